@@ -1,0 +1,176 @@
+"""fp64 CPU oracle of the head-wise sparse attention layer (TEST INFRASTRUCTURE ONLY).
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may import this
+package.  It wraps oracle/rtp_oracle.c (plain C, fp64) through ctypes and shares no code
+with the CUDA library.  What each function computes, and which passage of the pages it
+follows, is written in rtp_oracle.c.
+
+Parity pins: every function here is pinned by tests/test_oracle_pins.py (closed forms,
+brute force on tiny inputs, library routines, invariants); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        P = C.c_void_p
+        i64, i32, f64 = C.c_int64, C.c_int, C.c_double
+        L.orc_head_rows.restype = C.c_int
+        L.orc_head_rows.argtypes = [P, P, i64, i64, i32, i32, i32, P, i64, P, i64, i32, P, P, f64,
+                                    i64, i64, f64, f64, i64, P, P, P, P, P, P, i64, P, i64, i32]
+        L.orc_topp.restype = i64
+        L.orc_topp.argtypes = [P, i64, f64, P, P, P, P, P]
+        L.orc_rope.restype = None
+        L.orc_rope.argtypes = [P, f64, i32, f64, P]
+        L.orc_index_scores.restype = None
+        L.orc_index_scores.argtypes = [P, i64, i64, i32, i32, i32, P, P, P, P]
+        L.orc_max_threads.restype = C.c_int
+        L.orc_max_threads.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def max_threads() -> int:
+    return int(lib().orc_max_threads())
+
+
+def rope(x: np.ndarray, pos: float, base: float = 1.0e6) -> np.ndarray:
+    """Rotate-half RoPE of one fp64 vector at position ``pos``."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    lib().orc_rope(_p(x), float(pos), int(x.shape[0]), float(base), _p(y))
+    return y
+
+
+@dataclass
+class TopP:
+    count: int
+    order: np.ndarray  # key order (s desc, j asc); order[:count] is the selected set
+    pi: np.ndarray  # softmax mass per key
+    mass: float  # cumulative mass of the selected set
+    pi_t: float  # mass of the last member
+    cum_prev: float  # cumulative mass of the first count-1 members
+
+    @property
+    def selected(self) -> np.ndarray:
+        return np.sort(self.order[: self.count])
+
+
+def topp(scores: np.ndarray, p: float) -> TopP:
+    """Top-p selection over a score vector (the retrieval-head selection rule)."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    n = s.shape[0]
+    order = np.empty(max(n, 1), dtype=np.int64)
+    pi = np.empty(max(n, 1), dtype=np.float64)
+    mass = C.c_double()
+    pt = C.c_double()
+    cp = C.c_double()
+    K = lib().orc_topp(_p(s), n, float(p), _p(order), _p(pi), C.byref(mass), C.byref(pt), C.byref(cp))
+    return TopP(int(K), order[:n], pi[:n], mass.value, pt.value, cp.value)
+
+
+def index_scores(k_seq: np.ndarray, g: int, q_vec: np.ndarray, wq: np.ndarray, wk: np.ndarray,
+                 n: Optional[int] = None) -> np.ndarray:
+    """Pre-RoPE index scores of one query against keys 0..n-1 of KV head g.
+
+    k_seq: bf16 bits [N][Hkv][D] of one sequence; q_vec: bf16 bits [D]; wq/wk: fp32 [D][r].
+    """
+    k_seq = np.ascontiguousarray(k_seq, dtype=np.uint16)
+    N, Hkv, D = k_seq.shape
+    n = N if n is None else n
+    r = wq.shape[1]
+    q_vec = np.ascontiguousarray(q_vec, dtype=np.uint16)
+    wq = np.ascontiguousarray(wq, dtype=np.float32)
+    wk = np.ascontiguousarray(wk, dtype=np.float32)
+    s = np.empty(n, dtype=np.float64)
+    lib().orc_index_scores(_p(k_seq), n, Hkv * D, g, D, r, _p(q_vec), _p(wq), _p(wk), _p(s))
+    return s
+
+
+@dataclass
+class Rows:
+    out: np.ndarray  # [nrows][D]
+    count: np.ndarray  # [nrows]
+    mass: np.ndarray
+    pi_t: np.ndarray
+    cum_prev: np.ndarray
+    sel: Optional[list]  # per row: ascending selected positions (None if not requested)
+    pi: Optional[np.ndarray]  # [nrows][max_pos+1] index-softmax masses (retrieval, optional)
+
+
+def head_rows(k_seq: np.ndarray, v_seq: np.ndarray, q_rows: np.ndarray, positions: Sequence[int], *,
+              g: int, retrieval: bool, wq: Optional[np.ndarray] = None, wk: Optional[np.ndarray] = None,
+              top_p: float = 0.9, window: int = 8192, n_sink: int = 4, rope_base: float = 1.0e6,
+              sm_scale: Optional[float] = None, pos_offset: int = 0, want_sel: bool = True,
+              want_pi: bool = False, threads: Optional[int] = None) -> Rows:
+    """Oracle output of one query head for several query rows of one sequence.
+
+    k_seq, v_seq: bf16 bits [N][Hkv][D] (pre-RoPE keys); q_rows: bf16 bits [nrows][D];
+    positions: absolute position of each row (its own key is at that position).
+    """
+    k_seq = np.ascontiguousarray(k_seq, dtype=np.uint16)
+    v_seq = np.ascontiguousarray(v_seq, dtype=np.uint16)
+    N, Hkv, D = k_seq.shape
+    q_rows = np.ascontiguousarray(np.atleast_2d(q_rows), dtype=np.uint16)
+    pos = np.ascontiguousarray(np.asarray(positions, dtype=np.int64))
+    nrows = pos.shape[0]
+    r = 16 if wq is None else wq.shape[1]
+    if retrieval:
+        wq = np.ascontiguousarray(wq, dtype=np.float32)
+        wk = np.ascontiguousarray(wk, dtype=np.float32)
+    scale = 1.0 / np.sqrt(D) if sm_scale is None else sm_scale
+    out = np.zeros((nrows, D), dtype=np.float64)
+    cnt = np.zeros(nrows, dtype=np.int64)
+    mass = np.zeros(nrows)
+    pit = np.zeros(nrows)
+    cpv = np.zeros(nrows)
+    maxpos = int(pos.max()) if nrows else 0
+    cap = (maxpos + 1) if retrieval else (window + n_sink + 1)
+    sel = np.zeros((nrows, cap), dtype=np.int64) if want_sel else None
+    pi = np.zeros((nrows, maxpos + 1), dtype=np.float64) if (want_pi and retrieval) else None
+    th = max_threads() if threads is None else threads
+    rc = lib().orc_head_rows(
+        _p(k_seq), _p(v_seq), N, Hkv * D, g, D, r, _p(q_rows), q_rows.shape[1], _p(pos), nrows,
+        1 if retrieval else 0, _p(wq) if retrieval else None, _p(wk) if retrieval else None,
+        float(top_p), int(window), int(n_sink), float(rope_base), float(scale), int(pos_offset),
+        _p(out), _p(cnt), _p(mass), _p(pit), _p(cpv), _p(sel), cap if want_sel else 0,
+        _p(pi), (maxpos + 1) if pi is not None else 0, int(th))
+    if rc != 0:
+        raise ValueError("oracle: a row position lies outside the key range")
+    sels = [sel[t, : min(int(cnt[t]), cap)].copy() for t in range(nrows)] if want_sel else None
+    return Rows(out, cnt, mass, pit, cpv, sels, pi)
+
+
+def layer_rows(inputs, b: int, h: int, rows: Sequence[int], *, top_p: Optional[float] = None,
+               want_sel: bool = True, want_pi: bool = False, threads: Optional[int] = None,
+               pos_offset: int = 0) -> Rows:
+    """Oracle output of query head h of sequence b for chunk rows ``rows`` of a generated workload
+    (synth.LayerInputs): row i sits at position prefix + i."""
+    s = inputs.spec
+    rows = np.asarray(rows, dtype=np.int64)
+    retrieval = h in s.retrieval_heads
+    slot = s.retrieval_heads.index(h) if retrieval else 0
+    return head_rows(
+        inputs.k[b], inputs.v[b], inputs.q[b, rows, h], s.prefix + rows, g=s.kv_head(h),
+        retrieval=retrieval, wq=inputs.wq[slot] if retrieval else None,
+        wk=inputs.wk[slot] if retrieval else None, top_p=s.top_p if top_p is None else top_p,
+        window=s.window, n_sink=s.n_sink, rope_base=s.rope_base, want_sel=want_sel,
+        want_pi=want_pi, threads=threads, pos_offset=pos_offset)
