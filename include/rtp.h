@@ -1,0 +1,156 @@
+/*
+ * rtp.h -- C ABI of the head-wise sparse attention layer (RTPurbo) on NVIDIA B200 (sm_100a).
+ *
+ * The layer follows "Full Attention Strikes Back" (arXiv:2605.16928) as described on the
+ * pages it was built from:
+ *   - heads split into retrieval heads (~15%, keep the full KV cache) and local heads
+ *     (~85%, sliding window plus attention sinks)      -- techwalker page, section 2;
+ *   - retrieval heads score every causal key with a 16-dim pre-RoPE indexer
+ *     s_j = (Wq_h^T q).(Wk_h^T k_j)                    -- techwalker page, section 3;
+ *     ngjoo digest, "Core method" (pre-RoPE projections);
+ *   - they keep the smallest highest-score set whose index-softmax mass is >= p, ties to
+ *     the lower position                                -- zhichai page, insight 3;
+ *     techwalker page, section 4 (dynamic top-p);
+ *   - and run exact RoPE'd attention in the full head dim over that set
+ *                                                        -- techwalker page, section 3;
+ *   - local heads attend to the last W keys plus the first S keys
+ *                                                        -- techwalker page, section 8
+ *     (window 8192, 4 sinks).
+ *
+ * Conventions shared by every entry point
+ *   - All device pointers are plain CUDA device addresses on the layer's device; every
+ *     call is asynchronous and ordered on the stream it is given.  Nothing synchronises
+ *     the stream except rtp_check.
+ *   - The caller owns q/k/v/out and the streams.  The layer owns its KV cache, index-key
+ *     cache, weight copies and all scratch, and frees them in rtp_destroy.
+ *   - Argument errors are detected on the host before any launch and return RTP_EINVAL
+ *     (or RTP_ECAPACITY) without side effects.  Errors found by a kernel (a selection
+ *     larger than max_select, a value outside the fp16 cache range, a bounded wait that
+ *     ran out) are recorded in a device word and reported by the next rtp_check.
+ *   - No call allocates device memory after rtp_create.
+ *   - rtp_last_error returns a host string describing the most recent failure of a call
+ *     on that layer; it stays valid until the next call on the layer.
+ *   - A layer is not thread-safe: calls on one layer must be serialised by the caller and
+ *     issued on streams whose work does not overlap on the GPU.
+ */
+#ifndef RTP_H_
+#define RTP_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RTP_OK = 0,
+  RTP_EINVAL = 1,     /* bad argument (NULL pointer, unsupported size, p outside (0,1], ...) */
+  RTP_ENOMEM = 2,     /* device allocation failed in rtp_create */
+  RTP_ECAPACITY = 3,  /* append would exceed max_seq; nothing was written */
+  RTP_EOVERFLOW = 4,  /* a selected set exceeded max_select; it was truncated */
+  RTP_ECUDA = 5,      /* a CUDA runtime call or launch failed */
+  RTP_ETIMEOUT = 6,   /* a bounded in-kernel wait gave up; results of that call are invalid */
+  RTP_EINTERNAL = 7,  /* an internal consistency check failed */
+  RTP_ERANGE = 8      /* a RoPE'd key or a value lies outside the fp16 cache range */
+} rtp_status;
+
+typedef struct rtp_layer rtp_layer; /* opaque; owned by the library */
+
+typedef struct {
+  int32_t batch;              /* B >= 1 sequences; they share one length */
+  int32_t n_q_heads;          /* Hq >= 1 */
+  int32_t n_kv_heads;         /* Hkv >= 1, divides Hq (GQA: q head h reads KV head h / (Hq/Hkv)) */
+  int32_t head_dim;           /* D; must be 128 */
+  int32_t index_dim;          /* r; must be 16 */
+  int64_t max_seq;            /* KV capacity per sequence (positions 0..max_seq-1) */
+  const uint8_t* head_class;  /* HOST [Hq]: 1 = retrieval head, 0 = local head; copied */
+  float top_p;                /* p in (0, 1]; p == 1 keeps every causal key */
+  int32_t window;             /* W >= 1: a local head sees keys j with i - j < W */
+  int32_t n_sink;             /* S >= 0: ... and keys j < S */
+  double rope_base;           /* RoPE base (1e6 in the pages' models) */
+  float sm_scale;             /* attention scale; 0 selects 1/sqrt(D) */
+  const float* wq_index;      /* HOST [Hr][D][r] fp32, retrieval heads in ascending order; copied */
+  const float* wk_index;      /* HOST [Hr][D][r] fp32; copied */
+  int64_t max_select;         /* capacity of one selected set; 0 selects max_seq */
+  int32_t max_chunk;          /* largest prefill chunk C; 0 selects 16384 */
+} rtp_config;
+
+/* Optional decode statistics, DEVICE arrays [B][Hr] (retrieval heads ascending).  Any
+ * member may be NULL. */
+typedef struct {
+  int32_t* sel_count;  /* |J|, capped at max_select */
+  float* sel_mass;     /* index-softmax mass of J (>= p) */
+  float* threshold;    /* index-softmax mass of the last member of J */
+  int32_t* sel_index;  /* [B][Hr][sel_index_cap]: the first min(|J|, cap) positions of J, ascending */
+  int64_t sel_index_cap;
+} rtp_decode_stats;
+
+/* Optional prefill statistics, DEVICE array [B][C][Hr]. */
+typedef struct {
+  int32_t* sel_count;
+} rtp_prefill_stats;
+
+/* Device-side view of the layer's caches (for tests and tools; read-only use). */
+typedef struct {
+  const void* k;    /* fp16 [B][Hkv][max_seq][D]: RoPE'd keys */
+  const void* v;    /* fp16 [B][Hkv][max_seq][D] */
+  const float* idx; /* fp32 [B][Hr][max_seq][r]: pre-RoPE index keys Wk_h^T k_j */
+  int64_t max_seq;
+  int32_t n_retrieval;
+} rtp_cache_view;
+
+/* Create a layer on the current CUDA device: validates cfg, allocates the caches and all
+ * scratch, uploads the weights.  Synchronous.  On success *out receives the layer. */
+rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out);
+
+/* Release everything the layer owns.  Synchronises the device first.  NULL is a no-op. */
+rtp_status rtp_destroy(rtp_layer* layer);
+
+/* Append T >= 1 tokens to every sequence (positions len .. len+T-1): k, v are DEVICE bf16
+ * [B][T][Hkv][D], k pre-RoPE.  Writes RoPE(k) and v into the fp16 KV cache and, for every
+ * retrieval head h, the pre-RoPE index key Wk_h^T k into the index cache (the pages' 16-dim
+ * indexer: techwalker page section 3; ngjoo digest, pre-RoPE projections).  Advances the
+ * length by T.  RTP_ECAPACITY (nothing written) if len + T > max_seq. */
+rtp_status rtp_append_kv(rtp_layer* layer, const void* k, const void* v, int32_t T,
+                         cudaStream_t stream);
+
+/* One decode step for every sequence: q is DEVICE bf16 [B][Hq][D] pre-RoPE at position
+ * len-1 (append its own key first).  out is DEVICE fp32 [B][Hq][D].  Retrieval heads run
+ * index scoring, exact top-p selection and sparse attention; local heads run window+sink
+ * attention.  stats may be NULL. */
+rtp_status rtp_decode(rtp_layer* layer, const void* q, float* out, const rtp_decode_stats* stats,
+                      cudaStream_t stream);
+
+/* Chunked prefill: the last C appended tokens are the chunk; q is DEVICE bf16 [B][C][Hq][D]
+ * pre-RoPE, row i at position len-C+i.  Every row runs its own top-p selection over its causal
+ * prefix (retrieval heads) or its own window (local heads).  out is DEVICE fp32 [B][C][Hq][D].
+ * Requires 1 <= C <= min(len, max_chunk).  stats may be NULL. */
+rtp_status rtp_prefill_chunk(rtp_layer* layer, const void* q, int32_t C, float* out,
+                             const rtp_prefill_stats* stats, cudaStream_t stream);
+
+/* Change p for later calls (0 < p <= 1).  Takes effect in stream order of later calls. */
+rtp_status rtp_set_top_p(rtp_layer* layer, float top_p);
+
+/* Current sequence length (host-side counter; advanced by rtp_append_kv). */
+int64_t rtp_seq_len(const rtp_layer* layer);
+
+/* Forget every token (length back to 0); the caches are overwritten by later appends. */
+rtp_status rtp_reset(rtp_layer* layer);
+
+/* Synchronise `stream`, then report and clear errors recorded by kernels since the last
+ * check (RTP_EOVERFLOW, RTP_ERANGE, RTP_ETIMEOUT, ...). */
+rtp_status rtp_check(rtp_layer* layer, cudaStream_t stream);
+
+/* Device pointers of the caches. */
+rtp_status rtp_get_cache(const rtp_layer* layer, rtp_cache_view* view);
+
+/* Host string for the last failure on this layer ("" if none).  layer may be NULL, which
+ * returns the last failure of rtp_create in this thread. */
+const char* rtp_last_error(const rtp_layer* layer);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTP_H_ */

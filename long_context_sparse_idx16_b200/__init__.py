@@ -1,0 +1,262 @@
+"""Python binding of librtp (include/rtp.h): the head-wise sparse attention layer on B200.
+
+Argument marshalling only.  Every step of the layer runs in the CUDA kernels of
+librtp.so; PyTorch provides device memory and the current stream.  Importing the
+package does not need a GPU, but every call does, and the library must have been built
+(``python -m long_context_sparse_idx16_b200.build``): there is no fallback of any kind.
+
+The module-level functions carry the C names (rtp_create, rtp_append_kv, rtp_decode,
+rtp_prefill_chunk, rtp_destroy, ...); ``Layer`` wraps them for torch tensors.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librtp.so")
+
+RTP_OK, RTP_EINVAL, RTP_ENOMEM, RTP_ECAPACITY, RTP_EOVERFLOW = 0, 1, 2, 3, 4
+RTP_ECUDA, RTP_ETIMEOUT, RTP_EINTERNAL, RTP_ERANGE = 5, 6, 7, 8
+STATUS_NAMES = {0: "RTP_OK", 1: "RTP_EINVAL", 2: "RTP_ENOMEM", 3: "RTP_ECAPACITY", 4: "RTP_EOVERFLOW",
+                5: "RTP_ECUDA", 6: "RTP_ETIMEOUT", 7: "RTP_EINTERNAL", 8: "RTP_ERANGE"}
+
+
+class rtp_config(C.Structure):
+    _fields_ = [
+        ("batch", C.c_int32), ("n_q_heads", C.c_int32), ("n_kv_heads", C.c_int32),
+        ("head_dim", C.c_int32), ("index_dim", C.c_int32), ("max_seq", C.c_int64),
+        ("head_class", C.c_void_p), ("top_p", C.c_float), ("window", C.c_int32),
+        ("n_sink", C.c_int32), ("rope_base", C.c_double), ("sm_scale", C.c_float),
+        ("wq_index", C.c_void_p), ("wk_index", C.c_void_p), ("max_select", C.c_int64),
+        ("max_chunk", C.c_int32),
+    ]
+
+
+class rtp_decode_stats(C.Structure):
+    _fields_ = [("sel_count", C.c_void_p), ("sel_mass", C.c_void_p), ("threshold", C.c_void_p),
+                ("sel_index", C.c_void_p), ("sel_index_cap", C.c_int64)]
+
+
+class rtp_prefill_stats(C.Structure):
+    _fields_ = [("sel_count", C.c_void_p)]
+
+
+class rtp_cache_view(C.Structure):
+    _fields_ = [("k", C.c_void_p), ("v", C.c_void_p), ("idx", C.c_void_p), ("max_seq", C.c_int64),
+                ("n_retrieval", C.c_int32)]
+
+
+class RTPError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """The loaded librtp.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"librtp.so is missing at {LIB_PATH}; build it with "
+                              "`python -m long_context_sparse_idx16_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        P, i32, i64, f32 = C.c_void_p, C.c_int32, C.c_int64, C.c_float
+        sigs = {
+            "rtp_create": ([C.POINTER(rtp_config), C.POINTER(C.c_void_p)], C.c_int),
+            "rtp_destroy": ([P], C.c_int),
+            "rtp_append_kv": ([P, P, P, i32, P], C.c_int),
+            "rtp_decode": ([P, P, P, C.POINTER(rtp_decode_stats), P], C.c_int),
+            "rtp_prefill_chunk": ([P, P, i32, P, C.POINTER(rtp_prefill_stats), P], C.c_int),
+            "rtp_set_top_p": ([P, f32], C.c_int),
+            "rtp_seq_len": ([P], i64),
+            "rtp_reset": ([P], C.c_int),
+            "rtp_check": ([P, P], C.c_int),
+            "rtp_get_cache": ([P, C.POINTER(rtp_cache_view)], C.c_int),
+            "rtp_last_error": ([P], C.c_char_p),
+        }
+        for name, (args, res) in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(st: int, layer=None) -> None:
+    if st != RTP_OK:
+        msg = lib().rtp_last_error(layer)
+        raise RTPError(st, msg.decode() if msg else "")
+
+
+# ---------------------------------------------------------------- C names
+
+
+def rtp_create(cfg: rtp_config) -> C.c_void_p:
+    h = C.c_void_p()
+    _check(lib().rtp_create(C.byref(cfg), C.byref(h)))
+    return h
+
+
+def rtp_destroy(layer) -> None:
+    _check(lib().rtp_destroy(layer))
+
+
+def rtp_append_kv(layer, k_ptr: int, v_ptr: int, T: int, stream: int) -> None:
+    _check(lib().rtp_append_kv(layer, k_ptr, v_ptr, T, stream), layer)
+
+
+def rtp_decode(layer, q_ptr: int, out_ptr: int, stats: Optional[rtp_decode_stats], stream: int) -> None:
+    _check(lib().rtp_decode(layer, q_ptr, out_ptr, C.byref(stats) if stats is not None else None, stream), layer)
+
+
+def rtp_prefill_chunk(layer, q_ptr: int, C_rows: int, out_ptr: int, stats: Optional[rtp_prefill_stats],
+                      stream: int) -> None:
+    _check(lib().rtp_prefill_chunk(layer, q_ptr, C_rows, out_ptr,
+                                   C.byref(stats) if stats is not None else None, stream), layer)
+
+
+def rtp_set_top_p(layer, p: float) -> None:
+    _check(lib().rtp_set_top_p(layer, p), layer)
+
+
+def rtp_seq_len(layer) -> int:
+    return int(lib().rtp_seq_len(layer))
+
+
+def rtp_reset(layer) -> None:
+    _check(lib().rtp_reset(layer), layer)
+
+
+def rtp_check(layer, stream: int) -> int:
+    """Synchronise the stream; return the status of errors recorded by kernels."""
+    return int(lib().rtp_check(layer, stream))
+
+
+def rtp_get_cache(layer) -> rtp_cache_view:
+    v = rtp_cache_view()
+    _check(lib().rtp_get_cache(layer, C.byref(v)), layer)
+    return v
+
+
+def rtp_last_error(layer=None) -> str:
+    m = lib().rtp_last_error(layer)
+    return m.decode() if m else ""
+
+
+# ---------------------------------------------------------------- torch convenience
+
+
+def _stream_handle(stream=None) -> int:
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+class Layer:
+    """One sparse attention layer: owns a librtp layer on the current CUDA device."""
+
+    def __init__(self, *, batch: int, n_q_heads: int, n_kv_heads: int, head_class: Sequence[int],
+                 wq: Optional[np.ndarray], wk: Optional[np.ndarray], top_p: float, window: int,
+                 n_sink: int, max_seq: int, rope_base: float = 1.0e6, sm_scale: float = 0.0,
+                 max_select: int = 0, max_chunk: int = 0):
+        self._hc = np.ascontiguousarray(np.asarray(head_class, dtype=np.uint8))
+        self.n_retrieval = int(self._hc.sum())
+        self._wq = None if wq is None else np.ascontiguousarray(wq, dtype=np.float32)
+        self._wk = None if wk is None else np.ascontiguousarray(wk, dtype=np.float32)
+        cfg = rtp_config(
+            batch=batch, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads, head_dim=128, index_dim=16,
+            max_seq=max_seq, head_class=self._hc.ctypes.data, top_p=top_p, window=window,
+            n_sink=n_sink, rope_base=rope_base, sm_scale=sm_scale,
+            wq_index=self._wq.ctypes.data if self._wq is not None else None,
+            wk_index=self._wk.ctypes.data if self._wk is not None else None,
+            max_select=max_select, max_chunk=max_chunk)
+        self.batch, self.n_q_heads, self.n_kv_heads = batch, n_q_heads, n_kv_heads
+        self.handle = rtp_create(cfg)
+
+    @classmethod
+    def from_spec(cls, spec, inputs=None, *, max_seq: Optional[int] = None, **kw):
+        """A layer shaped like a synthetic workload spec (weights from `inputs`)."""
+        wq = inputs.wq if inputs is not None else None
+        wk = inputs.wk if inputs is not None else None
+        return cls(batch=spec.batch, n_q_heads=spec.n_q_heads, n_kv_heads=spec.n_kv_heads,
+                   head_class=spec.head_class, wq=wq, wk=wk, top_p=spec.top_p, window=spec.window,
+                   n_sink=spec.n_sink, max_seq=max_seq or spec.n_total, rope_base=spec.rope_base, **kw)
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            rtp_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def seq_len(self) -> int:
+        return rtp_seq_len(self.handle)
+
+    def set_top_p(self, p: float) -> None:
+        rtp_set_top_p(self.handle, p)
+
+    def reset(self) -> None:
+        rtp_reset(self.handle)
+
+    def append_kv(self, k, v, stream=None) -> None:
+        """k, v: torch bf16 CUDA tensors [B][T][Hkv][128] (k pre-RoPE)."""
+        assert k.is_cuda and k.is_contiguous() and v.is_contiguous()
+        rtp_append_kv(self.handle, k.data_ptr(), v.data_ptr(), int(k.shape[1]), _stream_handle(stream))
+
+    def decode(self, q, out=None, stats: bool = False, sel_cap: int = 0, stream=None):
+        """q: torch bf16 CUDA tensor [B][Hq][128] at position len-1.  Returns out (fp32) and,
+        with stats=True, (sel_count, sel_mass, threshold, sel_index) per (b, retrieval head);
+        sel_index holds the first sel_cap selected positions (None when sel_cap == 0)."""
+        import torch
+
+        assert q.is_cuda and q.is_contiguous()
+        if out is None:
+            out = torch.empty((self.batch, self.n_q_heads, 128), dtype=torch.float32, device=q.device)
+        st = None
+        tensors = None
+        if stats and self.n_retrieval:
+            shp = (self.batch, self.n_retrieval)
+            idx = (torch.full((self.batch, self.n_retrieval, sel_cap), -1, dtype=torch.int32, device=q.device)
+                   if sel_cap > 0 else None)
+            tensors = (torch.empty(shp, dtype=torch.int32, device=q.device),
+                       torch.empty(shp, dtype=torch.float32, device=q.device),
+                       torch.empty(shp, dtype=torch.float32, device=q.device), idx)
+            st = rtp_decode_stats(tensors[0].data_ptr(), tensors[1].data_ptr(), tensors[2].data_ptr(),
+                                  idx.data_ptr() if idx is not None else None, sel_cap)
+        rtp_decode(self.handle, q.data_ptr(), out.data_ptr(), st, _stream_handle(stream))
+        return (out, tensors) if stats else out
+
+    def prefill_chunk(self, q, out=None, stats: bool = False, stream=None):
+        """q: torch bf16 CUDA tensor [B][C][Hq][128]; row i at position len-C+i."""
+        import torch
+
+        assert q.is_cuda and q.is_contiguous()
+        Cr = int(q.shape[1])
+        if out is None:
+            out = torch.empty((self.batch, Cr, self.n_q_heads, 128), dtype=torch.float32, device=q.device)
+        st = None
+        cnt = None
+        if stats and self.n_retrieval:
+            cnt = torch.empty((self.batch, Cr, self.n_retrieval), dtype=torch.int32, device=q.device)
+            st = rtp_prefill_stats(cnt.data_ptr())
+        rtp_prefill_chunk(self.handle, q.data_ptr(), Cr, out.data_ptr(), st, _stream_handle(stream))
+        return (out, cnt) if stats else out
+
+    def check(self, stream=None) -> int:
+        return rtp_check(self.handle, _stream_handle(stream))
+
+    def cache(self) -> rtp_cache_view:
+        return rtp_get_cache(self.handle)

@@ -1,0 +1,145 @@
+// append_qprep.cu -- K/V append with RoPE and 16-dim index keys; query preparation.
+//
+// Append (rtp_append_kv): for each new token at position pos and KV head g,
+//   K[g][pos] = fp16(RoPE(k, pos)), V[g][pos] = fp16(v), and for every retrieval head h
+//   whose KV head is g: IDX[h][pos] = Wk_h^T k (pre-RoPE, fp32).
+// The indexer projects pre-RoPE keys (ngjoo digest, core method: "low-dimensional pre-RoPE
+// projections"; aitntnews page, finding 2: project D=128 down to r=16 so that the
+// high-frequency RoPE components do not disturb long-range matching).
+//
+// Query prep: q_rot = RoPE(q, pos) in fp32 and q_idx = Wq_h^T q (pre-RoPE) for retrieval heads.
+//
+// RoPE is the rotate-half form: pair (c, c + D/2) turns by pos * base^(-2c/D).  The angle is
+// formed and reduced in fp64 (pos reaches 2^20, where an fp32 angle is off by ~0.06 rad),
+// then the rotation runs in fp32.
+#include "rtp_device.cuh"
+#include "rtp_internal.h"
+
+namespace rtp {
+
+namespace {
+
+constexpr float kFp16Max = 65504.f;
+
+__global__ void __launch_bounds__(256) append_kv_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int T, int Hkv,
+    int Hr, int64_t pos0, int64_t max_seq, const double* __restrict__ theta,
+    const float* __restrict__ wk, const int16_t* __restrict__ ret_head, int group,
+    __half* __restrict__ kc, __half* __restrict__ vc, float* __restrict__ idx,
+    uint32_t* __restrict__ err) {
+  const int t = blockIdx.x;  // token within the appended block
+  const int b = blockIdx.y;
+  const int64_t pos = pos0 + t;
+  extern __shared__ float ks[];  // [Hkv][D] pre-RoPE key (fp32)
+  __shared__ float cs[kHalfD], sn[kHalfD];
+
+  const __nv_bfloat16* kt = k + ((int64_t)b * T + t) * Hkv * kD;
+  const __nv_bfloat16* vt = v + ((int64_t)b * T + t) * Hkv * kD;
+  for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) ks[i] = __bfloat162float(kt[i]);
+  if (threadIdx.x < kHalfD) {
+    double a = (double)pos * theta[threadIdx.x];
+    double s_, c_;
+    sincos(a, &s_, &c_);
+    cs[threadIdx.x] = (float)c_;
+    sn[threadIdx.x] = (float)s_;
+  }
+  __syncthreads();
+
+  bool bad = false;
+  for (int i = threadIdx.x; i < Hkv * kHalfD; i += blockDim.x) {
+    const int g = i / kHalfD, c = i % kHalfD;
+    const float x0 = ks[g * kD + c], x1 = ks[g * kD + c + kHalfD];
+    const float y0 = x0 * cs[c] - x1 * sn[c];
+    const float y1 = x1 * cs[c] + x0 * sn[c];
+    bad |= !(fabsf(y0) <= kFp16Max) || !(fabsf(y1) <= kFp16Max);
+    __half* dst = kc + (((int64_t)b * Hkv + g) * max_seq + pos) * kD;
+    dst[c] = __float2half_rn(y0);
+    dst[c + kHalfD] = __float2half_rn(y1);
+  }
+  for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) {
+    const int g = i / kD, d = i % kD;
+    const float x = __bfloat162float(vt[i]);
+    bad |= !(fabsf(x) <= kFp16Max);
+    vc[(((int64_t)b * Hkv + g) * max_seq + pos) * kD + d] = __float2half_rn(x);
+  }
+  // index keys: Hr x r outputs, each a 128-term fp32 dot product in a fixed order
+  for (int o = threadIdx.x; o < Hr * kR; o += blockDim.x) {
+    const int hr = o / kR, c = o % kR;
+    const int g = ret_head[hr] / group;
+    const float* w = wk + (int64_t)hr * kD * kR + c;
+    const float* x = ks + g * kD;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < kD; ++d) acc = fmaf(w[d * kR], x[d], acc);
+    idx[(((int64_t)b * Hr + hr) * max_seq + pos) * kR + c] = acc;
+  }
+  if (bad) atomicOr(err, kErrRange);
+}
+
+// One CTA per (row, batch): RoPE'd fp32 query for every head, pre-RoPE index query for the
+// retrieval heads.
+__global__ void __launch_bounds__(128) q_prep_kernel(
+    const __nv_bfloat16* __restrict__ q, int rows, int Hq, int Hr, int64_t pos0,
+    const double* __restrict__ theta, const float* __restrict__ wq,
+    const int16_t* __restrict__ ret_head, float* __restrict__ q_rot, float* __restrict__ q_idx) {
+  const int i = blockIdx.x, b = blockIdx.y;
+  const int64_t pos = pos0 + i;
+  __shared__ float cs[kHalfD], sn[kHalfD];
+  __shared__ float qs[kD];
+  if (threadIdx.x < kHalfD) {
+    double a = (double)pos * theta[threadIdx.x];
+    double s_, c_;
+    sincos(a, &s_, &c_);
+    cs[threadIdx.x] = (float)c_;
+    sn[threadIdx.x] = (float)s_;
+  }
+  __syncthreads();
+  const int64_t row = (int64_t)b * rows + i;
+  const __nv_bfloat16* qr = q + row * Hq * kD;
+  for (int h = 0; h < Hq; ++h) {
+    const float x = __bfloat162float(qr[h * kD + threadIdx.x]);
+    const float xp = __bfloat162float(qr[h * kD + (threadIdx.x ^ kHalfD)]);
+    const int c = threadIdx.x & (kHalfD - 1);
+    // first half: x*cos - partner*sin; second half: x*cos + partner*sin
+    const float y = threadIdx.x < kHalfD ? x * cs[c] - xp * sn[c] : x * cs[c] + xp * sn[c];
+    q_rot[(row * Hq + h) * kD + threadIdx.x] = y;
+  }
+  for (int hr = 0; hr < Hr; ++hr) {
+    const int h = ret_head[hr];
+    __syncthreads();
+    qs[threadIdx.x] = __bfloat162float(qr[h * kD + threadIdx.x]);
+    __syncthreads();
+    // 16 outputs x 8 partial sums of 16 dims each
+    const int c = threadIdx.x >> 3, part = threadIdx.x & 7;
+    const float* w = wq + (int64_t)hr * kD * kR + c;
+    float acc = 0.f;
+#pragma unroll
+    for (int d = part * 16; d < part * 16 + 16; ++d) acc = fmaf(w[d * kR], qs[d], acc);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (part == 0) q_idx[(row * Hr + hr) * kR + c] = acc;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T,
+                             cudaStream_t st) {
+  dim3 grid(T, L->B);
+  size_t smem = (size_t)L->Hkv * kD * sizeof(float);
+  append_kv_kernel<<<grid, 256, smem, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta,
+                                            L->wk, L->d_ret_head, L->group, L->kc, L->vc, L->idx,
+                                            L->err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, int64_t pos0,
+                          cudaStream_t st) {
+  dim3 grid(rows, L->B);
+  q_prep_kernel<<<grid, 128, 0, st>>>(q, rows, L->Hq, L->Hr, pos0, L->theta, L->wq, L->d_ret_head,
+                                      L->q_rot, L->q_idx);
+  return cudaGetLastError();
+}
+
+}  // namespace rtp

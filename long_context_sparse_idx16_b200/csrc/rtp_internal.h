@@ -1,0 +1,109 @@
+// rtp_internal.h -- layer state and kernel launch entry points (host side, internal).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "rtp.h"
+
+namespace rtp {
+
+// Work-split and scratch sizes of the fused decode index-stream + top-p select kernel.
+constexpr int kSelThreads = 1024;
+constexpr int kSelBins = 2048;   // level-1 score bins (width 1/64 below the row max) and radix digits
+constexpr int kSelMaxSeg = 64;   // (problem, CTA) segments one CTA may hold
+
+// Sparse-attention gather (decode): indices per work item.
+constexpr int kGatherChunk = 128;
+constexpr int kGatherThreads = 256;
+
+// Window + sink decode attention: keys per CTA tile and threads.
+constexpr int kSwaTile = 128;
+constexpr int kSwaThreads = 128;
+
+}  // namespace rtp
+
+struct rtp_layer {
+  // configuration
+  int B = 0, Hq = 0, Hkv = 0, Hr = 0, group = 0;
+  int64_t max_seq = 0, max_select = 0, len = 0;
+  int max_chunk = 0;
+  float top_p = 0.9f, sm_scale = 0.f;
+  double rope_base = 1e6;
+  int W = 0, S = 0;
+  std::vector<int> ret_heads;        // retrieval slot -> q head
+  std::vector<int> head_slot;        // q head -> retrieval slot or -1
+  int device = 0, sm_count = 0;
+  size_t smem_optin = 0;
+
+  // caches
+  __half* kc = nullptr;  // [B][Hkv][max_seq][D] RoPE'd keys
+  __half* vc = nullptr;  // [B][Hkv][max_seq][D]
+  float* idx = nullptr;  // [B][Hr][max_seq][r]
+  float* wq = nullptr;   // [Hr][D][r]
+  float* wk = nullptr;   // [Hr][D][r]
+  double* theta = nullptr;  // [D/2] RoPE frequencies base^(-2c/D)
+  int16_t* d_head_slot = nullptr;  // [Hq]
+  int16_t* d_ret_head = nullptr;   // [Hr]
+  int16_t* d_loc_head = nullptr;   // [Hkv][kMaxGroup] local q heads of each KV head (-1 pad)
+  int32_t* d_loc_cnt = nullptr;    // [Hkv]
+  int n_local = 0;
+
+  // decode scratch
+  float* q_rot = nullptr;    // [B*max_rows][Hq][D] fp32 RoPE'd queries
+  float* q_idx = nullptr;    // [B*max_rows][Hr][r]
+  int32_t* sel_idx = nullptr;  // [B*Hr][max_select]
+  int32_t* sel_cnt = nullptr;  // [B*Hr]
+  float* sel_mass = nullptr;   // [B*Hr]
+  float* sel_thr = nullptr;    // [B*Hr]
+  float* seg_max = nullptr;    // [P + G]
+  unsigned long long* h1_mass = nullptr;  // [P][bins]
+  uint32_t* h1_cnt = nullptr;
+  unsigned long long* hr_mass = nullptr;  // [2][P][bins]
+  uint32_t* hr_cnt = nullptr;
+  uint32_t* slot_cnt = nullptr;  // [P + G][2]
+  uint32_t* bar = nullptr;       // [2] grid barrier count, generation
+  float* gscores = nullptr;      // [P][max_seq] when scores do not fit in shared memory
+  size_t gscores_elems = 0;
+  float* gpart = nullptr;        // gather partials [items][D + 2]
+  int64_t gpart_items = 0;
+  uint32_t* gticket = nullptr;   // [B*Hr]
+  float* spart = nullptr;        // window partials
+  int64_t spart_elems = 0;
+  uint32_t* sticket = nullptr;   // [B*Hkv]
+  uint32_t* err = nullptr;       // device error word
+
+  std::string last_error;
+};
+
+namespace rtp {
+
+rtp_status fail(rtp_layer* L, rtp_status st, const std::string& msg);
+rtp_status cuda_fail(rtp_layer* L, cudaError_t e, const char* what);
+
+// Kernel launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T,
+                             cudaStream_t st);
+cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, int64_t pos0,
+                          cudaStream_t st);
+cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st);
+cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, float* out, cudaStream_t st);
+cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st);
+cudaError_t launch_iota_rows(int32_t* dst, int64_t cap, int rows, int64_t n, cudaStream_t st);
+cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st);
+
+// Selection kernel geometry for the current length (host-side; also sizes scratch).
+struct SelectGeom {
+  int grid = 0;
+  int64_t per_cta = 0;
+  bool smem_scores = true;
+  size_t smem_bytes = 0;
+};
+SelectGeom select_geometry(const rtp_layer* L, int64_t N);
+size_t select_fixed_smem();
+
+}  // namespace rtp

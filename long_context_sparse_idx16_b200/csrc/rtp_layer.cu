@@ -1,0 +1,337 @@
+// rtp_layer.cu -- the C ABI: layer creation, validation, memory layout and call sequencing.
+//
+// Memory layout in HBM (one layer):
+//   K cache  fp16 [B][Hkv][max_seq][128]  RoPE'd keys (written once by append)
+//   V cache  fp16 [B][Hkv][max_seq][128]
+//   IDX      fp32 [B][Hr][max_seq][16]    pre-RoPE index keys, one 64-byte row per key
+// fp16 (not bf16) caches: values are O(1)..O(100); fp16's 11-bit significand keeps the
+// rounding of RoPE'd keys, of the fp16 query and of the probabilities fed to the tensor
+// cores near 2.4e-4 each, which the 1e-3 relative-L2 output tolerance needs.  Inputs stay
+// bf16; bf16 -> fp16 is exact inside fp16's range, and append flags anything outside it.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+#include <vector>
+
+#include "rtp_device.cuh"
+#include "rtp_internal.h"
+
+namespace rtp {
+
+int64_t swa_part_elems(const rtp_layer* L);
+
+static thread_local std::string g_create_error;
+
+rtp_status fail(rtp_layer* L, rtp_status st, const std::string& msg) {
+  if (L) L->last_error = msg;
+  else g_create_error = msg;
+  return st;
+}
+
+rtp_status cuda_fail(rtp_layer* L, cudaError_t e, const char* what) {
+  std::string m = std::string(what) + ": " + cudaGetErrorString(e);
+  return fail(L, RTP_ECUDA, m);
+}
+
+template <typename T>
+static cudaError_t dalloc(T** p, size_t elems) {
+  *p = nullptr;
+  if (elems == 0) elems = 1;
+  return cudaMalloc((void**)p, elems * sizeof(T));
+}
+
+static void free_all(rtp_layer* L) {
+  void* ptrs[] = {L->kc, L->vc, L->idx, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
+                  L->d_loc_head, L->d_loc_cnt, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
+                  L->sel_mass, L->sel_thr, L->seg_max, L->h1_mass, L->h1_cnt, L->hr_mass,
+                  L->hr_cnt, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
+                  L->sticket, L->err};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+}  // namespace rtp
+
+using namespace rtp;
+
+extern "C" {
+
+rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
+  if (!cfg || !out) return fail(nullptr, RTP_EINVAL, "rtp_create: NULL argument");
+  *out = nullptr;
+  const rtp_config& c = *cfg;
+  if (c.batch < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads != 0)
+    return fail(nullptr, RTP_EINVAL, "rtp_create: need batch >= 1 and n_kv_heads dividing n_q_heads");
+  if (c.head_dim != kD || c.index_dim != kR)
+    return fail(nullptr, RTP_EINVAL, "rtp_create: head_dim must be 128 and index_dim 16");
+  if (c.n_q_heads / c.n_kv_heads > kMaxGroup)
+    return fail(nullptr, RTP_EINVAL, "rtp_create: at most 16 query heads per KV head");
+  if (c.max_seq < 1 || c.max_seq > (int64_t)INT32_MAX)
+    return fail(nullptr, RTP_EINVAL, "rtp_create: max_seq must be in [1, 2^31)");
+  if (!c.head_class) return fail(nullptr, RTP_EINVAL, "rtp_create: head_class is NULL");
+  if (!(c.top_p > 0.f && c.top_p <= 1.f)) return fail(nullptr, RTP_EINVAL, "rtp_create: top_p must be in (0, 1]");
+  if (c.window < 1 || c.n_sink < 0) return fail(nullptr, RTP_EINVAL, "rtp_create: need window >= 1, n_sink >= 0");
+  if (!(c.rope_base > 1.0)) return fail(nullptr, RTP_EINVAL, "rtp_create: rope_base must be > 1");
+  if (c.sm_scale < 0.f) return fail(nullptr, RTP_EINVAL, "rtp_create: sm_scale must be >= 0");
+  if (c.max_select < 0 || c.max_select > c.max_seq)
+    return fail(nullptr, RTP_EINVAL, "rtp_create: max_select must be in [0, max_seq]");
+  if (c.max_chunk < 0) return fail(nullptr, RTP_EINVAL, "rtp_create: max_chunk must be >= 0");
+
+  rtp_layer* L = new rtp_layer();
+  L->B = c.batch;
+  L->Hq = c.n_q_heads;
+  L->Hkv = c.n_kv_heads;
+  L->group = c.n_q_heads / c.n_kv_heads;
+  L->max_seq = c.max_seq;
+  L->max_select = c.max_select ? c.max_select : c.max_seq;
+  L->max_chunk = c.max_chunk ? c.max_chunk : 16384;
+  L->top_p = c.top_p;
+  L->sm_scale = c.sm_scale > 0.f ? c.sm_scale : 1.0f / sqrtf((float)kD);
+  L->rope_base = c.rope_base;
+  L->W = c.window;
+  L->S = c.n_sink;
+  L->head_slot.assign(L->Hq, -1);
+  std::vector<int16_t> loc_head((size_t)L->Hkv * kMaxGroup, (int16_t)-1);
+  std::vector<int32_t> loc_cnt(L->Hkv, 0);
+  for (int h = 0; h < L->Hq; ++h) {
+    if (c.head_class[h] > 1) {
+      delete L;
+      return fail(nullptr, RTP_EINVAL, "rtp_create: head_class entries must be 0 or 1");
+    }
+    if (c.head_class[h] == 1) {
+      L->head_slot[h] = (int)L->ret_heads.size();
+      L->ret_heads.push_back(h);
+    } else {
+      const int g = h / L->group;
+      loc_head[(size_t)g * kMaxGroup + loc_cnt[g]++] = (int16_t)h;
+      ++L->n_local;
+    }
+  }
+  L->Hr = (int)L->ret_heads.size();
+  if (L->Hr > 0 && (!c.wq_index || !c.wk_index)) {
+    delete L;
+    return fail(nullptr, RTP_EINVAL, "rtp_create: retrieval heads need wq_index and wk_index");
+  }
+  if ((int64_t)L->B * L->Hr > 2048) {
+    delete L;
+    return fail(nullptr, RTP_EINVAL, "rtp_create: batch * retrieval heads must be <= 2048");
+  }
+  cudaError_t e = cudaGetDevice(&L->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&L->sm_count, cudaDevAttrMultiProcessorCount, L->device);
+  int optin = 0;
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, L->device);
+  if (e != cudaSuccess) {
+    delete L;
+    return cuda_fail(nullptr, e, "rtp_create: device query");
+  }
+  L->smem_optin = (size_t)optin;
+
+  const int64_t B = L->B, Hkv = L->Hkv, Hr = L->Hr, Hq = L->Hq, P = B * Hr;
+  const int64_t rows = B * L->max_chunk;
+  const int64_t G = L->sm_count;
+  // Largest per-CTA score count the shared-memory variant can hold; beyond it the
+  // selection keeps scores in global scratch.
+  const int64_t smem_cap = ((int64_t)L->smem_optin - (int64_t)select_fixed_smem()) / 4;
+  const bool need_gscores = P * L->max_seq > smem_cap * G;
+  const int64_t gitems = P * ((L->max_seq + kGatherChunk - 1) / kGatherChunk);
+
+#define RTP_ALLOC(ptr, n)                                         \
+  do {                                                            \
+    if (e == cudaSuccess) e = dalloc(&(ptr), (size_t)(n));         \
+  } while (0)
+  e = cudaSuccess;
+  RTP_ALLOC(L->kc, B * Hkv * L->max_seq * kD);
+  RTP_ALLOC(L->vc, B * Hkv * L->max_seq * kD);
+  RTP_ALLOC(L->idx, P * L->max_seq * kR);
+  RTP_ALLOC(L->wq, Hr * kD * kR);
+  RTP_ALLOC(L->wk, Hr * kD * kR);
+  RTP_ALLOC(L->theta, kHalfD);
+  RTP_ALLOC(L->d_head_slot, Hq);
+  RTP_ALLOC(L->d_ret_head, Hr);
+  RTP_ALLOC(L->d_loc_head, Hkv * kMaxGroup);
+  RTP_ALLOC(L->d_loc_cnt, Hkv);
+  RTP_ALLOC(L->q_rot, rows * Hq * kD);
+  RTP_ALLOC(L->q_idx, rows * Hr * kR);
+  RTP_ALLOC(L->sel_idx, P * L->max_select);
+  RTP_ALLOC(L->sel_cnt, P);
+  RTP_ALLOC(L->sel_mass, P);
+  RTP_ALLOC(L->sel_thr, P);
+  RTP_ALLOC(L->seg_max, P + G);
+  RTP_ALLOC(L->h1_mass, P * kSelBins);
+  RTP_ALLOC(L->h1_cnt, P * kSelBins);
+  RTP_ALLOC(L->hr_mass, 3 * P * kSelBins);
+  RTP_ALLOC(L->hr_cnt, 3 * P * kSelBins);
+  RTP_ALLOC(L->slot_cnt, 2 * (P + G));
+  RTP_ALLOC(L->bar, 2);
+  if (need_gscores) {
+    L->gscores_elems = (size_t)(P * L->max_seq);
+    RTP_ALLOC(L->gscores, L->gscores_elems);
+  }
+  L->gpart_items = gitems;
+  RTP_ALLOC(L->gpart, gitems * (kD + 2));
+  RTP_ALLOC(L->gticket, P);
+  L->spart_elems = swa_part_elems(L);
+  RTP_ALLOC(L->spart, L->spart_elems);
+  RTP_ALLOC(L->err, 1);
+#undef RTP_ALLOC
+  if (e != cudaSuccess) {
+    free_all(L);
+    delete L;
+    return fail(nullptr, RTP_ENOMEM, std::string("rtp_create: device allocation failed: ") + cudaGetErrorString(e));
+  }
+
+  // weights, maps, RoPE frequencies, zeroed counters
+  std::vector<double> theta(kHalfD);
+  for (int i = 0; i < kHalfD; ++i) theta[i] = pow(c.rope_base, -2.0 * (double)i / (double)kD);
+  std::vector<int16_t> slot16(Hq), ret16(Hr > 0 ? Hr : 1);
+  for (int h = 0; h < Hq; ++h) slot16[h] = (int16_t)L->head_slot[h];
+  for (int i = 0; i < Hr; ++i) ret16[i] = (int16_t)L->ret_heads[i];
+  if (Hr > 0) {
+    e = cudaMemcpy(L->wq, c.wq_index, sizeof(float) * Hr * kD * kR, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(L->wk, c.wk_index, sizeof(float) * Hr * kD * kR, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(L->d_ret_head, ret16.data(), sizeof(int16_t) * Hr, cudaMemcpyHostToDevice);
+  }
+  if (e == cudaSuccess) e = cudaMemcpy(L->theta, theta.data(), sizeof(double) * kHalfD, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(L->d_head_slot, slot16.data(), sizeof(int16_t) * Hq, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(L->d_loc_head, loc_head.data(), sizeof(int16_t) * Hkv * kMaxGroup, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(L->d_loc_cnt, loc_cnt.data(), sizeof(int32_t) * Hkv, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(L->bar, 0, 2 * sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(L->gticket, 0, sizeof(uint32_t) * (P > 0 ? P : 1));
+  if (e == cudaSuccess) e = cudaMemset(L->err, 0, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(L->sel_cnt, 0, sizeof(int32_t) * (P > 0 ? P : 1));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    free_all(L);
+    delete L;
+    return cuda_fail(nullptr, e, "rtp_create: upload");
+  }
+  *out = L;
+  return RTP_OK;
+}
+
+rtp_status rtp_destroy(rtp_layer* L) {
+  if (!L) return RTP_OK;
+  cudaDeviceSynchronize();
+  free_all(L);
+  delete L;
+  return RTP_OK;
+}
+
+rtp_status rtp_append_kv(rtp_layer* L, const void* k, const void* v, int32_t T, cudaStream_t stream) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_append_kv: layer is NULL");
+  if (!k || !v) return fail(L, RTP_EINVAL, "rtp_append_kv: k or v is NULL");
+  if (T < 1) return fail(L, RTP_EINVAL, "rtp_append_kv: T must be >= 1");
+  if (L->len + T > L->max_seq) return fail(L, RTP_ECAPACITY, "rtp_append_kv: max_seq exceeded");
+  cudaError_t e = launch_append_kv(L, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, T, stream);
+  if (e != cudaSuccess) return cuda_fail(L, e, "rtp_append_kv: launch");
+  L->len += T;
+  L->last_error.clear();
+  return RTP_OK;
+}
+
+rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_stats* stats, cudaStream_t stream) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_decode: layer is NULL");
+  if (!q || !out) return fail(L, RTP_EINVAL, "rtp_decode: q or out is NULL");
+  if (L->len < 1) return fail(L, RTP_EINVAL, "rtp_decode: the cache is empty (append the token first)");
+  cudaError_t e = launch_q_prep(L, (const __nv_bfloat16*)q, 1, L->len - 1, stream);
+  if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: q_prep");
+  if (L->Hr > 0) {
+    // p == 1 keeps every causal key: the gather reads positions 0..len-1 directly
+    const bool dense = L->top_p >= 1.f;
+    e = dense ? launch_dense_stats(L, stream) : launch_decode_select(L, stream);
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: select");
+    e = launch_decode_gather(L, dense, out, stream);
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: gather");
+    if (stats) {
+      const size_t P = (size_t)L->B * L->Hr;
+      if (stats->sel_count)
+        e = cudaMemcpyAsync(stats->sel_count, L->sel_cnt, P * 4, cudaMemcpyDeviceToDevice, stream);
+      if (e == cudaSuccess && stats->sel_mass)
+        e = cudaMemcpyAsync(stats->sel_mass, L->sel_mass, P * 4, cudaMemcpyDeviceToDevice, stream);
+      if (e == cudaSuccess && stats->threshold)
+        e = cudaMemcpyAsync(stats->threshold, L->sel_thr, P * 4, cudaMemcpyDeviceToDevice, stream);
+      if (e == cudaSuccess && stats->sel_index && stats->sel_index_cap > 0) {
+        if (dense) {
+          e = launch_iota_rows(stats->sel_index, stats->sel_index_cap, (int)P, L->len, stream);
+        } else {
+          const int64_t w = stats->sel_index_cap < L->max_select ? stats->sel_index_cap : L->max_select;
+          e = cudaMemcpy2DAsync(stats->sel_index, (size_t)stats->sel_index_cap * 4, L->sel_idx,
+                                (size_t)L->max_select * 4, (size_t)w * 4, P, cudaMemcpyDeviceToDevice, stream);
+        }
+      }
+      if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: stats");
+    }
+  }
+  if (L->n_local > 0) {
+    e = launch_decode_swa(L, out, stream);
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: window attention");
+  }
+  L->last_error.clear();
+  return RTP_OK;
+}
+
+rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out, const rtp_prefill_stats* stats,
+                             cudaStream_t stream) {
+  (void)stats;
+  (void)stream;
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_prefill_chunk: layer is NULL");
+  if (!q || !out) return fail(L, RTP_EINVAL, "rtp_prefill_chunk: q or out is NULL");
+  if (C < 1 || C > L->max_chunk || C > L->len)
+    return fail(L, RTP_EINVAL, "rtp_prefill_chunk: need 1 <= C <= min(len, max_chunk)");
+  return fail(L, RTP_EINTERNAL, "rtp_prefill_chunk: not built yet");
+}
+
+rtp_status rtp_set_top_p(rtp_layer* L, float top_p) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_set_top_p: layer is NULL");
+  if (!(top_p > 0.f && top_p <= 1.f)) return fail(L, RTP_EINVAL, "rtp_set_top_p: top_p must be in (0, 1]");
+  L->top_p = top_p;
+  return RTP_OK;
+}
+
+int64_t rtp_seq_len(const rtp_layer* L) { return L ? L->len : -1; }
+
+rtp_status rtp_reset(rtp_layer* L) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_reset: layer is NULL");
+  L->len = 0;
+  return RTP_OK;
+}
+
+rtp_status rtp_check(rtp_layer* L, cudaStream_t stream) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_check: layer is NULL");
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(L, e, "rtp_check: stream");
+  uint32_t w = 0;
+  e = cudaMemcpy(&w, L->err, sizeof w, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(L, e, "rtp_check: read error word");
+  if (w == 0) return RTP_OK;
+  cudaMemset(L->err, 0, sizeof(uint32_t));
+  if (w & kErrTimeout) {
+    // a barrier gave up: its counters are inconsistent; start the next launch from zero
+    cudaMemset(L->bar, 0, 2 * sizeof(uint32_t));
+    cudaMemset(L->gticket, 0, sizeof(uint32_t) * (size_t)(L->B * L->Hr > 0 ? L->B * L->Hr : 1));
+    return fail(L, RTP_ETIMEOUT, "a bounded in-kernel wait gave up");
+  }
+  if (w & kErrInternal) return fail(L, RTP_EINTERNAL, "an internal consistency check failed");
+  if (w & kErrOverflow) return fail(L, RTP_EOVERFLOW, "a selected set exceeded max_select and was truncated");
+  if (w & kErrRange) return fail(L, RTP_ERANGE, "a key or value lies outside the fp16 cache range");
+  return fail(L, RTP_EINTERNAL, "unknown device error");
+}
+
+rtp_status rtp_get_cache(const rtp_layer* L, rtp_cache_view* view) {
+  if (!L || !view) return fail(nullptr, RTP_EINVAL, "rtp_get_cache: NULL argument");
+  view->k = L->kc;
+  view->v = L->vc;
+  view->idx = L->idx;
+  view->max_seq = L->max_seq;
+  view->n_retrieval = L->Hr;
+  return RTP_OK;
+}
+
+const char* rtp_last_error(const rtp_layer* L) {
+  return L ? L->last_error.c_str() : g_create_error.c_str();
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+"""Helpers shared by the GPU parity tests: drive the CUDA layer through the C ABI on a
+seeded workload and compare with the fp64 oracle under the stated tolerances.
+
+Tolerances (from the method statement):
+  * selected index sets identical except for keys whose oracle probability lies within
+    1e-6 of the threshold probability (the mass of the last member);  keys at the mass
+    boundary may also move when the oracle's cumulative mass before or after the last
+    member lies within 1e-6 of p (fp summation may legitimately move the cut there);
+  * selected mass (oracle probabilities over the GPU's set) >= p - 1e-5;
+  * attention outputs within 1e-2 max-abs and 1e-3 relative L2.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+
+SET_TOL = 1e-6
+MASS_TOL = 1e-5
+ABS_TOL = 1e-2
+REL_L2_TOL = 1e-3
+
+
+def torch_bf16(bits: np.ndarray, device="cuda"):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def build_cache(layer, x, upto: int, chunk: int = 1 << 16):
+    """Append positions [layer.seq_len, upto) of workload x to the layer."""
+    start = layer.seq_len
+    for t0 in range(start, upto, chunk):
+        t1 = min(upto, t0 + chunk)
+        layer.append_kv(torch_bf16(x.k[:, t0:t1]), torch_bf16(x.v[:, t0:t1]))
+
+
+def check_selection(gpu_sel: np.ndarray, ref: "oracle.Rows", t: int, p: float, what: str):
+    """Compare a GPU selected set (ascending positions) with oracle row t (needs ref.pi)."""
+    o_sel = ref.sel[t]
+    pi = ref.pi[t]
+    diff = np.setxor1d(gpu_sel, o_sel)
+    pt = ref.pi_t[t]
+    boundary = abs(ref.cum_prev[t] - p) <= SET_TOL or abs(ref.mass[t] - p) <= SET_TOL
+    bad = [j for j in diff if abs(pi[j] - pt) > SET_TOL]
+    if bad and boundary:
+        # at a mass boundary the cut may move by one key: the first key outside the oracle set
+        rest = np.ones(pi.shape[0], dtype=bool)
+        rest[o_sel] = False
+        p_next = float(pi[rest].max()) if rest.any() else pt
+        bad = [j for j in bad if abs(pi[j] - p_next) > SET_TOL]
+    assert not bad, (f"{what}: {len(bad)} selected keys differ beyond tolerance, e.g. {bad[:5]} "
+                     f"pi={[float(pi[j]) for j in bad[:5]]} pi_t={pt} |gpu|={len(gpu_sel)} |ref|={len(o_sel)}")
+    mass = float(pi[gpu_sel].sum()) if len(gpu_sel) else 0.0
+    assert mass >= p - MASS_TOL, f"{what}: selected mass {mass} < p - 1e-5 (p={p})"
+    return len(diff)
+
+
+def check_outputs(gpu: np.ndarray, ref: np.ndarray, what: str):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite outputs"
+    err = np.abs(gpu - ref)
+    rel = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err.max() <= ABS_TOL, f"{what}: max-abs error {err.max():.3e} > {ABS_TOL}"
+    assert rel <= REL_L2_TOL, f"{what}: relative L2 error {rel:.3e} > {REL_L2_TOL}"
+    return float(err.max()), float(rel)
+
+
+def run_decode(x, *, top_p=None, heads=None, batches=None, max_select=0, sel_cap=None, layer=None):
+    """Decode the workload's query row on the GPU and check it against the oracle.
+
+    Returns a dict of GPU outputs and the per-(b, h) comparison summaries.
+    """
+    import torch
+
+    from long_context_sparse_idx16_b200 import Layer
+
+    s = x.spec
+    N = s.n_total
+    p = s.top_p if top_p is None else top_p
+    own = layer is None
+    if own:
+        layer = Layer.from_spec(s, x, max_seq=N, max_chunk=1, max_select=max_select)
+        build_cache(layer, x, N)
+    else:
+        layer.set_top_p(p)
+    layer.set_top_p(p)
+    q = torch_bf16(x.q[:, 0])
+    cap = N if sel_cap is None else sel_cap
+    out, st = layer.decode(q, stats=True, sel_cap=cap)
+    assert layer.check() == 0, "kernel error word set"
+    out = out.cpu().numpy()
+    cnt = st[0].cpu().numpy() if st else None
+    mass = st[1].cpu().numpy() if st else None
+    idx = st[3].cpu().numpy() if st else None
+    heads = range(s.n_q_heads) if heads is None else heads
+    batches = range(s.batch) if batches is None else batches
+    refs, gpus = [], []
+    summary = {}
+    for b in batches:
+        for h in heads:
+            r = oracle.layer_rows(x, b, h, [0], top_p=p, want_pi=h in s.retrieval_heads)
+            refs.append(r.out[0])
+            gpus.append(out[b, h])
+            if h in s.retrieval_heads:
+                slot = s.retrieval_heads.index(h)
+                k = int(cnt[b, slot])
+                sel = idx[b, slot, :k].astype(np.int64)
+                assert np.all(np.diff(sel) > 0), "selected positions must be strictly ascending"
+                nd = check_selection(sel, r, 0, p, f"b={b} h={h}")
+                assert abs(float(mass[b, slot]) - float(r.pi[0][sel].sum())) <= 1e-5
+                summary[(b, h)] = (k, int(r.count[0]), nd)
+    err = check_outputs(np.stack(gpus), np.stack(refs), f"{s.name} p={p}")
+    if own:
+        layer.close()
+    return {"out": out, "count": cnt, "summary": summary, "err": err}

@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every entry point include/*.h declares, lays out its
+structs as a C compiler does, and rejects bad arguments on the host (no GPU needed)."""
+import ctypes as C
+import glob
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import long_context_sparse_idx16_b200 as rtp
+from long_context_sparse_idx16_b200 import build as rtp_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rtp_build.build()
+    return rtp.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b(rtp_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "rtp_create" in names and "rtp_prefill_chunk" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", rtp.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\b(rtp_\w+)\b", out))
+    assert set(names) <= exported
+
+
+def test_struct_layout_matches_c():
+    src = r'''
+#include <stddef.h>
+#include <stdio.h>
+#include "rtp.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(rtp_config), offsetof(rtp_config, max_seq),
+         offsetof(rtp_config, rope_base), offsetof(rtp_config, wq_index),
+         offsetof(rtp_config, max_select), offsetof(rtp_config, max_chunk));
+  printf("%zu %zu %zu\n", sizeof(rtp_decode_stats), offsetof(rtp_decode_stats, sel_index_cap),
+         sizeof(rtp_cache_view));
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "p.c")
+        open(c, "w").write(src)
+        exe = os.path.join(d, "p")
+        subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include", c, "-o", exe])
+        a, b = subprocess.check_output([exe], text=True).splitlines()
+    cfg = rtp.rtp_config
+    assert [int(t) for t in a.split()] == [C.sizeof(cfg), cfg.max_seq.offset, cfg.rope_base.offset,
+                                          cfg.wq_index.offset, cfg.max_select.offset, cfg.max_chunk.offset]
+    st = rtp.rtp_decode_stats
+    assert [int(t) for t in b.split()] == [C.sizeof(st), st.sel_index_cap.offset, C.sizeof(rtp.rtp_cache_view)]
+
+
+def _cfg(**kw):
+    import numpy as np
+
+    hc = np.array([1, 0, 0, 0], dtype=np.uint8)
+    w = np.zeros((1, 128, 16), dtype=np.float32)
+    base = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, index_dim=16, max_seq=64,
+                head_class=hc.ctypes.data, top_p=0.9, window=8, n_sink=2, rope_base=1e6, sm_scale=0.0,
+                wq_index=w.ctypes.data, wk_index=w.ctypes.data, max_select=0, max_chunk=0)
+    base.update(kw)
+    return rtp.rtp_config(**base), (hc, w)
+
+
+@pytest.mark.parametrize("bad", [dict(head_dim=64), dict(index_dim=8), dict(top_p=0.0), dict(top_p=1.5),
+                                 dict(n_kv_heads=3), dict(window=0), dict(n_sink=-1), dict(max_seq=0),
+                                 dict(max_select=65), dict(batch=0), dict(head_class=None),
+                                 dict(n_q_heads=64, n_kv_heads=2), dict(rope_base=1.0)])
+def test_create_rejects_bad_config_on_host(lib, bad):
+    cfg, keep = _cfg(**bad)
+    h = C.c_void_p()
+    st = lib.rtp_create(C.byref(cfg), C.byref(h))
+    assert st == rtp.RTP_EINVAL
+    assert h.value is None
+    assert rtp.rtp_last_error(None).startswith("rtp_create")
+
+
+def test_calls_on_null_layer_are_rejected(lib):
+    assert lib.rtp_append_kv(None, None, None, 1, None) == rtp.RTP_EINVAL
+    assert lib.rtp_decode(None, None, None, None, None) == rtp.RTP_EINVAL
+    assert lib.rtp_prefill_chunk(None, None, 1, None, None, None) == rtp.RTP_EINVAL
+    assert lib.rtp_set_top_p(None, 0.5) == rtp.RTP_EINVAL
+    assert lib.rtp_seq_len(None) == -1
+    assert lib.rtp_destroy(None) == rtp.RTP_OK
+    assert lib.rtp_create(None, None) == rtp.RTP_EINVAL
