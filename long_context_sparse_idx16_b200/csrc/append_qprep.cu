@@ -36,13 +36,7 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
   const __nv_bfloat16* kt = k + ((int64_t)b * T + t) * Hkv * kD;
   const __nv_bfloat16* vt = v + ((int64_t)b * T + t) * Hkv * kD;
   for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) ks[i] = __bfloat162float(kt[i]);
-  if (threadIdx.x < kHalfD) {
-    double a = (double)pos * theta[threadIdx.x];
-    double s_, c_;
-    sincos(a, &s_, &c_);
-    cs[threadIdx.x] = (float)c_;
-    sn[threadIdx.x] = (float)s_;
-  }
+  if (threadIdx.x < kHalfD) rope_cos_sin(pos, theta[threadIdx.x], &cs[threadIdx.x], &sn[threadIdx.x]);
   __syncthreads();
 
   bool bad = false;
@@ -76,49 +70,56 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
   if (bad) atomicOr(err, kErrRange);
 }
 
-// One CTA per (row, batch): RoPE'd fp32 query for every head, pre-RoPE index query for the
-// retrieval heads.
+// One CTA per (row, batch, group of kQHeads heads): RoPE'd fp32 query for each head, and the
+// pre-RoPE index query Wq_h^T q for the retrieval heads among them.
+constexpr int kQHeads = 4;
+
 __global__ void __launch_bounds__(128) q_prep_kernel(
     const __nv_bfloat16* __restrict__ q, int rows, int Hq, int Hr, int64_t pos0,
     const double* __restrict__ theta, const float* __restrict__ wq,
-    const int16_t* __restrict__ ret_head, float* __restrict__ q_rot, float* __restrict__ q_idx) {
-  const int i = blockIdx.x, b = blockIdx.y;
+    const int16_t* __restrict__ head_slot, float* __restrict__ q_rot, float* __restrict__ q_idx) {
+  const int i = blockIdx.x, b = blockIdx.y, h0 = blockIdx.z * kQHeads;
   const int64_t pos = pos0 + i;
+  const int d = threadIdx.x;
   __shared__ float cs[kHalfD], sn[kHalfD];
-  __shared__ float qs[kD];
-  if (threadIdx.x < kHalfD) {
-    double a = (double)pos * theta[threadIdx.x];
-    double s_, c_;
-    sincos(a, &s_, &c_);
-    cs[threadIdx.x] = (float)c_;
-    sn[threadIdx.x] = (float)s_;
-  }
-  __syncthreads();
+  __shared__ float qs[kQHeads][kD];
   const int64_t row = (int64_t)b * rows + i;
   const __nv_bfloat16* qr = q + row * Hq * kD;
-  for (int h = 0; h < Hq; ++h) {
-    const float x = __bfloat162float(qr[h * kD + threadIdx.x]);
-    const float xp = __bfloat162float(qr[h * kD + (threadIdx.x ^ kHalfD)]);
-    const int c = threadIdx.x & (kHalfD - 1);
-    // first half: x*cos - partner*sin; second half: x*cos + partner*sin
-    const float y = threadIdx.x < kHalfD ? x * cs[c] - xp * sn[c] : x * cs[c] + xp * sn[c];
-    q_rot[(row * Hq + h) * kD + threadIdx.x] = y;
+  float x[kQHeads], xp[kQHeads];
+#pragma unroll
+  for (int u = 0; u < kQHeads; ++u) {
+    const int h = h0 + u;
+    x[u] = h < Hq ? __bfloat162float(qr[h * kD + d]) : 0.f;
+    xp[u] = h < Hq ? __bfloat162float(qr[h * kD + (d ^ kHalfD)]) : 0.f;
   }
-  for (int hr = 0; hr < Hr; ++hr) {
-    const int h = ret_head[hr];
-    __syncthreads();
-    qs[threadIdx.x] = __bfloat162float(qr[h * kD + threadIdx.x]);
-    __syncthreads();
-    // 16 outputs x 8 partial sums of 16 dims each
-    const int c = threadIdx.x >> 3, part = threadIdx.x & 7;
-    const float* w = wq + (int64_t)hr * kD * kR + c;
+  if (d < kHalfD) rope_cos_sin(pos, theta[d], &cs[d], &sn[d]);
+#pragma unroll
+  for (int u = 0; u < kQHeads; ++u) qs[u][d] = x[u];
+  __syncthreads();
+  const int c = d & (kHalfD - 1);
+#pragma unroll
+  for (int u = 0; u < kQHeads; ++u) {
+    const int h = h0 + u;
+    if (h >= Hq) break;
+    // first half: x*cos - partner*sin; second half: x*cos + partner*sin
+    const float y = d < kHalfD ? x[u] * cs[c] - xp[u] * sn[c] : x[u] * cs[c] + xp[u] * sn[c];
+    q_rot[(row * Hq + h) * kD + d] = y;
+  }
+  // index queries: 16 outputs x 8 partial sums of 16 dims each
+  const int o = d >> 3, part = d & 7;
+  for (int u = 0; u < kQHeads; ++u) {
+    const int h = h0 + u;
+    if (h >= Hq) break;
+    const int hr = head_slot[h];
+    if (hr < 0) continue;
+    const float* w = wq + (int64_t)hr * kD * kR + o;
     float acc = 0.f;
 #pragma unroll
-    for (int d = part * 16; d < part * 16 + 16; ++d) acc = fmaf(w[d * kR], qs[d], acc);
+    for (int e = part * 16; e < part * 16 + 16; ++e) acc = fmaf(w[e * kR], qs[u][e], acc);
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
     acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-    if (part == 0) q_idx[(row * Hr + hr) * kR + c] = acc;
+    if (part == 0) q_idx[(row * Hr + hr) * kR + o] = acc;
   }
 }
 
@@ -136,8 +137,8 @@ cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const _
 
 cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, int64_t pos0,
                           cudaStream_t st) {
-  dim3 grid(rows, L->B);
-  q_prep_kernel<<<grid, 128, 0, st>>>(q, rows, L->Hq, L->Hr, pos0, L->theta, L->wq, L->d_ret_head,
+  dim3 grid(rows, L->B, (L->Hq + kQHeads - 1) / kQHeads);
+  q_prep_kernel<<<grid, 128, 0, st>>>(q, rows, L->Hq, L->Hr, pos0, L->theta, L->wq, L->d_head_slot,
                                       L->q_rot, L->q_idx);
   return cudaGetLastError();
 }

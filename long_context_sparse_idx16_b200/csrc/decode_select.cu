@@ -5,30 +5,42 @@
 //      scores s_j = qidx . IDX[p][j] (techwalker page, section 3: the 16-dim "radar");
 //   2. finds the exact top-p set: the shortest prefix of the order (s desc, j asc) whose
 //      index-softmax mass reaches p (zhichai page, insight 3; techwalker page, section 4),
-//      without sorting -- by mass histograms, as the pages' kernel does (techwalker page,
-//      section 6: 256 buckets, no sort, fused with scoring), refined until the cut is exact;
+//      without a full sort -- by a mass histogram, as the pages' kernel does (techwalker
+//      page, section 6: buckets instead of sorting, fused with scoring), refined until the
+//      cut is exact;
 //   3. writes the selected positions in ascending order.
 //
 // B200 design
 //   * One cooperative grid of <= #SM CTAs x 1024 threads.  The flat (problem, key) range is
-//     split evenly; each CTA keeps its scores in shared memory (up to ~50K per CTA, 7.4M per
-//     launch), so the histogram passes never touch HBM again.  Larger launches keep the
-//     scores in a global scratch array (L2-resident at these sizes) instead.
-//   * The index stream uses 16-byte non-allocating loads: four threads own one 64-byte row,
-//     so every warp load is a fully coalesced 512-byte segment.
-//   * Softmax masses are exp(s - m) in fp32, quantised to 64-bit fixed point (2^sc scale with
-//     N * 2^sc < 2^63).  Integer sums are exact and associative, so the selection is
-//     deterministic and identical however the work is split; integer atomics build the
-//     histograms.  The quantisation error on the total mass is below N * 2^-(sc+1)
-//     (< 1.2e-7 of the largest key's mass at N = 2^20).
-//   * Level 1: 2048 bins of width 1/64 in (m - s) (last bin: everything 32 or more below
-//     the max).  Levels 2-4: radix digits (11, 11, 10 bits) of the order-preserving key bits
-//     of the elements in the crossing bin.  Each level stops early when its crossing group
-//     holds a single key.  After the last level the cut score t is exact; ties at t are
-//     taken in ascending position order.
-//   * Grid barriers are bounded waits (about 1 s); on timeout the error word records
-//     RTP_ETIMEOUT and the kernel returns.
-#include <cooperative_groups.h>
+//     split evenly; each CTA keeps its scores in shared memory (up to ~47K per CTA, ~7M per
+//     launch), so the selection passes never touch HBM again.  Larger launches keep the
+//     scores in a global scratch array instead.
+//   * The index stream uses 16-byte non-allocating loads, eight in flight per thread: four
+//     threads own one 64-byte row, so every warp load is a fully coalesced 512-byte segment.
+//   * Masses are exp(s - m) in fp32, quantised to 64-bit fixed point (scale 2^sc with
+//     N * 2^sc <= 2^62) and accumulated with 32-bit integer atomics (low word with carry into
+//     the high word): integer sums are exact and order-independent, so the selection is
+//     deterministic however the work is split.  The quantisation error on the total mass is
+//     below N * 2^-(sc+1) of the largest key's mass (< 1.2e-7 at N = 2^20).
+//   * Level 1: 1024 bins of width 1/64 for (m - s) < 16 (shared atomics, and the key joins its
+//     warp's ordered keep list), one coarse bin for 16..32 (per-thread register sums: no atomics
+//     for the bulk of the keys).  Later passes walk only the keep lists.  Keys 32 or more below
+//     the max are never counted: each carries at most e^-32 of the top key's mass, their
+//     quantised mass is 0 whenever N > 2^16, and for smaller N their total stays below
+//     (1 - p) * Z for every fp32 p < 1 (1 - p >= 2^-24), so they can never be needed to reach
+//     p and the cut never falls among them.
+//   * The keys of the crossing bin (usually a handful, at most 1024 on the fast path) are
+//     gathered into a list that every CTA of the problem sorts in shared memory (bitonic, warp
+//     shuffles below distance 32) to locate the exact cut key t and how many keys tied at t
+//     are taken (lowest positions first).  Larger crossing bins (massive exact ties) fall back
+//     to three radix levels over the key bits, 11/11/10 bits.
+//   * After the cut the selection is a key comparison: key > t, or key == t among the first
+//     n_need tied positions.  Ordered compaction is two ballot passes per warp.
+//   * Four grid barriers on the fast path (max, histogram, candidates, counts), three more on
+//     the fallback.  Every barrier wait is bounded (about 1 s); on timeout the error word records
+//     RTP_ETIMEOUT and the kernel returns.  Scratch histograms are zeroed by the launch that
+//     last read them, so a launch starts on clean scratch without a memset.
+#include <type_traits>
 
 #include "rtp_device.cuh"
 #include "rtp_internal.h"
@@ -40,10 +52,20 @@ namespace {
 constexpr int kBins = kSelBins;
 constexpr int kThreads = kSelThreads;
 constexpr int kWarps = kThreads / 32;
+constexpr int kCand = kSelCand;  // crossing-bin keys resolved by sorting
 constexpr float kLog2e = 1.4426950408889634f;
-// radix levels inside the crossing bin: key bits [31:21], [20:10], [9:0]
+constexpr int kUnroll = 8;  // 16-byte loads in flight per thread in the index stream
+constexpr int kFine = 1024;  // level-1 bins of width 1/64 covering (m - s) in [0, 16); bin kFine: [16, 32)
+
+// radix fallback inside the crossing bin: key bits [31:21], [20:10], [9:0]
 __device__ __forceinline__ int level_shift(int l) { return l == 0 ? 21 : (l == 1 ? 10 : 0); }
 __device__ __forceinline__ int level_bits(int l) { return l == 2 ? 10 : 11; }
+
+struct Hist3 {  // a 2048-bin mass histogram in global memory: exact 64-bit mass as (hi, lo) words
+  uint32_t* lo;
+  uint32_t* hi;
+  uint32_t* cnt;
+};
 
 struct SelectArgs {
   const float* idx;
@@ -59,47 +81,108 @@ struct SelectArgs {
   int32_t* sel_cnt;
   float* sel_mass;
   float* sel_thr;
-  float* seg_max;  // [P + G]
-  unsigned long long* h1_mass;
-  uint32_t* h1_cnt;
-  unsigned long long* hr_mass;  // [3][P][bins]
-  uint32_t* hr_cnt;
-  uint32_t* slot_cnt;  // [P + G][2]
-  uint32_t* bar;
+  float* seg_max;     // [P + G]
+  Hist3 h1;           // [P][bins]
+  Hist3 hr;           // [3][P][bins] radix fallback levels
+  uint32_t* cand_cnt;         // [P]
+  unsigned long long* cand;   // [P][kCand] packed (key << 32) | ~j
+  uint32_t* slot_cnt;         // [P + G][2]: (gt, eq) per (problem, CTA)
+  unsigned long long* bar;    // [2]: grid barrier arrival counter (monotonic), exit counter
+  uint32_t* keep;             // global keep lists when the scores live in global memory
+  uint32_t* flags;            // [1]: some problem needs the radix fallback
   uint32_t* err;
   float* gscores;
 };
 
 struct Seg {
   int p;
-  int done;      // 1 once the tie group is known
-  int shift_f;   // 32: tie group = the whole crossing bin; else key >> shift_f == prefix
+  int radix;     // 1: crossing bin too large for the candidate list (fallback path)
+  int full;      // 1: a warp's keep list overflowed; later passes scan the whole chunk
+  int kbase;     // this segment's keep lists start at keep[kbase]; warp w at + w * kcap
+  int kcap;      // keep-list capacity per warp
   int bstar;
+  uint32_t prefix;
   int64_t jlo, jhi, off;
   float m;
-  uint32_t prefix;
-  unsigned long long Z, T, rem, e_t, n_need;
+  uint32_t t_key;
+  unsigned long long Z, T, rem, e_t, n_need, msel;
 };
 
 struct Smem {
-  unsigned long long hm[kBins];
+  union {
+    struct {
+      uint32_t lo[kBins];
+      uint32_t hi[kBins];
+    } w;
+    unsigned long long m[kBins];
+  } h;
   uint32_t hc[kBins];
+  unsigned long long sk[kCand];
   Seg seg[kSelMaxSeg];
   unsigned long long red64[kWarps];
   uint32_t red32[kWarps];
   float redf[kWarps];
-  int cross;
-  unsigned long long cross_above;
+  uint32_t wcnt[kSelMaxSeg][kWarps][2];  // (gt, eq) per warp chunk, then exclusive bases
+  uint32_t lcnt[kSelMaxSeg][kWarps];     // keep-list length per warp chunk
+  uint32_t slot[2 * kSelMaxGrid];
+  int cross, cut_idx;
+  unsigned long long cross_above, cut_cum;
   long long before, take;
-  uint32_t slot[2 * kThreads];  // (gt, eq) counts of the CTAs that share a problem
 };
 
-__device__ __forceinline__ unsigned long long mass_of(float s, float m, float scale) {
-  return __float2ull_rn(fast_exp2((s - m) * kLog2e) * scale);
+// ---------------------------------------------------------------- small helpers
+
+// Fixed-point mass of a score: round(2^sc * exp(s - m)), as (hi, lo) 32-bit words.
+__device__ __forceinline__ void mass_words(float s, float m, float scale, uint32_t* hi, uint32_t* lo) {
+  const float q = fast_exp2((s - m) * kLog2e) * scale;  // < 2^63; an integer once >= 2^24
+  const float qh = floorf(q * 2.3283064365386963e-10f);  // q / 2^32
+  *hi = (uint32_t)qh;
+  *lo = __float2uint_rn(fmaf(qh, -4294967296.0f, q));
+}
+__device__ __forceinline__ unsigned long long mass64(float s, float m, float scale) {
+  uint32_t hi, lo;
+  mass_words(s, m, scale, &hi, &lo);
+  return ((unsigned long long)hi << 32) | lo;
 }
 __device__ __forceinline__ int bin_of(float s, float m) {
-  int b = (int)((m - s) * 64.f);
-  return b < kBins - 1 ? b : kBins - 1;
+  const float x = m - s;  // >= 0; NaN lands in the tail
+  if (x < 16.f) return (int)(x * 64.f);
+  if (x < 32.f) return kFine;
+  return kBins - 1;
+}
+
+// exact 64-bit add into a (hi, lo) pair of 32-bit counters with 32-bit atomics
+__device__ __forceinline__ void add_words(uint32_t* lo_w, uint32_t* hi_w, uint32_t hi, uint32_t lo) {
+  const uint32_t old = atomicAdd(lo_w, lo);
+  const uint32_t carry = (old + lo < old) ? 1u : 0u;
+  if (hi + carry) atomicAdd(hi_w, hi + carry);
+}
+
+// Monotonic grid barrier: one atomic per CTA on a 64-bit counter that only grows, then an
+// acquire spin until the counter reaches the next multiple of the grid size.  Bounded.
+__device__ __forceinline__ bool grid_sync(unsigned long long* bar, uint32_t nblocks, uint32_t* err) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    const unsigned long long old = atomicAdd(bar, 1ull);
+    const unsigned long long target = (old / nblocks + 1) * nblocks;
+    const long long t0 = clock64();
+    while (true) {
+      unsigned long long v;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(bar) : "memory");
+      if (v >= target) break;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicOr(err, kErrTimeout);
+        ok = 0;
+        break;
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
 }
 
 __device__ float block_max(float v, Smem& S) {
@@ -109,7 +192,7 @@ __device__ float block_max(float v, Smem& S) {
   if (l == 0) S.redf[w] = v;
   __syncthreads();
   if (w == 0) {
-    v = l < kWarps ? S.redf[l] : -INFINITY;
+    v = S.redf[l];
     v = warp_max(v);
     if (l == 0) S.redf[0] = v;
   }
@@ -124,7 +207,7 @@ __device__ unsigned long long block_sum_u64(unsigned long long v, Smem& S) {
   if (l == 0) S.red64[w] = v;
   __syncthreads();
   if (w == 0) {
-    v = l < kWarps ? S.red64[l] : 0ull;
+    v = S.red64[l];
     v = warp_sum(v);
     if (l == 0) S.red64[0] = v;
   }
@@ -132,15 +215,10 @@ __device__ unsigned long long block_sum_u64(unsigned long long v, Smem& S) {
   return S.red64[0];
 }
 
-// In S.hm order (reverse: index kBins-1 first), find the first position whose inclusive
-// cumulative mass reaches target.  Result: S.cross = bin, S.cross_above = mass before it.
-__device__ void find_crossing(Smem& S, bool reverse, unsigned long long target) {
+// Inclusive block scan of one u64 per thread (thread order); returns the inclusive value.
+__device__ unsigned long long block_incl_scan_u64(unsigned long long v, Smem& S) {
   const int t = threadIdx.x, w = t >> 5, l = t & 31;
-  const int p0 = 2 * t, p1 = 2 * t + 1;
-  const int b0 = reverse ? kBins - 1 - p0 : p0;
-  const int b1 = reverse ? kBins - 1 - p1 : p1;
-  const unsigned long long m0 = S.hm[b0], m1 = S.hm[b1];
-  unsigned long long incl = m0 + m1;
+  unsigned long long incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -148,7 +226,6 @@ __device__ void find_crossing(Smem& S, bool reverse, unsigned long long target) 
   }
   __syncthreads();
   if (l == 31) S.red64[w] = incl;
-  if (t == 0) S.cross = -1;
   __syncthreads();
   if (w == 0) {
     unsigned long long x = S.red64[l];
@@ -157,10 +234,23 @@ __device__ void find_crossing(Smem& S, bool reverse, unsigned long long target) 
       unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
       if (l >= o) x += y;
     }
-    S.red64[l] = x;  // inclusive warp totals
+    S.red64[l] = x;
   }
   __syncthreads();
-  const unsigned long long base = (w > 0 ? S.red64[w - 1] : 0ull) + incl - (m0 + m1);
+  return (w > 0 ? S.red64[w - 1] : 0ull) + incl;
+}
+
+// In S.h.m order (reverse: index kBins-1 first), find the first position whose inclusive
+// cumulative mass reaches target.  Result: S.cross = bin (-1 if none), S.cross_above = mass
+// before it.
+__device__ void find_crossing(Smem& S, bool reverse, unsigned long long target) {
+  const int t = threadIdx.x;
+  const int b0 = reverse ? kBins - 1 - 2 * t : 2 * t;
+  const int b1 = reverse ? b0 - 1 : b0 + 1;
+  const unsigned long long m0 = S.h.m[b0], m1 = S.h.m[b1];
+  if (t == 0) S.cross = -1;
+  const unsigned long long incl = block_incl_scan_u64(m0 + m1, S);
+  const unsigned long long base = incl - (m0 + m1);
   if (base < target && base + m0 >= target) {
     S.cross = b0;
     S.cross_above = base;
@@ -171,57 +261,69 @@ __device__ void find_crossing(Smem& S, bool reverse, unsigned long long target) 
   __syncthreads();
 }
 
-__device__ __forceinline__ void zero_smem_hist(Smem& S) {
+__device__ __forceinline__ void zero_words(Smem& S) {
   for (int i = threadIdx.x; i < kBins; i += kThreads) {
-    S.hm[i] = 0ull;
+    S.h.w.lo[i] = 0u;
+    S.h.w.hi[i] = 0u;
     S.hc[i] = 0u;
   }
 }
 
-__device__ __forceinline__ void flush_hist(Smem& S, unsigned long long* gm, uint32_t* gc) {
+__device__ __forceinline__ void flush_words(Smem& S, const Hist3& g, int64_t base) {
   for (int i = threadIdx.x; i < kBins; i += kThreads) {
     const uint32_t c = S.hc[i];
     if (c) {
-      atomicAdd(gm + i, S.hm[i]);
-      atomicAdd(gc + i, c);
+      add_words(g.lo + base + i, g.hi + base + i, S.h.w.hi[i], S.h.w.lo[i]);
+      atomicAdd(g.cnt + base + i, c);
     }
   }
 }
 
-__device__ __forceinline__ void load_hist(Smem& S, const unsigned long long* gm, const uint32_t* gc) {
+// Load a global histogram as 64-bit masses + counts (then synchronise).
+__device__ __forceinline__ void load_hist(Smem& S, const Hist3& g, int64_t base) {
   for (int i = threadIdx.x; i < kBins; i += kThreads) {
-    S.hm[i] = __ldcg(gm + i);
-    S.hc[i] = __ldcg(gc + i);
+    const uint32_t lo = __ldcg(g.lo + base + i), hi = __ldcg(g.hi + base + i);
+    S.hc[i] = __ldcg(g.cnt + base + i);
+    S.h.m[i] = ((unsigned long long)hi << 32) | lo;
   }
   __syncthreads();
 }
 
-// Exclusive block scan of a packed (gt << 16 | eq) counter; returns the exclusive prefix,
-// total in *tot.
-__device__ uint32_t block_scan_u32(uint32_t v, Smem& S, uint32_t* tot) {
-  const int t = threadIdx.x, w = t >> 5, l = t & 31;
-  uint32_t incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (l >= o) incl += y;
+__device__ __forceinline__ void zero_global_hist(const Hist3& g, int64_t n, int c, uint32_t G) {
+  for (int64_t i = (int64_t)c * kThreads + threadIdx.x; i < n; i += (int64_t)G * kThreads) {
+    g.lo[i] = 0u;
+    g.hi[i] = 0u;
+    g.cnt[i] = 0u;
   }
-  __syncthreads();
-  if (l == 31) S.red32[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    uint32_t x = S.red32[l];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (l >= o) x += y;
-    }
-    S.red32[l] = x;
-  }
-  __syncthreads();
-  *tot = S.red32[kWarps - 1];
-  return (w > 0 ? S.red32[w - 1] : 0u) + incl - v;
 }
+
+// Sort S.sk[0..n) descending (n a power of two, 32 <= n <= kCand); thread t ends with element t.
+__device__ unsigned long long bitonic_desc(Smem& S, int n, unsigned long long v) {
+  const int t = threadIdx.x;
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      unsigned long long pv;
+      if (j >= 32) {
+        __syncthreads();
+        if (t < n) S.sk[t] = v;
+        __syncthreads();
+        pv = t < n ? S.sk[t ^ j] : 0ull;
+      } else {
+        pv = __shfl_xor_sync(0xffffffffu, v, j);
+      }
+      const bool desc = (t & k) == 0;
+      const bool lower = (t & j) == 0;
+      const unsigned long long hi_v = v > pv ? v : pv, lo_v = v > pv ? pv : v;
+      v = (lower == desc) ? hi_v : lo_v;
+    }
+  }
+  return v;
+}
+
+// first CTA that holds keys of problem p
+__device__ __forceinline__ int cf_of(int p, const SelectArgs& a) { return (int)(((int64_t)p * a.N) / a.L); }
+
+// ---------------------------------------------------------------- the kernel
 
 template <bool kSmemScores>
 __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a) {
@@ -229,14 +331,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
   const int c = blockIdx.x;
   const uint32_t G = gridDim.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t total = (int64_t)a.P * a.N;
   const int64_t r0 = (int64_t)c * a.L;
   const int64_t r1 = min(total, r0 + a.L);
   float* sc = kSmemScores ? reinterpret_cast<float*>(smem_raw + sizeof(Smem)) : a.gscores + r0;
+  // Keep lists: 16-bit in shared memory after the scores, 32-bit in global memory otherwise.
+  using KeepT = typename std::conditional<kSmemScores, uint16_t, uint32_t>::type;
+  KeepT* keep = kSmemScores ? reinterpret_cast<KeepT*>(smem_raw + sizeof(Smem) + 4 * ((a.L + 3) / 4 * 4))
+                            : reinterpret_cast<KeepT*>(a.keep + r0);
   const float scale = __uint_as_float((uint32_t)(127 + a.sc_bits) << 23);  // 2^sc
+  const int64_t nh = (int64_t)a.P * kBins;
 
-  // ---- segments of this CTA
+  // ---- segments of this CTA: [jlo, jhi) of problem p, stored at sc[off ...]
   int nseg = 0;
   if (r0 < r1) {
     const int p_first = (int)(r0 / a.N), p_last = (int)((r1 - 1) / a.N);
@@ -247,27 +354,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
       s.jlo = max((int64_t)0, r0 - (int64_t)s.p * a.N);
       s.jhi = min(a.N, r1 - (int64_t)s.p * a.N);
       s.off = (int64_t)s.p * a.N + s.jlo - r0;
-      s.done = 0;
-      s.shift_f = 32;
+      s.radix = 0;
+      s.full = 0;
       s.prefix = 0;
     }
   }
   __syncthreads();
-
-  // ---- phase A: zero global histograms; stream index keys -> scores, segment maxima
-  {
-    const int64_t nh = (int64_t)a.P * kBins;
-    for (int64_t i = (int64_t)c * kThreads + tid; i < nh; i += (int64_t)G * kThreads) {
-      a.h1_mass[i] = 0ull;
-      a.h1_cnt[i] = 0u;
-      a.hr_mass[i] = 0ull;
-      a.hr_cnt[i] = 0u;
-      a.hr_mass[nh + i] = 0ull;
-      a.hr_cnt[nh + i] = 0u;
-      a.hr_mass[2 * nh + i] = 0ull;
-      a.hr_cnt[2 * nh + i] = 0u;
+  if (tid == 0) {  // per-warp keep capacity: a quarter of the warp chunk, rounded up
+    int acc = 0;
+    for (int si = 0; si < nseg; ++si) {
+      const int rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
+      const int wlen = (rows + kWarps - 1) / kWarps;
+      S.seg[si].kcap = (wlen + 3) / 4;
+      S.seg[si].kbase = acc;
+      acc += kWarps * S.seg[si].kcap;
     }
   }
+  __syncthreads();
+
+  // ---- phase A: stream index keys -> scores, segment maxima
   const int quad = tid >> 2, part = tid & 3;
   for (int si = 0; si < nseg; ++si) {
     const Seg s = S.seg[si];
@@ -277,16 +382,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     float mx = -INFINITY;
     // The trip count is the same for every thread (the shuffles below are full-warp);
     // rows past the end are loaded as zeros and not stored.
-    for (int64_t base = 0; base < rows; base += 4 * (kThreads / 4)) {
+    for (int64_t base = 0; base < rows; base += kUnroll * (kThreads / 4)) {
       const int64_t k0 = base + quad;
-      float4 v[4];
+      float4 v[kUnroll];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kUnroll; ++u) {
         const int64_t k = k0 + u * (kThreads / 4);
         v[u] = k < rows ? ld_stream_f4(src + k * 4 + part) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kUnroll; ++u) {
         float d = v[u].x * qv.x;
         d = fmaf(v[u].y, qv.y, d);
         d = fmaf(v[u].z, qv.z, d);
@@ -304,182 +409,316 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     mx = block_max(mx, S);
     if (tid == 0) a.seg_max[s.p + c] = mx;
   }
-  if (!grid_barrier(a.bar, a.bar + 1, G, a.err)) return;
+  if (!grid_sync(a.bar, G, a.err)) return;
 
-  // ---- phase B: row maxima; level-1 mass histograms
+  // ---- phase B: row maxima; level-1 mass histogram; keep lists.  Warp w walks a contiguous
+  // chunk of the segment.  Keys within 16 of the max join the warp's ordered keep list (their
+  // fine-bin masses are added afterwards from the list, every lane busy); keys 16..32 below the
+  // max add their exact mass to a per-thread register sum for the single coarse bin.
+  const bool small_mass = a.sc_bits <= 54;  // then every coarse-bin mass fits 32 bits
   for (int si = 0; si < nseg; ++si) {
     const int p = S.seg[si].p;
-    const int cf = (int)(((int64_t)p * a.N) / a.L), cl = (int)(((int64_t)p * a.N + a.N - 1) / a.L);
+    const int cf = cf_of(p, a), cl = (int)(((int64_t)p * a.N + a.N - 1) / a.L);
     float mv = -INFINITY;
     for (int cc = cf + tid; cc <= cl; cc += kThreads) mv = fmaxf(mv, __ldcg(a.seg_max + p + cc));
     const float m = block_max(mv, S);
-    zero_smem_hist(S);
+    zero_words(S);
     if (tid == 0) S.seg[si].m = m;
     __syncthreads();
-    const Seg& s = S.seg[si];
-    const int64_t rows = s.jhi - s.jlo;
-    for (int64_t k = tid; k < rows; k += kThreads) {
-      const float v = sc[s.off + k];
-      const int b = bin_of(v, m);
-      atomicAdd(&S.hm[b], mass_of(v, m, scale));
-      atomicAdd(&S.hc[b], 1u);
-    }
-    __syncthreads();
-    flush_hist(S, a.h1_mass + (int64_t)p * kBins, a.h1_cnt + (int64_t)p * kBins);
-    __syncthreads();
-  }
-  if (!grid_barrier(a.bar, a.bar + 1, G, a.err)) return;
-
-  // ---- phase C: total mass, target, crossing bin; radix level 0 inside it
-  for (int si = 0; si < nseg; ++si) {
-    const int p = S.seg[si].p;
-    load_hist(S, a.h1_mass + (int64_t)p * kBins, a.h1_cnt + (int64_t)p * kBins);
-    unsigned long long part_sum = 0;
-    for (int i = tid; i < kBins; i += kThreads) part_sum += S.hm[i];
-    const unsigned long long Z = block_sum_u64(part_sum, S);
-    unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
-    if (T < 1ull) T = 1ull;
-    if (T > Z) T = Z;
-    find_crossing(S, false, T);
-    if (tid == 0) {
-      Seg& s = S.seg[si];
-      s.Z = Z;
-      s.T = T;
-      s.bstar = S.cross;
-      s.rem = T - S.cross_above;
-      if (S.cross < 0) {
-        atomicOr(a.err, kErrInternal);
-        s.bstar = 0;
-        s.rem = 1;
-      }
-      if (S.hc[s.bstar] == 1u) {  // a single key carries the cut
-        s.done = 1;
-        s.shift_f = 32;
-        s.e_t = S.hm[s.bstar];
-        s.n_need = 1;
-      }
-    }
-    __syncthreads();
-    const Seg& s = S.seg[si];
-    if (s.done) continue;
-    zero_smem_hist(S);
-    __syncthreads();
-    const int64_t rows = s.jhi - s.jlo;
-    for (int64_t k = tid; k < rows; k += kThreads) {
-      const float v = sc[s.off + k];
-      if (bin_of(v, s.m) != s.bstar) continue;
-      const uint32_t d = order_key(v) >> level_shift(0);
-      atomicAdd(&S.hm[d], mass_of(v, s.m, scale));
-      atomicAdd(&S.hc[d], 1u);
-    }
-    __syncthreads();
-    flush_hist(S, a.hr_mass + (int64_t)p * kBins, a.hr_cnt + (int64_t)p * kBins);
-    __syncthreads();
-  }
-  if (!grid_barrier(a.bar, a.bar + 1, G, a.err)) return;
-
-  // ---- phases D, E: radix levels 1 and 2 (after reading levels 0 and 1)
-  for (int lev = 1; lev <= 2; ++lev) {
-    const int64_t nh = (int64_t)a.P * kBins;
-    for (int si = 0; si < nseg; ++si) {
-      const Seg s0 = S.seg[si];
-      if (s0.done) continue;
-      const int p = s0.p;
-      load_hist(S, a.hr_mass + (lev - 1) * nh + (int64_t)p * kBins,
-                a.hr_cnt + (lev - 1) * nh + (int64_t)p * kBins);
-      find_crossing(S, true, s0.rem);
-      if (tid == 0) {
-        Seg& s = S.seg[si];
-        const int d = S.cross < 0 ? 0 : S.cross;
-        if (S.cross < 0) atomicOr(a.err, kErrInternal);
-        s.prefix = (lev == 1) ? (uint32_t)d : ((s.prefix << level_bits(lev - 1)) | (uint32_t)d);
-        s.rem -= S.cross_above;
-        s.shift_f = level_shift(lev - 1);
-        if (S.hc[d] == 1u) {
-          s.done = 1;
-          s.e_t = S.hm[d];
-          s.n_need = 1;
+    const int off = (int)S.seg[si].off, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
+    const int wlen = (rows + kWarps - 1) / kWarps;
+    const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
+    const int kcap = S.seg[si].kcap;
+    KeepT* kl = keep + S.seg[si].kbase + warp * kcap;
+    unsigned long long coarse = 0;
+    int nkeep = 0;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int k0 = w_lo; k0 < w_hi; k0 += 32) {
+      const int k = k0 + lane;
+      const float v = k < w_hi ? sc[off + k] : -INFINITY;
+      const float x = m - v;
+      const bool fine = x < 16.f;
+      if (!fine && x < 32.f) {
+        if (small_mass) {
+          coarse += __float2uint_rn(fast_exp2((v - m) * kLog2e) * scale);
+        } else {
+          coarse += mass64(v, m, scale);
         }
       }
-      __syncthreads();
-      const Seg& s = S.seg[si];
-      if (s.done) continue;
-      zero_smem_hist(S);
-      __syncthreads();
-      const int64_t rows = s.jhi - s.jlo;
-      for (int64_t k = tid; k < rows; k += kThreads) {
-        const float v = sc[s.off + k];
-        if (bin_of(v, s.m) != s.bstar) continue;
-        const uint32_t key = order_key(v);
-        if ((key >> s.shift_f) != s.prefix) continue;
-        const uint32_t d = (key >> level_shift(lev)) & ((1u << level_bits(lev)) - 1u);
-        atomicAdd(&S.hm[d], mass_of(v, s.m, scale));
-        atomicAdd(&S.hc[d], 1u);
+      const uint32_t bf = __ballot_sync(0xffffffffu, fine);
+      if (fine) {
+        const int pos = nkeep + __popc(bf & lt);
+        if (pos < kcap) {
+          kl[pos] = (KeepT)k;
+        } else {  // list full: count this key now
+          uint32_t hi, lo;
+          mass_words(v, m, scale, &hi, &lo);
+          add_words(&S.h.w.lo[(int)(x * 64.f)], &S.h.w.hi[(int)(x * 64.f)], hi, lo);
+        }
       }
-      __syncthreads();
-      flush_hist(S, a.hr_mass + lev * nh + (int64_t)p * kBins, a.hr_cnt + lev * nh + (int64_t)p * kBins);
-      __syncthreads();
+      nkeep += __popc(bf);
     }
-    if (!grid_barrier(a.bar, a.bar + 1, G, a.err)) return;
+    if (lane == 0) {
+      S.lcnt[si][warp] = (uint32_t)min(nkeep, kcap);
+      if (nkeep > kcap) S.seg[si].full = 1;
+    }
+    const int nl = min(nkeep, kcap);
+    __syncwarp();  // list entries written by other lanes of this warp
+    for (int i = lane; i < nl; i += 32) {
+      const float v = sc[off + (int)kl[i]];
+      const float x = m - v;
+      uint32_t hi, lo;
+      mass_words(v, m, scale, &hi, &lo);
+      add_words(&S.h.w.lo[(int)(x * 64.f)], &S.h.w.hi[(int)(x * 64.f)], hi, lo);
+    }
+    coarse = warp_sum(coarse);
+    if (lane == 0 && coarse) add_words(&S.h.w.lo[kFine], &S.h.w.hi[kFine], (uint32_t)(coarse >> 32), (uint32_t)coarse);
+    __syncthreads();
+    for (int i = tid; i <= kFine; i += kThreads) {
+      const uint32_t lo = S.h.w.lo[i], hi = S.h.w.hi[i];
+      if (lo | hi) add_words(a.h1.lo + (int64_t)p * kBins + i, a.h1.hi + (int64_t)p * kBins + i, hi, lo);
+    }
+    __syncthreads();
   }
+  if (!grid_sync(a.bar, G, a.err)) return;
 
-  // ---- phase F: exact cut from level 2; count keys above the tie group and in it
-  {
-    const int64_t nh = (int64_t)a.P * kBins;
-    for (int si = 0; si < nseg; ++si) {
-      const Seg s0 = S.seg[si];
-      const int p = s0.p;
-      if (!s0.done) {
-        load_hist(S, a.hr_mass + 2 * nh + (int64_t)p * kBins, a.hr_cnt + 2 * nh + (int64_t)p * kBins);
-        find_crossing(S, true, s0.rem);
+  // ---- phase C: total mass, target, crossing bin; its keys become candidates.  A crossing in
+  // the coarse bin, or more than kCand keys in the crossing bin, takes the radix fallback.
+  for (int si = 0; si < nseg; ++si) {
+    const int p = S.seg[si].p;
+    for (int i = tid; i < kBins; i += kThreads) {
+      uint32_t lo = 0, hi = 0;
+      if (i <= kFine) {
+        lo = __ldcg(a.h1.lo + (int64_t)p * kBins + i);
+        hi = __ldcg(a.h1.hi + (int64_t)p * kBins + i);
+      }
+      S.h.m[i] = ((unsigned long long)hi << 32) | lo;
+    }
+    __syncthreads();
+    {  // one scan gives Z (the total), then T, then the crossing bin
+      const unsigned long long m0 = S.h.m[2 * tid], m1 = S.h.m[2 * tid + 1];
+      if (tid == 0) S.cross = -1;
+      const unsigned long long incl = block_incl_scan_u64(m0 + m1, S);
+      const unsigned long long Z = S.red64[kWarps - 1];
+      unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
+      if (T < 1ull) T = 1ull;
+      if (T > Z) T = Z;
+      const unsigned long long base = incl - (m0 + m1);
+      if (base < T && base + m0 >= T) {
+        S.cross = 2 * tid;
+        S.cross_above = base;
+      } else if (base + m0 < T && base + m0 + m1 >= T) {
+        S.cross = 2 * tid + 1;
+        S.cross_above = base + m0;
+      }
+      if (tid == 0) {
+        S.seg[si].Z = Z;
+        S.seg[si].T = T;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      Seg& sg = S.seg[si];
+      if (S.cross < 0) {
+        atomicOr(a.err, kErrInternal);
+        S.cross = 0;
+        S.cross_above = 0;
+      }
+      sg.bstar = S.cross;
+      sg.rem = sg.T - S.cross_above;
+      // the coarse bin cannot be resolved from the keep lists: force the fallback
+      if (S.cross == kFine) {
+        atomicOr(a.flags, 1u);
+        if (c == cf_of(p, a)) atomicAdd(a.cand_cnt + p, (uint32_t)kCand + 1u);
+      }
+    }
+    __syncthreads();
+    const int bstar = S.seg[si].bstar;
+    if (bstar < kFine) {
+      const int off = (int)S.seg[si].off, jlo = (int)S.seg[si].jlo, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
+      const float m = S.seg[si].m;
+      const bool full = S.seg[si].full;
+      const int wlen = (rows + kWarps - 1) / kWarps;
+      const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
+      const KeepT* kl = keep + S.seg[si].kbase + warp * S.seg[si].kcap;
+      const int n_it = full ? (w_hi - w_lo) : (int)S.lcnt[si][warp];
+      for (int i = lane; i < n_it; i += 32) {
+        const int k = full ? w_lo + i : (int)kl[i];
+        const float v = sc[off + k];
+        if (bin_of(v, m) != bstar) continue;
+        const uint32_t slot = atomicAdd(a.cand_cnt + p, 1u);
+        if (slot < (uint32_t)kCand)
+          a.cand[(int64_t)p * kCand + slot] = ((unsigned long long)order_key(v) << 32) | (0xFFFFFFFFu - (uint32_t)(jlo + k));
+        else
+          atomicOr(a.flags, 1u);
+      }
+    }
+    __syncthreads();
+  }
+  if (!grid_sync(a.bar, G, a.err)) return;
+
+  // ---- phase D: exact cut.  Problems whose crossing bin fits the candidate list sort it;
+  // the others (decided identically by every CTA from the global counts) refine by radix.
+  if (tid == 0) S.cut_idx = (int)__ldcg(a.flags);
+  __syncthreads();
+  const bool fallback = S.cut_idx != 0;
+  __syncthreads();
+  for (int si = 0; si < nseg; ++si) {
+    const int p = S.seg[si].p;
+    // one round trip: the count and the candidate slots together
+    const unsigned long long vraw = tid < kCand ? __ldcg(a.cand + (int64_t)p * kCand + tid) : 0ull;
+    const uint32_t ncand = __ldcg(a.cand_cnt + p);
+    if (tid == 0) S.seg[si].radix = ncand > (uint32_t)kCand;
+    if (ncand > (uint32_t)kCand) continue;
+    const int nc = (int)ncand;
+    const float m = S.seg[si].m;
+    const unsigned long long rem = S.seg[si].rem;
+    int n = 32;
+    while (n < nc) n <<= 1;
+    const unsigned long long v = bitonic_desc(S, n, tid < nc ? vraw : 0ull);
+    // masses in sorted order; the cut is the first key whose running mass reaches rem
+    const uint32_t key = (uint32_t)(v >> 32);
+    unsigned long long mq = 0ull;
+    if (tid < nc) mq = mass64(key_to_float(key), m, scale);
+    const unsigned long long cum = block_incl_scan_u64(mq, S);
+    if (tid == 0) S.cut_idx = -1;
+    __syncthreads();
+    if (tid < nc && cum >= rem && cum - mq < rem) {
+      S.cut_idx = tid;
+      S.cut_cum = cum;
+      S.seg[si].t_key = key;
+      S.seg[si].e_t = mq;
+    }
+    __syncthreads();
+    if (tid < nc) S.sk[tid] = v;  // publish the sorted keys to find the start of the tie run
+    __syncthreads();
+    if (tid == 0) {
+      Seg& sg = S.seg[si];
+      int ci = S.cut_idx;
+      if (ci < 0) {  // unreachable with exact sums; keep every candidate
+        atomicOr(a.err, kErrInternal);
+        ci = nc - 1;
+        sg.t_key = (uint32_t)(S.sk[ci] >> 32);
+        sg.e_t = mass64(key_to_float(sg.t_key), sg.m, scale);
+        S.cut_cum = sg.rem;
+      }
+      int lo = ci;
+      while (lo > 0 && (uint32_t)(S.sk[lo - 1] >> 32) == sg.t_key) --lo;
+      sg.n_need = (unsigned long long)(ci - lo + 1);
+      sg.msel = (sg.T - sg.rem) + S.cut_cum;
+    }
+    __syncthreads();
+  }
+  __syncthreads();
+  if (fallback) {
+    // radix levels over the key bits of the crossing bin: build level l, sync, read it
+    for (int lev = 0; lev <= 2; ++lev) {
+      for (int si = 0; si < nseg; ++si) {
+        if (!S.seg[si].radix) continue;
+        const int p = S.seg[si].p;
+        const int off = (int)S.seg[si].off, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
+        const int bstar = S.seg[si].bstar;
+        const float m = S.seg[si].m;
+        const uint32_t prefix = S.seg[si].prefix;
+        const int sh = lev > 0 ? level_shift(lev - 1) : 32;
+        zero_words(S);
+        __syncthreads();
+        for (int k = tid; k < rows; k += kThreads) {
+          const float v = sc[off + k];
+          if (bin_of(v, m) != bstar) continue;
+          const uint32_t key = order_key(v);
+          if (sh < 32 && (key >> sh) != prefix) continue;
+          const uint32_t d = (key >> level_shift(lev)) & ((1u << level_bits(lev)) - 1u);
+          uint32_t hi, lo;
+          mass_words(v, m, scale, &hi, &lo);
+          add_words(&S.h.w.lo[d], &S.h.w.hi[d], hi, lo);
+          atomicAdd(&S.hc[d], 1u);
+        }
+        __syncthreads();
+        flush_words(S, a.hr, (int64_t)lev * nh + (int64_t)p * kBins);
+        __syncthreads();
+      }
+      if (!grid_sync(a.bar, G, a.err)) return;
+      for (int si = 0; si < nseg; ++si) {
+        if (!S.seg[si].radix) continue;
+        const int p = S.seg[si].p;
+        load_hist(S, a.hr, (int64_t)lev * nh + (int64_t)p * kBins);
+        find_crossing(S, true, S.seg[si].rem);
         if (tid == 0) {
-          Seg& s = S.seg[si];
-          const int d = S.cross < 0 ? 0 : S.cross;
-          if (S.cross < 0 || S.hc[d] == 0u) atomicOr(a.err, kErrInternal);
-          s.prefix = (s.prefix << level_bits(2)) | (uint32_t)d;
-          s.rem -= S.cross_above;
-          s.shift_f = 0;
-          const uint32_t cnt = S.hc[d] ? S.hc[d] : 1u;
-          s.e_t = S.hm[d] / cnt;  // equal keys carry equal masses
-          s.n_need = s.e_t ? (s.rem + s.e_t - 1) / s.e_t : (unsigned long long)cnt;
-          if (s.n_need > cnt) s.n_need = cnt;
-          s.done = 1;
+          Seg& sg = S.seg[si];
+          int d = S.cross;
+          if (d < 0 || S.hc[d] == 0u) {
+            atomicOr(a.err, kErrInternal);
+            d = d < 0 ? 0 : d;
+          }
+          sg.prefix = (lev == 0) ? (uint32_t)d : ((sg.prefix << level_bits(lev)) | (uint32_t)d);
+          sg.rem -= S.cross_above;
+          if (lev == 2) {  // full key: every member of the group has the same mass
+            const uint32_t cnt = S.hc[d] ? S.hc[d] : 1u;
+            sg.t_key = sg.prefix;
+            sg.e_t = S.h.m[d] / cnt;
+            sg.n_need = sg.e_t ? (sg.rem + sg.e_t - 1) / sg.e_t : (unsigned long long)cnt;
+            if (sg.n_need > cnt) sg.n_need = cnt;
+            sg.msel = (sg.T - sg.rem) + sg.n_need * sg.e_t;
+          }
         }
         __syncthreads();
       }
-      const Seg& s = S.seg[si];
-      uint32_t gt = 0, eq = 0;
-      const int64_t rows = s.jhi - s.jlo;
-      for (int64_t k = tid; k < rows; k += kThreads) {
-        const float v = sc[s.off + k];
-        const int b = bin_of(v, s.m);
-        if (b < s.bstar) {
-          ++gt;
-        } else if (b == s.bstar) {
-          if (s.shift_f == 32) {
-            ++eq;
-          } else {
-            const uint32_t kk = order_key(v) >> s.shift_f;
-            gt += kk > s.prefix;
-            eq += kk == s.prefix;
-          }
-        }
-      }
-      gt = (uint32_t)block_sum_u64(gt, S);
-      eq = (uint32_t)block_sum_u64(eq, S);
-      if (tid == 0) {
-        a.slot_cnt[2 * (p + c)] = gt;
-        a.slot_cnt[2 * (p + c) + 1] = eq;
-      }
     }
   }
-  if (!grid_barrier(a.bar, a.bar + 1, G, a.err)) return;
+  // counts above the cut and at it, per warp (kept for the write pass) and per CTA.  The keep
+  // list holds every key above a fine-bin cut; a coarse-bin cut scans the whole chunk.
+  for (int si = 0; si < nseg; ++si) {
+    const int off = (int)S.seg[si].off, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
+    const uint32_t tk = S.seg[si].t_key;
+    const bool full = S.seg[si].bstar >= kFine || S.seg[si].full;
+    const int wlen = (rows + kWarps - 1) / kWarps;
+    const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
+    const KeepT* kl = keep + S.seg[si].kbase + warp * S.seg[si].kcap;
+    const int n_it = full ? (w_hi - w_lo) : (int)S.lcnt[si][warp];
+    uint32_t wg = 0, we = 0;
+    for (int i0 = 0; i0 < n_it; i0 += 32) {
+      const int i = i0 + lane;
+      uint32_t key = 0u;
+      if (i < n_it) key = order_key(sc[off + (full ? w_lo + i : (int)kl[i])]);
+      wg += __popc(__ballot_sync(0xffffffffu, i < n_it && key > tk));
+      we += __popc(__ballot_sync(0xffffffffu, i < n_it && key == tk));
+    }
+    if (lane == 0) {
+      S.wcnt[si][warp][0] = wg;
+      S.wcnt[si][warp][1] = we;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t g1 = warp_sum(S.wcnt[si][lane][0]), e1 = warp_sum(S.wcnt[si][lane][1]);
+      if (lane == 0) {
+        a.slot_cnt[2 * (S.seg[si].p + c)] = g1;
+        a.slot_cnt[2 * (S.seg[si].p + c) + 1] = e1;
+      }
+    }
+    __syncthreads();
+  }
+  if (!grid_sync(a.bar, G, a.err)) return;
+  // Every CTA has passed its last barrier: the last one to get here rewinds the barrier
+  // counter so the next launch (whatever its grid size) starts from zero.
+  if (tid == 0 && atomicAdd(a.bar + 1, 1ull) == (unsigned long long)(G - 1)) {
+    a.bar[0] = 0ull;
+    a.bar[1] = 0ull;
+  }
 
-  // ---- phase G: offsets across CTAs, ordered compaction of the selected positions
+  // ---- phase E: offsets across CTAs; ordered compaction; clean the scratch for the next launch
+  for (int64_t i = (int64_t)c * kThreads + tid; i < nh; i += (int64_t)G * kThreads) {
+    a.h1.lo[i] = 0u;
+    a.h1.hi[i] = 0u;
+  }
+  if (fallback) zero_global_hist(a.hr, 3 * nh, c, G);
+  for (int i = c * kThreads + tid; i < a.P; i += G * kThreads) a.cand_cnt[i] = 0u;
+  if (c == 0 && tid == 0) a.flags[0] = 0u;
+
   for (int si = 0; si < nseg; ++si) {
     const Seg& s = S.seg[si];
     const int p = s.p;
-    const int cf = (int)(((int64_t)p * a.N) / a.L), cl = (int)(((int64_t)p * a.N + a.N - 1) / a.L);
+    const int cf = cf_of(p, a), cl = (int)(((int64_t)p * a.N + a.N - 1) / a.L);
     for (int cc = cf + tid; cc <= c; cc += kThreads) {
       S.slot[2 * (cc - cf)] = __ldcg(a.slot_cnt + 2 * (p + cc));
       S.slot[2 * (cc - cf) + 1] = __ldcg(a.slot_cnt + 2 * (p + cc) + 1);
@@ -500,50 +739,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
       take = take < 0 ? 0 : (take > e_own ? e_own : take);
       S.before = before;
       S.take = take;
+      uint32_t g_acc = 0, e_acc = 0;  // exclusive warp bases
+      for (int w = 0; w < kWarps; ++w) {
+        const uint32_t g1 = S.wcnt[si][w][0], e1 = S.wcnt[si][w][1];
+        S.wcnt[si][w][0] = g_acc;
+        S.wcnt[si][w][1] = e_acc;
+        g_acc += g1;
+        e_acc += e1;
+      }
+      if (c == cl) {
+        const long long K = before + g_acc + take;
+        a.sel_cnt[p] = (int32_t)(K < a.max_select ? K : a.max_select);
+        a.sel_mass[p] = (float)((double)s.msel / (double)s.Z);
+        a.sel_thr[p] = (float)((double)s.e_t / (double)s.Z);
+      }
     }
     __syncthreads();
+    // write positions in ascending order: warp lists in warp order, ballots within 32-key steps
     const long long before = S.before, take = S.take;
-    long long gt_run = 0, eq_run = 0;
-    const int64_t rows = s.jhi - s.jlo;
-    for (int64_t k0 = 0; k0 < rows; k0 += kThreads) {
-      const int64_t k = k0 + tid;
-      uint32_t isgt = 0, iseq = 0;
-      if (k < rows) {
-        const float v = sc[s.off + k];
-        const int b = bin_of(v, s.m);
-        if (b < s.bstar) {
-          isgt = 1;
-        } else if (b == s.bstar) {
-          if (s.shift_f == 32) {
-            iseq = 1;
-          } else {
-            const uint32_t kk = order_key(v) >> s.shift_f;
-            isgt = kk > s.prefix;
-            iseq = kk == s.prefix;
-          }
-        }
+    const int off = (int)s.off, rows = (int)(s.jhi - s.jlo), jlo = (int)s.jlo;
+    const uint32_t tk = s.t_key;
+    const bool full = s.bstar >= kFine || s.full;
+    const int wlen = (rows + kWarps - 1) / kWarps;
+    const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
+    const KeepT* kl = keep + s.kbase + warp * s.kcap;
+    const int n_it = full ? (w_hi - w_lo) : (int)S.lcnt[si][warp];
+    long long g_run = S.wcnt[si][warp][0], e_run = S.wcnt[si][warp][1];
+    const uint32_t lt = (1u << lane) - 1u;
+    int32_t* dst = a.sel_idx + (int64_t)p * a.max_select;
+    for (int i0 = 0; i0 < n_it; i0 += 32) {
+      const int i = i0 + lane;
+      int k = 0;
+      uint32_t key = 0u;
+      if (i < n_it) {
+        k = full ? w_lo + i : (int)kl[i];
+        key = order_key(sc[off + k]);
       }
-      uint32_t tot;
-      const uint32_t ex = block_scan_u32((isgt << 16) | iseq, S, &tot);
-      const long long gt_b = gt_run + (ex >> 16), eq_b = eq_run + (ex & 0xFFFFu);
-      const bool take_me = isgt || (iseq && eq_b < take);
-      if (take_me) {
-        const long long pos = before + gt_b + (eq_b < take ? eq_b : take);
-        if (pos < a.max_select) {
-          a.sel_idx[(int64_t)p * a.max_select + pos] = (int32_t)(s.jlo + k);
-        } else {
-          atomicOr(a.err, kErrOverflow);
-        }
+      const bool isg = i < n_it && key > tk;
+      const bool ise = i < n_it && key == tk;
+      const uint32_t bg = __ballot_sync(0xffffffffu, isg), be = __ballot_sync(0xffffffffu, ise);
+      const long long g_le = g_run + __popc(bg & lt), e_le = e_run + __popc(be & lt);
+      if (isg || (ise && e_le < take)) {
+        const long long pos = before + g_le + (e_le < take ? e_le : take);
+        if (pos < a.max_select) dst[pos] = jlo + k;
+        else atomicOr(a.err, kErrOverflow);
       }
-      gt_run += tot >> 16;
-      eq_run += tot & 0xFFFFu;
-    }
-    if (c == cl && tid == 0) {
-      const long long K = before + gt_run + take;
-      a.sel_cnt[p] = (int32_t)(K < a.max_select ? K : a.max_select);
-      const unsigned long long msel = (s.T - s.rem) + s.n_need * s.e_t;
-      a.sel_mass[p] = (float)((double)msel / (double)s.Z);
-      a.sel_thr[p] = (float)((double)s.e_t / (double)s.Z);
+      g_run += __popc(bg);
+      e_run += __popc(be);
     }
     __syncthreads();
   }
@@ -552,6 +794,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
 }  // namespace
 
 size_t select_fixed_smem() { return (sizeof(Smem) + 127) / 128 * 128; }
+
+// scores (fp32) + keep lists (16-bit, a quarter of the keys plus per-warp rounding)
+size_t select_var_smem(int64_t per) {
+  return 4 * (size_t)((per + 3) / 4 * 4) + 2 * (size_t)(per / 4 + kWarps * (2 * kSelMaxSeg + 2));
+}
 
 SelectGeom select_geometry(const rtp_layer* L, int64_t N) {
   SelectGeom g;
@@ -567,7 +814,7 @@ SelectGeom select_geometry(const rtp_layer* L, int64_t N) {
   g.grid = G;
   g.per_cta = per;
   const size_t fixed = select_fixed_smem();
-  const size_t need = fixed + (size_t)per * sizeof(float);
+  const size_t need = fixed + select_var_smem(per);
   g.smem_scores = need <= L->smem_optin;
   g.smem_bytes = g.smem_scores ? need : fixed;
   return g;
@@ -593,16 +840,19 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   a.sel_mass = L->sel_mass;
   a.sel_thr = L->sel_thr;
   a.seg_max = L->seg_max;
-  a.h1_mass = L->h1_mass;
-  a.h1_cnt = L->h1_cnt;
-  a.hr_mass = L->hr_mass;
-  a.hr_cnt = L->hr_cnt;
+  const int64_t nh = (int64_t)a.P * kBins;
+  a.h1 = Hist3{L->sel_words, L->sel_words + nh, L->sel_words + 2 * nh};
+  a.hr = Hist3{L->sel_words + 3 * nh, L->sel_words + 6 * nh, L->sel_words + 9 * nh};
+  a.cand_cnt = L->cand_cnt;
+  a.cand = L->cand;
   a.slot_cnt = L->slot_cnt;
   a.bar = L->bar;
   a.err = L->err;
   a.gscores = L->gscores;
+  a.keep = L->sel_keep;
+  a.flags = L->sel_flags;
   if (!g.smem_scores && L->gscores == nullptr) return cudaErrorInvalidValue;
-  if (g.grid > L->sm_count) return cudaErrorInvalidValue;
+  if (g.grid > L->sm_count || g.grid > kSelMaxGrid) return cudaErrorInvalidValue;
   void* args[] = {&a};
   const void* fn = g.smem_scores ? (const void*)decode_select_kernel<true> : (const void*)decode_select_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem_bytes);
@@ -611,8 +861,7 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, g.smem_bytes);
   if (e != cudaSuccess) return e;
   if (occ < 1 || g.grid > occ * L->sm_count) return cudaErrorCooperativeLaunchTooLarge;
-  e = cudaLaunchCooperativeKernel(fn, dim3(g.grid), dim3(kThreads), args, g.smem_bytes, st);
-  return e;
+  return cudaLaunchCooperativeKernel(fn, dim3(g.grid), dim3(kThreads), args, g.smem_bytes, st);
 }
 
 }  // namespace rtp

@@ -24,6 +24,19 @@ enum : uint32_t {
 // Bounded-wait limit for grid barriers: about one second at the B200 clock.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
+// cos/sin of the RoPE angle pos * theta.  The angle is formed in fp64 (pos reaches 2^20, where
+// an fp32 product is off by ~0.06 rad) and reduced to [-pi, pi] by Cody-Waite subtraction of
+// k * 2pi with 2pi split into two doubles; the short reduced angle then goes to fp32 sincosf.
+__device__ __forceinline__ void rope_cos_sin(int64_t pos, double theta, float* c, float* s) {
+  const double kTwoPiHi = 6.283185307179586;        // 2pi rounded to double
+  const double kTwoPiLo = 2.4492935982947064e-16;   // 2pi - kTwoPiHi
+  const double a = (double)pos * theta;
+  const double k = rint(a * (1.0 / 6.283185307179586));
+  double r = fma(-k, kTwoPiHi, a);
+  r = fma(-k, kTwoPiLo, r);
+  sincosf((float)r, s, c);
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -15,7 +15,9 @@ namespace rtp {
 // Work-split and scratch sizes of the fused decode index-stream + top-p select kernel.
 constexpr int kSelThreads = 1024;
 constexpr int kSelBins = 2048;   // level-1 score bins (width 1/64 below the row max) and radix digits
-constexpr int kSelMaxSeg = 64;   // (problem, CTA) segments one CTA may hold
+constexpr int kSelMaxSeg = 16;   // (problem, CTA) segments one CTA may hold
+constexpr int kSelCand = 1024;   // crossing-bin keys resolved by an in-CTA sort
+constexpr int kSelMaxGrid = 256; // CTAs of the selection grid (<= SM count)
 
 // Sparse-attention gather (decode): indices per work item.
 constexpr int kGatherChunk = 128;
@@ -61,12 +63,13 @@ struct rtp_layer {
   float* sel_mass = nullptr;   // [B*Hr]
   float* sel_thr = nullptr;    // [B*Hr]
   float* seg_max = nullptr;    // [P + G]
-  unsigned long long* h1_mass = nullptr;  // [P][bins]
-  uint32_t* h1_cnt = nullptr;
-  unsigned long long* hr_mass = nullptr;  // [2][P][bins]
-  uint32_t* hr_cnt = nullptr;
+  uint32_t* sel_words = nullptr;  // [12][P][bins]: level-1 and radix histograms (lo, hi, count)
+  uint32_t* cand_cnt = nullptr;   // [P]
+  unsigned long long* cand = nullptr;  // [P][kSelCand]
+  uint32_t* sel_keep = nullptr;   // [P][max_seq] keep lists of the selection (global-score mode)
+  uint32_t* sel_flags = nullptr;  // [1] radix fallback flag
   uint32_t* slot_cnt = nullptr;  // [P + G][2]
-  uint32_t* bar = nullptr;       // [2] grid barrier count, generation
+  unsigned long long* bar = nullptr;  // [2] grid barrier arrival / exit counters
   float* gscores = nullptr;      // [P][max_seq] when scores do not fit in shared memory
   size_t gscores_elems = 0;
   float* gpart = nullptr;        // gather partials [items][D + 2]
@@ -105,5 +108,6 @@ struct SelectGeom {
 };
 SelectGeom select_geometry(const rtp_layer* L, int64_t N);
 size_t select_fixed_smem();
+size_t select_var_smem(int64_t per);
 
 }  // namespace rtp

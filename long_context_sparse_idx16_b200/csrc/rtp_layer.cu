@@ -42,11 +42,21 @@ static cudaError_t dalloc(T** p, size_t elems) {
   return cudaMalloc((void**)p, elems * sizeof(T));
 }
 
+// Selection scratch that kernels expect zeroed on entry (they re-zero it after use).
+static cudaError_t reset_select_scratch(rtp_layer* L) {
+  const size_t P = (size_t)L->B * L->Hr > 0 ? (size_t)L->B * L->Hr : 1;
+  cudaError_t e = cudaMemset(L->sel_words, 0, 12 * P * kSelBins * sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(L->cand_cnt, 0, P * sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(L->bar, 0, 2 * sizeof(unsigned long long));
+  if (e == cudaSuccess) e = cudaMemset(L->sel_flags, 0, sizeof(uint32_t));
+  return e;
+}
+
 static void free_all(rtp_layer* L) {
   void* ptrs[] = {L->kc, L->vc, L->idx, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
                   L->d_loc_head, L->d_loc_cnt, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
-                  L->sel_mass, L->sel_thr, L->seg_max, L->h1_mass, L->h1_cnt, L->hr_mass,
-                  L->hr_cnt, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
+                  L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
+                  L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
                   L->sticket, L->err};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -133,7 +143,7 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   const int64_t G = L->sm_count;
   // Largest per-CTA score count the shared-memory variant can hold; beyond it the
   // selection keeps scores in global scratch.
-  const int64_t smem_cap = ((int64_t)L->smem_optin - (int64_t)select_fixed_smem()) / 4;
+  const int64_t smem_cap = ((int64_t)L->smem_optin - (int64_t)select_fixed_smem() - 2 * 32 * 34) * 2 / 9;
   const bool need_gscores = P * L->max_seq > smem_cap * G;
   const int64_t gitems = P * ((L->max_seq + kGatherChunk - 1) / kGatherChunk);
 
@@ -159,10 +169,11 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   RTP_ALLOC(L->sel_mass, P);
   RTP_ALLOC(L->sel_thr, P);
   RTP_ALLOC(L->seg_max, P + G);
-  RTP_ALLOC(L->h1_mass, P * kSelBins);
-  RTP_ALLOC(L->h1_cnt, P * kSelBins);
-  RTP_ALLOC(L->hr_mass, 3 * P * kSelBins);
-  RTP_ALLOC(L->hr_cnt, 3 * P * kSelBins);
+  RTP_ALLOC(L->sel_words, 12 * P * kSelBins);
+  RTP_ALLOC(L->cand_cnt, P);
+  RTP_ALLOC(L->cand, P * kSelCand);
+  RTP_ALLOC(L->sel_keep, P * L->max_seq);
+  RTP_ALLOC(L->sel_flags, 1);
   RTP_ALLOC(L->slot_cnt, 2 * (P + G));
   RTP_ALLOC(L->bar, 2);
   if (need_gscores) {
@@ -198,7 +209,7 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   if (e == cudaSuccess)
     e = cudaMemcpy(L->d_loc_head, loc_head.data(), sizeof(int16_t) * Hkv * kMaxGroup, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(L->d_loc_cnt, loc_cnt.data(), sizeof(int32_t) * Hkv, cudaMemcpyHostToDevice);
-  if (e == cudaSuccess) e = cudaMemset(L->bar, 0, 2 * sizeof(uint32_t));
+  if (e == cudaSuccess) e = reset_select_scratch(L);
   if (e == cudaSuccess) e = cudaMemset(L->gticket, 0, sizeof(uint32_t) * (P > 0 ? P : 1));
   if (e == cudaSuccess) e = cudaMemset(L->err, 0, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(L->sel_cnt, 0, sizeof(int32_t) * (P > 0 ? P : 1));
@@ -310,7 +321,7 @@ rtp_status rtp_check(rtp_layer* L, cudaStream_t stream) {
   cudaMemset(L->err, 0, sizeof(uint32_t));
   if (w & kErrTimeout) {
     // a barrier gave up: its counters are inconsistent; start the next launch from zero
-    cudaMemset(L->bar, 0, 2 * sizeof(uint32_t));
+    reset_select_scratch(L);
     cudaMemset(L->gticket, 0, sizeof(uint32_t) * (size_t)(L->B * L->Hr > 0 ? L->B * L->Hr : 1));
     return fail(L, RTP_ETIMEOUT, "a bounded in-kernel wait gave up");
   }
