@@ -1,0 +1,399 @@
+"""Benchmark of the head-wise sparse attention layer (RTPurbo) on B200.
+
+One JSON line on rank 0 (see --help).  A step is one decode token of the 128K workload:
+B = 8 sequences of N = 131072 keys, 32 query / 4 KV heads (D = 128), 5 retrieval heads (r = 16,
+p = 0.9) and 27 local heads (W = 8192, S = 4), seeded synthetic data shaped like the pages'
+workloads.  Each step appends the token's K/V (RoPE + index keys) and runs the decode
+(index stream, exact top-p, sparse attention, window + sink attention), through the C ABI.
+Before every step the length is rolled back by one, so every step sees exactly N keys.
+
+value   = decode microseconds per token (step time / B; all ranks' tokens / max rank time)
+e2e     = the same through the C ABI with the step's q/k/v copied from pinned host memory
+          and the output copied back, inside the timed region
+roofline= the dominant kernel (fused index stream + top-p select): algorithmic bytes (the
+          16-dim fp32 index keys, 64 B per key per retrieval head per sequence) per launch over
+          its mean device time from CUDA events on its launch stream
+--impl reference: the fp64 CPU oracle as it stands, on this host's cores, same metric.
+
+Multi-GPU: the layer does not shard; --gpus N runs N independent replicas (one per GPU).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RTPurbo attn layer: decode µs/token & prefill ms at 128K/1M; % of roofline"
+DECODE_WORKLOADS = ("decode_128k", "decode_1m")
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _profile_traffic(kernel_src: str):
+    """Per-launch DRAM traffic of the select kernel from the committed ncu summary, if the
+    kernel source has not changed since that capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_select_128k.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    want = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    traffic = None
+    src_hash = None
+    for line in text.splitlines():
+        if line.startswith("- source sha256[:16]:"):
+            src_hash = line.split(":", 1)[1].strip()
+        if line.startswith("- dram bytes per launch (read + write):"):
+            traffic = float(line.split(":", 1)[1].strip().split()[0])
+    return traffic if (src_hash == want and traffic) else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: int):
+        self.gpu = gpu
+        self.proc = None
+        self.path = os.path.join("/tmp", f"rtp_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(x, seconds: float = 12.0):
+    """Time the fp64 oracle (as it stands) on the decode step of whole sequences until about
+    `seconds` of CPU work; returns (us per token, cores, description)."""
+    import oracle
+
+    s = x.spec
+    t0 = time.perf_counter()
+    done = 0
+    for b in range(s.batch):
+        for h in range(s.n_q_heads):
+            oracle.layer_rows(x, b, h, [0], want_sel=False)
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return dt / done * 1e6, oracle.max_threads(), f"decode step of {done} of {s.batch} sequences, all {s.n_q_heads} heads"
+
+
+def run_reference(args):
+    """The oracle arm.  Each step runs the oracle on one retrieval head and one local head of one
+    sequence (cycling over all of them); the token time is estimated as
+    mean(retrieval head) x Hr + mean(local head) x Hl, which is unbiased for any step count."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import oracle
+
+    x = _generate(args)
+    s = x.spec
+    ret = [(b, h) for b in range(s.batch) for h in s.retrieval_heads]
+    loc = [(b, h) for b in range(s.batch) for h in range(s.n_q_heads) if h not in s.retrieval_heads]
+    budget = 200.0
+
+    def one(i):
+        t = []
+        for units in (ret, loc):
+            if not units:
+                t.append(0.0)
+                continue
+            b, h = units[i % len(units)]
+            t0 = time.perf_counter()
+            oracle.layer_rows(x, b, h, [0], want_sel=False)
+            t.append(time.perf_counter() - t0)
+        return t
+
+    for i in range(args.warmup):
+        one(i)
+    tr = tl = 0.0
+    n = 0
+    t_start = time.perf_counter()
+    for i in range(args.steps):
+        a, b = one(args.warmup + i)
+        tr += a
+        tl += b
+        n += 1
+        if time.perf_counter() - t_start > budget:
+            break
+    dt = time.perf_counter() - t_start
+    nr, nl = len(s.retrieval_heads), s.n_q_heads - len(s.retrieval_heads)
+    us_token = (tr / n * nr + tl / n * nl) * 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us_token, "unit": "us/token", "n_gpus": args.gpus,
+        "steps": n, "warmup": args.warmup, "ms_per_step": dt / n * 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(s, args.gpus),
+        "cpu_baseline": {"value": us_token, "unit": "us/token", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"{n} steps of one retrieval head + one local head of one sequence, cycling over "
+                                   f"all heads and sequences; token time = mean per class x heads per class"
+                                   + (" (stopped at the time budget)" if n < args.steps else "")},
+        "e2e": {"value": us_token, "unit": "us/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _generate(args):
+    import synth
+
+    return synth.generate(_spec(args))
+
+
+def _spec(args):
+    import synth
+
+    ov = {}
+    if args.batch:
+        base = synth.spec(args.workload)
+        ov["batch"] = args.batch
+        if base.needles and len(base.needles) > 1:
+            ov["needles"] = tuple(base.needles[i % len(base.needles)] for i in range(args.batch))
+    return synth.spec(args.workload, **ov)
+
+
+def _config(s, n_gpus):
+    return {"workload": (f"{s.name}: decode, B={s.batch}, N={s.n_total}, {s.n_q_heads} q / {s.n_kv_heads} kv heads, "
+                         f"D={s.head_dim}, {len(s.retrieval_heads)} retrieval heads r={s.index_dim} p={s.top_p}, "
+                         f"local W={s.window} S={s.n_sink}"),
+            "global_batch": s.batch * n_gpus, "seq_len": s.n_total, "parallelism": f"replicas x{n_gpus}",
+            "l2": "inputs larger than L2 (KV cache %.2f GiB + index keys %.0f MB per GPU)" % (
+                2 * s.batch * s.n_kv_heads * s.n_total * s.head_dim * 2 / 2**30,
+                s.batch * len(s.retrieval_heads) * s.n_total * s.index_dim * 4 / 1e6)}
+
+
+def run_gpu(args):
+    import numpy as np
+    import torch
+
+    import synth
+    from long_context_sparse_idx16_b200 import Layer
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    s = _spec(args)
+    x = synth.generate(s)
+    N, B = s.n_total, s.batch
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    layer = Layer.from_spec(s, x, max_seq=N, max_chunk=1)
+    for t0 in range(0, N - 1, 1 << 16):
+        t1 = min(N - 1, t0 + (1 << 16))
+        layer.append_kv(bf16(x.k[:, t0:t1]).to(dev), bf16(x.v[:, t0:t1]).to(dev))
+    k_tok = bf16(x.k[:, N - 1:N]).to(dev).contiguous()
+    v_tok = bf16(x.v[:, N - 1:N]).to(dev).contiguous()
+    q = bf16(x.q[:, 0]).to(dev).contiguous()
+    out = torch.empty((B, s.n_q_heads, 128), dtype=torch.float32, device=dev)
+
+    def step():
+        layer.truncate(N - 1)
+        layer.append_kv(k_tok, v_tok)
+        layer.decode(q, out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert layer.check() == 0
+    _, st = layer.decode(q, out, stats=True)
+    counts = st[0].cpu().numpy().ravel()
+
+    # ---- device-timed region (no per-kernel events inside it)
+    clocks = ClockSampler(local)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    assert layer.check() == 0
+    ms = _max_over_ranks(ms, world, dev)
+
+    # ---- the same steps again with a CUDA event pair around every kernel launch (on its
+    # launch stream): per-kernel device time for the roofline and the launch count
+    layer.profile(True)
+    layer.profile_read()  # drop anything recorded before
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    sel_ms, sel_n = layer.profile_read("decode_select")
+    rest_ms, rest_n = layer.profile_read(None)
+    layer.profile(False)
+    all_n = sel_n + rest_n
+
+    # ---- end-to-end through the C ABI with host buffers
+    q_h = torch.empty_like(q, device="cpu").pin_memory()
+    k_h = torch.empty_like(k_tok, device="cpu").pin_memory()
+    v_h = torch.empty_like(v_tok, device="cpu").pin_memory()
+    o_h = torch.empty_like(out, device="cpu").pin_memory()
+    q_h.copy_(q.cpu())
+    k_h.copy_(k_tok.cpu())
+    v_h.copy_(v_tok.cpu())
+    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(k_tok), torch.empty_like(v_tok)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        layer.truncate(N - 1)
+        layer.append_kv(k_d, v_d)
+        layer.decode(q_d, out)
+        o_h.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(f0.elapsed_time(f1), world, dev)
+    assert np.isfinite(o_h.numpy()).all()
+
+    tokens = B * args.steps * world
+    value = ms * 1e3 / tokens  # us per token: all ranks' tokens over the max rank time
+    e2e = e2e_ms * 1e3 / tokens
+    peak, peak_kind = _peaks()
+    P = B * len(s.retrieval_heads)
+    sel_bytes = P * N * s.index_dim * 4  # fp32 index keys streamed per launch
+    sel_us = sel_ms * 1e3 / max(sel_n, 1)
+    achieved = sel_bytes / (sel_us * 1e-6) / 1e9
+    traffic = _profile_traffic(os.path.join(ROOT, "long_context_sparse_idx16_b200", "csrc", "decode_select.cu"))
+    # whole-step algorithmic bytes: index keys + window/sink K/V rows + selected K/V rows
+    n_local_kv = s.n_kv_heads  # every KV head serves local heads in this layout
+    win_keys = min(N, s.window + s.n_sink)
+    step_bytes = sel_bytes + B * n_local_kv * win_keys * 512 + int(counts.sum()) * 512
+    line = {
+        "metric": METRIC, "value": value, "unit": "us/token", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(s, world),
+        "roofline": {"bound": "hbm", "kernel": "decode_select (fused index stream + exact top-p)",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "bytes_per_launch": sel_bytes,
+                     "us_per_launch": sel_us},
+        "step_roofline": {"bytes_per_step": step_bytes, "roofline_us_per_step": step_bytes / (peak * 1e9) * 1e6,
+                          "frac": step_bytes / (peak * 1e9) / (ms / args.steps * 1e-3)},
+        "e2e": {"value": e2e, "unit": "us/token", "h2d_bytes_per_step": int(q.numel() * 2 + k_tok.numel() * 2 * 2),
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": int(all_n),  # kernels of this library per timed region (one pass of --steps steps)
+        "selected_tokens": {"min": int(counts.min()), "median": float(np.median(counts)), "max": int(counts.max())},
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        v, cores, desc = cpu_oracle_sample(x)
+        line["cpu_baseline"] = {"value": v, "unit": "us/token", "cores": cores, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=DECODE_WORKLOADS, default="decode_128k",
+                    help="measured workload (the default is the headline one; others are for profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="override the sequence count (profiling cases)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

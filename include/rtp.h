@@ -138,6 +138,19 @@ int64_t rtp_seq_len(const rtp_layer* layer);
 /* Forget every token (length back to 0); the caches are overwritten by later appends. */
 rtp_status rtp_reset(rtp_layer* layer);
 
+/* Roll the length back to new_len <= current length (e.g. to re-run a step or drop rejected
+ * speculative tokens); later appends overwrite the dropped positions.  RTP_EINVAL if
+ * new_len is negative or above the current length. */
+rtp_status rtp_truncate(rtp_layer* layer, int64_t new_len);
+
+/* Per-kernel device timing.  While enabled, the library records a CUDA event pair on the
+ * launch stream around every kernel it launches.  rtp_profile_read synchronises on the
+ * recorded events, returns the summed device time (ms) and launch count of the named kernel
+ * ("append_kv", "q_prep", "decode_select", "decode_gather", "decode_swa", "swa_merge",
+ * "dense_fill", "prefill_*"; NULL: all kernels together), and clears that kernel's record. */
+rtp_status rtp_profile_enable(rtp_layer* layer, int on);
+rtp_status rtp_profile_read(rtp_layer* layer, const char* kernel, double* total_ms, int64_t* launches);
+
 /* Synchronise `stream`, then report and clear errors recorded by kernels since the last
  * check (RTP_EOVERFLOW, RTP_ERANGE, RTP_ETIMEOUT, ...). */
 rtp_status rtp_check(rtp_layer* layer, cudaStream_t stream);

@@ -79,6 +79,9 @@ def lib() -> C.CDLL:
             "rtp_reset": ([P], C.c_int),
             "rtp_check": ([P, P], C.c_int),
             "rtp_get_cache": ([P, C.POINTER(rtp_cache_view)], C.c_int),
+            "rtp_truncate": ([P, i64], C.c_int),
+            "rtp_profile_enable": ([P, C.c_int], C.c_int),
+            "rtp_profile_read": ([P, C.c_char_p, C.POINTER(C.c_double), C.POINTER(C.c_int64)], C.c_int),
             "rtp_last_error": ([P], C.c_char_p),
         }
         for name, (args, res) in sigs.items():
@@ -132,6 +135,22 @@ def rtp_seq_len(layer) -> int:
 
 def rtp_reset(layer) -> None:
     _check(lib().rtp_reset(layer), layer)
+
+
+def rtp_truncate(layer, new_len: int) -> None:
+    _check(lib().rtp_truncate(layer, new_len), layer)
+
+
+def rtp_profile_enable(layer, on: bool) -> None:
+    _check(lib().rtp_profile_enable(layer, 1 if on else 0), layer)
+
+
+def rtp_profile_read(layer, kernel: Optional[str]):
+    """(total device ms, launches) of the named kernel since the last read (clears it)."""
+    ms = C.c_double()
+    n = C.c_int64()
+    _check(lib().rtp_profile_read(layer, kernel.encode() if kernel else None, C.byref(ms), C.byref(n)), layer)
+    return ms.value, n.value
 
 
 def rtp_check(layer, stream: int) -> int:
@@ -210,6 +229,15 @@ class Layer:
 
     def reset(self) -> None:
         rtp_reset(self.handle)
+
+    def truncate(self, new_len: int) -> None:
+        rtp_truncate(self.handle, new_len)
+
+    def profile(self, on: bool) -> None:
+        rtp_profile_enable(self.handle, on)
+
+    def profile_read(self, kernel: Optional[str] = None):
+        return rtp_profile_read(self.handle, kernel)
 
     def append_kv(self, k, v, stream=None) -> None:
         """k, v: torch bf16 CUDA tensors [B][T][Hkv][128] (k pre-RoPE)."""

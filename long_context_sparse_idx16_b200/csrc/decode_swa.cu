@@ -362,9 +362,13 @@ cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st) {
   const size_t smem = tile_smem > merge_smem ? tile_smem : merge_smem;
   cudaError_t e = cudaFuncSetAttribute(decode_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_swa_kernel<<<dim3(a.n_chunks, L->Hkv, L->B), kThreads, smem, st>>>(a);
-  e = cudaGetLastError();
+  {
+    ProfScope ps(const_cast<rtp_layer*>(L), "decode_swa", st);
+    decode_swa_kernel<<<dim3(a.n_chunks, L->Hkv, L->B), kThreads, smem, st>>>(a);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess || a.n_chunks == 1) return e;
+  ProfScope ps(const_cast<rtp_layer*>(L), "swa_merge", st);
   swa_merge_kernel<<<dim3(kMaxGroup, L->Hkv, L->B), 256, 0, st>>>(L->spart, a.n_chunks, L->Hkv, L->Hq,
                                                                 L->d_loc_head, L->d_loc_cnt, out);
   return cudaGetLastError();

@@ -5,7 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <map>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "rtp.h"
@@ -80,10 +82,25 @@ struct rtp_layer {
   uint32_t* sticket = nullptr;   // [B*Hkv]
   uint32_t* err = nullptr;       // device error word
 
+  // per-kernel event timing (rtp_profile_enable)
+  bool prof_on = false;
+  std::map<std::string, std::vector<std::pair<cudaEvent_t, cudaEvent_t>>> prof;
+  std::vector<cudaEvent_t> prof_pool;
+
   std::string last_error;
 };
 
 namespace rtp {
+
+// Scoped event pair around one kernel launch when profiling is on.
+struct ProfScope {
+  rtp_layer* L;
+  const char* name;
+  cudaStream_t st;
+  cudaEvent_t e0 = nullptr;
+  ProfScope(rtp_layer* L_, const char* n, cudaStream_t s);
+  ~ProfScope();
+};
 
 rtp_status fail(rtp_layer* L, rtp_status st, const std::string& msg);
 rtp_status cuda_fail(rtp_layer* L, cudaError_t e, const char* what);

@@ -52,7 +52,45 @@ static cudaError_t reset_select_scratch(rtp_layer* L) {
   return e;
 }
 
+static cudaEvent_t prof_event(rtp_layer* L) {
+  if (!L->prof_pool.empty()) {
+    cudaEvent_t e = L->prof_pool.back();
+    L->prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+ProfScope::ProfScope(rtp_layer* L_, const char* n, cudaStream_t s) : L(L_), name(n), st(s) {
+  if (L && L->prof_on) {
+    e0 = prof_event(L);
+    cudaEventRecord(e0, st);
+  }
+}
+
+ProfScope::~ProfScope() {
+  if (e0) {
+    cudaEvent_t e1 = prof_event(L);
+    cudaEventRecord(e1, st);
+    L->prof[name].push_back({e0, e1});
+  }
+}
+
+static void prof_release(rtp_layer* L) {
+  for (auto& kv : L->prof)
+    for (auto& pr : kv.second) {
+      cudaEventDestroy(pr.first);
+      cudaEventDestroy(pr.second);
+    }
+  L->prof.clear();
+  for (cudaEvent_t e : L->prof_pool) cudaEventDestroy(e);
+  L->prof_pool.clear();
+}
+
 static void free_all(rtp_layer* L) {
+  prof_release(L);
   void* ptrs[] = {L->kc, L->vc, L->idx, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
                   L->d_loc_head, L->d_loc_cnt, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
@@ -236,7 +274,11 @@ rtp_status rtp_append_kv(rtp_layer* L, const void* k, const void* v, int32_t T, 
   if (!k || !v) return fail(L, RTP_EINVAL, "rtp_append_kv: k or v is NULL");
   if (T < 1) return fail(L, RTP_EINVAL, "rtp_append_kv: T must be >= 1");
   if (L->len + T > L->max_seq) return fail(L, RTP_ECAPACITY, "rtp_append_kv: max_seq exceeded");
-  cudaError_t e = launch_append_kv(L, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, T, stream);
+  cudaError_t e;
+  {
+    ProfScope ps(L, "append_kv", stream);
+    e = launch_append_kv(L, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, T, stream);
+  }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_append_kv: launch");
   L->len += T;
   L->last_error.clear();
@@ -247,14 +289,24 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_decode: layer is NULL");
   if (!q || !out) return fail(L, RTP_EINVAL, "rtp_decode: q or out is NULL");
   if (L->len < 1) return fail(L, RTP_EINVAL, "rtp_decode: the cache is empty (append the token first)");
-  cudaError_t e = launch_q_prep(L, (const __nv_bfloat16*)q, 1, L->len - 1, stream);
+  cudaError_t e;
+  {
+    ProfScope ps(L, "q_prep", stream);
+    e = launch_q_prep(L, (const __nv_bfloat16*)q, 1, L->len - 1, stream);
+  }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: q_prep");
   if (L->Hr > 0) {
     // p == 1 keeps every causal key: the gather reads positions 0..len-1 directly
     const bool dense = L->top_p >= 1.f;
-    e = dense ? launch_dense_stats(L, stream) : launch_decode_select(L, stream);
+    {
+      ProfScope ps(L, dense ? "dense_fill" : "decode_select", stream);
+      e = dense ? launch_dense_stats(L, stream) : launch_decode_select(L, stream);
+    }
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: select");
-    e = launch_decode_gather(L, dense, out, stream);
+    {
+      ProfScope ps(L, "decode_gather", stream);
+      e = launch_decode_gather(L, dense, out, stream);
+    }
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: gather");
     if (stats) {
       const size_t P = (size_t)L->B * L->Hr;
@@ -277,7 +329,7 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
     }
   }
   if (L->n_local > 0) {
-    e = launch_decode_swa(L, out, stream);
+    e = launch_decode_swa(L, out, stream);  // times itself ("decode_swa", "swa_merge")
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: window attention");
   }
   L->last_error.clear();
@@ -303,6 +355,45 @@ rtp_status rtp_set_top_p(rtp_layer* L, float top_p) {
 }
 
 int64_t rtp_seq_len(const rtp_layer* L) { return L ? L->len : -1; }
+
+rtp_status rtp_truncate(rtp_layer* L, int64_t new_len) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_truncate: layer is NULL");
+  if (new_len < 0 || new_len > L->len) return fail(L, RTP_EINVAL, "rtp_truncate: need 0 <= new_len <= length");
+  L->len = new_len;
+  return RTP_OK;
+}
+
+rtp_status rtp_profile_enable(rtp_layer* L, int on) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_profile_enable: layer is NULL");
+  L->prof_on = on != 0;
+  return RTP_OK;
+}
+
+rtp_status rtp_profile_read(rtp_layer* L, const char* kernel, double* total_ms, int64_t* launches) {
+  if (!L || !total_ms || !launches) return fail(L, RTP_EINVAL, "rtp_profile_read: NULL argument");
+  double ms = 0.0;
+  int64_t n = 0;
+  for (auto it = L->prof.begin(); it != L->prof.end();) {
+    if (kernel && it->first != kernel) {
+      ++it;
+      continue;
+    }
+    for (auto& pr : it->second) {
+      cudaError_t e = cudaEventSynchronize(pr.second);
+      if (e != cudaSuccess) return cuda_fail(L, e, "rtp_profile_read");
+      float t = 0.f;
+      cudaEventElapsedTime(&t, pr.first, pr.second);
+      ms += t;
+      ++n;
+      L->prof_pool.push_back(pr.first);
+      L->prof_pool.push_back(pr.second);
+    }
+    it = L->prof.erase(it);
+  }
+  *total_ms = ms;
+  *launches = n;
+  return RTP_OK;
+}
 
 rtp_status rtp_reset(rtp_layer* L) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_reset: layer is NULL");
