@@ -158,6 +158,28 @@ rtp_status rtp_check(rtp_layer* layer, cudaStream_t stream);
 /* Device pointers of the caches. */
 rtp_status rtp_get_cache(const rtp_layer* layer, rtp_cache_view* view);
 
+/* Exact attention over caller-given key lists, with no layer and no device allocation.
+ * (No counterpart on the pages: this serves callers that cannot allocate device memory --
+ * code running while a CUDA graph is captured, engines that own all device memory through
+ * their own pool, processes whose device memory is fully committed.)
+ *
+ * For each problem p < P (one decode query): o_p = softmax_j(sm_scale * q_p . K_j) V_j over the
+ * positions j = idx[p][0 .. min(cnt[p], max_count)).  K_j and V_j are fp16 rows of 128 values at
+ * k / v + kv_block[p] * kv_stride + j * 128 (kv_block NULL: block p); q is DEVICE fp32 [P][128]
+ * (already RoPE'd), idx DEVICE int32 [P][idx_stride], cnt DEVICE int32 [P], out DEVICE fp32
+ * [P][128].  Rows of the layer's cache (rtp_get_cache) can be passed directly.
+ *
+ * Scratch: one built-in device array of about 2.1 MB (4096 work items of 128 keys); the call
+ * returns RTP_EINVAL without launching when P * ceil(max_count / 128) exceeds 4096 or P > 2048.
+ * The first call on each device (with that device current) looks the array's address up and
+ * caches it: make that first call before any stream capture.  Every call on a device shares the
+ * array, so calls whose kernels overlap on the GPU race; serialise them (one stream).  Errors
+ * are reported through rtp_last_error(NULL). */
+rtp_status rtp_gather_attn_noalloc(const void* k, const void* v, const int32_t* kv_block, int64_t kv_stride,
+                                   const float* q, const int32_t* idx, int64_t idx_stride,
+                                   const int32_t* cnt, int32_t P, int64_t max_count, float sm_scale,
+                                   float* out, cudaStream_t stream);
+
 /* Host string for the last failure on this layer ("" if none).  layer may be NULL, which
  * returns the last failure of rtp_create in this thread. */
 const char* rtp_last_error(const rtp_layer* layer);

@@ -80,6 +80,7 @@ def lib() -> C.CDLL:
             "rtp_check": ([P, P], C.c_int),
             "rtp_get_cache": ([P, C.POINTER(rtp_cache_view)], C.c_int),
             "rtp_truncate": ([P, i64], C.c_int),
+            "rtp_gather_attn_noalloc": ([P, P, P, i64, P, P, i64, P, i32, i64, f32, P, P], C.c_int),
             "rtp_profile_enable": ([P, C.c_int], C.c_int),
             "rtp_profile_read": ([P, C.c_char_p, C.POINTER(C.c_double), C.POINTER(C.c_int64)], C.c_int),
             "rtp_last_error": ([P], C.c_char_p),
@@ -151,6 +152,14 @@ def rtp_profile_read(layer, kernel: Optional[str]):
     n = C.c_int64()
     _check(lib().rtp_profile_read(layer, kernel.encode() if kernel else None, C.byref(ms), C.byref(n)), layer)
     return ms.value, n.value
+
+
+def rtp_gather_attn_noalloc(k_ptr: int, v_ptr: int, kv_block_ptr: Optional[int], kv_stride: int, q_ptr: int,
+                            idx_ptr: int, idx_stride: int, cnt_ptr: int, P: int, max_count: int,
+                            sm_scale: float, out_ptr: int, stream: int) -> None:
+    """Attention over caller-given key lists without any device allocation (see rtp.h)."""
+    _check(lib().rtp_gather_attn_noalloc(k_ptr, v_ptr, kv_block_ptr, kv_stride, q_ptr, idx_ptr, idx_stride,
+                                         cnt_ptr, P, max_count, sm_scale, out_ptr, stream))
 
 
 def rtp_check(layer, stream: int) -> int:
