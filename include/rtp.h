@@ -86,9 +86,17 @@ typedef struct {
   int64_t sel_index_cap;
 } rtp_decode_stats;
 
-/* Optional prefill statistics, DEVICE array [B][C][Hr]. */
+/* Optional prefill statistics, DEVICE arrays (retrieval heads ascending).  Any member may be
+ * NULL.  sel_bitmap holds, for every row i and retrieval head, bitmap_words 32-bit words: bit
+ * (j % 32) of word j / 32 is set iff key j is in row i's selected set.  Words the kernel writes:
+ * those covering keys 0 .. (last position of the row's 64-row tile), rounded up to 64 keys and
+ * capped at bitmap_words; the caller zeroes the rest.  Keys past 32 * bitmap_words are not
+ * reported (the selection itself is unaffected). */
 typedef struct {
-  int32_t* sel_count;
+  int32_t* sel_count;    /* [B][C][Hr] |J_i| */
+  float* sel_mass;       /* [B][C][Hr] index-softmax mass of J_i (>= p) */
+  uint32_t* sel_bitmap;  /* [B][C][Hr][bitmap_words] */
+  int64_t bitmap_words;
 } rtp_prefill_stats;
 
 /* Device-side view of the layer's caches (for tests and tools; read-only use). */

@@ -42,7 +42,8 @@ class rtp_decode_stats(C.Structure):
 
 
 class rtp_prefill_stats(C.Structure):
-    _fields_ = [("sel_count", C.c_void_p)]
+    _fields_ = [("sel_count", C.c_void_p), ("sel_mass", C.c_void_p), ("sel_bitmap", C.c_void_p),
+                ("bitmap_words", C.c_int64)]
 
 
 class rtp_cache_view(C.Structure):
@@ -276,8 +277,11 @@ class Layer:
         rtp_decode(self.handle, q.data_ptr(), out.data_ptr(), st, _stream_handle(stream))
         return (out, tensors) if stats else out
 
-    def prefill_chunk(self, q, out=None, stats: bool = False, stream=None):
-        """q: torch bf16 CUDA tensor [B][C][Hq][128]; row i at position len-C+i."""
+    def prefill_chunk(self, q, out=None, stats: bool = False, bitmap_words: int = 0, stream=None):
+        """q: torch bf16 CUDA tensor [B][C][Hq][128]; row i at position len-C+i.
+
+        With stats, also returns (sel_count [B][C][Hr] int32, sel_mass [B][C][Hr] fp32,
+        sel_bitmap [B][C][Hr][bitmap_words] int32 or None)."""
         import torch
 
         assert q.is_cuda and q.is_contiguous()
@@ -285,12 +289,17 @@ class Layer:
         if out is None:
             out = torch.empty((self.batch, Cr, self.n_q_heads, 128), dtype=torch.float32, device=q.device)
         st = None
-        cnt = None
+        tensors = None
         if stats and self.n_retrieval:
-            cnt = torch.empty((self.batch, Cr, self.n_retrieval), dtype=torch.int32, device=q.device)
-            st = rtp_prefill_stats(cnt.data_ptr())
+            shp = (self.batch, Cr, self.n_retrieval)
+            bm = (torch.zeros(shp + (bitmap_words,), dtype=torch.int32, device=q.device)
+                  if bitmap_words > 0 else None)
+            tensors = (torch.empty(shp, dtype=torch.int32, device=q.device),
+                       torch.empty(shp, dtype=torch.float32, device=q.device), bm)
+            st = rtp_prefill_stats(tensors[0].data_ptr(), tensors[1].data_ptr(),
+                                   bm.data_ptr() if bm is not None else None, bitmap_words)
         rtp_prefill_chunk(self.handle, q.data_ptr(), Cr, out.data_ptr(), st, _stream_handle(stream))
-        return (out, cnt) if stats else out
+        return (out, tensors) if stats else out
 
     def check(self, stream=None) -> int:
         return rtp_check(self.handle, _stream_handle(stream))

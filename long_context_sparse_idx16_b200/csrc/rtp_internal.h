@@ -55,6 +55,7 @@ struct rtp_layer {
   int16_t* d_ret_head = nullptr;   // [Hr]
   int16_t* d_loc_head = nullptr;   // [Hkv][kMaxGroup] local q heads of each KV head (-1 pad)
   int32_t* d_loc_cnt = nullptr;    // [Hkv]
+  int16_t* d_local_list = nullptr; // [n_local] local q heads, ascending
   int n_local = 0;
 
   // decode scratch
@@ -115,6 +116,9 @@ cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, float* out, cud
 cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st);
 cudaError_t launch_iota_rows(int32_t* dst, int64_t cap, int rows, int64_t n, cudaStream_t st);
 cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st);
+cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStream_t st);
+cudaError_t launch_prefill_retrieval(const rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,
+                                     cudaStream_t st);
 
 // Selection kernel geometry for the current length (host-side; also sizes scratch).
 struct SelectGeom {

@@ -92,7 +92,7 @@ static void prof_release(rtp_layer* L) {
 static void free_all(rtp_layer* L) {
   prof_release(L);
   void* ptrs[] = {L->kc, L->vc, L->idx, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
-                  L->d_loc_head, L->d_loc_cnt, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
+                  L->d_loc_head, L->d_loc_cnt, L->d_local_list, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
                   L->sticket, L->err};
@@ -200,6 +200,7 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   RTP_ALLOC(L->d_ret_head, Hr);
   RTP_ALLOC(L->d_loc_head, Hkv * kMaxGroup);
   RTP_ALLOC(L->d_loc_cnt, Hkv);
+  RTP_ALLOC(L->d_local_list, L->n_local);
   RTP_ALLOC(L->q_rot, rows * Hq * kD);
   RTP_ALLOC(L->q_idx, rows * Hr * kR);
   RTP_ALLOC(L->sel_idx, P * L->max_select);
@@ -247,6 +248,13 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   if (e == cudaSuccess)
     e = cudaMemcpy(L->d_loc_head, loc_head.data(), sizeof(int16_t) * Hkv * kMaxGroup, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(L->d_loc_cnt, loc_cnt.data(), sizeof(int32_t) * Hkv, cudaMemcpyHostToDevice);
+  {
+    std::vector<int16_t> local_list;
+    for (int h = 0; h < Hq; ++h)
+      if (c.head_class[h] == 0) local_list.push_back((int16_t)h);
+    if (e == cudaSuccess && !local_list.empty())
+      e = cudaMemcpy(L->d_local_list, local_list.data(), sizeof(int16_t) * local_list.size(), cudaMemcpyHostToDevice);
+  }
   if (e == cudaSuccess) e = reset_select_scratch(L);
   if (e == cudaSuccess) e = cudaMemset(L->gticket, 0, sizeof(uint32_t) * (P > 0 ? P : 1));
   if (e == cudaSuccess) e = cudaMemset(L->err, 0, sizeof(uint32_t));
@@ -338,13 +346,30 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
 
 rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out, const rtp_prefill_stats* stats,
                              cudaStream_t stream) {
-  (void)stats;
-  (void)stream;
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_prefill_chunk: layer is NULL");
   if (!q || !out) return fail(L, RTP_EINVAL, "rtp_prefill_chunk: q or out is NULL");
   if (C < 1 || C > L->max_chunk || C > L->len)
     return fail(L, RTP_EINVAL, "rtp_prefill_chunk: need 1 <= C <= min(len, max_chunk)");
-  return fail(L, RTP_EINTERNAL, "rtp_prefill_chunk: not built yet");
+  if (stats && stats->sel_bitmap && stats->bitmap_words < 1)
+    return fail(L, RTP_EINVAL, "rtp_prefill_chunk: sel_bitmap needs bitmap_words >= 1");
+  cudaError_t e;
+  {
+    ProfScope ps(L, "q_prep", stream);
+    e = launch_q_prep(L, (const __nv_bfloat16*)q, C, L->len - C, stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: q_prep");
+  if (L->Hr > 0) {
+    ProfScope ps(L, "prefill_retrieval", stream);
+    e = launch_prefill_retrieval(L, C, out, stats, stream);
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: retrieval heads");
+  }
+  if (L->n_local > 0) {
+    ProfScope ps(L, "prefill_local", stream);
+    e = launch_prefill_local(L, C, out, stream);
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: local heads");
+  }
+  L->last_error.clear();
+  return RTP_OK;
 }
 
 rtp_status rtp_set_top_p(rtp_layer* L, float top_p) {

@@ -38,6 +38,8 @@ def lib():
         L.orc_rope.argtypes = [P, f64, i32, f64, P]
         L.orc_index_scores.restype = None
         L.orc_index_scores.argtypes = [P, i64, i64, i32, i32, i32, P, P, P, P]
+        L.orc_attend_set.restype = None
+        L.orc_attend_set.argtypes = [P, P, i64, i32, i32, P, i64, f64, f64, i64, P, i64, P]
         L.orc_max_threads.restype = C.c_int
         L.orc_max_threads.argtypes = []
         _lib = L
@@ -174,3 +176,22 @@ def layer_rows(inputs, b: int, h: int, rows: Sequence[int], *, top_p: Optional[f
         wk=inputs.wk[slot] if retrieval else None, top_p=s.top_p if top_p is None else top_p,
         window=s.window, n_sink=s.n_sink, rope_base=s.rope_base, want_sel=want_sel,
         want_pi=want_pi, threads=threads, pos_offset=pos_offset)
+
+
+def attend_set(inputs, b: int, h: int, row: int, sel: Sequence[int], *, pos_offset: int = 0) -> np.ndarray:
+    """Exact attention of chunk row ``row`` of query head h (sequence b) over the key set ``sel``
+    (no selection step): for checking an output whose set legitimately differs from the
+    oracle's own."""
+    s = inputs.spec
+    k_seq = np.ascontiguousarray(inputs.k[b], dtype=np.uint16)
+    v_seq = np.ascontiguousarray(inputs.v[b], dtype=np.uint16)
+    N, Hkv, D = k_seq.shape
+    q = np.ascontiguousarray(inputs.q[b, row, h], dtype=np.uint16)
+    J = np.ascontiguousarray(np.asarray(sel, dtype=np.int64))
+    pos = s.prefix + int(row)
+    if J.size and (J.min() < 0 or J.max() > pos):
+        raise ValueError("attend_set: a key lies outside the row's causal range")
+    out = np.zeros(D, dtype=np.float64)
+    lib().orc_attend_set(_p(k_seq), _p(v_seq), Hkv * D, s.kv_head(h), D, _p(q), pos, float(s.rope_base),
+                         1.0 / np.sqrt(D), int(pos_offset), _p(J), int(J.size), _p(out))
+    return out

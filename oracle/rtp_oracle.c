@@ -304,6 +304,30 @@ int orc_head_rows(const uint16_t* k, const uint16_t* v, int64_t n_keys, int64_t 
   return 0;
 }
 
+/*
+ * Exact attention of one query row (bf16 bits q, pre-RoPE, at absolute position pos) over a
+ * given key set J: the final step of both head classes on its own, for comparing a result
+ * whose set legitimately differs from the oracle's (a cut exactly at the mass boundary).
+ */
+void orc_attend_set(const uint16_t* k, const uint16_t* v, int64_t kv_stride, int g, int D,
+                    const uint16_t* q, int64_t pos, double rope_base, double sm_scale,
+                    int64_t pos_offset, const int64_t* J, int64_t nJ, double* out) {
+  orc_kv kv;
+  kv.k = k + (int64_t)g * D;
+  kv.v = v + (int64_t)g * D;
+  kv.stride = kv_stride;
+  kv.D = D;
+  kv.base = rope_base;
+  kv.pos_offset = pos_offset;
+  kv.rot_tab = NULL;
+  kv.tab_lo = 0;
+  kv.tab_hi = -1;
+  double qv[512], qr[512];
+  for (int d = 0; d < D; ++d) qv[d] = orc_bf16(q[d]);
+  orc_rope(qv, (double)(pos + pos_offset), D, rope_base, qr);
+  orc_attend(qr, &kv, J, nJ, sm_scale, out);
+}
+
 /* Index scores s_j = (Wq^T q).(Wk^T k_j) for j < n (pre-RoPE), fp64. */
 void orc_index_scores(const uint16_t* k, int64_t n, int64_t kv_stride, int g, int D, int r,
                       const uint16_t* q, const float* wq, const float* wk, double* s) {

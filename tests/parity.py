@@ -7,7 +7,11 @@ Tolerances (from the method statement):
     boundary may also move when the oracle's cumulative mass before or after the last
     member lies within 1e-6 of p (fp summation may legitimately move the cut there);
   * selected mass (oracle probabilities over the GPU's set) >= p - 1e-5;
-  * attention outputs within 1e-2 max-abs and 1e-3 relative L2.
+  * attention outputs within 1e-2 max-abs and 1e-3 relative L2 -- against the oracle's output,
+    or, for a row whose set legitimately differs from the oracle's, against the oracle's exact
+    attention over the GPU's set.
+
+p crosses the C ABI as fp32, so the oracle is given the same fp32 value.
 """
 from __future__ import annotations
 
@@ -19,6 +23,11 @@ SET_TOL = 1e-6
 MASS_TOL = 1e-5
 ABS_TOL = 1e-2
 REL_L2_TOL = 1e-3
+
+
+def p32(p: float) -> float:
+    """The value p takes after crossing the ABI as a C float."""
+    return float(np.float32(p))
 
 
 def torch_bf16(bits: np.ndarray, device="cuda"):
@@ -100,18 +109,93 @@ def run_decode(x, *, top_p=None, heads=None, batches=None, max_select=0, sel_cap
     summary = {}
     for b in batches:
         for h in heads:
-            r = oracle.layer_rows(x, b, h, [0], top_p=p, want_pi=h in s.retrieval_heads)
-            refs.append(r.out[0])
+            r = oracle.layer_rows(x, b, h, [0], top_p=p32(p), want_pi=h in s.retrieval_heads)
+            ref_out = r.out[0]
             gpus.append(out[b, h])
             if h in s.retrieval_heads:
                 slot = s.retrieval_heads.index(h)
                 k = int(cnt[b, slot])
                 sel = idx[b, slot, :k].astype(np.int64)
                 assert np.all(np.diff(sel) > 0), "selected positions must be strictly ascending"
-                nd = check_selection(sel, r, 0, p, f"b={b} h={h}")
+                nd = check_selection(sel, r, 0, p32(p), f"b={b} h={h}")
                 assert abs(float(mass[b, slot]) - float(r.pi[0][sel].sum())) <= 1e-5
+                if nd:
+                    ref_out = oracle.attend_set(x, b, h, 0, sel)
                 summary[(b, h)] = (k, int(r.count[0]), nd)
+            refs.append(ref_out)
     err = check_outputs(np.stack(gpus), np.stack(refs), f"{s.name} p={p}")
     if own:
         layer.close()
     return {"out": out, "count": cnt, "summary": summary, "err": err}
+
+
+def bitmap_positions(words: np.ndarray, n: int) -> np.ndarray:
+    """Ascending positions j < n whose bit is set in a little-endian 32-bit word bitmap."""
+    bits = np.unpackbits(np.ascontiguousarray(words).view(np.uint8), bitorder="little")[:n]
+    return np.flatnonzero(bits).astype(np.int64)
+
+
+def run_prefill(x, *, top_p=None, rows=None, heads=None, batches=None, bitmap=True, layer=None,
+                check_sets=True, exact_sets=False):
+    """Prefill the workload's chunk on the GPU (one call, C = chunk) and check the given rows
+    (default: all) of the given heads against the oracle.  exact_sets: the GPU's sets must equal
+    the oracle's (for exact ties, where the order rule alone decides)."""
+    import torch
+
+    from long_context_sparse_idx16_b200 import Layer
+
+    s = x.spec
+    N, C = s.n_total, s.chunk
+    p = s.top_p if top_p is None else top_p
+    own = layer is None
+    if own:
+        layer = Layer.from_spec(s, x, max_seq=N, max_chunk=C)
+        build_cache(layer, x, N)
+    layer.set_top_p(p)
+    words = (N + 31) // 32 if bitmap else 0
+    q = torch_bf16(x.q)
+    out, st = layer.prefill_chunk(q, stats=True, bitmap_words=words)
+    assert layer.check() == 0, "kernel error word set"
+    rows = np.arange(C) if rows is None else np.asarray(rows)
+    rows_t = torch.as_tensor(rows, device=out.device)
+    out_r = out[:, rows_t].cpu().numpy()
+    cnt = st[0][:, rows_t].cpu().numpy() if st else None
+    mass = st[1][:, rows_t].cpu().numpy() if st else None
+    heads = range(s.n_q_heads) if heads is None else heads
+    batches = range(s.batch) if batches is None else batches
+    summary = {}
+    refs, gpus = [], []
+    for b in batches:
+        for h in heads:
+            ret = h in s.retrieval_heads
+            r = oracle.layer_rows(x, b, h, rows, top_p=p32(p), want_pi=ret and check_sets)
+            ref_out = r.out.copy()
+            refs.append(ref_out)
+            gpus.append(out_r[b, :, h])
+            if not ret:
+                continue
+            slot = s.retrieval_heads.index(h)
+            ndiff = 0
+            for t, i in enumerate(rows):
+                k = int(cnt[b, t, slot])
+                if not check_sets:
+                    continue
+                pos = s.prefix + int(i)
+                if st[2] is not None:
+                    sel = bitmap_positions(st[2][b, int(i), slot].cpu().numpy(), pos + 1)
+                    assert len(sel) == k, f"b={b} h={h} row={i}: bitmap has {len(sel)} keys, count {k}"
+                    if exact_sets:
+                        assert np.array_equal(sel, r.sel[t]), f"b={b} h={h} row={i}: set differs"
+                    nd = check_selection(sel, r, t, p32(p), f"b={b} h={h} row={i}")
+                    assert abs(float(mass[b, t, slot]) - float(r.pi[t][sel].sum())) <= MASS_TOL, \
+                        f"b={b} h={h} row={i}: mass {mass[b, t, slot]} vs {r.pi[t][sel].sum()}"
+                    if nd:
+                        ref_out[t] = oracle.attend_set(x, b, h, int(i), sel)
+                    ndiff += nd
+                else:
+                    assert float(mass[b, t, slot]) >= p - MASS_TOL
+            summary[(b, h)] = (cnt[b, :, slot].copy(), r.count.copy(), ndiff)
+    err = check_outputs(np.stack(gpus), np.stack(refs), f"{s.name} prefill p={p}")
+    if own:
+        layer.close()
+    return {"out": out_r, "count": cnt, "summary": summary, "err": err}

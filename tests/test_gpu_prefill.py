@@ -1,0 +1,104 @@
+"""GPU chunked-prefill parity: every row of the chunk runs its own top-p selection (retrieval
+heads) or its own window (local heads); the CUDA path through the C ABI against the fp64 oracle."""
+import numpy as np
+import pytest
+
+import synth
+from parity import build_cache, run_prefill, torch_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def small(name="prefill_32k", **kw):
+    base = dict(prefix=0, chunk=300, window=96, n_clusters=8, needles=(64,))
+    base.update(kw)
+    return synth.generate(synth.spec(name, **base))
+
+
+def test_prefill_small_from_empty():
+    # 300 rows = four full 64-row tiles and a ragged tail of 44; keys 0..299
+    run_prefill(small())
+
+
+def test_prefill_small_with_prefix():
+    # rows at positions 1000..1199 over a 1200-key cache; rows of one tile need different cuts
+    run_prefill(small(prefix=1000, chunk=200, window=128))
+
+
+@pytest.mark.parametrize("p", [0.05, 0.5, 0.95, 0.999, 1.0])
+def test_prefill_p_sweep(p):
+    run_prefill(small(prefix=700, chunk=130, needles=()), top_p=p)
+
+
+def test_prefill_all_ties():
+    # every index score is exactly 0: each row keeps the lowest ceil(p (pos+1)) positions
+    x = small(prefix=500, chunk=150, zero_index_weights=True, needles=())
+    res = run_prefill(x, exact_sets=True)
+    p = float(np.float32(0.9))  # p as the ABI carries it
+    for (b, h), (cnt, cnt_ref, nd) in res["summary"].items():
+        pos = x.spec.prefix + np.arange(x.spec.chunk)
+        assert np.array_equal(cnt, np.ceil(p * (pos + 1)).astype(np.int64)) and nd == 0
+
+
+@pytest.mark.parametrize("W,S", [(1, 0), (1, 4), (7, 0), (100000, 4), (64, 70)])
+def test_prefill_window_shapes(W, S):
+    run_prefill(small(prefix=400, chunk=140, window=W, n_sink=S))
+
+
+def test_prefill_single_row_and_gqa_shapes():
+    run_prefill(small(prefix=999, chunk=1))
+    run_prefill(small(prefix=300, chunk=100, n_kv_heads=8))  # MHA
+    run_prefill(small(prefix=300, chunk=100, n_q_heads=16, n_kv_heads=1, retrieval_heads=(3, 9, 15)))
+
+
+def test_prefill_two_chunks_in_sequence():
+    # the second chunk's rows see the first chunk's keys through the cache
+    from long_context_sparse_idx16_b200 import Layer
+
+    x = small(prefix=0, chunk=512)
+    s = x.spec
+    layer = Layer.from_spec(s, x, max_seq=s.n_total, max_chunk=256)
+    build_cache(layer, x, 256)
+    first = layer.prefill_chunk(torch_bf16(x.q[:, :256]))
+    build_cache(layer, x, 512)
+    second = layer.prefill_chunk(torch_bf16(x.q[:, 256:]))
+    assert layer.check() == 0
+    import torch
+
+    whole = torch.cat([first, second], dim=1).cpu().numpy()
+    import oracle
+    from parity import check_outputs
+
+    for h in range(s.n_q_heads):
+        rows = np.arange(0, 512, 37)
+        ref = oracle.layer_rows(x, 0, h, rows).out
+        check_outputs(whole[0, rows, h], ref, f"two chunks h={h}")
+    layer.close()
+
+
+def test_prefill_multi_tile_keys_batch2():
+    # keys span many 64-key tiles; B=2 with needles planted in different heads
+    run_prefill(small(batch=2, prefix=1800, chunk=260, window=512, needles=(1, 16)))
+
+
+def test_prefill_deterministic():
+    x = small(prefix=600, chunk=128)
+    a = run_prefill(x)["out"]
+    b = run_prefill(x)["out"]
+    assert np.array_equal(a, b)
+
+
+@pytest.mark.slow
+def test_prefill_32k_full_sampled_rows():
+    # the full 32K chunk (B=1, C=32768 from an empty cache); rows sampled across the chunk
+    x = synth.generate(synth.spec("prefill_32k"))
+    rows = [0, 1, 63, 64, 4095, 4096, 8191, 8192, 16383, 20000, 32700, 32767]
+    run_prefill(x, rows=rows, heads=[0, 1, 7, 13, 19, 26, 31])
+
+
+@pytest.mark.slow
+def test_prefill_1m_full_sampled_rows():
+    # a 16384-row chunk on a 1032192-key prefix; counts and outputs on sampled rows
+    x = synth.generate(synth.spec("prefill_1m"))
+    rows = [0, 5, 8191, 8192, 16383]
+    run_prefill(x, rows=rows, heads=[0, 2, 13, 26], bitmap=False)

@@ -300,6 +300,27 @@ def test_sparse_attention_equals_attention_over_the_selected_set():
         assert np.allclose(res.out[t], ref, atol=1e-10)
 
 
+def test_attend_set_single_key_and_arbitrary_sets():
+    # one key: the softmax weight is 1, so the output is that key's value row exactly
+    s = synth.spec("prefill_32k", chunk=64, prefix=100, window=32, needles=())
+    x = synth.generate(s)
+    vf = bf16_bits_to_f32(x.v[0]).astype(np.float64)
+    for h, row, j in [(0, 0, 0), (9, 5, 77), (31, 63, 163)]:
+        out = oracle.attend_set(x, 0, h, row, [j])
+        assert np.array_equal(out, vf[j, s.kv_head(h)])
+    # an arbitrary set: brute-force attention over exactly those keys
+    kf = bf16_bits_to_f32(x.k[0]).astype(np.float64)
+    qf = bf16_bits_to_f32(x.q[0]).astype(np.float64)
+    rng = np.random.default_rng(3)
+    for h, row in [(2, 10), (26, 60)]:
+        i = s.prefix + row
+        J = sorted(rng.choice(i + 1, size=37, replace=False).tolist())
+        ref = _brute_attention(qf[row, h], kf[:, s.kv_head(h)], vf[:, s.kv_head(h)], i, J)
+        assert np.allclose(oracle.attend_set(x, 0, h, row, J), ref, atol=1e-10)
+    with pytest.raises(ValueError):
+        oracle.attend_set(x, 0, 0, 0, [s.prefix + 1])  # a key after the row
+
+
 def test_gqa_maps_heads_to_their_kv_head():
     s = synth.spec("toy_decode_4k", n_kv_heads=8, retrieval_heads=(0, 5), prefix=255, window=64,
                    needles=())
