@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "RTPurbo attn layer: decode µs/token & prefill ms at 128K/1M; % of roofline"
 DECODE_WORKLOADS = ("decode_128k", "decode_1m")
+PREFILL_WORKLOADS = ("prefill_32k", "prefill_1m")
 
 
 def _peaks():
@@ -42,6 +43,17 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def _tensor_peak():
+    """Dense 16-bit tensor peak (TFLOP/s): the measured cuBLAS bf16 burst figure (fp16 runs at
+    the same nominal rate), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (bf16 burst; fp16 has the same nominal rate)"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def _profile_traffic(kernel_src: str):
@@ -144,6 +156,40 @@ def cpu_oracle_sample(x, seconds: float = 12.0):
     return dt / done * 1e6, oracle.max_threads(), f"decode step of {done} of {s.batch} sequences, all {s.n_q_heads} heads"
 
 
+def cpu_oracle_prefill_sample(x, seconds: float = 12.0):
+    """Time the fp64 oracle (as it stands) on chunk rows spread over the chunk, one retrieval
+    and one local head per row, until about `seconds`; returns (ms per chunk, cores,
+    description), the chunk time being mean row time per class x rows x heads per class."""
+    import numpy as np
+
+    import oracle
+
+    s = x.spec
+    C = s.chunk
+    Hr = len(s.retrieval_heads)
+    loc = [h for h in range(s.n_q_heads) if h not in s.retrieval_heads]
+    rows = np.linspace(0, C - 1, 64).astype(np.int64)
+    tr = tl = 0.0
+    n = 0
+    t_start = time.perf_counter()
+    for i, row in enumerate(rows):
+        b = i % s.batch
+        t0 = time.perf_counter()
+        oracle.layer_rows(x, b, s.retrieval_heads[i % Hr], [int(row)], want_sel=False)
+        t1 = time.perf_counter()
+        if loc:
+            oracle.layer_rows(x, b, loc[i % len(loc)], [int(row)], want_sel=False)
+        t2 = time.perf_counter()
+        tr += t1 - t0
+        tl += t2 - t1
+        n += 1
+        if t2 - t_start >= seconds:
+            break
+    ms = (tr / n * Hr + tl / n * len(loc)) * C * s.batch * 1e3
+    return ms, oracle.max_threads(), (f"{n} chunk rows spread over the chunk, one retrieval and one local head each; "
+                                      f"chunk time = mean row time per class x {C} rows x heads per class x {s.batch}")
+
+
 def run_reference(args):
     """The oracle arm.  Each step runs the oracle on one retrieval head and one local head of one
     sequence (cycling over all of them); the token time is estimated as
@@ -155,6 +201,8 @@ def run_reference(args):
 
     x = _generate(args)
     s = x.spec
+    if args.workload in PREFILL_WORKLOADS:
+        return _run_reference_prefill(args, x)
     ret = [(b, h) for b in range(s.batch) for h in s.retrieval_heads]
     loc = [(b, h) for b in range(s.batch) for h in range(s.n_q_heads) if h not in s.retrieval_heads]
     budget = 200.0
@@ -199,6 +247,71 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _run_reference_prefill(args, x):
+    """Oracle arm for a prefill workload: each step runs one retrieval-head row and one
+    local-head row (rows and heads cycling over the chunk); chunk time = mean row time per
+    class x rows x heads per class x sequences."""
+    import numpy as np
+
+    import oracle
+
+    s = x.spec
+    C = s.chunk
+    Hr = len(s.retrieval_heads)
+    loc = [h for h in range(s.n_q_heads) if h not in s.retrieval_heads]
+    rows = np.linspace(0, C - 1, 97).astype(np.int64)
+    budget = 200.0
+
+    def one(i):
+        row, b = int(rows[i % len(rows)]), i % s.batch
+        t0 = time.perf_counter()
+        oracle.layer_rows(x, b, s.retrieval_heads[i % Hr], [row], want_sel=False)
+        t1 = time.perf_counter()
+        if loc:
+            oracle.layer_rows(x, b, loc[i % len(loc)], [row], want_sel=False)
+        return t1 - t0, time.perf_counter() - t1
+
+    for i in range(args.warmup):
+        one(i)
+    tr = tl = 0.0
+    n = 0
+    t_start = time.perf_counter()
+    for i in range(args.steps):
+        a, b = one(args.warmup + i)
+        tr += a
+        tl += b
+        n += 1
+        if time.perf_counter() - t_start > budget:
+            break
+    dt = time.perf_counter() - t_start
+    ms = (tr / n * Hr + tl / n * len(loc)) * C * s.batch * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": ms, "unit": "ms/chunk", "n_gpus": args.gpus,
+        "steps": n, "warmup": args.warmup, "ms_per_step": dt / n * 1e3, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _prefill_config(s, args.gpus),
+        "cpu_baseline": {"value": ms, "unit": "ms/chunk", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"{n} steps of one retrieval-head row + one local-head row, cycling over rows "
+                                   f"spread across the chunk; chunk time = mean row time per class x rows x heads"
+                                   + (" (stopped at the time budget)" if n < args.steps else "")},
+        "e2e": {"value": ms, "unit": "ms/chunk", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _prefill_config(s, n_gpus):
+    Hr = len(s.retrieval_heads)
+    return {"workload": (f"{s.name}: chunked prefill, B={s.batch}, prefix={s.prefix}, chunk={s.chunk}, "
+                         f"{s.n_q_heads} q / {s.n_kv_heads} kv heads, D={s.head_dim}, {Hr} retrieval heads "
+                         f"r={s.index_dim} p={s.top_p}, local W={s.window} S={s.n_sink}"),
+            "global_batch": s.batch * n_gpus, "seq_len": s.n_total, "parallelism": f"replicas x{n_gpus}",
+            "l2": "inputs larger than L2 (q %.0f MB, q_rot %.0f MB and out %.0f MB per step)" % (
+                s.batch * s.chunk * s.n_q_heads * s.head_dim * 2 / 1e6,
+                s.batch * s.chunk * s.n_q_heads * s.head_dim * 4 / 1e6,
+                s.batch * s.chunk * s.n_q_heads * s.head_dim * 4 / 1e6)}
 
 
 def _generate(args):
@@ -377,13 +490,171 @@ def run_gpu(args):
     return 0
 
 
+def _local_pairs(s) -> int:
+    """Sum over chunk rows of the local-head key count |J_i| (sinks + window, causal)."""
+    import numpy as np
+
+    pos = s.prefix + np.arange(s.chunk, dtype=np.int64)
+    sinks = np.minimum(s.n_sink, pos + 1)
+    w0 = np.maximum(s.n_sink, pos - s.window + 1)
+    return int((sinks + np.maximum(0, pos - w0 + 1)).sum())
+
+
+def run_prefill_gpu(args):
+    """A step is one chunked-prefill call of the workload: the chunk's K/V are appended
+    (RoPE + index keys) after the length is rolled back to the prefix, then every row of the
+    chunk runs its selection / window and attention."""
+    import numpy as np
+    import torch
+
+    import synth
+    from long_context_sparse_idx16_b200 import Layer
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    s = _spec(args)
+    x = synth.generate(s)
+    N, B, P, C = s.n_total, s.batch, s.prefix, s.chunk
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    layer = Layer.from_spec(s, x, max_seq=N, max_chunk=C)
+    for t0 in range(0, P, 1 << 16):
+        t1 = min(P, t0 + (1 << 16))
+        layer.append_kv(bf16(x.k[:, t0:t1]).to(dev), bf16(x.v[:, t0:t1]).to(dev))
+    k_c = bf16(x.k[:, P:N]).to(dev).contiguous()
+    v_c = bf16(x.v[:, P:N]).to(dev).contiguous()
+    q = bf16(x.q).to(dev).contiguous()
+    out = torch.empty((B, C, s.n_q_heads, 128), dtype=torch.float32, device=dev)
+
+    def step():
+        layer.truncate(P)
+        layer.append_kv(k_c, v_c)
+        layer.prefill_chunk(q, out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert layer.check() == 0
+    _, st = layer.prefill_chunk(q, out, stats=True)
+    counts = st[0].cpu().numpy()
+    assert layer.check() == 0
+
+    clocks = ClockSampler(local)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
+    assert layer.check() == 0
+
+    layer.profile(True)
+    layer.profile_read()
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    per = {}
+    for k in ("prefill_retrieval", "prefill_local", "append_kv", "q_prep"):
+        per[k] = layer.profile_read(k)
+    rest_ms, rest_n = layer.profile_read(None)
+    layer.profile(False)
+    all_n = sum(n for _, n in per.values()) + rest_n
+
+    # end to end: q and the chunk's K/V from pinned host memory, the output back to the host
+    q_h = q.cpu().pin_memory()
+    k_h = k_c.cpu().pin_memory()
+    v_h = v_c.cpu().pin_memory()
+    o_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(k_c), torch.empty_like(v_c)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        layer.truncate(P)
+        layer.append_kv(k_d, v_d)
+        layer.prefill_chunk(q_d, out)
+        o_h.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(f0.elapsed_time(f1), world, dev)
+
+    chunks = B * args.steps * world
+    value = ms / (args.steps)  # ms per chunk call (B sequences each) on one GPU
+    peak, peak_kind = _tensor_peak()
+    Hr = len(s.retrieval_heads)
+    Hl = s.n_q_heads - Hr
+    local_flops = 4 * s.head_dim * _local_pairs(s) * Hl * B
+    ret_flops = 4 * s.head_dim * int(counts.sum())
+    kern = {}
+    for k, (kms, kn) in per.items():
+        kern[k] = {"ms_per_launch": kms / max(kn, 1), "launches": kn}
+    lk, rk = kern["prefill_local"], kern["prefill_retrieval"]
+    dom = "prefill_local" if lk["ms_per_launch"] >= rk["ms_per_launch"] else "prefill_retrieval"
+    dom_flops = local_flops if dom == "prefill_local" else ret_flops
+    achieved = dom_flops / (kern[dom]["ms_per_launch"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "ms/chunk", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 mma / f32", "data": "synthetic",
+        "config": _prefill_config(s, world),
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "flops_per_launch": dom_flops, "ms_per_launch": kern[dom]["ms_per_launch"]},
+        "kernels": kern,
+        "flops": {"local_attention": local_flops, "retrieval_attention": ret_flops,
+                  "index_scores": Hr * B * (C * P + C * (C + 1) // 2)},
+        "e2e": {"value": e2e_ms / args.steps, "unit": "ms/chunk",
+                "h2d_bytes_per_step": int((q.numel() + k_c.numel() + v_c.numel()) * 2),
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": int(all_n),
+        "selected_tokens": {"min": int(counts.min()), "median": float(np.median(counts)), "max": int(counts.max()),
+                            "mean": float(counts.mean())},
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        v, cores, desc = cpu_oracle_prefill_sample(x)
+        line["cpu_baseline"] = {"value": v, "unit": "ms/chunk", "cores": cores, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=DECODE_WORKLOADS, default="decode_128k",
+    ap.add_argument("--workload", choices=DECODE_WORKLOADS + PREFILL_WORKLOADS, default="decode_128k",
                     help="measured workload (the default is the headline one; others are for profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -392,6 +663,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload in PREFILL_WORKLOADS:
+        return run_prefill_gpu(args)
     return run_gpu(args)
 
 

@@ -28,3 +28,16 @@ def test_bench_help():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True, text=True,
                        timeout=120, cwd=ROOT)
     assert r.returncode == 0 and "--impl" in r.stdout
+
+
+@pytest.mark.slow
+def test_reference_arm_prefill_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "3", "--workload", "prefill_32k"],
+                       capture_output=True, text=True, timeout=900, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "ms/chunk" and d["value"] > 0
+    assert "prefill_32k" in d["config"]["workload"]
