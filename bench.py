@@ -571,7 +571,7 @@ def run_prefill_gpu(args):
         step()
     torch.cuda.synchronize()
     per = {}
-    for k in ("prefill_retrieval", "prefill_local", "append_kv", "q_prep"):
+    for k in ("prefill_select", "prefill_attn", "prefill_local", "append_kv", "q_prep"):
         per[k] = layer.profile_read(k)
     rest_ms, rest_n = layer.profile_read(None)
     layer.profile(False)
@@ -614,8 +614,8 @@ def run_prefill_gpu(args):
     kern = {}
     for k, (kms, kn) in per.items():
         kern[k] = {"ms_per_launch": kms / max(kn, 1), "launches": kn}
-    lk, rk = kern["prefill_local"], kern["prefill_retrieval"]
-    dom = "prefill_local" if lk["ms_per_launch"] >= rk["ms_per_launch"] else "prefill_retrieval"
+    lk, rk = kern["prefill_local"], kern["prefill_attn"]
+    dom = "prefill_local" if lk["ms_per_launch"] >= rk["ms_per_launch"] else "prefill_attn"
     dom_flops = local_flops if dom == "prefill_local" else ret_flops
     achieved = dom_flops / (kern[dom]["ms_per_launch"] * 1e-3) / 1e12
     line = {

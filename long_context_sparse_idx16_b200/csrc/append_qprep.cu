@@ -2,7 +2,8 @@
 //
 // Append (rtp_append_kv): for each new token at position pos and KV head g,
 //   K[g][pos] = fp16(RoPE(k, pos)), V[g][pos] = fp16(v), and for every retrieval head h
-//   whose KV head is g: IDX[h][pos] = Wk_h^T k (pre-RoPE, fp32).
+//   whose KV head is g: IDX[h][pos] = Wk_h^T k (pre-RoPE, fp32), also kept split as fp16
+//   hi + lo for the tensor-core scoring of prefill.
 // The indexer projects pre-RoPE keys (ngjoo digest, core method: "low-dimensional pre-RoPE
 // projections"; aitntnews page, finding 2: project D=128 down to r=16 so that the
 // high-frequency RoPE components do not disturb long-range matching).
@@ -26,7 +27,7 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
     int Hr, int64_t pos0, int64_t max_seq, const double* __restrict__ theta,
     const float* __restrict__ wk, const int16_t* __restrict__ ret_head, int group,
     __half* __restrict__ kc, __half* __restrict__ vc, float* __restrict__ idx,
-    uint32_t* __restrict__ err) {
+    __half* __restrict__ idx_hl, uint32_t* __restrict__ err) {
   const int t = blockIdx.x;  // token within the appended block
   const int b = blockIdx.y;
   const int64_t pos = pos0 + t;
@@ -65,7 +66,12 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
     float acc = 0.f;
 #pragma unroll 8
     for (int d = 0; d < kD; ++d) acc = fmaf(w[d * kR], x[d], acc);
-    idx[(((int64_t)b * Hr + hr) * max_seq + pos) * kR + c] = acc;
+    const int64_t row = ((int64_t)b * Hr + hr) * max_seq + pos;
+    idx[row * kR + c] = acc;
+    // the same key split as fp16 hi + lo, for the tensor-core scoring of prefill
+    const __half h = __float2half_rn(acc);
+    idx_hl[row * (2 * kR) + c] = h;
+    idx_hl[row * (2 * kR) + kR + c] = __float2half_rn(acc - __half2float(h));
   }
   if (bad) atomicOr(err, kErrRange);
 }
@@ -131,7 +137,7 @@ cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const _
   size_t smem = (size_t)L->Hkv * kD * sizeof(float);
   append_kv_kernel<<<grid, 256, smem, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta,
                                             L->wk, L->d_ret_head, L->group, L->kc, L->vc, L->idx,
-                                            L->err);
+                                            L->idx_hl, L->err);
   return cudaGetLastError();
 }
 

@@ -62,8 +62,9 @@ __device__ __forceinline__ void fa_stage(unsigned char* ksm, unsigned char* vsm,
   }
 }
 
-// One key tile: visible(r, t) says whether row r (0..63 within the CTA) may attend to tile key t.
-template <typename VisFn>
+// One key tile: visible(r, t) says whether row r (0..63 within the CTA) may attend to tile key t
+// (not consulted when kMasked is false: every row sees every key of the tile).
+template <bool kMasked = true, typename VisFn>
 __device__ __forceinline__ void fa_tile(FaAcc& A, const uint32_t qa[8][4], const unsigned char* ksm,
                                         const unsigned char* vsm, float scale_log2, VisFn visible) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gr = lane >> 2, tq = lane & 3;
@@ -90,8 +91,13 @@ __device__ __forceinline__ void fa_tile(FaAcc& A, const uint32_t qa[8][4], const
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int t = nt * 8 + 2 * tq + e;
-      s[nt][e] = visible(r0, t) ? s[nt][e] * scale_log2 : -INFINITY;
-      s[nt][2 + e] = visible(r1, t) ? s[nt][2 + e] * scale_log2 : -INFINITY;
+      if (kMasked) {
+        s[nt][e] = visible(r0, t) ? s[nt][e] * scale_log2 : -INFINITY;
+        s[nt][2 + e] = visible(r1, t) ? s[nt][2 + e] * scale_log2 : -INFINITY;
+      } else {
+        s[nt][e] *= scale_log2;
+        s[nt][2 + e] *= scale_log2;
+      }
       mx0 = fmaxf(mx0, s[nt][e]);
       mx1 = fmaxf(mx1, s[nt][2 + e]);
     }

@@ -70,12 +70,23 @@ __global__ void __launch_bounds__(kFaThreads) prefill_local_kernel(LocalArgs a) 
     __syncthreads();
     const unsigned char* ks = sm + (t & 1) * 2 * kFaTileBytes;
     const int64_t u0 = (int64_t)t * kFaKeys;
-    fa_tile(A, qa, ks, ks + kFaTileBytes, a.scale_log2, [&](int r, int tt) {
+    auto vis = [&](int r, int tt) {
       const int64_t u = u0 + tt;
       if (r >= nrows || u >= n_keys) return false;
       const int64_t j = pos_of(u), pos = pos_min + r;
       return j <= pos && (j < a.S || pos - j < a.W);
-    });
+    };
+    // a tile whose keys every row of the CTA sees needs no mask: a full tile of one segment
+    // (sinks or window), with its last key at or before the first row and, for window keys,
+    // its first key inside the last row's window
+    bool full = false;
+    if (nrows == kFaRows && u0 + kFaKeys <= n_keys) {
+      const int64_t j_lo = pos_of(u0), j_hi = pos_of(u0 + kFaKeys - 1);
+      const bool one_seg = (u0 + kFaKeys <= s_cnt) || (u0 >= s_cnt);
+      full = one_seg && j_hi <= pos_min && (j_hi < a.S || pos_max - j_lo < a.W);
+    }
+    if (full) fa_tile<false>(A, qa, ks, ks + kFaTileBytes, a.scale_log2, vis);
+    else fa_tile<true>(A, qa, ks, ks + kFaTileBytes, a.scale_log2, vis);
     __syncthreads();
   }
   float* obase = a.out + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD;

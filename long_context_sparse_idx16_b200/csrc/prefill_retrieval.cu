@@ -1,47 +1,51 @@
-// prefill_retrieval.cu -- retrieval heads in chunked prefill: per-row top-p + sparse attention.
+// prefill_retrieval.cu -- retrieval heads in chunked prefill: per-row exact top-p, then sparse
+// attention over the selected keys.
 //
 // Every query row i of the chunk (position pos = len - C + i) runs its own selection over its
-// causal prefix j <= pos: pre-RoPE index scores s_j = qidx_i . IDX[j] (techwalker page,
-// section 3), the shortest prefix of the order (s desc, j asc) whose index-softmax mass reaches
-// p (zhichai page, insight 3; techwalker page, section 4), then exact RoPE'd attention over
-// that set.  (The pages' own prefill keeps retrieval heads dense -- techwalker page, limits;
-// ngjoo digest, limitations -- the per-row selection here is the chunked-prefill counterpart
-// of the decode selection.)
+// causal prefix j <= pos: pre-RoPE index scores s_j = qidx_i . kidx_j (techwalker page, section
+// 3), the shortest prefix of the order (s desc, j asc) whose index-softmax mass reaches p
+// (zhichai page, insight 3; techwalker page, section 4), then exact RoPE'd attention over that
+// set.  (The pages' own prefill keeps retrieval heads dense -- techwalker page, Q&A; ngjoo
+// digest, limitations -- the per-row selection here is the chunked-prefill counterpart of the
+// decode selection.)
 //
-// One CTA per (64-row tile, retrieval head, sequence), 128 threads.  Rows are independent,
-// so every step stays inside the CTA:
-//   * scoring: thread t owns row t % 64 and half (t / 64) of every 64-key index tile (staged in
-//     shared memory, read as broadcasts); a score is a fixed-order fp32 dot product, so every
-//     pass -- and the attention mask -- recomputes bit-identical scores;
-//   * pass A: row maxima;  pass B: fixed-point mass histogram (64 bins of width 1/4 below the
-//     max, keys 16..32 below summed apart, the rest negligible -- same argument as the decode
-//     selection) -> total mass Z, target T = ceil(p Z), crossing bin;
-//   * refinement passes: inside the crossing bin, 64-way splits of the order-key range (exact
-//     integer arithmetic) until a row's range holds <= 32 keys, which are sorted to give the
-//     exact cut key t and tie cutoff; a range that shrinks to one key value with more members
-//     is an exact tie, resolved by an ordered count of the tied positions;
-//   * attention pass: for each key tile the selection mask (s > t, or s == t and j <= cutoff)
-//     is recomputed; tiles no row selects are skipped, the others run on tensor cores
-//     (fa_tile.cuh) with the mask.
+// Two kernels, one CTA per (64-row tile, retrieval head, sequence), 128 threads each; scores
+// come from index_mma.cuh (tensor cores, identical bits in every pass):
+//
+//  prefill_select_kernel -- the exact cut (t_key, tiecut) of each row, in passes over the
+//    row's causal keys, all arithmetic exact in 64-bit fixed point (mass of key j =
+//    round(2^sc * e^(s_j - m)), sc = 62 - ceil(log2 len)):
+//      A  row maxima m;
+//      B  16 bins of m - s rounded to an integer (the last one holding everything from 14.5
+//         down) -> Z, T = ceil(p Z), crossing bin, whose exact order-key range is found by
+//         bisection;
+//      R  refinement: the crossing range of order keys is split 16 ways by bit slices, with
+//         the mass of each slice and the first keys of the range captured; once a row's
+//         range holds <= 16 keys they are sorted (key desc, j asc) for the exact cut; a range
+//         that shrinks to one key value is an exact tie group, resolved by
+//      T  an ordered count of the tied positions.
+//  prefill_attn_kernel -- recomputes the scores, applies each row's cut, ORs the rows' masks
+//    of every 64-key tile into the tile's union, compacts the union keys of successive tiles
+//    into 64-key chunks (positions + per-row bits) and runs the attention tiles (fa_tile.cuh)
+//    on the gathered K/V rows of each full chunk; tiles no row selects cost only their scores.
 #include "fa_tile.cuh"
+#include "index_mma.cuh"
 #include "rtp_internal.h"
 
 namespace rtp {
 
 namespace {
 
-constexpr int kRows = kFaRows;          // 64 query rows per CTA
-constexpr int kKeys = 64;               // index keys per tile
-constexpr int kThreads = kFaThreads;    // 128: two threads per row
-constexpr int kHalf = kKeys / 2;        // keys per thread per tile
-constexpr int kBins = 64;
-constexpr int kCandPerThread = 16;
+constexpr int kRows = 64;
+constexpr int kThreads = kIdxThreads;  // 128
+constexpr int kBins = 16;
+constexpr int kCand = 4;               // candidates captured per thread and row slot
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum : int { kModeHist = 0, kModeKeys = 1, kModeTie = 2, kModeDone = 3 };
+enum : int { kModeKeys = 1, kModeTie = 2, kModeDone = 3 };
 
 struct RetArgs {
-  const float* idx;           // [B][Hr][max_seq][r]
+  const __half* idx;          // [B][Hr][max_seq][hi r | lo r]: the split index cache
   const __half* kc;
   const __half* vc;
   int64_t max_seq;
@@ -52,6 +56,7 @@ struct RetArgs {
   const int16_t* ret_head;    // [Hr]
   const float* q_rot;         // [B][C][Hq][D]
   const float* q_idx;         // [B][C][Hr][r]
+  uint2* cut;                 // [B][Hr][C]: (t_key, tiecut)
   float scale_log2;
   float* out;                 // [B][C][Hq][D]
   int32_t* sel_count;         // [B][C][Hr] or nullptr
@@ -61,423 +66,669 @@ struct RetArgs {
   uint32_t* err;
 };
 
-struct RowSel {
+struct RowS {
   float m;
-  int mode;
-  int bin1;           // crossing level-1 bin (kBins: the 16..32 band)
-  int found;          // tie mode: cutoff located
-  uint32_t klo, khi;  // current order-key range (inclusive) inside bin1
-  uint32_t t_key;     // exact cut key
-  int tiecut;         // positions j <= tiecut with key t_key are selected
-  unsigned long long Z, rem, n_need, tie_before;
+  int mode, cb, shift, found, tiecut;
+  uint32_t klo, khi, t_key;
+  unsigned long long Z, rem, above, n_need, tie_before;
 };
 
-// Per-thread arrays are stored [item][thread] so that a warp touching item i of its own rows
-// hits consecutive words.
-struct SmemR {
-  RowSel row[kRows];
-  float ik[2][kKeys][kR];                          // index key tiles (8 KB)
-  unsigned long long cand[kCandPerThread][kThreads];  // refinement candidates (16 KB)
-  unsigned long long coarse[kThreads];
-  int ncand[kThreads];
-  uint32_t mask[kRows][2];                         // per-row 64-key masks (two halves)
-  union {
-    unsigned long long hist[kBins][kThreads];      // 64 KB: per-thread mass histograms
-    unsigned char kv[2 * kFaTileBytes];            // 32 KB: one K and one V tile
-  } u;
+// Per-thread exact histograms: a 64-bit mass is added as three 21-bit limbs with shared-memory
+// reductions (no read-modify-write chains); limb sums stay below 2^32 because every thread
+// folds its carries at least every kFoldTiles tiles (at most 16 keys per row slot per tile).
+constexpr int kLimbs = 3;
+constexpr int kFoldTiles = 128;
+
+struct SmemSel {
+  IdxRing st;                                     // 12 KB
+  uint32_t h[kBins][2][kLimbs][kThreads];         // 48 KB
+  unsigned long long cand[kCand][2][kThreads];    // 8 KB
+  int nc[2][kThreads];
+  RowS row[kRows];
 };
 
-__device__ __forceinline__ unsigned long long mass64(float s, float m, float scale) {
-  const float q = fast_exp2((s - m) * kLog2e) * scale;
-  const float qh = floorf(q * 2.3283064365386963e-10f);
-  const uint32_t hi = (uint32_t)qh, lo = __float2uint_rn(fmaf(qh, -4294967296.0f, q));
-  return ((unsigned long long)hi << 32) | lo;
+__device__ __forceinline__ void red_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// level-1 bin of a score below the row max: 0..63 (width 1/4), kBins (16..32), kBins+1 (tail)
-__device__ __forceinline__ int bin1_of(float s, float m) {
-  const float x = m - s;
-  if (x < 16.f) return (int)(x * 4.f);
-  if (x < 32.f) return kBins;
-  return kBins + 1;
+// Add mass v to bin b of row slot sl of this thread (three limb reductions).
+__device__ __forceinline__ void hist_add(SmemSel& S, int b, int sl, int tid, unsigned long long v) {
+  const uint32_t a0 = smem_u32(&S.h[b][sl][0][tid]);
+  red_add(a0, (uint32_t)v & 0x1FFFFFu);
+  red_add(a0 + kThreads * 4, (uint32_t)(v >> 21) & 0x1FFFFFu);
+  red_add(a0 + 2 * kThreads * 4, (uint32_t)(v >> 42));
 }
 
-__device__ __forceinline__ float score16(const float* qt, const float* k) {
-  const float4* k4 = reinterpret_cast<const float4*>(k);
-  float s = 0.f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const float4 v = k4[c];
-    s = fmaf(qt[4 * c + 0], v.x, s);
-    s = fmaf(qt[4 * c + 1], v.y, s);
-    s = fmaf(qt[4 * c + 2], v.z, s);
-    s = fmaf(qt[4 * c + 3], v.w, s);
-  }
-  return s + 0.0f;  // -0 -> +0: equal scores get equal order keys
+__device__ __forceinline__ unsigned long long hist_get(const SmemSel& S, int b, int sl, int t) {
+  return (unsigned long long)S.h[b][sl][0][t] + ((unsigned long long)S.h[b][sl][1][t] << 21) +
+         ((unsigned long long)S.h[b][sl][2][t] << 42);
 }
 
-// Order-key range [lo, hi] that contains every score whose level-1 bin is b (with margin;
-// membership is always re-tested with bin1_of).
-__device__ __forceinline__ void bin_key_range(float m, int b, uint32_t* lo, uint32_t* hi) {
-  const float x_lo = b < kBins ? 0.25f * b : 16.f;
-  const float x_hi = b < kBins ? 0.25f * (b + 1) : 32.f;
-  const float eps = 4.f * fmaxf(fabsf(m), 32.f) * 1.1920929e-7f;
-  *lo = order_key(m - x_hi - eps);
-  *hi = order_key(m - x_lo + eps);
-}
-
-// Stage index-key tile t (keys t*64 .. +63, zero beyond nkeys) into buffer buf.
-__device__ __forceinline__ void stage_ik(SmemR& S, int buf, const float* base, int64_t t, int64_t nkeys) {
-  const int tid = threadIdx.x;
-#pragma unroll
-  for (int i = 0; i < (kKeys * kR / 4) / kThreads; ++i) {  // 2 x 16 bytes per thread
-    const int idx = i * kThreads + tid;
-    const int r = idx >> 2, c4 = idx & 3;
-    const int64_t j = t * kKeys + r;
-    const bool ok = j < nkeys;
-    cp_async16(&S.ik[buf][r][c4 * 4], base + (ok ? j : 0) * kR + c4 * 4, ok ? 16 : 0);
-  }
-  cp_async_commit();
-}
-
-// Run f(j, s) over this thread's keys j <= pos (its half of every tile), tiles double-buffered.
-template <typename F>
-__device__ __forceinline__ void scan_keys(SmemR& S, const float* ibase, int64_t nkeys, int64_t pos, bool active,
-                                          const float* qt, F f) {
-  const int hf = threadIdx.x >> 6;
-  const int64_t ntiles = (nkeys + kKeys - 1) / kKeys;
-  stage_ik(S, 0, ibase, 0, nkeys);
-  for (int64_t t = 0; t < ntiles; ++t) {
-    if (t + 1 < ntiles) {
-      stage_ik(S, (t + 1) & 1, ibase, t + 1, nkeys);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+// Fold this thread's limb carries (its own entries only; same-thread order suffices).
+__device__ __forceinline__ void hist_fold(SmemSel& S, int tid) {
+  for (int b = 0; b < kBins; ++b)
+    for (int sl = 0; sl < 2; ++sl) {
+      const unsigned long long v = hist_get(S, b, sl, tid);
+      S.h[b][sl][0][tid] = (uint32_t)v & 0x1FFFFFu;
+      S.h[b][sl][1][tid] = (uint32_t)(v >> 21) & 0x1FFFFFu;
+      S.h[b][sl][2][tid] = (uint32_t)(v >> 42);
     }
-    __syncthreads();
-    if (active) {
-      const int buf = t & 1;
-#pragma unroll 4
-      for (int k = 0; k < kHalf; ++k) {
-        const int64_t j = t * kKeys + hf * kHalf + k;
-        if (j > pos) break;
-        f(j, score16(qt, S.ik[buf][hf * kHalf + k]));
+}
+
+__device__ __forceinline__ void hist_zero(SmemSel& S, int tid) {
+  for (int b = 0; b < kBins; ++b)
+    for (int sl = 0; sl < 2; ++sl)
+      for (int l = 0; l < kLimbs; ++l) S.h[b][sl][l][tid] = 0u;
+}
+
+// Fixed-point mass of a score s below the row max m: e^(s - m) * 2^sc truncated to an integer
+// (scale = 2^sc as a float, exact).
+__device__ __forceinline__ unsigned long long mass64(float s, float m, float scale) {
+  return __float2ull_rz(fast_exp2((s - m) * kLog2e) * scale);
+}
+
+// level-1 bin of x = m - s >= 0: x rounded to the nearest integer (adding 2^23 does the rounding),
+// with everything from 14.5 down in the last bin.  Non-increasing in s.
+__device__ __forceinline__ int bin1_of(float x) {
+  const uint32_t r = __float_as_uint(x + 8388608.0f) - 0x4B000000u;
+  return (int)min(r, (uint32_t)(kBins - 1));
+}
+
+// Exact order-key range [lo, hi] of the finite scores s <= m whose level-1 bin is b (bisection
+// on the monotone map key -> bin).
+__device__ __forceinline__ void bin_key_range(float m, int b, uint32_t* lo, uint32_t* hi) {
+  const uint32_t kmin = order_key(-3.4028234663852886e38f), kmax = order_key(m);
+  auto bin_of_key = [&](uint32_t k) { return bin1_of(m - key_to_float(k)); };
+  // first key with bin <= b
+  uint32_t l = kmin, h = kmax;
+  while (l < h) {
+    const uint32_t mid = l + ((h - l) >> 1);
+    if (bin_of_key(mid) <= b) h = mid;
+    else l = mid + 1;
+  }
+  *lo = l;
+  // last key with bin >= b: one below the first key with bin < b (kmax + 1 if none)
+  if (b == 0) {
+    *hi = kmax;
+    return;
+  }
+  l = *lo;
+  h = kmax;
+  if (bin_of_key(h) >= b) {
+    *hi = h;
+    return;
+  }
+  while (l < h) {
+    const uint32_t mid = l + ((h - l) >> 1);
+    if (bin_of_key(mid) < b) h = mid;
+    else l = mid + 1;
+  }
+  *hi = l - 1;
+}
+
+__device__ __forceinline__ int slice_shift(uint32_t klo, uint32_t khi) {
+  const uint32_t d = khi - klo;  // span - 1
+  const int bits = 32 - __clz(d);
+  return bits > 4 ? bits - 4 : 0;
+}
+
+struct RowCtx {
+  int tid, warp, gr, tq;
+  int ra, rb;          // CTA rows of slot 0 / 1
+  int64_t pa, pb;      // their positions (-1: inactive row)
+  int64_t pos_lo;      // position of CTA row 0 (every active row is at or after it)
+  int64_t nkeys;       // keys the CTA's rows can see
+};
+
+__device__ __forceinline__ RowCtx row_ctx(const RetArgs& a, int i0, int nrows) {
+  RowCtx x;
+  x.tid = threadIdx.x;
+  x.warp = x.tid >> 5;
+  x.gr = (x.tid & 31) >> 2;
+  x.tq = x.tid & 3;
+  x.ra = 16 * x.warp + x.gr;
+  x.rb = x.ra + 8;
+  x.pa = x.ra < nrows ? a.P0 + i0 + x.ra : -1;
+  x.pb = x.rb < nrows ? a.P0 + i0 + x.rb : -1;
+  x.pos_lo = a.P0 + i0;
+  x.nkeys = a.P0 + i0 + nrows;
+  return x;
+}
+
+// Pipelined walk over the index tiles of keys [0, nkeys): body(t, stage) runs once tile t is
+// in ring stage `stage` (kIdxStages - 1 tiles in flight, one barrier per tile).
+template <typename Body>
+__device__ __forceinline__ void idx_walk(IdxRing& R, const __half* base, int64_t nkeys, Body body) {
+  const int64_t ntiles = (nkeys + kIdxKeys - 1) / kIdxKeys;
+#pragma unroll
+  for (int s = 0; s < kIdxStages - 1; ++s) {
+    if (s < ntiles) idx_issue(R, s, base, s, nkeys);
+    cp_async_commit();
+  }
+  for (int64_t t = 0; t < ntiles; ++t) {
+    cp_async_wait<kIdxStages - 2>();
+    __syncthreads();  // tile t landed for every thread; stage (t - 1) % kIdxStages is free
+    const int64_t tn = t + kIdxStages - 1;
+    if (tn < ntiles) idx_issue(R, (int)(tn % kIdxStages), base, tn, nkeys);
+    cp_async_commit();
+    body(t, (int)(t % kIdxStages));
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+}
+
+// Run f(slot, j, s) over this thread's causal (row, key) pairs, tile by tile; fold() runs
+// after every kFoldTiles tiles.
+template <typename F, typename G>
+__device__ __forceinline__ void scan(IdxRing& S, const RowCtx& x, const __half* ibase, const uint32_t qh[4],
+                                     const uint32_t ql[4], F f, G fold) {
+  idx_walk(S, ibase, x.nkeys, [&](int64_t t, int stage) {
+    if (t > 0 && t % kFoldTiles == 0) fold();
+    float c[8][4];
+    idx_scores(c, qh, ql, S, stage);
+    const int64_t base = t * kIdxKeys;
+    // causal limits of the two rows inside this tile (-1: none, 63: all)
+    const int la = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pa - base));
+    const int lb = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pb - base));
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int p = 8 * nt + 2 * x.tq + e;
+        if (p <= la) f(0, base + p, c[nt][e]);
+        if (p <= lb) f(1, base + p, c[nt][2 + e]);
       }
     }
-    __syncthreads();
-  }
+  });
 }
 
-// Exact top-p cut of each row of the tile: on return S.row[r] holds (t_key, tiecut) such that
-// key j of row r is selected iff order_key(s_j) > t_key, or == t_key and j <= tiecut.
-__device__ void select_rows(SmemR& S, const RetArgs& a, const float* ibase, const float* qt, int64_t pos,
-                            int64_t nkeys, bool active, float scale) {
-  const int tid = threadIdx.x, r = tid & (kRows - 1), hf = tid >> 6;
+// As scan, for passes that touch few keys: gate(slot, s) is evaluated branch-free for every
+// pair, and f runs only on pairs that pass it, after one warp vote per tile.
+template <typename Gate, typename F, typename G>
+__device__ __forceinline__ void scan_gated(IdxRing& S, const RowCtx& x, const __half* ibase, const uint32_t qh[4],
+                                           const uint32_t ql[4], Gate gate, F f, G fold) {
+  idx_walk(S, ibase, x.nkeys, [&](int64_t t, int stage) {
+    if (t > 0 && t % kFoldTiles == 0) fold();
+    float c[8][4];
+    idx_scores(c, qh, ql, S, stage);
+    const int64_t base = t * kIdxKeys;
+    const int la = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pa - base));
+    const int lb = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pb - base));
+    uint32_t hit = 0;  // bit 2*(2nt+e)+slot
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int p = 8 * nt + 2 * x.tq + e;
+        const int k = 2 * nt + e;
+        hit |= (uint32_t)(p <= la && gate(0, c[nt][e])) << (2 * k);
+        hit |= (uint32_t)(p <= lb && gate(1, c[nt][2 + e])) << (2 * k + 1);
+      }
+    }
+    if (!__any_sync(0xffffffffu, hit != 0u)) return;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int p = 8 * nt + 2 * x.tq + e;
+        const int k = 2 * nt + e;
+        if (hit & (1u << (2 * k))) f(0, base + p, c[nt][e]);
+        if (hit & (1u << (2 * k + 1))) f(1, base + p, c[nt][2 + e]);
+      }
+    }
+  });
+}
 
-  // ---- pass A: row maxima
-  float mx = -INFINITY;
-  scan_keys(S, ibase, nkeys, pos, active, qt, [&](int64_t, float s) { mx = fmaxf(mx, s); });
-  S.u.hist[0][tid] = __float_as_uint(mx);  // exchange of the two halves
-  __syncthreads();
-  if (hf == 0) {
-    RowSel& R = S.row[r];
-    R.m = fmaxf(mx, __uint_as_float((uint32_t)S.u.hist[0][tid + kRows]));
-    R.mode = active ? kModeHist : kModeDone;
-    R.found = 0;
-    R.tie_before = 0;
+__global__ void __launch_bounds__(kThreads) prefill_select_kernel(RetArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  SmemSel& S = *reinterpret_cast<SmemSel*>(smem_raw);
+  const int tile = gridDim.x - 1 - blockIdx.x, hr = blockIdx.y, b = blockIdx.z;  // longest rows first
+  const int i0 = tile * kRows;
+  const int nrows = min(kRows, a.C - i0);
+  const RowCtx x = row_ctx(a, i0, nrows);
+  const int tid = x.tid;
+  const bool owner = x.tq == 0;
+  const float scale = __uint_as_float((uint32_t)(127 + a.sc_bits) << 23);  // 2^sc_bits
+  const __half* ibase = a.idx + ((int64_t)b * a.Hr + hr) * a.max_seq * (2 * kR);
+  uint2* cut = a.cut + ((int64_t)b * a.Hr + hr) * a.C + i0;
+
+  if (a.top_p >= 1.f) {  // p = 1 keeps every causal key (also those whose mass rounds to 0)
+    if (owner) {
+      if (x.pa >= 0) cut[x.ra] = make_uint2(0u, 0x7FFFFFFFu);
+      if (x.pb >= 0) cut[x.rb] = make_uint2(0u, 0x7FFFFFFFu);
+      if (a.sel_mass) {
+        if (x.pa >= 0) a.sel_mass[((int64_t)b * a.C + i0 + x.ra) * a.Hr + hr] = 1.f;
+        if (x.pb >= 0) a.sel_mass[((int64_t)b * a.C + i0 + x.rb) * a.Hr + hr] = 1.f;
+      }
+    }
+    return;
   }
-  __syncthreads();
 
-  // ---- pass B: level-1 mass histogram -> Z, T = ceil(p Z), crossing bin
+  uint32_t qh[4], ql[4];
   {
-    const float m = S.row[r].m;
-    for (int i = 0; i < kBins; ++i) S.u.hist[i][tid] = 0ull;
-    unsigned long long co = 0;
-    scan_keys(S, ibase, nkeys, pos, active, qt, [&](int64_t, float s) {
-      const int bb = bin1_of(s, m);
-      if (bb < kBins) S.u.hist[bb][tid] += mass64(s, m, scale);
-      else if (bb == kBins) co += mass64(s, m, scale);
-    });
-    S.coarse[tid] = co;
-    __syncthreads();
-    if (hf == 0 && active) {
-      RowSel& R = S.row[r];
-      unsigned long long Z = S.coarse[tid] + S.coarse[tid + kRows];
+    const int64_t qs = (int64_t)a.Hr * kR;
+    const float* q0 = a.q_idx + ((int64_t)b * a.C + i0) * qs + (int64_t)hr * kR;
+    idx_load_q(qh, ql, x.pa >= 0 ? q0 + x.ra * qs : nullptr, x.pb >= 0 ? q0 + x.rb * qs : nullptr);
+  }
+
+  // ---- pass A: row maxima (the 4 threads of a quad share their two rows)
+  float m[2] = {-INFINITY, -INFINITY};
+  scan(S.st, x, ibase, qh, ql, [&](int sl, int64_t, float s) { m[sl] = fmaxf(m[sl], s); }, [] {});
+#pragma unroll
+  for (int sl = 0; sl < 2; ++sl) {
+    m[sl] = fmaxf(m[sl], __shfl_xor_sync(0xffffffffu, m[sl], 1));
+    m[sl] = fmaxf(m[sl], __shfl_xor_sync(0xffffffffu, m[sl], 2));
+  }
+
+  // ---- pass B: 16 bins of width 1 below the max -> Z, T, crossing bin
+  hist_zero(S, tid);
+  scan(S.st, x, ibase, qh, ql, [&](int sl, int64_t, float s) {
+    hist_add(S, bin1_of(m[sl] - s), sl, tid, mass64(s, m[sl], scale));
+  }, [&] { hist_fold(S, tid); });
+  if (owner) {
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      const int r = sl ? x.rb : x.ra;
+      RowS& R = S.row[r];
+      R.m = m[sl];
+      R.found = 0;
+      R.tie_before = 0;
+      if ((sl ? x.pb : x.pa) < 0) {
+        R.mode = kModeDone;
+        continue;
+      }
+      unsigned long long hb[kBins];
+      unsigned long long Z = 0;
       for (int i = 0; i < kBins; ++i) {
-        S.u.hist[i][tid] += S.u.hist[i][tid + kRows];
-        Z += S.u.hist[i][tid];
+        hb[i] = hist_get(S, i, sl, tid) + hist_get(S, i, sl, tid + 1) + hist_get(S, i, sl, tid + 2) +
+                hist_get(S, i, sl, tid + 3);
+        Z += hb[i];
       }
       unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
       if (T < 1ull) T = 1ull;
       if (T > Z) T = Z;
       unsigned long long cum = 0;
-      int cb = kBins;  // bins run from the highest scores down
+      int cb = kBins - 1;  // bins run from the highest scores down
       for (int i = 0; i < kBins; ++i) {
-        if (cum + S.u.hist[i][tid] >= T) {
+        if (cum + hb[i] >= T) {
           cb = i;
           break;
         }
-        cum += S.u.hist[i][tid];
+        cum += hb[i];
       }
       R.Z = Z;
-      R.bin1 = cb;
+      R.cb = cb;
       R.rem = T - cum;
-      bin_key_range(R.m, cb, &R.klo, &R.khi);
+      R.above = cum;
+      bin_key_range(m[sl], cb, &R.klo, &R.khi);
+      R.shift = slice_shift(R.klo, R.khi);
       R.mode = kModeKeys;
     }
-    __syncthreads();
   }
+  __syncthreads();
 
-  // ---- refinement: split the key range of the crossing bin 64 ways until <= 2 x 16 keys remain
-  for (int level = 0; level < 8; ++level) {
-    const int need = (hf == 0 && S.row[r].mode == kModeKeys) ? 1 : 0;
+  // ---- refinement: 16-way bit slices of the crossing key range until <= 16 keys remain
+  for (int level = 0; level < 10; ++level) {
+    const int need = (S.row[x.ra].mode == kModeKeys) || (S.row[x.rb].mode == kModeKeys);
     if (!__syncthreads_or(need)) break;
-    const bool mine = active && S.row[r].mode == kModeKeys;
-    const float m = S.row[r].m;
-    const int b1 = S.row[r].bin1;
-    const uint32_t klo = S.row[r].klo, khi = S.row[r].khi;
-    const unsigned long long span = (unsigned long long)(khi - klo) + 1ull;
-    for (int i = 0; i < kBins; ++i) S.u.hist[i][tid] = 0ull;
-    int nc = 0;
-    scan_keys(S, ibase, nkeys, pos, mine, qt, [&](int64_t j, float s) {
-      if (bin1_of(s, m) != b1) return;
+    bool mine[2];
+    int sh[2];
+    uint32_t klo[2], khi[2];
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      const RowS& R = S.row[sl ? x.rb : x.ra];
+      mine[sl] = R.mode == kModeKeys;
+      sh[sl] = R.shift;
+      klo[sl] = R.klo;
+      khi[sl] = R.khi;
+    }
+    hist_zero(S, tid);
+    int nc[2] = {0, 0};
+    RowCtx xm = x;  // rows outside refinement see no keys
+    if (!mine[0]) xm.pa = -1;
+    if (!mine[1]) xm.pb = -1;
+    const uint32_t span[2] = {khi[0] - klo[0], khi[1] - klo[1]};
+    scan_gated(S.st, xm, ibase, qh, ql, [&](int sl, float s) { return order_key(s) - klo[sl] <= span[sl]; },
+               [&](int sl, int64_t j, float s) {
       const uint32_t key = order_key(s);
-      if (key < klo || key > khi) return;
-      const int sub = (int)(((unsigned long long)(key - klo) * kBins) / span);  // 0 = lowest keys
-      S.u.hist[sub][tid] += mass64(s, m, scale);
-      if (nc < kCandPerThread) S.cand[nc][tid] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)j);
-      ++nc;
-    });
-    S.ncand[tid] = nc;
+      {
+        hist_add(S, (int)((key - klo[sl]) >> sh[sl]), sl, tid, mass64(s, m[sl], scale));
+        if (nc[sl] < kCand) S.cand[nc[sl]][sl][tid] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)j);
+        ++nc[sl];
+      }
+    }, [&] { hist_fold(S, tid); });
+    S.nc[0][tid] = nc[0];
+    S.nc[1][tid] = nc[1];
     __syncthreads();
-    if (hf == 0 && mine) {
-      RowSel& W = S.row[r];
-      const int n0 = S.ncand[tid], n1 = S.ncand[tid + kRows];
-      if (n0 <= kCandPerThread && n1 <= kCandPerThread) {
-        // few keys left: the exact cut from the candidates sorted by (key desc, j asc)
-        unsigned long long c[2 * kCandPerThread];
-        int n = 0;
-        for (int i = 0; i < n0; ++i) c[n++] = S.cand[i][tid];
-        for (int i = 0; i < n1; ++i) c[n++] = S.cand[i][tid + kRows];
-        for (int i = 1; i < n; ++i) {
-          const unsigned long long v = c[i];
-          int k = i - 1;
-          while (k >= 0 && c[k] < v) {
-            c[k + 1] = c[k];
-            --k;
+    if (owner) {
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        if (!mine[sl]) continue;
+        RowS& W = S.row[sl ? x.rb : x.ra];
+        const int n0 = S.nc[sl][tid], n1 = S.nc[sl][tid + 1], n2 = S.nc[sl][tid + 2], n3 = S.nc[sl][tid + 3];
+        if (n0 <= kCand && n1 <= kCand && n2 <= kCand && n3 <= kCand) {
+          // every key of the range is a captured candidate: exact cut by sorting them
+          unsigned long long c[4 * kCand];
+          int n = 0;
+          const int nq[4] = {n0, n1, n2, n3};
+          for (int q = 0; q < 4; ++q)
+            for (int i = 0; i < nq[q]; ++i) c[n++] = S.cand[i][sl][tid + q];
+          for (int i = 1; i < n; ++i) {  // insertion sort, descending: key desc, then j asc
+            const unsigned long long v = c[i];
+            int k = i - 1;
+            while (k >= 0 && c[k] < v) {
+              c[k + 1] = c[k];
+              --k;
+            }
+            c[k + 1] = v;
           }
-          c[k + 1] = v;
-        }
-        unsigned long long cum = 0;
-        int ci = -1;
-        for (int i = 0; i < n; ++i) {
-          cum += mass64(key_to_float((uint32_t)(c[i] >> 32)), m, scale);
-          if (cum >= W.rem) {
-            ci = i;
-            break;
+          unsigned long long cum = 0;
+          int ci = -1;
+          for (int i = 0; i < n; ++i) {
+            cum += mass64(key_to_float((uint32_t)(c[i] >> 32)), m[sl], scale);
+            if (cum >= W.rem) {
+              ci = i;
+              break;
+            }
           }
-        }
-        if (ci < 0) {  // cannot happen: the range was chosen to hold at least rem
-          atomicOr(a.err, kErrInternal);
-          W.t_key = 0xFFFFFFFFu;
-          W.tiecut = -1;
-        } else {
-          W.t_key = (uint32_t)(c[ci] >> 32);
-          W.tiecut = (int)(0xFFFFFFFFu - (uint32_t)c[ci]);
-        }
-        W.mode = kModeDone;
-      } else {
-        unsigned long long cum = 0;
-        int cs = -1;
-        for (int i = kBins - 1; i >= 0; --i) {  // highest sub-range first
-          const unsigned long long hs = S.u.hist[i][tid] + S.u.hist[i][tid + kRows];
-          if (cum + hs >= W.rem) {
-            cs = i;
-            break;
+          if (ci < 0) {  // not reached: the range was chosen to hold at least rem
+            atomicOr(a.err, kErrInternal);
+            W.t_key = 0xFFFFFFFFu;
+            W.tiecut = -1;
+          } else {
+            W.t_key = (uint32_t)(c[ci] >> 32);
+            W.tiecut = (int)(0xFFFFFFFFu - (uint32_t)c[ci]);
+            W.above += cum;
           }
-          cum += hs;
-        }
-        if (cs < 0) {
-          atomicOr(a.err, kErrInternal);
-          W.t_key = 0xFFFFFFFFu;
-          W.tiecut = -1;
           W.mode = kModeDone;
         } else {
-          const uint32_t nlo = klo + (uint32_t)(((unsigned long long)cs * span + kBins - 1) / kBins);
-          const uint32_t nhi = klo + (uint32_t)((((unsigned long long)(cs + 1)) * span + kBins - 1) / kBins) - 1u;
-          W.rem -= cum;
-          W.klo = nlo;
-          W.khi = nhi;
-          if (nlo == nhi) {  // one key value with more than 32 members: an exact tie group
-            W.t_key = nlo;
-            const unsigned long long e = mass64(key_to_float(nlo), m, scale);
-            W.n_need = e ? (W.rem + e - 1) / e : 1ull;
-            W.mode = kModeTie;
+          unsigned long long cum = 0;
+          int cs = -1;
+          for (int i = kBins - 1; i >= 0; --i) {  // highest slice first
+            const unsigned long long hs = hist_get(S, i, sl, tid) + hist_get(S, i, sl, tid + 1) +
+                                          hist_get(S, i, sl, tid + 2) + hist_get(S, i, sl, tid + 3);
+            if (cum + hs >= W.rem) {
+              cs = i;
+              break;
+            }
+            cum += hs;
+          }
+          if (cs < 0) {
+            atomicOr(a.err, kErrInternal);
+            W.t_key = 0xFFFFFFFFu;
+            W.tiecut = -1;
+            W.mode = kModeDone;
+          } else {
+            const uint32_t nlo = W.klo + ((uint32_t)cs << W.shift);
+            const uint32_t top = nlo + ((1u << W.shift) - 1u);
+            const uint32_t nhi = top < W.khi && top >= nlo ? top : W.khi;
+            W.rem -= cum;
+            W.above += cum;
+            W.klo = nlo;
+            W.khi = nhi;
+            W.shift = slice_shift(nlo, nhi);
+            if (nlo == nhi) {  // one key value with more than 16 members: an exact tie group
+              W.t_key = nlo;
+              const unsigned long long e = mass64(key_to_float(nlo), m[sl], scale);
+              W.n_need = e ? (W.rem + e - 1) / e : 1ull;
+              W.mode = kModeTie;
+            }
           }
         }
       }
     }
     __syncthreads();
   }
-  if (hf == 0 && active && S.row[r].mode == kModeKeys) {  // not reached: six levels split 32 bits
-    atomicOr(a.err, kErrInternal);
-    S.row[r].t_key = 0xFFFFFFFFu;
-    S.row[r].tiecut = -1;
-    S.row[r].mode = kModeDone;
+  if (owner) {
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      RowS& W = S.row[sl ? x.rb : x.ra];
+      if (W.mode == kModeKeys) {  // not reached: ten 16-way levels split 32 bits
+        atomicOr(a.err, kErrInternal);
+        W.t_key = 0xFFFFFFFFu;
+        W.tiecut = -1;
+        W.mode = kModeDone;
+      }
+    }
   }
-  __syncthreads();
 
-  // ---- exact ties: the cutoff is the position of the n_need-th tied key in ascending order
-  const int need = (hf == 0 && S.row[r].mode == kModeTie) ? 1 : 0;
-  if (!__syncthreads_or(need)) return;
-  const bool mine = active && S.row[r].mode == kModeTie;
-  const uint32_t tk = S.row[r].t_key;
-  const float m = S.row[r].m;
-  const int b1 = S.row[r].bin1;
-  const int64_t ntiles = (nkeys + kKeys - 1) / kKeys;
-  for (int64_t t = 0; t < ntiles; ++t) {
-    stage_ik(S, 0, ibase, t, nkeys);
-    cp_async_wait<0>();
-    __syncthreads();
-    uint32_t bits = 0;
-    if (mine) {
-      for (int k = 0; k < kHalf; ++k) {
-        const int64_t j = t * kKeys + hf * kHalf + k;
-        if (j > pos) break;
-        const float s = score16(qt, S.ik[0][hf * kHalf + k]);
-        if (bin1_of(s, m) == b1 && order_key(s) == tk) bits |= 1u << k;
+  // ---- exact ties: the cutoff is the n_need-th tied position in ascending order
+  {
+    const int need = S.row[x.ra].mode == kModeTie || S.row[x.rb].mode == kModeTie;
+    if (__syncthreads_or(need)) {
+      bool mine[2];
+      uint32_t tk[2];
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        const RowS& R = S.row[sl ? x.rb : x.ra];
+        mine[sl] = R.mode == kModeTie;
+        tk[sl] = R.t_key;
       }
-    }
-    S.mask[r][hf] = bits;
-    __syncthreads();
-    if (hf == 0 && mine) {
-      RowSel& W = S.row[r];
-      if (!W.found) {
-        const unsigned long long mk = ((unsigned long long)S.mask[r][1] << 32) | S.mask[r][0];
-        const int cnt = __popcll(mk);
-        if (W.tie_before + cnt >= W.n_need) {
-          int want = (int)(W.n_need - W.tie_before);
-          unsigned long long x = mk;
-          while (--want > 0) x &= x - 1;  // drop the lowest (want - 1) set bits
-          W.tiecut = (int)(t * kKeys + (__ffsll((long long)x) - 1));
-          W.found = 1;
+      idx_walk(S.st, ibase, x.nkeys, [&](int64_t t, int stage) {
+        float c[8][4];
+        idx_scores(c, qh, ql, S.st, stage);
+        unsigned long long mk[2] = {0ull, 0ull};
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int p = 8 * nt + 2 * x.tq + e;
+            const int64_t j = t * kIdxKeys + p;
+#pragma unroll
+            for (int sl = 0; sl < 2; ++sl) {
+              const float s = c[nt][2 * sl + e];
+              if (mine[sl] && j <= (sl ? x.pb : x.pa) && order_key(s) == tk[sl])
+                mk[sl] |= 1ull << p;
+            }
+          }
         }
-        W.tie_before += cnt;
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 1);
+          mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 2);
+        }
+        if (owner) {
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            if (!mine[sl]) continue;
+            RowS& W = S.row[sl ? x.rb : x.ra];
+            if (W.found) continue;
+            const int cnt = __popcll(mk[sl]);
+            if (W.tie_before + cnt >= W.n_need) {
+              int want = (int)(W.n_need - W.tie_before);
+              unsigned long long v = mk[sl];
+              while (--want > 0) v &= v - 1;  // drop the lowest (want - 1) set bits
+              W.tiecut = (int)(t * kIdxKeys + (__ffsll((long long)v) - 1));
+              W.found = 1;
+            }
+            W.tie_before += cnt;
+          }
+        }
+      });
+      if (owner) {
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          if (!mine[sl]) continue;
+          RowS& W = S.row[sl ? x.rb : x.ra];
+          if (!W.found) {
+            atomicOr(a.err, kErrInternal);
+            W.tiecut = 0x7FFFFFFF;
+          } else {
+            W.above += (unsigned long long)W.n_need * mass64(key_to_float(W.t_key), m[sl], scale);
+          }
+          W.mode = kModeDone;
+        }
       }
     }
-    __syncthreads();
   }
-  if (hf == 0 && mine) {
-    if (!S.row[r].found) {
-      atomicOr(a.err, kErrInternal);
-      S.row[r].tiecut = 0x7FFFFFFF;
+
+  if (owner) {
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      const int r = sl ? x.rb : x.ra;
+      if ((sl ? x.pb : x.pa) < 0) continue;
+      const RowS& W = S.row[r];
+      cut[r] = make_uint2(W.t_key, (uint32_t)W.tiecut);
+      if (a.sel_mass)
+        a.sel_mass[((int64_t)b * a.C + i0 + r) * a.Hr + hr] = (float)((double)W.above / (double)W.Z);
     }
-    S.row[r].mode = kModeDone;
   }
-  __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads) prefill_retrieval_kernel(RetArgs a) {
+// ------------------------------------------------------------------ sparse attention
+
+struct SmemAttn {
+  IdxRing st;                           // 12 KB
+  unsigned char kv[2 * kFaTileBytes];   // 32 KB: gathered K and V rows of one chunk
+  uint32_t cm[kRows][4];                // per-row bits of the (up to 128) chunk slots
+  int32_t jl[128];                      // chunk slot -> key position
+  unsigned long long wun[4];            // per-warp union of the tile's row masks
+};
+
+__global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  SmemR& S = *reinterpret_cast<SmemR*>(smem_raw);
-  const int tile = blockIdx.x, hr = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, r = tid & (kRows - 1), hf = tid >> 6, warp = tid >> 5;
-  const int h = a.ret_head[hr], g = h / a.group;
+  SmemAttn& S = *reinterpret_cast<SmemAttn*>(smem_raw);
+  const int tile = gridDim.x - 1 - blockIdx.x, hr = blockIdx.y, b = blockIdx.z;  // longest rows first
   const int i0 = tile * kRows;
   const int nrows = min(kRows, a.C - i0);
-  const bool active = r < nrows;
-  const int64_t pos = a.P0 + i0 + r;                 // this thread's row position
-  const int64_t pos_max = a.P0 + i0 + nrows - 1;
-  const int64_t nkeys = pos_max + 1;
-  const float scale = __uint_as_float((uint32_t)(127 + a.sc_bits) << 23);
-  const float* ibase = a.idx + ((int64_t)b * a.Hr + hr) * a.max_seq * kR;
-
-  float qt[kR];
-  {
-    const float* qp = a.q_idx + (((int64_t)b * a.C + (active ? i0 + r : i0)) * a.Hr + hr) * kR;
-#pragma unroll
-    for (int c = 0; c < kR; ++c) qt[c] = qp[c];
-  }
-
-  if (a.top_p < 1.f) {
-    select_rows(S, a, ibase, qt, pos, nkeys, active, scale);
-  } else {  // p = 1 keeps every causal key (also those whose mass rounds to 0)
-    if (hf == 0) {
-      S.row[r].t_key = 0u;
-      S.row[r].tiecut = 0x7FFFFFFF;
-    }
-    __syncthreads();
-  }
-
-  // ---- attention over the selected keys of each row
+  const RowCtx x = row_ctx(a, i0, nrows);
+  const int tid = x.tid;
+  const bool owner = x.tq == 0;
+  const int h = a.ret_head[hr], g = h / a.group;
+  const __half* ibase = a.idx + ((int64_t)b * a.Hr + hr) * a.max_seq * (2 * kR);
   const __half* kb = a.kc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
   const __half* vb = a.vc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
   const int64_t qs = (int64_t)a.Hq * kD;
+
+  uint32_t qh[4], ql[4];
+  {
+    const int64_t is = (int64_t)a.Hr * kR;
+    const float* q0 = a.q_idx + ((int64_t)b * a.C + i0) * is + (int64_t)hr * kR;
+    idx_load_q(qh, ql, x.pa >= 0 ? q0 + x.ra * is : nullptr, x.pb >= 0 ? q0 + x.rb * is : nullptr);
+  }
+  const uint2* cut = a.cut + ((int64_t)b * a.Hr + hr) * a.C + i0;
+  uint32_t tk[2];
+  int64_t tc[2];
+  {
+    const uint2 ca = x.pa >= 0 ? cut[x.ra] : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+    const uint2 cbv = x.pb >= 0 ? cut[x.rb] : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+    tk[0] = ca.x;
+    tc[0] = (int32_t)ca.y;
+    tk[1] = cbv.x;
+    tc[1] = (int32_t)cbv.y;
+  }
+  uint32_t* brow[2] = {nullptr, nullptr};
+  if (a.bitmap && owner) {
+    if (x.pa >= 0) brow[0] = a.bitmap + (((int64_t)b * a.C + i0 + x.ra) * a.Hr + hr) * a.bitmap_words;
+    if (x.pb >= 0) brow[1] = a.bitmap + (((int64_t)b * a.C + i0 + x.rb) * a.Hr + hr) * a.bitmap_words;
+  }
+
   uint32_t qa[8][4];
-  fa_load_q(qa, a.q_rot + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD, qs, warp * 16, nrows);
+  fa_load_q(qa, a.q_rot + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD, qs, x.warp * 16, nrows);
   FaAcc A;
   fa_init(A);
-  const uint32_t tk = S.row[r].t_key;
-  const int tcut = S.row[r].tiecut;
-  const bool want_mass = a.sel_mass != nullptr && a.top_p < 1.f;
-  const float m = want_mass ? S.row[r].m : 0.f;
-  uint32_t* brow = (a.bitmap && active) ? a.bitmap + (((int64_t)b * a.C + i0 + r) * a.Hr + hr) * a.bitmap_words
-                                        : nullptr;
-  int nsel = 0;
-  unsigned long long msum = 0;
-  const int64_t ntiles = (nkeys + kKeys - 1) / kKeys;
-  for (int64_t t = 0; t < ntiles; ++t) {
-    stage_ik(S, 0, ibase, t, nkeys);
-    cp_async_wait<0>();
-    __syncthreads();
-    uint32_t bits = 0;
-    if (active) {
-      for (int k = 0; k < kHalf; ++k) {
-        const int64_t j = t * kKeys + hf * kHalf + k;
-        if (j > pos) break;
-        const float s = score16(qt, S.ik[0][hf * kHalf + k]);
-        const uint32_t key = order_key(s);
-        if (key > tk || (key == tk && j <= tcut)) {
-          bits |= 1u << k;
-          if (want_mass) msum += mass64(s, m, scale);
-        }
-      }
-      const int64_t w = 2 * t + hf;
-      if (brow && w < a.bitmap_words) brow[w] = bits;
-    }
-    S.mask[r][hf] = bits;
-    nsel += __popc(bits);
-    if (!__syncthreads_or(bits != 0u)) continue;  // no row selects a key of this tile
-    fa_stage(S.u.kv, S.u.kv + kFaTileBytes, kb, vb, (int)min((int64_t)kKeys, nkeys - t * kKeys),
-             [&](int rr) { return t * kKeys + rr; });
+
+  for (int i = tid; i < kRows * 4; i += kThreads) (&S.cm[0][0])[i] = 0u;
+  int fill = 0;
+  int nsel[2] = {0, 0};
+
+  auto flush = [&](int n) {
+    fa_stage(S.kv, S.kv + kFaTileBytes, kb, vb, n, [&](int r) { return (int64_t)S.jl[r]; });
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
-    fa_tile(A, qa, S.u.kv, S.u.kv + kFaTileBytes, a.scale_log2,
-            [&](int rr, int tt) { return ((S.mask[rr][tt >> 5] >> (tt & 31)) & 1u) != 0u; });
+    fa_tile(A, qa, S.kv, S.kv + kFaTileBytes, a.scale_log2,
+            [&](int r, int tt) { return ((S.cm[r][tt >> 5] >> (tt & 31)) & 1u) != 0u; });
     __syncthreads();
-  }
-  fa_store(A, a.out + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD, qs, warp * 16, nrows);
-  if (a.sel_count || a.sel_mass) {
-    S.ncand[tid] = nsel;
-    S.coarse[tid] = msum;
-    __syncthreads();
-    if (hf == 0 && active) {
-      const int64_t o = ((int64_t)b * a.C + i0 + r) * a.Hr + hr;
-      if (a.sel_count) a.sel_count[o] = S.ncand[tid] + S.ncand[tid + kRows];
-      if (a.sel_mass)
-        a.sel_mass[o] = a.top_p < 1.f ? (float)((double)(S.coarse[tid] + S.coarse[tid + kRows]) / (double)S.row[r].Z)
-                                      : 1.f;
+    // slots 64 .. 127 move down to 0 .. 63
+    for (int i = tid; i < kRows; i += kThreads) {
+      S.cm[i][0] = S.cm[i][2];
+      S.cm[i][1] = S.cm[i][3];
+      S.cm[i][2] = S.cm[i][3] = 0u;
     }
+    if (tid < 64) S.jl[tid] = S.jl[64 + tid];
+    __syncthreads();
+  };
+
+  idx_walk(S.st, ibase, x.nkeys, [&](int64_t t, int stage) {
+    float c[8][4];
+    idx_scores(c, qh, ql, S.st, stage);
+    unsigned long long mk[2] = {0ull, 0ull};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int p = 8 * nt + 2 * x.tq + e;
+        const int64_t j = t * kIdxKeys + p;
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          const uint32_t key = order_key(c[nt][2 * sl + e]);
+          const bool sel = j <= (sl ? x.pb : x.pa) && (key > tk[sl] || (key == tk[sl] && j <= tc[sl]));
+          if (sel) mk[sl] |= 1ull << p;
+        }
+      }
+    }
+    // this thread's selected keys, before the quad's masks are combined
+    const unsigned long long own0 = mk[0], own1 = mk[1];
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 1);
+      mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 2);
+    }
+    if (owner) {
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        nsel[sl] += __popcll(mk[sl]);
+        if (brow[sl]) {
+          const int64_t w = 2 * t;
+          if (w < a.bitmap_words) brow[sl][w] = (uint32_t)mk[sl];
+          if (w + 1 < a.bitmap_words) brow[sl][w + 1] = (uint32_t)(mk[sl] >> 32);
+        }
+      }
+    }
+    unsigned long long u = mk[0] | mk[1];
+    u |= __shfl_xor_sync(0xffffffffu, u, 4);
+    u |= __shfl_xor_sync(0xffffffffu, u, 8);
+    u |= __shfl_xor_sync(0xffffffffu, u, 16);
+    if ((tid & 31) == 0) S.wun[x.warp] = u;
+    __syncthreads();
+    const unsigned long long U = S.wun[0] | S.wun[1] | S.wun[2] | S.wun[3];
+    if (U == 0ull) return;  // uniform: no row selects a key of this tile
+    // append the tile's union keys to the chunk: slot = fill + rank of the key in U
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      unsigned long long v = sl ? own1 : own0;
+      const int r = sl ? x.rb : x.ra;
+      while (v) {
+        const int p = __ffsll((long long)v) - 1;
+        v &= v - 1;
+        const int slot = fill + __popcll(U & ((1ull << p) - 1ull));
+        atomicOr(&S.cm[r][slot >> 5], 1u << (slot & 31));
+      }
+    }
+    if (tid < 64 && ((U >> tid) & 1ull))
+      S.jl[fill + __popcll(U & ((1ull << tid) - 1ull))] = (int32_t)(t * kIdxKeys + tid);
+    fill += __popcll(U);
+    __syncthreads();
+    if (fill >= 64) {
+      flush(64);
+      fill -= 64;
+    }
+  });
+  if (fill > 0) flush(fill);
+  fa_store(A, a.out + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD, qs, x.warp * 16, nrows);
+  if (a.sel_count && owner) {
+    if (x.pa >= 0) a.sel_count[((int64_t)b * a.C + i0 + x.ra) * a.Hr + hr] = nsel[0];
+    if (x.pb >= 0) a.sel_count[((int64_t)b * a.C + i0 + x.rb) * a.Hr + hr] = nsel[1];
   }
 }
 
 }  // namespace
 
-cudaError_t launch_prefill_retrieval(const rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,
+cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,
                                      cudaStream_t st) {
   RetArgs a;
-  a.idx = L->idx;
+  a.idx = L->idx_hl;
   a.kc = L->kc;
   a.vc = L->vc;
   a.max_seq = L->max_seq;
@@ -494,6 +745,7 @@ cudaError_t launch_prefill_retrieval(const rtp_layer* L, int C, float* out, cons
   a.ret_head = L->d_ret_head;
   a.q_rot = L->q_rot;
   a.q_idx = L->q_idx;
+  a.cut = L->pf_cut;
   a.scale_log2 = L->sm_scale * 1.4426950408889634f;
   a.out = out;
   a.sel_count = stats ? stats->sel_count : nullptr;
@@ -501,12 +753,26 @@ cudaError_t launch_prefill_retrieval(const rtp_layer* L, int C, float* out, cons
   a.bitmap = stats ? stats->sel_bitmap : nullptr;
   a.bitmap_words = stats ? stats->bitmap_words : 0;
   a.err = L->err;
-  const size_t smem = sizeof(SmemR);
-  cudaError_t e = cudaFuncSetAttribute(prefill_retrieval_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   dim3 grid((C + kRows - 1) / kRows, L->Hr, L->B);
-  prefill_retrieval_kernel<<<grid, kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  cudaError_t e;
+  {
+    ProfScope ps(L, "prefill_select", st);
+    e = cudaFuncSetAttribute(prefill_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(SmemSel));
+    if (e != cudaSuccess) return e;
+    prefill_select_kernel<<<grid, kThreads, sizeof(SmemSel), st>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  {
+    ProfScope ps(L, "prefill_attn", st);
+    e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(SmemAttn));
+    if (e != cudaSuccess) return e;
+    prefill_attn_kernel<<<grid, kThreads, sizeof(SmemAttn), st>>>(a);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace rtp

@@ -56,6 +56,8 @@ struct rtp_layer {
   int16_t* d_loc_head = nullptr;   // [Hkv][kMaxGroup] local q heads of each KV head (-1 pad)
   int32_t* d_loc_cnt = nullptr;    // [Hkv]
   int16_t* d_local_list = nullptr; // [n_local] local q heads, ascending
+  __half* idx_hl = nullptr;        // [B][Hr][max_seq][2 r]: index keys split as fp16 hi | lo
+  uint2* pf_cut = nullptr;         // [B][Hr][max_chunk] prefill per-row cut (t_key, tiecut)
   int n_local = 0;
 
   // decode scratch
@@ -117,7 +119,7 @@ cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st);
 cudaError_t launch_iota_rows(int32_t* dst, int64_t cap, int rows, int64_t n, cudaStream_t st);
 cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st);
 cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStream_t st);
-cudaError_t launch_prefill_retrieval(const rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,
+cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,
                                      cudaStream_t st);
 
 // Selection kernel geometry for the current length (host-side; also sizes scratch).

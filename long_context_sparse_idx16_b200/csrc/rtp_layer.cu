@@ -92,7 +92,7 @@ static void prof_release(rtp_layer* L) {
 static void free_all(rtp_layer* L) {
   prof_release(L);
   void* ptrs[] = {L->kc, L->vc, L->idx, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
-                  L->d_loc_head, L->d_loc_cnt, L->d_local_list, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
+                  L->d_loc_head, L->d_loc_cnt, L->d_local_list, L->pf_cut, L->idx_hl, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
                   L->sticket, L->err};
@@ -201,6 +201,8 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   RTP_ALLOC(L->d_loc_head, Hkv * kMaxGroup);
   RTP_ALLOC(L->d_loc_cnt, Hkv);
   RTP_ALLOC(L->d_local_list, L->n_local);
+  RTP_ALLOC(L->idx_hl, (int64_t)B * Hr * L->max_seq * 2 * kR);
+  RTP_ALLOC(L->pf_cut, (int64_t)B * (Hr > 0 ? Hr : 1) * L->max_chunk);
   RTP_ALLOC(L->q_rot, rows * Hq * kD);
   RTP_ALLOC(L->q_idx, rows * Hr * kR);
   RTP_ALLOC(L->sel_idx, P * L->max_select);
@@ -359,8 +361,7 @@ rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out,
   }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: q_prep");
   if (L->Hr > 0) {
-    ProfScope ps(L, "prefill_retrieval", stream);
-    e = launch_prefill_retrieval(L, C, out, stats, stream);
+    e = launch_prefill_retrieval(L, C, out, stats, stream);  // profiled as prefill_select + prefill_attn
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: retrieval heads");
   }
   if (L->n_local > 0) {
