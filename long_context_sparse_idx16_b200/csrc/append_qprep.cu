@@ -57,21 +57,30 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
     bad |= !(fabsf(x) <= kFp16Max);
     vc[(((int64_t)b * Hkv + g) * max_seq + pos) * kD + d] = __float2half_rn(x);
   }
-  // index keys: Hr x r outputs, each a 128-term fp32 dot product in a fixed order
-  for (int o = threadIdx.x; o < Hr * kR; o += blockDim.x) {
-    const int hr = o / kR, c = o % kR;
+  // index keys: Hr x r outputs, each a 128-term fp32 dot product in a fixed order: 8 lanes
+  // of a warp take 16 dims each, then a fixed butterfly sums the 8 partials
+  const int lane = threadIdx.x & 31;
+  for (int o0 = (threadIdx.x >> 5) * 4; o0 < Hr * kR; o0 += (blockDim.x >> 5) * 4) {
+    const int o = o0 + (lane >> 3), part = lane & 7;
+    const bool live = o < Hr * kR;
+    const int hr = live ? o / kR : 0, c = o % kR;
     const int g = ret_head[hr] / group;
     const float* w = wk + (int64_t)hr * kD * kR + c;
     const float* x = ks + g * kD;
     float acc = 0.f;
-#pragma unroll 8
-    for (int d = 0; d < kD; ++d) acc = fmaf(w[d * kR], x[d], acc);
-    const int64_t row = ((int64_t)b * Hr + hr) * max_seq + pos;
-    idx[row * kR + c] = acc;
-    // the same key split as fp16 hi + lo, for the tensor-core scoring of prefill
-    const __half h = __float2half_rn(acc);
-    idx_hl[row * (2 * kR) + c] = h;
-    idx_hl[row * (2 * kR) + kR + c] = __float2half_rn(acc - __half2float(h));
+#pragma unroll
+    for (int d = part * 16; d < part * 16 + 16; ++d) acc = fmaf(w[d * kR], x[d], acc);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (live && part == 0) {
+      const int64_t row = ((int64_t)b * Hr + hr) * max_seq + pos;
+      idx[row * kR + c] = acc;
+      // the same key split as fp16 hi + lo, for the tensor-core scoring of prefill
+      const __half h = __float2half_rn(acc);
+      idx_hl[row * (2 * kR) + c] = h;
+      idx_hl[row * (2 * kR) + kR + c] = __float2half_rn(acc - __half2float(h));
+    }
   }
   if (bad) atomicOr(err, kErrRange);
 }

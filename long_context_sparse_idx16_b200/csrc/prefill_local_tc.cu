@@ -1,0 +1,334 @@
+// prefill_local_tc.cu -- local heads in chunked prefill on 5th-generation tensor cores.
+//
+// Local heads attend only to nearby tokens and a few attention sinks (techwalker page, section
+// 2; section 8: window 8192 with 4 sinks).  Query row i of the chunk sits at position
+// pos = len - C + i and sees keys j <= pos with pos - j < W or j < S.
+//
+// One CTA per (128-row tile, local head, sequence), 128 threads; thread r owns query row r
+// and TMEM lane r.  The tile's keys -- the sinks, then the union of its rows' windows -- are
+// taken in 64-key steps t, software-pipelined so the tensor cores, the copies and the softmax
+// overlap:
+//   * K/V rows go through a ring of four 128-byte-swizzled stages (cp.async), steps t + 1 ..
+//     t + 3 loading while step t computes;
+//   * S_t = Q K_t^T (tcgen05.mma, M 128, N 64, K 16 per instruction, Q and K from shared
+//     memory) lands in one of two TMEM buffers; S_{t+1} is issued before the softmax of S_t;
+//   * each thread reads its row of S_t from TMEM, applies the window mask and forms
+//     P = exp2(S - m) in fp16 (two P buffers) against a reference max m that only moves when
+//     the row max exceeds it by more than 8 (in log2 units): then the running sum and the
+//     output accumulator in TMEM are rescaled (this bounds P by 2^8);
+//   * O += P_t V_t (tcgen05.mma, M 128, N 128, V read as an MN-major operand) accumulates in
+//     TMEM across all steps and is read once at the end.
+// Completions are tracked with mbarriers (tcgen05.commit); every wait is bounded, and on
+// timeout the error word is set and the CTA leaves after freeing its TMEM.
+#include "rtp_internal.h"
+#include "tc_umma.cuh"
+
+namespace rtp {
+
+namespace {
+
+constexpr int kRowsT = 128;   // query rows per CTA (= TMEM lanes)
+constexpr int kKeysT = 64;    // keys per step
+constexpr int kThreadsT = 128;
+constexpr int kRing = 4;      // K/V stages: step t computes while t + 1 .. t + 3 load
+constexpr uint32_t kTmemCols = 256;  // S0 [0,64), S1 [64,128), O [128,256)
+constexpr float kRescale = 8.f;      // log2 headroom before the reference max moves
+constexpr uint32_t kQBytes = kRowsT * 256;   // 32 KB
+constexpr uint32_t kKVBytes = kKeysT * 256;  // 16 KB per K or V tile
+constexpr uint32_t kPBytes = kRowsT * 128;   // 16 KB
+// layout: Q | (K, V) x kRing | P x 2 | mbarriers (S0, S1, O0, O1), TMEM base
+constexpr uint32_t kOffRing = kQBytes;
+constexpr uint32_t kStageBytes = 2 * kKVBytes;
+constexpr uint32_t kOffP = kOffRing + kRing * kStageBytes;
+constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
+constexpr uint32_t kSmemT = kOffBar + 64;
+
+__device__ __forceinline__ uint32_t pack_half2_tc(float x, float y) {
+  __half2 h = __floats2half2_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+struct LocalTcArgs {
+  const __half* kc;
+  const __half* vc;
+  int64_t max_seq;
+  int Hkv, Hq, group, C;
+  int64_t P0;
+  int W, S;
+  const int16_t* local_heads;
+  const float* q_rot;  // [B][C][Hq][D]
+  float scale_log2;
+  float* out;          // [B][C][Hq][D]
+  uint32_t* err;
+};
+
+__global__ void __launch_bounds__(kThreadsT, 1) prefill_local_tc_kernel(LocalTcArgs a) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t barS0 = sbase + kOffBar, barO0 = barS0 + 16;  // barS[i] = barS0 + 8i, barO likewise
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + 32);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tile = blockIdx.x, b = blockIdx.z;
+  const int h = a.local_heads[blockIdx.y], g = h / a.group;
+  const int i0 = tile * kRowsT;
+  const int nrows = min(kRowsT, a.C - i0);
+  const int64_t pos_min = a.P0 + i0, pos_max = pos_min + nrows - 1;
+  const int64_t s_cnt = min((int64_t)a.S, pos_max + 1);
+  int64_t w_lo = pos_min - a.W + 1;
+  if (w_lo < s_cnt) w_lo = s_cnt;
+  const int64_t n_keys = s_cnt + (pos_max - w_lo + 1);
+  auto pos_of = [&](int64_t u) -> int64_t { return u < s_cnt ? u : w_lo + (u - s_cnt); };
+  const __half* kb = a.kc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
+  const __half* vb = a.vc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
+  const int64_t qs = (int64_t)a.Hq * kD;
+  const int r = tid;
+  const bool live = r < nrows;
+  const int64_t pos = pos_min + r;
+
+  // the swizzle is a function of address bits: the tiles must sit on 1024-byte boundaries
+  if (sbase & 1023u) {
+    if (tid == 0) atomicOr(a.err, kErrInternal);
+    return;
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(barS0 + 8 * i, 1);
+  }
+
+  // query row r as fp16 into the swizzled Q tile (zero rows past the chunk)
+  {
+    const float* qrow = a.q_rot + ((int64_t)b * a.C + i0 + (live ? r : 0)) * qs + (int64_t)h * kD;
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (live) {
+        const float4 x0 = *reinterpret_cast<const float4*>(qrow + 8 * c);
+        const float4 x1 = *reinterpret_cast<const float4*>(qrow + 8 * c + 4);
+        v.x = pack_half2_tc(x0.x, x0.y);
+        v.y = pack_half2_tc(x0.z, x0.w);
+        v.z = pack_half2_tc(x1.x, x1.y);
+        v.w = pack_half2_tc(x1.z, x1.w);
+      }
+      *reinterpret_cast<uint4*>(sm + sw128_off(r, c, kRowsT)) = v;
+    }
+  }
+
+  const int n_steps = (int)((n_keys + kKeysT - 1) / kKeysT);
+  auto stage = [&](int t) {  // K and V rows of step t into ring slot t % kRing; always commits
+    if (t < n_steps) {
+      const int64_t u0 = (int64_t)t * kKeysT;
+      unsigned char* ks = sm + kOffRing + (t % kRing) * kStageBytes;
+      unsigned char* vs = ks + kKVBytes;
+#pragma unroll
+      for (int i = 0; i < (kKeysT * 16) / kThreadsT; ++i) {
+        const int idx = i * kThreadsT + tid;
+        const int key = idx >> 4, c = idx & 15;
+        const int64_t u = u0 + key;
+        const bool ok = u < n_keys;
+        const int64_t p = ok ? pos_of(u) : 0;
+        cp_async16(ks + sw128_off(key, c, kKeysT), kb + p * kD + c * 8, ok ? 16 : 0);
+        cp_async16(vs + sw128_off(key, c, kKeysT), vb + p * kD + c * 8, ok ? 16 : 0);
+      }
+    }
+    cp_async_commit();
+  };
+  constexpr uint32_t kIdS = umma_idesc_f16(kKeysT, false);
+  constexpr uint32_t kIdO = umma_idesc_f16(kD, true);
+  auto issue_s = [&](uint32_t tmem, int t) {  // S_t = Q K_t^T into TMEM buffer t & 1 (one thread)
+    tc_fence_after();
+    const uint32_t k0 = sbase + kOffRing + (t % kRing) * kStageBytes;
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {
+      const uint64_t ad = umma_desc(sbase + (kk >> 2) * (kRowsT * 128) + (kk & 3) * 32, 16, 1024);
+      const uint64_t bd = umma_desc(k0 + (kk >> 2) * (kKeysT * 128) + (kk & 3) * 32, 16, 1024);
+      umma_f16(tmem + (uint32_t)((t & 1) * kKeysT), ad, bd, kIdS, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(barS0 + 8 * (t & 1));
+  };
+
+  stage(0);
+  stage(1);
+  stage(2);
+  cp_async_wait<2>();  // step 0 landed
+  fence_async_smem();
+  __syncthreads();  // Q and step 0 in shared memory, mbarriers initialised, TMEM base written
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  if (tid == 0) issue_s(tmem, 0);
+
+  float m_ref = -INFINITY, l = 0.f;
+  bool ok = true;
+  for (int t = 0; t < n_steps; ++t) {
+    // ---- K_{t+1} landed -> issue S_{t+1} (its buffer was last read by the softmax of t - 1)
+    if (t + 1 < n_steps) {
+      cp_async_wait<1>();  // everything but step t + 2
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) issue_s(tmem, t + 1);
+    }
+    // ---- softmax of S_t
+    ok = __syncthreads_and(mbar_wait(barS0 + 8 * (t & 1), (uint32_t)(t >> 1) & 1u));
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t sAddr = tmem + lane_off + (uint32_t)((t & 1) * kKeysT);
+    const int64_t u0 = (int64_t)t * kKeysT;
+    bool full = false;  // every row of the CTA sees every key of the step
+    if (nrows == kRowsT && u0 + kKeysT <= n_keys) {
+      const int64_t j_lo = pos_of(u0), j_hi = pos_of(u0 + kKeysT - 1);
+      const bool one_seg = (u0 + kKeysT <= s_cnt) || (u0 >= s_cnt);
+      full = one_seg && j_hi <= pos_min && (j_hi < a.S || pos_max - j_lo < a.W);
+    }
+    auto score = [&](int c, float x) -> float {
+      x *= a.scale_log2;
+      if (full) return x;
+      const int64_t u = u0 + c;
+      if (!live || u >= n_keys) return -INFINITY;
+      const int64_t j = pos_of(u);
+      return (j <= pos && (j < a.S || pos - j < a.W)) ? x : -INFINITY;
+    };
+    float sv[kKeysT];
+    tmem_ld32(sAddr, sv);
+    tmem_ld32(sAddr + 32, sv + 32);
+    tmem_ld_wait();
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kKeysT; ++c) {
+      sv[c] = score(c, sv[c]);
+      mx = fmaxf(mx, sv[c]);
+    }
+    // the reference max moves only when this step's max exceeds it by more than kRescale
+    const bool move = mx > m_ref + kRescale;
+    if (__syncthreads_or(move && t > 0)) {
+      // rescale the output accumulator: every P V issued so far must have completed
+      ok = __syncthreads_and(mbar_wait(barO0 + 8 * ((t - 1) & 1), (uint32_t)((t - 1) >> 1) & 1u));
+      if (!ok) break;
+      tc_fence_after();
+      // tcgen05.ld / st are warp-collective: every thread runs them, rows that keep their
+      // reference max with factor 1
+      const float cf = move ? fast_exp2(m_ref - mx) : 1.f;
+      const uint32_t oAddr = tmem + lane_off + 128u;
+#pragma unroll
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        float ov[32];
+        tmem_ld32(oAddr + c0, ov);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] *= cf;
+        tmem_st32(oAddr + c0, ov);
+      }
+      tmem_st_wait();
+    }
+    if (move) {
+      l *= fast_exp2(m_ref - mx);  // 0 while m_ref is still -inf
+      m_ref = mx;
+    }
+    // P_t into P buffer t & 1, last read by P V of step t - 2
+    if (t >= 2) {
+      ok = __syncthreads_and(mbar_wait(barO0 + 8 * (t & 1), (uint32_t)((t - 2) >> 1) & 1u));
+      if (!ok) break;
+    }
+    float rs = 0.f;
+    unsigned char* pbuf = sm + kOffP + (t & 1) * kPBytes;
+#pragma unroll
+    for (int q = 0; q < kKeysT / 8; ++q) {
+      float pv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        pv[e] = m_ref == -INFINITY ? 0.f : fast_exp2(sv[8 * q + e] - m_ref);
+        rs += pv[e];
+      }
+      uint4 w;
+      w.x = pack_half2_tc(pv[0], pv[1]);
+      w.y = pack_half2_tc(pv[2], pv[3]);
+      w.z = pack_half2_tc(pv[4], pv[5]);
+      w.w = pack_half2_tc(pv[6], pv[7]);
+      *reinterpret_cast<uint4*>(pbuf + sw128_off(r, q, kRowsT)) = w;
+    }
+    l += rs;
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- O += P_t V_t (one thread); V is read MN-major (rows = keys)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t v0 = sbase + kOffRing + (t % kRing) * kStageBytes + kKVBytes;
+      const uint32_t p0 = sbase + kOffP + (t & 1) * kPBytes;
+#pragma unroll
+      for (int kk = 0; kk < kKeysT / 16; ++kk) {
+        const uint64_t ad = umma_desc(p0 + kk * 32, 16, 1024);
+        const uint64_t bd = umma_desc(v0 + kk * 2048, kKeysT * 128, 1024);
+        umma_f16(tmem + 128u, ad, bd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(barO0 + 8 * (t & 1));
+    }
+    // ---- ring slot of step t + 3 held step t - 1, whose P V must be done before it is refilled
+    if (t >= 1) {
+      ok = __syncthreads_and(mbar_wait(barO0 + 8 * ((t - 1) & 1), (uint32_t)((t - 1) >> 1) & 1u));
+      if (!ok) break;
+    }
+    stage(t + 3);
+  }
+
+  if (ok && n_steps > 0) {
+    const int tl = n_steps - 1;
+    ok = __syncthreads_and(mbar_wait(barO0 + 8 * (tl & 1), (uint32_t)(tl >> 1) & 1u));
+  }
+  if (ok) {
+    tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float* orow = a.out + ((int64_t)b * a.C + i0 + (live ? r : 0)) * qs + (int64_t)h * kD;
+    const uint32_t oAddr = tmem + lane_off + 128u;
+#pragma unroll
+    for (int c0 = 0; c0 < kD; c0 += 32) {
+      float ov[32];
+      tmem_ld32(oAddr + c0, ov);
+      tmem_ld_wait();
+      if (live) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(orow + c0 + i) =
+              make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+      }
+    }
+  } else if (tid == 0) {
+    atomicOr(a.err, kErrTimeout);
+  }
+  cp_async_wait<0>();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_free(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStream_t st) {
+  LocalTcArgs a;
+  a.kc = L->kc;
+  a.vc = L->vc;
+  a.max_seq = L->max_seq;
+  a.Hkv = L->Hkv;
+  a.Hq = L->Hq;
+  a.group = L->group;
+  a.C = C;
+  a.P0 = L->len - C;
+  a.W = L->W;
+  a.S = L->S;
+  a.local_heads = L->d_local_list;
+  a.q_rot = L->q_rot;
+  a.scale_log2 = L->sm_scale * 1.4426950408889634f;
+  a.out = out;
+  a.err = L->err;
+  cudaError_t e = cudaFuncSetAttribute(prefill_local_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemT);
+  if (e != cudaSuccess) return e;
+  dim3 grid((C + kRowsT - 1) / kRowsT, L->n_local, L->B);
+  prefill_local_tc_kernel<<<grid, kThreadsT, kSmemT, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace rtp

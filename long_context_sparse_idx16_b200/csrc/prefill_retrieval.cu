@@ -578,11 +578,13 @@ __global__ void __launch_bounds__(kThreads) prefill_select_kernel(RetArgs a) {
 // ------------------------------------------------------------------ sparse attention
 
 struct SmemAttn {
-  IdxRing st;                           // 12 KB
-  unsigned char kv[2 * kFaTileBytes];   // 32 KB: gathered K and V rows of one chunk
-  uint32_t cm[kRows][4];                // per-row bits of the (up to 128) chunk slots
-  int32_t jl[128];                      // chunk slot -> key position
-  unsigned long long wun[4];            // per-warp union of the tile's row masks
+  IdxRing st;                             // 12 KB
+  unsigned char kv[2][2 * kFaTileBytes];  // 64 KB: gathered K and V rows of two chunks in flight
+  uint32_t cm[kRows][4];                  // per-row bits of the (up to 128) filling slots
+  int32_t jl[128];                        // filling slot -> key position
+  uint32_t cmc[2][kRows][2];              // per-row bits of the two issued chunks
+  int32_t jlc[2][64];                     // their key positions
+  unsigned long long wun[2][4];           // per-warp union of a tile's row masks (two tiles)
 };
 
 __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
@@ -632,44 +634,94 @@ __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
   int fill = 0;
   int nsel[2] = {0, 0};
 
-  auto flush = [&](int n) {
-    fa_stage(S.kv, S.kv + kFaTileBytes, kb, vb, n, [&](int r) { return (int64_t)S.jl[r]; });
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    fa_tile(A, qa, S.kv, S.kv + kFaTileBytes, a.scale_log2,
-            [&](int r, int tt) { return ((S.cm[r][tt >> 5] >> (tt & 31)) & 1u) != 0u; });
-    __syncthreads();
-    // slots 64 .. 127 move down to 0 .. 63
+  // Chunks are double-buffered: issuing chunk n starts its K/V gather, and only then is chunk
+  // n - 1 (gathered meanwhile) run through the attention tile.
+  int pend = -1;  // buffer of the issued chunk not yet attended (-1: none)
+  int nbuf = 0;   // buffer the next chunk goes to
+  auto attend = [&](int buf) {
+    fa_tile(A, qa, S.kv[buf], S.kv[buf] + kFaTileBytes, a.scale_log2,
+            [&](int r, int tt) { return ((S.cmc[buf][r][tt >> 5] >> (tt & 31)) & 1u) != 0u; });
+  };
+  auto issue = [&](int n) {  // move filling slots 0 .. n-1 into a chunk buffer and gather it
+    const int k = nbuf;
     for (int i = tid; i < kRows; i += kThreads) {
+      S.cmc[k][i][0] = S.cm[i][0];
+      S.cmc[k][i][1] = S.cm[i][1];
       S.cm[i][0] = S.cm[i][2];
       S.cm[i][1] = S.cm[i][3];
       S.cm[i][2] = S.cm[i][3] = 0u;
     }
-    if (tid < 64) S.jl[tid] = S.jl[64 + tid];
+    if (tid < 64) {
+      S.jlc[k][tid] = tid < n ? S.jl[tid] : 0;
+      S.jl[tid] = S.jl[64 + tid];
+    }
     __syncthreads();
+    fa_stage(S.kv[k], S.kv[k] + kFaTileBytes, kb, vb, n, [&](int r) { return (int64_t)S.jlc[k][r]; });
+    cp_async_commit();
+    if (pend >= 0) {
+      cp_async_wait<1>();  // everything but this chunk's gather has landed
+      __syncthreads();
+      attend(pend);
+      __syncthreads();
+    }
+    pend = k;
+    nbuf ^= 1;
+  };
+
+  // The union of tile t is published in shared memory and appended to the chunk during tile
+  // t + 1, after that tile's ring barrier: one barrier per tile.
+  unsigned long long own_prev[2] = {0ull, 0ull};
+  auto append = [&](int64_t t) {  // tile t's union keys -> chunk slots fill, fill + 1, ...
+    const int pb = (int)(t & 1);
+    const unsigned long long U = S.wun[pb][0] | S.wun[pb][1] | S.wun[pb][2] | S.wun[pb][3];
+    if (U == 0ull) return;  // uniform: no row selects a key of this tile
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      unsigned long long v = own_prev[sl];
+      const int r = sl ? x.rb : x.ra;
+      while (v) {
+        const int p = __ffsll((long long)v) - 1;
+        v &= v - 1;
+        const int slot = fill + __popcll(U & ((1ull << p) - 1ull));
+        atomicOr(&S.cm[r][slot >> 5], 1u << (slot & 31));
+      }
+    }
+    if (tid < 64 && ((U >> tid) & 1ull))
+      S.jl[fill + __popcll(U & ((1ull << tid) - 1ull))] = (int32_t)(t * kIdxKeys + tid);
+    fill += __popcll(U);
+    if (fill >= 64) {
+      __syncthreads();  // every slot of the chunk is written
+      issue(64);
+      fill -= 64;
+    }
   };
 
   idx_walk(S.st, ibase, x.nkeys, [&](int64_t t, int stage) {
+    if (t > 0) append(t - 1);
     float c[8][4];
     idx_scores(c, qh, ql, S.st, stage);
+    const int64_t base = t * kIdxKeys;
+    const int la = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pa - base));
+    const int lb = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pb - base));
+    const int ca = (int)max((int64_t)-1, min((int64_t)kIdxKeys, tc[0] - base));
+    const int cbt = (int)max((int64_t)-1, min((int64_t)kIdxKeys, tc[1] - base));
     unsigned long long mk[2] = {0ull, 0ull};
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int p = 8 * nt + 2 * x.tq + e;
-        const int64_t j = t * kIdxKeys + p;
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
           const uint32_t key = order_key(c[nt][2 * sl + e]);
-          const bool sel = j <= (sl ? x.pb : x.pa) && (key > tk[sl] || (key == tk[sl] && j <= tc[sl]));
-          if (sel) mk[sl] |= 1ull << p;
+          const int lim = sl ? lb : la, cut_p = sl ? cbt : ca;
+          const bool sel = p <= lim && (key > tk[sl] || (key == tk[sl] && p <= cut_p));
+          mk[sl] |= (unsigned long long)sel << p;
         }
       }
     }
-    // this thread's selected keys, before the quad's masks are combined
-    const unsigned long long own0 = mk[0], own1 = mk[1];
+    own_prev[0] = mk[0];  // this thread's selected keys, appended during the next tile
+    own_prev[1] = mk[1];
 #pragma unroll
     for (int sl = 0; sl < 2; ++sl) {
       mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 1);
@@ -690,32 +742,19 @@ __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
     u |= __shfl_xor_sync(0xffffffffu, u, 4);
     u |= __shfl_xor_sync(0xffffffffu, u, 8);
     u |= __shfl_xor_sync(0xffffffffu, u, 16);
-    if ((tid & 31) == 0) S.wun[x.warp] = u;
-    __syncthreads();
-    const unsigned long long U = S.wun[0] | S.wun[1] | S.wun[2] | S.wun[3];
-    if (U == 0ull) return;  // uniform: no row selects a key of this tile
-    // append the tile's union keys to the chunk: slot = fill + rank of the key in U
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      unsigned long long v = sl ? own1 : own0;
-      const int r = sl ? x.rb : x.ra;
-      while (v) {
-        const int p = __ffsll((long long)v) - 1;
-        v &= v - 1;
-        const int slot = fill + __popcll(U & ((1ull << p) - 1ull));
-        atomicOr(&S.cm[r][slot >> 5], 1u << (slot & 31));
-      }
-    }
-    if (tid < 64 && ((U >> tid) & 1ull))
-      S.jl[fill + __popcll(U & ((1ull << tid) - 1ull))] = (int32_t)(t * kIdxKeys + tid);
-    fill += __popcll(U);
-    __syncthreads();
-    if (fill >= 64) {
-      flush(64);
-      fill -= 64;
-    }
+    if ((tid & 31) == 0) S.wun[t & 1][x.warp] = u;
   });
-  if (fill > 0) flush(fill);
+  {
+    const int64_t ntiles = (x.nkeys + kIdxKeys - 1) / kIdxKeys;  // the walk ended with a barrier
+    append(ntiles - 1);
+  }
+  __syncthreads();
+  if (fill > 0) issue(fill);
+  if (pend >= 0) {
+    cp_async_wait<0>();
+    __syncthreads();
+    attend(pend);
+  }
   fa_store(A, a.out + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD, qs, x.warp * 16, nrows);
   if (a.sel_count && owner) {
     if (x.pa >= 0) a.sel_count[((int64_t)b * a.C + i0 + x.ra) * a.Hr + hr] = nsel[0];
