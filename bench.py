@@ -413,9 +413,16 @@ def run_gpu(args):
         step()
     torch.cuda.synchronize()
     sel_ms, sel_n = layer.profile_read("decode_select")
+    kern = {"decode_select": {"us_per_launch": sel_ms * 1e3 / max(sel_n, 1), "launches": sel_n}}
+    other_n = 0
+    for k in ("append_kv", "q_prep", "decode_gather", "decode_swa", "swa_merge", "dense_fill"):
+        kms, kn = layer.profile_read(k)
+        if kn:
+            kern[k] = {"us_per_launch": kms * 1e3 / kn, "launches": kn}
+        other_n += kn
     rest_ms, rest_n = layer.profile_read(None)
     layer.profile(False)
-    all_n = sel_n + rest_n
+    all_n = sel_n + other_n + rest_n
 
     # ---- end-to-end through the C ABI with host buffers
     q_h = torch.empty_like(q, device="cpu").pin_memory()
@@ -475,6 +482,7 @@ def run_gpu(args):
                           "frac": step_bytes / (peak * 1e9) / (ms / args.steps * 1e-3)},
         "e2e": {"value": e2e, "unit": "us/token", "h2d_bytes_per_step": int(q.numel() * 2 + k_tok.numel() * 2 * 2),
                 "d2h_bytes_per_step": int(out.numel() * 4)},
+        "kernels": kern,
         "gpu_launches": int(all_n),  # kernels of this library per timed region (one pass of --steps steps)
         "selected_tokens": {"min": int(counts.min()), "median": float(np.median(counts)), "max": int(counts.max())},
         "clocks": clk,
