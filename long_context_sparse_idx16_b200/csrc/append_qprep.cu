@@ -22,6 +22,9 @@ namespace {
 
 constexpr float kFp16Max = 65504.f;
 
+// Retrieval heads whose index weights are staged in shared memory at once (8 KB each).
+constexpr int kWHeads = 8;
+
 __global__ void __launch_bounds__(256) append_kv_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int T, int Hkv,
     int Hr, int64_t pos0, int64_t max_seq, const double* __restrict__ theta,
@@ -31,16 +34,28 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
   const int t = blockIdx.x;  // token within the appended block
   const int b = blockIdx.y;
   const int64_t pos = pos0 + t;
-  extern __shared__ float ks[];  // [Hkv][D] pre-RoPE key (fp32)
+  extern __shared__ float smem_f[];
+  float* ks = smem_f;                 // [Hkv][D] pre-RoPE key (fp32)
+  float* ws = smem_f + Hkv * kD;      // [<= kWHeads][D][r] index weights
   __shared__ float cs[kHalfD], sn[kHalfD];
 
   const __nv_bfloat16* kt = k + ((int64_t)b * T + t) * Hkv * kD;
   const __nv_bfloat16* vt = v + ((int64_t)b * T + t) * Hkv * kD;
+  // every global read of the token is issued before any is used: one memory round trip
+  const int nw = min(Hr, kWHeads);
+  for (int i = threadIdx.x; i < nw * kD * kR / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(ws)[i] = reinterpret_cast<const float4*>(wk)[i];
   for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) ks[i] = __bfloat162float(kt[i]);
   if (threadIdx.x < kHalfD) rope_cos_sin(pos, theta[threadIdx.x], &cs[threadIdx.x], &sn[threadIdx.x]);
+  bool bad = false;
+  for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) {
+    const int g = i / kD, d = i % kD;
+    const float x = __bfloat162float(vt[i]);
+    bad |= !(fabsf(x) <= kFp16Max);
+    vc[(((int64_t)b * Hkv + g) * max_seq + pos) * kD + d] = __float2half_rn(x);
+  }
   __syncthreads();
 
-  bool bad = false;
   for (int i = threadIdx.x; i < Hkv * kHalfD; i += blockDim.x) {
     const int g = i / kHalfD, c = i % kHalfD;
     const float x0 = ks[g * kD + c], x1 = ks[g * kD + c + kHalfD];
@@ -51,35 +66,28 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
     dst[c] = __float2half_rn(y0);
     dst[c + kHalfD] = __float2half_rn(y1);
   }
-  for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) {
-    const int g = i / kD, d = i % kD;
-    const float x = __bfloat162float(vt[i]);
-    bad |= !(fabsf(x) <= kFp16Max);
-    vc[(((int64_t)b * Hkv + g) * max_seq + pos) * kD + d] = __float2half_rn(x);
-  }
-  // index keys: Hr x r outputs, each a 128-term fp32 dot product in a fixed order: 8 lanes
-  // of a warp take 16 dims each, then a fixed butterfly sums the 8 partials
-  const int lane = threadIdx.x & 31;
-  for (int o0 = (threadIdx.x >> 5) * 4; o0 < Hr * kR; o0 += (blockDim.x >> 5) * 4) {
-    const int o = o0 + (lane >> 3), part = lane & 7;
-    const bool live = o < Hr * kR;
-    const int hr = live ? o / kR : 0, c = o % kR;
-    const int g = ret_head[hr] / group;
-    const float* w = wk + (int64_t)hr * kD * kR + c;
-    const float* x = ks + g * kD;
-    float acc = 0.f;
-#pragma unroll
-    for (int d = part * 16; d < part * 16 + 16; ++d) acc = fmaf(w[d * kR], x[d], acc);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-    if (live && part == 0) {
+  // index keys: Hr x r outputs, one thread each, a 128-term fp32 dot product in a fixed order
+  for (int h0 = 0; h0 < Hr; h0 += kWHeads) {
+    const int nh = min(Hr - h0, kWHeads);
+    if (h0 > 0) {  // later groups of heads (more than kWHeads retrieval heads)
+      __syncthreads();
+      for (int i = threadIdx.x; i < nh * kD * kR / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(ws)[i] = reinterpret_cast<const float4*>(wk + (int64_t)h0 * kD * kR)[i];
+      __syncthreads();
+    }
+    for (int o = threadIdx.x; o < nh * kR; o += blockDim.x) {
+      const int hl = o / kR, c = o % kR, hr = h0 + hl;
+      const float* w = ws + hl * kD * kR + c;
+      const float* x = ks + (ret_head[hr] / group) * kD;
+      float acc = 0.f;
+#pragma unroll 16
+      for (int d = 0; d < kD; ++d) acc = fmaf(w[d * kR], x[d], acc);
       const int64_t row = ((int64_t)b * Hr + hr) * max_seq + pos;
       idx[row * kR + c] = acc;
       // the same key split as fp16 hi + lo, for the tensor-core scoring of prefill
-      const __half h = __float2half_rn(acc);
-      idx_hl[row * (2 * kR) + c] = h;
-      idx_hl[row * (2 * kR) + kR + c] = __float2half_rn(acc - __half2float(h));
+      const __half hh = __float2half_rn(acc);
+      idx_hl[row * (2 * kR) + c] = hh;
+      idx_hl[row * (2 * kR) + kR + c] = __float2half_rn(acc - __half2float(hh));
     }
   }
   if (bad) atomicOr(err, kErrRange);
@@ -143,7 +151,10 @@ __global__ void __launch_bounds__(128) q_prep_kernel(
 cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T,
                              cudaStream_t st) {
   dim3 grid(T, L->B);
-  size_t smem = (size_t)L->Hkv * kD * sizeof(float);
+  const int nw = L->Hr < kWHeads ? L->Hr : kWHeads;
+  const size_t smem = ((size_t)L->Hkv * kD + (size_t)nw * kD * kR) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(append_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   append_kv_kernel<<<grid, 256, smem, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta,
                                             L->wk, L->d_ret_head, L->group, L->kc, L->vc, L->idx,
                                             L->idx_hl, L->err);
