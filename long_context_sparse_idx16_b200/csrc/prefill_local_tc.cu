@@ -227,13 +227,29 @@ __global__ void __launch_bounds__(kThreadsT, 2) prefill_local_tc_kernel(LocalTcA
       d_hi = cl((int64_t)a.S - 1 - base);
       e_lo = cl(pos - a.W + 1 - base);
     }
+    // a step whose keys every row of the CTA sees (one segment, last key at or before the
+    // first row, first key inside the last row's window) needs no mask
+    bool full = false;
+    if (nrows == kRowsT && u0 + kKeysT <= n_keys) {
+      const int64_t j_lo = pos_of(u0), j_hi = pos_of(u0 + kKeysT - 1);
+      const bool one_seg = (u0 + kKeysT <= s_cnt) || (u0 >= s_cnt);
+      full = one_seg && j_hi <= pos_min && (j_hi < a.S || pos_max - j_lo < a.W);
+    }
     float mx = -INFINITY;
+    if (full) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int c = 32 * half + i;
-      const bool vis = c <= s_hi || (c >= w_a && c <= w_b && (c <= d_hi || c >= e_lo));
-      sv[i] = vis ? sv[i] * a.scale_log2 : -INFINITY;
-      mx = fmaxf(mx, sv[i]);
+      for (int i = 0; i < 32; ++i) {
+        sv[i] *= a.scale_log2;
+        mx = fmaxf(mx, sv[i]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int c = 32 * half + i;
+        const bool vis = c <= s_hi || (c >= w_a && c <= w_b && (c <= d_hi || c >= e_lo));
+        sv[i] = vis ? sv[i] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sv[i]);
+      }
     }
     mx = fmaxf(mx, swap_half(sCol, mx));  // the row max over both halves
     // the reference max moves only when the row max exceeds it by more than kRescale
@@ -262,12 +278,14 @@ __global__ void __launch_bounds__(kThreadsT, 2) prefill_local_tc_kernel(LocalTcA
     // ---- P_t (this half's four 16-byte chunks)
     float rs = 0.f;
     unsigned char* pbuf = sm + kOffP;
+    // a row with no visible key yet has m_ref = -inf and only -inf scores: exp2(-inf - 0) = 0
+    const float mref = m_ref == -INFINITY ? 0.f : m_ref;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       float pv[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        pv[e] = m_ref == -INFINITY ? 0.f : fast_exp2(sv[8 * q + e] - m_ref);
+        pv[e] = fast_exp2(sv[8 * q + e] - mref);
         rs += pv[e];
       }
       uint4 w;
