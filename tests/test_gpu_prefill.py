@@ -102,3 +102,37 @@ def test_prefill_1m_full_sampled_rows():
     x = synth.generate(synth.spec("prefill_1m"))
     rows = [0, 5, 8191, 8192, 16383]
     run_prefill(x, rows=rows, heads=[0, 2, 13, 26], bitmap=False)
+
+
+def test_prefill_bitmap_needs_words():
+    # a bitmap pointer with no room is an argument error, caught before any launch
+    import torch
+
+    from long_context_sparse_idx16_b200 import Layer, RTPError, rtp_prefill_chunk, rtp_prefill_stats
+
+    x = small(prefix=100, chunk=64)
+    s = x.spec
+    layer = Layer.from_spec(s, x, max_seq=s.n_total, max_chunk=s.chunk)
+    build_cache(layer, x, s.n_total)
+    q = torch_bf16(x.q)
+    out = torch.empty((s.batch, s.chunk, s.n_q_heads, 128), dtype=torch.float32, device="cuda")
+    bm = torch.zeros(16, dtype=torch.int32, device="cuda")
+    st = rtp_prefill_stats(None, None, bm.data_ptr(), 0)
+    with pytest.raises(RTPError):
+        rtp_prefill_chunk(layer.handle, q.data_ptr(), s.chunk, out.data_ptr(), st, 0)
+    assert layer.check() == 0
+    layer.close()
+
+
+def test_prefill_chunk_larger_than_cache_is_rejected():
+    import torch
+
+    from long_context_sparse_idx16_b200 import Layer, RTPError
+
+    x = small(prefix=0, chunk=128)
+    s = x.spec
+    layer = Layer.from_spec(s, x, max_seq=s.n_total, max_chunk=s.chunk)
+    build_cache(layer, x, 64)  # only half the chunk's keys appended
+    with pytest.raises(RTPError):
+        layer.prefill_chunk(torch_bf16(x.q))
+    layer.close()
