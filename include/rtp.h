@@ -126,7 +126,8 @@ rtp_status rtp_append_kv(rtp_layer* layer, const void* k, const void* v, int32_t
 /* One decode step for every sequence: q is DEVICE bf16 [B][Hq][D] pre-RoPE at position
  * len-1 (append its own key first).  out is DEVICE fp32 [B][Hq][D].  Retrieval heads run
  * index scoring, exact top-p selection and sparse attention; local heads run window+sink
- * attention.  stats may be NULL. */
+ * attention, on an internal stream forked from `stream` (an event) after the selection and
+ * joined back (an event) before the call's work ends in `stream` order.  stats may be NULL. */
 rtp_status rtp_decode(rtp_layer* layer, const void* q, float* out, const rtp_decode_stats* stats,
                       cudaStream_t stream);
 

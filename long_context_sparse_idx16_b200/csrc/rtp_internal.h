@@ -57,7 +57,11 @@ struct rtp_layer {
   int32_t* d_loc_cnt = nullptr;    // [Hkv]
   int16_t* d_local_list = nullptr; // [n_local] local q heads, ascending
   __half* idx_hl = nullptr;        // [B][Hr][max_seq][2 r]: index keys split as fp16 hi | lo
-  uint2* pf_cut = nullptr;         // [B][Hr][max_chunk] prefill per-row cut (t_key, tiecut)
+  uint2* pf_cut = nullptr;
+  // decode: the local heads' window attention runs on a second stream, forked after the
+  // selection and joined back, so it overlaps the retrieval heads' gather attention
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;         // [B][Hr][max_chunk] prefill per-row cut (t_key, tiecut)
   int n_local = 0;
 
   // decode scratch

@@ -91,6 +91,11 @@ static void prof_release(rtp_layer* L) {
 
 static void free_all(rtp_layer* L) {
   prof_release(L);
+  if (L->ev_fork) cudaEventDestroy(L->ev_fork);
+  if (L->ev_join) cudaEventDestroy(L->ev_join);
+  if (L->side) cudaStreamDestroy(L->side);
+  L->ev_fork = L->ev_join = nullptr;
+  L->side = nullptr;
   void* ptrs[] = {L->kc, L->vc, L->idx, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
                   L->d_loc_head, L->d_loc_cnt, L->d_local_list, L->pf_cut, L->idx_hl, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
@@ -257,6 +262,9 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
     if (e == cudaSuccess && !local_list.empty())
       e = cudaMemcpy(L->d_local_list, local_list.data(), sizeof(int16_t) * local_list.size(), cudaMemcpyHostToDevice);
   }
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_join, cudaEventDisableTiming);
   if (e == cudaSuccess) e = reset_select_scratch(L);
   if (e == cudaSuccess) e = cudaMemset(L->gticket, 0, sizeof(uint32_t) * (P > 0 ? P : 1));
   if (e == cudaSuccess) e = cudaMemset(L->err, 0, sizeof(uint32_t));
@@ -305,6 +313,7 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
     e = launch_q_prep(L, (const __nv_bfloat16*)q, 1, L->len - 1, stream);
   }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: q_prep");
+  bool forked = false;
   if (L->Hr > 0) {
     // p == 1 keeps every causal key: the gather reads positions 0..len-1 directly
     const bool dense = L->top_p >= 1.f;
@@ -313,11 +322,22 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
       e = dense ? launch_dense_stats(L, stream) : launch_decode_select(L, stream);
     }
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: select");
+    if (L->n_local > 0) {  // the window attention needs only q_prep: fork it off here
+      e = cudaEventRecord(L->ev_fork, stream);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_fork, 0);
+      if (e == cudaSuccess) e = launch_decode_swa(L, out, L->side);
+      if (e == cudaSuccess) e = cudaEventRecord(L->ev_join, L->side);
+      if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: window attention");
+      forked = true;
+    }
     {
       ProfScope ps(L, "decode_gather", stream);
       e = launch_decode_gather(L, dense, out, stream);
     }
-    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: gather");
+    if (e != cudaSuccess) {
+      if (forked) cudaStreamWaitEvent(stream, L->ev_join, 0);
+      return cuda_fail(L, e, "rtp_decode: gather");
+    }
     if (stats) {
       const size_t P = (size_t)L->B * L->Hr;
       if (stats->sel_count)
@@ -335,10 +355,16 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
                                 (size_t)L->max_select * 4, (size_t)w * 4, P, cudaMemcpyDeviceToDevice, stream);
         }
       }
-      if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: stats");
+      if (e != cudaSuccess) {
+        if (forked) cudaStreamWaitEvent(stream, L->ev_join, 0);
+        return cuda_fail(L, e, "rtp_decode: stats");
+      }
     }
   }
-  if (L->n_local > 0) {
+  if (forked) {
+    e = cudaStreamWaitEvent(stream, L->ev_join, 0);  // join: the output is complete in stream order
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: join");
+  } else if (L->n_local > 0) {
     e = launch_decode_swa(L, out, stream);  // times itself ("decode_swa", "swa_merge")
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: window attention");
   }
