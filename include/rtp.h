@@ -134,7 +134,8 @@ rtp_status rtp_decode(rtp_layer* layer, const void* q, float* out, const rtp_dec
 /* Chunked prefill: the last C appended tokens are the chunk; q is DEVICE bf16 [B][C][Hq][D]
  * pre-RoPE, row i at position len-C+i.  Every row runs its own top-p selection over its causal
  * prefix (retrieval heads) or its own window (local heads).  out is DEVICE fp32 [B][C][Hq][D].
- * Requires 1 <= C <= min(len, max_chunk).  stats may be NULL. */
+ * Requires 1 <= C <= min(len, max_chunk).  The local heads run on an internal stream forked
+ * from `stream` (an event) and joined back (an event).  stats may be NULL. */
 rtp_status rtp_prefill_chunk(rtp_layer* layer, const void* q, int32_t C, float* out,
                              const rtp_prefill_stats* stats, cudaStream_t stream);
 
@@ -153,7 +154,8 @@ rtp_status rtp_reset(rtp_layer* layer);
 rtp_status rtp_truncate(rtp_layer* layer, int64_t new_len);
 
 /* Per-kernel device timing.  While enabled, the library records a CUDA event pair on the
- * launch stream around every kernel it launches.  rtp_profile_read synchronises on the
+ * launch stream around every kernel it launches, and runs every kernel on the call's stream
+ * in order (no internal fork), so each recorded time belongs to one kernel alone.  rtp_profile_read synchronises on the
  * recorded events, returns the summed device time (ms) and launch count of the named kernel
  * ("append_kv", "q_prep", "decode_select", "decode_gather", "decode_swa", "swa_merge",
  * "dense_fill", "prefill_*"; NULL: all kernels together), and clears that kernel's record. */

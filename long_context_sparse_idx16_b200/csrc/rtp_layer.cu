@@ -322,7 +322,7 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
       e = dense ? launch_dense_stats(L, stream) : launch_decode_select(L, stream);
     }
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: select");
-    if (L->n_local > 0) {  // the window attention needs only q_prep: fork it off here
+    if (L->n_local > 0 && !L->prof_on) {  // the window attention needs only q_prep: fork it off
       e = cudaEventRecord(L->ev_fork, stream);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_fork, 0);
       if (e == cudaSuccess) e = launch_decode_swa(L, out, L->side);
@@ -386,13 +386,29 @@ rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out,
     e = launch_q_prep(L, (const __nv_bfloat16*)q, C, L->len - C, stream);
   }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: q_prep");
+  // with both head classes, the local heads run on the internal stream (forked after q_prep,
+  // launched after the retrieval kernels) so they fill the SMs the retrieval kernels leave
+  const bool fork = L->Hr > 0 && L->n_local > 0 && !L->prof_on;
+  if (fork) {
+    e = cudaEventRecord(L->ev_fork, stream);
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: fork");
+  }
   if (L->Hr > 0) {
     e = launch_prefill_retrieval(L, C, out, stats, stream);  // profiled as prefill_select + prefill_attn
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: retrieval heads");
   }
   if (L->n_local > 0) {
-    ProfScope ps(L, "prefill_local", stream);
-    e = launch_prefill_local(L, C, out, stream);
+    cudaStream_t ls = fork ? L->side : stream;
+    if (fork) e = cudaStreamWaitEvent(ls, L->ev_fork, 0);
+    if (e == cudaSuccess) {
+      ProfScope ps(L, "prefill_local", ls);
+      e = launch_prefill_local(L, C, out, ls);
+    }
+    if (fork && e == cudaSuccess) e = cudaEventRecord(L->ev_join, ls);
+    if (fork) {
+      const cudaError_t j = cudaStreamWaitEvent(stream, L->ev_join, 0);
+      if (e == cudaSuccess) e = j;
+    }
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: local heads");
   }
   L->last_error.clear();
