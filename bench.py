@@ -1,6 +1,6 @@
 """Benchmark of the head-wise sparse attention layer (RTPurbo) on B200.
 
-One JSON line on rank 0 (see --help).  A step is one decode token of the 128K workload:
+One JSON line on rank 0 (see --help).  By default a step is one decode token of the 128K workload:
 B = 8 sequences of N = 131072 keys, 32 query / 4 KV heads (D = 128), 5 retrieval heads (r = 16,
 p = 0.9) and 27 local heads (W = 8192, S = 4), seeded synthetic data shaped like the pages'
 workloads.  Each step appends the token's K/V (RoPE + index keys) and runs the decode
@@ -13,6 +13,10 @@ e2e     = the same through the C ABI with the step's q/k/v copied from pinned ho
 roofline= the dominant kernel (fused index stream + top-p select): algorithmic bytes (the
           16-dim fp32 index keys, 64 B per key per retrieval head per sequence) per launch over
           its mean device time from CUDA events on its launch stream
+--workload prefill_32k | prefill_1m: a step is one chunked-prefill call (the chunk's K/V
+          appended, then every row's selection / window and attention), value in ms per chunk;
+          the roofline is the slower of the local-head tcgen05 kernel (flops 4 D sum_i |J_i|
+          per head) and the retrieval attention kernel (4 D per selected pair)
 --impl reference: the fp64 CPU oracle as it stands, on this host's cores, same metric.
 
 Multi-GPU: the layer does not shard; --gpus N runs N independent replicas (one per GPU).
