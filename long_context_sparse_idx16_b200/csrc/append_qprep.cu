@@ -115,6 +115,19 @@ __global__ void __launch_bounds__(128) q_prep_kernel(
     x[u] = h < Hq ? __bfloat162float(qr[h * kD + d]) : 0.f;
     xp[u] = h < Hq ? __bfloat162float(qr[h * kD + (d ^ kHalfD)]) : 0.f;
   }
+  // this thread's index weights (16 dims of one output per retrieval head), read together with
+  // q so the kernel waits on memory once
+  const int o = d >> 3, part = d & 7;
+  int hrs[kQHeads];
+  float wv[kQHeads][16];
+#pragma unroll
+  for (int u = 0; u < kQHeads; ++u) {
+    const int h = h0 + u;
+    hrs[u] = h < Hq ? head_slot[h] : -1;
+    const float* w = wq + (int64_t)(hrs[u] < 0 ? 0 : hrs[u]) * kD * kR + o;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) wv[u][e] = hrs[u] < 0 ? 0.f : w[(part * 16 + e) * kR];
+  }
   if (d < kHalfD) rope_cos_sin(pos, theta[d], &cs[d], &sn[d]);
 #pragma unroll
   for (int u = 0; u < kQHeads; ++u) qs[u][d] = x[u];
@@ -129,16 +142,13 @@ __global__ void __launch_bounds__(128) q_prep_kernel(
     q_rot[(row * Hq + h) * kD + d] = y;
   }
   // index queries: 16 outputs x 8 partial sums of 16 dims each
-  const int o = d >> 3, part = d & 7;
+#pragma unroll
   for (int u = 0; u < kQHeads; ++u) {
-    const int h = h0 + u;
-    if (h >= Hq) break;
-    const int hr = head_slot[h];
-    if (hr < 0) continue;
-    const float* w = wq + (int64_t)hr * kD * kR + o;
+    const int hr = hrs[u];
+    if (hr < 0) continue;  // uniform over the CTA: the head (or its absence) is blockIdx-derived
     float acc = 0.f;
 #pragma unroll
-    for (int e = part * 16; e < part * 16 + 16; ++e) acc = fmaf(w[e * kR], qs[u][e], acc);
+    for (int e = 0; e < 16; ++e) acc = fmaf(wv[u][e], qs[u][part * 16 + e], acc);
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
     acc += __shfl_xor_sync(0xffffffffu, acc, 4);
