@@ -41,3 +41,18 @@ def test_reference_arm_prefill_json_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "ms/chunk" and d["value"] > 0
     assert "prefill_32k" in d["config"]["workload"]
+
+
+def test_local_pairs_matches_brute_force():
+    # the local-head flop count of the prefill roofline: sum over chunk rows of |J_i|
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+
+    for prefix, chunk, W, S in [(0, 300, 96, 4), (1000, 200, 128, 4), (400, 140, 1, 0), (400, 140, 64, 70),
+                                (0, 50, 100000, 4)]:
+        s = synth.spec("prefill_32k", prefix=prefix, chunk=chunk, window=W, n_sink=S)
+        brute = 0
+        for i in range(prefix, prefix + chunk):
+            brute += sum(1 for j in range(i + 1) if i - j < W or j < S)
+        assert bench._local_pairs(s) == brute
