@@ -73,7 +73,7 @@ def _profile_traffic(kernel_src: str):
     src_hash = None
     for line in text.splitlines():
         if line.startswith("- source sha256[:16]:"):
-            src_hash = line.split(":", 1)[1].strip()
+            src_hash = line.rsplit(":", 1)[1].strip()
         if line.startswith("- dram bytes per launch (read + write):"):
             traffic = float(line.split(":", 1)[1].strip().split()[0])
     return traffic if (src_hash == want and traffic) else None

@@ -56,3 +56,26 @@ def test_local_pairs_matches_brute_force():
         for i in range(prefix, prefix + chunk):
             brute += sum(1 for j in range(i + 1) if i - j < W or j < S)
         assert bench._local_pairs(s) == brute
+
+
+def test_profile_traffic_follows_the_kernel_source(tmp_path):
+    # the committed ncu summary gives the select kernel's DRAM bytes only while the kernel
+    # source still hashes to the value recorded beside them
+    sys.path.insert(0, ROOT)
+    import bench
+
+    src = os.path.join(ROOT, "long_context_sparse_idx16_b200", "csrc", "decode_select.cu")
+    text = open(os.path.join(ROOT, "profiles", "decode_select_128k.md")).read()
+    rec = [ln for ln in text.splitlines() if ln.startswith("- dram bytes per launch")]
+    assert len(rec) == 1
+    want = float(rec[0].rsplit(":", 1)[1].split()[0])
+    got = bench._profile_traffic(src)
+    changed = tmp_path / "decode_select.cu"
+    changed.write_bytes(open(src, "rb").read() + b"\n")
+    assert bench._profile_traffic(str(changed)) is None
+    import hashlib
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if ("- source sha256[:16]: " + h) in text:
+        assert got == want
+    else:
+        assert got is None
