@@ -102,9 +102,29 @@ def test_decode_1m_full_size(p):
 
 
 def test_decode_128k_full_size():
+    # Full 128K decode workload (B=8), decoded twice on one layer: the selection scratch is
+    # cleaned by each launch for the next, and the exact selection makes both launches give
+    # the same bits.  The layer is then checked against the oracle.
+    import torch
+
+    from long_context_sparse_idx16_b200 import Layer
+    from parity import build_cache, torch_bf16
+
     x = synth.generate(synth.spec("decode_128k"))
-    heads = list(x.spec.retrieval_heads) + [2, 12, 20, 31]
-    run_decode(x, heads=heads)
+    s = x.spec
+    layer = Layer.from_spec(s, x, max_chunk=1)
+    build_cache(layer, x, s.n_total)
+    q = torch_bf16(x.q[:, 0])
+    o1, st1 = layer.decode(q, stats=True, sel_cap=s.n_total)
+    o2, st2 = layer.decode(q, stats=True, sel_cap=s.n_total)
+    torch.cuda.synchronize()
+    assert layer.check() == 0
+    assert torch.equal(o1, o2)
+    for a, b in zip(st1, st2):
+        assert torch.equal(a, b)
+    heads = list(s.retrieval_heads) + [2, 12, 20, 31]
+    run_decode(x, heads=heads, layer=layer)
+    layer.close()
 
 
 _state = {}
