@@ -82,7 +82,9 @@ def _cfg(**kw):
 @pytest.mark.parametrize("bad", [dict(head_dim=64), dict(index_dim=8), dict(top_p=0.0), dict(top_p=1.5),
                                  dict(n_kv_heads=3), dict(window=0), dict(n_sink=-1), dict(max_seq=0),
                                  dict(max_select=65), dict(batch=0), dict(head_class=None),
-                                 dict(n_q_heads=64, n_kv_heads=2), dict(rope_base=1.0)])
+                                 dict(n_q_heads=64, n_kv_heads=2), dict(rope_base=1.0), dict(sm_scale=-1.0),
+                                 dict(max_chunk=-1), dict(max_seq=1 << 31), dict(wq_index=None),
+                                 dict(wk_index=None), dict(top_p=float("nan")), dict(max_select=-1)])
 def test_create_rejects_bad_config_on_host(lib, bad):
     cfg, keep = _cfg(**bad)
     h = C.c_void_p()
@@ -100,3 +102,20 @@ def test_calls_on_null_layer_are_rejected(lib):
     assert lib.rtp_seq_len(None) == -1
     assert lib.rtp_destroy(None) == rtp.RTP_OK
     assert lib.rtp_create(None, None) == rtp.RTP_EINVAL
+
+
+def test_create_rejects_bad_head_maps_on_host(lib):
+    import numpy as np
+
+    # a class entry other than 0 (local) or 1 (retrieval)
+    hc = np.array([1, 2, 0, 0], dtype=np.uint8)
+    cfg, keep = _cfg(head_class=hc.ctypes.data)
+    h = C.c_void_p()
+    assert lib.rtp_create(C.byref(cfg), C.byref(h)) == rtp.RTP_EINVAL
+    assert h.value is None
+    # more (sequence, retrieval head) problems than the selection scratch is laid out for
+    hc = np.ones(16, dtype=np.uint8)
+    cfg, keep = _cfg(batch=129, n_q_heads=16, n_kv_heads=1, head_class=hc.ctypes.data)
+    assert lib.rtp_create(C.byref(cfg), C.byref(h)) == rtp.RTP_EINVAL
+    assert h.value is None
+    assert "2048" in rtp.rtp_last_error(None)
