@@ -189,6 +189,30 @@ def _stream_handle(stream=None) -> int:
     return int(s.cuda_stream)
 
 
+def _need(t, name: str, shape, dtype, device) -> None:
+    """Raise unless t is a contiguous tensor of exactly this shape, dtype and device: the
+    library reads and writes raw device pointers sized from the layer's configuration."""
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device != device:
+        raise ValueError(f"{name}: expected a tensor on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+
+
+def _dim(t, name: str, ndim: int, axis: int) -> int:
+    """Size of one axis of a tensor that must have ndim dimensions."""
+    if getattr(t, "dim", None) is None or t.dim() != ndim:
+        raise ValueError(f"{name}: expected a {ndim}-dimensional tensor")
+    return int(t.shape[axis])
+
+
 class Layer:
     """One sparse attention layer: owns a librtp layer on the current CUDA device."""
 
@@ -209,6 +233,9 @@ class Layer:
             max_select=max_select, max_chunk=max_chunk)
         self.batch, self.n_q_heads, self.n_kv_heads = batch, n_q_heads, n_kv_heads
         self.handle = rtp_create(cfg)
+        import torch
+
+        self.device = torch.device("cuda", torch.cuda.current_device())  # where rtp_create put it
 
     @classmethod
     def from_spec(cls, spec, inputs=None, *, max_seq: Optional[int] = None, **kw):
@@ -251,8 +278,12 @@ class Layer:
 
     def append_kv(self, k, v, stream=None) -> None:
         """k, v: torch bf16 CUDA tensors [B][T][Hkv][128] (k pre-RoPE)."""
-        assert k.is_cuda and k.is_contiguous() and v.is_contiguous()
-        rtp_append_kv(self.handle, k.data_ptr(), v.data_ptr(), int(k.shape[1]), _stream_handle(stream))
+        import torch
+
+        T = _dim(k, "k", 4, 1)
+        _need(k, "k", (self.batch, T, self.n_kv_heads, 128), torch.bfloat16, self.device)
+        _need(v, "v", (self.batch, T, self.n_kv_heads, 128), torch.bfloat16, self.device)
+        rtp_append_kv(self.handle, k.data_ptr(), v.data_ptr(), T, _stream_handle(stream))
 
     def decode(self, q, out=None, stats: bool = False, sel_cap: int = 0, stream=None):
         """q: torch bf16 CUDA tensor [B][Hq][128] at position len-1.  Returns out (fp32) and,
@@ -260,9 +291,12 @@ class Layer:
         sel_index holds the first sel_cap selected positions (None when sel_cap == 0)."""
         import torch
 
-        assert q.is_cuda and q.is_contiguous()
+        _need(q, "q", (self.batch, self.n_q_heads, 128), torch.bfloat16, self.device)
         if out is None:
             out = torch.empty((self.batch, self.n_q_heads, 128), dtype=torch.float32, device=q.device)
+        _need(out, "out", (self.batch, self.n_q_heads, 128), torch.float32, self.device)
+        if sel_cap < 0:
+            raise ValueError("sel_cap must be >= 0")
         st = None
         tensors = None
         if stats and self.n_retrieval:
@@ -284,10 +318,13 @@ class Layer:
         sel_bitmap [B][C][Hr][bitmap_words] int32 or None)."""
         import torch
 
-        assert q.is_cuda and q.is_contiguous()
-        Cr = int(q.shape[1])
+        Cr = _dim(q, "q", 4, 1)
+        _need(q, "q", (self.batch, Cr, self.n_q_heads, 128), torch.bfloat16, self.device)
         if out is None:
             out = torch.empty((self.batch, Cr, self.n_q_heads, 128), dtype=torch.float32, device=q.device)
+        _need(out, "out", (self.batch, Cr, self.n_q_heads, 128), torch.float32, self.device)
+        if bitmap_words < 0:
+            raise ValueError("bitmap_words must be >= 0")
         st = None
         tensors = None
         if stats and self.n_retrieval:
