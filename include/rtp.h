@@ -19,8 +19,9 @@
  *
  * Conventions shared by every entry point
  *   - All device pointers are plain CUDA device addresses on the layer's device; every
- *     call is asynchronous and ordered on the stream it is given.  Nothing synchronises
- *     the stream except rtp_check.
+ *     call is asynchronous and ordered on the stream it is given.  Of the per-call entry
+ *     points only rtp_check synchronises its stream (and rtp_profile_read waits for the
+ *     profiled kernels); rtp_create and rtp_destroy synchronise the device.
  *   - The caller owns q/k/v/out and the streams.  The layer owns its KV cache, index-key
  *     cache, weight copies and all scratch, and frees them in rtp_destroy.
  *   - Argument errors are detected on the host before any launch and return RTP_EINVAL
