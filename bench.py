@@ -60,6 +60,38 @@ def _tensor_peak():
         return 1590.0, "fallback"
 
 
+# MUFU (ex2) issue rate per SM per clock on B200, the unit the prefill selection's exponentials
+# run on; the peak is this rate times the SM count times the sampled SM clock.
+MUFU_EX2_PER_CLK_SM = 16
+
+
+def _prefill_roofline(kern: dict, flops: dict, exps: int, sm_mhz, n_sm: int, tensor_peak: float,
+                      tensor_peak_kind: str) -> dict:
+    """Roofline object of the prefill chunk's dominant kernel (the one with the longest time).
+
+    The selection (prefill_select) evaluates one exponential per causal (row, key) pair and
+    is bound by the exp (MUFU) and integer pipes, so it is reported as "alu" against
+    MUFU_EX2_PER_CLK_SM x SMs x clock.  The attention kernels are reported against the dense
+    16-bit tensor peak with their algorithmic flops (4 D per attended pair)."""
+    cands = [k for k in ("prefill_select", "prefill_attn", "prefill_local") if kern.get(k, {}).get("ms_per_launch", 0) > 0]
+    dom = max(cands, key=lambda k: kern[k]["ms_per_launch"])
+    ms = kern[dom]["ms_per_launch"]
+    if dom == "prefill_select":
+        mhz = float(sm_mhz) if sm_mhz else 1965.0
+        peak = MUFU_EX2_PER_CLK_SM * n_sm * mhz * 1e6 / 1e9
+        achieved = exps / (ms * 1e-3) / 1e9
+        return {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
+                "peak_kind": f"derived: {MUFU_EX2_PER_CLK_SM} ex2 per clock per SM x {n_sm} SMs x "
+                             f"{mhz:.0f} MHz ({'sampled' if sm_mhz else 'nominal max'} SM clock)",
+                "unit": "Gexp/s", "frac": achieved / peak, "traffic": None,
+                "exps_per_launch": int(exps), "ms_per_launch": ms}
+    f = flops["local_attention"] if dom == "prefill_local" else flops["retrieval_attention"]
+    achieved = f / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tensor_peak,
+            "peak_kind": tensor_peak_kind, "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": None,
+            "flops_per_launch": int(f), "ms_per_launch": ms}
+
+
 def _profile_traffic(kernel_src: str):
     """Per-launch DRAM traffic of the select kernel from the committed ncu summary, if the
     kernel source has not changed since that capture (else None)."""
@@ -626,21 +658,25 @@ def run_prefill_gpu(args):
     kern = {}
     for k, (kms, kn) in per.items():
         kern[k] = {"ms_per_launch": kms / max(kn, 1), "launches": kn}
-    lk, rk = kern["prefill_local"], kern["prefill_attn"]
-    dom = "prefill_local" if lk["ms_per_launch"] >= rk["ms_per_launch"] else "prefill_attn"
-    dom_flops = local_flops if dom == "prefill_local" else ret_flops
-    achieved = dom_flops / (kern[dom]["ms_per_launch"] * 1e-3) / 1e12
+    flops = {"local_attention": local_flops, "retrieval_attention": ret_flops,
+             "index_scores": Hr * B * (C * P + C * (C + 1) // 2)}
+    roof = _prefill_roofline(kern, flops, flops["index_scores"], clk.get("sm_mhz"),
+                             torch.cuda.get_device_properties(dev).multi_processor_count, peak, peak_kind)
+    # the tensor-core kernels, each against the tensor peak
+    tensor = {}
+    for k, f in (("prefill_local", local_flops), ("prefill_attn", ret_flops)):
+        if k in kern and kern[k]["ms_per_launch"] > 0:
+            a_ = f / (kern[k]["ms_per_launch"] * 1e-3) / 1e12
+            tensor[k] = {"achieved_tflops": a_, "frac": a_ / peak, "flops_per_launch": int(f)}
     line = {
         "metric": METRIC, "value": value, "unit": "ms/chunk", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16 mma / f32", "data": "synthetic",
         "config": _prefill_config(s, world),
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                     "flops_per_launch": dom_flops, "ms_per_launch": kern[dom]["ms_per_launch"]},
+        "roofline": roof,
+        "tensor_kernels": tensor,
         "kernels": kern,
-        "flops": {"local_attention": local_flops, "retrieval_attention": ret_flops,
-                  "index_scores": Hr * B * (C * P + C * (C + 1) // 2)},
+        "flops": flops,
         "e2e": {"value": e2e_ms / args.steps, "unit": "ms/chunk",
                 "h2d_bytes_per_step": int((q.numel() + k_c.numel() + v_c.numel()) * 2),
                 "d2h_bytes_per_step": int(out.numel() * 4)},

@@ -79,3 +79,23 @@ def test_profile_traffic_follows_the_kernel_source(tmp_path):
         assert got == want
     else:
         assert got is None
+
+
+def test_prefill_roofline_follows_the_dominant_kernel():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    flops = {"local_attention": 3.0e12, "retrieval_attention": 6.0e9, "index_scores": 2.0e9}
+    kern = {"prefill_select": {"ms_per_launch": 10.0}, "prefill_attn": {"ms_per_launch": 5.0},
+            "prefill_local": {"ms_per_launch": 6.0}, "q_prep": {"ms_per_launch": 99.0}}
+    r = bench._prefill_roofline(kern, flops, 2.0e9, 2000.0, 148, 1650.0, "measured")
+    # the selection dominates: one exp per causal pair against 16 ex2 / clock / SM
+    assert r["kernel"] == "prefill_select" and r["bound"] == "alu" and r["unit"] == "Gexp/s"
+    assert abs(r["achieved"] - 2.0e9 / 10e-3 / 1e9) < 1e-9
+    assert abs(r["peak"] - 16 * 148 * 2000.0e6 / 1e9) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+    # the local heads dominate: tensor roofline with their flops
+    kern["prefill_local"]["ms_per_launch"] = 20.0
+    r = bench._prefill_roofline(kern, flops, 2.0e9, None, 148, 1650.0, "measured")
+    assert r["kernel"] == "prefill_local" and r["bound"] == "tensor"
+    assert abs(r["achieved"] - 3.0e12 / 20e-3 / 1e12) < 1e-9 and r["peak"] == 1650.0
