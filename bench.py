@@ -15,8 +15,10 @@ roofline= the dominant kernel (fused index stream + top-p select): algorithmic b
           its mean device time from CUDA events on its launch stream
 --workload prefill_32k | prefill_1m: a step is one chunked-prefill call (the chunk's K/V
           appended, then every row's selection / window and attention), value in ms per chunk;
-          the roofline is the slower of the local-head tcgen05 kernel (flops 4 D sum_i |J_i|
-          per head) and the retrieval attention kernel (4 D per selected pair)
+          the roofline is the chunk's longest kernel: the selection against the MUFU peak
+          (one exp per causal (row, key) pair), or the local-head tcgen05 kernel (flops
+          4 D sum_i |J_i| per head) or the retrieval attention kernel (4 D per selected pair)
+          against the tensor peak
 --impl reference: the fp64 CPU oracle as it stands, on this host's cores, same metric.
 
 Multi-GPU: the layer does not shard; --gpus N runs N independent replicas (one per GPU).
