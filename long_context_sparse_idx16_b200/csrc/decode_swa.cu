@@ -314,10 +314,13 @@ __global__ void __launch_bounds__(256) swa_merge_kernel(const float* __restrict_
 
 }  // namespace
 
-// Chunking: enough CTAs to cover the SMs about twice, in whole 128-key tiles.
+// Chunking, in whole 128-key tiles: at most two CTAs per SM over the whole grid, so the grid
+// runs as one wave (the kernel's registers -- about 254 per thread at 128 threads -- let two
+// CTAs share an SM; a third CTA on any SM would wait for a second wave).
 static void swa_chunks(const rtp_layer* L, int64_t nJ, int64_t* chunk_keys, int* n_chunks) {
   const int64_t pairs = (int64_t)L->B * L->Hkv;
-  const int64_t want = (2LL * L->sm_count + pairs - 1) / pairs;  // chunks per (b, g)
+  int64_t want = (2LL * L->sm_count) / pairs;  // chunks per (b, g)
+  if (want < 1) want = 1;
   int64_t ck = (nJ + want - 1) / want;
   ck = (ck + kTile - 1) / kTile * kTile;
   if (ck < kTile) ck = kTile;
@@ -325,7 +328,8 @@ static void swa_chunks(const rtp_layer* L, int64_t nJ, int64_t* chunk_keys, int*
   *n_chunks = (int)((nJ + ck - 1) / ck);
 }
 
-// Upper bound on chunks for any length: chunk_keys >= nJ / want, so n_chunks <= want.
+// Upper bound on chunks for any length: chunk_keys >= nJ / want, so n_chunks <= want, and
+// want is at most this.
 static int64_t swa_max_chunks(const rtp_layer* L) {
   const int64_t pairs = (int64_t)L->B * L->Hkv;
   return (2LL * L->sm_count + pairs - 1) / pairs;
