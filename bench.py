@@ -67,6 +67,36 @@ def _tensor_peak():
 MUFU_EX2_PER_CLK_SM = 16
 
 
+def _prefill_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of the prefill selection at the 32K chunk, from the committed ncu
+    summary, while its sources are unchanged since the capture (else None).  Other kernels and
+    the 1M chunk have no capture whose bytes would scale: the 32K index keys sit in L2, the
+    1M ones do not."""
+    if kernel != "prefill_select" or workload != "prefill_32k":
+        return None
+    try:
+        text = open(os.path.join(ROOT, "profiles", "prefill_kernels_32k.md")).read()
+    except OSError:
+        return None
+    traffic, srcs = None, None
+    for line in text.splitlines():
+        if line.startswith("- prefill_select dram bytes per launch (read + write):"):
+            traffic = float(line.rsplit(":", 1)[1].strip().split()[0])
+        if line.startswith("- prefill_select sources sha256[:16]:"):
+            srcs = line.split("sha256[:16]:", 1)[1].strip()
+    if traffic is None or srcs is None:
+        return None
+    for item in srcs.split(","):
+        name, want = item.split()
+        path = os.path.join(ROOT, "long_context_sparse_idx16_b200", "csrc", name)
+        try:
+            if hashlib.sha256(open(path, "rb").read()).hexdigest()[:16] != want:
+                return None
+        except OSError:
+            return None
+    return traffic
+
+
 def _prefill_roofline(kern: dict, flops: dict, exps: int, sm_mhz, n_sm: int, tensor_peak: float,
                       tensor_peak_kind: str) -> dict:
     """Roofline object of the prefill chunk's dominant kernel (the one with the longest time).
@@ -664,6 +694,7 @@ def run_prefill_gpu(args):
              "index_scores": Hr * B * (C * P + C * (C + 1) // 2)}
     roof = _prefill_roofline(kern, flops, flops["index_scores"], clk.get("sm_mhz"),
                              torch.cuda.get_device_properties(dev).multi_processor_count, peak, peak_kind)
+    roof["traffic"] = _prefill_traffic(roof["kernel"], s.name)
     # the tensor-core kernels, each against the tensor peak
     tensor = {}
     for k, f in (("prefill_local", local_flops), ("prefill_attn", ret_flops)):

@@ -99,3 +99,13 @@ def test_prefill_roofline_follows_the_dominant_kernel():
     r = bench._prefill_roofline(kern, flops, 2.0e9, None, 148, 1650.0, "measured")
     assert r["kernel"] == "prefill_local" and r["bound"] == "tensor"
     assert abs(r["achieved"] - 3.0e12 / 20e-3 / 1e12) < 1e-9 and r["peak"] == 1650.0
+
+
+def test_prefill_traffic_only_for_the_captured_kernel_and_chunk():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    t = bench._prefill_traffic("prefill_select", "prefill_32k")
+    assert t is None or t == 24222464.0  # None once the kernel sources change
+    assert bench._prefill_traffic("prefill_select", "prefill_1m") is None
+    assert bench._prefill_traffic("prefill_local", "prefill_32k") is None
