@@ -692,7 +692,7 @@ def run_prefill_gpu(args):
         kern[k] = {"ms_per_launch": kms / max(kn, 1), "launches": kn}
     flops = {"local_attention": local_flops, "retrieval_attention": ret_flops,
              "index_scores": Hr * B * (C * P + C * (C + 1) // 2)}
-    roof = _prefill_roofline(kern, flops, flops["index_scores"], clk.get("sm_mhz"),
+    roof = _prefill_roofline(kern, flops, flops["index_scores"], (clk or {}).get("sm_mhz"),
                              torch.cuda.get_device_properties(dev).multi_processor_count, peak, peak_kind)
     roof["traffic"] = _prefill_traffic(roof["kernel"], s.name)
     # the tensor-core kernels, each against the tensor peak
