@@ -41,10 +41,11 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
 
   const __nv_bfloat16* kt = k + ((int64_t)b * T + t) * Hkv * kD;
   const __nv_bfloat16* vt = v + ((int64_t)b * T + t) * Hkv * kD;
-  // every global read of the token is issued before any is used: one memory round trip
+  // every global read of the token is issued before any is used: one memory round trip (the
+  // index weights go straight to shared memory with cp.async, all copies in flight at once)
   const int nw = min(Hr, kWHeads);
-  for (int i = threadIdx.x; i < nw * kD * kR / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(ws)[i] = reinterpret_cast<const float4*>(wk)[i];
+  for (int i = threadIdx.x; i < nw * kD * kR / 4; i += blockDim.x) cp_async16(ws + 4 * i, wk + 4 * i, 16);
+  cp_async_commit();
   for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) ks[i] = __bfloat162float(kt[i]);
   if (threadIdx.x < kHalfD) rope_cos_sin(pos, theta[threadIdx.x], &cs[threadIdx.x], &sn[threadIdx.x]);
   bool bad = false;
@@ -54,6 +55,7 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
     bad |= !(fabsf(x) <= kFp16Max);
     vc[(((int64_t)b * Hkv + g) * max_seq + pos) * kD + d] = __float2half_rn(x);
   }
+  cp_async_wait<0>();
   __syncthreads();
 
   for (int i = threadIdx.x; i < Hkv * kHalfD; i += blockDim.x) {
