@@ -92,12 +92,22 @@ typedef struct {
  * (j % 32) of word j / 32 is set iff key j is in row i's selected set.  Words the kernel writes:
  * those covering keys 0 .. (last position of the row's 64-row tile), rounded up to 64 keys and
  * capped at bitmap_words; the caller zeroes the rest.  Keys past 32 * bitmap_words are not
- * reported (the selection itself is unaffected). */
+ * reported (the selection itself is unaffected).
+ *
+ * Row-subset positions (cheap at any chunk size, where a full bitmap is not): for each of the
+ * n_rows distinct chunk rows listed in `rows` (DEVICE int32, 0 <= row < C; other values are
+ * ignored) and each retrieval head, row_sel receives the row's selected positions in
+ * ascending order, the first min(|J_i|, row_sel_cap) of them; |J_i| itself is in sel_count,
+ * which must then be non-NULL.  Entries past the count are not written. */
 typedef struct {
   int32_t* sel_count;    /* [B][C][Hr] |J_i| */
   float* sel_mass;       /* [B][C][Hr] index-softmax mass of J_i (>= p) */
   uint32_t* sel_bitmap;  /* [B][C][Hr][bitmap_words] */
   int64_t bitmap_words;
+  const int32_t* rows;   /* [n_rows] chunk rows whose selected positions are listed, or NULL */
+  int32_t n_rows;
+  int32_t* row_sel;      /* [B][n_rows][Hr][row_sel_cap] */
+  int64_t row_sel_cap;
 } rtp_prefill_stats;
 
 /* Device-side view of the layer's caches (for tests and tools; read-only use). */
@@ -143,6 +153,14 @@ rtp_status rtp_prefill_chunk(rtp_layer* layer, const void* q, int32_t C, float* 
 /* Change p for later calls (0 < p <= 1).  Takes effect in stream order of later calls. */
 rtp_status rtp_set_top_p(rtp_layer* layer, float top_p);
 
+/* Test knob: the limit, in SM clock cycles, on each wait of the decode selection's grid-wide
+ * barriers (0 restores the default, about one second).  A wait past its limit makes the
+ * kernel record RTP_ETIMEOUT and leave; the next rtp_check reports it and resets the
+ * selection's scratch, so later calls start clean.  A tiny limit makes the barrier give up
+ * at once, which is how the timeout path is tested.  The tensor-core completion waits of the
+ * prefill kernels keep their fixed limit.  RTP_EINVAL if cycles < 0. */
+rtp_status rtp_set_wait_limit(rtp_layer* layer, int64_t cycles);
+
 /* Current sequence length (host-side counter; advanced by rtp_append_kv). */
 int64_t rtp_seq_len(const rtp_layer* layer);
 
@@ -179,14 +197,20 @@ rtp_status rtp_get_cache(const rtp_layer* layer, rtp_cache_view* view);
  * positions j = idx[p][0 .. min(cnt[p], max_count)).  K_j and V_j are fp16 rows of 128 values at
  * k / v + kv_block[p] * kv_stride + j * 128 (kv_block NULL: block p); q is DEVICE fp32 [P][128]
  * (already RoPE'd), idx DEVICE int32 [P][idx_stride], cnt DEVICE int32 [P], out DEVICE fp32
- * [P][128].  Rows of the layer's cache (rtp_get_cache) can be passed directly.
+ * [P][128].  Rows of the layer's cache (rtp_get_cache) can be passed directly.  A problem whose
+ * count is <= 0 has an empty list; its output row is written as zeros.
+ *
+ * Alignment: k, v and q must be 16-byte aligned and kv_stride a multiple of 8 elements (rows
+ * are read as 16-byte vectors); otherwise RTP_EINVAL, nothing launched.  Every listed position
+ * must lie inside its block: positions are not checked.
  *
  * Scratch: one built-in device array of about 2.1 MB (4096 work items of 128 keys); the call
  * returns RTP_EINVAL without launching when P * ceil(max_count / 128) exceeds 4096 or P > 2048.
  * The first call on each device (with that device current) looks the array's address up and
- * caches it: make that first call before any stream capture.  Every call on a device shares the
- * array, so calls whose kernels overlap on the GPU race; serialise them (one stream).  Errors
- * are reported through rtp_last_error(NULL). */
+ * caches it for the life of the process (the cache assumes the device's primary context is
+ * never reset): make that first call before any stream capture.  Every call on a device shares
+ * the array, so calls whose kernels overlap on the GPU race; serialise them (one stream).
+ * Errors are reported through rtp_last_error(NULL). */
 rtp_status rtp_gather_attn_noalloc(const void* k, const void* v, const int32_t* kv_block, int64_t kv_stride,
                                    const float* q, const int32_t* idx, int64_t idx_stride,
                                    const int32_t* cnt, int32_t P, int64_t max_count, float sm_scale,

@@ -43,7 +43,8 @@ class rtp_decode_stats(C.Structure):
 
 class rtp_prefill_stats(C.Structure):
     _fields_ = [("sel_count", C.c_void_p), ("sel_mass", C.c_void_p), ("sel_bitmap", C.c_void_p),
-                ("bitmap_words", C.c_int64)]
+                ("bitmap_words", C.c_int64), ("rows", C.c_void_p), ("n_rows", C.c_int32),
+                ("row_sel", C.c_void_p), ("row_sel_cap", C.c_int64)]
 
 
 class rtp_cache_view(C.Structure):
@@ -76,6 +77,7 @@ def lib() -> C.CDLL:
             "rtp_decode": ([P, P, P, C.POINTER(rtp_decode_stats), P], C.c_int),
             "rtp_prefill_chunk": ([P, P, i32, P, C.POINTER(rtp_prefill_stats), P], C.c_int),
             "rtp_set_top_p": ([P, f32], C.c_int),
+            "rtp_set_wait_limit": ([P, i64], C.c_int),
             "rtp_seq_len": ([P], i64),
             "rtp_reset": ([P], C.c_int),
             "rtp_check": ([P, P], C.c_int),
@@ -129,6 +131,11 @@ def rtp_prefill_chunk(layer, q_ptr: int, C_rows: int, out_ptr: int, stats: Optio
 
 def rtp_set_top_p(layer, p: float) -> None:
     _check(lib().rtp_set_top_p(layer, p), layer)
+
+
+def rtp_set_wait_limit(layer, cycles: int) -> None:
+    """Test knob: clock-cycle limit of the decode selection's grid-barrier waits (0: default)."""
+    _check(lib().rtp_set_wait_limit(layer, int(cycles)), layer)
 
 
 def rtp_seq_len(layer) -> int:
@@ -264,6 +271,9 @@ class Layer:
     def set_top_p(self, p: float) -> None:
         rtp_set_top_p(self.handle, p)
 
+    def set_wait_limit(self, cycles: int) -> None:
+        rtp_set_wait_limit(self.handle, cycles)
+
     def reset(self) -> None:
         rtp_reset(self.handle)
 
@@ -311,11 +321,14 @@ class Layer:
         rtp_decode(self.handle, q.data_ptr(), out.data_ptr(), st, _stream_handle(stream))
         return (out, tensors) if stats else out
 
-    def prefill_chunk(self, q, out=None, stats: bool = False, bitmap_words: int = 0, stream=None):
+    def prefill_chunk(self, q, out=None, stats: bool = False, bitmap_words: int = 0, rows=None,
+                      row_sel_cap: int = 0, stream=None):
         """q: torch bf16 CUDA tensor [B][C][Hq][128]; row i at position len-C+i.
 
         With stats, also returns (sel_count [B][C][Hr] int32, sel_mass [B][C][Hr] fp32,
-        sel_bitmap [B][C][Hr][bitmap_words] int32 or None)."""
+        sel_bitmap [B][C][Hr][bitmap_words] int32 or None, row_sel [B][len(rows)][Hr][row_sel_cap]
+        int32 or None).  `rows` (distinct chunk rows) asks for those rows' selected positions,
+        ascending, the first row_sel_cap of each (unused entries stay -1)."""
         import torch
 
         Cr = _dim(q, "q", 4, 1)
@@ -325,16 +338,28 @@ class Layer:
         _need(out, "out", (self.batch, Cr, self.n_q_heads, 128), torch.float32, self.device)
         if bitmap_words < 0:
             raise ValueError("bitmap_words must be >= 0")
+        if rows is not None and (not stats or row_sel_cap < 1):
+            raise ValueError("rows needs stats=True and row_sel_cap >= 1")
         st = None
         tensors = None
         if stats and self.n_retrieval:
             shp = (self.batch, Cr, self.n_retrieval)
             bm = (torch.zeros(shp + (bitmap_words,), dtype=torch.int32, device=q.device)
                   if bitmap_words > 0 else None)
+            rl = rs = None
+            if rows is not None:
+                rl = torch.as_tensor(list(rows), dtype=torch.int32).to(q.device)
+                if rl.numel() < 1 or int(rl.min()) < 0 or int(rl.max()) >= Cr:
+                    raise ValueError("rows must be chunk rows in [0, C)")
+                rs = torch.full((self.batch, rl.numel(), self.n_retrieval, row_sel_cap), -1, dtype=torch.int32,
+                                device=q.device)
             tensors = (torch.empty(shp, dtype=torch.int32, device=q.device),
-                       torch.empty(shp, dtype=torch.float32, device=q.device), bm)
+                       torch.empty(shp, dtype=torch.float32, device=q.device), bm, rs)
             st = rtp_prefill_stats(tensors[0].data_ptr(), tensors[1].data_ptr(),
-                                   bm.data_ptr() if bm is not None else None, bitmap_words)
+                                   bm.data_ptr() if bm is not None else None, bitmap_words,
+                                   rl.data_ptr() if rl is not None else None, rl.numel() if rl is not None else 0,
+                                   rs.data_ptr() if rs is not None else None, row_sel_cap)
+            self._keep = rl  # the row list must outlive the asynchronous call
         rtp_prefill_chunk(self.handle, q.data_ptr(), Cr, out.data_ptr(), st, _stream_handle(stream))
         return (out, tensors) if stats else out
 

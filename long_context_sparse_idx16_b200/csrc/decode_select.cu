@@ -92,6 +92,7 @@ struct SelectArgs {
   uint32_t* flags;            // [1]: some problem needs the radix fallback
   uint32_t* err;
   float* gscores;
+  long long wait_limit;       // clock cycles a grid-barrier wait may take before it gives up
 };
 
 struct Seg {
@@ -159,8 +160,12 @@ __device__ __forceinline__ void add_words(uint32_t* lo_w, uint32_t* hi_w, uint32
 }
 
 // Monotonic grid barrier: one atomic per CTA on a 64-bit counter that only grows, then an
-// acquire spin until the counter reaches the next multiple of the grid size.  Bounded.
-__device__ __forceinline__ bool grid_sync(unsigned long long* bar, uint32_t nblocks, uint32_t* err) {
+// acquire spin until the counter reaches the next multiple of the grid size.  Bounded by
+// `limit` clock cycles.  A CTA that gives up has still arrived, so the CTAs that do pass the
+// barrier see every CTA's writes from before it; a CTA that gave up never arrives at the next
+// barrier, which therefore nobody passes.
+__device__ __forceinline__ bool grid_sync(unsigned long long* bar, uint32_t nblocks, uint32_t* err,
+                                          long long limit) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -173,7 +178,7 @@ __device__ __forceinline__ bool grid_sync(unsigned long long* bar, uint32_t nblo
       unsigned long long v;
       asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(bar) : "memory");
       if (v >= target) break;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         atomicOr(err, kErrTimeout);
         ok = 0;
         break;
@@ -409,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     mx = block_max(mx, S);
     if (tid == 0) a.seg_max[s.p + c] = mx;
   }
-  if (!grid_sync(a.bar, G, a.err)) return;
+  if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
 
   // ---- phase B: row maxima; level-1 mass histogram; keep lists.  Warp w walks a contiguous
   // chunk of the segment.  Keys within 16 of the max join the warp's ordered keep list (their
@@ -480,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     }
     __syncthreads();
   }
-  if (!grid_sync(a.bar, G, a.err)) return;
+  if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
 
   // ---- phase C: total mass, target, crossing bin; its keys become candidates.  A crossing in
   // the coarse bin, or more than kCand keys in the crossing bin, takes the radix fallback.
@@ -555,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     }
     __syncthreads();
   }
-  if (!grid_sync(a.bar, G, a.err)) return;
+  if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
 
   // ---- phase D: exact cut.  Problems whose crossing bin fits the candidate list sort it;
   // the others (decided identically by every CTA from the global counts) refine by radix.
@@ -638,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
         flush_words(S, a.hr, (int64_t)lev * nh + (int64_t)p * kBins);
         __syncthreads();
       }
-      if (!grid_sync(a.bar, G, a.err)) return;
+      if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
       for (int si = 0; si < nseg; ++si) {
         if (!S.seg[si].radix) continue;
         const int p = S.seg[si].p;
@@ -698,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     }
     __syncthreads();
   }
-  if (!grid_sync(a.bar, G, a.err)) return;
+  if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
   // Every CTA has passed its last barrier: the last one to get here rewinds the barrier
   // counter so the next launch (whatever its grid size) starts from zero.
   if (tid == 0 && atomicAdd(a.bar + 1, 1ull) == (unsigned long long)(G - 1)) {
@@ -851,6 +856,7 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   a.gscores = L->gscores;
   a.keep = L->sel_keep;
   a.flags = L->sel_flags;
+  a.wait_limit = L->wait_limit > 0 ? L->wait_limit : kWaitLimitCycles;
   if (!g.smem_scores && L->gscores == nullptr) return cudaErrorInvalidValue;
   if (g.grid > L->sm_count || g.grid > kSelMaxGrid) return cudaErrorInvalidValue;
   void* args[] = {&a};

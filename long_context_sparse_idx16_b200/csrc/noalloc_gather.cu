@@ -81,9 +81,23 @@ __global__ void __launch_bounds__(kThreads) noalloc_gather_kernel(Args a) {
   __syncthreads();
   const int total = min(s_base[a.P], kScratchItems);  // the host bounds it by kScratchItems
 
+  // a problem with an empty list has no work item: its output is defined as zeros
+  for (int p = blockIdx.x; p < a.P; p += gridDim.x)
+    if (s_base[p + 1] == s_base[p] && tid < kD) a.out[(int64_t)p * kD + tid] = 0.f;
+
   for (int it = blockIdx.x; it < total; it += gridDim.x) {
+    // the item's problem: the last p with s_base[p] <= it (then s_base[p + 1] > it; problems
+    // with empty lists share their base with the next problem and are skipped over)
     int p = 0;
-    while (p + 1 < a.P && s_base[p + 1] <= it) ++p;
+    for (int lo = 0, hi = a.P - 1; lo <= hi;) {
+      const int mid = (lo + hi) >> 1;
+      if (s_base[mid] <= it) {
+        p = mid;
+        lo = mid + 1;
+      } else {
+        hi = mid - 1;
+      }
+    }
     const int chunk = it - s_base[p];
     const int n_items = s_base[p + 1] - s_base[p];
     const int64_t K = min((int64_t)max(a.cnt[p], 0), a.max_count);
@@ -210,7 +224,9 @@ __global__ void __launch_bounds__(kThreads) noalloc_gather_kernel(Args a) {
   }
 }
 
-// Device address of the scratch array, looked up once per device.
+// Device address of the scratch array, looked up once per device and kept for the life of the
+// process: the cache assumes the device's primary context is never torn down (no
+// cudaDeviceReset between calls).
 std::mutex g_addr_mu;
 float* g_addr[kMaxDevices] = {};
 
@@ -231,6 +247,10 @@ extern "C" rtp_status rtp_gather_attn_noalloc(const void* k, const void* v, cons
     return fail(nullptr, RTP_EINVAL, "rtp_gather_attn_noalloc: need 1 <= P <= 2048");
   if (max_count < 1 || idx_stride < max_count || kv_stride < kD || !(sm_scale > 0.f))
     return fail(nullptr, RTP_EINVAL, "rtp_gather_attn_noalloc: bad max_count, strides or scale");
+  // K/V rows and queries are read as 16-byte vectors
+  if ((((uintptr_t)k | (uintptr_t)v | (uintptr_t)q) & 15u) != 0u || kv_stride % 8 != 0)
+    return fail(nullptr, RTP_EINVAL,
+                "rtp_gather_attn_noalloc: k, v and q must be 16-byte aligned and kv_stride a multiple of 8");
   const int64_t worst = (int64_t)P * ((max_count + kChunk - 1) / kChunk);
   if (worst > kScratchItems)
     return fail(nullptr, RTP_EINVAL,

@@ -63,6 +63,10 @@ struct RetArgs {
   float* sel_mass;            // [B][C][Hr] or nullptr
   uint32_t* bitmap;           // [B][C][Hr][bitmap_words] or nullptr
   int64_t bitmap_words;
+  const int32_t* rows;        // [n_rows] chunk rows whose positions are listed, or nullptr
+  int n_rows;
+  int32_t* row_sel;           // [B][n_rows][Hr][row_sel_cap]
+  int64_t row_sel_cap;
   uint32_t* err;
 };
 
@@ -585,6 +589,7 @@ struct SmemAttn {
   uint32_t cmc[2][kRows][2];              // per-row bits of the two issued chunks
   int32_t jlc[2][64];                     // their key positions
   unsigned long long wun[2][4];           // per-warp union of a tile's row masks (two tiles)
+  int32_t lslot[kRows];                   // row -> its entry in the listed rows (-1: not listed)
 };
 
 __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
@@ -631,6 +636,22 @@ __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
   fa_init(A);
 
   for (int i = tid; i < kRows * 4; i += kThreads) (&S.cm[0][0])[i] = 0u;
+  for (int i = tid; i < kRows; i += kThreads) S.lslot[i] = -1;
+  __syncthreads();
+  for (int i = tid; i < a.n_rows; i += kThreads) {
+    const int r = a.rows[i] - i0;
+    if (r >= 0 && r < nrows) S.lslot[r] = i;
+  }
+  __syncthreads();
+  int32_t* lrow[2] = {nullptr, nullptr};  // this owner's listed rows: where their positions go
+  if (a.row_sel && owner) {
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+      const int r = sl ? x.rb : x.ra;
+      const int li = (sl ? x.pb : x.pa) >= 0 ? S.lslot[r] : -1;
+      if (li >= 0) lrow[sl] = a.row_sel + (((int64_t)b * a.n_rows + li) * a.Hr + hr) * a.row_sel_cap;
+    }
+  }
   int fill = 0;
   int nsel[2] = {0, 0};
 
@@ -730,6 +751,15 @@ __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
     if (owner) {
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
+        if (lrow[sl]) {  // a listed row: its positions, ascending (tiles come in order)
+          unsigned long long v = mk[sl];
+          int n = nsel[sl];
+          while (v && n < a.row_sel_cap) {
+            const int p = __ffsll((long long)v) - 1;
+            v &= v - 1;
+            lrow[sl][n++] = (int32_t)(t * kIdxKeys + p);
+          }
+        }
         nsel[sl] += __popcll(mk[sl]);
         if (brow[sl]) {
           const int64_t w = 2 * t;
@@ -791,6 +821,10 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
   a.sel_mass = stats ? stats->sel_mass : nullptr;
   a.bitmap = stats ? stats->sel_bitmap : nullptr;
   a.bitmap_words = stats ? stats->bitmap_words : 0;
+  a.rows = stats ? stats->rows : nullptr;
+  a.n_rows = (stats && stats->rows) ? stats->n_rows : 0;
+  a.row_sel = (stats && stats->rows) ? stats->row_sel : nullptr;
+  a.row_sel_cap = (stats && stats->rows) ? stats->row_sel_cap : 0;
   a.err = L->err;
   dim3 grid((C + kRows - 1) / kRows, L->Hr, L->B);
   cudaError_t e;

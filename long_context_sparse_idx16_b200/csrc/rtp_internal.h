@@ -88,6 +88,7 @@ struct rtp_layer {
   int64_t spart_elems = 0;
   uint32_t* sticket = nullptr;   // [B*Hkv]
   uint32_t* err = nullptr;       // device error word
+  long long wait_limit = 0;      // decode grid-barrier wait limit in cycles (0: the default, ~1 s)
 
   // per-kernel event timing (rtp_profile_enable)
   bool prof_on = false;

@@ -380,6 +380,9 @@ rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out,
     return fail(L, RTP_EINVAL, "rtp_prefill_chunk: need 1 <= C <= min(len, max_chunk)");
   if (stats && stats->sel_bitmap && stats->bitmap_words < 1)
     return fail(L, RTP_EINVAL, "rtp_prefill_chunk: sel_bitmap needs bitmap_words >= 1");
+  if (stats && stats->rows &&
+      (stats->n_rows < 1 || !stats->row_sel || stats->row_sel_cap < 1 || !stats->sel_count))
+    return fail(L, RTP_EINVAL, "rtp_prefill_chunk: rows needs n_rows >= 1, row_sel, row_sel_cap >= 1 and sel_count");
   cudaError_t e;
   {
     ProfScope ps(L, "q_prep", stream);
@@ -419,6 +422,13 @@ rtp_status rtp_set_top_p(rtp_layer* L, float top_p) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_set_top_p: layer is NULL");
   if (!(top_p > 0.f && top_p <= 1.f)) return fail(L, RTP_EINVAL, "rtp_set_top_p: top_p must be in (0, 1]");
   L->top_p = top_p;
+  return RTP_OK;
+}
+
+rtp_status rtp_set_wait_limit(rtp_layer* L, int64_t cycles) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_set_wait_limit: layer is NULL");
+  if (cycles < 0) return fail(L, RTP_EINVAL, "rtp_set_wait_limit: cycles must be >= 0");
+  L->wait_limit = (long long)cycles;
   return RTP_OK;
 }
 

@@ -119,3 +119,28 @@ def test_create_rejects_bad_head_maps_on_host(lib):
     assert lib.rtp_create(C.byref(cfg), C.byref(h)) == rtp.RTP_EINVAL
     assert h.value is None
     assert "2048" in rtp.rtp_last_error(None)
+
+
+def test_noalloc_gather_rejects_misaligned_arguments_on_host(lib):
+    """The allocation-free attention reads K/V rows and queries as 16-byte vectors: a stride that
+    is not a multiple of 8 fp16 elements, or a K, V or q pointer off a 16-byte boundary, is
+    refused before any CUDA call (the pointers here are never dereferenced)."""
+    base = 1 << 20
+    args = dict(k=base, v=base + 4096, kv_block=None, kv_stride=128, q=base + 8192, idx=base + 12288,
+                idx_stride=16, cnt=base + 16384, P=1, max_count=16, sm_scale=0.088, out=base + 20480,
+                stream=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.rtp_gather_attn_noalloc(a["k"], a["v"], a["kv_block"], a["kv_stride"], a["q"], a["idx"],
+                                           a["idx_stride"], a["cnt"], a["P"], a["max_count"], a["sm_scale"],
+                                           a["out"], a["stream"])
+
+    assert call(kv_stride=130) == rtp.RTP_EINVAL
+    assert "16-byte" in rtp.rtp_last_error(None)
+    assert call(kv_stride=1028) == rtp.RTP_EINVAL
+    assert call(k=base + 8) == rtp.RTP_EINVAL
+    assert call(v=base + 4100) == rtp.RTP_EINVAL
+    assert call(q=base + 8196) == rtp.RTP_EINVAL
+    assert call(P=0) == rtp.RTP_EINVAL
+    assert call(idx_stride=8) == rtp.RTP_EINVAL

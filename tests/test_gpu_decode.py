@@ -99,6 +99,13 @@ def test_decode_1m_full_size(p):
     res = run_decode(x, top_p=p, heads=heads, layer=layer)
     counts = [v[0] for v in res["summary"].values()]
     assert max(counts) >= 100 and min(counts) <= 64  # budgets span orders of magnitude
+    span = _state.setdefault("decode_1m_counts", {})
+    span[p] = counts
+    if len(span) == 3:
+        # over the p sweep the set sizes span about 10 to 10^4 (needle-aimed queries keep a
+        # dozen keys, the Gaussian query about eight thousand at p = 0.95)
+        allc = [c for v in span.values() for c in v]
+        assert min(allc) <= 16 and max(allc) >= 8000, (min(allc), max(allc))
 
 
 def test_decode_128k_full_size():

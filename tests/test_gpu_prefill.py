@@ -88,20 +88,46 @@ def test_prefill_deterministic():
     assert np.array_equal(a, b)
 
 
+def _spread_rows(C: int, n: int, seed: int, tile: int = 64) -> np.ndarray:
+    """n distinct chunk rows: the first and last two, pairs across row-tile boundaries spread
+    over the chunk, and seeded random rows (even and odd rows alike)."""
+    rows = {0, 1, C - 2, C - 1}
+    n_tiles = (C + tile - 1) // tile
+    for k in np.linspace(1, n_tiles - 1, min(n_tiles - 1, n // 4)).astype(np.int64):
+        rows.update((int(k) * tile - 1, int(k) * tile))
+    rng = np.random.default_rng(seed)
+    while len(rows) < n:
+        rows.add(int(rng.integers(0, C)))
+    return np.array(sorted(r for r in rows if 0 <= r < C), dtype=np.int64)
+
+
+def test_prefill_row_lists_match_bitmap():
+    # the row-subset position lists give the same sets as the full bitmap (ragged tail included)
+    x = small(prefix=900, chunk=260, window=128)
+    rows = [0, 1, 63, 64, 65, 127, 128, 200, 255, 256, 259]
+    run_prefill(x, rows=rows, sets="rows")
+    run_prefill(x, rows=rows, sets="bitmap")
+
+
 @pytest.mark.slow
-def test_prefill_32k_full_sampled_rows():
-    # the full 32K chunk (B=1, C=32768 from an empty cache); rows sampled across the chunk
+def test_prefill_32k_full_every_retrieval_row():
+    # the full 32K chunk (B=1, C=32768 from an empty cache): every row of every retrieval head
+    # (sets through the bitmap, outputs), and 512 rows of every local head
     x = synth.generate(synth.spec("prefill_32k"))
-    rows = [0, 1, 63, 64, 4095, 4096, 8191, 8192, 16383, 20000, 32700, 32767]
-    run_prefill(x, rows=rows, heads=[0, 1, 7, 13, 19, 26, 31])
+    run_prefill(x, rows=None, local_rows=_spread_rows(x.spec.chunk, 512, seed=5), sets="bitmap")
 
 
 @pytest.mark.slow
 def test_prefill_1m_full_sampled_rows():
-    # a 16384-row chunk on a 1032192-key prefix; counts and outputs on sampled rows
+    # a 16384-row chunk on a 1032192-key prefix: 256 rows of each retrieval head with their sets
+    # (row lists), both query types, tile-boundary pairs and the first and last rows; 64 rows of
+    # each local head
     x = synth.generate(synth.spec("prefill_1m"))
-    rows = [0, 5, 8191, 8192, 16383]
-    run_prefill(x, rows=rows, heads=[0, 2, 13, 26], bitmap=False)
+    C = x.spec.chunk
+    rows = _spread_rows(C, 256, seed=6)
+    assert len(rows) >= 256 and {0, C - 1} <= set(rows.tolist())
+    assert (rows % 2 == 0).any() and (rows % 2 == 1).any()  # needle-aimed and N(0, 1) queries
+    run_prefill(x, rows=rows, local_rows=_spread_rows(C, 64, seed=7), sets="rows", row_block=64)
 
 
 def test_prefill_bitmap_needs_words():
@@ -117,7 +143,7 @@ def test_prefill_bitmap_needs_words():
     q = torch_bf16(x.q)
     out = torch.empty((s.batch, s.chunk, s.n_q_heads, 128), dtype=torch.float32, device="cuda")
     bm = torch.zeros(16, dtype=torch.int32, device="cuda")
-    st = rtp_prefill_stats(None, None, bm.data_ptr(), 0)
+    st = rtp_prefill_stats(None, None, bm.data_ptr(), 0, None, 0, None, 0)
     with pytest.raises(RTPError):
         rtp_prefill_chunk(layer.handle, q.data_ptr(), s.chunk, out.data_ptr(), st, 0)
     assert layer.check() == 0
