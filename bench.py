@@ -97,31 +97,45 @@ def _prefill_traffic(kernel: str, workload: str):
     return traffic
 
 
-def _prefill_roofline(kern: dict, flops: dict, exps: int, sm_mhz, n_sm: int, tensor_peak: float,
-                      tensor_peak_kind: str) -> dict:
-    """Roofline object of the prefill chunk's dominant kernel (the one with the longest time).
+def _prefill_rooflines(kern: dict, flops: dict, exps: int, exp_peak: dict, sm_mhz, tensor_peak: float,
+                       tensor_peak_kind: str) -> dict:
+    """Roofline objects of the prefill chunk's kernels.
 
-    The selection (prefill_select) evaluates one exponential per causal (row, key) pair and
-    is bound by the exp (MUFU) and integer pipes, so it is reported as "alu" against
-    MUFU_EX2_PER_CLK_SM x SMs x clock.  The attention kernels are reported against the dense
-    16-bit tensor peak with their algorithmic flops (4 D per attended pair)."""
-    cands = [k for k in ("prefill_select", "prefill_attn", "prefill_local") if kern.get(k, {}).get("ms_per_launch", 0) > 0]
-    dom = max(cands, key=lambda k: kern[k]["ms_per_launch"])
-    ms = kern[dom]["ms_per_launch"]
-    if dom == "prefill_select":
-        mhz = float(sm_mhz) if sm_mhz else 1965.0
-        peak = MUFU_EX2_PER_CLK_SM * n_sm * mhz * 1e6 / 1e9
+    prefill_select evaluates one exponential per causal (row, key) pair and is bound by the
+    exp (MUFU) and integer pipes: "alu" against the exponential rate measured on this GPU by the
+    ex2 probe (scaled to the SM clock sampled during the prefill).  prefill_attn and
+    prefill_local are "tensor" against the dense 16-bit peak with algorithmic flops (4 D per
+    attended pair).  "index_plus_sparse_attention" puts the retrieval heads' two kernels
+    together against the tensor peak: 2 r flops per causal (row, key) index score plus the
+    attention flops, over the two kernels' summed time."""
+    out = {}
+    if kern.get("prefill_select", {}).get("ms_per_launch", 0) > 0:
+        ms = kern["prefill_select"]["ms_per_launch"]
+        mhz = float(sm_mhz) if sm_mhz else float(exp_peak["sm_mhz"])
+        peak = exp_peak["per_clk_per_sm"] * exp_peak["sms"] * mhz * 1e6 / 1e9
         achieved = exps / (ms * 1e-3) / 1e9
-        return {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": peak,
-                "peak_kind": f"derived: {MUFU_EX2_PER_CLK_SM} ex2 per clock per SM x {n_sm} SMs x "
-                             f"{mhz:.0f} MHz ({'sampled' if sm_mhz else 'nominal max'} SM clock)",
-                "unit": "Gexp/s", "frac": achieved / peak, "traffic": None,
-                "exps_per_launch": int(exps), "ms_per_launch": ms}
-    f = flops["local_attention"] if dom == "prefill_local" else flops["retrieval_attention"]
-    achieved = f / (ms * 1e-3) / 1e12
-    return {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": tensor_peak,
-            "peak_kind": tensor_peak_kind, "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": None,
-            "flops_per_launch": int(f), "ms_per_launch": ms}
+        out["prefill_select"] = {
+            "bound": "alu", "kernel": "prefill_select", "achieved": achieved, "peak": peak,
+            "peak_kind": (f"measured: ex2 probe {exp_peak['per_clk_per_sm']:.2f} per clock per SM x "
+                          f"{exp_peak['sms']} SMs x {mhz:.0f} MHz ({'sampled' if sm_mhz else 'probe'} SM clock)"),
+            "unit": "Gexp/s", "frac": achieved / peak, "traffic": None, "exps_per_launch": int(exps),
+            "ms_per_launch": ms}
+    for k, f in (("prefill_attn", flops["retrieval_attention"]), ("prefill_local", flops["local_attention"])):
+        if kern.get(k, {}).get("ms_per_launch", 0) > 0:
+            ms = kern[k]["ms_per_launch"]
+            a = f / (ms * 1e-3) / 1e12
+            out[k] = {"bound": "tensor", "kernel": k, "achieved": a, "peak": tensor_peak,
+                      "peak_kind": tensor_peak_kind, "unit": "TFLOP/s", "frac": a / tensor_peak, "traffic": None,
+                      "flops_per_launch": int(f), "ms_per_launch": ms}
+    if "prefill_select" in out and "prefill_attn" in out:
+        ms = out["prefill_select"]["ms_per_launch"] + out["prefill_attn"]["ms_per_launch"]
+        f = flops["index_scores_flops"] + flops["retrieval_attention"]
+        a = f / (ms * 1e-3) / 1e12
+        out["index_plus_sparse_attention"] = {
+            "bound": "tensor", "kernels": ["prefill_select", "prefill_attn"], "achieved": a, "peak": tensor_peak,
+            "peak_kind": tensor_peak_kind, "unit": "TFLOP/s", "frac": a / tensor_peak, "flops_per_launch": int(f),
+            "ms_per_launch": ms}
+    return out
 
 
 def _profile_traffic(kernel_src: str):
@@ -144,18 +158,62 @@ def _profile_traffic(kernel_src: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+    """SM clock and throttle-reason sampling while a timed region runs (read-only).
+
+    NVML (the library nvidia-smi reads) is polled from a thread about every half millisecond,
+    so even a region of a few milliseconds gets samples; where NVML cannot be loaded,
+    nvidia-smi is run in the background instead (50 ms period)."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits, in the order of the names below
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
     def __init__(self, gpu: int):
         self.gpu = gpu
         self.proc = None
+        self.thread = None
+        self.rows = []
         self.path = os.path.join("/tmp", f"rtp_clocks_{os.getpid()}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
     def start(self):
+        import threading
+
+        try:
+            import pynvml
+
+            h = self._nvml_handle()
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._stop = threading.Event()
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((float(sm), float(smax), int(rs)))
+                    except Exception:
+                        pass
+                    time.sleep(0.0005)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
@@ -164,6 +222,16 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+            rows = self.rows
+            if not rows:
+                return None
+            sm = sorted(r[0] for r in rows)
+            reasons = sorted({n for r in rows for n, bit in self.REASONS if r[2] & bit})
+            return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                    "samples": len(rows), "source": "nvml"}
         if self.proc is None:
             return None
         time.sleep(0.06)
@@ -182,10 +250,10 @@ class ClockSampler:
             return None
         sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
         smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _ in self.REASONS]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi"}
 
 
 def _dist():
@@ -388,16 +456,17 @@ def _generate(args):
     return synth.generate(_spec(args))
 
 
-def _spec(args):
+def _spec(args, name=None):
     import synth
 
+    name = name or args.workload
     ov = {}
-    if args.batch:
-        base = synth.spec(args.workload)
+    if args.batch and name == args.workload:
+        base = synth.spec(name)
         ov["batch"] = args.batch
         if base.needles and len(base.needles) > 1:
             ov["needles"] = tuple(base.needles[i % len(base.needles)] for i in range(args.batch))
-    return synth.spec(args.workload, **ov)
+    return synth.spec(name, **ov)
 
 
 def _config(s, n_gpus):
@@ -410,99 +479,98 @@ def _config(s, n_gpus):
                 s.batch * len(s.retrieval_heads) * s.n_total * s.index_dim * 4 / 1e6)}
 
 
-def run_gpu(args):
+def _bf16(a):
     import numpy as np
     import torch
 
-    import synth
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+
+def measure_exp_rate(dev) -> dict:
+    """The exponential (MUFU ex2) issue rate of this GPU, from the library's ex2 probe timed
+    with CUDA events while nvidia-smi samples the SM clock: the peak the prefill selection's
+    roofline divides by."""
+    import torch
+
+    from long_context_sparse_idx16_b200 import rtp_probe_ex2
+
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks, iters = sms * 8, 4096
+    buf = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(3):
+        rtp_probe_ex2(blocks, iters, buf.data_ptr(), stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    best = None
+    n = 0
+    t_end = time.perf_counter() + 0.3
+    while time.perf_counter() < t_end:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        n = rtp_probe_ex2(blocks, iters, buf.data_ptr(), stream)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        best = ms if best is None else min(best, ms)
+    clk = clocks.stop()
+    mhz = (clk or {}).get("sm_mhz") or 1965.0
+    rate = n / (best * 1e-3)
+    return {"gexp_s": rate / 1e9, "per_clk_per_sm": rate / (sms * mhz * 1e6), "sms": sms, "sm_mhz": mhz,
+            "clock_source": "sampled" if clk and clk.get("sm_mhz") else "nominal max",
+            "exps_per_launch": int(n), "ms_per_launch": best}
+
+
+def _timed(step, steps: int, world: int, dev):
+    """Device time (ms, max over ranks) of exactly `steps` calls of step(), bracketed by a
+    barrier and a device synchronisation on both sides."""
+    import torch
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    return _max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+
+def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=None, cpu: bool = True):
+    """Decode lines of workload s, one per p in top_ps (default: the workload's p), all on one
+    layer.  A step appends the B new tokens and decodes their B queries; before every step the
+    length is rolled back by one, so every step sees exactly N keys."""
+    import numpy as np
+    import torch
+
     from long_context_sparse_idx16_b200 import Layer
 
-    world, rank, local = _dist()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    s = _spec(args)
-    x = synth.generate(s)
     N, B = s.n_total, s.batch
-
-    def bf16(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
-
     layer = Layer.from_spec(s, x, max_seq=N, max_chunk=1)
     for t0 in range(0, N - 1, 1 << 16):
         t1 = min(N - 1, t0 + (1 << 16))
-        layer.append_kv(bf16(x.k[:, t0:t1]).to(dev), bf16(x.v[:, t0:t1]).to(dev))
-    k_tok = bf16(x.k[:, N - 1:N]).to(dev).contiguous()
-    v_tok = bf16(x.v[:, N - 1:N]).to(dev).contiguous()
-    q = bf16(x.q[:, 0]).to(dev).contiguous()
+        layer.append_kv(_bf16(x.k[:, t0:t1]).to(dev), _bf16(x.v[:, t0:t1]).to(dev))
+    k_tok = _bf16(x.k[:, N - 1:N]).to(dev).contiguous()
+    v_tok = _bf16(x.v[:, N - 1:N]).to(dev).contiguous()
+    q = _bf16(x.q[:, 0]).to(dev).contiguous()
     out = torch.empty((B, s.n_q_heads, 128), dtype=torch.float32, device=dev)
+    q_h = q.cpu().pin_memory()
+    k_h = k_tok.cpu().pin_memory()
+    v_h = v_tok.cpu().pin_memory()
+    o_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(k_tok), torch.empty_like(v_tok)
 
     def step():
         layer.truncate(N - 1)
         layer.append_kv(k_tok, v_tok)
         layer.decode(q, out)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert layer.check() == 0
-    _, st = layer.decode(q, out, stats=True)
-    counts = st[0].cpu().numpy().ravel()
-
-    # ---- device-timed region (no per-kernel events inside it)
-    clocks = ClockSampler(local)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1)
-    assert layer.check() == 0
-    ms = _max_over_ranks(ms, world, dev)
-
-    # ---- the same steps again with a CUDA event pair around every kernel launch (on its
-    # launch stream): per-kernel device time for the roofline and the launch count
-    layer.profile(True)
-    layer.profile_read()  # drop anything recorded before
-    for _ in range(args.steps):
-        step()
-    torch.cuda.synchronize()
-    sel_ms, sel_n = layer.profile_read("decode_select")
-    kern = {"decode_select": {"us_per_launch": sel_ms * 1e3 / max(sel_n, 1), "launches": sel_n}}
-    other_n = 0
-    for k in ("append_kv", "q_prep", "decode_gather", "decode_swa", "swa_merge", "dense_fill"):
-        kms, kn = layer.profile_read(k)
-        if kn:
-            kern[k] = {"us_per_launch": kms * 1e3 / kn, "launches": kn}
-        other_n += kn
-    rest_ms, rest_n = layer.profile_read(None)
-    layer.profile(False)
-    all_n = sel_n + other_n + rest_n
-
-    # ---- end-to-end through the C ABI with host buffers
-    q_h = torch.empty_like(q, device="cpu").pin_memory()
-    k_h = torch.empty_like(k_tok, device="cpu").pin_memory()
-    v_h = torch.empty_like(v_tok, device="cpu").pin_memory()
-    o_h = torch.empty_like(out, device="cpu").pin_memory()
-    q_h.copy_(q.cpu())
-    k_h.copy_(k_tok.cpu())
-    v_h.copy_(v_tok.cpu())
-    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(k_tok), torch.empty_like(v_tok)
-
-    def e2e_step():
+    def e2e_step():  # the step's inputs from pinned host memory, the output back to the host
         q_d.copy_(q_h, non_blocking=True)
         k_d.copy_(k_h, non_blocking=True)
         v_d.copy_(v_h, non_blocking=True)
@@ -511,59 +579,77 @@ def run_gpu(args):
         layer.decode(q_d, out)
         o_h.copy_(out, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record()
-    for _ in range(args.steps):
-        e2e_step()
-    f1.record()
-    torch.cuda.synchronize()
-    e2e_ms = _max_over_ranks(f0.elapsed_time(f1), world, dev)
-    assert np.isfinite(o_h.numpy()).all()
-
-    tokens = B * args.steps * world
-    value = ms * 1e3 / tokens  # us per token: all ranks' tokens over the max rank time
-    e2e = e2e_ms * 1e3 / tokens
     peak, peak_kind = _peaks()
     P = B * len(s.retrieval_heads)
     sel_bytes = P * N * s.index_dim * 4  # fp32 index keys streamed per launch
-    sel_us = sel_ms * 1e3 / max(sel_n, 1)
-    achieved = sel_bytes / (sel_us * 1e-6) / 1e9
     traffic = _profile_traffic(os.path.join(ROOT, "long_context_sparse_idx16_b200", "csrc", "decode_select.cu"))
-    # whole-step algorithmic bytes: index keys + window/sink K/V rows + selected K/V rows
-    n_local_kv = s.n_kv_heads  # every KV head serves local heads in this layout
-    win_keys = min(N, s.window + s.n_sink)
-    step_bytes = sel_bytes + B * n_local_kv * win_keys * 512 + int(counts.sum()) * 512
-    line = {
-        "metric": METRIC, "value": value, "unit": "us/token", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(s, world),
-        "roofline": {"bound": "hbm", "kernel": "decode_select (fused index stream + exact top-p)",
-                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "bytes_per_launch": sel_bytes,
-                     "us_per_launch": sel_us},
-        "step_roofline": {"bytes_per_step": step_bytes, "roofline_us_per_step": step_bytes / (peak * 1e9) * 1e6,
-                          "frac": step_bytes / (peak * 1e9) / (ms / args.steps * 1e-3)},
-        "e2e": {"value": e2e, "unit": "us/token", "h2d_bytes_per_step": int(q.numel() * 2 + k_tok.numel() * 2 * 2),
-                "d2h_bytes_per_step": int(out.numel() * 4)},
-        "kernels": kern,
-        "gpu_launches": int(all_n),  # kernels of this library per timed region (one pass of --steps steps)
-        "selected_tokens": {"min": int(counts.min()), "median": float(np.median(counts)), "max": int(counts.max())},
-        "clocks": clk,
-    }
-    if rank == 0 and not args.no_cpu_baseline:
-        v, cores, desc = cpu_oracle_sample(x)
-        line["cpu_baseline"] = {"value": v, "unit": "us/token", "cores": cores, "kind": "oracle", "sample": desc}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    lines = []
+    for p in (top_ps or [s.top_p]):
+        layer.set_top_p(p)
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        assert layer.check() == 0
+        _, st = layer.decode(q, out, stats=True)
+        counts = st[0].cpu().numpy().ravel()
+        clocks = ClockSampler(dev.index or 0)
+        clocks.start()  # sampled during the timed region
+        ms = _timed(step, steps, world, dev)
+        clk = clocks.stop()
+        assert layer.check() == 0
+        # the same steps with a CUDA event pair around every kernel launch (on its launch
+        # stream): per-kernel device time for the roofline and the launch count
+        layer.profile(True)
+        layer.profile_read()  # drop anything recorded before
+        for _ in range(steps):
+            step()
+        torch.cuda.synchronize()
+        sel_ms, sel_n = layer.profile_read("decode_select")
+        kern = {"decode_select": {"us_per_launch": sel_ms * 1e3 / max(sel_n, 1), "launches": sel_n}}
+        other_n = 0
+        for k in ("append_kv", "q_prep", "decode_gather", "decode_swa", "swa_merge", "dense_fill"):
+            kms, kn = layer.profile_read(k)
+            if kn:
+                kern[k] = {"us_per_launch": kms * 1e3 / kn, "launches": kn}
+            other_n += kn
+        _, rest_n = layer.profile_read(None)
+        layer.profile(False)
+        for _ in range(warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        e2e_ms = _timed(e2e_step, steps, world, dev)
+        assert np.isfinite(o_h.numpy()).all()
+        tokens = B * steps * world
+        sel_us = sel_ms * 1e3 / max(sel_n, 1)
+        achieved = sel_bytes / (sel_us * 1e-6) / 1e9
+        win_keys = min(N, s.window + s.n_sink)
+        # whole-step algorithmic bytes: index keys + window/sink K/V rows + selected K/V rows
+        step_bytes = sel_bytes + B * s.n_kv_heads * win_keys * 512 + int(counts.sum()) * 512
+        lines.append({
+            "value": ms * 1e3 / tokens, "unit": "us/token", "top_p": p, "steps": steps, "warmup": warmup,
+            "ms_per_step": ms / steps, "config": _config(s, world),
+            "roofline": {"bound": "hbm", "kernel": "decode_select (fused index stream + exact top-p)",
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic if s.name == "decode_128k" else None,
+                         "bytes_per_launch": sel_bytes, "us_per_launch": sel_us},
+            "step_roofline": {"bytes_per_step": step_bytes, "roofline_us_per_step": step_bytes / (peak * 1e9) * 1e6,
+                              "frac": step_bytes / (peak * 1e9) / (ms / steps * 1e-3)},
+            "e2e": {"value": e2e_ms * 1e3 / tokens, "unit": "us/token",
+                    "h2d_bytes_per_step": int(q.numel() * 2 + k_tok.numel() * 2 * 2),
+                    "d2h_bytes_per_step": int(out.numel() * 4)},
+            "kernels": kern,
+            "gpu_launches": int(sel_n + other_n + rest_n),
+            "selected_tokens": {"min": int(counts.min()), "median": float(np.median(counts)),
+                                "max": int(counts.max())},
+            "clocks": clk,
+        })
     layer.close()
-    if world > 1:
-        torch.distributed.destroy_process_group()
-    return 0
+    if cpu:
+        v, cores, desc = cpu_oracle_sample(x)
+        for ln in lines:
+            ln["cpu_baseline"] = {"value": v, "unit": "us/token", "cores": cores, "kind": "oracle",
+                                  "sample": desc + f" at p={s.top_p}"}
+    return lines
 
 
 def _local_pairs(s) -> int:
@@ -576,39 +662,23 @@ def _local_pairs(s) -> int:
     return int((sinks + np.maximum(0, pos - w0 + 1)).sum())
 
 
-def run_prefill_gpu(args):
-    """A step is one chunked-prefill call of the workload: the chunk's K/V are appended
-    (RoPE + index keys) after the length is rolled back to the prefix, then every row of the
-    chunk runs its selection / window and attention."""
+def measure_prefill(s, x, steps: int, warmup: int, world: int, dev, exp_peak: dict, *, cpu: bool = True):
+    """A step is one chunked-prefill call of the workload: the chunk's K/V are appended (RoPE +
+    index keys) after the length is rolled back to the prefix, then every row of the chunk runs
+    its selection / window and attention."""
     import numpy as np
     import torch
 
-    import synth
     from long_context_sparse_idx16_b200 import Layer
 
-    world, rank, local = _dist()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    s = _spec(args)
-    x = synth.generate(s)
     N, B, P, C = s.n_total, s.batch, s.prefix, s.chunk
-
-    def bf16(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
-
     layer = Layer.from_spec(s, x, max_seq=N, max_chunk=C)
     for t0 in range(0, P, 1 << 16):
         t1 = min(P, t0 + (1 << 16))
-        layer.append_kv(bf16(x.k[:, t0:t1]).to(dev), bf16(x.v[:, t0:t1]).to(dev))
-    k_c = bf16(x.k[:, P:N]).to(dev).contiguous()
-    v_c = bf16(x.v[:, P:N]).to(dev).contiguous()
-    q = bf16(x.q).to(dev).contiguous()
+        layer.append_kv(_bf16(x.k[:, t0:t1]).to(dev), _bf16(x.v[:, t0:t1]).to(dev))
+    k_c = _bf16(x.k[:, P:N]).to(dev).contiguous()
+    v_c = _bf16(x.v[:, P:N]).to(dev).contiguous()
+    q = _bf16(x.q).to(dev).contiguous()
     out = torch.empty((B, C, s.n_q_heads, 128), dtype=torch.float32, device=dev)
 
     def step():
@@ -616,7 +686,7 @@ def run_prefill_gpu(args):
         layer.append_kv(k_c, v_c)
         layer.prefill_chunk(q, out)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     assert layer.check() == 0
@@ -624,32 +694,20 @@ def run_prefill_gpu(args):
     counts = st[0].cpu().numpy()
     assert layer.check() == 0
 
-    clocks = ClockSampler(local)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()  # sampled during the timed region
+    ms = _timed(step, steps, world, dev)
     clk = clocks.stop()
-    ms = _max_over_ranks(e0.elapsed_time(e1), world, dev)
     assert layer.check() == 0
-
     layer.profile(True)
     layer.profile_read()
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     torch.cuda.synchronize()
     per = {}
     for k in ("prefill_select", "prefill_attn", "prefill_local", "append_kv", "q_prep"):
         per[k] = layer.profile_read(k)
-    rest_ms, rest_n = layer.profile_read(None)
+    _, rest_n = layer.profile_read(None)
     layer.profile(False)
     all_n = sum(n for _, n in per.values()) + rest_n
 
@@ -669,48 +727,34 @@ def run_prefill_gpu(args):
         layer.prefill_chunk(q_d, out)
         o_h.copy_(out, non_blocking=True)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         e2e_step()
     torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record()
-    for _ in range(args.steps):
-        e2e_step()
-    f1.record()
-    torch.cuda.synchronize()
-    e2e_ms = _max_over_ranks(f0.elapsed_time(f1), world, dev)
+    e2e_ms = _timed(e2e_step, steps, world, dev)
+    layer.close()
 
-    chunks = B * args.steps * world
-    value = ms / (args.steps)  # ms per chunk call (B sequences each) on one GPU
     peak, peak_kind = _tensor_peak()
     Hr = len(s.retrieval_heads)
     Hl = s.n_q_heads - Hr
-    local_flops = 4 * s.head_dim * _local_pairs(s) * Hl * B
-    ret_flops = 4 * s.head_dim * int(counts.sum())
-    kern = {}
-    for k, (kms, kn) in per.items():
-        kern[k] = {"ms_per_launch": kms / max(kn, 1), "launches": kn}
-    flops = {"local_attention": local_flops, "retrieval_attention": ret_flops,
-             "index_scores": Hr * B * (C * P + C * (C + 1) // 2)}
-    roof = _prefill_roofline(kern, flops, flops["index_scores"], (clk or {}).get("sm_mhz"),
-                             torch.cuda.get_device_properties(dev).multi_processor_count, peak, peak_kind)
-    roof["traffic"] = _prefill_traffic(roof["kernel"], s.name)
-    # the tensor-core kernels, each against the tensor peak
-    tensor = {}
-    for k, f in (("prefill_local", local_flops), ("prefill_attn", ret_flops)):
-        if k in kern and kern[k]["ms_per_launch"] > 0:
-            a_ = f / (kern[k]["ms_per_launch"] * 1e-3) / 1e12
-            tensor[k] = {"achieved_tflops": a_, "frac": a_ / peak, "flops_per_launch": int(f)}
+    pairs = Hr * B * (C * P + C * (C + 1) // 2)  # causal (row, key) index scores, all retrieval heads
+    flops = {"local_attention": 4 * s.head_dim * _local_pairs(s) * Hl * B,
+             "retrieval_attention": 4 * s.head_dim * int(counts.sum()),
+             "index_scores": pairs, "index_scores_flops": 2 * s.index_dim * pairs}
+    kern = {k: {"ms_per_launch": kms / max(kn, 1), "launches": kn} for k, (kms, kn) in per.items()}
+    roofs = _prefill_rooflines(kern, flops, pairs, exp_peak, (clk or {}).get("sm_mhz"), peak, peak_kind)
+    if "prefill_select" in roofs:
+        roofs["prefill_select"]["traffic"] = _prefill_traffic("prefill_select", s.name)
+    # the chunk's dominant kernel is the headline roofline
+    dom = max((k for k in ("prefill_select", "prefill_attn", "prefill_local") if k in roofs),
+              key=lambda k: roofs[k]["ms_per_launch"])
     line = {
-        "metric": METRIC, "value": value, "unit": "ms/chunk", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16 mma / f32", "data": "synthetic",
+        "value": ms / steps, "unit": "ms/chunk", "steps": steps, "warmup": warmup, "ms_per_step": ms / steps,
         "config": _prefill_config(s, world),
-        "roofline": roof,
-        "tensor_kernels": tensor,
+        "roofline": roofs[dom],
+        "rooflines": roofs,
         "kernels": kern,
         "flops": flops,
-        "e2e": {"value": e2e_ms / args.steps, "unit": "ms/chunk",
+        "e2e": {"value": e2e_ms / steps, "unit": "ms/chunk",
                 "h2d_bytes_per_step": int((q.numel() + k_c.numel() + v_c.numel()) * 2),
                 "d2h_bytes_per_step": int(out.numel() * 4)},
         "gpu_launches": int(all_n),
@@ -718,12 +762,68 @@ def run_prefill_gpu(args):
                             "mean": float(counts.mean())},
         "clocks": clk,
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if cpu:
         v, cores, desc = cpu_oracle_prefill_sample(x)
         line["cpu_baseline"] = {"value": v, "unit": "ms/chunk", "cores": cores, "kind": "oracle", "sample": desc}
+    return line
+
+
+# the workloads measured besides the headline one, with the steps each takes at most (a 1M
+# prefill chunk takes about a second)
+SUB_WORKLOADS = (("decode_1m", None), ("prefill_32k", 5), ("prefill_1m", 3))
+
+
+def run_gpu(args):
+    import torch
+
+    import synth
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    cpu = rank == 0 and not args.no_cpu_baseline
+    exp_peak = measure_exp_rate(dev)
+
+    def one(name, steps):
+        s = _spec(args, name)
+        x = synth.generate(s)
+        if name in PREFILL_WORKLOADS:
+            return [measure_prefill(s, x, steps, args.warmup, world, dev, exp_peak, cpu=cpu)]
+        return measure_decode(s, x, steps, args.warmup, world, dev, top_ps=list(s.p_sweep) if s.p_sweep else None,
+                              cpu=cpu)
+
+    head = one(args.workload, args.steps)
+    main = head[len(head) // 2] if args.workload == "decode_1m" else head[0]  # p = 0.9 of a sweep
+    decode = args.workload in DECODE_WORKLOADS
+    line = {"metric": METRIC, "value": main["value"], "unit": main["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if decode else "f16 mma / f32",
+            "data": "synthetic"}
+    line.update({k: v for k, v in main.items() if k not in ("value", "unit", "steps", "warmup", "ms_per_step")})
+    if args.workload == "decode_1m":
+        line["p_sweep"] = {f"p={ln['top_p']}": ln for ln in head}
+    line["exp_peak"] = exp_peak
+    if not args.only:
+        subs = {}
+        total = line["gpu_launches"]
+        for name, cap in SUB_WORKLOADS:
+            if name == args.workload:
+                continue
+            steps = args.steps if cap is None else max(1, min(args.steps, cap))
+            for ln in one(name, steps):
+                key = name if "top_p" not in ln or name != "decode_1m" else f"{name}_p{ln['top_p']}"
+                subs[key] = ln
+                total += ln["gpu_launches"]
+        line["workloads"] = subs
+        line["gpu_launches_all_workloads"] = int(total)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    layer.close()
     if world > 1:
         torch.distributed.destroy_process_group()
     return 0
@@ -732,11 +832,13 @@ def run_prefill_gpu(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=DECODE_WORKLOADS + PREFILL_WORKLOADS, default="decode_128k",
-                    help="measured workload (the default is the headline one; others are for profiling)")
+                    help="headline workload (the default is the one the value is quoted on)")
+    ap.add_argument("--only", action="store_true",
+                    help="measure the headline workload alone (no sub-records for the other workloads)")
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -744,8 +846,6 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
-    if args.workload in PREFILL_WORKLOADS:
-        return run_prefill_gpu(args)
     return run_gpu(args)
 
 

@@ -216,6 +216,14 @@ rtp_status rtp_gather_attn_noalloc(const void* k, const void* v, const int32_t* 
                                    const int32_t* cnt, int32_t P, int64_t max_count, float sm_scale,
                                    float* out, cudaStream_t stream);
 
+/* Measurement probe, not part of the method: launches `blocks` CTAs of 256 threads that each
+ * evaluate 8 * iters dependent-free chains of ex2.approx (the exponential the prefill selection
+ * uses once per causal (row, key) pair), writing one float per thread to out (DEVICE,
+ * blocks * 256 floats).  *n_exp receives the number of exponentials launched; the caller times
+ * the launch on `stream` with CUDA events to measure the exponential issue rate that bounds
+ * the prefill selection.  RTP_EINVAL on a non-positive size or a NULL pointer. */
+rtp_status rtp_probe_ex2(int32_t blocks, int32_t iters, float* out, int64_t* n_exp, cudaStream_t stream);
+
 /* Host string for the last failure on this layer ("" if none).  layer may be NULL, which
  * returns the last failure of rtp_create in this thread. */
 const char* rtp_last_error(const rtp_layer* layer);

@@ -87,6 +87,7 @@ def lib() -> C.CDLL:
             "rtp_profile_enable": ([P, C.c_int], C.c_int),
             "rtp_profile_read": ([P, C.c_char_p, C.POINTER(C.c_double), C.POINTER(C.c_int64)], C.c_int),
             "rtp_last_error": ([P], C.c_char_p),
+            "rtp_probe_ex2": ([i32, i32, P, C.POINTER(C.c_int64), P], C.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -168,6 +169,13 @@ def rtp_gather_attn_noalloc(k_ptr: int, v_ptr: int, kv_block_ptr: Optional[int],
     """Attention over caller-given key lists without any device allocation (see rtp.h)."""
     _check(lib().rtp_gather_attn_noalloc(k_ptr, v_ptr, kv_block_ptr, kv_stride, q_ptr, idx_ptr, idx_stride,
                                          cnt_ptr, P, max_count, sm_scale, out_ptr, stream))
+
+
+def rtp_probe_ex2(blocks: int, iters: int, out_ptr: int, stream: int) -> int:
+    """Launch the exponential-rate probe; returns the number of exponentials it evaluates."""
+    n = C.c_int64()
+    _check(lib().rtp_probe_ex2(blocks, iters, out_ptr, C.byref(n), stream))
+    return n.value
 
 
 def rtp_check(layer, stream: int) -> int:

@@ -81,24 +81,32 @@ def test_profile_traffic_follows_the_kernel_source(tmp_path):
         assert got is None
 
 
-def test_prefill_roofline_follows_the_dominant_kernel():
+def test_prefill_rooflines_per_kernel():
     sys.path.insert(0, ROOT)
     import bench
 
-    flops = {"local_attention": 3.0e12, "retrieval_attention": 6.0e9, "index_scores": 2.0e9}
+    flops = {"local_attention": 3.0e12, "retrieval_attention": 6.0e9, "index_scores": 2.0e9,
+             "index_scores_flops": 6.4e10}
     kern = {"prefill_select": {"ms_per_launch": 10.0}, "prefill_attn": {"ms_per_launch": 5.0},
             "prefill_local": {"ms_per_launch": 6.0}, "q_prep": {"ms_per_launch": 99.0}}
-    r = bench._prefill_roofline(kern, flops, 2.0e9, 2000.0, 148, 1650.0, "measured")
-    # the selection dominates: one exp per causal pair against 16 ex2 / clock / SM
-    assert r["kernel"] == "prefill_select" and r["bound"] == "alu" and r["unit"] == "Gexp/s"
-    assert abs(r["achieved"] - 2.0e9 / 10e-3 / 1e9) < 1e-9
-    assert abs(r["peak"] - 16 * 148 * 2000.0e6 / 1e9) < 1e-9
-    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
-    # the local heads dominate: tensor roofline with their flops
-    kern["prefill_local"]["ms_per_launch"] = 20.0
-    r = bench._prefill_roofline(kern, flops, 2.0e9, None, 148, 1650.0, "measured")
-    assert r["kernel"] == "prefill_local" and r["bound"] == "tensor"
-    assert abs(r["achieved"] - 3.0e12 / 20e-3 / 1e12) < 1e-9 and r["peak"] == 1650.0
+    exp_peak = {"per_clk_per_sm": 16.0, "sms": 148, "sm_mhz": 1965.0}
+    r = bench._prefill_rooflines(kern, flops, 2.0e9, exp_peak, 2000.0, 1650.0, "measured")
+    # the selection: one exp per causal pair against the probe's rate at the sampled clock
+    sel = r["prefill_select"]
+    assert sel["bound"] == "alu" and sel["unit"] == "Gexp/s"
+    assert abs(sel["achieved"] - 2.0e9 / 10e-3 / 1e9) < 1e-9
+    assert abs(sel["peak"] - 16 * 148 * 2000.0e6 / 1e9) < 1e-9
+    assert abs(sel["frac"] - sel["achieved"] / sel["peak"]) < 1e-12
+    # the attention kernels: tensor rooflines with their algorithmic flops
+    assert r["prefill_local"]["bound"] == "tensor" and r["prefill_local"]["peak"] == 1650.0
+    assert abs(r["prefill_local"]["achieved"] - 3.0e12 / 6e-3 / 1e12) < 1e-9
+    assert abs(r["prefill_attn"]["achieved"] - 6.0e9 / 5e-3 / 1e12) < 1e-9
+    # the retrieval heads' two kernels together against the tensor peak
+    agg = r["index_plus_sparse_attention"]
+    assert abs(agg["achieved"] - (6.4e10 + 6.0e9) / 15e-3 / 1e12) < 1e-9
+    # without a sampled clock the probe's own clock is used
+    r = bench._prefill_rooflines(kern, flops, 2.0e9, exp_peak, None, 1650.0, "measured")
+    assert abs(r["prefill_select"]["peak"] - 16 * 148 * 1965.0e6 / 1e9) < 1e-9
 
 
 def test_prefill_traffic_only_for_the_captured_kernel_and_chunk():
