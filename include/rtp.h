@@ -90,8 +90,8 @@ typedef struct {
 /* Optional prefill statistics, DEVICE arrays (retrieval heads ascending).  Any member may be
  * NULL.  sel_bitmap holds, for every row i and retrieval head, bitmap_words 32-bit words: bit
  * (j % 32) of word j / 32 is set iff key j is in row i's selected set.  Words the kernel writes:
- * those covering keys 0 .. (last position of the row's 64-row tile), rounded up to 64 keys and
- * capped at bitmap_words; the caller zeroes the rest.  Keys past 32 * bitmap_words are not
+ * those covering keys 0 .. (last position of the row's 128-row tile), rounded up to 64 keys
+ * and capped at bitmap_words; the caller zeroes the rest.  Keys past 32 * bitmap_words are not
  * reported (the selection itself is unaffected).
  *
  * Row-subset positions (cheap at any chunk size, where a full bitmap is not): for each of the

@@ -9,45 +9,46 @@
 // digest, limitations -- the per-row selection here is the chunked-prefill counterpart of the
 // decode selection.)
 //
-// Two kernels, one CTA per (64-row tile, retrieval head, sequence), 128 threads each; scores
-// come from index_mma.cuh (tensor cores, identical bits in every pass):
+// Both kernels take 128-row tiles (one CTA per (row tile, retrieval head, sequence)) and score
+// 64-key tiles on the tensor cores (index_tc.cuh: three tcgen05.mma into TMEM, key tiles
+// copied by TMA), so both see identical score bits:
 //
-//  prefill_select_kernel -- the exact cut (t_key, tiecut) of each row, in passes over the
-//    row's causal keys, all arithmetic exact in 64-bit fixed point (mass of key j =
-//    round(2^sc * e^(s_j - m)), sc = 62 - ceil(log2 len)):
+//  prefill_select_kernel -- 128 threads, one query row per thread (its TMEM lane).  The exact
+//    cut (t_key, tiecut) of each row, in walks over the row's causal keys, all masses exact in
+//    64-bit fixed point (mass of key j = trunc(2^sc * e^(s_j - m)), sc = 62 - ceil(log2 len)),
+//    each row's histograms in its own shared-memory column (no atomics):
 //      A  row maxima m;
 //      B  16 bins of m - s rounded to an integer (the last one holding everything from 14.5
 //         down) -> Z, T = ceil(p Z), crossing bin, whose exact order-key range is found by
 //         bisection;
-//      R  refinement: the crossing range of order keys is split 16 ways by bit slices, with
-//         the mass of each slice and the first keys of the range captured; once a row's
+//      R  refinement: the crossing range of order keys is split 32 ways by bit slices, with
+//         the mass of each slice and the first 16 keys of the range captured; once a row's
 //         range holds <= 16 keys they are sorted (key desc, j asc) for the exact cut; a range
 //         that shrinks to one key value is an exact tie group, resolved by
 //      T  an ordered count of the tied positions.
-//  prefill_attn_kernel -- recomputes the scores, applies each row's cut, ORs the rows' masks
-//    of every 64-key tile into the tile's union, compacts the union keys of successive tiles
-//    into 64-key chunks (positions + per-row bits) and runs the attention tiles (fa_tile.cuh)
-//    on the gathered K/V rows of each full chunk; tiles no row selects cost only their scores.
-#include "fa_tile.cuh"
-#include "index_mma.cuh"
+//  prefill_attn_kernel -- 256 threads, two per row (each on half of a tile's 64 columns).
+//    Walks the key tiles in order: the index scores of tile t + 1 (computed one tile ahead)
+//    and each row's cut give the rows' selection masks; a tile no row selects is skipped,
+//    otherwise its K and V rows come in by TMA, S = Q K^T runs on the tensor cores into TMEM,
+//    the masked online softmax forms P in shared memory and O += P V accumulates in TMEM.
+#include "index_tc.cuh"
 #include "rtp_internal.h"
 
 namespace rtp {
 
 namespace {
 
-constexpr int kRows = 64;
-constexpr int kThreads = kIdxThreads;  // 128
-constexpr int kBins = 16;
-constexpr int kCand = 4;               // candidates captured per thread and row slot
+constexpr int kRowsR = kTcRows;  // 128 query rows per CTA (TMEM lanes)
+constexpr int kKeysR = kTcKeys;  // 64 keys per tile
+constexpr int kBins = 16;        // pass B: bins of width 1 below the row max
+constexpr int kSlices = 32;      // refinement: slices of the crossing key range per level
+constexpr int kCand = 16;        // keys captured per row in a refinement walk
+constexpr int kLevels = 8;       // refinement levels (5 key bits each, with margin)
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int { kModeKeys = 1, kModeTie = 2, kModeDone = 3 };
 
 struct RetArgs {
-  const __half* idx;          // [B][Hr][max_seq][hi r | lo r]: the split index cache
-  const __half* kc;
-  const __half* vc;
   int64_t max_seq;
   int Hkv, Hq, Hr, group, C;
   int64_t P0;
@@ -70,93 +71,36 @@ struct RetArgs {
   uint32_t* err;
 };
 
-struct RowS {
-  float m;
-  int mode, cb, shift, found, tiecut;
-  uint32_t klo, khi, t_key;
-  unsigned long long Z, rem, above, n_need, tie_before;
-};
-
-// Per-thread exact histograms: a 64-bit mass is added as three 21-bit limbs with shared-memory
-// reductions (no read-modify-write chains); limb sums stay below 2^32 because every thread
-// folds its carries at least every kFoldTiles tiles (at most 16 keys per row slot per tile).
-constexpr int kLimbs = 3;
-constexpr int kFoldTiles = 128;
-
-struct SmemSel {
-  IdxRing st;                                     // 12 KB
-  uint32_t h[kBins][2][kLimbs][kThreads];         // 48 KB
-  unsigned long long cand[kCand][2][kThreads];    // 8 KB
-  int nc[2][kThreads];
-  RowS row[kRows];
-};
-
-__device__ __forceinline__ void red_add(uint32_t addr, uint32_t v) {
-  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-// Add mass v to bin b of row slot sl of this thread (three limb reductions).
-__device__ __forceinline__ void hist_add(SmemSel& S, int b, int sl, int tid, unsigned long long v) {
-  const uint32_t a0 = smem_u32(&S.h[b][sl][0][tid]);
-  red_add(a0, (uint32_t)v & 0x1FFFFFu);
-  red_add(a0 + kThreads * 4, (uint32_t)(v >> 21) & 0x1FFFFFu);
-  red_add(a0 + 2 * kThreads * 4, (uint32_t)(v >> 42));
-}
-
-__device__ __forceinline__ unsigned long long hist_get(const SmemSel& S, int b, int sl, int t) {
-  return (unsigned long long)S.h[b][sl][0][t] + ((unsigned long long)S.h[b][sl][1][t] << 21) +
-         ((unsigned long long)S.h[b][sl][2][t] << 42);
-}
-
-// Fold this thread's limb carries (its own entries only; same-thread order suffices).
-__device__ __forceinline__ void hist_fold(SmemSel& S, int tid) {
-  for (int b = 0; b < kBins; ++b)
-    for (int sl = 0; sl < 2; ++sl) {
-      const unsigned long long v = hist_get(S, b, sl, tid);
-      S.h[b][sl][0][tid] = (uint32_t)v & 0x1FFFFFu;
-      S.h[b][sl][1][tid] = (uint32_t)(v >> 21) & 0x1FFFFFu;
-      S.h[b][sl][2][tid] = (uint32_t)(v >> 42);
-    }
-}
-
-__device__ __forceinline__ void hist_zero(SmemSel& S, int tid) {
-  for (int b = 0; b < kBins; ++b)
-    for (int sl = 0; sl < 2; ++sl)
-      for (int l = 0; l < kLimbs; ++l) S.h[b][sl][l][tid] = 0u;
-}
-
 // Fixed-point mass of a score s below the row max m: e^(s - m) * 2^sc truncated to an integer
 // (scale = 2^sc as a float, exact).
 __device__ __forceinline__ unsigned long long mass64(float s, float m, float scale) {
   return __float2ull_rz(fast_exp2((s - m) * kLog2e) * scale);
 }
 
-// level-1 bin of x = m - s >= 0: x rounded to the nearest integer (adding 2^23 does the rounding),
-// with everything from 14.5 down in the last bin.  Non-increasing in s.
+// pass-B bin of x = m - s >= 0: x rounded to the nearest integer (adding 2^23 does the
+// rounding), with everything from 14.5 down in the last bin.  Non-increasing in s.
 __device__ __forceinline__ int bin1_of(float x) {
   const uint32_t r = __float_as_uint(x + 8388608.0f) - 0x4B000000u;
   return (int)min(r, (uint32_t)(kBins - 1));
 }
 
-// Exact order-key range [lo, hi] of the finite scores s <= m whose level-1 bin is b (bisection
+// Exact order-key range [lo, hi] of the finite scores s <= m whose pass-B bin is b (bisection
 // on the monotone map key -> bin).
 __device__ __forceinline__ void bin_key_range(float m, int b, uint32_t* lo, uint32_t* hi) {
   const uint32_t kmin = order_key(-3.4028234663852886e38f), kmax = order_key(m);
   auto bin_of_key = [&](uint32_t k) { return bin1_of(m - key_to_float(k)); };
-  // first key with bin <= b
-  uint32_t l = kmin, h = kmax;
+  uint32_t l = kmin, h = kmax;  // first key with bin <= b
   while (l < h) {
     const uint32_t mid = l + ((h - l) >> 1);
     if (bin_of_key(mid) <= b) h = mid;
     else l = mid + 1;
   }
   *lo = l;
-  // last key with bin >= b: one below the first key with bin < b (kmax + 1 if none)
   if (b == 0) {
     *hi = kmax;
     return;
   }
-  l = *lo;
+  l = *lo;  // last key with bin >= b: one below the first key with bin < b
   h = kmax;
   if (bin_of_key(h) >= b) {
     *hi = h;
@@ -170,625 +114,711 @@ __device__ __forceinline__ void bin_key_range(float m, int b, uint32_t* lo, uint
   *hi = l - 1;
 }
 
+// slices of 2^shift keys cover [klo, khi] in at most kSlices pieces
 __device__ __forceinline__ int slice_shift(uint32_t klo, uint32_t khi) {
-  const uint32_t d = khi - klo;  // span - 1
-  const int bits = 32 - __clz(d);
-  return bits > 4 ? bits - 4 : 0;
+  const int bits = 32 - __clz(khi - klo);
+  return bits > 5 ? bits - 5 : 0;
 }
 
-struct RowCtx {
-  int tid, warp, gr, tq;
-  int ra, rb;          // CTA rows of slot 0 / 1
-  int64_t pa, pb;      // their positions (-1: inactive row)
-  int64_t pos_lo;      // position of CTA row 0 (every active row is at or after it)
-  int64_t nkeys;       // keys the CTA's rows can see
+// last causal column of a 64-key tile for a row at position pos (-1: none)
+__device__ __forceinline__ int causal_lim(int64_t pos, int64_t t) {
+  return (int)max((int64_t)-1, min((int64_t)(kKeysR - 1), pos - t * kKeysR));
+}
+
+// ------------------------------------------------------------------ exact per-row top-p
+
+constexpr int kPsThreads = kRowsR;  // one thread per row
+constexpr uint32_t kSelStages = 4;   // key tiles of the TMA ring
+constexpr uint32_t kSOffQ = 0;                                       // query tile, 8 KB
+constexpr uint32_t kSOffK = kSOffQ + kTcQBytes;                      // key ring, 4 x 4 KB
+constexpr uint32_t kSOffH = kSOffK + kSelStages * kTcKBytes;         // [slice][row] u64, 32 KB
+constexpr uint32_t kSOffC = kSOffH + kSlices * kRowsR * 8;           // [cand][row] u64, 16 KB
+constexpr uint32_t kSOffBar = kSOffC + kCand * kRowsR * 8;           // full[4], done[2], TMEM base
+constexpr uint32_t kSelSmem = kSOffBar + 64;
+constexpr uint32_t kSelTmemCols = 128;                               // two 64-column score buffers
+
+// Walks over the key tiles [0, ntiles) of one (sequence, retrieval head): thread 0 keeps
+// kSelStages TMA copies in flight and issues the scores of tile t + 1 before tile t is read;
+// body(t, s) gets this thread's row's 64 scores of tile t.  g counts tiles over all walks
+// (mbarrier phases).  A wait that runs out clears ok in every thread; later walks then do
+// nothing, and drain() waits (bounded) for the copies and MMAs still in flight.
+struct SelWalk {
+  uint32_t sbase, tmem, lane_addr;
+  const CUtensorMap* map;
+  int64_t row0;
+  uint32_t g;
+  bool ok;
+  uint32_t inflight_lo, inflight_hi;  // tiles [lo, hi) whose copies thread 0 has not waited on
+  bool mma_pending;                   // scores of tile g issued and not waited on
+
+  __device__ uint32_t full_bar(uint32_t gt) const { return sbase + kSOffBar + 8u * (gt % kSelStages); }
+  __device__ uint32_t done_bar(uint32_t gt) const { return sbase + kSOffBar + 32u + 8u * (gt & 1u); }
+  __device__ uint32_t ktile(uint32_t gt) const { return sbase + kSOffK + (gt % kSelStages) * kTcKBytes; }
+
+  template <typename Body>
+  __device__ __forceinline__ void run(int64_t ntiles, Body body) {
+    const int tid = threadIdx.x;
+    if (!ok || ntiles <= 0) return;
+    bool okw = true;
+    if (tid == 0) {
+      inflight_lo = g;
+      for (int64_t i = 0; i < (int64_t)kSelStages && i < ntiles; ++i)
+        tc_load_keys(ktile(g + (uint32_t)i), map, row0, i, full_bar(g + (uint32_t)i));
+      inflight_hi = g + (uint32_t)min((int64_t)kSelStages, ntiles);
+      okw = mbar_wait(full_bar(g), (g / kSelStages) & 1u);
+      inflight_lo = g + 1;
+      if (okw) tc_issue_scores(tmem + (g & 1u) * kTcKeys, sbase + kSOffQ, ktile(g), done_bar(g));
+      mma_pending = okw;
+    }
+    for (int64_t t = 0; t < ntiles; ++t) {
+      const uint32_t gt = g + (uint32_t)t;
+      bool issued_next = false;  // thread 0: the scores of tile gt + 1 are in flight
+      if (tid == 0 && t + 1 < ntiles && okw) {
+        okw = mbar_wait(full_bar(gt + 1), ((gt + 1) / kSelStages) & 1u);
+        inflight_lo = gt + 2;
+        if (okw) {
+          tc_issue_scores(tmem + ((gt + 1) & 1u) * kTcKeys, sbase + kSOffQ, ktile(gt + 1), done_bar(gt + 1));
+          issued_next = true;
+        }
+      }
+      if (tid != 0 || mma_pending) okw = mbar_wait(done_bar(gt), (gt >> 1) & 1u) && okw;
+      tc_fence_after();
+      float s[kTcKeys];
+      __syncwarp();  // the loads are warp-collective: reconverge after thread 0's work
+      tmem_ld32(lane_addr + (gt & 1u) * kTcKeys, s);
+      tmem_ld32(lane_addr + (gt & 1u) * kTcKeys + 32u, s + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      if (!__syncthreads_and(okw ? 1 : 0)) {
+        ok = false;
+        if (tid == 0) mma_pending = issued_next;  // drain() waits for the scores of tile gt + 1
+        g = gt + 1;
+        return;
+      }
+      if (tid == 0) {
+        mma_pending = issued_next;
+        if (t + kSelStages < ntiles) {  // the stage of tile gt is free: its scores are done
+          tc_load_keys(ktile(gt), map, row0, t + kSelStages, full_bar(gt));
+          inflight_hi = gt + kSelStages + 1;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kTcKeys; ++i) s[i] += 0.0f;  // -0 -> +0: equal scores, equal order keys
+      body(t, s);
+    }
+    g += (uint32_t)ntiles;
+  }
+
+  // after a timeout: wait (bounded) for the copies and the scores still in flight
+  __device__ void drain() {
+    if (threadIdx.x != 0) return;
+    for (uint32_t gt = inflight_lo; gt < inflight_hi; ++gt) mbar_wait(full_bar(gt), (gt / kSelStages) & 1u);
+    if (mma_pending) mbar_wait(done_bar(g), (g >> 1) & 1u);
+  }
 };
 
-__device__ __forceinline__ RowCtx row_ctx(const RetArgs& a, int i0, int nrows) {
-  RowCtx x;
-  x.tid = threadIdx.x;
-  x.warp = x.tid >> 5;
-  x.gr = (x.tid & 31) >> 2;
-  x.tq = x.tid & 3;
-  x.ra = 16 * x.warp + x.gr;
-  x.rb = x.ra + 8;
-  x.pa = x.ra < nrows ? a.P0 + i0 + x.ra : -1;
-  x.pb = x.rb < nrows ? a.P0 + i0 + x.rb : -1;
-  x.pos_lo = a.P0 + i0;
-  x.nkeys = a.P0 + i0 + nrows;
-  return x;
-}
-
-// Pipelined walk over the index tiles of keys [0, nkeys): body(t, stage) runs once tile t is
-// in ring stage `stage` (kIdxStages - 1 tiles in flight, one barrier per tile).
-template <typename Body>
-__device__ __forceinline__ void idx_walk(IdxRing& R, const __half* base, int64_t nkeys, Body body) {
-  const int64_t ntiles = (nkeys + kIdxKeys - 1) / kIdxKeys;
-#pragma unroll
-  for (int s = 0; s < kIdxStages - 1; ++s) {
-    if (s < ntiles) idx_issue(R, s, base, s, nkeys);
-    cp_async_commit();
-  }
-  for (int64_t t = 0; t < ntiles; ++t) {
-    cp_async_wait<kIdxStages - 2>();
-    __syncthreads();  // tile t landed for every thread; stage (t - 1) % kIdxStages is free
-    const int64_t tn = t + kIdxStages - 1;
-    if (tn < ntiles) idx_issue(R, (int)(tn % kIdxStages), base, tn, nkeys);
-    cp_async_commit();
-    body(t, (int)(t % kIdxStages));
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-}
-
-// Run f(slot, j, s) over this thread's causal (row, key) pairs, tile by tile; fold() runs
-// after every kFoldTiles tiles.
-template <typename F, typename G>
-__device__ __forceinline__ void scan(IdxRing& S, const RowCtx& x, const __half* ibase, const uint32_t qh[4],
-                                     const uint32_t ql[4], F f, G fold) {
-  idx_walk(S, ibase, x.nkeys, [&](int64_t t, int stage) {
-    if (t > 0 && t % kFoldTiles == 0) fold();
-    float c[8][4];
-    idx_scores(c, qh, ql, S, stage);
-    const int64_t base = t * kIdxKeys;
-    // causal limits of the two rows inside this tile (-1: none, 63: all)
-    const int la = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pa - base));
-    const int lb = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pb - base));
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int p = 8 * nt + 2 * x.tq + e;
-        if (p <= la) f(0, base + p, c[nt][e]);
-        if (p <= lb) f(1, base + p, c[nt][2 + e]);
-      }
-    }
-  });
-}
-
-// As scan, for passes that touch few keys: gate(slot, s) is evaluated branch-free for every
-// pair, and f runs only on pairs that pass it, after one warp vote per tile.
-template <typename Gate, typename F, typename G>
-__device__ __forceinline__ void scan_gated(IdxRing& S, const RowCtx& x, const __half* ibase, const uint32_t qh[4],
-                                           const uint32_t ql[4], Gate gate, F f, G fold) {
-  idx_walk(S, ibase, x.nkeys, [&](int64_t t, int stage) {
-    if (t > 0 && t % kFoldTiles == 0) fold();
-    float c[8][4];
-    idx_scores(c, qh, ql, S, stage);
-    const int64_t base = t * kIdxKeys;
-    const int la = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pa - base));
-    const int lb = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pb - base));
-    uint32_t hit = 0;  // bit 2*(2nt+e)+slot
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int p = 8 * nt + 2 * x.tq + e;
-        const int k = 2 * nt + e;
-        hit |= (uint32_t)(p <= la && gate(0, c[nt][e])) << (2 * k);
-        hit |= (uint32_t)(p <= lb && gate(1, c[nt][2 + e])) << (2 * k + 1);
-      }
-    }
-    if (!__any_sync(0xffffffffu, hit != 0u)) return;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int p = 8 * nt + 2 * x.tq + e;
-        const int k = 2 * nt + e;
-        if (hit & (1u << (2 * k))) f(0, base + p, c[nt][e]);
-        if (hit & (1u << (2 * k + 1))) f(1, base + p, c[nt][2 + e]);
-      }
-    }
-  });
-}
-
-__global__ void __launch_bounds__(kThreads) prefill_select_kernel(RetArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  SmemSel& S = *reinterpret_cast<SmemSel*>(smem_raw);
+__global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
+                                                                     const __grid_constant__ CUtensorMap tm_idx) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const uint32_t sbase = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int tile = gridDim.x - 1 - blockIdx.x, hr = blockIdx.y, b = blockIdx.z;  // longest rows first
-  const int i0 = tile * kRows;
-  const int nrows = min(kRows, a.C - i0);
-  const RowCtx x = row_ctx(a, i0, nrows);
-  const int tid = x.tid;
-  const bool owner = x.tq == 0;
+  const int i0 = tile * kRowsR;
+  const int nrows = min(kRowsR, a.C - i0);
+  const bool live = tid < nrows;
+  const int64_t pos = live ? a.P0 + i0 + tid : -1;
+  const int64_t nkeys = a.P0 + i0 + nrows;
+  const int64_t ntiles = (nkeys + kKeysR - 1) / kKeysR;
   const float scale = __uint_as_float((uint32_t)(127 + a.sc_bits) << 23);  // 2^sc_bits
-  const __half* ibase = a.idx + ((int64_t)b * a.Hr + hr) * a.max_seq * (2 * kR);
   uint2* cut = a.cut + ((int64_t)b * a.Hr + hr) * a.C + i0;
+  float* mass_out = (a.sel_mass && live) ? a.sel_mass + ((int64_t)b * a.C + i0 + tid) * a.Hr + hr : nullptr;
 
   if (a.top_p >= 1.f) {  // p = 1 keeps every causal key (also those whose mass rounds to 0)
-    if (owner) {
-      if (x.pa >= 0) cut[x.ra] = make_uint2(0u, 0x7FFFFFFFu);
-      if (x.pb >= 0) cut[x.rb] = make_uint2(0u, 0x7FFFFFFFu);
-      if (a.sel_mass) {
-        if (x.pa >= 0) a.sel_mass[((int64_t)b * a.C + i0 + x.ra) * a.Hr + hr] = 1.f;
-        if (x.pb >= 0) a.sel_mass[((int64_t)b * a.C + i0 + x.rb) * a.Hr + hr] = 1.f;
-      }
+    if (live) {
+      cut[tid] = make_uint2(0u, 0x7FFFFFFFu);
+      if (mass_out) *mass_out = 1.f;
     }
     return;
   }
-
-  uint32_t qh[4], ql[4];
+  if (sbase & 127u) {  // TMA destinations and operand tiles need aligned shared memory
+    if (tid == 0) atomicOr(a.err, kErrInternal);
+    return;
+  }
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSOffBar + 48);
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kSelTmemCols);
+  if (tid == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(sbase + kSOffBar + 8u * i, 1);
+    fence_mbar_init();
+  }
   {
-    const int64_t qs = (int64_t)a.Hr * kR;
-    const float* q0 = a.q_idx + ((int64_t)b * a.C + i0) * qs + (int64_t)hr * kR;
-    idx_load_q(qh, ql, x.pa >= 0 ? q0 + x.ra * qs : nullptr, x.pb >= 0 ? q0 + x.rb * qs : nullptr);
+    const float* qrow = a.q_idx + (((int64_t)b * a.C + i0 + (live ? tid : 0)) * a.Hr + hr) * kR;
+    tc_put_query(sm + kSOffQ, tid, live ? qrow : nullptr);
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  SelWalk W;
+  W.sbase = sbase;
+  W.tmem = tmem;
+  W.lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  W.map = &tm_idx;
+  W.row0 = ((int64_t)b * a.Hr + hr) * a.max_seq;
+  W.g = 0;
+  W.ok = true;
+  W.inflight_lo = W.inflight_hi = 0;
+  W.mma_pending = false;
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(sm + kSOffH) + tid;  // [slice * 128]
+  unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kSOffC) + tid;  // [k * 128]
+
+  // ---- pass A: the row max
+  float m = -INFINITY;
+  W.run(ntiles, [&](int64_t t, const float* s) {
+    const int lim = causal_lim(pos, t);
+#pragma unroll
+    for (int c = 0; c < kKeysR; ++c)
+      if (c <= lim) m = fmaxf(m, s[c]);
+  });
+
+  // ---- pass B: 16 bins of width 1 below the max (the last, most populated bin in a register)
+  for (int i = 0; i < kBins; ++i) hist[i * kRowsR] = 0ull;
+  unsigned long long far = 0ull;
+  W.run(ntiles, [&](int64_t t, const float* s) {
+    const int lim = causal_lim(pos, t);
+#pragma unroll
+    for (int c = 0; c < kKeysR; ++c) {
+      if (c <= lim) {
+        const int bi = bin1_of(m - s[c]);
+        const unsigned long long ms = mass64(s[c], m, scale);
+        if (bi == kBins - 1) far += ms;
+        else hist[bi * kRowsR] += ms;
+      }
+    }
+  });
+  int mode = kModeDone, shift = 0, tiecut = -1;
+  uint32_t klo = 0u, khi = 0u, t_key = 0xFFFFFFFFu;
+  unsigned long long Z = 0ull, rem = 0ull, above = 0ull, n_need = 0ull;
+  if (live) {
+    unsigned long long hb[kBins];
+    for (int i = 0; i < kBins - 1; ++i) {
+      hb[i] = hist[i * kRowsR];
+      Z += hb[i];
+    }
+    hb[kBins - 1] = far;
+    Z += far;
+    unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
+    if (T < 1ull) T = 1ull;
+    if (T > Z) T = Z;
+    unsigned long long cum = 0ull;
+    int cb = kBins - 1;  // bins run from the highest scores down
+    for (int i = 0; i < kBins; ++i) {
+      if (cum + hb[i] >= T) {
+        cb = i;
+        break;
+      }
+      cum += hb[i];
+    }
+    rem = T - cum;
+    above = cum;
+    bin_key_range(m, cb, &klo, &khi);
+    shift = slice_shift(klo, khi);
+    mode = kModeKeys;
   }
 
-  // ---- pass A: row maxima (the 4 threads of a quad share their two rows)
-  float m[2] = {-INFINITY, -INFINITY};
-  scan(S.st, x, ibase, qh, ql, [&](int sl, int64_t, float s) { m[sl] = fmaxf(m[sl], s); }, [] {});
+  // ---- refinement: 32-way bit slices of the crossing key range until <= 16 keys remain
+  for (int level = 0; level < kLevels; ++level) {
+    if (!__syncthreads_or(mode == kModeKeys)) break;
+    const bool mine = mode == kModeKeys;
+    if (mine)
+      for (int i = 0; i < kSlices; ++i) hist[i * kRowsR] = 0ull;
+    int nc = 0;
+    const uint32_t span = khi - klo;
+    W.run(ntiles, [&](int64_t t, const float* s) {
+      if (!mine) return;
+      const int lim = causal_lim(pos, t);
 #pragma unroll
-  for (int sl = 0; sl < 2; ++sl) {
-    m[sl] = fmaxf(m[sl], __shfl_xor_sync(0xffffffffu, m[sl], 1));
-    m[sl] = fmaxf(m[sl], __shfl_xor_sync(0xffffffffu, m[sl], 2));
-  }
-
-  // ---- pass B: 16 bins of width 1 below the max -> Z, T, crossing bin
-  hist_zero(S, tid);
-  scan(S.st, x, ibase, qh, ql, [&](int sl, int64_t, float s) {
-    hist_add(S, bin1_of(m[sl] - s), sl, tid, mass64(s, m[sl], scale));
-  }, [&] { hist_fold(S, tid); });
-  if (owner) {
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      const int r = sl ? x.rb : x.ra;
-      RowS& R = S.row[r];
-      R.m = m[sl];
-      R.found = 0;
-      R.tie_before = 0;
-      if ((sl ? x.pb : x.pa) < 0) {
-        R.mode = kModeDone;
-        continue;
+      for (int c = 0; c < kKeysR; ++c) {
+        const uint32_t key = order_key(s[c]);
+        if (c <= lim && key - klo <= span) {
+          hist[(int)((key - klo) >> shift) * kRowsR] += mass64(s[c], m, scale);
+          if (nc < kCand)
+            cand[nc * kRowsR] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)(t * kKeysR + c));
+          ++nc;
+        }
       }
-      unsigned long long hb[kBins];
-      unsigned long long Z = 0;
-      for (int i = 0; i < kBins; ++i) {
-        hb[i] = hist_get(S, i, sl, tid) + hist_get(S, i, sl, tid + 1) + hist_get(S, i, sl, tid + 2) +
-                hist_get(S, i, sl, tid + 3);
-        Z += hb[i];
+    });
+    if (!mine) continue;
+    if (nc <= kCand) {
+      // every key of the range is a captured candidate: exact cut by sorting them
+      unsigned long long cv[kCand];
+      for (int i = 0; i < nc; ++i) cv[i] = cand[i * kRowsR];
+      for (int i = 1; i < nc; ++i) {  // insertion sort, descending: key desc, then j asc
+        const unsigned long long v = cv[i];
+        int k = i - 1;
+        while (k >= 0 && cv[k] < v) {
+          cv[k + 1] = cv[k];
+          --k;
+        }
+        cv[k + 1] = v;
       }
-      unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
-      if (T < 1ull) T = 1ull;
-      if (T > Z) T = Z;
-      unsigned long long cum = 0;
-      int cb = kBins - 1;  // bins run from the highest scores down
-      for (int i = 0; i < kBins; ++i) {
-        if (cum + hb[i] >= T) {
-          cb = i;
+      unsigned long long cum = 0ull;
+      int ci = -1;
+      for (int i = 0; i < nc; ++i) {
+        cum += mass64(key_to_float((uint32_t)(cv[i] >> 32)), m, scale);
+        if (cum >= rem) {
+          ci = i;
           break;
         }
-        cum += hb[i];
       }
-      R.Z = Z;
-      R.cb = cb;
-      R.rem = T - cum;
-      R.above = cum;
-      bin_key_range(m[sl], cb, &R.klo, &R.khi);
-      R.shift = slice_shift(R.klo, R.khi);
-      R.mode = kModeKeys;
-    }
-  }
-  __syncthreads();
-
-  // ---- refinement: 16-way bit slices of the crossing key range until <= 16 keys remain
-  for (int level = 0; level < 10; ++level) {
-    const int need = (S.row[x.ra].mode == kModeKeys) || (S.row[x.rb].mode == kModeKeys);
-    if (!__syncthreads_or(need)) break;
-    bool mine[2];
-    int sh[2];
-    uint32_t klo[2], khi[2];
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      const RowS& R = S.row[sl ? x.rb : x.ra];
-      mine[sl] = R.mode == kModeKeys;
-      sh[sl] = R.shift;
-      klo[sl] = R.klo;
-      khi[sl] = R.khi;
-    }
-    hist_zero(S, tid);
-    int nc[2] = {0, 0};
-    RowCtx xm = x;  // rows outside refinement see no keys
-    if (!mine[0]) xm.pa = -1;
-    if (!mine[1]) xm.pb = -1;
-    const uint32_t span[2] = {khi[0] - klo[0], khi[1] - klo[1]};
-    scan_gated(S.st, xm, ibase, qh, ql, [&](int sl, float s) { return order_key(s) - klo[sl] <= span[sl]; },
-               [&](int sl, int64_t j, float s) {
-      const uint32_t key = order_key(s);
-      {
-        hist_add(S, (int)((key - klo[sl]) >> sh[sl]), sl, tid, mass64(s, m[sl], scale));
-        if (nc[sl] < kCand) S.cand[nc[sl]][sl][tid] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)j);
-        ++nc[sl];
+      if (ci < 0) {  // not reached: the range was chosen to hold at least rem
+        atomicOr(a.err, kErrInternal);
+        t_key = 0xFFFFFFFFu;
+        tiecut = -1;
+      } else {
+        t_key = (uint32_t)(cv[ci] >> 32);
+        tiecut = (int)(0xFFFFFFFFu - (uint32_t)cv[ci]);
+        above += cum;
       }
-    }, [&] { hist_fold(S, tid); });
-    S.nc[0][tid] = nc[0];
-    S.nc[1][tid] = nc[1];
-    __syncthreads();
-    if (owner) {
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        if (!mine[sl]) continue;
-        RowS& W = S.row[sl ? x.rb : x.ra];
-        const int n0 = S.nc[sl][tid], n1 = S.nc[sl][tid + 1], n2 = S.nc[sl][tid + 2], n3 = S.nc[sl][tid + 3];
-        if (n0 <= kCand && n1 <= kCand && n2 <= kCand && n3 <= kCand) {
-          // every key of the range is a captured candidate: exact cut by sorting them
-          unsigned long long c[4 * kCand];
-          int n = 0;
-          const int nq[4] = {n0, n1, n2, n3};
-          for (int q = 0; q < 4; ++q)
-            for (int i = 0; i < nq[q]; ++i) c[n++] = S.cand[i][sl][tid + q];
-          for (int i = 1; i < n; ++i) {  // insertion sort, descending: key desc, then j asc
-            const unsigned long long v = c[i];
-            int k = i - 1;
-            while (k >= 0 && c[k] < v) {
-              c[k + 1] = c[k];
-              --k;
-            }
-            c[k + 1] = v;
-          }
-          unsigned long long cum = 0;
-          int ci = -1;
-          for (int i = 0; i < n; ++i) {
-            cum += mass64(key_to_float((uint32_t)(c[i] >> 32)), m[sl], scale);
-            if (cum >= W.rem) {
-              ci = i;
-              break;
-            }
-          }
-          if (ci < 0) {  // not reached: the range was chosen to hold at least rem
-            atomicOr(a.err, kErrInternal);
-            W.t_key = 0xFFFFFFFFu;
-            W.tiecut = -1;
-          } else {
-            W.t_key = (uint32_t)(c[ci] >> 32);
-            W.tiecut = (int)(0xFFFFFFFFu - (uint32_t)c[ci]);
-            W.above += cum;
-          }
-          W.mode = kModeDone;
-        } else {
-          unsigned long long cum = 0;
-          int cs = -1;
-          for (int i = kBins - 1; i >= 0; --i) {  // highest slice first
-            const unsigned long long hs = hist_get(S, i, sl, tid) + hist_get(S, i, sl, tid + 1) +
-                                          hist_get(S, i, sl, tid + 2) + hist_get(S, i, sl, tid + 3);
-            if (cum + hs >= W.rem) {
-              cs = i;
-              break;
-            }
-            cum += hs;
-          }
-          if (cs < 0) {
-            atomicOr(a.err, kErrInternal);
-            W.t_key = 0xFFFFFFFFu;
-            W.tiecut = -1;
-            W.mode = kModeDone;
-          } else {
-            const uint32_t nlo = W.klo + ((uint32_t)cs << W.shift);
-            const uint32_t top = nlo + ((1u << W.shift) - 1u);
-            const uint32_t nhi = top < W.khi && top >= nlo ? top : W.khi;
-            W.rem -= cum;
-            W.above += cum;
-            W.klo = nlo;
-            W.khi = nhi;
-            W.shift = slice_shift(nlo, nhi);
-            if (nlo == nhi) {  // one key value with more than 16 members: an exact tie group
-              W.t_key = nlo;
-              const unsigned long long e = mass64(key_to_float(nlo), m[sl], scale);
-              W.n_need = e ? (W.rem + e - 1) / e : 1ull;
-              W.mode = kModeTie;
-            }
-          }
+      mode = kModeDone;
+    } else {
+      unsigned long long cum = 0ull;
+      int cs = -1;
+      for (int i = kSlices - 1; i >= 0; --i) {  // highest slice first
+        const unsigned long long hs = hist[i * kRowsR];
+        if (cum + hs >= rem) {
+          cs = i;
+          break;
+        }
+        cum += hs;
+      }
+      if (cs < 0) {
+        atomicOr(a.err, kErrInternal);
+        t_key = 0xFFFFFFFFu;
+        tiecut = -1;
+        mode = kModeDone;
+      } else {
+        const uint32_t nlo = klo + ((uint32_t)cs << shift);
+        const uint32_t top = nlo + ((1u << shift) - 1u);
+        const uint32_t nhi = top < khi && top >= nlo ? top : khi;
+        rem -= cum;
+        above += cum;
+        klo = nlo;
+        khi = nhi;
+        shift = slice_shift(nlo, nhi);
+        if (nlo == nhi) {  // one key value with more than 16 members: an exact tie group
+          t_key = nlo;
+          const unsigned long long e = mass64(key_to_float(nlo), m, scale);
+          n_need = e ? (rem + e - 1) / e : 1ull;
+          mode = kModeTie;
         }
       }
     }
-    __syncthreads();
   }
-  if (owner) {
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      RowS& W = S.row[sl ? x.rb : x.ra];
-      if (W.mode == kModeKeys) {  // not reached: ten 16-way levels split 32 bits
-        atomicOr(a.err, kErrInternal);
-        W.t_key = 0xFFFFFFFFu;
-        W.tiecut = -1;
-        W.mode = kModeDone;
-      }
-    }
+  if (mode == kModeKeys) {  // not reached: eight 32-way levels split 32 bits
+    atomicOr(a.err, kErrInternal);
+    t_key = 0xFFFFFFFFu;
+    tiecut = -1;
+    mode = kModeDone;
   }
 
   // ---- exact ties: the cutoff is the n_need-th tied position in ascending order
-  {
-    const int need = S.row[x.ra].mode == kModeTie || S.row[x.rb].mode == kModeTie;
-    if (__syncthreads_or(need)) {
-      bool mine[2];
-      uint32_t tk[2];
+  if (__syncthreads_or(mode == kModeTie)) {
+    const bool mine = mode == kModeTie;
+    unsigned long long before = 0ull;
+    bool found = false;
+    W.run(ntiles, [&](int64_t t, const float* s) {
+      if (!mine || found) return;
+      const int lim = causal_lim(pos, t);
 #pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        const RowS& R = S.row[sl ? x.rb : x.ra];
-        mine[sl] = R.mode == kModeTie;
-        tk[sl] = R.t_key;
-      }
-      idx_walk(S.st, ibase, x.nkeys, [&](int64_t t, int stage) {
-        float c[8][4];
-        idx_scores(c, qh, ql, S.st, stage);
-        unsigned long long mk[2] = {0ull, 0ull};
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int p = 8 * nt + 2 * x.tq + e;
-            const int64_t j = t * kIdxKeys + p;
-#pragma unroll
-            for (int sl = 0; sl < 2; ++sl) {
-              const float s = c[nt][2 * sl + e];
-              if (mine[sl] && j <= (sl ? x.pb : x.pa) && order_key(s) == tk[sl])
-                mk[sl] |= 1ull << p;
-            }
+      for (int c = 0; c < kKeysR; ++c) {
+        if (c <= lim && order_key(s[c]) == t_key && !found) {
+          if (++before == n_need) {
+            tiecut = (int)(t * kKeysR + c);
+            found = true;
           }
-        }
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 1);
-          mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 2);
-        }
-        if (owner) {
-#pragma unroll
-          for (int sl = 0; sl < 2; ++sl) {
-            if (!mine[sl]) continue;
-            RowS& W = S.row[sl ? x.rb : x.ra];
-            if (W.found) continue;
-            const int cnt = __popcll(mk[sl]);
-            if (W.tie_before + cnt >= W.n_need) {
-              int want = (int)(W.n_need - W.tie_before);
-              unsigned long long v = mk[sl];
-              while (--want > 0) v &= v - 1;  // drop the lowest (want - 1) set bits
-              W.tiecut = (int)(t * kIdxKeys + (__ffsll((long long)v) - 1));
-              W.found = 1;
-            }
-            W.tie_before += cnt;
-          }
-        }
-      });
-      if (owner) {
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          if (!mine[sl]) continue;
-          RowS& W = S.row[sl ? x.rb : x.ra];
-          if (!W.found) {
-            atomicOr(a.err, kErrInternal);
-            W.tiecut = 0x7FFFFFFF;
-          } else {
-            W.above += (unsigned long long)W.n_need * mass64(key_to_float(W.t_key), m[sl], scale);
-          }
-          W.mode = kModeDone;
         }
       }
+    });
+    if (mine) {
+      if (!found) {
+        atomicOr(a.err, kErrInternal);
+        tiecut = 0x7FFFFFFF;
+      } else {
+        above += n_need * mass64(key_to_float(t_key), m, scale);
+      }
+      mode = kModeDone;
     }
   }
 
-  if (owner) {
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      const int r = sl ? x.rb : x.ra;
-      if ((sl ? x.pb : x.pa) < 0) continue;
-      const RowS& W = S.row[r];
-      cut[r] = make_uint2(W.t_key, (uint32_t)W.tiecut);
-      if (a.sel_mass)
-        a.sel_mass[((int64_t)b * a.C + i0 + r) * a.Hr + hr] = (float)((double)W.above / (double)W.Z);
-    }
+  if (!W.ok) {
+    W.drain();
+    if (tid == 0) atomicOr(a.err, kErrTimeout);
+  } else if (live) {
+    cut[tid] = make_uint2(t_key, (uint32_t)tiecut);
+    if (mass_out) *mass_out = (float)((double)above / (double)Z);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_free(tmem, kSelTmemCols);
   }
 }
 
 // ------------------------------------------------------------------ sparse attention
 
-struct SmemAttn {
-  IdxRing st;                             // 12 KB
-  unsigned char kv[2][2 * kFaTileBytes];  // 64 KB: gathered K and V rows of two chunks in flight
-  uint32_t cm[kRows][4];                  // per-row bits of the (up to 128) filling slots
-  int32_t jl[128];                        // filling slot -> key position
-  uint32_t cmc[2][kRows][2];              // per-row bits of the two issued chunks
-  int32_t jlc[2][64];                     // their key positions
-  unsigned long long wun[2][4];           // per-warp union of a tile's row masks (two tiles)
-  int32_t lslot[kRows];                   // row -> its entry in the listed rows (-1: not listed)
-};
+constexpr int kAttThreads = 256;          // two threads per row
+constexpr uint32_t kAttTmemCols = 256;    // index scores [0,64), S [64,128), O [128,256)
+constexpr uint32_t kColIdx = 0, kColS = 64, kColO = 128;
+constexpr float kRescale = 11.f;          // log2 headroom before the reference max moves (P <= 2^11)
+constexpr uint32_t kIdxStages = 3;
+constexpr uint32_t kAOffQ = 0;                                  // Q tile (128-byte swizzle), 32 KB
+constexpr uint32_t kAOffIQ = kAOffQ + kRowsR * 256;              // index query tile, 8 KB
+constexpr uint32_t kAOffIK = kAOffIQ + kTcQBytes;                // index key ring, 3 x 4 KB
+constexpr uint32_t kAOffK = kAOffIK + kIdxStages * kTcKBytes;    // K tile, 16 KB
+constexpr uint32_t kAOffV = kAOffK + kKeysR * 256;               // V tile, 16 KB
+constexpr uint32_t kAOffP = kAOffV + kKeysR * 256;               // P tile, 16 KB
+constexpr uint32_t kAOffX = kAOffP + kRowsR * 128;               // mask exchange [2][128] u32, count [128]
+constexpr uint32_t kAOffBar = kAOffX + 3 * kRowsR * 4;           // ifull[3], idone, kfull, vfull, sdone, odone
+constexpr uint32_t kAttSmem = kAOffBar + 8 * 8 + 16;
+static_assert(kAOffK % 1024 == 0 && kAOffV % 1024 == 0 && kAOffP % 1024 == 0, "swizzled tiles need 1 KB alignment");
+constexpr uint32_t kKVTileBytes = kKeysR * 256;
 
-__global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  SmemAttn& S = *reinterpret_cast<SmemAttn*>(smem_raw);
+__device__ __forceinline__ uint32_t pack_half2_r(float x, float y) {
+  __half2 h = __floats2half2_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
+                                                                       const __grid_constant__ CUtensorMap tm_idx,
+                                                                       const __grid_constant__ CUtensorMap tm_k,
+                                                                       const __grid_constant__ CUtensorMap tm_v) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const uint32_t sbase = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int half = tid >> 7, r = tid & (kRowsR - 1);
   const int tile = gridDim.x - 1 - blockIdx.x, hr = blockIdx.y, b = blockIdx.z;  // longest rows first
-  const int i0 = tile * kRows;
-  const int nrows = min(kRows, a.C - i0);
-  const RowCtx x = row_ctx(a, i0, nrows);
-  const int tid = x.tid;
-  const bool owner = x.tq == 0;
+  const int i0 = tile * kRowsR;
+  const int nrows = min(kRowsR, a.C - i0);
+  const bool live = r < nrows;
+  const int64_t pos = live ? a.P0 + i0 + r : -1;
+  const int64_t nkeys = a.P0 + i0 + nrows;
+  const int64_t nt = (nkeys + kKeysR - 1) / kKeysR;
   const int h = a.ret_head[hr], g = h / a.group;
-  const __half* ibase = a.idx + ((int64_t)b * a.Hr + hr) * a.max_seq * (2 * kR);
-  const __half* kb = a.kc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
-  const __half* vb = a.vc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
   const int64_t qs = (int64_t)a.Hq * kD;
+  const int64_t idx_row0 = ((int64_t)b * a.Hr + hr) * a.max_seq;
+  const int64_t kv_row0 = ((int64_t)b * a.Hkv + g) * a.max_seq;
+  const uint32_t barI = sbase + kAOffBar, barIdone = barI + 24, barK = barI + 32, barV = barI + 40,
+                 barS = barI + 48, barO = barI + 56;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kAOffBar + 64);
+  uint32_t* xm = reinterpret_cast<uint32_t*>(sm + kAOffX);  // [2][128]: half 1's masks of a tile
+  int32_t* xcnt = reinterpret_cast<int32_t*>(sm + kAOffX + 2 * kRowsR * 4);
 
-  uint32_t qh[4], ql[4];
+  if (sbase & 1023u) {  // the swizzle is a function of address bits: tiles on 1 KB boundaries
+    if (tid == 0) atomicOr(a.err, kErrInternal);
+    return;
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kAttTmemCols);
+  if (tid == 0) {
+    for (int i = 0; i < 8; ++i) mbar_init(barI + 8u * i, 1);
+    fence_mbar_init();
+  }
+  // query rows: RoPE'd q as fp16 into the swizzled Q tile (each half writes 8 of the row's 16
+  // chunks); the index queries (hi | lo) into the index query tile (half 0)
   {
-    const int64_t is = (int64_t)a.Hr * kR;
-    const float* q0 = a.q_idx + ((int64_t)b * a.C + i0) * is + (int64_t)hr * kR;
-    idx_load_q(qh, ql, x.pa >= 0 ? q0 + x.ra * is : nullptr, x.pb >= 0 ? q0 + x.rb * is : nullptr);
-  }
-  const uint2* cut = a.cut + ((int64_t)b * a.Hr + hr) * a.C + i0;
-  uint32_t tk[2];
-  int64_t tc[2];
-  {
-    const uint2 ca = x.pa >= 0 ? cut[x.ra] : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-    const uint2 cbv = x.pb >= 0 ? cut[x.rb] : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-    tk[0] = ca.x;
-    tc[0] = (int32_t)ca.y;
-    tk[1] = cbv.x;
-    tc[1] = (int32_t)cbv.y;
-  }
-  uint32_t* brow[2] = {nullptr, nullptr};
-  if (a.bitmap && owner) {
-    if (x.pa >= 0) brow[0] = a.bitmap + (((int64_t)b * a.C + i0 + x.ra) * a.Hr + hr) * a.bitmap_words;
-    if (x.pb >= 0) brow[1] = a.bitmap + (((int64_t)b * a.C + i0 + x.rb) * a.Hr + hr) * a.bitmap_words;
-  }
-
-  uint32_t qa[8][4];
-  fa_load_q(qa, a.q_rot + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD, qs, x.warp * 16, nrows);
-  FaAcc A;
-  fa_init(A);
-
-  for (int i = tid; i < kRows * 4; i += kThreads) (&S.cm[0][0])[i] = 0u;
-  for (int i = tid; i < kRows; i += kThreads) S.lslot[i] = -1;
-  __syncthreads();
-  for (int i = tid; i < a.n_rows; i += kThreads) {
-    const int r = a.rows[i] - i0;
-    if (r >= 0 && r < nrows) S.lslot[r] = i;
-  }
-  __syncthreads();
-  int32_t* lrow[2] = {nullptr, nullptr};  // this owner's listed rows: where their positions go
-  if (a.row_sel && owner) {
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      const int r = sl ? x.rb : x.ra;
-      const int li = (sl ? x.pb : x.pa) >= 0 ? S.lslot[r] : -1;
-      if (li >= 0) lrow[sl] = a.row_sel + (((int64_t)b * a.n_rows + li) * a.Hr + hr) * a.row_sel_cap;
+    const float* qrow = a.q_rot + ((int64_t)b * a.C + i0 + (live ? r : 0)) * qs + (int64_t)h * kD;
+#pragma unroll 4
+    for (int cc = 0; cc < 8; ++cc) {
+      const int c = 8 * half + cc;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (live) {
+        const float4 x0 = *reinterpret_cast<const float4*>(qrow + 8 * c);
+        const float4 x1 = *reinterpret_cast<const float4*>(qrow + 8 * c + 4);
+        v.x = pack_half2_r(x0.x, x0.y);
+        v.y = pack_half2_r(x0.z, x0.w);
+        v.z = pack_half2_r(x1.x, x1.y);
+        v.w = pack_half2_r(x1.z, x1.w);
+      }
+      *reinterpret_cast<uint4*>(sm + kAOffQ + sw128_off(r, c, kRowsR)) = v;
+    }
+    if (half == 0) {
+      const float* iq = a.q_idx + (((int64_t)b * a.C + i0 + (live ? r : 0)) * a.Hr + hr) * kR;
+      tc_put_query(sm + kAOffIQ, r, live ? iq : nullptr);
     }
   }
-  int fill = 0;
-  int nsel[2] = {0, 0};
+  // this row's cut
+  uint32_t tk = 0xFFFFFFFFu;
+  int64_t tcut = -1;
+  if (live) {
+    const uint2 cv = a.cut[((int64_t)b * a.Hr + hr) * a.C + i0 + r];
+    tk = cv.x;
+    tcut = (int32_t)cv.y;
+  }
+  // outputs of the selection statistics
+  uint32_t* brow = (a.bitmap && live) ? a.bitmap + (((int64_t)b * a.C + i0 + r) * a.Hr + hr) * a.bitmap_words : nullptr;
+  int32_t* lrow = nullptr;  // a listed row: where half 0 writes its positions
+  if (a.row_sel && live && half == 0) {
+    for (int i = 0; i < a.n_rows; ++i)
+      if (a.rows[i] == i0 + r) lrow = a.row_sel + (((int64_t)b * a.n_rows + i) * a.Hr + hr) * a.row_sel_cap;
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
 
-  // Chunks are double-buffered: issuing chunk n starts its K/V gather, and only then is chunk
-  // n - 1 (gathered meanwhile) run through the attention tile.
-  int pend = -1;  // buffer of the issued chunk not yet attended (-1: none)
-  int nbuf = 0;   // buffer the next chunk goes to
-  auto attend = [&](int buf) {
-    fa_tile(A, qa, S.kv[buf], S.kv[buf] + kFaTileBytes, a.scale_log2,
-            [&](int r, int tt) { return ((S.cmc[buf][r][tt >> 5] >> (tt & 31)) & 1u) != 0u; });
+  // phase counters of the mbarriers (each completion is waited exactly once, in order)
+  uint32_t n_idone = 0, n_k = 0, n_v = 0, n_s = 0, n_o = 0;
+  bool okw = true, ok = true, any_pv = false;
+  auto ikt = [&](int64_t t) { return sbase + kAOffIK + (uint32_t)(t % kIdxStages) * kTcKBytes; };
+  auto load_kv = [&](uint32_t bar, uint32_t dst, const CUtensorMap* map, int64_t t) {
+    mbar_expect_tx(bar, kKVTileBytes);
+    const int y = (int)(kv_row0 + t * kKeysR);
+    tma_load_2d(dst, map, 0, y, bar);
+    tma_load_2d(dst + kKeysR * 128, map, 64, y, bar);
   };
-  auto issue = [&](int n) {  // move filling slots 0 .. n-1 into a chunk buffer and gather it
-    const int k = nbuf;
-    for (int i = tid; i < kRows; i += kThreads) {
-      S.cmc[k][i][0] = S.cm[i][0];
-      S.cmc[k][i][1] = S.cm[i][1];
-      S.cm[i][0] = S.cm[i][2];
-      S.cm[i][1] = S.cm[i][3];
-      S.cm[i][2] = S.cm[i][3] = 0u;
+  // this thread's selection mask of tile t (its 32 columns) from the index scores in TMEM
+  auto read_mask = [&](int64_t t) -> uint32_t {
+    okw = mbar_wait(barIdone, n_idone & 1u) && okw;
+    ++n_idone;
+    tc_fence_after();
+    __syncwarp();
+    float s[32];
+    tmem_ld32(lane_addr + kColIdx + 32u * half, s);
+    tmem_ld_wait();
+    const int lim = causal_lim(pos, t) - 32 * half;
+    uint32_t mk = 0u;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int64_t j = t * kKeysR + 32 * half + i;
+      const uint32_t key = order_key(s[i] + 0.0f);
+      const bool sel = i <= lim && (key > tk || (key == tk && j <= tcut));
+      mk |= (uint32_t)sel << i;
     }
-    if (tid < 64) {
-      S.jlc[k][tid] = tid < n ? S.jl[tid] : 0;
-      S.jl[tid] = S.jl[64 + tid];
-    }
+    return mk;
+  };
+  // exchange one float per row between the two halves through TMEM columns of the S buffer
+  // that both have already read
+  auto swap_half = [&](float v) -> float {
+    float w[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] = v;
+    __syncwarp();
+    tmem_st32(lane_addr + kColS + 32u * half, w);
+    tmem_st_wait();
+    tc_fence_before();
     __syncthreads();
-    fa_stage(S.kv[k], S.kv[k] + kFaTileBytes, kb, vb, n, [&](int r) { return (int64_t)S.jlc[k][r]; });
-    cp_async_commit();
-    if (pend >= 0) {
-      cp_async_wait<1>();  // everything but this chunk's gather has landed
-      __syncthreads();
-      attend(pend);
-      __syncthreads();
-    }
-    pend = k;
-    nbuf ^= 1;
+    tc_fence_after();
+    tmem_ld32(lane_addr + kColS + 32u * (1 - half), w);
+    tmem_ld_wait();
+    return w[0];
   };
 
-  // The union of tile t is published in shared memory and appended to the chunk during tile
-  // t + 1, after that tile's ring barrier: one barrier per tile.
-  unsigned long long own_prev[2] = {0ull, 0ull};
-  auto append = [&](int64_t t) {  // tile t's union keys -> chunk slots fill, fill + 1, ...
-    const int pb = (int)(t & 1);
-    const unsigned long long U = S.wun[pb][0] | S.wun[pb][1] | S.wun[pb][2] | S.wun[pb][3];
-    if (U == 0ull) return;  // uniform: no row selects a key of this tile
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      unsigned long long v = own_prev[sl];
-      const int r = sl ? x.rb : x.ra;
-      while (v) {
-        const int p = __ffsll((long long)v) - 1;
+  // ---- prologue: index key tiles 0..2 in flight, the scores of tile 0, its masks
+  if (tid == 0) {
+    for (int64_t i = 0; i < (int64_t)kIdxStages && i < nt; ++i)
+      tc_load_keys(ikt(i), &tm_idx, idx_row0, i, barI + 8u * (uint32_t)i);
+    okw = mbar_wait(barI, 0u);
+    if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(0), barIdone);
+  }
+  uint32_t mask_cur = read_mask(0);
+  tc_fence_before();
+  if (half == 1) xm[r] = mask_cur;
+  bool any_cur = __syncthreads_or(mask_cur != 0u) != 0;
+  ok = __syncthreads_and(okw ? 1 : 0) != 0;
+  if (ok && tid == 0) {
+    if (nt > 1) {
+      okw = mbar_wait(barI + 8u, 0u);
+      if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(1), barIdone);
+    }
+    if (nt > 3) tc_load_keys(ikt(3), &tm_idx, idx_row0, 3, barI);  // stage 0: tile 0 is scored
+    if (any_cur) load_kv(barK, sbase + kAOffK, &tm_k, 0);
+  }
+
+  float m_ref = -INFINITY, l = 0.f;  // reference max of row r; this half's share of the sum
+  int nsel = 0;
+  int64_t lbase = 0;  // listed positions written so far (half 0 of a listed row)
+  for (int64_t t = 0; ok && t < nt; ++t) {
+    // ---- statistics of tile t: count, bitmap words, listed positions
+    nsel += __popc(mask_cur);
+    if (brow) {
+      const int64_t w = 2 * t + half;
+      if (w < a.bitmap_words) brow[w] = mask_cur;
+    }
+    if (lrow) {  // half 0 writes both halves' positions, ascending
+      uint32_t v = mask_cur;
+      while (v && lbase < a.row_sel_cap) {
+        const int p = __ffs(v) - 1;
         v &= v - 1;
-        const int slot = fill + __popcll(U & ((1ull << p) - 1ull));
-        atomicOr(&S.cm[r][slot >> 5], 1u << (slot & 31));
+        lrow[lbase++] = (int32_t)(t * kKeysR + p);
+      }
+      v = xm[(t & 1) * kRowsR + r];
+      while (v && lbase < a.row_sel_cap) {
+        const int p = __ffs(v) - 1;
+        v &= v - 1;
+        lrow[lbase++] = (int32_t)(t * kKeysR + 32 + p);
       }
     }
-    if (tid < 64 && ((U >> tid) & 1ull))
-      S.jl[fill + __popcll(U & ((1ull << tid) - 1ull))] = (int32_t)(t * kIdxKeys + tid);
-    fill += __popcll(U);
-    if (fill >= 64) {
-      __syncthreads();  // every slot of the chunk is written
-      issue(64);
-      fill -= 64;
-    }
-  };
-
-  idx_walk(S.st, ibase, x.nkeys, [&](int64_t t, int stage) {
-    if (t > 0) append(t - 1);
-    float c[8][4];
-    idx_scores(c, qh, ql, S.st, stage);
-    const int64_t base = t * kIdxKeys;
-    const int la = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pa - base));
-    const int lb = (int)max((int64_t)-1, min((int64_t)(kIdxKeys - 1), x.pb - base));
-    const int ca = (int)max((int64_t)-1, min((int64_t)kIdxKeys, tc[0] - base));
-    const int cbt = (int)max((int64_t)-1, min((int64_t)kIdxKeys, tc[1] - base));
-    unsigned long long mk[2] = {0ull, 0ull};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int p = 8 * nt + 2 * x.tq + e;
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          const uint32_t key = order_key(c[nt][2 * sl + e]);
-          const int lim = sl ? lb : la, cut_p = sl ? cbt : ca;
-          const bool sel = p <= lim && (key > tk[sl] || (key == tk[sl] && p <= cut_p));
-          mk[sl] |= (unsigned long long)sel << p;
-        }
+    // ---- (a) the masks of tile t + 1 (scored one tile ahead); the scores of tile t + 2
+    uint32_t mask_next = 0u;
+    bool any_next = false;
+    if (t + 1 < nt) {
+      mask_next = read_mask(t + 1);
+      tc_fence_before();
+      if (half == 1) xm[((t + 1) & 1) * kRowsR + r] = mask_next;
+      any_next = __syncthreads_or(mask_next != 0u) != 0;
+      if (tid == 0 && t + 2 < nt && okw) {
+        okw = mbar_wait(barI + 8u * (uint32_t)((t + 2) % kIdxStages), (uint32_t)(((t + 2) / kIdxStages) & 1));
+        if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(t + 2), barIdone);
+        if (t + 4 < nt)  // the stage of tile t + 1 is free: its scores are done
+          tc_load_keys(ikt(t + 4), &tm_idx, idx_row0, t + 4, barI + 8u * (uint32_t)((t + 4) % kIdxStages));
       }
     }
-    own_prev[0] = mk[0];  // this thread's selected keys, appended during the next tile
-    own_prev[1] = mk[1];
+    // ---- (b) attention over tile t
+    if (any_cur) {
+      if (tid == 0) {
+        if (any_pv && okw) okw = mbar_wait(barO, (n_o - 1) & 1u);  // V and P are free
+        if (okw) load_kv(barV, sbase + kAOffV, &tm_v, t);
+        if (okw) okw = mbar_wait(barK, n_k & 1u);
+        if (okw) {
+          tc_fence_after();
+          constexpr uint32_t kIdS = umma_idesc_f16(kKeysR, false);
 #pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-      mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 1);
-      mk[sl] |= __shfl_xor_sync(0xffffffffu, mk[sl], 2);
-    }
-    if (owner) {
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        if (lrow[sl]) {  // a listed row: its positions, ascending (tiles come in order)
-          unsigned long long v = mk[sl];
-          int n = nsel[sl];
-          while (v && n < a.row_sel_cap) {
-            const int p = __ffsll((long long)v) - 1;
-            v &= v - 1;
-            lrow[sl][n++] = (int32_t)(t * kIdxKeys + p);
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t ad = umma_desc(sbase + kAOffQ + (kk >> 2) * (kRowsR * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = umma_desc(sbase + kAOffK + (kk >> 2) * (kKeysR * 128) + (kk & 3) * 32, 16, 1024);
+            umma_f16(tmem + kColS, ad, bd, kIdS, kk > 0 ? 1u : 0u);
           }
+          umma_commit(barS);
         }
-        nsel[sl] += __popcll(mk[sl]);
-        if (brow[sl]) {
-          const int64_t w = 2 * t;
-          if (w < a.bitmap_words) brow[sl][w] = (uint32_t)mk[sl];
-          if (w + 1 < a.bitmap_words) brow[sl][w + 1] = (uint32_t)(mk[sl] >> 32);
+      }
+      ++n_k;
+      okw = mbar_wait(barS, n_s & 1u) && okw;
+      ++n_s;
+      tc_fence_after();
+      __syncwarp();
+      float sv[32];
+      tmem_ld32(lane_addr + kColS + 32u * half, sv);
+      tmem_ld_wait();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        sv[i] = ((mask_cur >> i) & 1u) ? sv[i] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sv[i]);
+      }
+      mx = fmaxf(mx, swap_half(mx));  // the row max over both halves (also orders the S reads)
+      // S of tile t is done, and so is P V of the previous tile: K, P and O are free
+      if (tid == 0 && any_next && okw) load_kv(barK, sbase + kAOffK, &tm_k, t + 1);
+      const bool move = mx > m_ref + kRescale;
+      if (any_pv && __any_sync(0xffffffffu, move)) {
+        const float cf = move ? fast_exp2(m_ref - mx) : 1.f;  // warp-collective ld / st below
+        const uint32_t oAddr = lane_addr + kColO + 64u * half;
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          float ov[32];
+          tmem_ld32(oAddr + c0, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= cf;
+          tmem_st32(oAddr + c0, ov);
+        }
+        tmem_st_wait();
+      }
+      if (move) {
+        l *= fast_exp2(m_ref - mx);  // 0 while m_ref is still -inf
+        m_ref = mx;
+      }
+      float rs = 0.f;
+      const float mref = m_ref == -INFINITY ? 0.f : m_ref;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float pv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pv[e] = fast_exp2(sv[8 * q + e] - mref);
+          rs += pv[e];
+        }
+        uint4 w;
+        w.x = pack_half2_r(pv[0], pv[1]);
+        w.y = pack_half2_r(pv[2], pv[3]);
+        w.z = pack_half2_r(pv[4], pv[5]);
+        w.w = pack_half2_r(pv[6], pv[7]);
+        *reinterpret_cast<uint4*>(sm + kAOffP + sw128_off(r, 4 * half + q, kRowsR)) = w;
+      }
+      l += rs;
+      fence_async_smem();
+      tc_fence_before();
+      ok = __syncthreads_and(okw ? 1 : 0) != 0;
+      if (!ok) break;
+      // ---- O += P V (one thread); V is read MN-major (rows = keys)
+      if (tid == 0) {
+        okw = mbar_wait(barV, n_v & 1u);
+        if (okw) {
+          tc_fence_after();
+          constexpr uint32_t kIdO = umma_idesc_f16(kD, true);
+#pragma unroll
+          for (int kk = 0; kk < kKeysR / 16; ++kk) {
+            const uint64_t ad = umma_desc(sbase + kAOffP + kk * 32, 16, 1024);
+            const uint64_t bd = umma_desc(sbase + kAOffV + kk * 2048, kKeysR * 128, 1024);
+            umma_f16(tmem + kColO, ad, bd, kIdO, (any_pv || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(barO);
+        }
+      }
+      ++n_v;
+      ++n_o;
+      any_pv = true;
+    } else if (tid == 0 && any_next && okw) {
+      load_kv(barK, sbase + kAOffK, &tm_k, t + 1);  // K is free: every earlier S has completed
+    }
+    mask_cur = mask_next;
+    any_cur = any_next;
+    ok = __syncthreads_and(okw ? 1 : 0) != 0;
+  }
+
+  if (ok && any_pv) {
+    if (tid == 0) okw = mbar_wait(barO, (n_o - 1) & 1u);
+    ok = __syncthreads_and(okw ? 1 : 0) != 0;
+  }
+  if (ok) {
+    tc_fence_after();
+    const float lt = l + swap_half(l);
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+    float* orow = a.out + ((int64_t)b * a.C + i0 + (live ? r : 0)) * qs + (int64_t)h * kD + 64 * half;
+    const uint32_t oAddr = lane_addr + kColO + 64u * half;
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+      float ov[32];
+      tmem_ld32(oAddr + c0, ov);
+      tmem_ld_wait();
+      if (live) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (any_pv) o4 = make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+          *reinterpret_cast<float4*>(orow + c0 + i) = o4;
         }
       }
     }
-    unsigned long long u = mk[0] | mk[1];
-    u |= __shfl_xor_sync(0xffffffffu, u, 4);
-    u |= __shfl_xor_sync(0xffffffffu, u, 8);
-    u |= __shfl_xor_sync(0xffffffffu, u, 16);
-    if ((tid & 31) == 0) S.wun[t & 1][x.warp] = u;
-  });
-  {
-    const int64_t ntiles = (x.nkeys + kIdxKeys - 1) / kIdxKeys;  // the walk ended with a barrier
-    append(ntiles - 1);
-  }
-  __syncthreads();
-  if (fill > 0) issue(fill);
-  if (pend >= 0) {
-    cp_async_wait<0>();
+    // selected counts: half 1 hands its count to half 0
+    if (half == 1) xcnt[r] = nsel;
     __syncthreads();
-    attend(pend);
+    if (half == 0 && live && a.sel_count) a.sel_count[((int64_t)b * a.C + i0 + r) * a.Hr + hr] = nsel + xcnt[r];
+  } else if (tid == 0) {
+    atomicOr(a.err, kErrTimeout);
+    // wait (bounded) for the copies and MMAs this CTA may still have in flight: the next
+    // phase of every barrier that has one pending
+    mbar_wait(barIdone, n_idone & 1u);
+    mbar_wait(barS, n_s & 1u);
+    if (any_pv) mbar_wait(barO, (n_o - 1) & 1u);
   }
-  fa_store(A, a.out + ((int64_t)b * a.C + i0) * qs + (int64_t)h * kD, qs, x.warp * 16, nrows);
-  if (a.sel_count && owner) {
-    if (x.pa >= 0) a.sel_count[((int64_t)b * a.C + i0 + x.ra) * a.Hr + hr] = nsel[0];
-    if (x.pb >= 0) a.sel_count[((int64_t)b * a.C + i0 + x.rb) * a.Hr + hr] = nsel[1];
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_free(tmem, kAttTmemCols);
   }
 }
 
@@ -796,10 +826,8 @@ __global__ void __launch_bounds__(kThreads) prefill_attn_kernel(RetArgs a) {
 
 cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,
                                      cudaStream_t st) {
+  if (!L->tm_ready) return cudaErrorInvalidValue;
   RetArgs a;
-  a.idx = L->idx_hl;
-  a.kc = L->kc;
-  a.vc = L->vc;
   a.max_seq = L->max_seq;
   a.Hkv = L->Hkv;
   a.Hq = L->Hq;
@@ -821,28 +849,26 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
   a.sel_mass = stats ? stats->sel_mass : nullptr;
   a.bitmap = stats ? stats->sel_bitmap : nullptr;
   a.bitmap_words = stats ? stats->bitmap_words : 0;
-  a.rows = stats ? stats->rows : nullptr;
+  a.rows = (stats && stats->rows) ? stats->rows : nullptr;
   a.n_rows = (stats && stats->rows) ? stats->n_rows : 0;
   a.row_sel = (stats && stats->rows) ? stats->row_sel : nullptr;
   a.row_sel_cap = (stats && stats->rows) ? stats->row_sel_cap : 0;
   a.err = L->err;
-  dim3 grid((C + kRows - 1) / kRows, L->Hr, L->B);
+  dim3 grid((C + kRowsR - 1) / kRowsR, L->Hr, L->B);
   cudaError_t e;
   {
     ProfScope ps(L, "prefill_select", st);
-    e = cudaFuncSetAttribute(prefill_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(SmemSel));
+    e = cudaFuncSetAttribute(prefill_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelSmem);
     if (e != cudaSuccess) return e;
-    prefill_select_kernel<<<grid, kThreads, sizeof(SmemSel), st>>>(a);
+    prefill_select_kernel<<<grid, kPsThreads, kSelSmem, st>>>(a, L->tm_idx);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   {
     ProfScope ps(L, "prefill_attn", st);
-    e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(SmemAttn));
+    e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttSmem);
     if (e != cudaSuccess) return e;
-    prefill_attn_kernel<<<grid, kThreads, sizeof(SmemAttn), st>>>(a);
+    prefill_attn_kernel<<<grid, kAttThreads, kAttSmem, st>>>(a, L->tm_idx, L->tm_k, L->tm_v);
     e = cudaGetLastError();
   }
   return e;

@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "rtp.h"
+#include "tma.cuh"
 
 namespace rtp {
 
@@ -57,6 +58,11 @@ struct rtp_layer {
   int32_t* d_loc_cnt = nullptr;    // [Hkv]
   int16_t* d_local_list = nullptr; // [n_local] local q heads, ascending
   __half* idx_hl = nullptr;        // [B][Hr][max_seq][2 r]: index keys split as fp16 hi | lo
+  // TMA tensor maps of the prefill kernels: the split index cache as [rows][4 chunks][8 values]
+  // (64-key boxes per chunk), the K and V caches as [rows][128 values] (64-key x 64-value boxes,
+  // 128-byte swizzle)
+  CUtensorMap tm_idx, tm_k, tm_v;
+  bool tm_ready = false;
   uint2* pf_cut = nullptr;
   // decode: the local heads' window attention runs on a second stream, forked after the
   // selection and joined back, so it overlaps the retrieval heads' gather attention

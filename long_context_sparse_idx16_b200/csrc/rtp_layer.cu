@@ -262,6 +262,24 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
     if (e == cudaSuccess && !local_list.empty())
       e = cudaMemcpy(L->d_local_list, local_list.data(), sizeof(int16_t) * local_list.size(), cudaMemcpyHostToDevice);
   }
+  // tensor maps of the prefill kernels (the caches never move)
+  {
+    const uint64_t kv_rows = (uint64_t)(B * Hkv * L->max_seq);
+    const uint64_t kv_dims[2] = {(uint64_t)kD, kv_rows}, kv_str[1] = {(uint64_t)kD * 2};
+    const uint32_t kv_box[2] = {64u, 64u};
+    bool okm = tma_encode(&L->tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, L->kc, kv_dims, kv_str, kv_box,
+                          CU_TENSOR_MAP_SWIZZLE_128B) &&
+               tma_encode(&L->tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, L->vc, kv_dims, kv_str, kv_box,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    if (okm && Hr > 0) {
+      const uint64_t idx_dims[3] = {8u, 4u, (uint64_t)(P * L->max_seq)}, idx_str[2] = {16u, (uint64_t)(4 * kR)};
+      const uint32_t idx_box[3] = {8u, 1u, 64u};
+      okm = tma_encode(&L->tm_idx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, L->idx_hl, idx_dims, idx_str, idx_box,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    L->tm_ready = okm;
+    if (!okm && e == cudaSuccess) e = cudaErrorInvalidValue;
+  }
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_fork, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_join, cudaEventDisableTiming);

@@ -16,7 +16,7 @@ def small(name="prefill_32k", **kw):
 
 
 def test_prefill_small_from_empty():
-    # 300 rows = four full 64-row tiles and a ragged tail of 44; keys 0..299
+    # 300 rows = two full 128-row tiles and a ragged tail of 44; keys 0..299
     run_prefill(small())
 
 
@@ -88,7 +88,7 @@ def test_prefill_deterministic():
     assert np.array_equal(a, b)
 
 
-def _spread_rows(C: int, n: int, seed: int, tile: int = 64) -> np.ndarray:
+def _spread_rows(C: int, n: int, seed: int, tile: int = 128) -> np.ndarray:
     """n distinct chunk rows: the first and last two, pairs across row-tile boundaries spread
     over the chunk, and seeded random rows (even and odd rows alike)."""
     rows = {0, 1, C - 2, C - 1}
