@@ -26,6 +26,7 @@ Multi-GPU: the layer does not shard; --gpus N runs N independent replicas (one p
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -581,7 +582,8 @@ def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=Non
 
     peak, peak_kind = _peaks()
     P = B * len(s.retrieval_heads)
-    sel_bytes = P * N * s.index_dim * 4  # fp32 index keys streamed per launch
+    key_bytes = 2 if getattr(s, "index_bf16", False) else 4
+    sel_bytes = P * N * s.index_dim * key_bytes  # index keys streamed per launch (fp32 or bf16)
     traffic = _profile_traffic(os.path.join(ROOT, "long_context_sparse_idx16_b200", "csrc", "decode_select.cu"))
     lines = []
     for p in (top_ps or [s.top_p]):
@@ -768,9 +770,12 @@ def measure_prefill(s, x, steps: int, warmup: int, world: int, dev, exp_peak: di
     return line
 
 
-# the workloads measured besides the headline one, with the steps each takes at most (a 1M
-# prefill chunk takes about a second)
-SUB_WORKLOADS = (("decode_1m", None), ("prefill_32k", 5), ("prefill_1m", 3))
+# the workloads measured besides the headline one: (record name, workload, layer options,
+# the steps each takes at most -- a 1M prefill chunk takes about a second -- and the p values)
+SUB_WORKLOADS = (("decode_1m", "decode_1m", {}, None, None),
+                 ("decode_1m_bf16_index", "decode_1m", {"index_bf16": True}, None, (0.9,)),
+                 ("prefill_32k", "prefill_32k", {}, 5, None),
+                 ("prefill_1m", "prefill_1m", {}, 3, None))
 
 
 def run_gpu(args):
@@ -790,13 +795,15 @@ def run_gpu(args):
     cpu = rank == 0 and not args.no_cpu_baseline
     exp_peak = measure_exp_rate(dev)
 
-    def one(name, steps):
+    def one(name, steps, opts=None, ps=None):
         s = _spec(args, name)
+        if opts:
+            s = dataclasses.replace(s, **opts)
         x = synth.generate(s)
         if name in PREFILL_WORKLOADS:
             return [measure_prefill(s, x, steps, args.warmup, world, dev, exp_peak, cpu=cpu)]
-        return measure_decode(s, x, steps, args.warmup, world, dev, top_ps=list(s.p_sweep) if s.p_sweep else None,
-                              cpu=cpu)
+        ps = ps or (list(s.p_sweep) if s.p_sweep else None)
+        return measure_decode(s, x, steps, args.warmup, world, dev, top_ps=list(ps) if ps else None, cpu=cpu)
 
     head = one(args.workload, args.steps)
     main = head[len(head) // 2] if args.workload == "decode_1m" else head[0]  # p = 0.9 of a sweep
@@ -812,12 +819,14 @@ def run_gpu(args):
     if not args.only:
         subs = {}
         total = line["gpu_launches"]
-        for name, cap in SUB_WORKLOADS:
-            if name == args.workload:
+        for rec, name, opts, cap, ps in SUB_WORKLOADS:
+            if name == args.workload and not opts:
                 continue
             steps = args.steps if cap is None else max(1, min(args.steps, cap))
-            for ln in one(name, steps):
-                key = name if "top_p" not in ln or name != "decode_1m" else f"{name}_p{ln['top_p']}"
+            for ln in one(name, steps, opts, ps):
+                key = rec if name not in DECODE_WORKLOADS else f"{rec}_p{ln['top_p']}"
+                if opts:
+                    ln["layer_options"] = opts
                 subs[key] = ln
                 total += ln["gpu_launches"]
         line["workloads"] = subs

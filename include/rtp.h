@@ -75,6 +75,16 @@ typedef struct {
   const float* wk_index;      /* HOST [Hr][D][r] fp32; copied */
   int64_t max_select;         /* capacity of one selected set; 0 selects max_seq */
   int32_t max_chunk;          /* largest prefill chunk C; 0 selects 16384 */
+  int32_t index_bf16;         /* 0: index keys stored in fp32; 1: in bf16, rounded to nearest
+                                 even from an fp64 projection (half the decode index stream;
+                                 the selection then follows the rounded keys) */
+  int32_t prefill_dense;      /* 1: in prefill, retrieval heads attend to every causal key (the
+                                 pages' own prefill, techwalker page Q&A; ngjoo digest,
+                                 limitations); decode keeps its selection.  0: per-row selection */
+  int64_t top_k;              /* 0: top-p selection; k > 0: retrieval heads keep the first
+                                 min(k, n) keys of the order (s desc, j asc) instead -- the
+                                 pages' fixed-budget ablation (techwalker page, section 4);
+                                 sel_mass and threshold are then reported as -1 */
 } rtp_config;
 
 /* Optional decode statistics, DEVICE arrays [B][Hr] (retrieval heads ascending).  Any
@@ -114,9 +124,10 @@ typedef struct {
 typedef struct {
   const void* k;    /* fp16 [B][Hkv][max_seq][D]: RoPE'd keys */
   const void* v;    /* fp16 [B][Hkv][max_seq][D] */
-  const float* idx; /* fp32 [B][Hr][max_seq][r]: pre-RoPE index keys Wk_h^T k_j */
+  const float* idx; /* fp32 [B][Hr][max_seq][r]: pre-RoPE index keys Wk_h^T k_j (NULL with bf16 keys) */
   int64_t max_seq;
   int32_t n_retrieval;
+  const void* idx_bf16; /* bf16 [B][Hr][max_seq][r] when the layer stores bf16 index keys, else NULL */
 } rtp_cache_view;
 
 /* Create a layer on the current CUDA device: validates cfg, allocates the caches and all

@@ -32,7 +32,8 @@ class rtp_config(C.Structure):
         ("head_class", C.c_void_p), ("top_p", C.c_float), ("window", C.c_int32),
         ("n_sink", C.c_int32), ("rope_base", C.c_double), ("sm_scale", C.c_float),
         ("wq_index", C.c_void_p), ("wk_index", C.c_void_p), ("max_select", C.c_int64),
-        ("max_chunk", C.c_int32),
+        ("max_chunk", C.c_int32), ("index_bf16", C.c_int32), ("prefill_dense", C.c_int32),
+        ("top_k", C.c_int64),
     ]
 
 
@@ -49,7 +50,7 @@ class rtp_prefill_stats(C.Structure):
 
 class rtp_cache_view(C.Structure):
     _fields_ = [("k", C.c_void_p), ("v", C.c_void_p), ("idx", C.c_void_p), ("max_seq", C.c_int64),
-                ("n_retrieval", C.c_int32)]
+                ("n_retrieval", C.c_int32), ("idx_bf16", C.c_void_p)]
 
 
 class RTPError(RuntimeError):
@@ -234,7 +235,8 @@ class Layer:
     def __init__(self, *, batch: int, n_q_heads: int, n_kv_heads: int, head_class: Sequence[int],
                  wq: Optional[np.ndarray], wk: Optional[np.ndarray], top_p: float, window: int,
                  n_sink: int, max_seq: int, rope_base: float = 1.0e6, sm_scale: float = 0.0,
-                 max_select: int = 0, max_chunk: int = 0):
+                 max_select: int = 0, max_chunk: int = 0, index_bf16: bool = False,
+                 prefill_dense: bool = False, top_k: int = 0):
         self._hc = np.ascontiguousarray(np.asarray(head_class, dtype=np.uint8))
         self.n_retrieval = int(self._hc.sum())
         self._wq = None if wq is None else np.ascontiguousarray(wq, dtype=np.float32)
@@ -245,7 +247,8 @@ class Layer:
             n_sink=n_sink, rope_base=rope_base, sm_scale=sm_scale,
             wq_index=self._wq.ctypes.data if self._wq is not None else None,
             wk_index=self._wk.ctypes.data if self._wk is not None else None,
-            max_select=max_select, max_chunk=max_chunk)
+            max_select=max_select, max_chunk=max_chunk, index_bf16=1 if index_bf16 else 0,
+            prefill_dense=1 if prefill_dense else 0, top_k=int(top_k))
         self.batch, self.n_q_heads, self.n_kv_heads = batch, n_q_heads, n_kv_heads
         self.handle = rtp_create(cfg)
         import torch
@@ -259,7 +262,9 @@ class Layer:
         wk = inputs.wk if inputs is not None else None
         return cls(batch=spec.batch, n_q_heads=spec.n_q_heads, n_kv_heads=spec.n_kv_heads,
                    head_class=spec.head_class, wq=wq, wk=wk, top_p=spec.top_p, window=spec.window,
-                   n_sink=spec.n_sink, max_seq=max_seq or spec.n_total, rope_base=spec.rope_base, **kw)
+                   n_sink=spec.n_sink, max_seq=max_seq or spec.n_total, rope_base=spec.rope_base,
+                   index_bf16=getattr(spec, "index_bf16", False),
+                   prefill_dense=getattr(spec, "prefill_dense", False), top_k=getattr(spec, "top_k", 0), **kw)
 
     def close(self) -> None:
         if getattr(self, "handle", None):

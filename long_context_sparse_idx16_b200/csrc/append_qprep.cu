@@ -2,8 +2,9 @@
 //
 // Append (rtp_append_kv): for each new token at position pos and KV head g,
 //   K[g][pos] = fp16(RoPE(k, pos)), V[g][pos] = fp16(v), and for every retrieval head h
-//   whose KV head is g: IDX[h][pos] = Wk_h^T k (pre-RoPE, fp32), also kept split as fp16
-//   hi + lo for the tensor-core scoring of prefill.
+//   whose KV head is g: IDX[h][pos] = Wk_h^T k (pre-RoPE; stored in fp32, or in bf16 when the
+//   layer keeps bf16 index keys), also kept split as fp16 hi + lo for the tensor-core scoring
+//   of prefill.
 // The indexer projects pre-RoPE keys (ngjoo digest, core method: "low-dimensional pre-RoPE
 // projections"; aitntnews page, finding 2: project D=128 down to r=16 so that the
 // high-frequency RoPE components do not disturb long-range matching).
@@ -25,11 +26,12 @@ constexpr float kFp16Max = 65504.f;
 // Retrieval heads whose index weights are staged in shared memory at once (8 KB each).
 constexpr int kWHeads = 8;
 
+template <bool kBf16>
 __global__ void __launch_bounds__(256) append_kv_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int T, int Hkv,
     int Hr, int64_t pos0, int64_t max_seq, const double* __restrict__ theta,
     const float* __restrict__ wk, const int16_t* __restrict__ ret_head, int group,
-    __half* __restrict__ kc, __half* __restrict__ vc, float* __restrict__ idx,
+    __half* __restrict__ kc, __half* __restrict__ vc, float* __restrict__ idx, __nv_bfloat16* __restrict__ idx_b,
     __half* __restrict__ idx_hl, uint32_t* __restrict__ err) {
   const int t = blockIdx.x;  // token within the appended block
   const int b = blockIdx.y;
@@ -81,11 +83,23 @@ __global__ void __launch_bounds__(256) append_kv_kernel(
       const int hl = o / kR, c = o % kR, hr = h0 + hl;
       const float* w = ws + hl * kD * kR + c;
       const float* x = ks + (ret_head[hr] / group) * kD;
-      float acc = 0.f;
-#pragma unroll 16
-      for (int d = 0; d < kD; ++d) acc = fmaf(w[d * kR], x[d], acc);
       const int64_t row = ((int64_t)b * Hr + hr) * max_seq + pos;
-      idx[row * kR + c] = acc;
+      float acc;
+      if (kBf16) {
+        // bf16 storage: the projection in fp64, then one rounding to the nearest bf16 (even on
+        // ties), so the stored key is the exact projection's bf16 rounding
+        double a64 = 0.0;
+#pragma unroll 16
+        for (int d = 0; d < kD; ++d) a64 = fma((double)w[d * kR], (double)x[d], a64);
+        const __nv_bfloat16 kb = __double2bfloat16(a64);
+        idx_b[row * kR + c] = kb;
+        acc = __bfloat162float(kb);
+      } else {
+        acc = 0.f;
+#pragma unroll 16
+        for (int d = 0; d < kD; ++d) acc = fmaf(w[d * kR], x[d], acc);
+        idx[row * kR + c] = acc;
+      }
       // the same key split as fp16 hi + lo, for the tensor-core scoring of prefill
       const __half hh = __float2half_rn(acc);
       idx_hl[row * (2 * kR) + c] = hh;
@@ -165,11 +179,11 @@ cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const _
   dim3 grid(T, L->B);
   const int nw = L->Hr < kWHeads ? L->Hr : kWHeads;
   const size_t smem = ((size_t)L->Hkv * kD + (size_t)nw * kD * kR) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(append_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto fn = L->index_bf16 ? append_kv_kernel<true> : append_kv_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  append_kv_kernel<<<grid, 256, smem, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta,
-                                            L->wk, L->d_ret_head, L->group, L->kc, L->vc, L->idx,
-                                            L->idx_hl, L->err);
+  fn<<<grid, 256, smem, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta, L->wk, L->d_ret_head,
+                              L->group, L->kc, L->vc, L->idx, L->idx_b, L->idx_hl, L->err);
   return cudaGetLastError();
 }
 

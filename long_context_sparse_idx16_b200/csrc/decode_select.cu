@@ -1,7 +1,8 @@
 // decode_select.cu -- decode-time index scoring fused with the exact top-p selection.
 //
 // For every problem p = (sequence b, retrieval head h) the kernel
-//   1. streams the 16-dim index keys IDX[p][0..N) from HBM and computes the pre-RoPE
+//   1. streams the 16-dim index keys IDX[p][0..N) (fp32, or bf16 when the layer stores bf16
+//      keys: half the bytes) from HBM and computes the pre-RoPE
 //      scores s_j = qidx . IDX[p][j] (techwalker page, section 3: the 16-dim "radar");
 //   2. finds the exact top-p set: the shortest prefix of the order (s desc, j asc) whose
 //      index-softmax mass reaches p (zhichai page, insight 3; techwalker page, section 4),
@@ -68,7 +69,8 @@ struct Hist3 {  // a 2048-bin mass histogram in global memory: exact 64-bit mass
 };
 
 struct SelectArgs {
-  const float* idx;
+  const float* idx;           // fp32 index keys, or
+  const __nv_bfloat16* idx_b; // bf16 index keys (one of the two is set)
   int64_t idx_pstride;  // floats between problems (max_seq * r)
   const float* q_idx;   // [P][r]
   int P;
@@ -330,7 +332,7 @@ __device__ __forceinline__ int cf_of(int p, const SelectArgs& a) { return (int)(
 
 // ---------------------------------------------------------------- the kernel
 
-template <bool kSmemScores>
+template <bool kSmemScores, bool kBf16>
 __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
@@ -377,34 +379,64 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   }
   __syncthreads();
 
-  // ---- phase A: stream index keys -> scores, segment maxima
-  const int quad = tid >> 2, part = tid & 3;
+  // ---- phase A: stream index keys -> scores, segment maxima.  fp32 keys: four threads per
+  // 64-byte key row, 16 bytes each; bf16 keys: two threads per 32-byte row.
+  constexpr int kPer = kBf16 ? 2 : 4;      // threads per key
+  constexpr int kKeysIt = kThreads / kPer;  // keys per unrolled step
+  const int quad = tid / kPer, part = tid % kPer;
   for (int si = 0; si < nseg; ++si) {
     const Seg s = S.seg[si];
     const int64_t rows = s.jhi - s.jlo;
-    const float4* src = reinterpret_cast<const float4*>(a.idx + (int64_t)s.p * a.idx_pstride) + s.jlo * 4;
-    const float4 qv = reinterpret_cast<const float4*>(a.q_idx + (int64_t)s.p * kR)[part];
+    const float4* src = kBf16 ? reinterpret_cast<const float4*>(a.idx_b + (int64_t)s.p * a.idx_pstride) + s.jlo * 2
+                              : reinterpret_cast<const float4*>(a.idx + (int64_t)s.p * a.idx_pstride) + s.jlo * 4;
+    float qv[kBf16 ? 8 : 4];
+    {
+      const float4* qp = reinterpret_cast<const float4*>(a.q_idx + (int64_t)s.p * kR) + part * (kBf16 ? 2 : 1);
+#pragma unroll
+      for (int i = 0; i < (kBf16 ? 2 : 1); ++i) {
+        const float4 q4 = qp[i];
+        qv[4 * i] = q4.x;
+        qv[4 * i + 1] = q4.y;
+        qv[4 * i + 2] = q4.z;
+        qv[4 * i + 3] = q4.w;
+      }
+    }
     float mx = -INFINITY;
     // The trip count is the same for every thread (the shuffles below are full-warp);
     // rows past the end are loaded as zeros and not stored.
-    for (int64_t base = 0; base < rows; base += kUnroll * (kThreads / 4)) {
+    for (int64_t base = 0; base < rows; base += kUnroll * kKeysIt) {
       const int64_t k0 = base + quad;
       float4 v[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        const int64_t k = k0 + u * (kThreads / 4);
-        v[u] = k < rows ? ld_stream_f4(src + k * 4 + part) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int64_t k = k0 + u * kKeysIt;
+        v[u] = k < rows ? ld_stream_f4(src + k * kPer + part) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        float d = v[u].x * qv.x;
-        d = fmaf(v[u].y, qv.y, d);
-        d = fmaf(v[u].z, qv.z, d);
-        d = fmaf(v[u].w, qv.w, d);
-        d += __shfl_xor_sync(0xffffffffu, d, 1);
-        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        float d;
+        if constexpr (kBf16) {  // eight bf16 components
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+          float2 f = __bfloat1622float2(h[0]);
+          d = f.x * qv[0];
+          d = fmaf(f.y, qv[1], d);
+#pragma unroll
+          for (int e = 1; e < 4; ++e) {
+            f = __bfloat1622float2(h[e]);
+            d = fmaf(f.x, qv[2 * e], d);
+            d = fmaf(f.y, qv[2 * e + 1], d);
+          }
+          d += __shfl_xor_sync(0xffffffffu, d, 1);
+        } else {  // four fp32 components
+          d = v[u].x * qv[0];
+          d = fmaf(v[u].y, qv[1], d);
+          d = fmaf(v[u].z, qv[2], d);
+          d = fmaf(v[u].w, qv[3], d);
+          d += __shfl_xor_sync(0xffffffffu, d, 1);
+          d += __shfl_xor_sync(0xffffffffu, d, 2);
+        }
         d += 0.0f;  // -0 -> +0: equal scores must get equal order keys
-        const int64_t k = k0 + u * (kThreads / 4);
+        const int64_t k = k0 + u * kKeysIt;
         if (k < rows) {
           mx = fmaxf(mx, d);
           if (part == 0) sc[s.off + k] = d;
@@ -830,6 +862,7 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   const SelectGeom g = select_geometry(L, N);
   SelectArgs a;
   a.idx = L->idx;
+  a.idx_b = L->idx_b;
   a.idx_pstride = L->max_seq * kR;
   a.q_idx = L->q_idx;
   a.P = L->B * L->Hr;
@@ -860,7 +893,11 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   if (!g.smem_scores && L->gscores == nullptr) return cudaErrorInvalidValue;
   if (g.grid > L->sm_count || g.grid > kSelMaxGrid) return cudaErrorInvalidValue;
   void* args[] = {&a};
-  const void* fn = g.smem_scores ? (const void*)decode_select_kernel<true> : (const void*)decode_select_kernel<false>;
+  const void* fn = L->index_bf16
+                       ? (g.smem_scores ? (const void*)decode_select_kernel<true, true>
+                                        : (const void*)decode_select_kernel<false, true>)
+                       : (g.smem_scores ? (const void*)decode_select_kernel<true, false>
+                                        : (const void*)decode_select_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem_bytes);
   if (e != cudaSuccess) return e;
   int occ = 0;

@@ -1,4 +1,6 @@
-// prefill_local_tc.cu -- local heads in chunked prefill on 5th-generation tensor cores.
+// prefill_local_tc.cu -- local heads in chunked prefill on 5th-generation tensor cores (and
+// the retrieval heads too, with a window covering every causal key, when the layer runs the
+// pages' own dense prefill for them).
 //
 // Local heads attend only to nearby tokens and a few attention sinks (techwalker page, section
 // 2; section 8: window 8192 with 4 sinks).  Query row i of the chunk sits at position
@@ -354,7 +356,10 @@ __global__ void __launch_bounds__(kThreadsT, 2) prefill_local_tc_kernel(LocalTcA
 
 }  // namespace
 
-cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStream_t st) {
+// The kernel over a list of heads with a given window and sink count: the local heads, or (the
+// pages' own prefill) the retrieval heads with a window that covers every causal key.
+static cudaError_t launch_prefill_heads(const rtp_layer* L, int C, float* out, cudaStream_t st,
+                                        const int16_t* heads, int n_heads, int W, int S) {
   LocalTcArgs a;
   a.kc = L->kc;
   a.vc = L->vc;
@@ -364,9 +369,9 @@ cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStre
   a.group = L->group;
   a.C = C;
   a.P0 = L->len - C;
-  a.W = L->W;
-  a.S = L->S;
-  a.local_heads = L->d_local_list;
+  a.W = W;
+  a.S = S;
+  a.local_heads = heads;
   a.q_rot = L->q_rot;
   a.scale_log2 = L->sm_scale * 1.4426950408889634f;
   a.out = out;
@@ -374,9 +379,18 @@ cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStre
   cudaError_t e = cudaFuncSetAttribute(prefill_local_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemT);
   if (e != cudaSuccess) return e;
-  dim3 grid((C + kRowsT - 1) / kRowsT, L->n_local, L->B);
+  dim3 grid((C + kRowsT - 1) / kRowsT, n_heads, L->B);
   prefill_local_tc_kernel<<<grid, kThreadsT, kSmemT, st>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStream_t st) {
+  return launch_prefill_heads(L, C, out, st, L->d_local_list, L->n_local, L->W, L->S);
+}
+
+cudaError_t launch_prefill_dense_retrieval(const rtp_layer* L, int C, float* out, cudaStream_t st) {
+  const int W = L->len < (int64_t)0x7FFFFFFF ? (int)L->len : 0x7FFFFFFF;  // every causal key
+  return launch_prefill_heads(L, C, out, st, L->d_ret_head, L->Hr, W, 0);
 }
 
 }  // namespace rtp

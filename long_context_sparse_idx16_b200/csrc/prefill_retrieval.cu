@@ -21,7 +21,7 @@
 //      B  16 bins of m - s rounded to an integer (the last one holding everything from 14.5
 //         down) -> Z, T = ceil(p Z), crossing bin, whose exact order-key range is found by
 //         bisection;
-//      R  refinement: the crossing range of order keys is split 32 ways by bit slices, with
+//      R  refinement: the crossing range of order keys is split 16 ways by bit slices, with
 //         the mass of each slice and the first 16 keys of the range captured; once a row's
 //         range holds <= 16 keys they are sorted (key desc, j asc) for the exact cut; a range
 //         that shrinks to one key value is an exact tie group, resolved by
@@ -41,9 +41,9 @@ namespace {
 constexpr int kRowsR = kTcRows;  // 128 query rows per CTA (TMEM lanes)
 constexpr int kKeysR = kTcKeys;  // 64 keys per tile
 constexpr int kBins = 16;        // pass B: bins of width 1 below the row max
-constexpr int kSlices = 32;      // refinement: slices of the crossing key range per level
+constexpr int kSlices = 16;      // refinement: slices of the crossing key range per level
 constexpr int kCand = 16;        // keys captured per row in a refinement walk
-constexpr int kLevels = 8;       // refinement levels (5 key bits each, with margin)
+constexpr int kLevels = 10;      // refinement levels (4 key bits each, with margin)
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int { kModeKeys = 1, kModeTie = 2, kModeDone = 3 };
@@ -53,6 +53,7 @@ struct RetArgs {
   int Hkv, Hq, Hr, group, C;
   int64_t P0;
   float top_p;
+  int64_t top_k;              // > 0: fixed budget (counts instead of masses)
   int sc_bits;
   const int16_t* ret_head;    // [Hr]
   const float* q_rot;         // [B][C][Hq][D]
@@ -114,10 +115,10 @@ __device__ __forceinline__ void bin_key_range(float m, int b, uint32_t* lo, uint
   *hi = l - 1;
 }
 
-// slices of 2^shift keys cover [klo, khi] in at most kSlices pieces
+// slices of 2^shift keys cover [klo, khi] in at most kSlices (16) pieces
 __device__ __forceinline__ int slice_shift(uint32_t klo, uint32_t khi) {
   const int bits = 32 - __clz(khi - klo);
-  return bits > 5 ? bits - 5 : 0;
+  return bits > 4 ? bits - 4 : 0;
 }
 
 // last causal column of a 64-key tile for a row at position pos (-1: none)
@@ -128,31 +129,33 @@ __device__ __forceinline__ int causal_lim(int64_t pos, int64_t t) {
 // ------------------------------------------------------------------ exact per-row top-p
 
 constexpr int kPsThreads = kRowsR;  // one thread per row
-constexpr uint32_t kSelStages = 4;   // key tiles of the TMA ring
+constexpr uint32_t kSelStages = 3;   // key tiles of the TMA ring
 constexpr uint32_t kSOffQ = 0;                                       // query tile, 8 KB
-constexpr uint32_t kSOffK = kSOffQ + kTcQBytes;                      // key ring, 4 x 4 KB
-constexpr uint32_t kSOffH = kSOffK + kSelStages * kTcKBytes;         // [slice][row] u64, 32 KB
+constexpr uint32_t kSOffK = kSOffQ + kTcQBytes;                      // key ring, 3 x 4 KB
+constexpr uint32_t kSOffH = kSOffK + kSelStages * kTcKBytes;         // [slice][row] u64, 16 KB
 constexpr uint32_t kSOffC = kSOffH + kSlices * kRowsR * 8;           // [cand][row] u64, 16 KB
-constexpr uint32_t kSOffBar = kSOffC + kCand * kRowsR * 8;           // full[4], done[2], TMEM base
-constexpr uint32_t kSelSmem = kSOffBar + 64;
+constexpr uint32_t kSOffBar = kSOffC + kCand * kRowsR * 8;           // full[3], done[2], TMEM base
+constexpr uint32_t kSelSmem = kSOffBar + 64;  // about 54 KB: four CTAs (4 x 128 TMEM columns) per SM
+static_assert(kSelStages <= 3, "the barrier block holds three stage barriers");
 constexpr uint32_t kSelTmemCols = 128;                               // two 64-column score buffers
 
 // Walks over the key tiles [0, ntiles) of one (sequence, retrieval head): thread 0 keeps
 // kSelStages TMA copies in flight and issues the scores of tile t + 1 before tile t is read;
-// body(t, s) gets this thread's row's 64 scores of tile t.  g counts tiles over all walks
+// body(t, c0, s, lim) gets this thread's row's scores of tile t in groups of 16 (columns c0 ..
+// c0 + 15, s[0..15]) and the last causal column lim of the tile.  g counts tiles over all walks
 // (mbarrier phases).  A wait that runs out clears ok in every thread; later walks then do
 // nothing, and drain() waits (bounded) for the copies and MMAs still in flight.
 struct SelWalk {
   uint32_t sbase, tmem, lane_addr;
   const CUtensorMap* map;
-  int64_t row0;
+  int64_t row0, pos;  // pos: this thread's row position (-1: no row)
   uint32_t g;
   bool ok;
   uint32_t inflight_lo, inflight_hi;  // tiles [lo, hi) whose copies thread 0 has not waited on
   bool mma_pending;                   // scores of tile g issued and not waited on
 
   __device__ uint32_t full_bar(uint32_t gt) const { return sbase + kSOffBar + 8u * (gt % kSelStages); }
-  __device__ uint32_t done_bar(uint32_t gt) const { return sbase + kSOffBar + 32u + 8u * (gt & 1u); }
+  __device__ uint32_t done_bar(uint32_t gt) const { return sbase + kSOffBar + 24u + 8u * (gt & 1u); }
   __device__ uint32_t ktile(uint32_t gt) const { return sbase + kSOffK + (gt % kSelStages) * kTcKBytes; }
 
   template <typename Body>
@@ -185,8 +188,8 @@ struct SelWalk {
       tc_fence_after();
       float s[kTcKeys];
       __syncwarp();  // the loads are warp-collective: reconverge after thread 0's work
-      tmem_ld32(lane_addr + (gt & 1u) * kTcKeys, s);
-      tmem_ld32(lane_addr + (gt & 1u) * kTcKeys + 32u, s + 32);
+#pragma unroll
+      for (int q = 0; q < kTcKeys / 16; ++q) tmem_ld16(lane_addr + (gt & 1u) * kTcKeys + 16u * q, s + 16 * q);
       tmem_ld_wait();
       tc_fence_before();
       if (!__syncthreads_and(okw ? 1 : 0)) {
@@ -204,7 +207,11 @@ struct SelWalk {
       }
 #pragma unroll
       for (int i = 0; i < kTcKeys; ++i) s[i] += 0.0f;  // -0 -> +0: equal scores, equal order keys
-      body(t, s);
+      // the body sees the tile in four 16-column groups (a smaller unrolled body), told whether
+      // every column of the group is causal for this row
+      const int lim = causal_lim(pos, t);
+#pragma unroll
+      for (int q = 0; q < kTcKeys / 16; ++q) body(t, 16 * q, s + 16 * q, lim);
     }
     g += (uint32_t)ntiles;
   }
@@ -233,7 +240,8 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
   uint2* cut = a.cut + ((int64_t)b * a.Hr + hr) * a.C + i0;
   float* mass_out = (a.sel_mass && live) ? a.sel_mass + ((int64_t)b * a.C + i0 + tid) * a.Hr + hr : nullptr;
 
-  if (a.top_p >= 1.f) {  // p = 1 keeps every causal key (also those whose mass rounds to 0)
+  const bool topk = a.top_k > 0;  // fixed budget: every key weighs 1, the target is min(k, n)
+  if (!topk && a.top_p >= 1.f) {  // p = 1 keeps every causal key (also those whose mass rounds to 0)
     if (live) {
       cut[tid] = make_uint2(0u, 0x7FFFFFFFu);
       if (mass_out) *mass_out = 1.f;
@@ -247,7 +255,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSOffBar + 48);
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kSelTmemCols);
   if (tid == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(sbase + kSOffBar + 8u * i, 1);
+    for (int i = 0; i < 5; ++i) mbar_init(sbase + kSOffBar + 8u * i, 1);
     fence_mbar_init();
   }
   {
@@ -265,32 +273,40 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
   W.lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
   W.map = &tm_idx;
   W.row0 = ((int64_t)b * a.Hr + hr) * a.max_seq;
+  W.pos = pos;
   W.g = 0;
   W.ok = true;
   W.inflight_lo = W.inflight_hi = 0;
   W.mma_pending = false;
+  // the weight a key adds to the histograms: its fixed-point softmax mass, or 1 with a fixed
+  // budget (then the sums are counts)
+  auto weight = [&](float s, float mx) -> unsigned long long { return topk ? 1ull : mass64(s, mx, scale); };
   unsigned long long* hist = reinterpret_cast<unsigned long long*>(sm + kSOffH) + tid;  // [slice * 128]
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kSOffC) + tid;  // [k * 128]
 
   // ---- pass A: the row max
-  float m = -INFINITY;
-  W.run(ntiles, [&](int64_t t, const float* s) {
-    const int lim = causal_lim(pos, t);
+  float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four chains: no serial max
+  W.run(ntiles, [&](int64_t t, int c0, const float* s, int lim) {
+    if (lim >= c0 + 15) {
 #pragma unroll
-    for (int c = 0; c < kKeysR; ++c)
-      if (c <= lim) m = fmaxf(m, s[c]);
+      for (int c = 0; c < 16; ++c) mq[c & 3] = fmaxf(mq[c & 3], s[c]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        if (c0 + c <= lim) mq[c & 3] = fmaxf(mq[c & 3], s[c]);
+    }
   });
+  const float m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
 
   // ---- pass B: 16 bins of width 1 below the max (the last, most populated bin in a register)
   for (int i = 0; i < kBins; ++i) hist[i * kRowsR] = 0ull;
   unsigned long long far = 0ull;
-  W.run(ntiles, [&](int64_t t, const float* s) {
-    const int lim = causal_lim(pos, t);
+  W.run(ntiles, [&](int64_t t, int c0, const float* s, int lim) {
 #pragma unroll
-    for (int c = 0; c < kKeysR; ++c) {
-      if (c <= lim) {
+    for (int c = 0; c < 16; ++c) {
+      if (c0 + c <= lim) {
         const int bi = bin1_of(m - s[c]);
-        const unsigned long long ms = mass64(s[c], m, scale);
+        const unsigned long long ms = weight(s[c], m);
         if (bi == kBins - 1) far += ms;
         else hist[bi * kRowsR] += ms;
       }
@@ -307,7 +323,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
     }
     hb[kBins - 1] = far;
     Z += far;
-    unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
+    unsigned long long T = topk ? (unsigned long long)a.top_k : (unsigned long long)ceil((double)a.top_p * (double)Z);
     if (T < 1ull) T = 1ull;
     if (T > Z) T = Z;
     unsigned long long cum = 0ull;
@@ -326,7 +342,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
     mode = kModeKeys;
   }
 
-  // ---- refinement: 32-way bit slices of the crossing key range until <= 16 keys remain
+  // ---- refinement: 16-way bit slices of the crossing key range until <= 16 keys remain
   for (int level = 0; level < kLevels; ++level) {
     if (!__syncthreads_or(mode == kModeKeys)) break;
     const bool mine = mode == kModeKeys;
@@ -334,16 +350,15 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
       for (int i = 0; i < kSlices; ++i) hist[i * kRowsR] = 0ull;
     int nc = 0;
     const uint32_t span = khi - klo;
-    W.run(ntiles, [&](int64_t t, const float* s) {
+    W.run(ntiles, [&](int64_t t, int c0, const float* s, int lim) {
       if (!mine) return;
-      const int lim = causal_lim(pos, t);
 #pragma unroll
-      for (int c = 0; c < kKeysR; ++c) {
+      for (int c = 0; c < 16; ++c) {
         const uint32_t key = order_key(s[c]);
-        if (c <= lim && key - klo <= span) {
-          hist[(int)((key - klo) >> shift) * kRowsR] += mass64(s[c], m, scale);
+        if (c0 + c <= lim && key - klo <= span) {
+          hist[(int)((key - klo) >> shift) * kRowsR] += weight(s[c], m);
           if (nc < kCand)
-            cand[nc * kRowsR] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)(t * kKeysR + c));
+            cand[nc * kRowsR] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)(t * kKeysR + c0 + c));
           ++nc;
         }
       }
@@ -365,7 +380,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
       unsigned long long cum = 0ull;
       int ci = -1;
       for (int i = 0; i < nc; ++i) {
-        cum += mass64(key_to_float((uint32_t)(cv[i] >> 32)), m, scale);
+        cum += weight(key_to_float((uint32_t)(cv[i] >> 32)), m);
         if (cum >= rem) {
           ci = i;
           break;
@@ -408,14 +423,14 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
         shift = slice_shift(nlo, nhi);
         if (nlo == nhi) {  // one key value with more than 16 members: an exact tie group
           t_key = nlo;
-          const unsigned long long e = mass64(key_to_float(nlo), m, scale);
+          const unsigned long long e = weight(key_to_float(nlo), m);
           n_need = e ? (rem + e - 1) / e : 1ull;
           mode = kModeTie;
         }
       }
     }
   }
-  if (mode == kModeKeys) {  // not reached: eight 32-way levels split 32 bits
+  if (mode == kModeKeys) {  // not reached: ten 16-way levels split 32 bits
     atomicOr(a.err, kErrInternal);
     t_key = 0xFFFFFFFFu;
     tiecut = -1;
@@ -427,14 +442,13 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
     const bool mine = mode == kModeTie;
     unsigned long long before = 0ull;
     bool found = false;
-    W.run(ntiles, [&](int64_t t, const float* s) {
+    W.run(ntiles, [&](int64_t t, int c0, const float* s, int lim) {
       if (!mine || found) return;
-      const int lim = causal_lim(pos, t);
 #pragma unroll
-      for (int c = 0; c < kKeysR; ++c) {
-        if (c <= lim && order_key(s[c]) == t_key && !found) {
+      for (int c = 0; c < 16; ++c) {
+        if (c0 + c <= lim && order_key(s[c]) == t_key && !found) {
           if (++before == n_need) {
-            tiecut = (int)(t * kKeysR + c);
+            tiecut = (int)(t * kKeysR + c0 + c);
             found = true;
           }
         }
@@ -445,7 +459,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
         atomicOr(a.err, kErrInternal);
         tiecut = 0x7FFFFFFF;
       } else {
-        above += n_need * mass64(key_to_float(t_key), m, scale);
+        above += n_need * weight(key_to_float(t_key), m);
       }
       mode = kModeDone;
     }
@@ -456,7 +470,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
     if (tid == 0) atomicOr(a.err, kErrTimeout);
   } else if (live) {
     cut[tid] = make_uint2(t_key, (uint32_t)tiecut);
-    if (mass_out) *mass_out = (float)((double)above / (double)Z);
+    if (mass_out) *mass_out = topk ? -1.f : (float)((double)above / (double)Z);  // no masses with a fixed budget
   }
   tc_fence_before();
   __syncthreads();
@@ -836,6 +850,7 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
   a.C = C;
   a.P0 = L->len - C;
   a.top_p = L->top_p;
+  a.top_k = L->top_k;
   int lg = 0;
   while ((1ll << lg) < L->len) ++lg;
   a.sc_bits = 62 - lg;

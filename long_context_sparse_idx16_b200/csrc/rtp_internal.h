@@ -1,6 +1,7 @@
 // rtp_internal.h -- layer state and kernel launch entry points (host side, internal).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -26,6 +27,9 @@ constexpr int kSelMaxGrid = 256; // CTAs of the selection grid (<= SM count)
 constexpr int kGatherChunk = 128;
 constexpr int kGatherThreads = 256;
 
+// Fixed top-k decode selection (ablation mode): keys per chunk of its radix-select kernels.
+constexpr int kTopkChunk = 4096;
+
 // Window + sink decode attention: keys per CTA tile and threads.
 constexpr int kSwaTile = 128;
 constexpr int kSwaThreads = 128;
@@ -48,7 +52,14 @@ struct rtp_layer {
   // caches
   __half* kc = nullptr;  // [B][Hkv][max_seq][D] RoPE'd keys
   __half* vc = nullptr;  // [B][Hkv][max_seq][D]
-  float* idx = nullptr;  // [B][Hr][max_seq][r]
+  float* idx = nullptr;  // [B][Hr][max_seq][r] fp32 index keys (fp32 storage)
+  __nv_bfloat16* idx_b = nullptr;  // [B][Hr][max_seq][r] bf16 index keys (bf16 storage)
+  bool index_bf16 = false;
+  bool prefill_dense = false;       // retrieval heads dense in prefill (the pages' own prefill)
+  int64_t top_k = 0;                // > 0: fixed-budget selection instead of top-p
+  uint32_t* tk_keys = nullptr;      // [B*Hr][max_seq] order keys of the scores (top-k mode)
+  uint32_t* tk_hist = nullptr;      // [B*Hr][4][256] radix histograms (top-k mode)
+  uint32_t* tk_cnt = nullptr;       // [B*Hr][chunks][2] per-chunk counts (top-k mode)
   float* wq = nullptr;   // [Hr][D][r]
   float* wk = nullptr;   // [Hr][D][r]
   double* theta = nullptr;  // [D/2] RoPE frequencies base^(-2c/D)
@@ -125,6 +136,9 @@ cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const _
 cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, int64_t pos0,
                           cudaStream_t st);
 cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st);
+cudaError_t launch_decode_topk(rtp_layer* L, cudaStream_t st);
+cudaError_t launch_prefill_dense_retrieval(const rtp_layer* L, int C, float* out, cudaStream_t st);
+cudaError_t launch_prefill_dense_stats(const rtp_layer* L, int C, int32_t* cnt, float* mass, cudaStream_t st);
 cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, float* out, cudaStream_t st);
 cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st);
 cudaError_t launch_iota_rows(int32_t* dst, int64_t cap, int rows, int64_t n, cudaStream_t st);

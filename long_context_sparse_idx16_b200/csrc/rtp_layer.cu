@@ -96,15 +96,34 @@ static void free_all(rtp_layer* L) {
   if (L->side) cudaStreamDestroy(L->side);
   L->ev_fork = L->ev_join = nullptr;
   L->side = nullptr;
-  void* ptrs[] = {L->kc, L->vc, L->idx, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
+  void* ptrs[] = {L->kc, L->vc, L->idx, L->idx_b, L->wq, L->wk, L->theta, L->d_head_slot, L->d_ret_head,
                   L->d_loc_head, L->d_loc_cnt, L->d_local_list, L->pf_cut, L->idx_hl, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
-                  L->sticket, L->err};
+                  L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
 
+}  // namespace rtp
+
+namespace rtp {
+namespace {
+// With dense retrieval prefill row i (position P0 + i) keeps all its P0 + i + 1 causal keys.
+__global__ void prefill_dense_stats_kernel(int32_t* cnt, float* mass, int C, int Hr, int64_t P0, int64_t n) {
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n) return;
+  const int64_t i = (t / Hr) % C;
+  if (cnt) cnt[t] = (int32_t)(P0 + i + 1);
+  if (mass) mass[t] = 1.f;
+}
+}  // namespace
+
+cudaError_t launch_prefill_dense_stats(const rtp_layer* L, int C, int32_t* cnt, float* mass, cudaStream_t st) {
+  const int64_t n = (int64_t)L->B * C * L->Hr;
+  prefill_dense_stats_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cnt, mass, C, L->Hr, L->len - C, n);
+  return cudaGetLastError();
+}
 }  // namespace rtp
 
 using namespace rtp;
@@ -131,6 +150,10 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   if (c.max_select < 0 || c.max_select > c.max_seq)
     return fail(nullptr, RTP_EINVAL, "rtp_create: max_select must be in [0, max_seq]");
   if (c.max_chunk < 0) return fail(nullptr, RTP_EINVAL, "rtp_create: max_chunk must be >= 0");
+  if (c.index_bf16 != 0 && c.index_bf16 != 1) return fail(nullptr, RTP_EINVAL, "rtp_create: index_bf16 must be 0 or 1");
+  if (c.prefill_dense != 0 && c.prefill_dense != 1)
+    return fail(nullptr, RTP_EINVAL, "rtp_create: prefill_dense must be 0 or 1");
+  if (c.top_k < 0) return fail(nullptr, RTP_EINVAL, "rtp_create: top_k must be >= 0");
 
   rtp_layer* L = new rtp_layer();
   L->B = c.batch;
@@ -140,6 +163,9 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   L->max_seq = c.max_seq;
   L->max_select = c.max_select ? c.max_select : c.max_seq;
   L->max_chunk = c.max_chunk ? c.max_chunk : 16384;
+  L->index_bf16 = c.index_bf16 == 1;
+  L->prefill_dense = c.prefill_dense == 1;
+  L->top_k = c.top_k;
   L->top_p = c.top_p;
   L->sm_scale = c.sm_scale > 0.f ? c.sm_scale : 1.0f / sqrtf((float)kD);
   L->rope_base = c.rope_base;
@@ -197,7 +223,13 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   e = cudaSuccess;
   RTP_ALLOC(L->kc, B * Hkv * L->max_seq * kD);
   RTP_ALLOC(L->vc, B * Hkv * L->max_seq * kD);
-  RTP_ALLOC(L->idx, P * L->max_seq * kR);
+  if (L->top_k > 0 && Hr > 0) {
+    RTP_ALLOC(L->tk_keys, P * L->max_seq);
+    RTP_ALLOC(L->tk_hist, P * 4 * 256);
+    RTP_ALLOC(L->tk_cnt, P * 2 * ((L->max_seq + kTopkChunk - 1) / kTopkChunk));
+  }
+  if (L->index_bf16) RTP_ALLOC(L->idx_b, P * L->max_seq * kR);
+  else RTP_ALLOC(L->idx, P * L->max_seq * kR);
   RTP_ALLOC(L->wq, Hr * kD * kR);
   RTP_ALLOC(L->wk, Hr * kD * kR);
   RTP_ALLOC(L->theta, kHalfD);
@@ -334,10 +366,12 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
   bool forked = false;
   if (L->Hr > 0) {
     // p == 1 keeps every causal key: the gather reads positions 0..len-1 directly
-    const bool dense = L->top_p >= 1.f;
+    // p == 1 (without a fixed budget) keeps every causal key: the gather reads 0..len-1 directly
+    const bool dense = L->top_k == 0 && L->top_p >= 1.f;
     {
-      ProfScope ps(L, dense ? "dense_fill" : "decode_select", stream);
-      e = dense ? launch_dense_stats(L, stream) : launch_decode_select(L, stream);
+      ProfScope ps(L, dense ? "dense_fill" : (L->top_k > 0 ? "decode_topk" : "decode_select"), stream);
+      e = dense ? launch_dense_stats(L, stream)
+                : (L->top_k > 0 ? launch_decode_topk(L, stream) : launch_decode_select(L, stream));
     }
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: select");
     if (L->n_local > 0 && !L->prof_on) {  // the window attention needs only q_prep: fork it off
@@ -401,6 +435,9 @@ rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out,
   if (stats && stats->rows &&
       (stats->n_rows < 1 || !stats->row_sel || stats->row_sel_cap < 1 || !stats->sel_count))
     return fail(L, RTP_EINVAL, "rtp_prefill_chunk: rows needs n_rows >= 1, row_sel, row_sel_cap >= 1 and sel_count");
+  if (stats && L->prefill_dense && (stats->sel_bitmap || stats->rows))
+    return fail(L, RTP_EINVAL, "rtp_prefill_chunk: with dense retrieval prefill every causal key is selected; "
+                               "no bitmap or row lists are written");
   cudaError_t e;
   {
     ProfScope ps(L, "q_prep", stream);
@@ -414,7 +451,16 @@ rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out,
     e = cudaEventRecord(L->ev_fork, stream);
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: fork");
   }
-  if (L->Hr > 0) {
+  if (L->Hr > 0 && L->prefill_dense) {
+    // the pages' own prefill: retrieval heads attend to every causal key
+    {
+      ProfScope ps(L, "prefill_dense", stream);
+      e = launch_prefill_dense_retrieval(L, C, out, stream);
+    }
+    if (e == cudaSuccess && stats && (stats->sel_count || stats->sel_mass))
+      e = launch_prefill_dense_stats(L, C, stats->sel_count, stats->sel_mass, stream);
+    if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: retrieval heads (dense)");
+  } else if (L->Hr > 0) {
     e = launch_prefill_retrieval(L, C, out, stats, stream);  // profiled as prefill_select + prefill_attn
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: retrieval heads");
   }
@@ -523,6 +569,7 @@ rtp_status rtp_get_cache(const rtp_layer* L, rtp_cache_view* view) {
   view->k = L->kc;
   view->v = L->vc;
   view->idx = L->idx;
+  view->idx_bf16 = L->idx_b;
   view->max_seq = L->max_seq;
   view->n_retrieval = L->Hr;
   return RTP_OK;

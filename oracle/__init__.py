@@ -31,13 +31,17 @@ def lib():
         i64, i32, f64 = C.c_int64, C.c_int, C.c_double
         L.orc_head_rows.restype = C.c_int
         L.orc_head_rows.argtypes = [P, P, i64, i64, i32, i32, i32, P, i64, P, i64, i32, P, P, f64,
-                                    i64, i64, f64, f64, i64, P, P, P, P, P, P, i64, P, i64, i32]
+                                    i64, i64, f64, f64, i64, P, P, P, P, P, P, i64, P, i64, i32, i32, i64]
+        L.orc_topk.restype = i64
+        L.orc_topk.argtypes = [P, i64, i64, P, P, P, P, P]
         L.orc_topp.restype = i64
         L.orc_topp.argtypes = [P, i64, f64, P, P, P, P, P]
         L.orc_rope.restype = None
         L.orc_rope.argtypes = [P, f64, i32, f64, P]
         L.orc_index_scores.restype = None
-        L.orc_index_scores.argtypes = [P, i64, i64, i32, i32, i32, P, P, P, P]
+        L.orc_index_scores.argtypes = [P, i64, i64, i32, i32, i32, P, P, P, P, i32]
+        L.orc_round_bf16.restype = f64
+        L.orc_round_bf16.argtypes = [f64]
         L.orc_attend_set.restype = None
         L.orc_attend_set.argtypes = [P, P, i64, i32, i32, P, i64, f64, f64, i64, P, i64, P]
         L.orc_max_threads.restype = C.c_int
@@ -89,11 +93,30 @@ def topp(scores: np.ndarray, p: float) -> TopP:
     return TopP(int(K), order[:n], pi[:n], mass.value, pt.value, cp.value)
 
 
+def round_bf16(x: float) -> float:
+    """x rounded to the nearest bf16 value, ties to even (the bf16 index-key storage)."""
+    return float(lib().orc_round_bf16(float(x)))
+
+
+def topk(scores: np.ndarray, k: int) -> TopP:
+    """Fixed top-k selection over a score vector (the pages' fixed-budget ablation)."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    n = s.shape[0]
+    order = np.empty(max(n, 1), dtype=np.int64)
+    pi = np.empty(max(n, 1), dtype=np.float64)
+    mass = C.c_double()
+    pt = C.c_double()
+    cp = C.c_double()
+    K = lib().orc_topk(_p(s), n, int(k), _p(order), _p(pi), C.byref(mass), C.byref(pt), C.byref(cp))
+    return TopP(int(K), order[:n], pi[:n], mass.value, pt.value, cp.value)
+
+
 def index_scores(k_seq: np.ndarray, g: int, q_vec: np.ndarray, wq: np.ndarray, wk: np.ndarray,
-                 n: Optional[int] = None) -> np.ndarray:
+                 n: Optional[int] = None, index_bf16: bool = False) -> np.ndarray:
     """Pre-RoPE index scores of one query against keys 0..n-1 of KV head g.
 
     k_seq: bf16 bits [N][Hkv][D] of one sequence; q_vec: bf16 bits [D]; wq/wk: fp32 [D][r].
+    index_bf16: the index keys are stored in bf16 (each component rounded, ties to even).
     """
     k_seq = np.ascontiguousarray(k_seq, dtype=np.uint16)
     N, Hkv, D = k_seq.shape
@@ -103,7 +126,7 @@ def index_scores(k_seq: np.ndarray, g: int, q_vec: np.ndarray, wq: np.ndarray, w
     wq = np.ascontiguousarray(wq, dtype=np.float32)
     wk = np.ascontiguousarray(wk, dtype=np.float32)
     s = np.empty(n, dtype=np.float64)
-    lib().orc_index_scores(_p(k_seq), n, Hkv * D, g, D, r, _p(q_vec), _p(wq), _p(wk), _p(s))
+    lib().orc_index_scores(_p(k_seq), n, Hkv * D, g, D, r, _p(q_vec), _p(wq), _p(wk), _p(s), 1 if index_bf16 else 0)
     return s
 
 
@@ -122,7 +145,8 @@ def head_rows(k_seq: np.ndarray, v_seq: np.ndarray, q_rows: np.ndarray, position
               g: int, retrieval: bool, wq: Optional[np.ndarray] = None, wk: Optional[np.ndarray] = None,
               top_p: float = 0.9, window: int = 8192, n_sink: int = 4, rope_base: float = 1.0e6,
               sm_scale: Optional[float] = None, pos_offset: int = 0, want_sel: bool = True,
-              want_pi: bool = False, threads: Optional[int] = None) -> Rows:
+              want_pi: bool = False, threads: Optional[int] = None, index_bf16: bool = False,
+              top_k: int = 0) -> Rows:
     """Oracle output of one query head for several query rows of one sequence.
 
     k_seq, v_seq: bf16 bits [N][Hkv][D] (pre-RoPE keys); q_rows: bf16 bits [nrows][D];
@@ -154,7 +178,7 @@ def head_rows(k_seq: np.ndarray, v_seq: np.ndarray, q_rows: np.ndarray, position
         1 if retrieval else 0, _p(wq) if retrieval else None, _p(wk) if retrieval else None,
         float(top_p), int(window), int(n_sink), float(rope_base), float(scale), int(pos_offset),
         _p(out), _p(cnt), _p(mass), _p(pit), _p(cpv), _p(sel), cap if want_sel else 0,
-        _p(pi), (maxpos + 1) if pi is not None else 0, int(th))
+        _p(pi), (maxpos + 1) if pi is not None else 0, int(th), 1 if index_bf16 else 0, int(top_k))
     if rc != 0:
         raise ValueError("oracle: a row position lies outside the key range")
     sels = [sel[t, : min(int(cnt[t]), cap)].copy() for t in range(nrows)] if want_sel else None
@@ -170,12 +194,16 @@ def layer_rows(inputs, b: int, h: int, rows: Sequence[int], *, top_p: Optional[f
     rows = np.asarray(rows, dtype=np.int64)
     retrieval = h in s.retrieval_heads
     slot = s.retrieval_heads.index(h) if retrieval else 0
+    p = s.top_p if top_p is None else top_p
+    top_k = s.top_k
+    if s.prefill_dense and s.chunk > 1:  # the pages' own prefill: retrieval heads see every causal key
+        p, top_k = 1.0, 0
     return head_rows(
         inputs.k[b], inputs.v[b], inputs.q[b, rows, h], s.prefix + rows, g=s.kv_head(h),
         retrieval=retrieval, wq=inputs.wq[slot] if retrieval else None,
-        wk=inputs.wk[slot] if retrieval else None, top_p=s.top_p if top_p is None else top_p,
+        wk=inputs.wk[slot] if retrieval else None, top_p=p, top_k=top_k,
         window=s.window, n_sink=s.n_sink, rope_base=s.rope_base, want_sel=want_sel,
-        want_pi=want_pi, threads=threads, pos_offset=pos_offset)
+        want_pi=want_pi, threads=threads, pos_offset=pos_offset, index_bf16=s.index_bf16)
 
 
 def attend_set(inputs, b: int, h: int, row: int, sel: Sequence[int], *, pos_offset: int = 0) -> np.ndarray:

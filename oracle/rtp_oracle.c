@@ -24,6 +24,12 @@
  *   (P2 section 3 "full 128-dim exact computation on the selected tokens"):
  *       o = sum_{j in J} softmax_j( sm_scale * RoPE(q_i, i) . RoPE(k_j, j) ) v_j.
  *
+ *   With a fixed budget k > 0 instead of p (the pages' top-k ablation), J is the first
+ *   min(k, i + 1) keys of that order.
+ *
+ *   With bf16 index-key storage (an option of the layer), every component of kt_j is first
+ *   rounded to bf16, ties to even (orc_round_bf16); the query side stays fp64.
+ *
  *   RoPE is the rotate-half form: for c < D/2 the pair (c, c + D/2) turns by
  *   angle pos * base^(-2c/D).  The pages lose the formula in extraction; this is the
  *   plainest reading consistent with "low frequencies carry semantics" (P3 finding 2).
@@ -58,6 +64,23 @@ void orc_rope(const double* x, double pos, int D, double base, double* y) {
     y[c] = x[c] * cs - x[c + half] * sn;
     y[c + half] = x[c + half] * cs + x[c] * sn;
   }
+}
+
+/*
+ * x rounded to the nearest bf16 value (8 significant bits), ties to even: the storage of the
+ * index keys when the layer keeps them in bf16 (a storage choice the pages leave open; the
+ * aitntnews page, finding 2, calls the r = 16 indexer's cost "almost negligible").  Written
+ * from the definition: scale the significand to [128, 256), round half to even, scale back.
+ */
+double orc_round_bf16(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  int e;
+  double m = frexp(x, &e);        /* x = m * 2^e, 0.5 <= |m| < 1 */
+  double t = ldexp(m, 8);         /* |t| in [128, 256): the bf16 significand */
+  double f = floor(t);
+  double d = t - f;
+  if (d > 0.5 || (d == 0.5 && fmod(f, 2.0) != 0.0)) f += 1.0;
+  return ldexp(f, e - 8);
 }
 
 /* y[t] = sum_d W[d][t] x[d]: the 16-dim projection (W is [D][r], fp32). */
@@ -122,6 +145,32 @@ int64_t orc_topp(const double* s, int64_t n, double p, int64_t* order, double* p
   if (pi_t) *pi_t = last;
   if (cum_prev) *cum_prev = prev;
   free(pr);
+  return K;
+}
+
+/*
+ * Fixed top-k over scores s[0..n-1] (the ablation the techwalker page, section 4 and its
+ * Q&A, sets against dynamic top-p: a fixed budget of 4096 or 16384 tokens): J = the first
+ * min(k, n) keys of the order (s desc, j asc).  order / pi / mass / pi_t / cum_prev as for
+ * orc_topp (the masses are reported, not used for the cut).
+ */
+int64_t orc_topk(const double* s, int64_t n, int64_t k, int64_t* order, double* pi, double* mass, double* pi_t,
+                 double* cum_prev) {
+  if (n <= 0) return 0;
+  double* pw = (double*)malloc(sizeof(double) * (size_t)n);
+  orc_topp(s, n, 1.0, order, pw, NULL, NULL, NULL); /* the full order and every mass */
+  int64_t K = k < n ? k : n;
+  double cum = 0.0, prev = 0.0, last = 0.0;
+  for (int64_t t = 0; t < K; ++t) {
+    prev = cum;
+    last = pw[order[t]];
+    cum += last;
+  }
+  if (pi) memcpy(pi, pw, sizeof(double) * (size_t)n);
+  if (mass) *mass = cum;
+  if (pi_t) *pi_t = last;
+  if (cum_prev) *cum_prev = prev;
+  free(pw);
   return K;
 }
 
@@ -201,7 +250,7 @@ int orc_head_rows(const uint16_t* k, const uint16_t* v, int64_t n_keys, int64_t 
                   int64_t window, int64_t n_sink, double rope_base, double sm_scale,
                   int64_t pos_offset, double* out, int64_t* sel_count, double* sel_mass,
                   double* pi_t, double* cum_prev, int64_t* sel_idx, int64_t sel_cap,
-                  double* pi_all, int64_t pi_stride, int n_threads) {
+                  double* pi_all, int64_t pi_stride, int n_threads, int key_bf16, int64_t top_k) {
   if (nrows <= 0) return 0;
   int64_t maxpos = 0, minpos = pos[0];
   for (int64_t t = 0; t < nrows; ++t) {
@@ -250,6 +299,8 @@ int orc_head_rows(const uint16_t* k, const uint16_t* v, int64_t n_keys, int64_t 
       double x[512];
       for (int d = 0; d < D; ++d) x[d] = orc_bf16(kv.k[j * kv_stride + d]);
       orc_index_vec(x, wk, D, r, kt + j * r);
+      if (key_bf16)
+        for (int c = 0; c < r; ++c) kt[j * r + c] = orc_round_bf16(kt[j * r + c]);
     }
   }
 
@@ -273,7 +324,10 @@ int orc_head_rows(const uint16_t* k, const uint16_t* v, int64_t n_keys, int64_t 
       }
       J = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
       double ms = 0, pt = 0, cp = 0;
-      nJ = orc_topp(s, n, top_p, J, pi_all ? pi_all + t * pi_stride : NULL, &ms, &pt, &cp);
+      if (top_k > 0)
+        nJ = orc_topk(s, n, top_k, J, pi_all ? pi_all + t * pi_stride : NULL, &ms, &pt, &cp);
+      else
+        nJ = orc_topp(s, n, top_p, J, pi_all ? pi_all + t * pi_stride : NULL, &ms, &pt, &cp);
       sel_mass[t] = ms;
       pi_t[t] = pt;
       cum_prev[t] = cp;
@@ -328,9 +382,10 @@ void orc_attend_set(const uint16_t* k, const uint16_t* v, int64_t kv_stride, int
   orc_attend(qr, &kv, J, nJ, sm_scale, out);
 }
 
-/* Index scores s_j = (Wq^T q).(Wk^T k_j) for j < n (pre-RoPE), fp64. */
+/* Index scores s_j = (Wq^T q).(Wk^T k_j) for j < n (pre-RoPE), fp64; with key_bf16 each
+ * index-key component is first rounded to bf16 (the stored keys). */
 void orc_index_scores(const uint16_t* k, int64_t n, int64_t kv_stride, int g, int D, int r,
-                      const uint16_t* q, const float* wq, const float* wk, double* s) {
+                      const uint16_t* q, const float* wq, const float* wk, double* s, int key_bf16) {
   double qv[512], qt[64], x[512], kt[64];
   for (int d = 0; d < D; ++d) qv[d] = orc_bf16(q[d]);
   orc_index_vec(qv, wq, D, r, qt);
@@ -338,6 +393,8 @@ void orc_index_scores(const uint16_t* k, int64_t n, int64_t kv_stride, int g, in
     const uint16_t* kr = k + j * kv_stride + (int64_t)g * D;
     for (int d = 0; d < D; ++d) x[d] = orc_bf16(kr[d]);
     orc_index_vec(x, wk, D, r, kt);
+    if (key_bf16)
+      for (int c = 0; c < r; ++c) kt[c] = orc_round_bf16(kt[c]);
     double acc = 0.0;
     for (int c = 0; c < r; ++c) acc += qt[c] * kt[c];
     s[j] = acc;

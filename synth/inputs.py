@@ -91,6 +91,10 @@ class LayerSpec:
     # degenerate variants used by edge-case tests
     zero_index_weights: bool = False  # every index score is exactly 0 (all ties)
     p_sweep: Tuple[float, ...] = ()
+    # layer options the workload runs with (no effect on the generated numbers)
+    index_bf16: bool = False  # index keys stored in bf16 instead of fp32
+    top_k: int = 0  # > 0: retrieval heads keep a fixed budget of k keys instead of top-p
+    prefill_dense: bool = False  # retrieval heads attend to every causal key in prefill
 
     @property
     def group(self) -> int:

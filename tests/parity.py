@@ -44,7 +44,7 @@ def build_cache(layer, x, upto: int, chunk: int = 1 << 16):
         layer.append_kv(torch_bf16(x.k[:, t0:t1]), torch_bf16(x.v[:, t0:t1]))
 
 
-def check_selection(gpu_sel: np.ndarray, ref: "oracle.Rows", t: int, p: float, what: str):
+def check_selection(gpu_sel: np.ndarray, ref: "oracle.Rows", t: int, p: float, what: str, top_k: int = 0):
     """Compare a GPU selected set (ascending positions) with oracle row t (needs ref.pi).
 
     Returns the number of differing keys.  Besides the per-key rule, the count of differing keys
@@ -68,6 +68,9 @@ def check_selection(gpu_sel: np.ndarray, ref: "oracle.Rows", t: int, p: float, w
         n_band = int(np.count_nonzero(np.abs(pi - pt) <= SET_TOL))
         assert len(diff) <= n_band + 1, (f"{what}: {len(diff)} keys differ, more than the {n_band} keys "
                                          f"within 1e-6 of the threshold probability plus one")
+    if top_k > 0:  # a fixed budget: exactly min(k, n) keys, no mass target
+        assert len(gpu_sel) == len(o_sel), f"{what}: {len(gpu_sel)} keys selected, the budget gives {len(o_sel)}"
+        return len(diff)
     mass = float(pi[gpu_sel].sum()) if len(gpu_sel) else 0.0
     assert mass >= p - MASS_TOL, f"{what}: selected mass {mass} < p - 1e-5 (p={p})"
     return len(diff)
@@ -125,8 +128,9 @@ def run_decode(x, *, top_p=None, heads=None, batches=None, max_select=0, sel_cap
                 k = int(cnt[b, slot])
                 sel = idx[b, slot, :k].astype(np.int64)
                 assert np.all(np.diff(sel) > 0), "selected positions must be strictly ascending"
-                nd = check_selection(sel, r, 0, p32(p), f"b={b} h={h}")
-                assert abs(float(mass[b, slot]) - float(r.pi[0][sel].sum())) <= 1e-5
+                nd = check_selection(sel, r, 0, p32(p), f"b={b} h={h}", top_k=s.top_k)
+                if s.top_k == 0:
+                    assert abs(float(mass[b, slot]) - float(r.pi[0][sel].sum())) <= 1e-5
                 if nd:
                     ref_out = oracle.attend_set(x, b, h, 0, sel)
                 summary[(b, h)] = (k, int(r.count[0]), nd)
@@ -211,7 +215,10 @@ def run_prefill(x, *, top_p=None, rows=None, heads=None, batches=None, sets="bit
                     k = int(cnt[b0 + t])
                     pos = s.prefix + int(i)
                     if sets is None:
-                        assert float(mass[b0 + t]) >= p - MASS_TOL
+                        if s.prefill_dense:
+                            assert k == pos + 1, f"b={b} h={h} row={i}: dense prefill counts {k} keys"
+                        elif s.top_k == 0:
+                            assert float(mass[b0 + t]) >= p - MASS_TOL
                         continue
                     if sets == "bitmap":
                         sel = bitmap_positions(bm[t], pos + 1)
@@ -222,9 +229,10 @@ def run_prefill(x, *, top_p=None, rows=None, heads=None, batches=None, sets="bit
                             f"b={b} h={h} row={i}: listed positions not ascending inside the causal range"
                     if exact_sets:
                         assert np.array_equal(sel, r.sel[t]), f"b={b} h={h} row={i}: set differs"
-                    nd = check_selection(sel, r, t, p32(p), f"b={b} h={h} row={i}")
-                    assert abs(float(mass[b0 + t]) - float(r.pi[t][sel].sum())) <= MASS_TOL, \
-                        f"b={b} h={h} row={i}: mass {mass[b0 + t]} vs {r.pi[t][sel].sum()}"
+                    nd = check_selection(sel, r, t, p32(p), f"b={b} h={h} row={i}", top_k=s.top_k)
+                    if s.top_k == 0:
+                        assert abs(float(mass[b0 + t]) - float(r.pi[t][sel].sum())) <= MASS_TOL, \
+                            f"b={b} h={h} row={i}: mass {mass[b0 + t]} vs {r.pi[t][sel].sum()}"
                     if nd:
                         ref_out[t] = oracle.attend_set(x, b, h, int(i), sel)
                     ndiff += nd

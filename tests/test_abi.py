@@ -46,11 +46,13 @@ def test_struct_layout_matches_c():
 #include <stdio.h>
 #include "rtp.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(rtp_config), offsetof(rtp_config, max_seq),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(rtp_config), offsetof(rtp_config, max_seq),
          offsetof(rtp_config, rope_base), offsetof(rtp_config, wq_index),
-         offsetof(rtp_config, max_select), offsetof(rtp_config, max_chunk));
-  printf("%zu %zu %zu\n", sizeof(rtp_decode_stats), offsetof(rtp_decode_stats, sel_index_cap),
-         sizeof(rtp_cache_view));
+         offsetof(rtp_config, max_select), offsetof(rtp_config, max_chunk),
+         offsetof(rtp_config, index_bf16), offsetof(rtp_config, top_k));
+  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(rtp_decode_stats), offsetof(rtp_decode_stats, sel_index_cap),
+         sizeof(rtp_cache_view), offsetof(rtp_cache_view, idx_bf16), sizeof(rtp_prefill_stats),
+         offsetof(rtp_prefill_stats, row_sel_cap));
   return 0;
 }
 '''
@@ -62,9 +64,13 @@ int main(void) {
         a, b = subprocess.check_output([exe], text=True).splitlines()
     cfg = rtp.rtp_config
     assert [int(t) for t in a.split()] == [C.sizeof(cfg), cfg.max_seq.offset, cfg.rope_base.offset,
-                                          cfg.wq_index.offset, cfg.max_select.offset, cfg.max_chunk.offset]
+                                          cfg.wq_index.offset, cfg.max_select.offset, cfg.max_chunk.offset,
+                                          cfg.index_bf16.offset, cfg.top_k.offset]
     st = rtp.rtp_decode_stats
-    assert [int(t) for t in b.split()] == [C.sizeof(st), st.sel_index_cap.offset, C.sizeof(rtp.rtp_cache_view)]
+    ps = rtp.rtp_prefill_stats
+    assert [int(t) for t in b.split()] == [C.sizeof(st), st.sel_index_cap.offset, C.sizeof(rtp.rtp_cache_view),
+                                          rtp.rtp_cache_view.idx_bf16.offset, C.sizeof(ps),
+                                          ps.row_sel_cap.offset]
 
 
 def _cfg(**kw):
@@ -83,7 +89,7 @@ def _cfg(**kw):
                                  dict(n_kv_heads=3), dict(window=0), dict(n_sink=-1), dict(max_seq=0),
                                  dict(max_select=65), dict(batch=0), dict(head_class=None),
                                  dict(n_q_heads=64, n_kv_heads=2), dict(rope_base=1.0), dict(sm_scale=-1.0),
-                                 dict(max_chunk=-1), dict(max_seq=1 << 31), dict(wq_index=None),
+                                 dict(max_chunk=-1), dict(max_seq=1 << 31), dict(wq_index=None), dict(index_bf16=2), dict(top_k=-1), dict(prefill_dense=3),
                                  dict(wk_index=None), dict(top_p=float("nan")), dict(max_select=-1)])
 def test_create_rejects_bad_config_on_host(lib, bad):
     cfg, keep = _cfg(**bad)

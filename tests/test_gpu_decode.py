@@ -135,3 +135,42 @@ def test_decode_128k_full_size():
 
 
 _state = {}
+
+
+def test_decode_bf16_index_keys():
+    # bf16 index-key storage: the oracle rounds its fp64 index keys to bf16 the same way
+    run_decode(synth.generate(synth.spec("toy_decode_4k", index_bf16=True)))
+    run_decode(synth.generate(synth.spec("decode_128k", prefix=16383, index_bf16=True,
+                                         needles=(1, 16, 1024, 1, 16, 1024, 1, 16))))
+
+
+def test_decode_1m_bf16_index_keys():
+    # the full 1M workload with bf16 index keys (half the index stream), p = 0.9
+    x = synth.generate(synth.spec("decode_1m", index_bf16=True))
+    res = run_decode(x, top_p=0.9, heads=list(x.spec.retrieval_heads) + [1, 31])
+    counts = [v[0] for v in res["summary"].values()]
+    assert max(counts) >= 1000 and min(counts) <= 16
+
+
+@pytest.mark.parametrize("k", [1, 64, 700, 5000])
+def test_decode_fixed_top_k(k):
+    # the pages' fixed-budget ablation: each retrieval head keeps its k highest-scoring keys
+    # (5000 > N = 4096 keeps every key)
+    run_decode(synth.generate(synth.spec("toy_decode_4k", top_k=k)))
+
+
+def test_decode_fixed_top_k_ties_and_128k_layer():
+    # all index scores equal: the budget takes the lowest positions
+    x = synth.generate(synth.spec("toy_decode_4k", top_k=300, zero_index_weights=True, needles=()))
+    res = run_decode(x)
+    assert all(v[0] == 300 and v[2] == 0 for v in res["summary"].values())
+    run_decode(synth.generate(synth.spec("decode_128k", prefix=16383, top_k=4096,
+                                         needles=(1, 16, 1024, 1, 16, 1024, 1, 16))))
+
+
+@pytest.mark.parametrize("k", [4096, 16384])
+def test_decode_1m_fixed_top_k(k):
+    # the pages' budgets (4096 and 16384 tokens) at 1M keys
+    x = synth.generate(synth.spec("decode_1m", top_k=k))
+    res = run_decode(x, heads=list(x.spec.retrieval_heads) + [2])
+    assert all(v[0] == k for (b, h), v in res["summary"].items())

@@ -162,3 +162,29 @@ def test_prefill_chunk_larger_than_cache_is_rejected():
     with pytest.raises(RTPError):
         layer.prefill_chunk(torch_bf16(x.q))
     layer.close()
+
+
+def test_prefill_bf16_index_keys():
+    # bf16 index-key storage feeds the same tensor-core scoring (its hi/lo split is exact)
+    run_prefill(small(prefix=700, chunk=200, window=128, index_bf16=True))
+    run_prefill(small(prefix=0, chunk=260, index_bf16=True), top_p=0.5)
+
+
+def test_prefill_fixed_top_k():
+    run_prefill(small(prefix=600, chunk=200, window=128, top_k=40))
+    # all ties: each row keeps its lowest min(k, pos + 1) positions
+    x = small(prefix=0, chunk=150, zero_index_weights=True, needles=(), top_k=25)
+    res = run_prefill(x, exact_sets=True)
+    for (b, h), (cnt, cnt_ref, nd) in res["summary"].items():
+        assert np.array_equal(cnt, np.minimum(25, np.arange(150) + 1)) and nd == 0
+
+
+def test_prefill_dense_retrieval_heads():
+    # the pages' own prefill: retrieval heads attend to every causal key; decode still selects
+    from long_context_sparse_idx16_b200 import Layer
+    from parity import run_decode
+
+    x = small(prefix=500, chunk=180, window=64, prefill_dense=True)
+    run_prefill(x, sets=None)
+    xd = synth.generate(synth.spec("toy_decode_4k", prefill_dense=True))
+    run_decode(xd)

@@ -386,3 +386,85 @@ def test_many_needles_form_the_top_of_the_order():
         assert sel <= nset or nset <= sel
         checked += 1
     assert checked >= 5
+
+
+# ---------------------------------------------------------------- bf16 index-key storage
+
+
+def _bf16_nearest_by_enumeration(x: float) -> float:
+    """The bf16 value nearest to x, ties to the even significand: the bf16 neighbours of x
+    (from its float32 bits) compared in exact rational arithmetic."""
+    from fractions import Fraction
+
+    u = int(np.array([np.float32(x)]).view(np.uint32)[0]) & 0xFFFF0000
+    cands = []
+    for d in range(-2, 3):
+        v = (u + (d << 16)) & 0xFFFFFFFF
+        c = float(np.array([v], dtype=np.uint32).view(np.float32)[0])
+        if np.isfinite(c):
+            cands.append((c, v >> 16))
+    X = Fraction(x)
+    return min(cands, key=lambda cv: (abs(Fraction(cv[0]) - X), cv[1] & 1))[0]
+
+
+def test_round_bf16_matches_exact_nearest_even():
+    rng = np.random.default_rng(3)
+    xs = list(rng.standard_normal(3000) * 4.0) + list(rng.standard_normal(500) * 1e-3)
+    # exact halfway cases: 1 + 2^-8 lies between 1 and 1 + 2^-7 (even: 1); 1 + 3 * 2^-8 between
+    # 1 + 2^-7 and 1 + 2^-6 (even: 1 + 2^-6)
+    xs += [1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 0.0, 2.0, -0.5, 1 + 2 ** -9]
+    for x in xs:
+        assert oracle.round_bf16(x) == _bf16_nearest_by_enumeration(x), x
+    assert oracle.round_bf16(1 + 2 ** -8) == 1.0 and oracle.round_bf16(1 + 3 * 2 ** -8) == 1 + 2 ** -6
+
+
+def test_bf16_index_keys_change_scores_only_by_key_rounding():
+    # keys whose projections are exact in bf16 (weights and keys small dyadic numbers) give the
+    # same scores with fp32 and bf16 storage; a weight with more significant bits moves them
+    rng = np.random.default_rng(4)
+    D, r, n = 128, 16, 40
+    k = rng.integers(-4, 5, size=(n, 1, D)).astype(np.float32)
+    q = rng.integers(-4, 5, size=D).astype(np.float32)
+    wq = np.zeros((D, r), np.float32)
+    wk = np.zeros((D, r), np.float32)
+    for c in range(r):  # each index dim reads one key dim with weight 1/4: exact in bf16
+        wq[c, c] = wk[c, c] = 0.25
+    kb = synth.f32_to_bf16_bits(k)
+    qb = synth.f32_to_bf16_bits(q)
+    s32 = oracle.index_scores(kb, 0, qb, wq, wk)
+    s16 = oracle.index_scores(kb, 0, qb, wq, wk, index_bf16=True)
+    assert np.array_equal(s32, s16)
+    wk2 = wk.copy()
+    wk2[0, 0] = 0.25 + 2 ** -12  # 11 significant bits: bf16 storage rounds the key component
+    s32 = oracle.index_scores(kb, 0, qb, wq, wk2)
+    s16 = oracle.index_scores(kb, 0, qb, wq, wk2, index_bf16=True)
+    kt = k[:, 0].astype(np.float64) @ wk2.astype(np.float64)
+    qt = q.astype(np.float64) @ wq.astype(np.float64)
+    want = np.array([[oracle.round_bf16(v) for v in row] for row in kt]) @ qt
+    assert np.allclose(s16, want, rtol=0, atol=1e-12)
+    assert not np.array_equal(s32, s16)
+
+
+# ---------------------------------------------------------------- fixed top-k (ablation mode)
+
+
+def test_topk_equals_topp_at_the_mass_of_its_set():
+    # with distinct scores, the k highest keys are exactly the top-p set for p = their mass
+    # (the already pinned top-p rule), for every k
+    rng = np.random.default_rng(8)
+    s = rng.standard_normal(300) * 3.0
+    for k in (1, 2, 7, 50, 299):
+        tk = oracle.topk(s, k)
+        tp = oracle.topp(s, tk.mass * (1 - 1e-12))
+        assert tk.count == k and np.array_equal(tk.selected, tp.selected)
+        assert tk.mass == pytest.approx(float(np.sort(softmax(s))[::-1][:k].sum()), rel=1e-12)
+
+
+def test_topk_ties_and_limits():
+    s = np.zeros(40)
+    tk = oracle.topk(s, 9)
+    assert tk.count == 9 and np.array_equal(tk.selected, np.arange(9))  # all equal: lowest positions
+    s = np.array([1.0, 3.0, 3.0, 2.0, 3.0])
+    assert np.array_equal(oracle.topk(s, 2).selected, [1, 2])  # the tie at 3 goes to the lower positions
+    assert np.array_equal(oracle.topk(s, 4).selected, [1, 2, 3, 4])
+    assert oracle.topk(s, 99).count == 5  # k >= n keeps every key
