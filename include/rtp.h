@@ -187,7 +187,7 @@ rtp_status rtp_truncate(rtp_layer* layer, int64_t new_len);
  * launch stream around every kernel it launches, and runs every kernel on the call's stream
  * in order (no internal fork), so each recorded time belongs to one kernel alone.  rtp_profile_read synchronises on the
  * recorded events, returns the summed device time (ms) and launch count of the named kernel
- * ("append_kv", "q_prep", "decode_select", "decode_gather", "decode_swa", "swa_merge",
+ * ("append_kv", "q_prep", "decode_select", "decode_topk", "decode_gather", "decode_swa", "swa_merge",
  * "dense_fill", "prefill_*"; NULL: all kernels together), and clears that kernel's record. */
 rtp_status rtp_profile_enable(rtp_layer* layer, int on);
 rtp_status rtp_profile_read(rtp_layer* layer, const char* kernel, double* total_ms, int64_t* launches);

@@ -23,90 +23,99 @@ namespace {
 
 constexpr float kFp16Max = 65504.f;
 
-// Retrieval heads whose index weights are staged in shared memory at once (8 KB each).
-constexpr int kWHeads = 8;
+// Append work split: blockIdx.z == 0 writes RoPE(k) and v of up to kAppTok tokens; blockIdx.z
+// == 1 + hr computes retrieval head hr's index keys of the same tokens (its 8 KB of weights
+// read once for the group).  A one-token decode append is 1 + Hr small CTAs per sequence, all
+// in flight at once.
+constexpr int kAppThreads = 128;
+constexpr int kAppTok = 8;
 
 template <bool kBf16>
-__global__ void __launch_bounds__(256) append_kv_kernel(
+__global__ void __launch_bounds__(kAppThreads) append_kv_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int T, int Hkv,
     int Hr, int64_t pos0, int64_t max_seq, const double* __restrict__ theta,
     const float* __restrict__ wk, const int16_t* __restrict__ ret_head, int group,
     __half* __restrict__ kc, __half* __restrict__ vc, float* __restrict__ idx, __nv_bfloat16* __restrict__ idx_b,
     __half* __restrict__ idx_hl, uint32_t* __restrict__ err) {
-  const int t = blockIdx.x;  // token within the appended block
-  const int b = blockIdx.y;
-  const int64_t pos = pos0 + t;
-  extern __shared__ float smem_f[];
-  float* ks = smem_f;                 // [Hkv][D] pre-RoPE key (fp32)
-  float* ws = smem_f + Hkv * kD;      // [<= kWHeads][D][r] index weights
-  __shared__ float cs[kHalfD], sn[kHalfD];
-
-  const __nv_bfloat16* kt = k + ((int64_t)b * T + t) * Hkv * kD;
-  const __nv_bfloat16* vt = v + ((int64_t)b * T + t) * Hkv * kD;
-  // every global read of the token is issued before any is used: one memory round trip (the
-  // index weights go straight to shared memory with cp.async, all copies in flight at once)
-  const int nw = min(Hr, kWHeads);
-  for (int i = threadIdx.x; i < nw * kD * kR / 4; i += blockDim.x) cp_async16(ws + 4 * i, wk + 4 * i, 16);
-  cp_async_commit();
-  for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) ks[i] = __bfloat162float(kt[i]);
-  if (threadIdx.x < kHalfD) rope_cos_sin(pos, theta[threadIdx.x], &cs[threadIdx.x], &sn[threadIdx.x]);
-  bool bad = false;
-  for (int i = threadIdx.x; i < Hkv * kD; i += blockDim.x) {
-    const int g = i / kD, d = i % kD;
-    const float x = __bfloat162float(vt[i]);
-    bad |= !(fabsf(x) <= kFp16Max);
-    vc[(((int64_t)b * Hkv + g) * max_seq + pos) * kD + d] = __float2half_rn(x);
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-
-  for (int i = threadIdx.x; i < Hkv * kHalfD; i += blockDim.x) {
-    const int g = i / kHalfD, c = i % kHalfD;
-    const float x0 = ks[g * kD + c], x1 = ks[g * kD + c + kHalfD];
-    const float y0 = x0 * cs[c] - x1 * sn[c];
-    const float y1 = x1 * cs[c] + x0 * sn[c];
-    bad |= !(fabsf(y0) <= kFp16Max) || !(fabsf(y1) <= kFp16Max);
-    __half* dst = kc + (((int64_t)b * Hkv + g) * max_seq + pos) * kD;
-    dst[c] = __float2half_rn(y0);
-    dst[c + kHalfD] = __float2half_rn(y1);
-  }
-  // index keys: Hr x r outputs, one thread each, a 128-term fp32 dot product in a fixed order
-  for (int h0 = 0; h0 < Hr; h0 += kWHeads) {
-    const int nh = min(Hr - h0, kWHeads);
-    if (h0 > 0) {  // later groups of heads (more than kWHeads retrieval heads)
+  const int t0 = blockIdx.x * kAppTok, b = blockIdx.y, role = blockIdx.z;
+  const int nt = min(kAppTok, T - t0);
+  const int tid = threadIdx.x;
+  if (role == 0) {
+    // ---- K (RoPE'd) and V rows into the fp16 cache
+    __shared__ float cs[kHalfD], sn[kHalfD];
+    bool bad = false;
+    for (int u = 0; u < nt; ++u) {
+      const int t = t0 + u;
+      const int64_t pos = pos0 + t;
+      __syncthreads();  // the previous token's angles are consumed
+      if (tid < kHalfD) rope_cos_sin(pos, theta[tid], &cs[tid], &sn[tid]);
       __syncthreads();
-      for (int i = threadIdx.x; i < nh * kD * kR / 4; i += blockDim.x)
-        reinterpret_cast<float4*>(ws)[i] = reinterpret_cast<const float4*>(wk + (int64_t)h0 * kD * kR)[i];
-      __syncthreads();
-    }
-    for (int o = threadIdx.x; o < nh * kR; o += blockDim.x) {
-      const int hl = o / kR, c = o % kR, hr = h0 + hl;
-      const float* w = ws + hl * kD * kR + c;
-      const float* x = ks + (ret_head[hr] / group) * kD;
-      const int64_t row = ((int64_t)b * Hr + hr) * max_seq + pos;
-      float acc;
-      if (kBf16) {
-        // bf16 storage: the projection in fp64, then one rounding to the nearest bf16 (even on
-        // ties), so the stored key is the exact projection's bf16 rounding
-        double a64 = 0.0;
-#pragma unroll 16
-        for (int d = 0; d < kD; ++d) a64 = fma((double)w[d * kR], (double)x[d], a64);
-        const __nv_bfloat16 kb = __double2bfloat16(a64);
-        idx_b[row * kR + c] = kb;
-        acc = __bfloat162float(kb);
-      } else {
-        acc = 0.f;
-#pragma unroll 16
-        for (int d = 0; d < kD; ++d) acc = fmaf(w[d * kR], x[d], acc);
-        idx[row * kR + c] = acc;
+      const __nv_bfloat16* kt = k + ((int64_t)b * T + t) * Hkv * kD;
+      const __nv_bfloat16* vt = v + ((int64_t)b * T + t) * Hkv * kD;
+      for (int i = tid; i < Hkv * kD; i += kAppThreads) {
+        const int g = i / kD, d = i % kD;
+        const float x = __bfloat162float(vt[i]);
+        bad |= !(fabsf(x) <= kFp16Max);
+        vc[(((int64_t)b * Hkv + g) * max_seq + pos) * kD + d] = __float2half_rn(x);
       }
-      // the same key split as fp16 hi + lo, for the tensor-core scoring of prefill
+      for (int i = tid; i < Hkv * kHalfD; i += kAppThreads) {
+        const int g = i / kHalfD, c = i % kHalfD;
+        const float x0 = __bfloat162float(kt[g * kD + c]), x1 = __bfloat162float(kt[g * kD + c + kHalfD]);
+        const float y0 = x0 * cs[c] - x1 * sn[c];
+        const float y1 = x1 * cs[c] + x0 * sn[c];
+        bad |= !(fabsf(y0) <= kFp16Max) || !(fabsf(y1) <= kFp16Max);
+        __half* dst = kc + (((int64_t)b * Hkv + g) * max_seq + pos) * kD;
+        dst[c] = __float2half_rn(y0);
+        dst[c + kHalfD] = __float2half_rn(y1);
+      }
+    }
+    if (bad) atomicOr(err, kErrRange);
+    return;
+  }
+  // ---- index keys of retrieval head hr: 16 outputs x 8 partial sums of 16 dims, a fixed
+  // order (then a 3-step shuffle tree) so every append gives the same bits
+  const int hr = role - 1;
+  const int o = tid >> 3, part = tid & 7;
+  const int g = ret_head[hr] / group;
+  float w[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) w[e] = wk[((int64_t)hr * kD + part * 16 + e) * kR + o];
+  for (int u = 0; u < nt; ++u) {
+    const int t = t0 + u;
+    const int64_t pos = pos0 + t;
+    const __nv_bfloat16* kt = k + (((int64_t)b * T + t) * Hkv + g) * kD + part * 16;
+    float x[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[e] = __bfloat162float(kt[e]);
+    const int64_t row = ((int64_t)b * Hr + hr) * max_seq + pos;
+    float acc;
+    if (kBf16) {
+      // bf16 storage: the projection in fp64, then one rounding to the nearest bf16 (even on
+      // ties), so the stored key is the exact projection's bf16 rounding
+      double a64 = 0.0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) a64 = fma((double)w[e], (double)x[e], a64);
+      a64 += __shfl_xor_sync(0xffffffffu, a64, 1);
+      a64 += __shfl_xor_sync(0xffffffffu, a64, 2);
+      a64 += __shfl_xor_sync(0xffffffffu, a64, 4);
+      const __nv_bfloat16 kb = __double2bfloat16(a64);
+      if (part == 0) idx_b[row * kR + o] = kb;
+      acc = __bfloat162float(kb);
+    } else {
+      acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc = fmaf(w[e], x[e], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      if (part == 0) idx[row * kR + o] = acc;
+    }
+    if (part == 0) {  // the same key split as fp16 hi + lo, for the tensor-core scoring of prefill
       const __half hh = __float2half_rn(acc);
-      idx_hl[row * (2 * kR) + c] = hh;
-      idx_hl[row * (2 * kR) + kR + c] = __float2half_rn(acc - __half2float(hh));
+      idx_hl[row * (2 * kR) + o] = hh;
+      idx_hl[row * (2 * kR) + kR + o] = __float2half_rn(acc - __half2float(hh));
     }
   }
-  if (bad) atomicOr(err, kErrRange);
 }
 
 // One CTA per (row, batch, group of kQHeads heads): RoPE'd fp32 query for each head, and the
@@ -176,14 +185,10 @@ __global__ void __launch_bounds__(128) q_prep_kernel(
 
 cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T,
                              cudaStream_t st) {
-  dim3 grid(T, L->B);
-  const int nw = L->Hr < kWHeads ? L->Hr : kWHeads;
-  const size_t smem = ((size_t)L->Hkv * kD + (size_t)nw * kD * kR) * sizeof(float);
+  dim3 grid((T + kAppTok - 1) / kAppTok, L->B, 1 + L->Hr);
   auto fn = L->index_bf16 ? append_kv_kernel<true> : append_kv_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  fn<<<grid, 256, smem, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta, L->wk, L->d_ret_head,
-                              L->group, L->kc, L->vc, L->idx, L->idx_b, L->idx_hl, L->err);
+  fn<<<grid, kAppThreads, 0, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta, L->wk, L->d_ret_head,
+                                   L->group, L->kc, L->vc, L->idx, L->idx_b, L->idx_hl, L->err);
   return cudaGetLastError();
 }
 

@@ -22,8 +22,8 @@
 //         down) -> Z, T = ceil(p Z), crossing bin, whose exact order-key range is found by
 //         bisection;
 //      R  refinement: the crossing range of order keys is split 16 ways by bit slices, with
-//         the mass of each slice and the first 16 keys of the range captured; once a row's
-//         range holds <= 16 keys they are sorted (key desc, j asc) for the exact cut; a range
+//         the mass of each slice and the first 8 keys of the range captured; once a row's
+//         range holds <= 8 keys they are sorted (key desc, j asc) for the exact cut; a range
 //         that shrinks to one key value is an exact tie group, resolved by
 //      T  an ordered count of the tied positions.
 //  prefill_attn_kernel -- 256 threads, two per row (each on half of a tile's 64 columns).
@@ -42,7 +42,7 @@ constexpr int kRowsR = kTcRows;  // 128 query rows per CTA (TMEM lanes)
 constexpr int kKeysR = kTcKeys;  // 64 keys per tile
 constexpr int kBins = 16;        // pass B: bins of width 1 below the row max
 constexpr int kSlices = 16;      // refinement: slices of the crossing key range per level
-constexpr int kCand = 16;        // keys captured per row in a refinement walk
+constexpr int kCand = 8;         // keys captured per row in a refinement walk
 constexpr int kLevels = 10;      // refinement levels (4 key bits each, with margin)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -133,14 +133,17 @@ constexpr uint32_t kSelStages = 3;   // key tiles of the TMA ring
 constexpr uint32_t kSOffQ = 0;                                       // query tile, 8 KB
 constexpr uint32_t kSOffK = kSOffQ + kTcQBytes;                      // key ring, 3 x 4 KB
 constexpr uint32_t kSOffH = kSOffK + kSelStages * kTcKBytes;         // [slice][row] u64, 16 KB
-constexpr uint32_t kSOffC = kSOffH + kSlices * kRowsR * 8;           // [cand][row] u64, 16 KB
-constexpr uint32_t kSOffBar = kSOffC + kCand * kRowsR * 8;           // full[3], done[2], TMEM base
-constexpr uint32_t kSelSmem = kSOffBar + 64;  // about 54 KB: four CTAs (4 x 128 TMEM columns) per SM
+constexpr uint32_t kSOffC = kSOffH + kSlices * kRowsR * 8;           // [cand][row] u64, 8 KB
+constexpr uint32_t kSOffBar = kSOffC + kCand * kRowsR * 8;           // full[3], done, TMEM base
+constexpr uint32_t kSelSmem = kSOffBar + 64;  // about 44 KB: five CTAs (5 x 64 TMEM columns) per SM
 static_assert(kSelStages <= 3, "the barrier block holds three stage barriers");
-constexpr uint32_t kSelTmemCols = 128;                               // two 64-column score buffers
+// One 64-column TMEM score buffer per CTA: five CTAs fit an SM (TMEM 512 columns, shared
+// memory 228 KB), so the 640 CTAs of a 16K-row chunk with 5 retrieval heads run in one wave;
+// the scores of tile t + 1 are issued as soon as every thread has read tile t.
+constexpr uint32_t kSelTmemCols = 64;
 
 // Walks over the key tiles [0, ntiles) of one (sequence, retrieval head): thread 0 keeps
-// kSelStages TMA copies in flight and issues the scores of tile t + 1 before tile t is read;
+// kSelStages TMA copies in flight and issues the scores of tile t + 1 once tile t is read;
 // body(t, c0, s, lim) gets this thread's row's scores of tile t in groups of 16 (columns c0 ..
 // c0 + 15, s[0..15]) and the last causal column lim of the tile.  g counts tiles over all walks
 // (mbarrier phases).  A wait that runs out clears ok in every thread; later walks then do
@@ -155,7 +158,7 @@ struct SelWalk {
   bool mma_pending;                   // scores of tile g issued and not waited on
 
   __device__ uint32_t full_bar(uint32_t gt) const { return sbase + kSOffBar + 8u * (gt % kSelStages); }
-  __device__ uint32_t done_bar(uint32_t gt) const { return sbase + kSOffBar + 24u + 8u * (gt & 1u); }
+  __device__ uint32_t done_bar(uint32_t) const { return sbase + kSOffBar + 24u; }
   __device__ uint32_t ktile(uint32_t gt) const { return sbase + kSOffK + (gt % kSelStages) * kTcKBytes; }
 
   template <typename Body>
@@ -170,48 +173,48 @@ struct SelWalk {
       inflight_hi = g + (uint32_t)min((int64_t)kSelStages, ntiles);
       okw = mbar_wait(full_bar(g), (g / kSelStages) & 1u);
       inflight_lo = g + 1;
-      if (okw) tc_issue_scores(tmem + (g & 1u) * kTcKeys, sbase + kSOffQ, ktile(g), done_bar(g));
+      if (okw) tc_issue_scores(tmem, sbase + kSOffQ, ktile(g), done_bar(g));
       mma_pending = okw;
     }
     for (int64_t t = 0; t < ntiles; ++t) {
       const uint32_t gt = g + (uint32_t)t;
-      bool issued_next = false;  // thread 0: the scores of tile gt + 1 are in flight
-      if (tid == 0 && t + 1 < ntiles && okw) {
-        okw = mbar_wait(full_bar(gt + 1), ((gt + 1) / kSelStages) & 1u);
-        inflight_lo = gt + 2;
-        if (okw) {
-          tc_issue_scores(tmem + ((gt + 1) & 1u) * kTcKeys, sbase + kSOffQ, ktile(gt + 1), done_bar(gt + 1));
-          issued_next = true;
-        }
-      }
-      if (tid != 0 || mma_pending) okw = mbar_wait(done_bar(gt), (gt >> 1) & 1u) && okw;
+      // the scores of tile gt: one completion of the done barrier per tile (parity gt & 1)
+      if (tid != 0 || mma_pending) okw = mbar_wait(done_bar(gt), gt & 1u) && okw;
       tc_fence_after();
-      float s[kTcKeys];
       __syncwarp();  // the loads are warp-collective: reconverge after thread 0's work
+      // the body sees the tile in four 16-column groups, each loaded from TMEM on its own (one
+      // copy of the unrolled body per walk), with the last causal column lim of the tile
+      const int lim = causal_lim(pos, t);
+#pragma unroll 1
+      for (int q = 0; q < kTcKeys / 16; ++q) {
+        float s[16];
+        tmem_ld16(lane_addr + 16u * q, s);
+        tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < kTcKeys / 16; ++q) tmem_ld16(lane_addr + (gt & 1u) * kTcKeys + 16u * q, s + 16 * q);
-      tmem_ld_wait();
+        for (int i = 0; i < 16; ++i) s[i] += 0.0f;  // -0 -> +0: equal scores, equal order keys
+        body(t, 16 * q, s, lim);
+      }
       tc_fence_before();
+      // every thread has read tile gt: the buffer takes the scores of tile gt + 1 next
       if (!__syncthreads_and(okw ? 1 : 0)) {
         ok = false;
-        if (tid == 0) mma_pending = issued_next;  // drain() waits for the scores of tile gt + 1
+        if (tid == 0) mma_pending = false;
         g = gt + 1;
         return;
       }
       if (tid == 0) {
-        mma_pending = issued_next;
+        mma_pending = false;
         if (t + kSelStages < ntiles) {  // the stage of tile gt is free: its scores are done
           tc_load_keys(ktile(gt), map, row0, t + kSelStages, full_bar(gt));
           inflight_hi = gt + kSelStages + 1;
         }
+        if (t + 1 < ntiles) {
+          okw = mbar_wait(full_bar(gt + 1), ((gt + 1) / kSelStages) & 1u);
+          inflight_lo = gt + 2;
+          if (okw) tc_issue_scores(tmem, sbase + kSOffQ, ktile(gt + 1), done_bar(gt + 1));
+          mma_pending = okw;
+        }
       }
-#pragma unroll
-      for (int i = 0; i < kTcKeys; ++i) s[i] += 0.0f;  // -0 -> +0: equal scores, equal order keys
-      // the body sees the tile in four 16-column groups (a smaller unrolled body), told whether
-      // every column of the group is causal for this row
-      const int lim = causal_lim(pos, t);
-#pragma unroll
-      for (int q = 0; q < kTcKeys / 16; ++q) body(t, 16 * q, s + 16 * q, lim);
     }
     g += (uint32_t)ntiles;
   }
@@ -220,7 +223,7 @@ struct SelWalk {
   __device__ void drain() {
     if (threadIdx.x != 0) return;
     for (uint32_t gt = inflight_lo; gt < inflight_hi; ++gt) mbar_wait(full_bar(gt), (gt / kSelStages) & 1u);
-    if (mma_pending) mbar_wait(done_bar(g), (g >> 1) & 1u);
+    if (mma_pending) mbar_wait(done_bar(g), g & 1u);
   }
 };
 
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kSOffBar + 48);
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kSelTmemCols);
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(sbase + kSOffBar + 8u * i, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(sbase + kSOffBar + 8u * i, 1);
     fence_mbar_init();
   }
   {
