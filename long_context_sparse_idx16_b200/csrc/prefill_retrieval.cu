@@ -21,10 +21,13 @@
 //      B  16 bins of m - s rounded to an integer (the last one holding everything from 14.5
 //         down) -> Z, T = ceil(p Z), crossing bin, whose exact order-key range is found by
 //         bisection;
-//      R  refinement: the crossing range of order keys is split 16 ways by bit slices, with
-//         the mass of each slice and the first 8 keys of the range captured; once a row's
-//         range holds <= 8 keys they are sorted (key desc, j asc) for the exact cut; a range
-//         that shrinks to one key value is an exact tie group, resolved by
+//      R  refinement: each walk sums the mass of 16 bit slices of the crossing range of order
+//         keys and captures the range's keys (in position order) into a per-row global list;
+//         a row whose range holds at most 2048 keys finishes from its list (narrowing it 16
+//         ways at a time, then sorting the last <= 8 keys, key desc, j asc, for the exact cut;
+//         a single key value is an exact tie group, cut at its n-th position); otherwise the
+//         range narrows to the crossing slice for the next walk, and a range that shrinks to
+//         one key value with more members than the list holds is resolved by
 //      T  an ordered count of the tied positions.
 //  prefill_attn_kernel -- 256 threads, two per row (each on half of a tile's 64 columns).
 //    Walks the key tiles in order: the index scores of tile t + 1 (computed one tile ahead)
@@ -42,7 +45,8 @@ constexpr int kRowsR = kTcRows;  // 128 query rows per CTA (TMEM lanes)
 constexpr int kKeysR = kTcKeys;  // 64 keys per tile
 constexpr int kBins = 16;        // pass B: bins of width 1 below the row max
 constexpr int kSlices = 16;      // refinement: slices of the crossing key range per level
-constexpr int kCand = 8;         // keys captured per row in a refinement walk
+constexpr int kCand = 8;         // keys sorted in registers for the final cut
+constexpr int kCapG = kPfCapture; // keys of the crossing range captured per row in a refinement walk
 constexpr int kLevels = 10;      // refinement levels (4 key bits each, with margin)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -59,6 +63,7 @@ struct RetArgs {
   const float* q_rot;         // [B][C][Hq][D]
   const float* q_idx;         // [B][C][Hr][r]
   uint2* cut;                 // [B][Hr][C]: (t_key, tiecut)
+  unsigned long long* capture; // [B][Hr][C / 128][kCapG][128]: (key << 32 | ~j) of a row's crossing range
   float scale_log2;
   float* out;                 // [B][C][Hq][D]
   int32_t* sel_count;         // [B][C][Hr] or nullptr
@@ -133,9 +138,8 @@ constexpr uint32_t kSelStages = 3;   // key tiles of the TMA ring
 constexpr uint32_t kSOffQ = 0;                                       // query tile, 8 KB
 constexpr uint32_t kSOffK = kSOffQ + kTcQBytes;                      // key ring, 3 x 4 KB
 constexpr uint32_t kSOffH = kSOffK + kSelStages * kTcKBytes;         // [slice][row] u64, 16 KB
-constexpr uint32_t kSOffC = kSOffH + kSlices * kRowsR * 8;           // [cand][row] u64, 8 KB
-constexpr uint32_t kSOffBar = kSOffC + kCand * kRowsR * 8;           // full[3], done, TMEM base
-constexpr uint32_t kSelSmem = kSOffBar + 64;  // about 44 KB: five CTAs (5 x 64 TMEM columns) per SM
+constexpr uint32_t kSOffBar = kSOffH + kSlices * kRowsR * 8;         // full[3], done, TMEM base
+constexpr uint32_t kSelSmem = kSOffBar + 64;  // about 36 KB: five CTAs (5 x 64 TMEM columns) per SM
 static_assert(kSelStages <= 3, "the barrier block holds three stage barriers");
 // One 64-column TMEM score buffer per CTA: five CTAs fit an SM (TMEM 512 columns, shared
 // memory 228 KB), so the 640 CTAs of a 16K-row chunk with 5 retrieval heads run in one wave;
@@ -285,7 +289,9 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
   // budget (then the sums are counts)
   auto weight = [&](float s, float mx) -> unsigned long long { return topk ? 1ull : mass64(s, mx, scale); };
   unsigned long long* hist = reinterpret_cast<unsigned long long*>(sm + kSOffH) + tid;  // [slice * 128]
-  unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + kSOffC) + tid;  // [k * 128]
+  // this row's capture list, entry k at cap[k * 128] (the CTA's rows interleaved: coalesced)
+  unsigned long long* cap = a.capture + (((int64_t)b * a.Hr + hr) * ((a.C + kRowsR - 1) / kRowsR) + tile) *
+                                             (int64_t)kCapG * kRowsR + tid;
 
   // ---- pass A: the row max
   float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four chains: no serial max
@@ -345,7 +351,10 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
     mode = kModeKeys;
   }
 
-  // ---- refinement: 16-way bit slices of the crossing key range until <= 16 keys remain
+  // ---- refinement: each walk captures the keys of a row's crossing key range (in position
+  // order) into its global list while it sums the mass of 16 bit slices of the range.  A row
+  // whose range holds at most kCapG keys then finishes from its list alone (no further walk);
+  // otherwise its range narrows to the crossing slice for the next walk.
   for (int level = 0; level < kLevels; ++level) {
     if (!__syncthreads_or(mode == kModeKeys)) break;
     const bool mine = mode == kModeKeys;
@@ -360,43 +369,99 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
         const uint32_t key = order_key(s[c]);
         if (c0 + c <= lim && key - klo <= span) {
           hist[(int)((key - klo) >> shift) * kRowsR] += weight(s[c], m);
-          if (nc < kCand)
-            cand[nc * kRowsR] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)(t * kKeysR + c0 + c));
+          if (nc < kCapG)
+            cap[(int64_t)nc * kRowsR] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)(t * kKeysR + c0 + c));
           ++nc;
         }
       }
     });
     if (!mine) continue;
-    if (nc <= kCand) {
-      // every key of the range is a captured candidate: exact cut by sorting them
-      unsigned long long cv[kCand];
-      for (int i = 0; i < nc; ++i) cv[i] = cand[i * kRowsR];
-      for (int i = 1; i < nc; ++i) {  // insertion sort, descending: key desc, then j asc
-        const unsigned long long v = cv[i];
-        int k = i - 1;
-        while (k >= 0 && cv[k] < v) {
-          cv[k + 1] = cv[k];
-          --k;
+    if (nc <= kCapG) {
+      // every key of the range is in the list: narrow the range over the list until at most
+      // kCand keys remain (a single key value is an exact tie group), then sort those
+      int n_in = nc;
+      while (n_in > kCand && klo != khi) {
+        for (int i = 0; i < kSlices; ++i) hist[i * kRowsR] = 0ull;
+        const uint32_t sp = khi - klo;
+        for (int i = 0; i < nc; ++i) {
+          const uint32_t key = (uint32_t)(cap[(int64_t)i * kRowsR] >> 32);
+          if (key - klo <= sp) hist[(int)((key - klo) >> shift) * kRowsR] += weight(key_to_float(key), m);
         }
-        cv[k + 1] = v;
-      }
-      unsigned long long cum = 0ull;
-      int ci = -1;
-      for (int i = 0; i < nc; ++i) {
-        cum += weight(key_to_float((uint32_t)(cv[i] >> 32)), m);
-        if (cum >= rem) {
-          ci = i;
-          break;
+        unsigned long long cum = 0ull;
+        int cs = 0;
+        for (int i = kSlices - 1; i >= 0; --i) {  // highest slice first
+          const unsigned long long hs = hist[i * kRowsR];
+          if (cum + hs >= rem) {
+            cs = i;
+            break;
+          }
+          cum += hs;
         }
-      }
-      if (ci < 0) {  // not reached: the range was chosen to hold at least rem
-        atomicOr(a.err, kErrInternal);
-        t_key = 0xFFFFFFFFu;
-        tiecut = -1;
-      } else {
-        t_key = (uint32_t)(cv[ci] >> 32);
-        tiecut = (int)(0xFFFFFFFFu - (uint32_t)cv[ci]);
+        const uint32_t nlo = klo + ((uint32_t)cs << shift);
+        const uint32_t top = nlo + ((1u << shift) - 1u);
+        khi = top < khi && top >= nlo ? top : khi;
+        klo = nlo;
+        rem -= cum;
         above += cum;
+        shift = slice_shift(klo, khi);
+        n_in = 0;
+        for (int i = 0; i < nc; ++i) n_in += ((uint32_t)(cap[(int64_t)i * kRowsR] >> 32) - klo <= khi - klo) ? 1 : 0;
+      }
+      if (n_in <= kCand) {
+        unsigned long long cv[kCand];
+        int n = 0;
+        for (int i = 0; i < nc && n < kCand; ++i) {
+          const unsigned long long e = cap[(int64_t)i * kRowsR];
+          if ((uint32_t)(e >> 32) - klo <= khi - klo) cv[n++] = e;
+        }
+        for (int i = 1; i < n; ++i) {  // insertion sort, descending: key desc, then j asc
+          const unsigned long long v = cv[i];
+          int k = i - 1;
+          while (k >= 0 && cv[k] < v) {
+            cv[k + 1] = cv[k];
+            --k;
+          }
+          cv[k + 1] = v;
+        }
+        unsigned long long cum = 0ull;
+        int ci = -1;
+        for (int i = 0; i < n; ++i) {
+          cum += weight(key_to_float((uint32_t)(cv[i] >> 32)), m);
+          if (cum >= rem) {
+            ci = i;
+            break;
+          }
+        }
+        if (ci < 0) {  // not reached: the range was chosen to hold at least rem
+          atomicOr(a.err, kErrInternal);
+          t_key = 0xFFFFFFFFu;
+          tiecut = -1;
+        } else {
+          t_key = (uint32_t)(cv[ci] >> 32);
+          tiecut = (int)(0xFFFFFFFFu - (uint32_t)cv[ci]);
+          above += cum;
+        }
+      } else {
+        // one key value with more than kCand members: the n_need-th of them in position order
+        // (the list is in position order)
+        t_key = klo;
+        const unsigned long long e = weight(key_to_float(klo), m);
+        const unsigned long long need = e ? (rem + e - 1) / e : 1ull;
+        unsigned long long seen = 0ull;
+        tiecut = -1;
+        for (int i = 0; i < nc; ++i) {
+          const unsigned long long v = cap[(int64_t)i * kRowsR];
+          if ((uint32_t)(v >> 32) == klo && ++seen == need) {
+            tiecut = (int)(0xFFFFFFFFu - (uint32_t)v);
+            break;
+          }
+        }
+        if (tiecut < 0) {
+          atomicOr(a.err, kErrInternal);
+          tiecut = 0x7FFFFFFF;
+        } else {
+          above += need * e;
+        }
       }
       mode = kModeDone;
     } else {
@@ -424,7 +489,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
         klo = nlo;
         khi = nhi;
         shift = slice_shift(nlo, nhi);
-        if (nlo == nhi) {  // one key value with more than 16 members: an exact tie group
+        if (nlo == nhi) {  // one key value with more than kCapG members: an exact tie group
           t_key = nlo;
           const unsigned long long e = weight(key_to_float(nlo), m);
           n_need = e ? (rem + e - 1) / e : 1ull;
@@ -433,7 +498,7 @@ __global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
       }
     }
   }
-  if (mode == kModeKeys) {  // not reached: ten 16-way levels split 32 bits
+  if (mode == kModeKeys) {  // not reached: the walks narrow the range 16-fold each
     atomicOr(a.err, kErrInternal);
     t_key = 0xFFFFFFFFu;
     tiecut = -1;
@@ -861,6 +926,7 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
   a.q_rot = L->q_rot;
   a.q_idx = L->q_idx;
   a.cut = L->pf_cut;
+  a.capture = L->pf_capture;
   a.scale_log2 = L->sm_scale * 1.4426950408889634f;
   a.out = out;
   a.sel_count = stats ? stats->sel_count : nullptr;

@@ -27,6 +27,9 @@ constexpr int kSelMaxGrid = 256; // CTAs of the selection grid (<= SM count)
 constexpr int kGatherChunk = 128;
 constexpr int kGatherThreads = 256;
 
+// Prefill selection: keys of a row's crossing range captured per refinement walk.
+constexpr int kPfCapture = 2048;
+
 // Fixed top-k decode selection (ablation mode): keys per chunk of its radix-select kernels.
 constexpr int kTopkChunk = 4096;
 
@@ -75,6 +78,7 @@ struct rtp_layer {
   CUtensorMap tm_idx, tm_k, tm_v;
   bool tm_ready = false;
   uint2* pf_cut = nullptr;
+  unsigned long long* pf_capture = nullptr;  // [B][Hr][max_chunk / 128][kPfCapture][128] selection lists
   // decode: the local heads' window attention runs on a second stream, forked after the
   // selection and joined back, so it overlaps the retrieval heads' gather attention
   cudaStream_t side = nullptr;

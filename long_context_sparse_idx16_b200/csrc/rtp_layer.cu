@@ -100,7 +100,7 @@ static void free_all(rtp_layer* L) {
                   L->d_loc_head, L->d_loc_cnt, L->d_local_list, L->pf_cut, L->idx_hl, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
-                  L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt};
+                  L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt, L->pf_capture};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -240,6 +240,8 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   RTP_ALLOC(L->d_local_list, L->n_local);
   RTP_ALLOC(L->idx_hl, (int64_t)B * Hr * L->max_seq * 2 * kR);
   RTP_ALLOC(L->pf_cut, (int64_t)B * (Hr > 0 ? Hr : 1) * L->max_chunk);
+  if (Hr > 0 && !L->prefill_dense)
+    RTP_ALLOC(L->pf_capture, (int64_t)B * Hr * ((L->max_chunk + 127) / 128) * kPfCapture * 128);
   RTP_ALLOC(L->q_rot, rows * Hq * kD);
   RTP_ALLOC(L->q_idx, rows * Hr * kR);
   RTP_ALLOC(L->sel_idx, P * L->max_select);
