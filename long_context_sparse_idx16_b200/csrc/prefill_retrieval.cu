@@ -30,7 +30,9 @@
 //         one key value with more members than the list holds is resolved by
 //      T  an ordered count of the tied positions.
 //  prefill_attn_kernel -- 256 threads, two per row (each on half of a tile's 64 columns).
-//    Walks the key tiles in order: the index scores of tile t + 1 (computed one tile ahead)
+//    Rows with more than 256K keys split them over several CTAs (partial softmax states merged
+//    by the last CTA of the row tile).  Walks the key tiles in order: the index scores of tile
+//    t + 1 (computed one tile ahead)
 //    and each row's cut give the rows' selection masks; a tile no row selects is skipped,
 //    otherwise its K and V rows come in by TMA, S = Q K^T runs on the tensor cores into TMEM,
 //    the masked online softmax forms P in shared memory and O += P V accumulates in TMEM.
@@ -58,12 +60,16 @@ struct RetArgs {
   int64_t P0;
   float top_p;
   int64_t top_k;              // > 0: fixed budget (counts instead of masses)
-  int sc_bits;
+  int sc_bits;                // fixed-point scale of the selection masses (62 - ceil(log2 len))
   const int16_t* ret_head;    // [Hr]
   const float* q_rot;         // [B][C][Hq][D]
   const float* q_idx;         // [B][C][Hr][r]
   uint2* cut;                 // [B][Hr][C]: (t_key, tiecut)
   unsigned long long* capture; // [B][Hr][C / 128][kCapG][128]: (key << 32 | ~j) of a row's crossing range
+  int attn_splits;            // CTAs per row tile of the attention, each on attn_split_tiles key tiles
+  int64_t attn_split_tiles;
+  float* attn_part;           // [B][Hr][C / 128][attn_splits][128][4 + D]: (m, l, count, -, o) per row
+  uint32_t* attn_ticket;      // [B][Hr][C / 128]: splits of a row tile done (the last merges)
   float scale_log2;
   float* out;                 // [B][C][Hq][D]
   int32_t* sel_count;         // [B][C][Hr] or nullptr
@@ -566,6 +572,7 @@ constexpr uint32_t kAOffBar = kAOffX + 3 * kRowsR * 4;           // ifull[3], id
 constexpr uint32_t kAttSmem = kAOffBar + 8 * 8 + 16;
 static_assert(kAOffK % 1024 == 0 && kAOffV % 1024 == 0 && kAOffP % 1024 == 0, "swizzled tiles need 1 KB alignment");
 constexpr uint32_t kKVTileBytes = kKeysR * 256;
+constexpr int kPartStride = 4 + kD;  // floats per row of a split's partial: m, l, count, pad, o[D]
 
 __device__ __forceinline__ uint32_t pack_half2_r(float x, float y) {
   __half2 h = __floats2half2_rn(x, y);
@@ -580,13 +587,20 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
   const uint32_t sbase = smem_u32(sm);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int half = tid >> 7, r = tid & (kRowsR - 1);
-  const int tile = gridDim.x - 1 - blockIdx.x, hr = blockIdx.y, b = blockIdx.z;  // longest rows first
+  // a row tile's keys may be split over attn_splits CTAs (key tiles [tb, tb + ntl) each), whose
+  // partial (m, l, o) the last to finish merges; row tiles run longest first
+  const int n_split = a.attn_splits;
+  const int split = (int)(blockIdx.x % n_split);
+  const int n_tiles_c = (int)(gridDim.x / n_split);
+  const int tile = n_tiles_c - 1 - (int)(blockIdx.x / n_split), hr = blockIdx.y, b = blockIdx.z;
   const int i0 = tile * kRowsR;
   const int nrows = min(kRowsR, a.C - i0);
   const bool live = r < nrows;
   const int64_t pos = live ? a.P0 + i0 + r : -1;
   const int64_t nkeys = a.P0 + i0 + nrows;
   const int64_t nt = (nkeys + kKeysR - 1) / kKeysR;
+  const int64_t tb = (int64_t)split * a.attn_split_tiles;
+  const int64_t ntl = max((int64_t)0, min(nt, tb + a.attn_split_tiles) - tb);
   const int h = a.ret_head[hr], g = h / a.group;
   const int64_t qs = (int64_t)a.Hq * kD;
   const int64_t idx_row0 = ((int64_t)b * a.Hr + hr) * a.max_seq;
@@ -698,31 +712,37 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
     return w[0];
   };
 
-  // ---- prologue: index key tiles 0..2 in flight, the scores of tile 0, its masks
-  if (tid == 0) {
-    for (int64_t i = 0; i < (int64_t)kIdxStages && i < nt; ++i)
-      tc_load_keys(ikt(i), &tm_idx, idx_row0, i, barI + 8u * (uint32_t)i);
-    okw = mbar_wait(barI, 0u);
-    if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(0), barIdone);
-  }
-  uint32_t mask_cur = read_mask(0);
-  tc_fence_before();
-  if (half == 1) xm[r] = mask_cur;
-  bool any_cur = __syncthreads_or(mask_cur != 0u) != 0;
-  ok = __syncthreads_and(okw ? 1 : 0) != 0;
-  if (ok && tid == 0) {
-    if (nt > 1) {
-      okw = mbar_wait(barI + 8u, 0u);
-      if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(1), barIdone);
+  // ---- prologue: index key tiles tb .. tb + 2 in flight, the scores of tile tb, its masks
+  // (ring stages and barrier phases count tiles from tb; coordinates are absolute)
+  uint32_t mask_cur = 0u;
+  bool any_cur = false;
+  if (ntl > 0) {
+    if (tid == 0) {
+      for (int64_t i = 0; i < (int64_t)kIdxStages && i < ntl; ++i)
+        tc_load_keys(ikt(i), &tm_idx, idx_row0, tb + i, barI + 8u * (uint32_t)i);
+      okw = mbar_wait(barI, 0u);
+      if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(0), barIdone);
     }
-    if (nt > 3) tc_load_keys(ikt(3), &tm_idx, idx_row0, 3, barI);  // stage 0: tile 0 is scored
-    if (any_cur) load_kv(barK, sbase + kAOffK, &tm_k, 0);
+    mask_cur = read_mask(tb);
+    tc_fence_before();
+    if (half == 1) xm[(tb & 1) * kRowsR + r] = mask_cur;
+    any_cur = __syncthreads_or(mask_cur != 0u) != 0;
+    ok = __syncthreads_and(okw ? 1 : 0) != 0;
+    if (ok && tid == 0) {
+      if (ntl > 1) {
+        okw = mbar_wait(barI + 8u, 0u);
+        if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(1), barIdone);
+      }
+      if (ntl > 3) tc_load_keys(ikt(3), &tm_idx, idx_row0, tb + 3, barI);  // stage 0: tile tb is scored
+      if (any_cur) load_kv(barK, sbase + kAOffK, &tm_k, tb);
+    }
   }
 
   float m_ref = -INFINITY, l = 0.f;  // reference max of row r; this half's share of the sum
   int nsel = 0;
   int64_t lbase = 0;  // listed positions written so far (half 0 of a listed row)
-  for (int64_t t = 0; ok && t < nt; ++t) {
+  for (int64_t u = 0; ok && u < ntl; ++u) {
+    const int64_t t = tb + u;  // the absolute key tile
     // ---- statistics of tile t: count, bitmap words, listed positions
     nsel += __popc(mask_cur);
     if (brow) {
@@ -746,16 +766,16 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
     // ---- (a) the masks of tile t + 1 (scored one tile ahead); the scores of tile t + 2
     uint32_t mask_next = 0u;
     bool any_next = false;
-    if (t + 1 < nt) {
+    if (u + 1 < ntl) {
       mask_next = read_mask(t + 1);
       tc_fence_before();
       if (half == 1) xm[((t + 1) & 1) * kRowsR + r] = mask_next;
       any_next = __syncthreads_or(mask_next != 0u) != 0;
-      if (tid == 0 && t + 2 < nt && okw) {
-        okw = mbar_wait(barI + 8u * (uint32_t)((t + 2) % kIdxStages), (uint32_t)(((t + 2) / kIdxStages) & 1));
-        if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(t + 2), barIdone);
-        if (t + 4 < nt)  // the stage of tile t + 1 is free: its scores are done
-          tc_load_keys(ikt(t + 4), &tm_idx, idx_row0, t + 4, barI + 8u * (uint32_t)((t + 4) % kIdxStages));
+      if (tid == 0 && u + 2 < ntl && okw) {
+        okw = mbar_wait(barI + 8u * (uint32_t)((u + 2) % kIdxStages), (uint32_t)(((u + 2) / kIdxStages) & 1));
+        if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(u + 2), barIdone);
+        if (u + 4 < ntl)  // the stage of tile t + 1 is free: its scores are done
+          tc_load_keys(ikt(u + 4), &tm_idx, idx_row0, t + 4, barI + 8u * (uint32_t)((u + 4) % kIdxStages));
       }
     }
     // ---- (b) attention over tile t
@@ -867,27 +887,70 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
   if (ok) {
     tc_fence_after();
     const float lt = l + swap_half(l);
-    const float inv = lt > 0.f ? 1.f / lt : 0.f;
-    float* orow = a.out + ((int64_t)b * a.C + i0 + (live ? r : 0)) * qs + (int64_t)h * kD + 64 * half;
+    if (half == 1) xcnt[r] = nsel;  // selected counts: half 1 hands its count to half 0
+    __syncthreads();
+    const int cnt_row = nsel + xcnt[r];  // (half 0)
+    float ov[64];
     const uint32_t oAddr = lane_addr + kColO + 64u * half;
+    tmem_ld32(oAddr, ov);
+    tmem_ld32(oAddr + 32u, ov + 32);
+    tmem_ld_wait();
+    if (!any_pv) {
 #pragma unroll
-    for (int c0 = 0; c0 < 64; c0 += 32) {
-      float ov[32];
-      tmem_ld32(oAddr + c0, ov);
-      tmem_ld_wait();
+      for (int i = 0; i < 64; ++i) ov[i] = 0.f;
+    }
+    float* orow = a.out + ((int64_t)b * a.C + i0 + (live ? r : 0)) * qs + (int64_t)h * kD + 64 * half;
+    int32_t* crow = (a.sel_count && live && half == 0) ? a.sel_count + ((int64_t)b * a.C + i0 + r) * a.Hr + hr : nullptr;
+    if (n_split == 1) {
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
       if (live) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (any_pv) o4 = make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
-          *reinterpret_cast<float4*>(orow + c0 + i) = o4;
+        for (int i = 0; i < 64; i += 4)
+          *reinterpret_cast<float4*>(orow + i) = make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+      }
+      if (crow) *crow = cnt_row;
+    } else {
+      // this split's partial, then the last split of the row tile merges them all (log-sum-exp
+      // in base 2: the o and l of each split are relative to its reference max m)
+      const int64_t tix = ((int64_t)b * a.Hr + hr) * n_tiles_c + tile;
+      float* pt = a.attn_part + tix * n_split * (int64_t)kRowsR * kPartStride;
+      float* mine = pt + ((int64_t)split * kRowsR + r) * kPartStride;
+#pragma unroll
+      for (int i = 0; i < 64; i += 4)
+        *reinterpret_cast<float4*>(mine + 4 + 64 * half + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+      if (half == 0) *reinterpret_cast<float4*>(mine) = make_float4(m_ref, lt, __int_as_float(cnt_row), 0.f);
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) xcnt[0] = atomicAdd(a.attn_ticket + tix, 1u) == (uint32_t)(n_split - 1) ? 1 : 0;
+      __syncthreads();
+      if (xcnt[0]) {
+        __threadfence();
+        float M = -INFINITY;
+        for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, __ldcg(pt + ((int64_t)sp * kRowsR + r) * kPartStride));
+        float Ls = 0.f, o[64];
+        int cnt = 0;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) o[i] = 0.f;
+        for (int sp = 0; sp < n_split; ++sp) {
+          const float* q = pt + ((int64_t)sp * kRowsR + r) * kPartStride;
+          const float ms = __ldcg(q);
+          cnt += __float_as_int(__ldcg(q + 2));
+          if (ms == -INFINITY) continue;  // no selected key of this row in that split
+          const float f = fast_exp2(ms - M);
+          Ls += __ldcg(q + 1) * f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) o[i] += __ldcg(q + 4 + 64 * half + i) * f;
         }
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < 64; i += 4)
+            *reinterpret_cast<float4*>(orow + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        }
+        if (crow) *crow = cnt;
+        if (tid == 0) a.attn_ticket[tix] = 0u;
       }
     }
-    // selected counts: half 1 hands its count to half 0
-    if (half == 1) xcnt[r] = nsel;
-    __syncthreads();
-    if (half == 0 && live && a.sel_count) a.sel_count[((int64_t)b * a.C + i0 + r) * a.Hr + hr] = nsel + xcnt[r];
   } else if (tid == 0) {
     atomicOr(a.err, kErrTimeout);
     // wait (bounded) for the copies and MMAs this CTA may still have in flight: the next
@@ -927,6 +990,18 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
   a.q_idx = L->q_idx;
   a.cut = L->pf_cut;
   a.capture = L->pf_capture;
+  // long rows split their keys over several attention CTAs (one wave holds 2 per SM), unless a
+  // row's positions are to be listed in order
+  {
+    const int64_t nt_max = (L->len + kKeysR - 1) / kKeysR;
+    int64_t n_split = (nt_max + kAttSplitTiles - 1) / kAttSplitTiles;
+    if (n_split < 1 || (stats && stats->rows)) n_split = 1;
+    if (n_split > L->attn_split_max) n_split = L->attn_split_max;
+    a.attn_splits = (int)n_split;
+    a.attn_split_tiles = (nt_max + n_split - 1) / n_split;  // every key tile in some split
+  }
+  a.attn_part = L->attn_part;
+  a.attn_ticket = L->attn_ticket;
   a.scale_log2 = L->sm_scale * 1.4426950408889634f;
   a.out = out;
   a.sel_count = stats ? stats->sel_count : nullptr;
@@ -938,7 +1013,8 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
   a.row_sel = (stats && stats->rows) ? stats->row_sel : nullptr;
   a.row_sel_cap = (stats && stats->rows) ? stats->row_sel_cap : 0;
   a.err = L->err;
-  dim3 grid((C + kRowsR - 1) / kRowsR, L->Hr, L->B);
+  const dim3 grid((C + kRowsR - 1) / kRowsR, L->Hr, L->B);
+  const dim3 agrid(grid.x * a.attn_splits, L->Hr, L->B);
   cudaError_t e;
   {
     ProfScope ps(L, "prefill_select", st);
@@ -952,7 +1028,7 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
     ProfScope ps(L, "prefill_attn", st);
     e = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttSmem);
     if (e != cudaSuccess) return e;
-    prefill_attn_kernel<<<grid, kAttThreads, kAttSmem, st>>>(a, L->tm_idx, L->tm_k, L->tm_v);
+    prefill_attn_kernel<<<agrid, kAttThreads, kAttSmem, st>>>(a, L->tm_idx, L->tm_k, L->tm_v);
     e = cudaGetLastError();
   }
   return e;

@@ -29,6 +29,8 @@ constexpr int kGatherThreads = 256;
 
 // Prefill selection: keys of a row's crossing range captured per refinement walk.
 constexpr int kPfCapture = 2048;
+// Prefill attention: key tiles (64 keys) per CTA when long rows split their keys (256K keys).
+constexpr int kAttSplitTiles = 4096;
 
 // Fixed top-k decode selection (ablation mode): keys per chunk of its radix-select kernels.
 constexpr int kTopkChunk = 4096;
@@ -79,6 +81,9 @@ struct rtp_layer {
   bool tm_ready = false;
   uint2* pf_cut = nullptr;
   unsigned long long* pf_capture = nullptr;  // [B][Hr][max_chunk / 128][kPfCapture][128] selection lists
+  int attn_split_max = 1;          // key splits of a prefill attention row tile (max_seq / 256K)
+  float* attn_part = nullptr;      // [B][Hr][max_chunk / 128][attn_split_max][128][4 + D] partials
+  uint32_t* attn_ticket = nullptr; // [B][Hr][max_chunk / 128]
   // decode: the local heads' window attention runs on a second stream, forked after the
   // selection and joined back, so it overlaps the retrieval heads' gather attention
   cudaStream_t side = nullptr;

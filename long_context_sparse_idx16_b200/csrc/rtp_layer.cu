@@ -100,7 +100,8 @@ static void free_all(rtp_layer* L) {
                   L->d_loc_head, L->d_loc_cnt, L->d_local_list, L->pf_cut, L->idx_hl, L->q_rot, L->q_idx, L->sel_idx, L->sel_cnt,
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
-                  L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt, L->pf_capture};
+                  L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt, L->pf_capture, L->attn_part,
+                  L->attn_ticket};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -240,8 +241,17 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   RTP_ALLOC(L->d_local_list, L->n_local);
   RTP_ALLOC(L->idx_hl, (int64_t)B * Hr * L->max_seq * 2 * kR);
   RTP_ALLOC(L->pf_cut, (int64_t)B * (Hr > 0 ? Hr : 1) * L->max_chunk);
-  if (Hr > 0 && !L->prefill_dense)
-    RTP_ALLOC(L->pf_capture, (int64_t)B * Hr * ((L->max_chunk + 127) / 128) * kPfCapture * 128);
+  if (Hr > 0 && !L->prefill_dense) {
+    const int64_t row_tiles = (L->max_chunk + 127) / 128;
+    RTP_ALLOC(L->pf_capture, (int64_t)B * Hr * row_tiles * kPfCapture * 128);
+    const int64_t key_tiles = (L->max_seq + 63) / 64;
+    L->attn_split_max = (int)((key_tiles + kAttSplitTiles - 1) / kAttSplitTiles);
+    if (L->attn_split_max > 1) {
+      RTP_ALLOC(L->attn_part, (int64_t)B * Hr * row_tiles * L->attn_split_max * 128 * (4 + kD));
+      RTP_ALLOC(L->attn_ticket, (int64_t)B * Hr * row_tiles);
+      if (e == cudaSuccess) e = cudaMemset(L->attn_ticket, 0, sizeof(uint32_t) * (size_t)(B * Hr * row_tiles));
+    }
+  }
   RTP_ALLOC(L->q_rot, rows * Hq * kD);
   RTP_ALLOC(L->q_idx, rows * Hr * kR);
   RTP_ALLOC(L->sel_idx, P * L->max_select);
@@ -558,6 +568,8 @@ rtp_status rtp_check(rtp_layer* L, cudaStream_t stream) {
     // a barrier gave up: its counters are inconsistent; start the next launch from zero
     reset_select_scratch(L);
     cudaMemset(L->gticket, 0, sizeof(uint32_t) * (size_t)(L->B * L->Hr > 0 ? L->B * L->Hr : 1));
+    if (L->attn_ticket)
+      cudaMemset(L->attn_ticket, 0, sizeof(uint32_t) * (size_t)L->B * L->Hr * ((L->max_chunk + 127) / 128));
     return fail(L, RTP_ETIMEOUT, "a bounded in-kernel wait gave up");
   }
   if (w & kErrInternal) return fail(L, RTP_EINTERNAL, "an internal consistency check failed");

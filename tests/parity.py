@@ -116,7 +116,7 @@ def run_decode(x, *, top_p=None, heads=None, batches=None, max_select=0, sel_cap
     idx = st[3].cpu().numpy() if st else None
     heads = range(s.n_q_heads) if heads is None else heads
     batches = range(s.batch) if batches is None else batches
-    refs, gpus = [], []
+    refs, gpus, gpus2 = [], [], []
     summary = {}
     for b in batches:
         for h in heads:
@@ -181,18 +181,23 @@ def run_prefill(x, *, top_p=None, rows=None, heads=None, batches=None, sets="bit
         cap = int(st[0][:, torch.as_tensor(rows, device=out.device)].max()) + 1
         out2, st2 = layer.prefill_chunk(q, stats=True, rows=rows.tolist(), row_sel_cap=cap)
         assert layer.check() == 0, "kernel error word set"
-        assert torch.equal(out, out2) and torch.equal(st[0], st2[0]), "a repeated prefill call differs"
+        # the same selection; a chunk whose long rows split their keys over several attention
+        # CTAs (not done when rows are listed) differs from the listed call only in rounding, so
+        # both calls' outputs are compared with the oracle below
+        assert torch.equal(st[0], st2[0]), "a repeated prefill call selects differently"
         row_lists = st2[3].cpu().numpy()  # [B][len(rows)][Hr][cap]
     heads = range(s.n_q_heads) if heads is None else heads
     batches = range(s.batch) if batches is None else batches
     summary = {}
-    refs, gpus = [], []
+    refs, gpus, gpus2 = [], [], []
     for b in batches:
         for h in heads:
             ret = h in s.retrieval_heads
             hrows = rows if ret else local_rows
             rows_t = torch.as_tensor(hrows, device=out.device)
             out_h = out[b, rows_t, h].cpu().numpy()
+            if row_lists is not None:
+                gpus2.append(out2[b, rows_t, h].cpu().numpy())
             if not ret:
                 for b0 in range(0, len(hrows), row_block):
                     r = oracle.layer_rows(x, b, h, hrows[b0:b0 + row_block])
@@ -241,6 +246,8 @@ def run_prefill(x, *, top_p=None, rows=None, heads=None, batches=None, sets="bit
             gpus.append(out_h)
             summary[(b, h)] = (cnt.copy(), np.concatenate(counts_ref), ndiff)
     err = check_outputs(np.concatenate(gpus), np.concatenate(refs), f"{s.name} prefill p={p}")
+    if gpus2:
+        check_outputs(np.concatenate(gpus2), np.concatenate(refs), f"{s.name} prefill p={p}, listed rows")
     if own:
         layer.close()
     return {"out": out[:, torch.as_tensor(rows, device=out.device)].cpu().numpy(), "summary": summary, "err": err}

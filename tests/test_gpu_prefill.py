@@ -188,3 +188,10 @@ def test_prefill_dense_retrieval_heads():
     run_prefill(x, sets=None)
     xd = synth.generate(synth.spec("toy_decode_4k", prefill_dense=True))
     run_decode(xd)
+
+
+def test_prefill_long_rows_split_over_attention_ctas():
+    # 300K cached keys: each row tile's keys are split over two attention CTAs whose partial
+    # softmax states the last one merges; sets through the bitmap, outputs against the oracle
+    x = synth.generate(synth.spec("prefill_1m", prefix=300000, chunk=200))
+    run_prefill(x, rows=np.arange(0, 200, 3), local_rows=np.arange(0, 200, 25), heads=[0, 1, 13, 26], sets="bitmap")
