@@ -30,17 +30,27 @@
 //     quantised mass is 0 whenever N > 2^16, and for smaller N their total stays below
 //     (1 - p) * Z for every fp32 p < 1 (1 - p >= 2^-24), so they can never be needed to reach
 //     p and the cut never falls among them.
-//   * The keys of the crossing bin (usually a handful, at most 1024 on the fast path) are
-//     gathered into a list that every CTA of the problem sorts in shared memory (bitonic, warp
-//     shuffles below distance 32) to locate the exact cut key t and how many keys tied at t
-//     are taken (lowest positions first).  Larger crossing bins (massive exact ties) fall back
-//     to three radix levels over the key bits, 11/11/10 bits.
+//   * Each (problem, CTA) segment publishes its cumulative fine-bin key counts.  One CTA per
+//     problem (the one holding the middle of its keys) waits for all of them (an arrival count)
+//     and finds Z, the target and the crossing bin.  After the second barrier every CTA adds its
+//     crossing-bin keys (usually a handful, at most 1024 on the fast path) to the problem's
+//     candidate list, and the same CTA sorts the list in shared memory (bitonic, warp shuffles
+//     below distance 32) to locate the exact cut key t and how many keys tied at t are taken
+//     (lowest positions first), and from the cumulative counts and the sorted list the number of
+//     keys each CTA's predecessors select.  After the third barrier each CTA writes its own
+//     positions.
 //   * After the cut the selection is a key comparison: key > t, or key == t among the first
 //     n_need tied positions.  Ordered compaction is two ballot passes per warp.
-//   * Four grid barriers on the fast path (max, histogram, candidates, counts), three more on
-//     the fallback.  Every barrier wait is bounded (about 1 s); on timeout the error word records
-//     RTP_ETIMEOUT and the kernel returns.  Scratch histograms are zeroed by the launch that
-//     last read them, so a launch starts on clean scratch without a memset.
+//   * The ranges of the flat (problem, key) space follow the SM number when every SM holds one
+//     CTA: the even SM of each TPC takes a larger share (measured: it streams faster while both
+//     stream).
+//   * Three grid barriers on the fast path (max, histogram, cut).  A crossing in the coarse bin
+//     or one holding more keys than the sort takes (massive exact ties) sets the launch's
+//     fallback flag: then every CTA sorts the candidates of the problems that fit, and the
+//     others refine by three radix levels over the key bits (11/11/10), with five barriers
+//     after the second.  Every barrier wait is bounded (about 1 s); on timeout the error word
+//     records RTP_ETIMEOUT and the kernel returns.  Scratch histograms and lists are reset by
+//     the launch that last read them, so a launch starts on clean scratch without a memset.
 #include <type_traits>
 
 #include "rtp_device.cuh"
@@ -55,8 +65,11 @@ constexpr int kThreads = kSelThreads;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCand = kSelCand;  // crossing-bin keys resolved by sorting
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPsum = 8;     // words of a problem's summary
 constexpr int kUnroll = 8;  // 16-byte loads in flight per thread in the index stream
-constexpr int kFine = 1024;  // level-1 bins of width 1/64 covering (m - s) in [0, 16); bin kFine: [16, 32)
+constexpr int kFine = kSelFine;  // level-1 bins of width 1/64 covering (m - s) in [0, 16); bin kFine: [16, 32)
+static_assert(kFine == kThreads, "one fine bin per thread in the count scans");
+static_assert(kWarps == 32, "one lane per warp in the warp-base scans");
 
 // radix fallback inside the crossing bin: key bits [31:21], [20:10], [9:0]
 __device__ __forceinline__ int level_shift(int l) { return l == 0 ? 21 : (l == 1 ? 10 : 0); }
@@ -75,7 +88,10 @@ struct SelectArgs {
   const float* q_idx;   // [P][r]
   int P;
   int64_t N;
-  int64_t L;  // keys per CTA
+  int64_t L;   // keys of the longest CTA range (sizes the shared-memory score array)
+  int64_t Lp;  // keys per CTA pair (virtual indices 2k, 2k + 1) ...
+  int64_t Le;  // ... of which the even member takes the first Le
+  int use_smid;  // 1: the virtual index of a CTA is its SM (one CTA on every SM)
   int sc_bits;
   float top_p;
   int32_t* sel_idx;
@@ -84,14 +100,19 @@ struct SelectArgs {
   float* sel_mass;
   float* sel_thr;
   float* seg_max;     // [P + G]
-  Hist3 h1;           // [P][bins]
+  unsigned long long* h1;  // [P][bins]: level-1 masses (64-bit words)
   Hist3 hr;           // [3][P][bins] radix fallback levels
   uint32_t* cand_cnt;         // [P]
   unsigned long long* cand;   // [P][kCand] packed (key << 32) | ~j
   uint32_t* slot_cnt;         // [P + G][2]: (gt, eq) per (problem, CTA)
   unsigned long long* bar;    // [2]: grid barrier arrival counter (monotonic), exit counter
   uint32_t* keep;             // global keep lists when the scores live in global memory
-  uint32_t* flags;            // [1]: some problem needs the radix fallback
+  uint32_t* flags;            // [1]: == epoch when some problem of this launch needs the fallback
+  uint32_t epoch;             // this launch's number (never 0)
+  uint32_t* cum;              // [P + G][kFine]: cumulative fine-bin key counts per (problem, CTA)
+  unsigned long long* psum;   // [P][kPsum]: Z, T, rem, (crossing-bin keys << 32) | crossing bin, cut key
+  long long* cres;            // [P + G][2]: keys the CTAs before select, tied keys this CTA takes
+  uint32_t* pticket;          // [P]: CTAs of the problem done with phase B (the last resets it)
   uint32_t* err;
   float* gscores;
   long long wait_limit;       // clock cycles a grid-barrier wait may take before it gives up
@@ -100,7 +121,6 @@ struct SelectArgs {
 struct Seg {
   int p;
   int radix;     // 1: crossing bin too large for the candidate list (fallback path)
-  int full;      // 1: a warp's keep list overflowed; later passes scan the whole chunk
   int kbase;     // this segment's keep lists start at keep[kbase]; warp w at + w * kcap
   int kcap;      // keep-list capacity per warp
   int bstar;
@@ -127,6 +147,7 @@ struct Smem {
   float redf[kWarps];
   uint32_t wcnt[kSelMaxSeg][kWarps][2];  // (gt, eq) per warp chunk, then exclusive bases
   uint32_t lcnt[kSelMaxSeg][kWarps];     // keep-list length per warp chunk
+  uint32_t lres[kSelMaxSeg][kWarps];     // first key of the warp chunk its full keep list missed
   uint32_t slot[2 * kSelMaxGrid];
   int cross, cut_idx;
   unsigned long long cross_above, cut_cum;
@@ -134,6 +155,18 @@ struct Smem {
 };
 
 // ---------------------------------------------------------------- small helpers
+
+// The keys a pass over a warp chunk's fine keys visits: its keep list, then, when the list
+// filled up, every key from the first one it missed to the end of the chunk (keys that are not
+// fine fail every test those passes make).  `whole`: every key of the chunk (a cut in the coarse
+// bin, whose keys are not listed).
+__device__ __forceinline__ int visit_count(bool whole, int w_lo, int w_hi, int n_list, int res) {
+  return whole ? (w_hi - w_lo) : n_list + (w_hi - res);
+}
+template <typename KeepT>
+__device__ __forceinline__ int visit_key(int i, bool whole, int w_lo, const KeepT* kl, int n_list, int res) {
+  return whole ? w_lo + i : (i < n_list ? (int)kl[i] : res + (i - n_list));
+}
 
 // Fixed-point mass of a score: round(2^sc * exp(s - m)), as (hi, lo) 32-bit words.
 __device__ __forceinline__ void mass_words(float s, float m, float scale, uint32_t* hi, uint32_t* lo) {
@@ -190,6 +223,22 @@ __device__ __forceinline__ bool grid_sync(unsigned long long* bar, uint32_t nblo
   }
   __syncthreads();
   return s_ok != 0;
+}
+
+// Wait (bounded by `limit` clock cycles) until the counter reaches target; false, with
+// RTP_ETIMEOUT recorded, if it does not.  Only counters that co-resident CTAs of this
+// cooperative grid advance are waited on.
+__device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t target, uint32_t* err, long long limit) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (clock64() - t0 > limit) {
+      atomicOr(err, kErrTimeout);
+      return false;
+    }
+  }
 }
 
 __device__ float block_max(float v, Smem& S) {
@@ -327,8 +376,160 @@ __device__ unsigned long long bitonic_desc(Smem& S, int n, unsigned long long v)
   return v;
 }
 
-// first CTA that holds keys of problem p
-__device__ __forceinline__ int cf_of(int p, const SelectArgs& a) { return (int)(((int64_t)p * a.N) / a.L); }
+// CTA ranges of the flat (problem, key) index space: virtual CTA v starts at r_start(v); the
+// two members of a pair split Lp keys as Le + (Lp - Le).
+__device__ __forceinline__ int64_t r_start(int v, const SelectArgs& a) {
+  return (int64_t)(v >> 1) * a.Lp + ((v & 1) ? a.Le : 0);
+}
+// the CTA whose range holds flat index x
+__device__ __forceinline__ int cta_of(int64_t x, const SelectArgs& a) {
+  const int64_t k = x / a.Lp;
+  return (int)(2 * k + (x - k * a.Lp >= a.Le ? 1 : 0));
+}
+// first and last CTA that hold keys of problem p
+__device__ __forceinline__ int cf_of(int p, const SelectArgs& a) { return cta_of((int64_t)p * a.N, a); }
+__device__ __forceinline__ int cl_of(int p, const SelectArgs& a) { return cta_of((int64_t)p * a.N + a.N - 1, a); }
+
+// The virtual index of this CTA.  Of the two SMs of a TPC, the odd-numbered one streams about
+// 15% slower while both stream (measured), so with one CTA on every SM the ranges follow the SM
+// number: even SMs take the larger share of a pair.  Otherwise the block index.
+__device__ __forceinline__ int virtual_cta(const SelectArgs& a) {
+  if (a.use_smid) {
+    uint32_t smid, nsmid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    asm volatile("mov.u32 %0, %%nsmid;" : "=r"(nsmid));
+    if (nsmid == gridDim.x) return (int)smid;  // then the SM numbers are exactly 0 .. G-1
+  }
+  return (int)blockIdx.x;
+}
+
+// Z, the target T and the crossing bin of problem p, found once by its designated CTA after
+// every CTA of the problem has finished phase B (S.h.m holds the problem's level-1 masses, every CTA of the problem has
+// published its cumulative fine-bin counts).  A crossing in the coarse bin, or one holding more
+// than kCand keys, is left to the fallback path (the launch's flag).
+__device__ void select_summary(const SelectArgs& a, Smem& S, int p, int cf, int cl) {
+  const int tid = threadIdx.x;
+  // one scan gives Z (the total), then T, then the crossing bin
+  const unsigned long long m0 = S.h.m[2 * tid], m1 = S.h.m[2 * tid + 1];
+  if (tid == 0) S.cross = -1;
+  const unsigned long long incl = block_incl_scan_u64(m0 + m1, S);
+  const unsigned long long Z = S.red64[kWarps - 1];
+  unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
+  if (T < 1ull) T = 1ull;
+  if (T > Z) T = Z;
+  const unsigned long long base = incl - (m0 + m1);
+  if (base < T && base + m0 >= T) {
+    S.cross = 2 * tid;
+    S.cross_above = base;
+  } else if (base + m0 < T && base + m0 + m1 >= T) {
+    S.cross = 2 * tid + 1;
+    S.cross_above = base + m0;
+  }
+  __syncthreads();
+  if (tid == 0 && S.cross < 0) {
+    atomicOr(a.err, kErrInternal);
+    S.cross = 0;
+    S.cross_above = 0;
+  }
+  __syncthreads();
+  const int cross = S.cross;
+  // keys in the crossing bin, over the problem's CTAs
+  unsigned long long nk = 0;
+  if (cross < kFine) {
+    for (int cc = cf + tid; cc <= cl; cc += kThreads) {
+      const uint32_t* cu = a.cum + (int64_t)(p + cc) * kFine;
+      nk += __ldcg(cu + cross) - (cross > 0 ? __ldcg(cu + cross - 1) : 0u);
+    }
+  }
+  nk = block_sum_u64(nk, S);
+  if (tid == 0) {
+    unsigned long long* ps = a.psum + kPsum * (int64_t)p;
+    ps[0] = Z;
+    ps[1] = T;
+    ps[2] = T - S.cross_above;
+    ps[3] = (nk << 32) | (uint32_t)cross;
+    if (cross >= kFine || nk > (unsigned long long)kCand) atomicExch(a.flags, a.epoch);
+    a.pticket[p] = 0u;
+  }
+}
+
+// The exact cut of problem p, found once by its designated CTA after every CTA of the problem
+// has added its crossing-bin keys to the problem's candidate list: the candidates sorted (key desc, then position asc), the
+// cut key t and the number of tied keys taken; then, per CTA of the problem, the count of keys
+// its predecessors select (their keys above the crossing bin, from the cumulative counts, plus
+// their candidates above the cut and the ties taken) and how many of its own tied keys it
+// takes.  Also the problem's outputs (count, mass, threshold); the list is reset for the next
+// launch.
+__device__ void select_cut(const SelectArgs& a, Smem& S, int p, int cf, int cl, float m, float scale) {
+  const int tid = threadIdx.x;
+  unsigned long long* ps = a.psum + kPsum * (int64_t)p;
+  const unsigned long long Z = __ldcg(ps), T = __ldcg(ps + 1), rem = __ldcg(ps + 2);
+  const int cross = (int)(uint32_t)__ldcg(ps + 3);
+  const int nct = cl - cf + 1;
+  const unsigned long long vraw = tid < kCand ? __ldcg(a.cand + (int64_t)p * kCand + tid) : 0ull;
+  const int nc = min((int)__ldcg(a.cand_cnt + p), kCand);
+  // per CTA of the problem: keys above the crossing bin
+  for (int t = tid; t < nct; t += kThreads) {
+    const uint32_t* cu = a.cum + (int64_t)(p + cf + t) * kFine;
+    S.slot[t] = cross > 0 ? __ldcg(cu + cross - 1) : 0u;
+  }
+  int n = 32;
+  while (n < nc) n <<= 1;
+  const unsigned long long v = bitonic_desc(S, n, tid < nc ? vraw : 0ull);  // key desc, then position asc
+  // masses in sorted order; the cut is the first key whose running mass reaches rem
+  const uint32_t key = (uint32_t)(v >> 32);
+  unsigned long long mq = 0ull;
+  if (tid < nc) mq = mass64(key_to_float(key), m, scale);
+  const unsigned long long cum = block_incl_scan_u64(mq, S);
+  if (tid == 0) S.cut_idx = -1;
+  __syncthreads();
+  if (tid < nc && cum >= rem && cum - mq < rem) {
+    S.cut_idx = tid;
+    S.cut_cum = cum;
+  }
+  if (tid < nc) S.sk[tid] = v;
+  __syncthreads();
+  int ci = S.cut_idx;
+  if (ci < 0) {  // unreachable with exact sums; keep every candidate
+    if (tid == 0) atomicOr(a.err, kErrInternal);
+    ci = nc - 1;
+  }
+  // the cut key (an empty list, also unreachable, selects nothing from the crossing bin)
+  const uint32_t tk = ci >= 0 ? (uint32_t)(S.sk[ci] >> 32) : 0xFFFFFFFFu;
+  // the start of the tie run at the cut (sorted: equal keys are adjacent)
+  if (tid == 0) S.cross = ci + 1;
+  for (int t = tid; t < 2 * nct; t += kThreads) S.hc[t] = 0u;
+  __syncthreads();
+  if (tid < nc && key == tk && (tid == 0 || (uint32_t)(S.sk[tid - 1] >> 32) != tk)) S.cross = tid;
+  // per CTA: crossing-bin keys above the cut, and at it
+  if (tid < nc && key >= tk) {
+    const uint32_t j = 0xFFFFFFFFu - (uint32_t)v;
+    const int t = cta_of((int64_t)p * a.N + j, a) - cf;
+    atomicAdd(&S.hc[2 * t + (key == tk ? 1 : 0)], 1u);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const long long n_need = (long long)(ci - S.cross + 1);
+    long long before = 0, eq_seen = 0;
+    for (int t = 0; t < nct; ++t) {
+      const long long eq = S.hc[2 * t + 1];
+      long long take = n_need - eq_seen;
+      take = take < 0 ? 0 : (take > eq ? eq : take);
+      a.cres[2 * (int64_t)(p + cf + t)] = before;
+      a.cres[2 * (int64_t)(p + cf + t) + 1] = take;
+      before += (long long)S.slot[t] + (long long)S.hc[2 * t] + take;
+      eq_seen += eq;
+    }
+    const unsigned long long e_t = mass64(key_to_float(tk), m, scale);
+    const unsigned long long cut_cum = S.cut_idx >= 0 ? S.cut_cum : rem;
+    a.sel_cnt[p] = (int32_t)(before < a.max_select ? before : a.max_select);
+    a.sel_mass[p] = (float)((double)((T - rem) + cut_cum) / (double)Z);
+    a.sel_thr[p] = (float)((double)e_t / (double)Z);
+    ps[4] = tk;
+    a.cand_cnt[p] = 0u;
+    a.pticket[p] = 0u;
+  }
+}
 
 // ---------------------------------------------------------------- the kernel
 
@@ -336,12 +537,12 @@ template <bool kSmemScores, bool kBf16>
 __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
-  const int c = blockIdx.x;
+  const int c = virtual_cta(a);
   const uint32_t G = gridDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t total = (int64_t)a.P * a.N;
-  const int64_t r0 = (int64_t)c * a.L;
-  const int64_t r1 = min(total, r0 + a.L);
+  const int64_t r0 = min(total, r_start(c, a));
+  const int64_t r1 = min(total, r_start(c + 1, a));
   float* sc = kSmemScores ? reinterpret_cast<float*>(smem_raw + sizeof(Smem)) : a.gscores + r0;
   // Keep lists: 16-bit in shared memory after the scores, 32-bit in global memory otherwise.
   using KeepT = typename std::conditional<kSmemScores, uint16_t, uint32_t>::type;
@@ -362,17 +563,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
       s.jhi = min(a.N, r1 - (int64_t)s.p * a.N);
       s.off = (int64_t)s.p * a.N + s.jlo - r0;
       s.radix = 0;
-      s.full = 0;
       s.prefix = 0;
     }
   }
   __syncthreads();
-  if (tid == 0) {  // per-warp keep capacity: a quarter of the warp chunk, rounded up
+  if (tid == 0) {  // per-warp keep capacity: 3/8 of the warp chunk, rounded up
     int acc = 0;
     for (int si = 0; si < nseg; ++si) {
       const int rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
       const int wlen = (rows + kWarps - 1) / kWarps;
-      S.seg[si].kcap = (wlen + 3) / 4;
+      S.seg[si].kcap = (3 * wlen + 7) / 8;
       S.seg[si].kbase = acc;
       acc += kWarps * S.seg[si].kcap;
     }
@@ -448,14 +648,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   }
   if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
 
-  // ---- phase B: row maxima; level-1 mass histogram; keep lists.  Warp w walks a contiguous
-  // chunk of the segment.  Keys within 16 of the max join the warp's ordered keep list (their
-  // fine-bin masses are added afterwards from the list, every lane busy); keys 16..32 below the
-  // max add their exact mass to a per-thread register sum for the single coarse bin.
+  // ---- phase B: row maxima; level-1 mass histogram; keep lists; the fine keys by bin.  Warp w
+  // walks a contiguous chunk of the segment.  Keys within 16 of the max join the warp's ordered
+  // keep list (their fine-bin masses and counts are added afterwards from the list, every lane
+  // busy); keys 16..32 below the max add their exact mass to a per-thread register sum for the
+  // single coarse bin.  Each segment then publishes its cumulative fine-bin counts and its fine
+  // keys grouped by bin, so that after the next barrier any CTA can read the crossing bin's keys
+  // of every other CTA directly.  The last CTA of a problem to finish (a ticket) reads the
+  // problem's histogram and records Z, the target T, the crossing bin and its key count.
   const bool small_mass = a.sc_bits <= 54;  // then every coarse-bin mass fits 32 bits
   for (int si = 0; si < nseg; ++si) {
     const int p = S.seg[si].p;
-    const int cf = cf_of(p, a), cl = (int)(((int64_t)p * a.N + a.N - 1) / a.L);
+    const int cf = cf_of(p, a), cl = cl_of(p, a);
     float mv = -INFINITY;
     for (int cc = cf + tid; cc <= cl; cc += kThreads) mv = fmaxf(mv, __ldcg(a.seg_max + p + cc));
     const float m = block_max(mv, S);
@@ -463,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     if (tid == 0) S.seg[si].m = m;
     __syncthreads();
     const int off = (int)S.seg[si].off, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
+    const int jlo = (int)S.seg[si].jlo;
     const int wlen = (rows + kWarps - 1) / kWarps;
     const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
     const int kcap = S.seg[si].kcap;
@@ -470,6 +675,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     unsigned long long coarse = 0;
     int nkeep = 0;
     const uint32_t lt = (1u << lane) - 1u;
+    if (lane == 0) S.lres[si][warp] = (uint32_t)w_hi;
+    __syncwarp();
     for (int k0 = w_lo; k0 < w_hi; k0 += 32) {
       const int k = k0 + lane;
       const float v = k < w_hi ? sc[off + k] : -INFINITY;
@@ -487,18 +694,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
         const int pos = nkeep + __popc(bf & lt);
         if (pos < kcap) {
           kl[pos] = (KeepT)k;
-        } else {  // list full: count this key now
+        } else {  // list full: count this key now (later passes rescan from the first one)
+          if (pos == kcap) S.lres[si][warp] = (uint32_t)k;
           uint32_t hi, lo;
           mass_words(v, m, scale, &hi, &lo);
-          add_words(&S.h.w.lo[(int)(x * 64.f)], &S.h.w.hi[(int)(x * 64.f)], hi, lo);
+          const int bi = (int)(x * 64.f);
+          add_words(&S.h.w.lo[bi], &S.h.w.hi[bi], hi, lo);
+          atomicAdd(&S.hc[bi], 1u);
         }
       }
       nkeep += __popc(bf);
     }
-    if (lane == 0) {
-      S.lcnt[si][warp] = (uint32_t)min(nkeep, kcap);
-      if (nkeep > kcap) S.seg[si].full = 1;
-    }
+    if (lane == 0) S.lcnt[si][warp] = (uint32_t)min(nkeep, kcap);
     const int nl = min(nkeep, kcap);
     __syncwarp();  // list entries written by other lanes of this warp
     for (int i = lane; i < nl; i += 32) {
@@ -506,100 +713,212 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
       const float x = m - v;
       uint32_t hi, lo;
       mass_words(v, m, scale, &hi, &lo);
-      add_words(&S.h.w.lo[(int)(x * 64.f)], &S.h.w.hi[(int)(x * 64.f)], hi, lo);
+      const int bi = (int)(x * 64.f);
+      add_words(&S.h.w.lo[bi], &S.h.w.hi[bi], hi, lo);
+      atomicAdd(&S.hc[bi], 1u);
     }
     coarse = warp_sum(coarse);
     if (lane == 0 && coarse) add_words(&S.h.w.lo[kFine], &S.h.w.hi[kFine], (uint32_t)(coarse >> 32), (uint32_t)coarse);
     __syncthreads();
     for (int i = tid; i <= kFine; i += kThreads) {
       const uint32_t lo = S.h.w.lo[i], hi = S.h.w.hi[i];
-      if (lo | hi) add_words(a.h1.lo + (int64_t)p * kBins + i, a.h1.hi + (int64_t)p * kBins + i, hi, lo);
+      if (lo | hi) atomicAdd(a.h1 + (int64_t)p * kBins + i, ((unsigned long long)hi << 32) | lo);
+    }
+    // cumulative fine-bin counts of this segment (one bin per thread), published
+    a.cum[(int64_t)(p + c) * kFine + tid] = (uint32_t)block_incl_scan_u64(S.hc[tid], S);
+    // the problem's arrival count: its designated CTA (the one holding the middle of its keys,
+    // which holds no other problem whenever the problem spans three CTAs or more) waits for all
+    // of them and summarises the histogram.  Waits only point to CTAs' contributions to the same
+    // or lower-numbered problems, which no wait precedes, so they cannot form a cycle.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      atomicAdd(a.pticket + p, 1u);
+      S.cut_idx = c == cta_of((int64_t)p * a.N + a.N / 2, a) &&
+                          wait_count(a.pticket + p, (uint32_t)(cl - cf + 1), a.err, a.wait_limit)
+                      ? 1
+                      : 0;
+    }
+    __syncthreads();
+    if (S.cut_idx) {
+      __threadfence();
+      for (int i = tid; i < kBins; i += kThreads) {
+        unsigned long long v = 0ull;
+        if (i <= kFine) {
+          v = __ldcg(a.h1 + (int64_t)p * kBins + i);
+          a.h1[(int64_t)p * kBins + i] = 0ull;  // clean for the next launch
+        }
+        S.h.m[i] = v;
+      }
+      __syncthreads();
+      select_summary(a, S, p, cf, cl);
     }
     __syncthreads();
   }
   if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
 
-  // ---- phase C: total mass, target, crossing bin; its keys become candidates.  A crossing in
-  // the coarse bin, or more than kCand keys in the crossing bin, takes the radix fallback.
-  for (int si = 0; si < nseg; ++si) {
-    const int p = S.seg[si].p;
-    for (int i = tid; i < kBins; i += kThreads) {
-      uint32_t lo = 0, hi = 0;
-      if (i <= kFine) {
-        lo = __ldcg(a.h1.lo + (int64_t)p * kBins + i);
-        hi = __ldcg(a.h1.hi + (int64_t)p * kBins + i);
-      }
-      S.h.m[i] = ((unsigned long long)hi << 32) | lo;
-    }
+  // Unless some problem needs the fallback (the launch's flag): each CTA adds its crossing-bin
+  // keys to the problem's candidate list; the last CTA of the problem to do so finds the cut
+  // for all of them; after the barrier every CTA writes its own positions.
+  if (tid == 0) S.cut_idx = __ldcg(a.flags) == a.epoch ? 1 : 0;
+  __syncthreads();
+  if (S.cut_idx == 0) {
     __syncthreads();
-    {  // one scan gives Z (the total), then T, then the crossing bin
-      const unsigned long long m0 = S.h.m[2 * tid], m1 = S.h.m[2 * tid + 1];
-      if (tid == 0) S.cross = -1;
-      const unsigned long long incl = block_incl_scan_u64(m0 + m1, S);
-      const unsigned long long Z = S.red64[kWarps - 1];
-      unsigned long long T = (unsigned long long)ceil((double)a.top_p * (double)Z);
-      if (T < 1ull) T = 1ull;
-      if (T > Z) T = Z;
-      const unsigned long long base = incl - (m0 + m1);
-      if (base < T && base + m0 >= T) {
-        S.cross = 2 * tid;
-        S.cross_above = base;
-      } else if (base + m0 < T && base + m0 + m1 >= T) {
-        S.cross = 2 * tid + 1;
-        S.cross_above = base + m0;
-      }
-      if (tid == 0) {
-        S.seg[si].Z = Z;
-        S.seg[si].T = T;
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      Seg& sg = S.seg[si];
-      if (S.cross < 0) {
-        atomicOr(a.err, kErrInternal);
-        S.cross = 0;
-        S.cross_above = 0;
-      }
-      sg.bstar = S.cross;
-      sg.rem = sg.T - S.cross_above;
-      // the coarse bin cannot be resolved from the keep lists: force the fallback
-      if (S.cross == kFine) {
-        atomicOr(a.flags, 1u);
-        if (c == cf_of(p, a)) atomicAdd(a.cand_cnt + p, (uint32_t)kCand + 1u);
-      }
-    }
-    __syncthreads();
-    const int bstar = S.seg[si].bstar;
-    if (bstar < kFine) {
+    for (int si = 0; si < nseg; ++si) {
+      const int p = S.seg[si].p;
+      const int cf = cf_of(p, a), cl = cl_of(p, a);
+      const int bstar = (int)(uint32_t)__ldcg(a.psum + kPsum * (int64_t)p + 3);
       const int off = (int)S.seg[si].off, jlo = (int)S.seg[si].jlo, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
       const float m = S.seg[si].m;
-      const bool full = S.seg[si].full;
       const int wlen = (rows + kWarps - 1) / kWarps;
       const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
       const KeepT* kl = keep + S.seg[si].kbase + warp * S.seg[si].kcap;
-      const int n_it = full ? (w_hi - w_lo) : (int)S.lcnt[si][warp];
+      const int n_list = (int)S.lcnt[si][warp], res = (int)S.lres[si][warp];
+      const int n_it = visit_count(false, w_lo, w_hi, n_list, res);
       for (int i = lane; i < n_it; i += 32) {
-        const int k = full ? w_lo + i : (int)kl[i];
+        const int k = visit_key(i, false, w_lo, kl, n_list, res);
         const float v = sc[off + k];
         if (bin_of(v, m) != bstar) continue;
         const uint32_t slot = atomicAdd(a.cand_cnt + p, 1u);
         if (slot < (uint32_t)kCand)
           a.cand[(int64_t)p * kCand + slot] = ((unsigned long long)order_key(v) << 32) | (0xFFFFFFFFu - (uint32_t)(jlo + k));
-        else
-          atomicOr(a.flags, 1u);
+      }
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {  // arrive; the problem's designated CTA waits for all and finds the cut
+        atomicAdd(a.pticket + p, 1u);
+        S.cut_idx = c == cta_of((int64_t)p * a.N + a.N / 2, a) &&
+                            wait_count(a.pticket + p, (uint32_t)(cl - cf + 1), a.err, a.wait_limit)
+                        ? 1
+                        : 0;
+      }
+      __syncthreads();
+      if (S.cut_idx) {
+        __threadfence();
+        select_cut(a, S, p, cf, cl, m, scale);
+      }
+      __syncthreads();
+    }
+    if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
+    // every CTA has passed its last barrier: the last one to get here rewinds the barrier
+    // counter so the next launch (whatever its grid size) starts from zero
+    if (tid == 0 && atomicAdd(a.bar + 1, 1ull) == (unsigned long long)(G - 1)) {
+      a.bar[0] = 0ull;
+      a.bar[1] = 0ull;
+    }
+    for (int si = 0; si < nseg; ++si) {
+      const Seg& s = S.seg[si];
+      const int p = s.p;
+      const uint32_t tk = (uint32_t)__ldcg(a.psum + kPsum * (int64_t)p + 4);
+      const long long before = __ldcg(a.cres + 2 * (int64_t)(p + c)), take = __ldcg(a.cres + 2 * (int64_t)(p + c) + 1);
+      // per-warp counts over the keep list (or the whole chunk), exclusive warp bases, then the
+      // positions in ascending order: warp lists in warp order, ballots within 32-key steps
+      const int off = (int)s.off, rows = (int)(s.jhi - s.jlo), jlo = (int)s.jlo;
+      const int wlen = (rows + kWarps - 1) / kWarps;
+      const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
+      const KeepT* kl = keep + s.kbase + warp * s.kcap;
+      const int n_list = (int)S.lcnt[si][warp], res = (int)S.lres[si][warp];
+      const int n_it = visit_count(false, w_lo, w_hi, n_list, res);
+      uint32_t wg = 0, we = 0;
+      for (int i0 = 0; i0 < n_it; i0 += 32) {
+        const int i = i0 + lane;
+        uint32_t kk = 0u;
+        if (i < n_it) kk = order_key(sc[off + visit_key(i, false, w_lo, kl, n_list, res)]);
+        wg += __popc(__ballot_sync(0xffffffffu, i < n_it && kk > tk));
+        we += __popc(__ballot_sync(0xffffffffu, i < n_it && kk == tk));
+      }
+      if (lane == 0) {
+        S.wcnt[si][warp][0] = wg;
+        S.wcnt[si][warp][1] = we;
+      }
+      __syncthreads();
+      if (warp == 0) {  // exclusive warp bases (one warp, one lane per warp)
+        uint32_t g1 = S.wcnt[si][lane][0], e1 = S.wcnt[si][lane][1];
+        uint32_t gi = g1, ei = e1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t gy = __shfl_up_sync(0xffffffffu, gi, o), ey = __shfl_up_sync(0xffffffffu, ei, o);
+          if (lane >= o) {
+            gi += gy;
+            ei += ey;
+          }
+        }
+        S.wcnt[si][lane][0] = gi - g1;
+        S.wcnt[si][lane][1] = ei - e1;
+      }
+      __syncthreads();
+      long long g_run = S.wcnt[si][warp][0], e_run = S.wcnt[si][warp][1];
+      const uint32_t lt = (1u << lane) - 1u;
+      int32_t* dst = a.sel_idx + (int64_t)p * a.max_select;
+      for (int i0 = 0; i0 < n_it; i0 += 32) {
+        const int i = i0 + lane;
+        int k = 0;
+        uint32_t kk = 0u;
+        if (i < n_it) {
+          k = visit_key(i, false, w_lo, kl, n_list, res);
+          kk = order_key(sc[off + k]);
+        }
+        const bool isg = i < n_it && kk > tk;
+        const bool ise = i < n_it && kk == tk;
+        const uint32_t bg = __ballot_sync(0xffffffffu, isg), be = __ballot_sync(0xffffffffu, ise);
+        const long long g_le = g_run + __popc(bg & lt), e_le = e_run + __popc(be & lt);
+        if (isg || (ise && e_le < take)) {
+          const long long pos = before + g_le + (e_le < take ? e_le : take);
+          if (pos < a.max_select) dst[pos] = jlo + k;
+          else atomicOr(a.err, kErrOverflow);
+        }
+        g_run += __popc(bg);
+        e_run += __popc(be);
+      }
+      __syncthreads();
+    }
+    return;
+  }
+
+  // ---- fallback (some problem's crossing bin is the coarse bin or holds more than kCand keys;
+  // decided identically by every CTA from the launch's flag): the candidates of the problems
+  // that fit are gathered by atomics, the others refine by radix levels over the key bits.
+  for (int si = 0; si < nseg; ++si) {
+    const int p = S.seg[si].p;
+    if (tid == 0) {
+      Seg& sg = S.seg[si];
+      const unsigned long long* ps = a.psum + kPsum * (int64_t)p;
+      sg.Z = __ldcg(ps);
+      sg.T = __ldcg(ps + 1);
+      sg.rem = __ldcg(ps + 2);
+      const unsigned long long w3 = __ldcg(ps + 3);
+      sg.bstar = (int)(uint32_t)w3;
+      // the coarse bin cannot be resolved from the keep lists, nor a crossing bin with more keys
+      // than the candidate list holds: those problems refine by radix
+      sg.radix = sg.bstar >= kFine || (w3 >> 32) > (unsigned long long)kCand;
+      if (sg.radix && c == cf_of(p, a)) atomicAdd(a.cand_cnt + p, (uint32_t)kCand + 1u);
+    }
+    __syncthreads();
+    const int bstar = S.seg[si].bstar;
+    if (!S.seg[si].radix) {
+      const int off = (int)S.seg[si].off, jlo = (int)S.seg[si].jlo, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
+      const float m = S.seg[si].m;
+      const int wlen = (rows + kWarps - 1) / kWarps;
+      const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
+      const KeepT* kl = keep + S.seg[si].kbase + warp * S.seg[si].kcap;
+      const int n_list = (int)S.lcnt[si][warp], res = (int)S.lres[si][warp];
+      const int n_it = visit_count(false, w_lo, w_hi, n_list, res);
+      for (int i = lane; i < n_it; i += 32) {
+        const int k = visit_key(i, false, w_lo, kl, n_list, res);
+        const float v = sc[off + k];
+        if (bin_of(v, m) != bstar) continue;
+        const uint32_t slot = atomicAdd(a.cand_cnt + p, 1u);
+        if (slot < (uint32_t)kCand)
+          a.cand[(int64_t)p * kCand + slot] = ((unsigned long long)order_key(v) << 32) | (0xFFFFFFFFu - (uint32_t)(jlo + k));
       }
     }
     __syncthreads();
   }
   if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
 
-  // ---- phase D: exact cut.  Problems whose crossing bin fits the candidate list sort it;
-  // the others (decided identically by every CTA from the global counts) refine by radix.
-  if (tid == 0) S.cut_idx = (int)__ldcg(a.flags);
-  __syncthreads();
-  const bool fallback = S.cut_idx != 0;
-  __syncthreads();
+  // exact cut.  Problems whose crossing bin fits the candidate list sort it; the others
+  // (decided identically by every CTA from the global counts) refine by radix.
+  constexpr bool fallback = true;
   for (int si = 0; si < nseg; ++si) {
     const int p = S.seg[si].p;
     // one round trip: the count and the candidate slots together
@@ -708,16 +1027,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   for (int si = 0; si < nseg; ++si) {
     const int off = (int)S.seg[si].off, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
     const uint32_t tk = S.seg[si].t_key;
-    const bool full = S.seg[si].bstar >= kFine || S.seg[si].full;
+    const bool whole = S.seg[si].bstar >= kFine;
     const int wlen = (rows + kWarps - 1) / kWarps;
     const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
     const KeepT* kl = keep + S.seg[si].kbase + warp * S.seg[si].kcap;
-    const int n_it = full ? (w_hi - w_lo) : (int)S.lcnt[si][warp];
+    const int n_list = (int)S.lcnt[si][warp], res = (int)S.lres[si][warp];
+    const int n_it = visit_count(whole, w_lo, w_hi, n_list, res);
     uint32_t wg = 0, we = 0;
     for (int i0 = 0; i0 < n_it; i0 += 32) {
       const int i = i0 + lane;
       uint32_t key = 0u;
-      if (i < n_it) key = order_key(sc[off + (full ? w_lo + i : (int)kl[i])]);
+      if (i < n_it) key = order_key(sc[off + visit_key(i, whole, w_lo, kl, n_list, res)]);
       wg += __popc(__ballot_sync(0xffffffffu, i < n_it && key > tk));
       we += __popc(__ballot_sync(0xffffffffu, i < n_it && key == tk));
     }
@@ -744,18 +1064,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   }
 
   // ---- phase E: offsets across CTAs; ordered compaction; clean the scratch for the next launch
-  for (int64_t i = (int64_t)c * kThreads + tid; i < nh; i += (int64_t)G * kThreads) {
-    a.h1.lo[i] = 0u;
-    a.h1.hi[i] = 0u;
-  }
   if (fallback) zero_global_hist(a.hr, 3 * nh, c, G);
   for (int i = c * kThreads + tid; i < a.P; i += G * kThreads) a.cand_cnt[i] = 0u;
-  if (c == 0 && tid == 0) a.flags[0] = 0u;
 
   for (int si = 0; si < nseg; ++si) {
     const Seg& s = S.seg[si];
     const int p = s.p;
-    const int cf = cf_of(p, a), cl = (int)(((int64_t)p * a.N + a.N - 1) / a.L);
+    const int cf = cf_of(p, a), cl = cl_of(p, a);
     for (int cc = cf + tid; cc <= c; cc += kThreads) {
       S.slot[2 * (cc - cf)] = __ldcg(a.slot_cnt + 2 * (p + cc));
       S.slot[2 * (cc - cf) + 1] = __ldcg(a.slot_cnt + 2 * (p + cc) + 1);
@@ -796,11 +1111,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     const long long before = S.before, take = S.take;
     const int off = (int)s.off, rows = (int)(s.jhi - s.jlo), jlo = (int)s.jlo;
     const uint32_t tk = s.t_key;
-    const bool full = s.bstar >= kFine || s.full;
+    const bool whole = s.bstar >= kFine;
     const int wlen = (rows + kWarps - 1) / kWarps;
     const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
     const KeepT* kl = keep + s.kbase + warp * s.kcap;
-    const int n_it = full ? (w_hi - w_lo) : (int)S.lcnt[si][warp];
+    const int n_list = (int)S.lcnt[si][warp], res = (int)S.lres[si][warp];
+    const int n_it = visit_count(whole, w_lo, w_hi, n_list, res);
     long long g_run = S.wcnt[si][warp][0], e_run = S.wcnt[si][warp][1];
     const uint32_t lt = (1u << lane) - 1u;
     int32_t* dst = a.sel_idx + (int64_t)p * a.max_select;
@@ -809,7 +1125,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
       int k = 0;
       uint32_t key = 0u;
       if (i < n_it) {
-        k = full ? w_lo + i : (int)kl[i];
+        k = visit_key(i, whole, w_lo, kl, n_list, res);
         key = order_key(sc[off + k]);
       }
       const bool isg = i < n_it && key > tk;
@@ -832,9 +1148,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
 
 size_t select_fixed_smem() { return (sizeof(Smem) + 127) / 128 * 128; }
 
-// scores (fp32) + keep lists (16-bit, a quarter of the keys plus per-warp rounding)
+// scores (fp32) + keep lists (16-bit, 3/8 of the keys plus per-warp rounding)
 size_t select_var_smem(int64_t per) {
-  return 4 * (size_t)((per + 3) / 4 * 4) + 2 * (size_t)(per / 4 + kWarps * (2 * kSelMaxSeg + 2));
+  return 4 * (size_t)((per + 3) / 4 * 4) + 2 * (size_t)(per * 3 / 8 + 1 + kWarps * (2 * kSelMaxSeg + 2));
 }
 
 SelectGeom select_geometry(const rtp_layer* L, int64_t N) {
@@ -850,10 +1166,27 @@ SelectGeom select_geometry(const rtp_layer* L, int64_t N) {
   G = (int)((total + per - 1) / per);
   g.grid = G;
   g.per_cta = per;
+  g.pair = 2 * per;
+  g.even = per;
   const size_t fixed = select_fixed_smem();
   const size_t need = fixed + select_var_smem(per);
   g.smem_scores = need <= L->smem_optin;
   g.smem_bytes = g.smem_scores ? need : fixed;
+  // one CTA on every SM: the even SM of each TPC takes the larger share of a pair's keys, if
+  // the larger range still fits the same score storage and segment limit
+  if (G == L->sm_count && G >= 2) {
+    int64_t le = (int64_t)llround((double)(2 * per) * kSelEvenShare);
+    if (le > (int64_t)(kSelMaxSeg - 1) * N) le = (int64_t)(kSelMaxSeg - 1) * N;
+    if (le > per) {
+      const size_t need_e = fixed + select_var_smem(le);
+      if (!g.smem_scores || need_e <= L->smem_optin) {
+        g.even = le;
+        g.per_cta = le;
+        if (g.smem_scores) g.smem_bytes = need_e;
+        g.parity = true;
+      }
+    }
+  }
   return g;
 }
 
@@ -868,6 +1201,9 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   a.P = L->B * L->Hr;
   a.N = N;
   a.L = g.per_cta;
+  a.Lp = g.pair;
+  a.Le = g.even;
+  a.use_smid = 0;
   int lg = 0;
   while ((1ll << lg) < N) ++lg;
   a.sc_bits = 62 - lg;
@@ -879,7 +1215,7 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   a.sel_thr = L->sel_thr;
   a.seg_max = L->seg_max;
   const int64_t nh = (int64_t)a.P * kBins;
-  a.h1 = Hist3{L->sel_words, L->sel_words + nh, L->sel_words + 2 * nh};
+  a.h1 = reinterpret_cast<unsigned long long*>(L->sel_words);  // the first 2 * nh words
   a.hr = Hist3{L->sel_words + 3 * nh, L->sel_words + 6 * nh, L->sel_words + 9 * nh};
   a.cand_cnt = L->cand_cnt;
   a.cand = L->cand;
@@ -889,6 +1225,12 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   a.gscores = L->gscores;
   a.keep = L->sel_keep;
   a.flags = L->sel_flags;
+  if (++L->sel_epoch == 0u) L->sel_epoch = 1u;
+  a.epoch = L->sel_epoch;
+  a.cum = L->sel_cum;
+  a.psum = L->sel_psum;
+  a.cres = L->sel_cres;
+  a.pticket = L->sel_pticket;
   a.wait_limit = L->wait_limit > 0 ? L->wait_limit : kWaitLimitCycles;
   if (!g.smem_scores && L->gscores == nullptr) return cudaErrorInvalidValue;
   if (g.grid > L->sm_count || g.grid > kSelMaxGrid) return cudaErrorInvalidValue;
@@ -904,6 +1246,8 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, g.smem_bytes);
   if (e != cudaSuccess) return e;
   if (occ < 1 || g.grid > occ * L->sm_count) return cudaErrorCooperativeLaunchTooLarge;
+  // SM-numbered ranges need exactly one CTA on every SM; otherwise the same split by block index
+  if (g.parity) a.use_smid = occ == 1 ? 1 : 0;
   return cudaLaunchCooperativeKernel(fn, dim3(g.grid), dim3(kThreads), args, g.smem_bytes, st);
 }
 

@@ -21,7 +21,14 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelBins = 2048;   // level-1 score bins (width 1/64 below the row max) and radix digits
 constexpr int kSelMaxSeg = 16;   // (problem, CTA) segments one CTA may hold
 constexpr int kSelCand = 1024;   // crossing-bin keys resolved by an in-CTA sort
+constexpr int kSelFine = 1024;   // level-1 fine bins (width 1/64 below the row max, 16 deep)
 constexpr int kSelMaxGrid = 256; // CTAs of the selection grid (<= SM count)
+// Share of a CTA pair's keys taken by the even SM of a TPC when every SM holds one selection
+// CTA.  The two SMs of a TPC share its bandwidth unevenly: with equal key counts the index
+// stream took 57 us on even and 66 us on odd SMs; with a 0.537 share, 61.5 and 54.9 us (the odd
+// SM speeds up as its partner's share grows); with 0.521, 59.6 and 63.5 us.  Interpolating the
+// difference to zero gives 0.527.
+constexpr double kSelEvenShare = 0.527;
 
 // Sparse-attention gather (decode): indices per work item.
 constexpr int kGatherChunk = 128;
@@ -102,7 +109,12 @@ struct rtp_layer {
   uint32_t* cand_cnt = nullptr;   // [P]
   unsigned long long* cand = nullptr;  // [P][kSelCand]
   uint32_t* sel_keep = nullptr;   // [P][max_seq] keep lists of the selection (global-score mode)
-  uint32_t* sel_flags = nullptr;  // [1] radix fallback flag
+  uint32_t* sel_flags = nullptr;  // [1] radix fallback flag (the epoch of the launch that set it)
+  uint32_t sel_epoch = 0;         // launches of the decode selection (its flag epochs)
+  uint32_t* sel_cum = nullptr;    // [P + G][1024] cumulative fine-bin counts per (problem, CTA)
+  unsigned long long* sel_psum = nullptr;   // [P][8] per-problem crossing summaries and cut keys
+  long long* sel_cres = nullptr;            // [P + G][2] per-(problem, CTA) compaction offsets
+  uint32_t* sel_pticket = nullptr;          // [P] phase completion tickets
   uint32_t* slot_cnt = nullptr;  // [P + G][2]
   unsigned long long* bar = nullptr;  // [2] grid barrier arrival / exit counters
   float* gscores = nullptr;      // [P][max_seq] when scores do not fit in shared memory
@@ -159,7 +171,10 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
 // Selection kernel geometry for the current length (host-side; also sizes scratch).
 struct SelectGeom {
   int grid = 0;
-  int64_t per_cta = 0;
+  int64_t per_cta = 0;  // keys of the longest CTA range
+  int64_t pair = 0;     // keys per CTA pair
+  int64_t even = 0;     // keys of the even member of a pair
+  bool parity = false;  // pairs split unevenly (by SM number, one CTA on every SM)
   bool smem_scores = true;
   size_t smem_bytes = 0;
 };

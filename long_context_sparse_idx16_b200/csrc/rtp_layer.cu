@@ -49,6 +49,7 @@ static cudaError_t reset_select_scratch(rtp_layer* L) {
   if (e == cudaSuccess) e = cudaMemset(L->cand_cnt, 0, P * sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(L->bar, 0, 2 * sizeof(unsigned long long));
   if (e == cudaSuccess) e = cudaMemset(L->sel_flags, 0, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(L->sel_pticket, 0, P * sizeof(uint32_t));
   return e;
 }
 
@@ -101,7 +102,7 @@ static void free_all(rtp_layer* L) {
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
                   L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt, L->pf_capture, L->attn_part,
-                  L->attn_ticket};
+                  L->attn_ticket, L->sel_cum, L->sel_psum, L->sel_pticket, L->sel_cres};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -213,7 +214,7 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   const int64_t G = L->sm_count;
   // Largest per-CTA score count the shared-memory variant can hold; beyond it the
   // selection keeps scores in global scratch.
-  const int64_t smem_cap = ((int64_t)L->smem_optin - (int64_t)select_fixed_smem() - 2 * 32 * 34) * 2 / 9;
+  const int64_t smem_cap = ((int64_t)L->smem_optin - (int64_t)select_fixed_smem() - 2 * 32 * 34 - 2) * 4 / 19;
   const bool need_gscores = P * L->max_seq > smem_cap * G;
   const int64_t gitems = P * ((L->max_seq + kGatherChunk - 1) / kGatherChunk);
 
@@ -264,6 +265,10 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   RTP_ALLOC(L->cand, P * kSelCand);
   RTP_ALLOC(L->sel_keep, P * L->max_seq);
   RTP_ALLOC(L->sel_flags, 1);
+  RTP_ALLOC(L->sel_cum, (P + G) * kSelFine);
+  RTP_ALLOC(L->sel_psum, 8 * P);
+  RTP_ALLOC(L->sel_cres, 2 * (P + G));
+  RTP_ALLOC(L->sel_pticket, P);
   RTP_ALLOC(L->slot_cnt, 2 * (P + G));
   RTP_ALLOC(L->bar, 2);
   if (need_gscores) {
