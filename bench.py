@@ -69,11 +69,11 @@ MUFU_EX2_PER_CLK_SM = 16
 
 
 def _prefill_traffic(kernel: str, workload: str):
-    """Per-launch DRAM bytes of the prefill selection at the 32K chunk, from the committed ncu
-    summary, while its sources are unchanged since the capture (else None).  Other kernels and
-    the 1M chunk have no capture whose bytes would scale: the 32K index keys sit in L2, the
-    1M ones do not."""
-    if kernel != "prefill_select" or workload != "prefill_32k":
+    """Per-launch DRAM bytes of the prefill retrieval kernels at the 32K chunk, from the
+    committed ncu summary, while their sources are unchanged since the capture (else None).
+    The 1M chunk has no capture whose bytes would scale: the 32K index keys sit in L2, the 1M
+    ones do not."""
+    if kernel not in ("prefill_select", "prefill_attn") or workload != "prefill_32k":
         return None
     try:
         text = open(os.path.join(ROOT, "profiles", "prefill_kernels_32k.md")).read()
@@ -81,9 +81,9 @@ def _prefill_traffic(kernel: str, workload: str):
         return None
     traffic, srcs = None, None
     for line in text.splitlines():
-        if line.startswith("- prefill_select dram bytes per launch (read + write):"):
+        if line.startswith(f"- {kernel} dram bytes per launch (read + write):"):
             traffic = float(line.rsplit(":", 1)[1].strip().split()[0])
-        if line.startswith("- prefill_select sources sha256[:16]:"):
+        if line.startswith(f"- {kernel} sources sha256[:16]:"):
             srcs = line.split("sha256[:16]:", 1)[1].strip()
     if traffic is None or srcs is None:
         return None
@@ -137,6 +137,9 @@ def _prefill_rooflines(kern: dict, flops: dict, exps: int, exp_peak: dict, sm_mh
             "peak_kind": tensor_peak_kind, "unit": "TFLOP/s", "frac": a / tensor_peak, "flops_per_launch": int(f),
             "ms_per_launch": ms}
     return out
+
+
+_TRAFFIC_KEYS = 40 * 131072  # keys streamed by the launch the committed traffic figure is for
 
 
 def _profile_traffic(kernel_src: str):
@@ -632,7 +635,9 @@ def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=Non
             "ms_per_step": ms / steps, "config": _config(s, world),
             "roofline": {"bound": "hbm", "kernel": "decode_select (fused index stream + exact top-p)",
                          "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic if s.name == "decode_128k" else None,
+                         "frac": achieved / peak,
+                         # the capture streams fp32 keys; its bytes scale with the keys streamed
+                         "traffic": (traffic * P * N / _TRAFFIC_KEYS if traffic and key_bytes == 4 else None),
                          "bytes_per_launch": sel_bytes, "us_per_launch": sel_us},
             "step_roofline": {"bytes_per_step": step_bytes, "roofline_us_per_step": step_bytes / (peak * 1e9) * 1e6,
                               "frac": step_bytes / (peak * 1e9) / (ms / steps * 1e-3)},
@@ -746,6 +751,8 @@ def measure_prefill(s, x, steps: int, warmup: int, world: int, dev, exp_peak: di
     roofs = _prefill_rooflines(kern, flops, pairs, exp_peak, (clk or {}).get("sm_mhz"), peak, peak_kind)
     if "prefill_select" in roofs:
         roofs["prefill_select"]["traffic"] = _prefill_traffic("prefill_select", s.name)
+    if "prefill_attn" in roofs:
+        roofs["prefill_attn"]["traffic"] = _prefill_traffic("prefill_attn", s.name)
     # the chunk's dominant kernel is the headline roofline
     dom = max((k for k in ("prefill_select", "prefill_attn", "prefill_local") if k in roofs),
               key=lambda k: roofs[k]["ms_per_launch"])
