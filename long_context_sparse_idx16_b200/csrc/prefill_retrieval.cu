@@ -237,7 +237,7 @@ struct SelWalk {
   }
 };
 
-__global__ void __launch_bounds__(kPsThreads) prefill_select_kernel(RetArgs a,
+__global__ void __launch_bounds__(kPsThreads, 6) prefill_select_kernel(RetArgs a,
                                                                      const __grid_constant__ CUtensorMap tm_idx) {
   extern __shared__ __align__(1024) unsigned char sm[];
   const uint32_t sbase = smem_u32(sm);
@@ -568,7 +568,8 @@ constexpr uint32_t kAOffK = kAOffIK + kIdxStages * kTcKBytes;    // K tile, 16 K
 constexpr uint32_t kAOffV = kAOffK + kKeysR * 256;               // V tile, 16 KB
 constexpr uint32_t kAOffP = kAOffV + kKeysR * 256;               // P tile, 16 KB
 constexpr uint32_t kAOffX = kAOffP + kRowsR * 128;               // mask exchange [2][128] u32, count [128]
-constexpr uint32_t kAOffBar = kAOffX + 3 * kRowsR * 4;           // ifull[3], idone, kfull, vfull, sdone, odone
+constexpr uint32_t kAOffXf = kAOffX + 3 * kRowsR * 4;            // per-thread float exchange [256]
+constexpr uint32_t kAOffBar = kAOffXf + kAttThreads * 4;         // ifull[3], idone, kfull, vfull, sdone, odone
 constexpr uint32_t kAttSmem = kAOffBar + 8 * 8 + 16;
 static_assert(kAOffK % 1024 == 0 && kAOffV % 1024 == 0 && kAOffP % 1024 == 0, "swizzled tiles need 1 KB alignment");
 constexpr uint32_t kKVTileBytes = kKeysR * 256;
@@ -675,6 +676,15 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
     tma_load_2d(dst, map, 0, y, bar);
     tma_load_2d(dst + kKeysR * 128, map, 64, y, bar);
   };
+  // The row's cut as a float: key j is selected iff s_j > tf, or s_j == tf at a position
+  // j <= tcut.  Float order equals the order of the (canonical, +0 for -0) order keys.  A row
+  // without a cut has tk = 0xFFFFFFFF, whose float is a NaN that no score exceeds or equals;
+  // the cut of p = 1 is tk = 0, below every finite score (-inf here).
+  const float tf = tk == 0u ? -INFINITY : key_to_float(tk);
+  // columns 0 .. x of this thread's 32 (none for x < 0, all for x >= 31)
+  auto prefix_bits = [](int64_t x) -> uint32_t {
+    return x < 0 ? 0u : (x >= 31 ? 0xFFFFFFFFu : (2u << (uint32_t)x) - 1u);
+  };
   // this thread's selection mask of tile t (its 32 columns) from the index scores in TMEM
   auto read_mask = [&](int64_t t) -> uint32_t {
     okw = mbar_wait(barIdone, n_idone & 1u) && okw;
@@ -684,32 +694,25 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
     float s[32];
     tmem_ld32(lane_addr + kColIdx + 32u * half, s);
     tmem_ld_wait();
-    const int lim = causal_lim(pos, t) - 32 * half;
-    uint32_t mk = 0u;
+    const int64_t j0 = t * kKeysR + 32 * half;  // position of column 0
+    uint32_t gt[4] = {0u, 0u, 0u, 0u}, eq[4] = {0u, 0u, 0u, 0u};  // independent chains
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const int64_t j = t * kKeysR + 32 * half + i;
-      const uint32_t key = order_key(s[i] + 0.0f);
-      const bool sel = i <= lim && (key > tk || (key == tk && j <= tcut));
-      mk |= (uint32_t)sel << i;
+      gt[i & 3] |= (s[i] > tf ? 1u : 0u) << i;
+      eq[i & 3] |= (s[i] == tf ? 1u : 0u) << i;
     }
-    return mk;
+    const uint32_t g = (gt[0] | gt[1]) | (gt[2] | gt[3]), e = (eq[0] | eq[1]) | (eq[2] | eq[3]);
+    return (g | (e & prefix_bits(tcut - j0))) & prefix_bits(pos - j0);
   };
-  // exchange one float per row between the two halves through TMEM columns of the S buffer
-  // that both have already read
+  // exchange one float per row between the two halves (threads tid and tid ^ 128) through
+  // shared memory; consecutive calls are separated by at least one CTA barrier
+  float* xf = reinterpret_cast<float*>(sm + kAOffXf);
   auto swap_half = [&](float v) -> float {
-    float w[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) w[i] = v;
-    __syncwarp();
-    tmem_st32(lane_addr + kColS + 32u * half, w);
-    tmem_st_wait();
-    tc_fence_before();
+    xf[tid] = v;
+    tc_fence_before();  // also orders this thread's TMEM reads before the barrier
     __syncthreads();
     tc_fence_after();
-    tmem_ld32(lane_addr + kColS + 32u * (1 - half), w);
-    tmem_ld_wait();
-    return w[0];
+    return xf[tid ^ kRowsR];
   };
 
   // ---- prologue: index key tiles tb .. tb + 2 in flight, the scores of tile tb, its masks
@@ -770,7 +773,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
       mask_next = read_mask(t + 1);
       tc_fence_before();
       if (half == 1) xm[((t + 1) & 1) * kRowsR + r] = mask_next;
-      any_next = __syncthreads_or(mask_next != 0u) != 0;
+      // one barrier: does any row select a key of tile t + 1, and has any wait given up
+      const int f = __syncthreads_or((mask_next != 0u ? 1 : 0) | (okw ? 0 : 2));
+      any_next = (f & 1) != 0;
+      if (f & 2) ok = false;
       if (tid == 0 && u + 2 < ntl && okw) {
         okw = mbar_wait(barI + 8u * (uint32_t)((u + 2) % kIdxStages), (uint32_t)(((u + 2) / kIdxStages) & 1));
         if (okw) tc_issue_scores(tmem + kColIdx, sbase + kAOffIQ, ikt(u + 2), barIdone);
@@ -804,12 +810,13 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
       float sv[32];
       tmem_ld32(lane_addr + kColS + 32u * half, sv);
       tmem_ld_wait();
-      float mx = -INFINITY;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // independent chains
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         sv[i] = ((mask_cur >> i) & 1u) ? sv[i] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, sv[i]);
+        m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
       }
+      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       mx = fmaxf(mx, swap_half(mx));  // the row max over both halves (also orders the S reads)
       // S of tile t is done, and so is P V of the previous tile: K, P and O are free
       if (tid == 0 && any_next && okw) load_kv(barK, sbase + kAOffK, &tm_k, t + 1);
@@ -832,7 +839,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
         l *= fast_exp2(m_ref - mx);  // 0 while m_ref is still -inf
         m_ref = mx;
       }
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
       const float mref = m_ref == -INFINITY ? 0.f : m_ref;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -840,7 +847,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           pv[e] = fast_exp2(sv[8 * q + e] - mref);
-          rs += pv[e];
+          rs4[e & 3] += pv[e];
         }
         uint4 w;
         w.x = pack_half2_r(pv[0], pv[1]);
@@ -849,7 +856,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
         w.w = pack_half2_r(pv[6], pv[7]);
         *reinterpret_cast<uint4*>(sm + kAOffP + sw128_off(r, 4 * half + q, kRowsR)) = w;
       }
-      l += rs;
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       fence_async_smem();
       tc_fence_before();
       ok = __syncthreads_and(okw ? 1 : 0) != 0;
@@ -877,13 +884,12 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
     }
     mask_cur = mask_next;
     any_cur = any_next;
-    ok = __syncthreads_and(okw ? 1 : 0) != 0;
+    // (no barrier here: the next tile's mask barrier also carries the wait status; a wait that
+    // gives up after it is seen by the attention barrier of the tile that follows, or the exit)
   }
 
-  if (ok && any_pv) {
-    if (tid == 0) okw = mbar_wait(barO, (n_o - 1) & 1u);
-    ok = __syncthreads_and(okw ? 1 : 0) != 0;
-  }
+  if (ok && any_pv && tid == 0) okw = mbar_wait(barO, (n_o - 1) & 1u) && okw;
+  ok = __syncthreads_and((ok && okw) ? 1 : 0) != 0;
   if (ok) {
     tc_fence_after();
     const float lt = l + swap_half(l);
