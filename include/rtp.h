@@ -59,7 +59,7 @@ typedef enum {
 typedef struct rtp_layer rtp_layer; /* opaque; owned by the library */
 
 typedef struct {
-  int32_t batch;              /* B >= 1 sequences; they share one length */
+  int32_t batch;              /* B sequences, 1 <= B <= 256; each has its own length */
   int32_t n_q_heads;          /* Hq >= 1 */
   int32_t n_kv_heads;         /* Hkv >= 1, divides Hq (GQA: q head h reads KV head h / (Hq/Hkv)) */
   int32_t head_dim;           /* D; must be 128 */
@@ -137,26 +137,33 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out);
 /* Release everything the layer owns.  Synchronises the device first.  NULL is a no-op. */
 rtp_status rtp_destroy(rtp_layer* layer);
 
-/* Append T >= 1 tokens to every sequence (positions len .. len+T-1): k, v are DEVICE bf16
- * [B][T][Hkv][D], k pre-RoPE.  Writes RoPE(k) and v into the fp16 KV cache and, for every
- * retrieval head h, the pre-RoPE index key Wk_h^T k into the index cache (the pages' 16-dim
- * indexer: techwalker page section 3; ngjoo digest, pre-RoPE projections).  Advances the
- * length by T.  RTP_ECAPACITY (nothing written) if len + T > max_seq. */
+/* Append T >= 1 tokens to every sequence, each at its own positions len_b .. len_b+T-1: k, v
+ * are DEVICE bf16 [B][T][Hkv][D], k pre-RoPE.  Writes RoPE(k) and v into the fp16 KV cache and,
+ * for every retrieval head h, the pre-RoPE index key Wk_h^T k into the index cache (the pages'
+ * 16-dim indexer: techwalker page section 3; ngjoo digest, pre-RoPE projections).  Advances
+ * every length by T.  RTP_ECAPACITY (nothing written) if some len_b + T > max_seq. */
 rtp_status rtp_append_kv(rtp_layer* layer, const void* k, const void* v, int32_t T,
                          cudaStream_t stream);
 
-/* One decode step for every sequence: q is DEVICE bf16 [B][Hq][D] pre-RoPE at position
- * len-1 (append its own key first).  out is DEVICE fp32 [B][Hq][D].  Retrieval heads run
+/* Ragged batches: append T >= 1 tokens to sequence b alone (k, v DEVICE bf16 [T][Hkv][D], k
+ * pre-RoPE) at positions len_b .. len_b+T-1, and advance len_b by T.  RTP_EINVAL for b outside
+ * [0, B); RTP_ECAPACITY (nothing written) if len_b + T > max_seq. */
+rtp_status rtp_append_kv_seq(rtp_layer* layer, int32_t b, const void* k, const void* v, int32_t T,
+                             cudaStream_t stream);
+
+/* One decode step for every sequence: q is DEVICE bf16 [B][Hq][D] pre-RoPE, sequence b's row at
+ * position len_b-1 (append its own key first; every len_b >= 1, else RTP_EINVAL).  Sequences of
+ * a ragged batch select and attend over their own keys only.  out is DEVICE fp32 [B][Hq][D].  Retrieval heads run
  * index scoring, exact top-p selection and sparse attention; local heads run window+sink
  * attention, on an internal stream forked from `stream` (an event) after the selection and
  * joined back (an event) before the call's work ends in `stream` order.  stats may be NULL. */
 rtp_status rtp_decode(rtp_layer* layer, const void* q, float* out, const rtp_decode_stats* stats,
                       cudaStream_t stream);
 
-/* Chunked prefill: the last C appended tokens are the chunk; q is DEVICE bf16 [B][C][Hq][D]
- * pre-RoPE, row i at position len-C+i.  Every row runs its own top-p selection over its causal
+/* Chunked prefill: the last C appended tokens of every sequence are its chunk; q is DEVICE bf16
+ * [B][C][Hq][D] pre-RoPE, row i of sequence b at position len_b-C+i (ragged batches too).  Every row runs its own top-p selection over its causal
  * prefix (retrieval heads) or its own window (local heads).  out is DEVICE fp32 [B][C][Hq][D].
- * Requires 1 <= C <= min(len, max_chunk).  The local heads run on an internal stream forked
+ * Requires 1 <= C <= min(shortest len_b, max_chunk).  The local heads run on an internal stream forked
  * from `stream` (an event) and joined back (an event).  stats may be NULL. */
 rtp_status rtp_prefill_chunk(rtp_layer* layer, const void* q, int32_t C, float* out,
                              const rtp_prefill_stats* stats, cudaStream_t stream);
@@ -172,16 +179,24 @@ rtp_status rtp_set_top_p(rtp_layer* layer, float top_p);
  * prefill kernels keep their fixed limit.  RTP_EINVAL if cycles < 0. */
 rtp_status rtp_set_wait_limit(rtp_layer* layer, int64_t cycles);
 
-/* Current sequence length (host-side counter; advanced by rtp_append_kv). */
+/* The longest sequence's length (host-side counters advanced by the appends): the common
+ * length of a batch whose sequences have one.  -1 for a NULL layer. */
 int64_t rtp_seq_len(const rtp_layer* layer);
 
-/* Forget every token (length back to 0); the caches are overwritten by later appends. */
+/* Length of sequence b; -1 for a NULL layer or b outside [0, B). */
+int64_t rtp_seq_len_of(const rtp_layer* layer, int32_t b);
+
+/* Forget every token (every length back to 0); the caches are overwritten by later appends. */
 rtp_status rtp_reset(rtp_layer* layer);
 
-/* Roll the length back to new_len <= current length (e.g. to re-run a step or drop rejected
- * speculative tokens); later appends overwrite the dropped positions.  RTP_EINVAL if
- * new_len is negative or above the current length. */
+/* Roll every sequence longer than new_len back to new_len (e.g. to re-run a step or drop
+ * rejected speculative tokens); later appends overwrite the dropped positions.  RTP_EINVAL if
+ * new_len is negative or above the longest length. */
 rtp_status rtp_truncate(rtp_layer* layer, int64_t new_len);
+
+/* Roll sequence b back to new_len <= its length.  RTP_EINVAL for b outside [0, B) or new_len
+ * outside [0, len_b]. */
+rtp_status rtp_truncate_seq(rtp_layer* layer, int32_t b, int64_t new_len);
 
 /* Per-kernel device timing.  While enabled, the library records a CUDA event pair on the
  * launch stream around every kernel it launches, and runs every kernel on the call's stream

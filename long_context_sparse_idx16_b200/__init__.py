@@ -75,6 +75,9 @@ def lib() -> C.CDLL:
             "rtp_create": ([C.POINTER(rtp_config), C.POINTER(C.c_void_p)], C.c_int),
             "rtp_destroy": ([P], C.c_int),
             "rtp_append_kv": ([P, P, P, i32, P], C.c_int),
+            "rtp_append_kv_seq": ([P, i32, P, P, i32, P], C.c_int),
+            "rtp_seq_len_of": ([P, i32], i64),
+            "rtp_truncate_seq": ([P, i32, i64], C.c_int),
             "rtp_decode": ([P, P, P, C.POINTER(rtp_decode_stats), P], C.c_int),
             "rtp_prefill_chunk": ([P, P, i32, P, C.POINTER(rtp_prefill_stats), P], C.c_int),
             "rtp_set_top_p": ([P, f32], C.c_int),
@@ -121,6 +124,10 @@ def rtp_append_kv(layer, k_ptr: int, v_ptr: int, T: int, stream: int) -> None:
     _check(lib().rtp_append_kv(layer, k_ptr, v_ptr, T, stream), layer)
 
 
+def rtp_append_kv_seq(layer, b: int, k_ptr: int, v_ptr: int, T: int, stream: int) -> None:
+    _check(lib().rtp_append_kv_seq(layer, b, k_ptr, v_ptr, T, stream), layer)
+
+
 def rtp_decode(layer, q_ptr: int, out_ptr: int, stats: Optional[rtp_decode_stats], stream: int) -> None:
     _check(lib().rtp_decode(layer, q_ptr, out_ptr, C.byref(stats) if stats is not None else None, stream), layer)
 
@@ -142,6 +149,14 @@ def rtp_set_wait_limit(layer, cycles: int) -> None:
 
 def rtp_seq_len(layer) -> int:
     return int(lib().rtp_seq_len(layer))
+
+
+def rtp_seq_len_of(layer, b: int) -> int:
+    return int(lib().rtp_seq_len_of(layer, b))
+
+
+def rtp_truncate_seq(layer, b: int, new_len: int) -> None:
+    _check(lib().rtp_truncate_seq(layer, b, new_len), layer)
 
 
 def rtp_reset(layer) -> None:
@@ -292,6 +307,21 @@ class Layer:
 
     def truncate(self, new_len: int) -> None:
         rtp_truncate(self.handle, new_len)
+
+    def seq_len_of(self, b: int) -> int:
+        return rtp_seq_len_of(self.handle, b)
+
+    def truncate_seq(self, b: int, new_len: int) -> None:
+        rtp_truncate_seq(self.handle, b, new_len)
+
+    def append_kv_seq(self, b: int, k, v, stream=None) -> None:
+        """Append to sequence b alone: k, v torch bf16 CUDA tensors [T][Hkv][128] (k pre-RoPE)."""
+        import torch
+
+        T = _dim(k, "k", 3, 0)
+        _need(k, "k", (T, self.n_kv_heads, 128), torch.bfloat16, self.device)
+        _need(v, "v", (T, self.n_kv_heads, 128), torch.bfloat16, self.device)
+        rtp_append_kv_seq(self.handle, b, k.data_ptr(), v.data_ptr(), T, _stream_handle(stream))
 
     def profile(self, on: bool) -> None:
         rtp_profile_enable(self.handle, on)

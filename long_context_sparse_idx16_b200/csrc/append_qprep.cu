@@ -33,11 +33,12 @@ constexpr int kAppTok = 8;
 template <bool kBf16>
 __global__ void __launch_bounds__(kAppThreads) append_kv_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, int T, int Hkv,
-    int Hr, int64_t pos0, int64_t max_seq, const double* __restrict__ theta,
+    int Hr, const SeqPos pos0, int b0, int64_t max_seq, const double* __restrict__ theta,
     const float* __restrict__ wk, const int16_t* __restrict__ ret_head, int group,
     __half* __restrict__ kc, __half* __restrict__ vc, float* __restrict__ idx, __nv_bfloat16* __restrict__ idx_b,
     __half* __restrict__ idx_hl, uint32_t* __restrict__ err) {
-  const int t0 = blockIdx.x * kAppTok, b = blockIdx.y, role = blockIdx.z;
+  // bl: the sequence's slot in this call's k / v; b: its index in the layer (caches, positions)
+  const int t0 = blockIdx.x * kAppTok, bl = blockIdx.y, b = b0 + bl, role = blockIdx.z;
   const int nt = min(kAppTok, T - t0);
   const int tid = threadIdx.x;
   if (role == 0) {
@@ -46,12 +47,12 @@ __global__ void __launch_bounds__(kAppThreads) append_kv_kernel(
     bool bad = false;
     for (int u = 0; u < nt; ++u) {
       const int t = t0 + u;
-      const int64_t pos = pos0 + t;
+      const int64_t pos = (int64_t)pos0.v[b] + t;
       __syncthreads();  // the previous token's angles are consumed
       if (tid < kHalfD) rope_cos_sin(pos, theta[tid], &cs[tid], &sn[tid]);
       __syncthreads();
-      const __nv_bfloat16* kt = k + ((int64_t)b * T + t) * Hkv * kD;
-      const __nv_bfloat16* vt = v + ((int64_t)b * T + t) * Hkv * kD;
+      const __nv_bfloat16* kt = k + ((int64_t)bl * T + t) * Hkv * kD;
+      const __nv_bfloat16* vt = v + ((int64_t)bl * T + t) * Hkv * kD;
       for (int i = tid; i < Hkv * kD; i += kAppThreads) {
         const int g = i / kD, d = i % kD;
         const float x = __bfloat162float(vt[i]);
@@ -82,8 +83,8 @@ __global__ void __launch_bounds__(kAppThreads) append_kv_kernel(
   for (int e = 0; e < 16; ++e) w[e] = wk[((int64_t)hr * kD + part * 16 + e) * kR + o];
   for (int u = 0; u < nt; ++u) {
     const int t = t0 + u;
-    const int64_t pos = pos0 + t;
-    const __nv_bfloat16* kt = k + (((int64_t)b * T + t) * Hkv + g) * kD + part * 16;
+    const int64_t pos = (int64_t)pos0.v[b] + t;
+    const __nv_bfloat16* kt = k + (((int64_t)bl * T + t) * Hkv + g) * kD + part * 16;
     float x[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) x[e] = __bfloat162float(kt[e]);
@@ -123,11 +124,11 @@ __global__ void __launch_bounds__(kAppThreads) append_kv_kernel(
 constexpr int kQHeads = 4;
 
 __global__ void __launch_bounds__(128) q_prep_kernel(
-    const __nv_bfloat16* __restrict__ q, int rows, int Hq, int Hr, int64_t pos0,
+    const __nv_bfloat16* __restrict__ q, int rows, int Hq, int Hr, const SeqPos pos0,
     const double* __restrict__ theta, const float* __restrict__ wq,
     const int16_t* __restrict__ head_slot, float* __restrict__ q_rot, float* __restrict__ q_idx) {
   const int i = blockIdx.x, b = blockIdx.y, h0 = blockIdx.z * kQHeads;
-  const int64_t pos = pos0 + i;
+  const int64_t pos = (int64_t)pos0.v[b] + i;  // row i of sequence b
   const int d = threadIdx.x;
   __shared__ float cs[kHalfD], sn[kHalfD];
   __shared__ float qs[kQHeads][kD];
@@ -183,16 +184,22 @@ __global__ void __launch_bounds__(128) q_prep_kernel(
 
 }  // namespace
 
-cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T,
-                             cudaStream_t st) {
-  dim3 grid((T + kAppTok - 1) / kAppTok, L->B, 1 + L->Hr);
+SeqPos seq_pos(const rtp_layer* L, int64_t delta) {
+  SeqPos s{};
+  for (int b = 0; b < L->B; ++b) s.v[b] = (int32_t)(L->lens[b] + delta);
+  return s;
+}
+
+cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T, int b0,
+                             int nb, cudaStream_t st) {
+  dim3 grid((T + kAppTok - 1) / kAppTok, nb, 1 + L->Hr);
   auto fn = L->index_bf16 ? append_kv_kernel<true> : append_kv_kernel<false>;
-  fn<<<grid, kAppThreads, 0, st>>>(k, v, T, L->Hkv, L->Hr, L->len, L->max_seq, L->theta, L->wk, L->d_ret_head,
-                                   L->group, L->kc, L->vc, L->idx, L->idx_b, L->idx_hl, L->err);
+  fn<<<grid, kAppThreads, 0, st>>>(k, v, T, L->Hkv, L->Hr, seq_pos(L, 0), b0, L->max_seq, L->theta, L->wk,
+                                   L->d_ret_head, L->group, L->kc, L->vc, L->idx, L->idx_b, L->idx_hl, L->err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, int64_t pos0,
+cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, const SeqPos& pos0,
                           cudaStream_t st) {
   dim3 grid(rows, L->B, (L->Hq + kQHeads - 1) / kQHeads);
   q_prep_kernel<<<grid, 128, 0, st>>>(q, rows, L->Hq, L->Hr, pos0, L->theta, L->wq, L->d_head_slot,

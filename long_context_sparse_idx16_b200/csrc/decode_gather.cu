@@ -41,7 +41,7 @@ struct GatherArgs {
   const int16_t* ret_head;
   int P;
   int dense;
-  int64_t N;
+  SeqPos lens;  // each sequence's length (a dense step attends to all its keys)
   float scale_log2;
   float* part;
   uint32_t* ticket;
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kThreads) decode_gather_kernel(GatherArgs a) {
 
   // item prefix over problems: counts loaded in parallel, summed by one thread from smem
   for (int p = tid; p < a.P; p += kThreads) {
-    const int64_t K = a.dense ? a.N : (int64_t)a.sel_cnt[p];
+    const int64_t K = a.dense ? (int64_t)a.lens.v[p / a.Hr] : (int64_t)a.sel_cnt[p];
     s_base[p + 1] = (int)((K + kChunk - 1) / kChunk);
   }
   __syncthreads();
@@ -88,7 +88,8 @@ __global__ void __launch_bounds__(kThreads) decode_gather_kernel(GatherArgs a) {
     const int n_items = s_base[p + 1] - s_base[p];
     const int b = p / a.Hr, hr = p % a.Hr;
     const int h = a.ret_head[hr], g = h / a.group;
-    const int64_t K = a.dense ? a.N : (int64_t)a.sel_cnt[p];
+    const int64_t Nb = a.lens.v[b];  // this sequence's keys
+    const int64_t K = a.dense ? Nb : (int64_t)a.sel_cnt[p];
     const int64_t r_lo = (int64_t)chunk * kChunk;
     const int64_t r_hi = min(K, r_lo + kChunk);
 
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) decode_gather_kernel(GatherArgs a) {
       const int64_t r = r_lo + (warp * 2 + half) + 2 * kWarps * u;
       if (r < r_hi) {
         int64_t j = a.dense ? r : (int64_t)__ldg(ids + r);
-        if ((uint64_t)j >= (uint64_t)a.N) {  // never expected: a stale or corrupt list
+        if ((uint64_t)j >= (uint64_t)Nb) {  // never expected: a stale or corrupt list
           atomicOr(a.err, kErrInternal);
           j = 0;
         }
@@ -250,17 +251,19 @@ __global__ void __launch_bounds__(kThreads) decode_gather_kernel(GatherArgs a) {
 }
 
 // p == 1: every causal key is selected.
-__global__ void dense_stats_kernel(int32_t* cnt, float* mass, float* thr, int P, int64_t N) {
+__global__ void dense_stats_kernel(int32_t* cnt, float* mass, float* thr, int P, int Hr, const SeqPos lens) {
   const int p = blockIdx.x * blockDim.x + threadIdx.x;
   if (p < P) {
-    cnt[p] = (int32_t)N;
+    cnt[p] = lens.v[p / Hr];
     mass[p] = 1.0f;
     thr[p] = 0.0f;
   }
 }
 
-// dst[r][i] = i for i < min(n, cap): the selected list of a p == 1 step.
-__global__ void iota_rows_kernel(int32_t* dst, int64_t cap, int64_t n) {
+// dst[r][i] = i for i < min(n_r, cap), n_r the length of row r's sequence: the selected list of
+// a p == 1 step.
+__global__ void iota_rows_kernel(int32_t* dst, int64_t cap, int Hr, const SeqPos lens) {
+  const int64_t n = lens.v[blockIdx.y / Hr];
   const int64_t w = n < cap ? n : cap;
   int32_t* row = dst + (int64_t)blockIdx.y * cap;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < w; i += (int64_t)gridDim.x * blockDim.x)
@@ -269,14 +272,14 @@ __global__ void iota_rows_kernel(int32_t* dst, int64_t cap, int64_t n) {
 
 }  // namespace
 
-cudaError_t launch_iota_rows(int32_t* dst, int64_t cap, int rows, int64_t n, cudaStream_t st) {
-  iota_rows_kernel<<<dim3(64, rows), 256, 0, st>>>(dst, cap, n);
+cudaError_t launch_iota_rows(const rtp_layer* L, int32_t* dst, int64_t cap, cudaStream_t st) {
+  iota_rows_kernel<<<dim3(64, L->B * L->Hr), 256, 0, st>>>(dst, cap, L->Hr, seq_pos(L, 0));
   return cudaGetLastError();
 }
 
 cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st) {
   const int P = L->B * L->Hr;
-  dense_stats_kernel<<<(P + 127) / 128, 128, 0, st>>>(L->sel_cnt, L->sel_mass, L->sel_thr, P, L->len);
+  dense_stats_kernel<<<(P + 127) / 128, 128, 0, st>>>(L->sel_cnt, L->sel_mass, L->sel_thr, P, L->Hr, seq_pos(L, 0));
   return cudaGetLastError();
 }
 
@@ -296,7 +299,7 @@ cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, float* out, cud
   a.ret_head = L->d_ret_head;
   a.P = L->B * L->Hr;
   a.dense = dense ? 1 : 0;
-  a.N = L->len;
+  a.lens = seq_pos(L, 0);
   a.scale_log2 = L->sm_scale * 1.4426950408889634f;
   a.part = L->gpart;
   a.ticket = L->gticket;

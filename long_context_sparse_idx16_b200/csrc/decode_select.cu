@@ -92,6 +92,9 @@ struct SelectArgs {
   int64_t Lp;  // keys per CTA pair (virtual indices 2k, 2k + 1) ...
   int64_t Le;  // ... of which the even member takes the first Le
   int use_smid;  // 1: the virtual index of a CTA is its SM (one CTA on every SM)
+  int Hr;        // retrieval heads: problem p belongs to sequence p / Hr
+  SeqPos lens;   // each sequence's length; problems span N = the longest, keys past a
+                 // sequence's length score -inf (never counted, never selected)
   int sc_bits;
   float top_p;
   int32_t* sel_idx;
@@ -587,6 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   for (int si = 0; si < nseg; ++si) {
     const Seg s = S.seg[si];
     const int64_t rows = s.jhi - s.jlo;
+    // keys of the segment inside its sequence (a shorter sequence of a ragged batch)
+    const int64_t valid = max((int64_t)0, min(rows, (int64_t)a.lens.v[s.p / a.Hr] - s.jlo));
     const float4* src = kBf16 ? reinterpret_cast<const float4*>(a.idx_b + (int64_t)s.p * a.idx_pstride) + s.jlo * 2
                               : reinterpret_cast<const float4*>(a.idx + (int64_t)s.p * a.idx_pstride) + s.jlo * 4;
     float qv[kBf16 ? 8 : 4];
@@ -610,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int64_t k = k0 + u * kKeysIt;
-        v[u] = k < rows ? ld_stream_f4(src + k * kPer + part) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u] = k < valid ? ld_stream_f4(src + k * kPer + part) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
@@ -638,6 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
         d += 0.0f;  // -0 -> +0: equal scores must get equal order keys
         const int64_t k = k0 + u * kKeysIt;
         if (k < rows) {
+          if (k >= valid) d = -INFINITY;
           mx = fmaxf(mx, d);
           if (part == 0) sc[s.off + k] = d;
         }
@@ -1204,6 +1210,8 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   a.Lp = g.pair;
   a.Le = g.even;
   a.use_smid = 0;
+  a.Hr = L->Hr;
+  a.lens = seq_pos(L, 0);
   int lg = 0;
   while ((1ll << lg) < N) ++lg;
   a.sc_bits = 62 - lg;

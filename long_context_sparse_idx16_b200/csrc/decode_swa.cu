@@ -36,10 +36,10 @@ struct SwaArgs {
   const float* q_rot;        // [B][Hq][D]
   const int16_t* loc_head;   // [Hkv][16]
   const int32_t* loc_cnt;    // [Hkv]
-  int64_t N;                 // keys in cache; query at N-1
-  int64_t s_cnt, w0;         // sinks [0, s_cnt), window [w0, N)
-  int64_t nJ;
-  int64_t chunk_keys;
+  SeqPos lens;               // each sequence's length N_b; its query sits at N_b - 1
+  int64_t W, S;              // window and sinks: keys [0, min(S, N_b)) and [max(.., N_b - W), N_b)
+  int64_t chunk_keys;        // keys per chunk (chunks of the longest key set; a shorter
+                             // sequence's later chunks are empty)
   int n_chunks;
   float scale_log2;
   float* part;  // [B][Hkv][n_chunks][16][D+2]
@@ -105,8 +105,13 @@ __global__ void __launch_bounds__(kThreads) decode_swa_kernel(SwaArgs a) {
 
   const __half* kb = a.kc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
   const __half* vb = a.vc + ((int64_t)b * a.Hkv + g) * a.max_seq * kD;
+  // this sequence's key set J = [0, s_cnt) U [w0, N_b), enumerated by u = 0 .. nJ - 1
+  const int64_t Nb = a.lens.v[b];
+  const int64_t s_cnt = min(a.S, Nb);
+  const int64_t w0 = max(s_cnt, Nb - a.W);
+  const int64_t nJ = s_cnt + (Nb - w0);
   const int64_t u_lo = (int64_t)chunk * a.chunk_keys;
-  const int64_t u_hi = min(a.nJ, u_lo + a.chunk_keys);
+  const int64_t u_hi = min(nJ, u_lo + a.chunk_keys);
 
   for (int64_t t0 = u_lo; t0 < u_hi; t0 += kTile) {
     const int64_t wbase = t0 + warp * kWarpKeys;
@@ -117,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) decode_swa_kernel(SwaArgs a) {
       const int r = idx >> 4, ch = idx & 15;
       const int64_t u = wbase + r;
       const bool ok = u < u_hi;
-      const int64_t pos = u < a.s_cnt ? u : a.w0 + (u - a.s_cnt);
+      const int64_t pos = u < s_cnt ? u : w0 + (u - s_cnt);
       const int64_t safe = ok ? pos : 0;
       cp_async16(ksm + swz(r, ch), kb + safe * kD + ch * 8, ok ? 16 : 0);
       cp_async16(vsm + swz(r, ch), vb + safe * kD + ch * 8, ok ? 16 : 0);
@@ -349,14 +354,18 @@ cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st) {
   a.q_rot = L->q_rot;
   a.loc_head = L->d_loc_head;
   a.loc_cnt = L->d_loc_cnt;
-  a.N = L->len;
-  const int64_t i = L->len - 1;
-  a.s_cnt = L->S < L->len ? L->S : L->len;
-  int64_t w0 = i - L->W + 1;
-  if (w0 < a.s_cnt) w0 = a.s_cnt;
-  a.w0 = w0;
-  a.nJ = a.s_cnt + (L->len - w0);
-  swa_chunks(L, a.nJ, &a.chunk_keys, &a.n_chunks);
+  a.lens = seq_pos(L, 0);
+  a.W = L->W;
+  a.S = L->S;
+  // chunking of the longest sequence's key set (at most S + W keys)
+  int64_t nJ_max = 0;
+  for (int b = 0; b < L->B; ++b) {
+    const int64_t n = L->lens[b], sc = L->S < n ? L->S : n;
+    const int64_t w0 = n - L->W > sc ? n - L->W : sc;
+    const int64_t nj = sc + (n - w0);
+    nJ_max = nj > nJ_max ? nj : nJ_max;
+  }
+  swa_chunks(L, nJ_max, &a.chunk_keys, &a.n_chunks);
   if ((int64_t)L->B * L->Hkv * a.n_chunks * kMaxGroup * (kD + 2) > L->spart_elems) return cudaErrorInvalidValue;
   a.scale_log2 = L->sm_scale * 1.4426950408889634f;
   a.part = L->spart;

@@ -34,8 +34,9 @@ struct TopkArgs {
   const __nv_bfloat16* idx_b;   // bf16 index keys
   int64_t idx_pstride;
   const float* q_idx;           // [P][r]
-  int P;
-  int64_t N, k;
+  int P, Hr;
+  SeqPos lens;  // each sequence's length: problem p sees keys 0 .. lens[p / Hr] - 1
+  int64_t k;
   int nchunks;
   uint32_t* keys;               // [P][max_seq] order keys of the scores
   int64_t keys_pstride;
@@ -51,8 +52,10 @@ struct TopkArgs {
 
 // Digits fixed by the first `levels` levels of problem p, and how many keys are still needed
 // among the keys that match them (counted from the highest key down).
+__device__ __forceinline__ int64_t nkeys(const TopkArgs& a, int p) { return a.lens.v[p / a.Hr]; }
+
 __device__ void topk_state(const TopkArgs& a, int p, int levels, uint32_t* prefix, uint32_t* mask, int64_t* rem) {
-  int64_t need = min(a.k, a.N);
+  int64_t need = min(a.k, nkeys(a, p));
   uint32_t pre = 0u, msk = 0u;
   for (int l = 0; l < levels; ++l) {
     const uint32_t* h = a.hist + ((int64_t)p * kTkLevels + l) * 256;
@@ -86,7 +89,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_score_kernel(TopkArgs a) {
 #pragma unroll 4
   for (int u = 0; u < kTkPer; ++u) {
     const int64_t j = j0 + u * kTkThreads + tid;
-    if (j >= a.N) break;
+    if (j >= nkeys(a, p)) break;
     float s;
     if constexpr (kBf16) {
       const uint4* row = reinterpret_cast<const uint4*>(a.idx_b + (int64_t)p * a.idx_pstride + j * kR);
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_hist_kernel(TopkArgs a, int l
 #pragma unroll 4
   for (int u = 0; u < kTkPer; ++u) {
     const int64_t j = j0 + u * kTkThreads + tid;
-    if (j >= a.N) break;
+    if (j >= nkeys(a, p)) break;
     const uint32_t key = keys[j];
     if ((key & msk) == pre) atomicAdd(&h[(key >> sh) & 0xFFu], 1u);
   }
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_count_kernel(TopkArgs a) {
   uint32_t above = 0u, eq = 0u;
   for (int u = 0; u < kTkPer; ++u) {
     const int64_t j = j0 + u * kTkThreads + tid;
-    if (j >= a.N) break;
+    if (j >= nkeys(a, p)) break;
     const uint32_t key = keys[j];
     above += key > t ? 1u : 0u;
     eq += key == t ? 1u : 0u;
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_write_kernel(TopkArgs a) {
     s_before = before;
     s_eqbefore = eqb;
     if (c == a.nchunks - 1) {
-      const int64_t K = min(a.k, a.N);
+      const int64_t K = min(a.k, nkeys(a, p));
       if (K > a.max_select) atomicOr(a.err, kErrOverflow);
       a.sel_cnt[p] = (int32_t)(K < a.max_select ? K : a.max_select);
       if (a.sel_mass) a.sel_mass[p] = -1.f;  // the fixed budget does not sum masses
@@ -263,8 +266,8 @@ __global__ void __launch_bounds__(kTkThreads) topk_write_kernel(TopkArgs a) {
 #pragma unroll
   for (int i = 0; i < kTkPer; ++i) {
     const int64_t j = j0 + i;
-    kv[i] = j < a.N ? keys[j] : 0u;
-    const bool in = j < a.N;
+    const bool in = j < nkeys(a, p);
+    kv[i] = in ? keys[j] : 0u;
     above += (in && kv[i] > t) ? 1u : 0u;
     eq += (in && kv[i] == t) ? 1u : 0u;
   }
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(kTkThreads) topk_write_kernel(TopkArgs a) {
 #pragma unroll
   for (int i = 0; i < kTkPer; ++i) {
     const int64_t j = j0 + i;
-    if (j >= a.N) break;
+    if (j >= nkeys(a, p)) break;
     bool sel = kv[i] > t;
     if (kv[i] == t) {
       sel = tie_rank < need;
@@ -305,7 +308,8 @@ cudaError_t launch_decode_topk(rtp_layer* L, cudaStream_t st) {
   a.idx_pstride = L->max_seq * kR;
   a.q_idx = L->q_idx;
   a.P = L->B * L->Hr;
-  a.N = L->len;
+  a.Hr = L->Hr;
+  a.lens = seq_pos(L, 0);
   a.k = L->top_k;
   a.nchunks = (int)((L->len + kTopkChunk - 1) / kTopkChunk);
   a.keys = L->tk_keys;

@@ -56,7 +56,7 @@ struct LocalTcArgs {
   const __half* vc;
   int64_t max_seq;
   int Hkv, Hq, group, C;
-  int64_t P0;
+  SeqPos P0;  // per sequence: position of chunk row 0
   int W, S;
   const int16_t* local_heads;
   const float* q_rot;  // [B][C][Hq][D]
@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kThreadsT, 2) prefill_local_tc_kernel(LocalTcA
   const int h = a.local_heads[blockIdx.y], g = h / a.group;
   const int i0 = tile * kRowsT;
   const int nrows = min(kRowsT, a.C - i0);
-  const int64_t pos_min = a.P0 + i0, pos_max = pos_min + nrows - 1;
+  const int64_t pos_min = (int64_t)a.P0.v[b] + i0, pos_max = pos_min + nrows - 1;
   const int64_t s_cnt = min((int64_t)a.S, pos_max + 1);
   int64_t w_lo = pos_min - a.W + 1;
   if (w_lo < s_cnt) w_lo = s_cnt;
@@ -368,7 +368,7 @@ static cudaError_t launch_prefill_heads(const rtp_layer* L, int C, float* out, c
   a.Hq = L->Hq;
   a.group = L->group;
   a.C = C;
-  a.P0 = L->len - C;
+  a.P0 = seq_pos(L, -C);
   a.W = W;
   a.S = S;
   a.local_heads = heads;

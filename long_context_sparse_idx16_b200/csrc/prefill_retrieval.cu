@@ -57,7 +57,7 @@ enum : int { kModeKeys = 1, kModeTie = 2, kModeDone = 3 };
 struct RetArgs {
   int64_t max_seq;
   int Hkv, Hq, Hr, group, C;
-  int64_t P0;
+  SeqPos P0;                  // per sequence: position of chunk row 0 (its length - C)
   float top_p;
   int64_t top_k;              // > 0: fixed budget (counts instead of masses)
   int sc_bits;                // fixed-point scale of the selection masses (62 - ceil(log2 len))
@@ -246,8 +246,9 @@ __global__ void __launch_bounds__(kPsThreads, 6) prefill_select_kernel(RetArgs a
   const int i0 = tile * kRowsR;
   const int nrows = min(kRowsR, a.C - i0);
   const bool live = tid < nrows;
-  const int64_t pos = live ? a.P0 + i0 + tid : -1;
-  const int64_t nkeys = a.P0 + i0 + nrows;
+  const int64_t P0 = a.P0.v[b];
+  const int64_t pos = live ? P0 + i0 + tid : -1;
+  const int64_t nkeys = P0 + i0 + nrows;
   const int64_t ntiles = (nkeys + kKeysR - 1) / kKeysR;
   const float scale = __uint_as_float((uint32_t)(127 + a.sc_bits) << 23);  // 2^sc_bits
   uint2* cut = a.cut + ((int64_t)b * a.Hr + hr) * a.C + i0;
@@ -597,8 +598,9 @@ __global__ void __launch_bounds__(kAttThreads, 2) prefill_attn_kernel(RetArgs a,
   const int i0 = tile * kRowsR;
   const int nrows = min(kRowsR, a.C - i0);
   const bool live = r < nrows;
-  const int64_t pos = live ? a.P0 + i0 + r : -1;
-  const int64_t nkeys = a.P0 + i0 + nrows;
+  const int64_t P0 = a.P0.v[b];
+  const int64_t pos = live ? P0 + i0 + r : -1;
+  const int64_t nkeys = P0 + i0 + nrows;
   const int64_t nt = (nkeys + kKeysR - 1) / kKeysR;
   const int64_t tb = (int64_t)split * a.attn_split_tiles;
   const int64_t ntl = max((int64_t)0, min(nt, tb + a.attn_split_tiles) - tb);
@@ -985,7 +987,7 @@ cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_
   a.Hr = L->Hr;
   a.group = L->group;
   a.C = C;
-  a.P0 = L->len - C;
+  a.P0 = seq_pos(L, -C);
   a.top_p = L->top_p;
   a.top_k = L->top_k;
   int lg = 0;

@@ -42,6 +42,13 @@ constexpr int kAttSplitTiles = 4096;
 // Fixed top-k decode selection (ablation mode): keys per chunk of its radix-select kernels.
 constexpr int kTopkChunk = 4096;
 
+// Sequences of a layer, and their per-sequence positions passed to kernels by value (a
+// sequence's length, or the position of its first new row).
+constexpr int kMaxBatch = 256;
+struct SeqPos {
+  int32_t v[kMaxBatch];
+};
+
 // Window + sink decode attention: keys per CTA tile and threads.
 constexpr int kSwaTile = 128;
 constexpr int kSwaThreads = 128;
@@ -51,7 +58,9 @@ constexpr int kSwaThreads = 128;
 struct rtp_layer {
   // configuration
   int B = 0, Hq = 0, Hkv = 0, Hr = 0, group = 0;
-  int64_t max_seq = 0, max_select = 0, len = 0;
+  int64_t max_seq = 0, max_select = 0;
+  int64_t len = 0;                 // the longest sequence's length (sizes the launches)
+  std::vector<int64_t> lens;       // [B] each sequence's length (ragged batches)
   int max_chunk = 0;
   float top_p = 0.9f, sm_scale = 0.f;
   double rope_base = 1e6;
@@ -152,9 +161,12 @@ rtp_status fail(rtp_layer* L, rtp_status st, const std::string& msg);
 rtp_status cuda_fail(rtp_layer* L, cudaError_t e, const char* what);
 
 // Kernel launchers (return cudaGetLastError() of the launch).
-cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T,
-                             cudaStream_t st);
-cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, int64_t pos0,
+// per-sequence lengths plus delta (a sequence's decode row: delta -1; first prefill row: -C)
+SeqPos seq_pos(const rtp_layer* L, int64_t delta);
+// append T tokens to sequences b0 .. b0 + nb - 1 (k, v: [nb][T][Hkv][D]) at their own lengths
+cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const __nv_bfloat16* v, int T, int b0,
+                             int nb, cudaStream_t st);
+cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, const SeqPos& pos0,
                           cudaStream_t st);
 cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st);
 cudaError_t launch_decode_topk(rtp_layer* L, cudaStream_t st);
@@ -162,7 +174,7 @@ cudaError_t launch_prefill_dense_retrieval(const rtp_layer* L, int C, float* out
 cudaError_t launch_prefill_dense_stats(const rtp_layer* L, int C, int32_t* cnt, float* mass, cudaStream_t st);
 cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, float* out, cudaStream_t st);
 cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st);
-cudaError_t launch_iota_rows(int32_t* dst, int64_t cap, int rows, int64_t n, cudaStream_t st);
+cudaError_t launch_iota_rows(const rtp_layer* L, int32_t* dst, int64_t cap, cudaStream_t st);
 cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st);
 cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStream_t st);
 cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,

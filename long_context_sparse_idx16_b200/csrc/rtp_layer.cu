@@ -111,19 +111,20 @@ static void free_all(rtp_layer* L) {
 
 namespace rtp {
 namespace {
-// With dense retrieval prefill row i (position P0 + i) keeps all its P0 + i + 1 causal keys.
-__global__ void prefill_dense_stats_kernel(int32_t* cnt, float* mass, int C, int Hr, int64_t P0, int64_t n) {
+// With dense retrieval prefill row i of sequence b (position P0_b + i) keeps all its
+// P0_b + i + 1 causal keys.
+__global__ void prefill_dense_stats_kernel(int32_t* cnt, float* mass, int C, int Hr, const SeqPos P0, int64_t n) {
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= n) return;
-  const int64_t i = (t / Hr) % C;
-  if (cnt) cnt[t] = (int32_t)(P0 + i + 1);
+  const int64_t i = (t / Hr) % C, b = t / ((int64_t)Hr * C);
+  if (cnt) cnt[t] = (int32_t)(P0.v[b] + i + 1);
   if (mass) mass[t] = 1.f;
 }
 }  // namespace
 
 cudaError_t launch_prefill_dense_stats(const rtp_layer* L, int C, int32_t* cnt, float* mass, cudaStream_t st) {
   const int64_t n = (int64_t)L->B * C * L->Hr;
-  prefill_dense_stats_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cnt, mass, C, L->Hr, L->len - C, n);
+  prefill_dense_stats_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cnt, mass, C, L->Hr, seq_pos(L, -C), n);
   return cudaGetLastError();
 }
 }  // namespace rtp
@@ -138,6 +139,7 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   const rtp_config& c = *cfg;
   if (c.batch < 1 || c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads != 0)
     return fail(nullptr, RTP_EINVAL, "rtp_create: need batch >= 1 and n_kv_heads dividing n_q_heads");
+  if (c.batch > kMaxBatch) return fail(nullptr, RTP_EINVAL, "rtp_create: at most 256 sequences");
   if (c.head_dim != kD || c.index_dim != kR)
     return fail(nullptr, RTP_EINVAL, "rtp_create: head_dim must be 128 and index_dim 16");
   if (c.n_q_heads / c.n_kv_heads > kMaxGroup)
@@ -159,6 +161,7 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
 
   rtp_layer* L = new rtp_layer();
   L->B = c.batch;
+  L->lens.assign((size_t)c.batch, 0);
   L->Hq = c.n_q_heads;
   L->Hkv = c.n_kv_heads;
   L->group = c.n_q_heads / c.n_kv_heads;
@@ -354,6 +357,19 @@ rtp_status rtp_destroy(rtp_layer* L) {
   return RTP_OK;
 }
 
+namespace {
+void update_len(rtp_layer* L) {
+  int64_t mx = 0;
+  for (int64_t n : L->lens) mx = n > mx ? n : mx;
+  L->len = mx;
+}
+int64_t min_len(const rtp_layer* L) {
+  int64_t mn = L->lens.empty() ? 0 : L->lens[0];
+  for (int64_t n : L->lens) mn = n < mn ? n : mn;
+  return mn;
+}
+}  // namespace
+
 rtp_status rtp_append_kv(rtp_layer* L, const void* k, const void* v, int32_t T, cudaStream_t stream) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_append_kv: layer is NULL");
   if (!k || !v) return fail(L, RTP_EINVAL, "rtp_append_kv: k or v is NULL");
@@ -362,10 +378,30 @@ rtp_status rtp_append_kv(rtp_layer* L, const void* k, const void* v, int32_t T, 
   cudaError_t e;
   {
     ProfScope ps(L, "append_kv", stream);
-    e = launch_append_kv(L, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, T, stream);
+    e = launch_append_kv(L, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, T, 0, L->B, stream);
   }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_append_kv: launch");
-  L->len += T;
+  for (int64_t& n : L->lens) n += T;
+  update_len(L);
+  L->last_error.clear();
+  return RTP_OK;
+}
+
+rtp_status rtp_append_kv_seq(rtp_layer* L, int32_t b, const void* k, const void* v, int32_t T,
+                             cudaStream_t stream) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_append_kv_seq: layer is NULL");
+  if (b < 0 || b >= L->B) return fail(L, RTP_EINVAL, "rtp_append_kv_seq: sequence index out of range");
+  if (!k || !v) return fail(L, RTP_EINVAL, "rtp_append_kv_seq: k or v is NULL");
+  if (T < 1) return fail(L, RTP_EINVAL, "rtp_append_kv_seq: T must be >= 1");
+  if (L->lens[b] + T > L->max_seq) return fail(L, RTP_ECAPACITY, "rtp_append_kv_seq: max_seq exceeded");
+  cudaError_t e;
+  {
+    ProfScope ps(L, "append_kv", stream);
+    e = launch_append_kv(L, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, T, b, 1, stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(L, e, "rtp_append_kv_seq: launch");
+  L->lens[b] += T;
+  update_len(L);
   L->last_error.clear();
   return RTP_OK;
 }
@@ -373,11 +409,11 @@ rtp_status rtp_append_kv(rtp_layer* L, const void* k, const void* v, int32_t T, 
 rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_stats* stats, cudaStream_t stream) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_decode: layer is NULL");
   if (!q || !out) return fail(L, RTP_EINVAL, "rtp_decode: q or out is NULL");
-  if (L->len < 1) return fail(L, RTP_EINVAL, "rtp_decode: the cache is empty (append the token first)");
+  if (min_len(L) < 1) return fail(L, RTP_EINVAL, "rtp_decode: a sequence is empty (append its token first)");
   cudaError_t e;
   {
     ProfScope ps(L, "q_prep", stream);
-    e = launch_q_prep(L, (const __nv_bfloat16*)q, 1, L->len - 1, stream);
+    e = launch_q_prep(L, (const __nv_bfloat16*)q, 1, seq_pos(L, -1), stream);
   }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: q_prep");
   bool forked = false;
@@ -417,7 +453,7 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
         e = cudaMemcpyAsync(stats->threshold, L->sel_thr, P * 4, cudaMemcpyDeviceToDevice, stream);
       if (e == cudaSuccess && stats->sel_index && stats->sel_index_cap > 0) {
         if (dense) {
-          e = launch_iota_rows(stats->sel_index, stats->sel_index_cap, (int)P, L->len, stream);
+          e = launch_iota_rows(L, stats->sel_index, stats->sel_index_cap, stream);
         } else {
           const int64_t w = stats->sel_index_cap < L->max_select ? stats->sel_index_cap : L->max_select;
           e = cudaMemcpy2DAsync(stats->sel_index, (size_t)stats->sel_index_cap * 4, L->sel_idx,
@@ -445,8 +481,8 @@ rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out,
                              cudaStream_t stream) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_prefill_chunk: layer is NULL");
   if (!q || !out) return fail(L, RTP_EINVAL, "rtp_prefill_chunk: q or out is NULL");
-  if (C < 1 || C > L->max_chunk || C > L->len)
-    return fail(L, RTP_EINVAL, "rtp_prefill_chunk: need 1 <= C <= min(len, max_chunk)");
+  if (C < 1 || C > L->max_chunk || C > min_len(L))
+    return fail(L, RTP_EINVAL, "rtp_prefill_chunk: need 1 <= C <= min(shortest length, max_chunk)");
   if (stats && stats->sel_bitmap && stats->bitmap_words < 1)
     return fail(L, RTP_EINVAL, "rtp_prefill_chunk: sel_bitmap needs bitmap_words >= 1");
   if (stats && stats->rows &&
@@ -458,7 +494,7 @@ rtp_status rtp_prefill_chunk(rtp_layer* L, const void* q, int32_t C, float* out,
   cudaError_t e;
   {
     ProfScope ps(L, "q_prep", stream);
-    e = launch_q_prep(L, (const __nv_bfloat16*)q, C, L->len - C, stream);
+    e = launch_q_prep(L, (const __nv_bfloat16*)q, C, seq_pos(L, -C), stream);
   }
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_prefill_chunk: q_prep");
   // with both head classes, the local heads run on the internal stream (forked after q_prep,
@@ -515,10 +551,23 @@ rtp_status rtp_set_wait_limit(rtp_layer* L, int64_t cycles) {
 
 int64_t rtp_seq_len(const rtp_layer* L) { return L ? L->len : -1; }
 
+int64_t rtp_seq_len_of(const rtp_layer* L, int32_t b) { return (L && b >= 0 && b < L->B) ? L->lens[b] : -1; }
+
 rtp_status rtp_truncate(rtp_layer* L, int64_t new_len) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_truncate: layer is NULL");
   if (new_len < 0 || new_len > L->len) return fail(L, RTP_EINVAL, "rtp_truncate: need 0 <= new_len <= length");
-  L->len = new_len;
+  for (int64_t& n : L->lens) n = n < new_len ? n : new_len;
+  update_len(L);
+  return RTP_OK;
+}
+
+rtp_status rtp_truncate_seq(rtp_layer* L, int32_t b, int64_t new_len) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_truncate_seq: layer is NULL");
+  if (b < 0 || b >= L->B) return fail(L, RTP_EINVAL, "rtp_truncate_seq: sequence index out of range");
+  if (new_len < 0 || new_len > L->lens[b])
+    return fail(L, RTP_EINVAL, "rtp_truncate_seq: need 0 <= new_len <= the sequence's length");
+  L->lens[b] = new_len;
+  update_len(L);
   return RTP_OK;
 }
 
@@ -556,6 +605,7 @@ rtp_status rtp_profile_read(rtp_layer* L, const char* kernel, double* total_ms, 
 
 rtp_status rtp_reset(rtp_layer* L) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_reset: layer is NULL");
+  for (int64_t& n : L->lens) n = 0;
   L->len = 0;
   return RTP_OK;
 }

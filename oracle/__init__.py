@@ -206,17 +206,19 @@ def layer_rows(inputs, b: int, h: int, rows: Sequence[int], *, top_p: Optional[f
         want_pi=want_pi, threads=threads, pos_offset=pos_offset, index_bf16=s.index_bf16)
 
 
-def attend_set(inputs, b: int, h: int, row: int, sel: Sequence[int], *, pos_offset: int = 0) -> np.ndarray:
+def attend_set(inputs, b: int, h: int, row: int, sel: Sequence[int], *, pos_offset: int = 0,
+               pos: Optional[int] = None) -> np.ndarray:
     """Exact attention of chunk row ``row`` of query head h (sequence b) over the key set ``sel``
     (no selection step): for checking an output whose set legitimately differs from the
-    oracle's own."""
+    oracle's own.  pos: the row's position when it is not prefix + row (a sequence of a ragged
+    batch)."""
     s = inputs.spec
     k_seq = np.ascontiguousarray(inputs.k[b], dtype=np.uint16)
     v_seq = np.ascontiguousarray(inputs.v[b], dtype=np.uint16)
     N, Hkv, D = k_seq.shape
     q = np.ascontiguousarray(inputs.q[b, row, h], dtype=np.uint16)
     J = np.ascontiguousarray(np.asarray(sel, dtype=np.int64))
-    pos = s.prefix + int(row)
+    pos = s.prefix + int(row) if pos is None else int(pos)
     if J.size and (J.min() < 0 or J.max() > pos):
         raise ValueError("attend_set: a key lies outside the row's causal range")
     out = np.zeros(D, dtype=np.float64)
