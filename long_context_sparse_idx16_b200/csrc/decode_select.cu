@@ -609,16 +609,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     float mx = -INFINITY;
     // The trip count is the same for every thread (the shuffles below are full-warp);
     // rows past the end are loaded as zeros and not stored.
-    for (int64_t base = 0; base < rows; base += kUnroll * kKeysIt) {
+    // bf16 keys: four 16-byte loads in flight per thread (eight, with the bf16 unpacking, spill
+    // out of the 64 registers a thread has, which cost a third of the stream's speed)
+    constexpr int kU = kBf16 ? 4 : kUnroll;
+    for (int64_t base = 0; base < rows; base += kU * kKeysIt) {
       const int64_t k0 = base + quad;
-      float4 v[kUnroll];
+      float4 v[kU];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kU; ++u) {
         const int64_t k = k0 + u * kKeysIt;
         v[u] = k < valid ? ld_stream_f4(src + k * kPer + part) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kU; ++u) {
         float d;
         if constexpr (kBf16) {  // eight bf16 components
           const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
@@ -673,7 +676,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     if (tid == 0) S.seg[si].m = m;
     __syncthreads();
     const int off = (int)S.seg[si].off, rows = (int)(S.seg[si].jhi - S.seg[si].jlo);
-    const int jlo = (int)S.seg[si].jlo;
     const int wlen = (rows + kWarps - 1) / kWarps;
     const int w_lo = min(rows, warp * wlen), w_hi = min(rows, w_lo + wlen);
     const int kcap = S.seg[si].kcap;
