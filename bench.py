@@ -69,14 +69,14 @@ MUFU_EX2_PER_CLK_SM = 16
 
 
 def _prefill_traffic(kernel: str, workload: str):
-    """Per-launch DRAM bytes of the prefill retrieval kernels at the 32K chunk, from the
-    committed ncu summary, while their sources are unchanged since the capture (else None).
-    The 1M chunk has no capture whose bytes would scale: the 32K index keys sit in L2, the 1M
-    ones do not."""
-    if kernel not in ("prefill_select", "prefill_attn") or workload != "prefill_32k":
+    """Per-launch DRAM bytes of the prefill retrieval kernels at the 32K and the 1M chunk, from
+    the committed ncu summaries (each captured on its own workload), while their sources are
+    unchanged since the capture (else None)."""
+    files = {"prefill_32k": "prefill_kernels_32k.md", "prefill_1m": "prefill_kernels_1m.md"}
+    if kernel not in ("prefill_select", "prefill_attn") or workload not in files:
         return None
     try:
-        text = open(os.path.join(ROOT, "profiles", "prefill_kernels_32k.md")).read()
+        text = open(os.path.join(ROOT, "profiles", files[workload])).read()
     except OSError:
         return None
     traffic, srcs = None, None

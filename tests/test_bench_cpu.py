@@ -118,5 +118,7 @@ def test_prefill_traffic_only_for_the_captured_kernel_and_chunk():
     assert t is None or t == 623752704.0
     t = bench._prefill_traffic("prefill_attn", "prefill_32k")
     assert t is None or t == 245485056.0
-    assert bench._prefill_traffic("prefill_select", "prefill_1m") is None
+    t = bench._prefill_traffic("prefill_select", "prefill_1m")
+    assert t is None or t == 61888269824.0
+    assert bench._prefill_traffic("prefill_select", "decode_1m") is None
     assert bench._prefill_traffic("prefill_local", "prefill_32k") is None
