@@ -46,6 +46,14 @@ def lib():
         L.orc_attend_set.argtypes = [P, P, i64, i32, i32, P, i64, f64, f64, i64, P, i64, P]
         L.orc_max_threads.restype = C.c_int
         L.orc_max_threads.argtypes = []
+        L.orc_index_keys_bf16.restype = None
+        L.orc_index_keys_bf16.argtypes = [P, i64, i64, i32, i32, i32, P, P]
+        L.orc_index_query.restype = None
+        L.orc_index_query.argtypes = [P, i32, i32, P, P]
+        L.orc_kmeans.restype = None
+        L.orc_kmeans.argtypes = [P, i64, i32, i32, i32, P, P, P]
+        L.orc_cluster_select.restype = C.c_int
+        L.orc_cluster_select.argtypes = [P, P, P, i32, i32, f64, P, P, P]
         _lib = L
     return _lib
 
@@ -225,3 +233,82 @@ def attend_set(inputs, b: int, h: int, row: int, sel: Sequence[int], *, pos_offs
     lib().orc_attend_set(_p(k_seq), _p(v_seq), Hkv * D, s.kv_head(h), D, _p(q), pos, float(s.rope_base),
                          1.0 / np.sqrt(D), int(pos_offset), _p(J), int(J.size), _p(out))
     return out
+
+
+# ------------------------------------------------------------------ K-cache clustering
+
+
+def index_keys_bf16(k_seq: np.ndarray, g: int, wk: np.ndarray, n: Optional[int] = None) -> np.ndarray:
+    """Stored bf16 index keys kt_j = bf16(Wk^T k_j) of KV head g for j < n, fp64 [n][r]."""
+    k_seq = np.ascontiguousarray(k_seq, dtype=np.uint16)
+    N, Hkv, D = k_seq.shape
+    n = N if n is None else n
+    wk = np.ascontiguousarray(wk, dtype=np.float32)
+    r = wk.shape[1]
+    kt = np.empty((n, r), dtype=np.float64)
+    lib().orc_index_keys_bf16(_p(k_seq), n, Hkv * D, g, D, r, _p(wk), _p(kt))
+    return kt
+
+
+def index_query(q_vec: np.ndarray, wq: np.ndarray) -> np.ndarray:
+    """Index query Wq^T q of one bf16 query vector, fp64 [r]."""
+    q_vec = np.ascontiguousarray(q_vec, dtype=np.uint16)
+    wq = np.ascontiguousarray(wq, dtype=np.float32)
+    qt = np.empty(wq.shape[1], dtype=np.float64)
+    lib().orc_index_query(_p(q_vec), q_vec.shape[0], wq.shape[1], _p(wq), _p(qt))
+    return qt
+
+
+def kmeans(kt: np.ndarray, K: int, iters: int):
+    """Lloyd's k-means of the index keys kt [n][r] (readings in rtp_oracle.c): (centres [K][r],
+    cluster sizes [K], assignment [n])."""
+    kt = np.ascontiguousarray(kt, dtype=np.float64)
+    n, r = kt.shape
+    cent = np.empty((K, r), dtype=np.float64)
+    counts = np.empty(K, dtype=np.int64)
+    assign = np.empty(n, dtype=np.int32)
+    lib().orc_kmeans(_p(kt), n, r, K, iters, _p(cent), _p(counts), _p(assign))
+    return cent, counts, assign
+
+
+def cluster_select(qt: np.ndarray, cent: np.ndarray, counts: np.ndarray, p: float):
+    """Coarse match of an index query against the centres: (hit [K] bool, weight fractions [K],
+    weight fraction of the last cluster taken)."""
+    qt = np.ascontiguousarray(qt, dtype=np.float64)
+    cent = np.ascontiguousarray(cent, dtype=np.float64)
+    counts = np.ascontiguousarray(counts, dtype=np.int64)
+    K, r = cent.shape
+    hit = np.empty(K, dtype=np.int32)
+    w = np.empty(K, dtype=np.float64)
+    wt = np.zeros(1, dtype=np.float64)
+    lib().orc_cluster_select(_p(qt), _p(cent), _p(counts), K, r, float(p), _p(hit), _p(w), _p(wt))
+    return hit.astype(bool), w, float(wt[0])
+
+
+@dataclass
+class ClusterRow:
+    out: np.ndarray      # [D]
+    sel: np.ndarray      # ascending selected positions
+    hit: np.ndarray      # [K] clusters hit
+    w: np.ndarray        # [K] cluster weight fractions
+    w_t: float           # weight fraction of the last cluster taken
+    cent: np.ndarray
+    counts: np.ndarray
+    assign: np.ndarray
+
+
+def cluster_row(inputs, b: int, h: int, n: int, K: int, iters: int, p: float,
+                n_clustered: Optional[int] = None) -> ClusterRow:
+    """The clustered selection and attention of the decode query of retrieval head h, sequence
+    b, at position n - 1: keys 0 .. n_clustered - 1 clustered, the later ones always kept."""
+    s = inputs.spec
+    slot = s.retrieval_heads.index(h)
+    g = s.kv_head(h)
+    nc = n if n_clustered is None else n_clustered
+    kt = index_keys_bf16(inputs.k[b], g, inputs.wk[slot], nc)
+    cent, counts, assign = kmeans(kt, K, iters)
+    qt = index_query(inputs.q[b, 0, h], inputs.wq[slot])
+    hit, w, wt = cluster_select(qt, cent, counts, p)
+    sel = np.concatenate([np.flatnonzero(hit[assign]), np.arange(nc, n)]).astype(np.int64)
+    out = attend_set(inputs, b, h, 0, sel, pos=n - 1)
+    return ClusterRow(out, sel, hit, w, wt, cent, counts, assign)

@@ -401,6 +401,155 @@ void orc_index_scores(const uint16_t* k, int64_t n, int64_t kv_stride, int g, in
   }
 }
 
+/* ---------------------------------------------------------------- K-cache clustering
+ *
+ * The RTPurboV2 two-level funnel (aitntnews page, finding 3): the N cached tokens of a
+ * retrieval head are grouped into K semantic clusters in the r = 16 index space, a query is
+ * matched against the K cluster centres first, and exact attention then runs only over the
+ * tokens of the clusters it hits.  The page fixes none of the steps; the readings taken here:
+ *   - the clustered vectors are the stored bf16 index keys kt_j (the layer's bf16 option),
+ *     put on the fixed-point grid 2^-27 (xq = rint(kt * 2^27)) so that centre sums are exact
+ *     integers, whatever their order;
+ *   - Lloyd's k-means: centres start at the keys j_k = floor((2k + 1) n / (2K)); each pass
+ *     assigns every key to the centre of least squared distance (fp64, the 16 terms summed
+ *     in dimension order with fused multiply-adds; ties to the lower centre), then moves every
+ *     non-empty centre to the mean of its keys (integer sum / count * 2^-27); an empty
+ *     cluster keeps its centre; a final assignment follows the last pass;
+ *   - the coarse match: centre score c_k = qt . mu_k; a cluster weighs n_k exp(c_k - max c)
+ *     (its key count times the softmax weight of its centre: the mass its keys would carry if
+ *     they sat at the centre); clusters ordered by (c_k desc, k asc), the shortest prefix whose
+ *     weight reaches p of the total is hit (p >= 1: every non-empty cluster);
+ *   - keys cached after the clustering are always kept; the fine step is exact attention over
+ *     the hit clusters' keys and those. */
+
+#define ORC_CL_SCALE 134217728.0 /* 2^27 */
+
+/* kt_j = Wk^T k_j for j < n, each component rounded to bf16 (the stored keys). */
+void orc_index_keys_bf16(const uint16_t* k, int64_t n, int64_t kv_stride, int g, int D, int r,
+                         const float* wk, double* kt) {
+  double x[512];
+  for (int64_t j = 0; j < n; ++j) {
+    const uint16_t* kr = k + j * kv_stride + (int64_t)g * D;
+    for (int d = 0; d < D; ++d) x[d] = orc_bf16(kr[d]);
+    orc_index_vec(x, wk, D, r, kt + j * r);
+    for (int c = 0; c < r; ++c) kt[j * r + c] = orc_round_bf16(kt[j * r + c]);
+  }
+}
+
+static double orc_sqdist(const double* x, const double* mu, int r) {
+  double acc = 0.0;
+  for (int c = 0; c < r; ++c) {
+    const double d = x[c] - mu[c];
+    acc = fma(d, d, acc);
+  }
+  return acc;
+}
+
+/* qt = Wq^T q for one bf16 query (the index query, fp64). */
+void orc_index_query(const uint16_t* q, int D, int r, const float* wq, double* qt) {
+  double qv[512];
+  for (int d = 0; d < D; ++d) qv[d] = orc_bf16(q[d]);
+  orc_index_vec(qv, wq, D, r, qt);
+}
+
+/* Lloyd's k-means of the n keys kt[n][r] into K clusters (K <= n) with `iters` passes.
+ * cent[K][r] receives the centres, counts[K] the cluster sizes and assign[n] each key's
+ * cluster, all after the final assignment. */
+void orc_kmeans(const double* kt, int64_t n, int r, int K, int iters, double* cent, int64_t* counts,
+                int32_t* assign) {
+  double* xq = (double*)malloc(sizeof(double) * (size_t)n * (size_t)r);
+  int64_t* qi = (int64_t*)malloc(sizeof(int64_t) * (size_t)n * (size_t)r);
+  int64_t* sums = (int64_t*)malloc(sizeof(int64_t) * (size_t)K * (size_t)r);
+  for (int64_t i = 0; i < n * r; ++i) {
+    qi[i] = (int64_t)rint(kt[i] * ORC_CL_SCALE);
+    xq[i] = (double)qi[i] / ORC_CL_SCALE;
+  }
+  for (int k = 0; k < K; ++k) {
+    const int64_t j = ((int64_t)(2 * k + 1) * n) / (2 * (int64_t)K);
+    for (int c = 0; c < r; ++c) cent[(int64_t)k * r + c] = xq[j * r + c];
+  }
+  for (int it = 0; it <= iters; ++it) {
+    for (int64_t j = 0; j < n; ++j) {
+      int best = 0;
+      double bd = orc_sqdist(xq + j * r, cent, r);
+      for (int k = 1; k < K; ++k) {
+        const double d = orc_sqdist(xq + j * r, cent + (int64_t)k * r, r);
+        if (d < bd) {
+          bd = d;
+          best = k;
+        }
+      }
+      assign[j] = best;
+    }
+    for (int k = 0; k < K; ++k) counts[k] = 0;
+    for (int64_t i = 0; i < (int64_t)K * r; ++i) sums[i] = 0;
+    for (int64_t j = 0; j < n; ++j) {
+      counts[assign[j]] += 1;
+      for (int c = 0; c < r; ++c) sums[(int64_t)assign[j] * r + c] += qi[j * r + c];
+    }
+    if (it == iters) break; /* the final assignment: centres stay */
+    for (int k = 0; k < K; ++k)
+      if (counts[k] > 0)
+        for (int c = 0; c < r; ++c)
+          cent[(int64_t)k * r + c] = (double)sums[(int64_t)k * r + c] / (double)counts[k] / ORC_CL_SCALE;
+  }
+  free(xq);
+  free(qi);
+  free(sums);
+}
+
+typedef struct {
+  double c;
+  int k;
+} orc_cl;
+
+static int orc_cmp_cl(const void* a, const void* b) {
+  const orc_cl* x = (const orc_cl*)a;
+  const orc_cl* y = (const orc_cl*)b;
+  if (x->c > y->c) return -1;
+  if (x->c < y->c) return 1;
+  return x->k - y->k;
+}
+
+/* The coarse match of one index query qt[r] against K centres: hit[k] = 1 for the clusters
+ * taken.  w[k] (optional) receives each cluster's weight fraction; returns the number hit and
+ * *w_t the weight fraction of the last cluster taken. */
+int orc_cluster_select(const double* qt, const double* cent, const int64_t* counts, int K, int r, double p,
+                       int32_t* hit, double* w, double* w_t) {
+  orc_cl* o = (orc_cl*)malloc(sizeof(orc_cl) * (size_t)K);
+  int m = 0;
+  double cmax = -INFINITY;
+  for (int k = 0; k < K; ++k) {
+    hit[k] = 0;
+    if (w) w[k] = 0.0;
+    if (counts[k] <= 0) continue;
+    double acc = 0.0;
+    for (int c = 0; c < r; ++c) acc += qt[c] * cent[(int64_t)k * r + c];
+    o[m].c = acc;
+    o[m].k = k;
+    if (acc > cmax) cmax = acc;
+    ++m;
+  }
+  double tot = 0.0;
+  for (int i = 0; i < m; ++i) tot += (double)counts[o[i].k] * exp(o[i].c - cmax);
+  qsort(o, (size_t)m, sizeof(orc_cl), orc_cmp_cl);
+  double cum = 0.0, last = 0.0;
+  int taken = 0;
+  for (int i = 0; i < m; ++i) {
+    const double f = (double)counts[o[i].k] * exp(o[i].c - cmax) / tot;
+    if (w) w[o[i].k] = f;
+    if (taken == i && (p >= 1.0 || cum < p)) {
+      hit[o[i].k] = 1;
+      cum += f;
+      last = f;
+      taken = i + 1;
+    }
+  }
+  if (w_t) *w_t = last;
+  free(o);
+  return taken;
+}
+
 int orc_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -468,3 +468,142 @@ def test_topk_ties_and_limits():
     assert np.array_equal(oracle.topk(s, 2).selected, [1, 2])  # the tie at 3 goes to the lower positions
     assert np.array_equal(oracle.topk(s, 4).selected, [1, 2, 3, 4])
     assert oracle.topk(s, 99).count == 5  # k >= n keeps every key
+
+
+# ------------------------------------------------------------------ K-cache clustering
+
+
+def _bf16_keys(n, r=16, seed=0, blobs=None):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((n, r))
+    if blobs is not None:
+        x = x * 0.05 + blobs[rng.integers(0, len(blobs), n)]
+    return np.array([[oracle.round_bf16(v) for v in row] for row in x])
+
+
+def _quantised(kt):
+    return np.rint(kt * 2.0**27) / 2.0**27
+
+
+def test_kmeans_assigns_every_key_to_a_nearest_centre():
+    kt = _bf16_keys(600, seed=1)
+    for K, iters in [(5, 0), (9, 2), (16, 4)]:
+        cent, counts, assign = oracle.kmeans(kt, K, iters)
+        d = ((_quantised(kt)[:, None, :] - cent[None, :, :]) ** 2).sum(-1)
+        best = d.min(1)
+        assert np.all(np.abs(d[np.arange(len(kt)), assign] - best) <= 1e-12 * (1 + best))
+        # ties go to the lower centre: no strictly-lower-index centre is as near
+        for j in range(len(kt)):
+            near = np.flatnonzero(np.abs(d[j] - best[j]) <= 1e-12 * (1 + best[j]))
+            assert assign[j] == near.min()
+        assert counts.sum() == len(kt) and np.array_equal(np.bincount(assign, minlength=K), counts)
+
+
+def test_kmeans_objective_never_increases_over_passes():
+    kt = _bf16_keys(800, seed=2)
+    xq = _quantised(kt)
+    prev = None
+    for iters in range(6):
+        cent, counts, assign = oracle.kmeans(kt, 12, iters)
+        obj = ((xq - cent[assign]) ** 2).sum()
+        if prev is not None:
+            assert obj <= prev * (1 + 1e-12)
+        prev = obj
+
+
+def test_kmeans_closed_forms():
+    kt = _bf16_keys(300, seed=3)
+    xq = _quantised(kt)
+    # one cluster: its centre is the mean of every key (exact on the 2^-27 grid)
+    cent, counts, assign = oracle.kmeans(kt, 1, 3)
+    assert counts.tolist() == [300] and np.all(assign == 0)
+    assert np.allclose(cent[0], xq.mean(0), rtol=0, atol=1e-15)
+    # as many clusters as keys: every key starts as its own centre and stays there
+    cent, counts, assign = oracle.kmeans(kt, 300, 2)
+    assert np.array_equal(assign, np.arange(300)) and np.all(counts == 1)
+    assert np.array_equal(cent, xq)
+    # one pass from the evenly spaced start: the centres are the means of the first assignment
+    cent0, _, assign0 = oracle.kmeans(kt, 7, 0)
+    assert np.array_equal(cent0, xq[[(2 * k + 1) * 300 // 14 for k in range(7)]])
+    cent1, _, _ = oracle.kmeans(kt, 7, 1)
+    for k in range(7):
+        m = assign0 == k
+        assert np.allclose(cent1[k], xq[m].mean(0), rtol=0, atol=1e-15)
+
+
+def test_kmeans_separates_far_blobs():
+    blobs = np.zeros((3, 16))
+    blobs[0, 0], blobs[1, 1], blobs[2, 2] = 40.0, 40.0, 40.0
+    kt = _bf16_keys(450, seed=4, blobs=blobs)
+    cent, counts, assign = oracle.kmeans(kt, 3, 5)
+    near = np.argmax(np.abs(kt[:, :3]), axis=1)  # the blob each key came from
+    # a one-to-one map between clusters and blobs
+    pairs = {(int(a), int(b)) for a, b in zip(assign, near)}
+    assert len(pairs) == 3 and len({a for a, _ in pairs}) == 3
+
+
+def _brute_cluster_hit(qt, cent, counts, p):
+    """Smallest set of clusters, closed upward in centre score (with ties to the lower index),
+    whose weight reaches p of the total: by enumeration of every subset."""
+    import itertools
+
+    K = len(counts)
+    c = cent @ qt
+    live = [k for k in range(K) if counts[k] > 0]
+    cmax = max(c[k] for k in live)
+    wt = {k: counts[k] * np.exp(c[k] - cmax) for k in live}
+    tot = sum(wt.values())
+    best = None
+    for m in range(1, len(live) + 1):
+        for S in itertools.combinations(live, m):
+            Ss = set(S)
+            closed = all(((c[o], -o) <= (c[k], -k)) or (o in Ss) for k in Ss for o in live
+                         if (c[o], -o) > (c[k], -k))
+            if closed and sum(wt[k] for k in S) >= p * tot * (1 - 1e-12):
+                best = Ss
+                break
+        if best is not None:
+            break
+    return best
+
+
+def test_cluster_select_matches_enumeration():
+    rng = np.random.default_rng(5)
+    for trial in range(30):
+        K = int(rng.integers(2, 8))
+        cent = rng.standard_normal((K, 16))
+        counts = rng.integers(0, 50, K).astype(np.int64)
+        counts[rng.integers(0, K)] = 7  # at least one non-empty cluster
+        qt = rng.standard_normal(16)
+        p = float(rng.choice([0.3, 0.5, 0.8, 0.9, 0.99]))
+        hit, w, wt = oracle.cluster_select(qt, cent, counts, p)
+        assert set(np.flatnonzero(hit).tolist()) == _brute_cluster_hit(qt, cent, counts, p)
+        assert np.all(~hit[counts == 0])
+        assert abs(w.sum() - 1.0) < 1e-12 and w[hit].sum() >= p * (1 - 1e-12)
+
+
+def test_cluster_select_limits():
+    cent = np.eye(4, 16)
+    counts = np.array([5, 0, 3, 2], dtype=np.int64)
+    hit, w, _ = oracle.cluster_select(np.zeros(16), cent, counts, 1.0)
+    assert hit.tolist() == [True, False, True, True]  # p = 1: every non-empty cluster
+    # equal centre scores: weights are the sizes, taken in index order
+    hit, w, _ = oracle.cluster_select(np.zeros(16), cent, counts, 0.5)
+    assert hit.tolist() == [True, False, False, False] and np.allclose(w, counts / 10.0)
+    hit, _, _ = oracle.cluster_select(np.zeros(16), cent, counts, 0.6)
+    assert hit.tolist() == [True, False, True, False]
+
+
+def test_cluster_row_single_cluster_is_dense_attention():
+    # one cluster holds every key: the clustered row attends to all of them, as p = 1 does
+    s = synth.spec("toy_decode_4k", prefix=511, index_bf16=True)
+    x = synth.generate(s)
+    n = 512
+    r = oracle.cluster_row(x, 0, 0, n, 1, 2, 0.9)
+    assert np.array_equal(r.sel, np.arange(n))
+    ref = oracle.layer_rows(x, 0, 0, [0], top_p=1.0)
+    assert np.allclose(r.out, ref.out[0], rtol=0, atol=1e-12)
+    # keys cached after the clustering are always kept
+    r2 = oracle.cluster_row(x, 0, 0, n, 16, 2, 0.5, n_clustered=400)
+    assert np.all(np.isin(np.arange(400, n), r2.sel)) and np.all(np.diff(r2.sel) > 0)
+    assert set(r2.sel[r2.sel < 400].tolist()) == set(np.flatnonzero(r2.hit[r2.assign]).tolist())
