@@ -85,14 +85,20 @@ typedef struct {
                                  min(k, n) keys of the order (s desc, j asc) instead -- the
                                  pages' fixed-budget ablation (techwalker page, section 4);
                                  sel_mass and threshold are then reported as -1 */
+  int32_t n_clusters;         /* 0: no clustering.  K in [1, 1024]: the layer can cluster each
+                                 retrieval head's index keys into K clusters (rtp_cluster_build)
+                                 and then select by clusters in decode (RTPurboV2, aitntnews page,
+                                 finding 3).  Needs index_bf16 = 1 and top_k = 0 */
 } rtp_config;
 
 /* Optional decode statistics, DEVICE arrays [B][Hr] (retrieval heads ascending).  Any
  * member may be NULL. */
 typedef struct {
   int32_t* sel_count;  /* |J|, capped at max_select */
-  float* sel_mass;     /* index-softmax mass of J (>= p) */
-  float* threshold;    /* index-softmax mass of the last member of J */
+  float* sel_mass;     /* index-softmax mass of J (>= p); clustered selection: the weight
+                          fraction of the clusters hit (>= p) */
+  float* threshold;    /* index-softmax mass of the last member of J; clustered selection: the
+                          weight fraction of the last cluster taken */
   int32_t* sel_index;  /* [B][Hr][sel_index_cap]: the first min(|J|, cap) positions of J, ascending */
   int64_t sel_index_cap;
 } rtp_decode_stats;
@@ -129,6 +135,17 @@ typedef struct {
   int32_t n_retrieval;
   const void* idx_bf16; /* bf16 [B][Hr][max_seq][r] when the layer stores bf16 index keys, else NULL */
 } rtp_cache_view;
+
+/* Device-side view of a layer's K-cache clustering (read-only use).  P = B * Hr problems,
+ * retrieval heads ascending within a sequence. */
+typedef struct {
+  const double* centres;  /* fp64 [P][K][r] cluster centres in the index space */
+  const int32_t* counts;  /* [P][K] keys per cluster */
+  const uint16_t* assign; /* [P][max_seq] cluster of each clustered key (positions < rtp_cluster_len) */
+  int32_t n_clusters;     /* K (0: the layer cannot cluster) */
+  int32_t ready;          /* 1 while the clustering is in use by decode, else 0 */
+  int64_t max_seq;
+} rtp_cluster_view;
 
 /* Create a layer on the current CUDA device: validates cfg, allocates the caches and all
  * scratch, uploads the weights.  Synchronous.  On success *out receives the layer. */
@@ -198,12 +215,36 @@ rtp_status rtp_truncate(rtp_layer* layer, int64_t new_len);
  * outside [0, len_b]. */
 rtp_status rtp_truncate_seq(rtp_layer* layer, int32_t b, int64_t new_len);
 
+/* K-cache clustering (RTPurboV2, aitntnews page, finding 3: the two-level funnel).  For every
+ * sequence b and retrieval head, clusters the stored bf16 index keys of positions 0 .. len_b - 1
+ * into K = n_clusters clusters by Lloyd's k-means with `iters` passes (0..1000), and records
+ * len_b as the sequence's clustered length.  The keys are taken on the fixed-point grid 2^-27;
+ * centre k starts at key floor((2k+1) len_b / (2K)); each pass assigns every key to the centre
+ * of least squared distance (fp64, ties to the lower centre) and moves every non-empty centre
+ * to its keys' mean; a final assignment follows the last pass.  Every step is deterministic.
+ *
+ * From then on rtp_decode (for p < 1) selects by clusters: centre scores c_k = q~ . mu_k with
+ * the index query q~, cluster weights n_k exp(c_k - max c), clusters taken in (c desc, k asc)
+ * order while the weight before them is below p of the total; the selected set J is every
+ * clustered key of a hit cluster plus every key appended after the clustering, and the
+ * retrieval head attends exactly over J.  Truncating a sequence below its clustered length,
+ * rtp_reset or rtp_cluster_drop ends the clustered selection (decode returns to the per-key
+ * top-p).  RTP_EINVAL (nothing launched) if the layer has no n_clusters or no retrieval heads,
+ * iters is out of range, or some len_b is below K or above 2^21.  An index key of magnitude
+ * >= 2^15 is counted as 0 and reported as RTP_ERANGE by the next rtp_check. */
+rtp_status rtp_cluster_build(rtp_layer* layer, int32_t iters, cudaStream_t stream);
+rtp_status rtp_cluster_drop(rtp_layer* layer);
+/* Clustered length of sequence b (0 when no clustering is in use; -1 for a NULL layer or b
+ * outside [0, B)). */
+int64_t rtp_cluster_len(const rtp_layer* layer, int32_t b);
+rtp_status rtp_get_clusters(const rtp_layer* layer, rtp_cluster_view* view);
+
 /* Per-kernel device timing.  While enabled, the library records a CUDA event pair on the
  * launch stream around every kernel it launches, and runs every kernel on the call's stream
  * in order (no internal fork), so each recorded time belongs to one kernel alone.  rtp_profile_read synchronises on the
  * recorded events, returns the summed device time (ms) and launch count of the named kernel
  * ("append_kv", "q_prep", "decode_select", "decode_topk", "decode_gather", "decode_swa", "swa_merge",
- * "dense_fill", "prefill_*"; NULL: all kernels together), and clears that kernel's record. */
+ * "dense_fill", "cluster_*", "prefill_*"; NULL: all kernels together), and clears that kernel's record. */
 rtp_status rtp_profile_enable(rtp_layer* layer, int on);
 rtp_status rtp_profile_read(rtp_layer* layer, const char* kernel, double* total_ms, int64_t* launches);
 

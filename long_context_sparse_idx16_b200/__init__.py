@@ -33,7 +33,7 @@ class rtp_config(C.Structure):
         ("n_sink", C.c_int32), ("rope_base", C.c_double), ("sm_scale", C.c_float),
         ("wq_index", C.c_void_p), ("wk_index", C.c_void_p), ("max_select", C.c_int64),
         ("max_chunk", C.c_int32), ("index_bf16", C.c_int32), ("prefill_dense", C.c_int32),
-        ("top_k", C.c_int64),
+        ("top_k", C.c_int64), ("n_clusters", C.c_int32),
     ]
 
 
@@ -51,6 +51,19 @@ class rtp_prefill_stats(C.Structure):
 class rtp_cache_view(C.Structure):
     _fields_ = [("k", C.c_void_p), ("v", C.c_void_p), ("idx", C.c_void_p), ("max_seq", C.c_int64),
                 ("n_retrieval", C.c_int32), ("idx_bf16", C.c_void_p)]
+
+
+class rtp_cluster_view(C.Structure):
+    _fields_ = [("centres", C.c_void_p), ("counts", C.c_void_p), ("assign", C.c_void_p),
+                ("n_clusters", C.c_int32), ("ready", C.c_int32), ("max_seq", C.c_int64)]
+
+
+class _DeviceArray:
+    """A borrowed device array described by __cuda_array_interface__ (viewed by torch, no copy)."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(int(d) for d in shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 2, "strides": None}
 
 
 class RTPError(RuntimeError):
@@ -92,6 +105,10 @@ def lib() -> C.CDLL:
             "rtp_profile_read": ([P, C.c_char_p, C.POINTER(C.c_double), C.POINTER(C.c_int64)], C.c_int),
             "rtp_last_error": ([P], C.c_char_p),
             "rtp_probe_ex2": ([i32, i32, P, C.POINTER(C.c_int64), P], C.c_int),
+            "rtp_cluster_build": ([P, i32, P], C.c_int),
+            "rtp_cluster_drop": ([P], C.c_int),
+            "rtp_cluster_len": ([P, i32], i64),
+            "rtp_get_clusters": ([P, C.POINTER(rtp_cluster_view)], C.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -205,6 +222,24 @@ def rtp_get_cache(layer) -> rtp_cache_view:
     return v
 
 
+def rtp_cluster_build(layer, iters: int, stream: int) -> None:
+    _check(lib().rtp_cluster_build(layer, iters, stream), layer)
+
+
+def rtp_cluster_drop(layer) -> None:
+    _check(lib().rtp_cluster_drop(layer), layer)
+
+
+def rtp_cluster_len(layer, b: int) -> int:
+    return int(lib().rtp_cluster_len(layer, b))
+
+
+def rtp_get_clusters(layer) -> rtp_cluster_view:
+    v = rtp_cluster_view()
+    _check(lib().rtp_get_clusters(layer, C.byref(v)), layer)
+    return v
+
+
 def rtp_last_error(layer=None) -> str:
     m = lib().rtp_last_error(layer)
     return m.decode() if m else ""
@@ -251,7 +286,7 @@ class Layer:
                  wq: Optional[np.ndarray], wk: Optional[np.ndarray], top_p: float, window: int,
                  n_sink: int, max_seq: int, rope_base: float = 1.0e6, sm_scale: float = 0.0,
                  max_select: int = 0, max_chunk: int = 0, index_bf16: bool = False,
-                 prefill_dense: bool = False, top_k: int = 0):
+                 prefill_dense: bool = False, top_k: int = 0, n_clusters: int = 0):
         self._hc = np.ascontiguousarray(np.asarray(head_class, dtype=np.uint8))
         self.n_retrieval = int(self._hc.sum())
         self._wq = None if wq is None else np.ascontiguousarray(wq, dtype=np.float32)
@@ -263,7 +298,7 @@ class Layer:
             wq_index=self._wq.ctypes.data if self._wq is not None else None,
             wk_index=self._wk.ctypes.data if self._wk is not None else None,
             max_select=max_select, max_chunk=max_chunk, index_bf16=1 if index_bf16 else 0,
-            prefill_dense=1 if prefill_dense else 0, top_k=int(top_k))
+            prefill_dense=1 if prefill_dense else 0, top_k=int(top_k), n_clusters=int(n_clusters))
         self.batch, self.n_q_heads, self.n_kv_heads = batch, n_q_heads, n_kv_heads
         self.handle = rtp_create(cfg)
         import torch
@@ -411,3 +446,27 @@ class Layer:
 
     def cache(self) -> rtp_cache_view:
         return rtp_get_cache(self.handle)
+
+    def cluster_build(self, iters: int, stream=None) -> None:
+        """K-means of every sequence's index keys (rtp_cluster_build); decode then selects by clusters."""
+        rtp_cluster_build(self.handle, iters, _stream_handle(stream))
+
+    def cluster_drop(self) -> None:
+        rtp_cluster_drop(self.handle)
+
+    def cluster_len(self, b: int) -> int:
+        return rtp_cluster_len(self.handle, b)
+
+    def clusters(self):
+        """Device views of the clustering: centres fp64 [B][Hr][K][16], counts int32 [B][Hr][K] and
+        assign [B][Hr][max_seq] (uint16 cluster ids, returned widened to int32)."""
+        import torch
+
+        v = rtp_get_clusters(self.handle)
+        B, Hr, K = self.batch, self.n_retrieval, v.n_clusters
+        if K < 1 or Hr < 1:
+            raise RTPError(RTP_EINVAL, "the layer has no clustering")
+        cent = torch.as_tensor(_DeviceArray(v.centres, (B, Hr, K, 16), "<f8"), device=self.device)
+        counts = torch.as_tensor(_DeviceArray(v.counts, (B, Hr, K), "<i4"), device=self.device)
+        asg = torch.as_tensor(_DeviceArray(v.assign, (B, Hr, v.max_seq), "<i2"), device=self.device)
+        return {"centres": cent, "counts": counts, "assign": asg.to(torch.int32) & 0xFFFF, "ready": bool(v.ready)}

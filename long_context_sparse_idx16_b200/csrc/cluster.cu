@@ -1,0 +1,422 @@
+// cluster.cu -- K-cache clustering of the retrieval heads' index keys and the clustered decode
+// selection built on it (RTPurboV2, aitntnews page, finding 3: redundancy along the sequence,
+// the two-level funnel of a coarse match against K cluster centres and exact attention inside
+// the clusters hit).
+//
+// Clustering (rtp_cluster_build): Lloyd's k-means, per (sequence, retrieval head), of the stored
+// bf16 index keys kt_j in the r = 16 index space.  The keys are put on the fixed-point grid
+// 2^-27 (xq = rint(kt * 2^27) / 2^27, the integer numerators exact in int64), so a centre's sum
+// is an exact integer sum in whatever order the atomics add it, and every step repeats bit for
+// bit:
+//   init    centre k starts at key floor((2k + 1) n / (2K));
+//   assign  each key goes to the centre of least squared distance, the 16 fp64 terms (x - mu)^2
+//           accumulated by fused multiply-adds in dimension order; ties to the lower centre;
+//   update  every non-empty centre moves to (integer sum of its keys) / count / 2^27 (fp64,
+//           correctly rounded divisions); an empty centre stays;
+// and a final assignment after the last move gives the cluster sizes.
+//
+// Clustered decode: the centre scores c_k = q~ . mu_k (fp64, from the fp32 index query), the
+// cluster weights n_k exp(c_k - max c), the clusters taken in (c desc, k asc) order while the
+// weight before them is below p of the total; the selected set is every clustered key of a hit
+// cluster plus every key cached after the clustering, in ascending position order, which the
+// sparse-attention gather then attends to exactly.
+#include "rtp_device.cuh"
+#include "rtp_internal.h"
+
+namespace rtp {
+namespace {
+
+constexpr double kClScale = 134217728.0;  // 2^27
+constexpr double kClKeyLimit = 32768.0;   // |kt| < 2^15: sums of up to 2^21 keys stay in int64
+constexpr int kClThreads = 256;
+constexpr int kClAssignKeys = 256;        // keys per CTA of the assignment (one per thread)
+constexpr int kClAccumKeys = 16384;       // keys per CTA of the centre-sum accumulation
+
+// A stored bf16 index key component on the clustering grid; out-of-range values (and NaN) map
+// to 0 and are reported by the accumulation kernel.
+__device__ __forceinline__ double cl_grid(float f) {
+  const double x = (double)f;
+  return fabs(x) < kClKeyLimit ? rint(x * kClScale) / kClScale : 0.0;
+}
+
+__device__ __forceinline__ double cl_sqdist(const double* x, const double* mu) {
+  double acc = 0.0;
+#pragma unroll
+  for (int c = 0; c < kR; ++c) {
+    const double d = __dsub_rn(x[c], mu[c]);
+    acc = __fma_rn(d, d, acc);
+  }
+  return acc;
+}
+
+__global__ void cl_init_kernel(const __nv_bfloat16* __restrict__ idx, double* __restrict__ cent,
+                               unsigned long long* __restrict__ sum, unsigned long long* __restrict__ cnt, int K,
+                               int Hr, int64_t max_seq, const SeqPos lens) {
+  const int p = blockIdx.x;
+  const int64_t n = lens.v[p / Hr];
+  for (int i = threadIdx.x; i < K * kR; i += blockDim.x) {
+    const int k = i / kR, c = i % kR;
+    const int64_t j = ((int64_t)(2 * k + 1) * n) / (2 * (int64_t)K);
+    cent[(int64_t)p * K * kR + i] = cl_grid(__bfloat162float(idx[((int64_t)p * max_seq + j) * kR + c]));
+    sum[(int64_t)p * K * kR + i] = 0ull;
+  }
+  for (int k = threadIdx.x; k < K; k += blockDim.x) cnt[(int64_t)p * K + k] = 0ull;
+}
+
+// One key per thread against all K centres (staged in shared memory, read as broadcasts).
+// Four centres per step give four independent fma chains; each chain keeps dimension order.
+__global__ void __launch_bounds__(kClThreads) cl_assign_kernel(const __nv_bfloat16* __restrict__ idx,
+                                                               const double* __restrict__ cent,
+                                                               uint16_t* __restrict__ assign, int K, int Hr,
+                                                               int64_t max_seq, const SeqPos lens) {
+  extern __shared__ double s_cent[];  // [K][r]
+  const int p = blockIdx.y;
+  const int64_t n = lens.v[p / Hr];
+  const int64_t j0 = (int64_t)blockIdx.x * kClAssignKeys;
+  if (j0 >= n) return;  // the whole CTA leaves before its only barrier
+  const double2* cg = reinterpret_cast<const double2*>(cent + (int64_t)p * K * kR);
+  for (int i = threadIdx.x; i < K * kR / 2; i += kClThreads) reinterpret_cast<double2*>(s_cent)[i] = cg[i];
+  const int64_t j = j0 + threadIdx.x;
+  double x[kR];
+  if (j < n) {
+    const uint4* src = reinterpret_cast<const uint4*>(idx + ((int64_t)p * max_seq + j) * kR);
+    const uint4 u0 = src[0], u1 = src[1];
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // element 2i is the low half of word i
+      x[2 * i] = cl_grid(__uint_as_float(w[i] << 16));
+      x[2 * i + 1] = cl_grid(__uint_as_float(w[i] & 0xffff0000u));
+    }
+  }
+  __syncthreads();
+  if (j >= n) return;
+  int best = 0;
+  double bd = cl_sqdist(x, s_cent);
+  int k = 1;
+  for (; k + 3 < K; k += 4) {
+    const double d0 = cl_sqdist(x, s_cent + (k + 0) * kR);
+    const double d1 = cl_sqdist(x, s_cent + (k + 1) * kR);
+    const double d2 = cl_sqdist(x, s_cent + (k + 2) * kR);
+    const double d3 = cl_sqdist(x, s_cent + (k + 3) * kR);
+    if (d0 < bd) { bd = d0; best = k; }
+    if (d1 < bd) { bd = d1; best = k + 1; }
+    if (d2 < bd) { bd = d2; best = k + 2; }
+    if (d3 < bd) { bd = d3; best = k + 3; }
+  }
+  for (; k < K; ++k) {
+    const double d = cl_sqdist(x, s_cent + k * kR);
+    if (d < bd) { bd = d; best = k; }
+  }
+  assign[(int64_t)p * max_seq + j] = (uint16_t)best;
+}
+
+// Integer centre sums and counts of the current assignment: 16 lanes per key (one component
+// each) add into a CTA-private shared-memory table, flushed to the global sums by atomics.
+__global__ void __launch_bounds__(kClThreads) cl_accum_kernel(const __nv_bfloat16* __restrict__ idx,
+                                                              const uint16_t* __restrict__ assign,
+                                                              unsigned long long* __restrict__ sum,
+                                                              unsigned long long* __restrict__ cnt, int K, int Hr,
+                                                              int64_t max_seq, const SeqPos lens,
+                                                              uint32_t* __restrict__ err) {
+  extern __shared__ unsigned long long s_sum[];  // [K][r], then [K] counts as uint32
+  uint32_t* s_cnt = reinterpret_cast<uint32_t*>(s_sum + (size_t)K * kR);
+  const int p = blockIdx.y;
+  const int64_t n = lens.v[p / Hr];
+  const int64_t j0 = (int64_t)blockIdx.x * kClAccumKeys;
+  if (j0 >= n) return;
+  for (int i = threadIdx.x; i < K * kR; i += kClThreads) s_sum[i] = 0ull;
+  for (int i = threadIdx.x; i < K; i += kClThreads) s_cnt[i] = 0u;
+  __syncthreads();
+  const int c = threadIdx.x & (kR - 1);
+  const int64_t jend = n < j0 + kClAccumKeys ? n : j0 + kClAccumKeys;
+  bool bad = false;
+  for (int64_t j = j0 + (threadIdx.x >> 4); j < jend; j += kClThreads / kR) {
+    const int a = assign[(int64_t)p * max_seq + j];
+    const double x = (double)__bfloat162float(idx[((int64_t)p * max_seq + j) * kR + c]);
+    long long q = 0;
+    if (fabs(x) < kClKeyLimit) q = (long long)rint(x * kClScale);
+    else bad = true;
+    if (q != 0) atomicAdd(&s_sum[a * kR + c], (unsigned long long)q);
+    if (c == 0) atomicAdd(&s_cnt[a], 1u);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < K * kR; i += kClThreads)
+    if (s_sum[i] != 0ull) atomicAdd(&sum[(int64_t)p * K * kR + i], s_sum[i]);
+  for (int i = threadIdx.x; i < K; i += kClThreads)
+    if (s_cnt[i] != 0u) atomicAdd(&cnt[(int64_t)p * K + i], (unsigned long long)s_cnt[i]);
+  if (bad) atomicOr(err, kErrRange);
+}
+
+// Cluster sizes of the current assignment; with `move`, every non-empty centre moves to the
+// mean of its keys.  Clears the accumulators for the next pass.
+__global__ void cl_update_kernel(double* __restrict__ cent, unsigned long long* __restrict__ sum,
+                                 unsigned long long* __restrict__ cnt, int32_t* __restrict__ counts, int K,
+                                 int move) {
+  const int p = blockIdx.x;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    const int64_t pk = (int64_t)p * K + k;
+    const unsigned long long m = cnt[pk];
+    counts[pk] = (int32_t)m;
+    for (int c = 0; c < kR; ++c) {
+      if (move && m > 0ull)
+        cent[pk * kR + c] = __ddiv_rn(__ddiv_rn(__ll2double_rn((long long)sum[pk * kR + c]), __ull2double_rn(m)),
+                                      kClScale);
+      sum[pk * kR + c] = 0ull;
+    }
+    cnt[pk] = 0ull;
+  }
+}
+
+// ---------------------------------------------------------------- clustered decode selection
+
+constexpr int kClSelThreads = 1024;  // one thread per cluster (K <= 1024)
+constexpr int kClChunk = 4096;       // positions per CTA of the compaction
+
+template <typename T, typename Op>
+__device__ __forceinline__ T cl_block_reduce(T v, T* s_red, Op op) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();  // s_red may still be read by a previous reduction
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  v = s_red[0];
+  for (int w = 1; w < nw; ++w) v = op(v, s_red[w]);
+  return v;
+}
+
+struct DMax {
+  __device__ double operator()(double a, double b) const { return a > b ? a : b; }
+};
+struct DSum {
+  __device__ double operator()(double a, double b) const { return a + b; }
+};
+struct IMax {
+  __device__ int operator()(int a, int b) const { return a > b ? a : b; }
+};
+struct ISum {
+  __device__ int operator()(int a, int b) const { return a + b; }
+};
+
+// The coarse match of one problem's index query against its K centres: hit flags, the hit
+// clusters' weight fraction (sel_mass) and the weight fraction of the last cluster taken
+// (threshold).  A cluster's place in the (c desc, k asc) order and the weight before it come
+// from a direct count over all K clusters, so no sort is needed.
+__global__ void __launch_bounds__(kClSelThreads) cl_select_kernel(const float* __restrict__ q_idx,
+                                                                  const double* __restrict__ cent,
+                                                                  const int32_t* __restrict__ counts, int K,
+                                                                  float top_p, uint8_t* __restrict__ hit,
+                                                                  float* __restrict__ sel_mass,
+                                                                  float* __restrict__ sel_thr) {
+  __shared__ double s_c[kClSelThreads], s_w[kClSelThreads];
+  __shared__ double s_red[32];
+  __shared__ int s_ired[32];
+  const int p = blockIdx.x, k = threadIdx.x;
+  const bool live = k < K && counts[(int64_t)p * K + k] > 0;
+  double ck = -INFINITY;
+  if (live) {
+    const float* q = q_idx + (int64_t)p * kR;
+    const double* mu = cent + ((int64_t)p * K + k) * kR;
+    double acc = 0.0;
+#pragma unroll
+    for (int c = 0; c < kR; ++c) acc = __dadd_rn(acc, __dmul_rn((double)q[c], mu[c]));
+    ck = acc;
+  }
+  const double cmax = cl_block_reduce(ck, s_red, DMax());
+  const double wk = live ? (double)counts[(int64_t)p * K + k] * exp(ck - cmax) : 0.0;
+  s_c[k] = ck;
+  s_w[k] = wk;
+  const double tot = cl_block_reduce(wk, s_red, DSum());  // its barriers publish s_c, s_w
+  double before = 0.0;
+  int rank = 0;
+  if (live) {
+    for (int o = 0; o < K; ++o) {
+      const double co = s_c[o];
+      if (o != k && co != -INFINITY && (co > ck || (co == ck && o < k))) {  // -inf: empty cluster
+        before += s_w[o];
+        ++rank;
+      }
+    }
+  }
+  const bool h = live && (top_p >= 1.f || before / tot < (double)top_p);
+  if (k < K) hit[(int64_t)p * K + k] = h ? 1 : 0;
+  const double mass = cl_block_reduce(h ? wk : 0.0, s_red, DSum());
+  const int last = cl_block_reduce(h ? rank : -1, s_ired, IMax());
+  if (k == 0) sel_mass[p] = (float)(mass / tot);
+  if (h && rank == last) sel_thr[p] = (float)(wk / tot);
+}
+
+// Selected positions of problem p: clustered keys (j < ncl) of hit clusters, and every key
+// cached after the clustering (ncl <= j < n).
+__device__ __forceinline__ bool cl_take(const uint16_t* __restrict__ asg, const uint8_t* s_hit, int64_t j,
+                                        int64_t ncl, int64_t n) {
+  return j < n && (j >= ncl || s_hit[asg[j]] != 0);
+}
+
+// Per-chunk counts; the last CTA of a problem (ticket) turns them into exclusive offsets in
+// place and writes the set size.
+__global__ void __launch_bounds__(kClThreads) cl_count_kernel(const uint16_t* __restrict__ assign,
+                                                              const uint8_t* __restrict__ hit, int K, int Hr,
+                                                              int64_t max_seq, int64_t max_select,
+                                                              const SeqPos lens, const SeqPos ncl_b,
+                                                              int32_t* __restrict__ chunk,
+                                                              uint32_t* __restrict__ ticket,
+                                                              int32_t* __restrict__ sel_cnt,
+                                                              uint32_t* __restrict__ err) {
+  __shared__ uint8_t s_hit[1024];
+  __shared__ int s_red[32];
+  __shared__ bool s_last;
+  const int p = blockIdx.y, b = p / Hr;
+  const int64_t n = lens.v[b], ncl = ncl_b.v[b];
+  const int64_t j0 = (int64_t)blockIdx.x * kClChunk;
+  for (int i = threadIdx.x; i < K; i += kClThreads) s_hit[i] = hit[(int64_t)p * K + i];
+  __syncthreads();
+  const uint16_t* asg = assign + (int64_t)p * max_seq;
+  int c = 0;
+  for (int i = threadIdx.x; i < kClChunk; i += kClThreads) c += cl_take(asg, s_hit, j0 + i, ncl, n) ? 1 : 0;
+  c = cl_block_reduce(c, s_red, ISum());
+  const int nch = gridDim.x;
+  if (threadIdx.x == 0) {
+    chunk[(int64_t)p * nch + blockIdx.x] = c;
+    __threadfence();
+    s_last = atomicAdd(&ticket[p], 1u) == (uint32_t)(nch - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // exclusive scan of the nch counts, kClThreads at a time
+  __shared__ long long s_scan[kClThreads];
+  long long base = 0;
+  for (int t0 = 0; t0 < nch; t0 += kClThreads) {
+    const int t = t0 + threadIdx.x;
+    const long long v = t < nch ? (long long)*((volatile int32_t*)&chunk[(int64_t)p * nch + t]) : 0;
+    s_scan[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < kClThreads; o <<= 1) {
+      const long long add = threadIdx.x >= o ? s_scan[threadIdx.x - o] : 0;
+      __syncthreads();
+      s_scan[threadIdx.x] += add;
+      __syncthreads();
+    }
+    if (t < nch) chunk[(int64_t)p * nch + t] = (int32_t)(base + s_scan[threadIdx.x] - v);
+    base += s_scan[kClThreads - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    sel_cnt[p] = (int32_t)(base < max_select ? base : max_select);
+    if (base > max_select) atomicOr(err, kErrOverflow);
+    ticket[p] = 0u;
+  }
+}
+
+// Ordered write of the selected positions: positions of a chunk go in blocks of kClThreads, one
+// per thread; warp ballots and a scan of the per-warp counts give each its slot.
+__global__ void __launch_bounds__(kClThreads) cl_write_kernel(const uint16_t* __restrict__ assign,
+                                                              const uint8_t* __restrict__ hit, int K, int Hr,
+                                                              int64_t max_seq, int64_t max_select,
+                                                              const SeqPos lens, const SeqPos ncl_b,
+                                                              const int32_t* __restrict__ chunk,
+                                                              int32_t* __restrict__ sel_idx) {
+  __shared__ uint8_t s_hit[1024];
+  __shared__ int s_wc[kClThreads / 32];
+  const int p = blockIdx.y, b = p / Hr;
+  const int64_t n = lens.v[b], ncl = ncl_b.v[b];
+  const int64_t j0 = (int64_t)blockIdx.x * kClChunk;
+  if (j0 >= n) return;
+  for (int i = threadIdx.x; i < K; i += kClThreads) s_hit[i] = hit[(int64_t)p * K + i];
+  __syncthreads();
+  const uint16_t* asg = assign + (int64_t)p * max_seq;
+  int32_t* dst = sel_idx + (int64_t)p * max_select;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t base = chunk[(int64_t)p * gridDim.x + blockIdx.x];
+  for (int i0 = 0; i0 < kClChunk; i0 += kClThreads) {
+    const int64_t j = j0 + i0 + threadIdx.x;
+    const bool t = cl_take(asg, s_hit, j, ncl, n);
+    const uint32_t bal = __ballot_sync(0xffffffffu, t);
+    if (lane == 0) s_wc[warp] = __popc(bal);
+    __syncthreads();
+    int off = 0, tot = 0;
+    for (int w = 0; w < kClThreads / 32; ++w) {
+      off += w < warp ? s_wc[w] : 0;
+      tot += s_wc[w];
+    }
+    const int64_t slot = base + off + __popc(bal & ((1u << lane) - 1u));
+    if (t && slot < max_select) dst[slot] = (int32_t)j;
+    base += tot;
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_cluster_build(rtp_layer* L, int iters, cudaStream_t st) {
+  const int K = L->n_clusters, P = L->B * L->Hr;
+  const SeqPos lens = seq_pos(L, 0);
+  const int64_t nmax = L->len;
+  cudaError_t e;
+  {
+    ProfScope ps(L, "cluster_init", st);
+    cl_init_kernel<<<P, kClThreads, 0, st>>>(L->idx_b, L->cl_cent, L->cl_sum, L->cl_acc, K, L->Hr, L->max_seq, lens);
+    e = cudaGetLastError();
+  }
+  const size_t smem_a = (size_t)K * kR * sizeof(double);
+  const size_t smem_s = (size_t)K * kR * sizeof(unsigned long long) + (size_t)K * sizeof(uint32_t);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(cl_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(cl_accum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s);
+  const dim3 ga((unsigned)((nmax + kClAssignKeys - 1) / kClAssignKeys), (unsigned)P);
+  const dim3 gs((unsigned)((nmax + kClAccumKeys - 1) / kClAccumKeys), (unsigned)P);
+  for (int it = 0; it <= iters && e == cudaSuccess; ++it) {
+    {
+      ProfScope ps(L, "cluster_assign", st);
+      cl_assign_kernel<<<ga, kClThreads, smem_a, st>>>(L->idx_b, L->cl_cent, L->cl_assign, K, L->Hr, L->max_seq,
+                                                       lens);
+      e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) break;
+    {
+      ProfScope ps(L, "cluster_accum", st);
+      cl_accum_kernel<<<gs, kClThreads, smem_s, st>>>(L->idx_b, L->cl_assign, L->cl_sum, L->cl_acc, K, L->Hr,
+                                                      L->max_seq, lens, L->err);
+      e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) break;
+    {
+      ProfScope ps(L, "cluster_update", st);
+      cl_update_kernel<<<P, kClThreads, 0, st>>>(L->cl_cent, L->cl_sum, L->cl_acc, L->cl_count, K, it < iters ? 1 : 0);
+      e = cudaGetLastError();
+    }
+  }
+  return e;
+}
+
+cudaError_t launch_cluster_select(rtp_layer* L, cudaStream_t st) {
+  const int K = L->n_clusters, P = L->B * L->Hr;
+  const SeqPos lens = seq_pos(L, 0);
+  SeqPos ncl{};
+  for (int b = 0; b < L->B; ++b) ncl.v[b] = (int32_t)L->cl_len[(size_t)b];
+  cudaError_t e;
+  {
+    ProfScope ps(L, "cluster_select", st);
+    cl_select_kernel<<<P, kClSelThreads, 0, st>>>(L->q_idx, L->cl_cent, L->cl_count, K, L->top_p, L->cl_hit,
+                                                  L->sel_mass, L->sel_thr);
+    e = cudaGetLastError();
+  }
+  const dim3 g((unsigned)((L->len + kClChunk - 1) / kClChunk), (unsigned)P);
+  if (e == cudaSuccess) {
+    ProfScope ps(L, "cluster_count", st);
+    cl_count_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_hit, K, L->Hr, L->max_seq, L->max_select, lens, ncl,
+                                              L->cl_chunk, L->cl_ticket, L->sel_cnt, L->err);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) {
+    ProfScope ps(L, "cluster_write", st);
+    cl_write_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_hit, K, L->Hr, L->max_seq, L->max_select, lens, ncl,
+                                              L->cl_chunk, L->sel_idx);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+int64_t cluster_chunks(int64_t max_seq) { return (max_seq + kClChunk - 1) / kClChunk; }
+
+}  // namespace rtp

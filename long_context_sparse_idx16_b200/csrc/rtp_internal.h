@@ -137,6 +137,19 @@ struct rtp_layer {
   uint32_t* err = nullptr;       // device error word
   long long wait_limit = 0;      // decode grid-barrier wait limit in cycles (0: the default, ~1 s)
 
+  // K-cache clustering of the index keys (n_clusters > 0, bf16 index keys)
+  int n_clusters = 0;
+  bool cl_ready = false;                 // centres and assignments valid (rtp_cluster_build)
+  std::vector<int64_t> cl_len;           // [B] keys clustered per sequence
+  double* cl_cent = nullptr;             // [P][K][r] fp64 centres
+  int32_t* cl_count = nullptr;           // [P][K] cluster sizes
+  uint16_t* cl_assign = nullptr;         // [P][max_seq] cluster of each clustered key
+  unsigned long long* cl_sum = nullptr;  // [P][K][r] integer centre sums (two's complement)
+  unsigned long long* cl_acc = nullptr;  // [P][K] counts being accumulated
+  uint8_t* cl_hit = nullptr;             // [P][K] clusters hit by the current decode query
+  int32_t* cl_chunk = nullptr;           // [P][max_seq / 4096] selected counts, then offsets
+  uint32_t* cl_ticket = nullptr;         // [P]
+
   // per-kernel event timing (rtp_profile_enable)
   bool prof_on = false;
   std::map<std::string, std::vector<std::pair<cudaEvent_t, cudaEvent_t>>> prof;
@@ -176,6 +189,11 @@ cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, float* out, cud
 cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st);
 cudaError_t launch_iota_rows(const rtp_layer* L, int32_t* dst, int64_t cap, cudaStream_t st);
 cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st);
+// K-cache clustering: `iters` k-means passes over every sequence's keys 0 .. len_b - 1, and the
+// clustered decode selection (sel_idx, sel_cnt, sel_mass, sel_thr)
+cudaError_t launch_cluster_build(rtp_layer* L, int iters, cudaStream_t st);
+cudaError_t launch_cluster_select(rtp_layer* L, cudaStream_t st);
+int64_t cluster_chunks(int64_t max_seq);
 cudaError_t launch_prefill_local(const rtp_layer* L, int C, float* out, cudaStream_t st);
 cudaError_t launch_prefill_retrieval(rtp_layer* L, int C, float* out, const rtp_prefill_stats* stats,
                                      cudaStream_t st);

@@ -102,7 +102,8 @@ static void free_all(rtp_layer* L) {
                   L->sel_mass, L->sel_thr, L->seg_max, L->sel_words, L->cand_cnt, L->cand,
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
                   L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt, L->pf_capture, L->attn_part,
-                  L->attn_ticket, L->sel_cum, L->sel_psum, L->sel_pticket, L->sel_cres};
+                  L->attn_ticket, L->sel_cum, L->sel_psum, L->sel_pticket, L->sel_cres, L->cl_cent,
+                  L->cl_count, L->cl_assign, L->cl_sum, L->cl_acc, L->cl_hit, L->cl_chunk, L->cl_ticket};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -158,6 +159,10 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   if (c.prefill_dense != 0 && c.prefill_dense != 1)
     return fail(nullptr, RTP_EINVAL, "rtp_create: prefill_dense must be 0 or 1");
   if (c.top_k < 0) return fail(nullptr, RTP_EINVAL, "rtp_create: top_k must be >= 0");
+  if (c.n_clusters < 0 || c.n_clusters > 1024)
+    return fail(nullptr, RTP_EINVAL, "rtp_create: n_clusters must be in [0, 1024]");
+  if (c.n_clusters > 0 && (c.index_bf16 != 1 || c.top_k != 0))
+    return fail(nullptr, RTP_EINVAL, "rtp_create: n_clusters needs index_bf16 = 1 and top_k = 0");
 
   rtp_layer* L = new rtp_layer();
   L->B = c.batch;
@@ -171,6 +176,8 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   L->index_bf16 = c.index_bf16 == 1;
   L->prefill_dense = c.prefill_dense == 1;
   L->top_k = c.top_k;
+  L->n_clusters = c.n_clusters;
+  L->cl_len.assign((size_t)c.batch, 0);
   L->top_p = c.top_p;
   L->sm_scale = c.sm_scale > 0.f ? c.sm_scale : 1.0f / sqrtf((float)kD);
   L->rope_base = c.rope_base;
@@ -274,6 +281,18 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   RTP_ALLOC(L->sel_pticket, P);
   RTP_ALLOC(L->slot_cnt, 2 * (P + G));
   RTP_ALLOC(L->bar, 2);
+  if (L->n_clusters > 0 && Hr > 0) {
+    const int64_t K = L->n_clusters;
+    RTP_ALLOC(L->cl_cent, P * K * kR);
+    RTP_ALLOC(L->cl_count, P * K);
+    RTP_ALLOC(L->cl_assign, P * L->max_seq);
+    RTP_ALLOC(L->cl_sum, P * K * kR);
+    RTP_ALLOC(L->cl_acc, P * K);
+    RTP_ALLOC(L->cl_hit, P * K);
+    RTP_ALLOC(L->cl_chunk, P * cluster_chunks(L->max_seq));
+    RTP_ALLOC(L->cl_ticket, P);
+    if (e == cudaSuccess) e = cudaMemset(L->cl_ticket, 0, sizeof(uint32_t) * (size_t)P);
+  }
   if (need_gscores) {
     L->gscores_elems = (size_t)(P * L->max_seq);
     RTP_ALLOC(L->gscores, L->gscores_elems);
@@ -363,6 +382,11 @@ void update_len(rtp_layer* L) {
   for (int64_t n : L->lens) mx = n > mx ? n : mx;
   L->len = mx;
 }
+// A truncation below the clustered prefix of some sequence invalidates the clustering.
+void drop_stale_clusters(rtp_layer* L) {
+  for (int b = 0; b < L->B && L->cl_ready; ++b)
+    if (L->lens[(size_t)b] < L->cl_len[(size_t)b]) L->cl_ready = false;
+}
 int64_t min_len(const rtp_layer* L) {
   int64_t mn = L->lens.empty() ? 0 : L->lens[0];
   for (int64_t n : L->lens) mn = n < mn ? n : mn;
@@ -418,10 +442,11 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
   if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: q_prep");
   bool forked = false;
   if (L->Hr > 0) {
-    // p == 1 keeps every causal key: the gather reads positions 0..len-1 directly
     // p == 1 (without a fixed budget) keeps every causal key: the gather reads 0..len-1 directly
     const bool dense = L->top_k == 0 && L->top_p >= 1.f;
-    {
+    if (!dense && L->cl_ready) {
+      e = launch_cluster_select(L, stream);  // times its kernels itself ("cluster_*")
+    } else {
       ProfScope ps(L, dense ? "dense_fill" : (L->top_k > 0 ? "decode_topk" : "decode_select"), stream);
       e = dense ? launch_dense_stats(L, stream)
                 : (L->top_k > 0 ? launch_decode_topk(L, stream) : launch_decode_select(L, stream));
@@ -558,6 +583,7 @@ rtp_status rtp_truncate(rtp_layer* L, int64_t new_len) {
   if (new_len < 0 || new_len > L->len) return fail(L, RTP_EINVAL, "rtp_truncate: need 0 <= new_len <= length");
   for (int64_t& n : L->lens) n = n < new_len ? n : new_len;
   update_len(L);
+  drop_stale_clusters(L);
   return RTP_OK;
 }
 
@@ -568,6 +594,47 @@ rtp_status rtp_truncate_seq(rtp_layer* L, int32_t b, int64_t new_len) {
     return fail(L, RTP_EINVAL, "rtp_truncate_seq: need 0 <= new_len <= the sequence's length");
   L->lens[b] = new_len;
   update_len(L);
+  drop_stale_clusters(L);
+  return RTP_OK;
+}
+
+rtp_status rtp_cluster_build(rtp_layer* L, int32_t iters, cudaStream_t stream) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_cluster_build: layer is NULL");
+  if (L->n_clusters < 1 || L->Hr < 1)
+    return fail(L, RTP_EINVAL, "rtp_cluster_build: the layer has no n_clusters or no retrieval heads");
+  if (iters < 0 || iters > 1000) return fail(L, RTP_EINVAL, "rtp_cluster_build: iters must be in [0, 1000]");
+  for (int64_t n : L->lens) {
+    if (n < L->n_clusters) return fail(L, RTP_EINVAL, "rtp_cluster_build: a sequence has fewer keys than n_clusters");
+    if (n > ((int64_t)1 << 21)) return fail(L, RTP_EINVAL, "rtp_cluster_build: a sequence has more than 2^21 keys");
+  }
+  L->cl_ready = false;
+  const cudaError_t e = launch_cluster_build(L, iters, stream);
+  if (e != cudaSuccess) return cuda_fail(L, e, "rtp_cluster_build: launch");
+  L->cl_len = L->lens;
+  L->cl_ready = true;
+  L->last_error.clear();
+  return RTP_OK;
+}
+
+rtp_status rtp_cluster_drop(rtp_layer* L) {
+  if (!L) return fail(nullptr, RTP_EINVAL, "rtp_cluster_drop: layer is NULL");
+  L->cl_ready = false;
+  return RTP_OK;
+}
+
+int64_t rtp_cluster_len(const rtp_layer* L, int32_t b) {
+  if (!L || b < 0 || b >= L->B) return -1;
+  return L->cl_ready ? L->cl_len[(size_t)b] : 0;
+}
+
+rtp_status rtp_get_clusters(const rtp_layer* L, rtp_cluster_view* view) {
+  if (!L || !view) return fail(nullptr, RTP_EINVAL, "rtp_get_clusters: NULL argument");
+  view->centres = L->cl_cent;
+  view->counts = L->cl_count;
+  view->assign = L->cl_assign;
+  view->n_clusters = L->n_clusters;
+  view->ready = L->cl_ready ? 1 : 0;
+  view->max_seq = L->max_seq;
   return RTP_OK;
 }
 
@@ -607,6 +674,7 @@ rtp_status rtp_reset(rtp_layer* L) {
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_reset: layer is NULL");
   for (int64_t& n : L->lens) n = 0;
   L->len = 0;
+  L->cl_ready = false;
   return RTP_OK;
 }
 
@@ -623,6 +691,7 @@ rtp_status rtp_check(rtp_layer* L, cudaStream_t stream) {
     // a barrier gave up: its counters are inconsistent; start the next launch from zero
     reset_select_scratch(L);
     cudaMemset(L->gticket, 0, sizeof(uint32_t) * (size_t)(L->B * L->Hr > 0 ? L->B * L->Hr : 1));
+    if (L->cl_ticket) cudaMemset(L->cl_ticket, 0, sizeof(uint32_t) * (size_t)(L->B * L->Hr));
     if (L->attn_ticket)
       cudaMemset(L->attn_ticket, 0, sizeof(uint32_t) * (size_t)L->B * L->Hr * ((L->max_chunk + 127) / 128));
     return fail(L, RTP_ETIMEOUT, "a bounded in-kernel wait gave up");

@@ -50,6 +50,9 @@ int main(void) {
          offsetof(rtp_config, rope_base), offsetof(rtp_config, wq_index),
          offsetof(rtp_config, max_select), offsetof(rtp_config, max_chunk),
          offsetof(rtp_config, index_bf16), offsetof(rtp_config, top_k));
+  printf("%zu %zu %zu %zu %zu\n", offsetof(rtp_config, n_clusters), sizeof(rtp_cluster_view),
+         offsetof(rtp_cluster_view, n_clusters), offsetof(rtp_cluster_view, ready),
+         offsetof(rtp_cluster_view, max_seq));
   printf("%zu %zu %zu %zu %zu %zu\n", sizeof(rtp_decode_stats), offsetof(rtp_decode_stats, sel_index_cap),
          sizeof(rtp_cache_view), offsetof(rtp_cache_view, idx_bf16), sizeof(rtp_prefill_stats),
          offsetof(rtp_prefill_stats, row_sel_cap));
@@ -61,11 +64,14 @@ int main(void) {
         open(c, "w").write(src)
         exe = os.path.join(d, "p")
         subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include", c, "-o", exe])
-        a, b = subprocess.check_output([exe], text=True).splitlines()
+        a, c3, b = subprocess.check_output([exe], text=True).splitlines()
     cfg = rtp.rtp_config
     assert [int(t) for t in a.split()] == [C.sizeof(cfg), cfg.max_seq.offset, cfg.rope_base.offset,
                                           cfg.wq_index.offset, cfg.max_select.offset, cfg.max_chunk.offset,
                                           cfg.index_bf16.offset, cfg.top_k.offset]
+    cv = rtp.rtp_cluster_view
+    assert [int(t) for t in c3.split()] == [cfg.n_clusters.offset, C.sizeof(cv), cv.n_clusters.offset,
+                                           cv.ready.offset, cv.max_seq.offset]
     st = rtp.rtp_decode_stats
     ps = rtp.rtp_prefill_stats
     assert [int(t) for t in b.split()] == [C.sizeof(st), st.sel_index_cap.offset, C.sizeof(rtp.rtp_cache_view),
@@ -90,7 +96,9 @@ def _cfg(**kw):
                                  dict(max_select=65), dict(batch=0), dict(head_class=None),
                                  dict(n_q_heads=64, n_kv_heads=2), dict(rope_base=1.0), dict(sm_scale=-1.0),
                                  dict(max_chunk=-1), dict(max_seq=1 << 31), dict(wq_index=None), dict(index_bf16=2), dict(top_k=-1), dict(prefill_dense=3),
-                                 dict(wk_index=None), dict(top_p=float("nan")), dict(max_select=-1)])
+                                 dict(wk_index=None), dict(top_p=float("nan")), dict(max_select=-1),
+                                 dict(n_clusters=-1), dict(n_clusters=1025), dict(n_clusters=8),
+                                 dict(n_clusters=8, index_bf16=1, top_k=16)])
 def test_create_rejects_bad_config_on_host(lib, bad):
     cfg, keep = _cfg(**bad)
     h = C.c_void_p()
@@ -108,6 +116,10 @@ def test_calls_on_null_layer_are_rejected(lib):
     assert lib.rtp_seq_len(None) == -1
     assert lib.rtp_destroy(None) == rtp.RTP_OK
     assert lib.rtp_create(None, None) == rtp.RTP_EINVAL
+    assert lib.rtp_cluster_build(None, 4, None) == rtp.RTP_EINVAL
+    assert lib.rtp_cluster_drop(None) == rtp.RTP_EINVAL
+    assert lib.rtp_cluster_len(None, 0) == -1
+    assert lib.rtp_get_clusters(None, None) == rtp.RTP_EINVAL
 
 
 def test_create_rejects_bad_head_maps_on_host(lib):
