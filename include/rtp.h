@@ -141,10 +141,11 @@ typedef struct {
 typedef struct {
   const double* centres;  /* fp64 [P][K][r] cluster centres in the index space */
   const int32_t* counts;  /* [P][K] keys per cluster */
-  const uint16_t* assign; /* [P][max_seq] cluster of each clustered key (positions < rtp_cluster_len) */
+  const uint16_t* assign; /* [P][assign_stride] cluster of each clustered key (positions < rtp_cluster_len) */
   int32_t n_clusters;     /* K (0: the layer cannot cluster) */
   int32_t ready;          /* 1 while the clustering is in use by decode, else 0 */
   int64_t max_seq;
+  int64_t assign_stride;  /* entries per row of assign: max_seq rounded up to a multiple of 16 */
 } rtp_cluster_view;
 
 /* Create a layer on the current CUDA device: validates cfg, allocates the caches and all

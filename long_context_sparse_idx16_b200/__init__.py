@@ -55,7 +55,8 @@ class rtp_cache_view(C.Structure):
 
 class rtp_cluster_view(C.Structure):
     _fields_ = [("centres", C.c_void_p), ("counts", C.c_void_p), ("assign", C.c_void_p),
-                ("n_clusters", C.c_int32), ("ready", C.c_int32), ("max_seq", C.c_int64)]
+                ("n_clusters", C.c_int32), ("ready", C.c_int32), ("max_seq", C.c_int64),
+                ("assign_stride", C.c_int64)]
 
 
 class _DeviceArray:
@@ -468,5 +469,6 @@ class Layer:
             raise RTPError(RTP_EINVAL, "the layer has no clustering")
         cent = torch.as_tensor(_DeviceArray(v.centres, (B, Hr, K, 16), "<f8"), device=self.device)
         counts = torch.as_tensor(_DeviceArray(v.counts, (B, Hr, K), "<i4"), device=self.device)
-        asg = torch.as_tensor(_DeviceArray(v.assign, (B, Hr, v.max_seq), "<i2"), device=self.device)
-        return {"centres": cent, "counts": counts, "assign": asg.to(torch.int32) & 0xFFFF, "ready": bool(v.ready)}
+        asg = torch.as_tensor(_DeviceArray(v.assign, (B, Hr, v.assign_stride), "<i2"), device=self.device)
+        asg = asg[:, :, :v.max_seq].to(torch.int32) & 0xFFFF
+        return {"centres": cent, "counts": counts, "assign": asg, "ready": bool(v.ready)}

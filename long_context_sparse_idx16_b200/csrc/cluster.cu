@@ -67,8 +67,8 @@ __global__ void cl_init_kernel(const __nv_bfloat16* __restrict__ idx, double* __
 // Four centres per step give four independent fma chains; each chain keeps dimension order.
 __global__ void __launch_bounds__(kClThreads) cl_assign_kernel(const __nv_bfloat16* __restrict__ idx,
                                                                const double* __restrict__ cent,
-                                                               uint16_t* __restrict__ assign, int K, int Hr,
-                                                               int64_t max_seq, const SeqPos lens) {
+                                                               uint16_t* __restrict__ assign, int64_t a_stride,
+                                                               int K, int Hr, int64_t max_seq, const SeqPos lens) {
   extern __shared__ double s_cent[];  // [K][r]
   const int p = blockIdx.y;
   const int64_t n = lens.v[p / Hr];
@@ -107,13 +107,13 @@ __global__ void __launch_bounds__(kClThreads) cl_assign_kernel(const __nv_bfloat
     const double d = cl_sqdist(x, s_cent + k * kR);
     if (d < bd) { bd = d; best = k; }
   }
-  assign[(int64_t)p * max_seq + j] = (uint16_t)best;
+  assign[(int64_t)p * a_stride + j] = (uint16_t)best;
 }
 
 // Integer centre sums and counts of the current assignment: 16 lanes per key (one component
 // each) add into a CTA-private shared-memory table, flushed to the global sums by atomics.
 __global__ void __launch_bounds__(kClThreads) cl_accum_kernel(const __nv_bfloat16* __restrict__ idx,
-                                                              const uint16_t* __restrict__ assign,
+                                                              const uint16_t* __restrict__ assign, int64_t a_stride,
                                                               unsigned long long* __restrict__ sum,
                                                               unsigned long long* __restrict__ cnt, int K, int Hr,
                                                               int64_t max_seq, const SeqPos lens,
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kClThreads) cl_accum_kernel(const __nv_bfloat1
   const int64_t jend = n < j0 + kClAccumKeys ? n : j0 + kClAccumKeys;
   bool bad = false;
   for (int64_t j = j0 + (threadIdx.x >> 4); j < jend; j += kClThreads / kR) {
-    const int a = assign[(int64_t)p * max_seq + j];
+    const int a = assign[(int64_t)p * a_stride + j];
     const double x = (double)__bfloat162float(idx[((int64_t)p * max_seq + j) * kR + c]);
     long long q = 0;
     if (fabs(x) < kClKeyLimit) q = (long long)rint(x * kClScale);
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kClSelThreads) cl_select_kernel(const float* _
   __shared__ double s_c[kClSelThreads], s_w[kClSelThreads];
   __shared__ double s_red[32];
   __shared__ int s_ired[32];
-  const int p = blockIdx.x, k = threadIdx.x;
+  const int p = blockIdx.x, k = threadIdx.x;  // blockDim.x: K rounded up to a warp multiple
   const bool live = k < K && counts[(int64_t)p * K + k] > 0;
   double ck = -INFINITY;
   if (live) {
@@ -246,18 +246,47 @@ __global__ void __launch_bounds__(kClSelThreads) cl_select_kernel(const float* _
   if (h && rank == last) sel_thr[p] = (float)(wk / tot);
 }
 
+constexpr int kClPer = kClChunk / kClThreads;  // consecutive positions per thread of a chunk
+
+// The assignments of positions jb .. jb + 15 (jb a multiple of 16; rows padded to 16 entries),
+// loaded as two 16-byte vectors when any of them is clustered.
+__device__ __forceinline__ void cl_load16(const uint16_t* __restrict__ asg, uint16_t* av, int64_t jb, int64_t ncl) {
+  uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+  if (jb < ncl) {
+    const uint4* src = reinterpret_cast<const uint4*>(asg + jb);
+    u0 = __ldg(src);
+    u1 = __ldg(src + 1);
+  }
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    av[2 * i] = (uint16_t)(w[i] & 0xffffu);
+    av[2 * i + 1] = (uint16_t)(w[i] >> 16);
+  }
+}
+
 // Selected positions of problem p: clustered keys (j < ncl) of hit clusters, and every key
 // cached after the clustering (ncl <= j < n).
-__device__ __forceinline__ bool cl_take(const uint16_t* __restrict__ asg, const uint8_t* s_hit, int64_t j,
-                                        int64_t ncl, int64_t n) {
-  return j < n && (j >= ncl || s_hit[asg[j]] != 0);
+__device__ __forceinline__ bool cl_take(uint16_t a, const uint8_t* s_hit, int64_t j, int64_t ncl, int64_t n) {
+  return j < n && (j >= ncl || s_hit[a] != 0);
+}
+
+// Taken positions among this thread's kClPer consecutive ones, as a bit mask.
+__device__ __forceinline__ uint32_t cl_mask(const uint16_t* __restrict__ asg, const uint8_t* s_hit, int64_t jb,
+                                            int64_t ncl, int64_t n) {
+  uint16_t av[kClPer];
+  cl_load16(asg, av, jb, ncl);
+  uint32_t msk = 0u;
+#pragma unroll
+  for (int i = 0; i < kClPer; ++i) msk |= cl_take(av[i], s_hit, jb + i, ncl, n) ? (1u << i) : 0u;
+  return msk;
 }
 
 // Per-chunk counts; the last CTA of a problem (ticket) turns them into exclusive offsets in
 // place and writes the set size.
 __global__ void __launch_bounds__(kClThreads) cl_count_kernel(const uint16_t* __restrict__ assign,
-                                                              const uint8_t* __restrict__ hit, int K, int Hr,
-                                                              int64_t max_seq, int64_t max_select,
+                                                              int64_t a_stride, const uint8_t* __restrict__ hit,
+                                                              int K, int Hr, int64_t max_select,
                                                               const SeqPos lens, const SeqPos ncl_b,
                                                               int32_t* __restrict__ chunk,
                                                               uint32_t* __restrict__ ticket,
@@ -265,15 +294,14 @@ __global__ void __launch_bounds__(kClThreads) cl_count_kernel(const uint16_t* __
                                                               uint32_t* __restrict__ err) {
   __shared__ uint8_t s_hit[1024];
   __shared__ int s_red[32];
+  __shared__ long long s_scan[kClThreads];
   __shared__ bool s_last;
   const int p = blockIdx.y, b = p / Hr;
   const int64_t n = lens.v[b], ncl = ncl_b.v[b];
   const int64_t j0 = (int64_t)blockIdx.x * kClChunk;
   for (int i = threadIdx.x; i < K; i += kClThreads) s_hit[i] = hit[(int64_t)p * K + i];
   __syncthreads();
-  const uint16_t* asg = assign + (int64_t)p * max_seq;
-  int c = 0;
-  for (int i = threadIdx.x; i < kClChunk; i += kClThreads) c += cl_take(asg, s_hit, j0 + i, ncl, n) ? 1 : 0;
+  int c = __popc(cl_mask(assign + (int64_t)p * a_stride, s_hit, j0 + (int64_t)threadIdx.x * kClPer, ncl, n));
   c = cl_block_reduce(c, s_red, ISum());
   const int nch = gridDim.x;
   if (threadIdx.x == 0) {
@@ -285,7 +313,6 @@ __global__ void __launch_bounds__(kClThreads) cl_count_kernel(const uint16_t* __
   if (!s_last) return;
   __threadfence();
   // exclusive scan of the nch counts, kClThreads at a time
-  __shared__ long long s_scan[kClThreads];
   long long base = 0;
   for (int t0 = 0; t0 < nch; t0 += kClThreads) {
     const int t = t0 + threadIdx.x;
@@ -309,41 +336,43 @@ __global__ void __launch_bounds__(kClThreads) cl_count_kernel(const uint16_t* __
   }
 }
 
-// Ordered write of the selected positions: positions of a chunk go in blocks of kClThreads, one
-// per thread; warp ballots and a scan of the per-warp counts give each its slot.
+// Ordered write of the selected positions: thread t owns positions j0 + 16 t .. j0 + 16 t + 15;
+// a block scan of the per-thread counts gives each thread its first slot.
 __global__ void __launch_bounds__(kClThreads) cl_write_kernel(const uint16_t* __restrict__ assign,
-                                                              const uint8_t* __restrict__ hit, int K, int Hr,
-                                                              int64_t max_seq, int64_t max_select,
+                                                              int64_t a_stride, const uint8_t* __restrict__ hit,
+                                                              int K, int Hr, int64_t max_select,
                                                               const SeqPos lens, const SeqPos ncl_b,
                                                               const int32_t* __restrict__ chunk,
                                                               int32_t* __restrict__ sel_idx) {
   __shared__ uint8_t s_hit[1024];
-  __shared__ int s_wc[kClThreads / 32];
+  __shared__ int s_wsum[kClThreads / 32];
   const int p = blockIdx.y, b = p / Hr;
   const int64_t n = lens.v[b], ncl = ncl_b.v[b];
   const int64_t j0 = (int64_t)blockIdx.x * kClChunk;
   if (j0 >= n) return;
   for (int i = threadIdx.x; i < K; i += kClThreads) s_hit[i] = hit[(int64_t)p * K + i];
   __syncthreads();
-  const uint16_t* asg = assign + (int64_t)p * max_seq;
-  int32_t* dst = sel_idx + (int64_t)p * max_select;
+  const int64_t jb = j0 + (int64_t)threadIdx.x * kClPer;
+  uint32_t msk = cl_mask(assign + (int64_t)p * a_stride, s_hit, jb, ncl, n);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int64_t base = chunk[(int64_t)p * gridDim.x + blockIdx.x];
-  for (int i0 = 0; i0 < kClChunk; i0 += kClThreads) {
-    const int64_t j = j0 + i0 + threadIdx.x;
-    const bool t = cl_take(asg, s_hit, j, ncl, n);
-    const uint32_t bal = __ballot_sync(0xffffffffu, t);
-    if (lane == 0) s_wc[warp] = __popc(bal);
-    __syncthreads();
-    int off = 0, tot = 0;
-    for (int w = 0; w < kClThreads / 32; ++w) {
-      off += w < warp ? s_wc[w] : 0;
-      tot += s_wc[w];
-    }
-    const int64_t slot = base + off + __popc(bal & ((1u << lane) - 1u));
-    if (t && slot < max_select) dst[slot] = (int32_t)j;
-    base += tot;
-    __syncthreads();
+  const int c = __popc(msk);
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_wsum[warp] = incl;
+  __syncthreads();
+  int off = incl - c;
+  for (int w = 0; w < warp; ++w) off += s_wsum[w];
+  int64_t slot = (int64_t)chunk[(int64_t)p * gridDim.x + blockIdx.x] + off;
+  int32_t* dst = sel_idx + (int64_t)p * max_select;
+  while (msk) {
+    const int i = __ffs(msk) - 1;
+    msk &= msk - 1u;
+    if (slot < max_select) dst[slot] = (int32_t)(jb + i);
+    ++slot;
   }
 }
 
@@ -368,14 +397,14 @@ cudaError_t launch_cluster_build(rtp_layer* L, int iters, cudaStream_t st) {
   for (int it = 0; it <= iters && e == cudaSuccess; ++it) {
     {
       ProfScope ps(L, "cluster_assign", st);
-      cl_assign_kernel<<<ga, kClThreads, smem_a, st>>>(L->idx_b, L->cl_cent, L->cl_assign, K, L->Hr, L->max_seq,
-                                                       lens);
+      cl_assign_kernel<<<ga, kClThreads, smem_a, st>>>(L->idx_b, L->cl_cent, L->cl_assign, L->cl_stride, K, L->Hr,
+                                                       L->max_seq, lens);
       e = cudaGetLastError();
     }
     if (e != cudaSuccess) break;
     {
       ProfScope ps(L, "cluster_accum", st);
-      cl_accum_kernel<<<gs, kClThreads, smem_s, st>>>(L->idx_b, L->cl_assign, L->cl_sum, L->cl_acc, K, L->Hr,
+      cl_accum_kernel<<<gs, kClThreads, smem_s, st>>>(L->idx_b, L->cl_assign, L->cl_stride, L->cl_sum, L->cl_acc, K, L->Hr,
                                                       L->max_seq, lens, L->err);
       e = cudaGetLastError();
     }
@@ -397,21 +426,21 @@ cudaError_t launch_cluster_select(rtp_layer* L, cudaStream_t st) {
   cudaError_t e;
   {
     ProfScope ps(L, "cluster_select", st);
-    cl_select_kernel<<<P, kClSelThreads, 0, st>>>(L->q_idx, L->cl_cent, L->cl_count, K, L->top_p, L->cl_hit,
+    cl_select_kernel<<<P, (K + 31) / 32 * 32, 0, st>>>(L->q_idx, L->cl_cent, L->cl_count, K, L->top_p, L->cl_hit,
                                                   L->sel_mass, L->sel_thr);
     e = cudaGetLastError();
   }
   const dim3 g((unsigned)((L->len + kClChunk - 1) / kClChunk), (unsigned)P);
   if (e == cudaSuccess) {
     ProfScope ps(L, "cluster_count", st);
-    cl_count_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_hit, K, L->Hr, L->max_seq, L->max_select, lens, ncl,
-                                              L->cl_chunk, L->cl_ticket, L->sel_cnt, L->err);
+    cl_count_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_stride, L->cl_hit, K, L->Hr, L->max_select, lens,
+                                              ncl, L->cl_chunk, L->cl_ticket, L->sel_cnt, L->err);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) {
     ProfScope ps(L, "cluster_write", st);
-    cl_write_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_hit, K, L->Hr, L->max_seq, L->max_select, lens, ncl,
-                                              L->cl_chunk, L->sel_idx);
+    cl_write_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_stride, L->cl_hit, K, L->Hr, L->max_select, lens,
+                                              ncl, L->cl_chunk, L->sel_idx);
     e = cudaGetLastError();
   }
   return e;

@@ -30,9 +30,10 @@ constexpr int kSelMaxGrid = 256; // CTAs of the selection grid (<= SM count)
 // difference to zero gives 0.527.
 constexpr double kSelEvenShare = 0.527;
 
-// Sparse-attention gather (decode): indices per work item.
+// Sparse-attention gather (decode): the item kernel's chunk of selected positions and its
+// item cap per problem (the flat kernel needs two partials per CTA).
 constexpr int kGatherChunk = 128;
-constexpr int kGatherThreads = 256;
+constexpr int kGatherMaxItems = 64;
 
 // Prefill selection: keys of a row's crossing range captured per refinement walk.
 constexpr int kPfCapture = 2048;
@@ -143,7 +144,8 @@ struct rtp_layer {
   std::vector<int64_t> cl_len;           // [B] keys clustered per sequence
   double* cl_cent = nullptr;             // [P][K][r] fp64 centres
   int32_t* cl_count = nullptr;           // [P][K] cluster sizes
-  uint16_t* cl_assign = nullptr;         // [P][max_seq] cluster of each clustered key
+  uint16_t* cl_assign = nullptr;         // [P][cl_stride] cluster of each clustered key
+  int64_t cl_stride = 0;                 // max_seq rounded up to 16 entries (32-byte rows)
   unsigned long long* cl_sum = nullptr;  // [P][K][r] integer centre sums (two's complement)
   unsigned long long* cl_acc = nullptr;  // [P][K] counts being accumulated
   uint8_t* cl_hit = nullptr;             // [P][K] clusters hit by the current decode query
@@ -185,7 +187,9 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st);
 cudaError_t launch_decode_topk(rtp_layer* L, cudaStream_t st);
 cudaError_t launch_prefill_dense_retrieval(const rtp_layer* L, int C, float* out, cudaStream_t st);
 cudaError_t launch_prefill_dense_stats(const rtp_layer* L, int C, int32_t* cnt, float* mass, cudaStream_t st);
-cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, float* out, cudaStream_t st);
+// flat: the streaming kernel for long lists (p = 1, fixed top-k, clustered selection); else the
+// item kernel for the short lists of per-key top-p
+cudaError_t launch_decode_gather(const rtp_layer* L, bool dense, bool flat, float* out, cudaStream_t st);
 cudaError_t launch_dense_stats(const rtp_layer* L, cudaStream_t st);
 cudaError_t launch_iota_rows(const rtp_layer* L, int32_t* dst, int64_t cap, cudaStream_t st);
 cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st);

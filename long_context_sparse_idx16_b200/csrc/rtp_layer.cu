@@ -226,7 +226,11 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
   // selection keeps scores in global scratch.
   const int64_t smem_cap = ((int64_t)L->smem_optin - (int64_t)select_fixed_smem() - 2 * 32 * 34 - 2) * 4 / 19;
   const bool need_gscores = P * L->max_seq > smem_cap * G;
-  const int64_t gitems = P * ((L->max_seq + kGatherChunk - 1) / kGatherChunk);
+  // gather partials: the item kernel's items (at most 64 per problem), or two per CTA of the
+  // flat kernel
+  const int64_t gchunks = (L->max_seq + kGatherChunk - 1) / kGatherChunk;
+  const int64_t gitems_i = P * (gchunks < kGatherMaxItems ? gchunks : kGatherMaxItems);
+  const int64_t gitems = gitems_i > 2 * G ? gitems_i : 2 * G;
 
 #define RTP_ALLOC(ptr, n)                                         \
   do {                                                            \
@@ -285,7 +289,8 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
     const int64_t K = L->n_clusters;
     RTP_ALLOC(L->cl_cent, P * K * kR);
     RTP_ALLOC(L->cl_count, P * K);
-    RTP_ALLOC(L->cl_assign, P * L->max_seq);
+    L->cl_stride = (L->max_seq + 15) / 16 * 16;
+    RTP_ALLOC(L->cl_assign, P * L->cl_stride);
     RTP_ALLOC(L->cl_sum, P * K * kR);
     RTP_ALLOC(L->cl_acc, P * K);
     RTP_ALLOC(L->cl_hit, P * K);
@@ -462,7 +467,7 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
     }
     {
       ProfScope ps(L, "decode_gather", stream);
-      e = launch_decode_gather(L, dense, out, stream);
+      e = launch_decode_gather(L, dense, dense || L->top_k > 0 || L->cl_ready, out, stream);
     }
     if (e != cudaSuccess) {
       if (forked) cudaStreamWaitEvent(stream, L->ev_join, 0);
@@ -635,6 +640,7 @@ rtp_status rtp_get_clusters(const rtp_layer* L, rtp_cluster_view* view) {
   view->n_clusters = L->n_clusters;
   view->ready = L->cl_ready ? 1 : 0;
   view->max_seq = L->max_seq;
+  view->assign_stride = L->cl_stride;
   return RTP_OK;
 }
 

@@ -50,9 +50,9 @@ int main(void) {
          offsetof(rtp_config, rope_base), offsetof(rtp_config, wq_index),
          offsetof(rtp_config, max_select), offsetof(rtp_config, max_chunk),
          offsetof(rtp_config, index_bf16), offsetof(rtp_config, top_k));
-  printf("%zu %zu %zu %zu %zu\n", offsetof(rtp_config, n_clusters), sizeof(rtp_cluster_view),
+  printf("%zu %zu %zu %zu %zu %zu\n", offsetof(rtp_config, n_clusters), sizeof(rtp_cluster_view),
          offsetof(rtp_cluster_view, n_clusters), offsetof(rtp_cluster_view, ready),
-         offsetof(rtp_cluster_view, max_seq));
+         offsetof(rtp_cluster_view, max_seq), offsetof(rtp_cluster_view, assign_stride));
   printf("%zu %zu %zu %zu %zu %zu\n", sizeof(rtp_decode_stats), offsetof(rtp_decode_stats, sel_index_cap),
          sizeof(rtp_cache_view), offsetof(rtp_cache_view, idx_bf16), sizeof(rtp_prefill_stats),
          offsetof(rtp_prefill_stats, row_sel_cap));
@@ -71,7 +71,7 @@ int main(void) {
                                           cfg.index_bf16.offset, cfg.top_k.offset]
     cv = rtp.rtp_cluster_view
     assert [int(t) for t in c3.split()] == [cfg.n_clusters.offset, C.sizeof(cv), cv.n_clusters.offset,
-                                           cv.ready.offset, cv.max_seq.offset]
+                                           cv.ready.offset, cv.max_seq.offset, cv.assign_stride.offset]
     st = rtp.rtp_decode_stats
     ps = rtp.rtp_prefill_stats
     assert [int(t) for t in b.split()] == [C.sizeof(st), st.sel_index_cap.offset, C.sizeof(rtp.rtp_cache_view),

@@ -53,6 +53,17 @@ def test_decode_gqa_mha_and_wide_groups():
     run_decode(x)
 
 
+@pytest.mark.parametrize("p", [0.999, 1.0])
+def test_decode_long_selections_span_many_ctas(p):
+    # ~16K selected keys per problem: more than 64 gather chunks, so the gather's work items
+    # run over several chunks each (p = 1 through the dense path; p = 0.999 with all index
+    # scores tied, through the selected lists: the lowest ceil(0.999 N) positions)
+    x = synth.generate(synth.spec("decode_128k", batch=2, prefix=16383, needles=(), query_mode="gauss",
+                                  zero_index_weights=p < 1.0))
+    res = run_decode(x, top_p=p)
+    assert min(k for k, _, _ in res["summary"].values()) > 64 * 128
+
+
 def test_decode_128k_layer_short():
     # the 128K layer shape (B=8, 32/4 heads, 5 retrieval heads, W=8192) at 16K context
     x = synth.generate(synth.spec("decode_128k", prefix=16383,

@@ -84,11 +84,13 @@ def test_decode_ragged_fixed_top_k_and_bf16_keys():
     _ragged_decode(x, (4096, 500, 2000))
 
 
-def test_decode_ragged_128k_layer_shape():
-    # the 128K layer's shape (B=8, 32/4 heads, 5 retrieval heads) with eight different lengths
+@pytest.mark.parametrize("p", [0.9, 1.0])
+def test_decode_ragged_128k_layer_shape(p):
+    # the 128K layer's shape (B=8, 32/4 heads, 5 retrieval heads) with eight different lengths;
+    # at p = 1 the longer sequences span more than 64 gather chunks
     s = synth.spec("decode_128k", prefix=16383, needles=(1, 16, 1024, 1, 16, 1024, 1, 16))
     x = synth.generate(s)
-    _ragged_decode(x, (16384, 9000, 12345, 1, 16000, 8193, 4097, 300))
+    _ragged_decode(x, (16384, 9000, 12345, 1, 16000, 8193, 4097, 300), top_p=p)
 
 
 def test_prefill_ragged_lengths():
