@@ -545,20 +545,50 @@ def _timed(step, steps: int, world: int, dev):
     return _max_over_ranks(e0.elapsed_time(e1), world, dev)
 
 
-def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=None, cpu: bool = True):
+def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=None, cpu: bool = True,
+                   cluster_k: int = 0, cluster_iters: int = 4):
     """Decode lines of workload s, one per p in top_ps (default: the workload's p), all on one
     layer.  A step appends the B new tokens and decodes their B queries; before every step the
-    length is rolled back by one, so every step sees exactly N keys."""
+    length is rolled back by one, so every step sees exactly N keys.  cluster_k > 0: the first
+    N - 1 keys of every sequence are clustered into cluster_k clusters (timed once) and the
+    steps select by clusters; the key each step appends is kept as one cached after the
+    clustering."""
     import numpy as np
     import torch
 
     from long_context_sparse_idx16_b200 import Layer
 
     N, B = s.n_total, s.batch
-    layer = Layer.from_spec(s, x, max_seq=N, max_chunk=1)
+    layer = Layer.from_spec(s, x, max_seq=N, max_chunk=1, n_clusters=cluster_k)
     for t0 in range(0, N - 1, 1 << 16):
         t1 = min(N - 1, t0 + (1 << 16))
         layer.append_kv(_bf16(x.k[:, t0:t1]).to(dev), _bf16(x.v[:, t0:t1]).to(dev))
+    build = None
+    if cluster_k:
+        layer.cluster_build(cluster_iters)  # warm-up build
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        layer.cluster_build(cluster_iters)
+        e1.record()
+        torch.cuda.synchronize()
+        assert layer.check() == 0
+        layer.profile(True)
+        layer.profile_read()
+        layer.cluster_build(cluster_iters)
+        torch.cuda.synchronize()
+        bk = {}
+        for k in ("cluster_init", "cluster_assign", "cluster_accum", "cluster_update"):
+            kms, kn = layer.profile_read(k)
+            bk[k] = {"us_per_launch": kms * 1e3 / max(kn, 1), "launches": kn}
+        layer.profile(False)
+        P_ = B * len(s.retrieval_heads)
+        # fp64 work of one assignment pass: 16 subtractions + 16 fused multiply-adds per (key, centre)
+        flops = P_ * (N - 1) * cluster_k * 16 * 3
+        a_us = bk["cluster_assign"]["us_per_launch"]
+        build = {"ms": e0.elapsed_time(e1), "n_clusters": cluster_k, "iters": cluster_iters,
+                 "keys_per_problem": N - 1, "problems": P_, "kernels": bk,
+                 "assign_fp64_tflops": flops / (a_us * 1e-6) / 1e12}
     k_tok = _bf16(x.k[:, N - 1:N]).to(dev).contiguous()
     v_tok = _bf16(x.v[:, N - 1:N]).to(dev).contiguous()
     q = _bf16(x.q[:, 0]).to(dev).contiguous()
@@ -612,7 +642,8 @@ def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=Non
         sel_ms, sel_n = layer.profile_read("decode_select")
         kern = {"decode_select": {"us_per_launch": sel_ms * 1e3 / max(sel_n, 1), "launches": sel_n}}
         other_n = 0
-        for k in ("append_kv", "q_prep", "decode_topk", "decode_gather", "decode_swa", "swa_merge", "dense_fill"):
+        for k in ("append_kv", "q_prep", "decode_topk", "decode_gather", "decode_swa", "swa_merge", "dense_fill",
+                  "cluster_select", "cluster_count", "cluster_write"):
             kms, kn = layer.profile_read(k)
             if kn:
                 kern[k] = {"us_per_launch": kms * 1e3 / kn, "launches": kn}
@@ -626,19 +657,31 @@ def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=Non
         assert np.isfinite(o_h.numpy()).all()
         tokens = B * steps * world
         sel_us = sel_ms * 1e3 / max(sel_n, 1)
-        achieved = sel_bytes / (sel_us * 1e-6) / 1e9
+        achieved = sel_bytes / (sel_us * 1e-6) / 1e9 if sel_us > 0 else 0.0
         win_keys = min(N, s.window + s.n_sink)
         # whole-step algorithmic bytes: index keys + window/sink K/V rows + selected K/V rows
         step_bytes = sel_bytes + B * s.n_kv_heads * win_keys * 512 + int(counts.sum()) * 512
+        roof = {"bound": "hbm", "kernel": "decode_select (fused index stream + exact top-p)",
+                "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": achieved / peak,
+                # the capture streams fp32 keys; its bytes scale with the keys streamed
+                "traffic": (traffic * P * N / _TRAFFIC_KEYS if traffic and key_bytes == 4 else None),
+                "bytes_per_launch": sel_bytes, "us_per_launch": sel_us}
+        if cluster_k:
+            # the clusters' keys replace the index stream: centres, one 2-byte assignment per
+            # clustered key, then the selected K/V rows through the flat gather (the dominant kernel)
+            g_us = kern["decode_gather"]["us_per_launch"]
+            g_bytes = int(counts.sum()) * 512
+            g_ach = g_bytes / (g_us * 1e-6) / 1e9
+            roof = {"bound": "hbm", "kernel": "decode_gather (flat stream of the hit clusters' K/V rows)",
+                    "achieved": g_ach, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": g_ach / peak,
+                    "traffic": None, "bytes_per_launch": g_bytes, "us_per_launch": g_us}
+            step_bytes = (P * cluster_k * s.index_dim * 8 + P * (N - 1) * 2 + B * s.n_kv_heads * win_keys * 512
+                          + int(counts.sum()) * 512)
         lines.append({
             "value": ms * 1e3 / tokens, "unit": "us/token", "top_p": p, "steps": steps, "warmup": warmup,
             "ms_per_step": ms / steps, "config": _config(s, world),
-            "roofline": {"bound": "hbm", "kernel": "decode_select (fused index stream + exact top-p)",
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak,
-                         # the capture streams fp32 keys; its bytes scale with the keys streamed
-                         "traffic": (traffic * P * N / _TRAFFIC_KEYS if traffic and key_bytes == 4 else None),
-                         "bytes_per_launch": sel_bytes, "us_per_launch": sel_us},
+            "roofline": roof,
             "step_roofline": {"bytes_per_step": step_bytes, "roofline_us_per_step": step_bytes / (peak * 1e9) * 1e6,
                               "frac": step_bytes / (peak * 1e9) / (ms / steps * 1e-3)},
             "e2e": {"value": e2e_ms * 1e3 / tokens, "unit": "us/token",
@@ -650,8 +693,10 @@ def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=Non
                                 "max": int(counts.max())},
             "clocks": clk,
         })
+        if build:
+            lines[-1]["cluster_build"] = build
     layer.close()
-    if cpu:
+    if cpu and not cluster_k:
         v, cores, desc = cpu_oracle_sample(x)
         for ln in lines:
             ln["cpu_baseline"] = {"value": v, "unit": "us/token", "cores": cores, "kind": "oracle",
@@ -779,8 +824,12 @@ def measure_prefill(s, x, steps: int, warmup: int, world: int, dev, exp_peak: di
 
 # the workloads measured besides the headline one: (record name, workload, layer options,
 # the steps each takes at most -- a 1M prefill chunk takes about a second -- and the p values)
+# Layer-only options: cluster_k (K-cache clustering with that many clusters; K = 128 is the
+# page's example, 256 at 1M keeps about 4K keys per cluster).
 SUB_WORKLOADS = (("decode_1m", "decode_1m", {}, None, None),
                  ("decode_1m_bf16_index", "decode_1m", {"index_bf16": True}, None, (0.9,)),
+                 ("decode_1m_clustered", "decode_1m", {"index_bf16": True, "cluster_k": 256}, None, (0.9,)),
+                 ("decode_128k_clustered", "decode_128k", {"index_bf16": True, "cluster_k": 128}, None, None),
                  ("prefill_32k", "prefill_32k", {}, 5, None),
                  ("prefill_1m", "prefill_1m", {}, 3, None))
 
@@ -801,18 +850,29 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     cpu = rank == 0 and not args.no_cpu_baseline
     exp_peak = measure_exp_rate(dev)
+    decode_wl = args.workload in DECODE_WORKLOADS
+
+    generated = {}
 
     def one(name, steps, opts=None, ps=None):
+        opts = dict(opts or {})
+        layer_opts = {k: opts.pop(k) for k in list(opts) if k.startswith("cluster_")}
         s = _spec(args, name)
         if opts:
             s = dataclasses.replace(s, **opts)
-        x = synth.generate(s)
+        key = (name, tuple(sorted(opts.items())))
+        if key not in generated:  # inputs shared by the records of one spec
+            generated.clear()
+            generated[key] = synth.generate(s)
+        x = generated[key]
         if name in PREFILL_WORKLOADS:
             return [measure_prefill(s, x, steps, args.warmup, world, dev, exp_peak, cpu=cpu)]
         ps = ps or (list(s.p_sweep) if s.p_sweep else None)
-        return measure_decode(s, x, steps, args.warmup, world, dev, top_ps=list(ps) if ps else None, cpu=cpu)
+        return measure_decode(s, x, steps, args.warmup, world, dev, top_ps=list(ps) if ps else None, cpu=cpu,
+                              **layer_opts)
 
-    head = one(args.workload, args.steps)
+    head = one(args.workload, args.steps,
+               {"index_bf16": True, "cluster_k": args.cluster_k} if args.cluster_k and decode_wl else None)
     main = head[len(head) // 2] if args.workload == "decode_1m" else head[0]  # p = 0.9 of a sweep
     decode = args.workload in DECODE_WORKLOADS
     line = {"metric": METRIC, "value": main["value"], "unit": main["unit"], "n_gpus": world, "steps": args.steps,
@@ -822,6 +882,8 @@ def run_gpu(args):
     line.update({k: v for k, v in main.items() if k not in ("value", "unit", "steps", "warmup", "ms_per_step")})
     if args.workload == "decode_1m":
         line["p_sweep"] = {f"p={ln['top_p']}": ln for ln in head}
+    if args.cluster_k and decode_wl:
+        line["layer_options"] = {"index_bf16": True, "n_clusters": args.cluster_k}
     line["exp_peak"] = exp_peak
     if not args.only:
         subs = {}
@@ -857,6 +919,9 @@ def main():
                     help="measure the headline workload alone (no sub-records for the other workloads)")
     ap.add_argument("--batch", type=int, default=0, help="override the sequence count (profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cluster-k", type=int, default=0,
+                    help="decode workloads: K-cache clustering with K clusters (bf16 index keys) for the headline "
+                         "workload (profiling cases)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
