@@ -85,7 +85,15 @@ struct SelectArgs {
   const float* idx;           // fp32 index keys, or
   const __nv_bfloat16* idx_b; // bf16 index keys (one of the two is set)
   int64_t idx_pstride;  // floats between problems (max_seq * r)
-  const float* q_idx;   // [P][r]
+  const float* q_idx;   // [P][r], read when q_raw is NULL
+  // With q_raw set the kernel also does the query preparation: it writes the RoPE'd rows of
+  // every head (q_rot, for the attention kernels) and forms its own segments' index queries.
+  const __nv_bfloat16* q_raw;  // [B][Hq][D] pre-RoPE decode queries, or NULL
+  const double* theta;         // [D/2] RoPE frequencies
+  const float* wq;             // [Hr][D][r]
+  const int16_t* ret_head;     // [Hr] query head of each retrieval slot
+  int Hq;
+  float* q_rot;                // [B][Hq][D]
   int P;
   int64_t N;
   int64_t L;   // keys of the longest CTA range (sizes the shared-memory score array)
@@ -582,6 +590,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   }
   __syncthreads();
 
+  // ---- query preparation (q_raw set).  The index queries of this CTA's segments live in the
+  // candidate buffer, which is not used before the cut.
+  float* s_qt = reinterpret_cast<float*>(S.sk);  // [kSelMaxSeg][r]
+  if (a.q_raw) {
+    // RoPE'd rows b * Hq + h, 128 threads per row (rows spread over all CTAs): first half
+    // x cos - partner sin, second half x cos + partner sin, the angle reduced in fp64
+    const int n_rows = a.P / a.Hr * a.Hq, d = tid & (kD - 1);
+    for (int r = blockIdx.x * (kThreads / kD) + tid / kD; r < n_rows; r += gridDim.x * (kThreads / kD)) {
+      const int b = r / a.Hq;
+      const __nv_bfloat16* qr = a.q_raw + (int64_t)r * kD;
+      const float x = __bfloat162float(qr[d]), xp = __bfloat162float(qr[d ^ kHalfD]);
+      float cs, sn;
+      rope_cos_sin((int64_t)a.lens.v[b] - 1, a.theta[d & (kHalfD - 1)], &cs, &sn);
+      a.q_rot[(int64_t)r * kD + d] = d < kHalfD ? x * cs - xp * sn : x * cs + xp * sn;
+    }
+    // index query of segment w (warp w): lane l holds dims 4l .. 4l + 3 of q and their 16
+    // weights each, then the 16 sums are reduced over the warp
+    if (warp < nseg) {
+      const int p = S.seg[warp].p, hr = p % a.Hr;
+      const __nv_bfloat16* qr = a.q_raw + ((int64_t)(p / a.Hr) * a.Hq + a.ret_head[hr]) * kD + 4 * lane;
+      const float4* w4 = reinterpret_cast<const float4*>(a.wq + ((int64_t)hr * kD + 4 * lane) * kR);
+      float acc[kR];
+#pragma unroll
+      for (int o = 0; o < kR; ++o) acc[o] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float x = __bfloat162float(qr[i]);
+#pragma unroll
+        for (int o4 = 0; o4 < kR / 4; ++o4) {
+          const float4 w = w4[i * (kR / 4) + o4];
+          acc[4 * o4] = fmaf(x, w.x, acc[4 * o4]);
+          acc[4 * o4 + 1] = fmaf(x, w.y, acc[4 * o4 + 1]);
+          acc[4 * o4 + 2] = fmaf(x, w.z, acc[4 * o4 + 2]);
+          acc[4 * o4 + 3] = fmaf(x, w.w, acc[4 * o4 + 3]);
+        }
+      }
+#pragma unroll
+      for (int o = 0; o < kR; ++o) {
+#pragma unroll
+        for (int sh = 16; sh >= 1; sh >>= 1) acc[o] += __shfl_xor_sync(0xffffffffu, acc[o], sh);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int o = 0; o < kR; ++o) s_qt[warp * kR + o] = acc[o];
+      }
+    }
+    __syncthreads();
+  }
+
   // ---- phase A: stream index keys -> scores, segment maxima.  fp32 keys: four threads per
   // 64-byte key row, 16 bytes each; bf16 keys: two threads per 32-byte row.
   constexpr int kPer = kBf16 ? 2 : 4;      // threads per key
@@ -596,7 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
                               : reinterpret_cast<const float4*>(a.idx + (int64_t)s.p * a.idx_pstride) + s.jlo * 4;
     float qv[kBf16 ? 8 : 4];
     {
-      const float4* qp = reinterpret_cast<const float4*>(a.q_idx + (int64_t)s.p * kR) + part * (kBf16 ? 2 : 1);
+      const float4* qp = reinterpret_cast<const float4*>(a.q_raw ? s_qt + si * kR : a.q_idx + (int64_t)s.p * kR) +
+                         part * (kBf16 ? 2 : 1);
 #pragma unroll
       for (int i = 0; i < (kBf16 ? 2 : 1); ++i) {
         const float4 q4 = qp[i];
@@ -1198,7 +1256,7 @@ SelectGeom select_geometry(const rtp_layer* L, int64_t N) {
   return g;
 }
 
-cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
+cudaError_t launch_decode_select(rtp_layer* L, const __nv_bfloat16* q_raw, cudaStream_t st) {
   const int64_t N = L->len;
   const SelectGeom g = select_geometry(L, N);
   SelectArgs a;
@@ -1206,6 +1264,12 @@ cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st) {
   a.idx_b = L->idx_b;
   a.idx_pstride = L->max_seq * kR;
   a.q_idx = L->q_idx;
+  a.q_raw = q_raw;
+  a.theta = L->theta;
+  a.wq = L->wq;
+  a.ret_head = L->d_ret_head;
+  a.Hq = L->Hq;
+  a.q_rot = L->q_rot;
   a.P = L->B * L->Hr;
   a.N = N;
   a.L = g.per_cta;

@@ -183,7 +183,9 @@ cudaError_t launch_append_kv(const rtp_layer* L, const __nv_bfloat16* k, const _
                              int nb, cudaStream_t st);
 cudaError_t launch_q_prep(const rtp_layer* L, const __nv_bfloat16* q, int rows, const SeqPos& pos0,
                           cudaStream_t st);
-cudaError_t launch_decode_select(rtp_layer* L, cudaStream_t st);
+// q_raw: the decode queries ([B][Hq][D] bf16): the kernel then also writes q_rot and forms its
+// own index queries (no q_prep launch); NULL: it reads q_idx written by q_prep
+cudaError_t launch_decode_select(rtp_layer* L, const __nv_bfloat16* q_raw, cudaStream_t st);
 cudaError_t launch_decode_topk(rtp_layer* L, cudaStream_t st);
 cudaError_t launch_prefill_dense_retrieval(const rtp_layer* L, int C, float* out, cudaStream_t st);
 cudaError_t launch_prefill_dense_stats(const rtp_layer* L, int C, int32_t* cnt, float* mass, cudaStream_t st);

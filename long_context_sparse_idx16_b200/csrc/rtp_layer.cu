@@ -439,8 +439,11 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
   if (!L) return fail(nullptr, RTP_EINVAL, "rtp_decode: layer is NULL");
   if (!q || !out) return fail(L, RTP_EINVAL, "rtp_decode: q or out is NULL");
   if (min_len(L) < 1) return fail(L, RTP_EINVAL, "rtp_decode: a sequence is empty (append its token first)");
-  cudaError_t e;
-  {
+  cudaError_t e = cudaSuccess;
+  // per-key top-p: the selection kernel prepares the queries itself (RoPE'd rows for the
+  // attention kernels, its own index queries), so no query-prep launch precedes it
+  const bool per_key = L->Hr > 0 && L->top_k == 0 && L->top_p < 1.f && !L->cl_ready;
+  if (!per_key) {
     ProfScope ps(L, "q_prep", stream);
     e = launch_q_prep(L, (const __nv_bfloat16*)q, 1, seq_pos(L, -1), stream);
   }
@@ -454,10 +457,11 @@ rtp_status rtp_decode(rtp_layer* L, const void* q, float* out, const rtp_decode_
     } else {
       ProfScope ps(L, dense ? "dense_fill" : (L->top_k > 0 ? "decode_topk" : "decode_select"), stream);
       e = dense ? launch_dense_stats(L, stream)
-                : (L->top_k > 0 ? launch_decode_topk(L, stream) : launch_decode_select(L, stream));
+                : (L->top_k > 0 ? launch_decode_topk(L, stream)
+                                : launch_decode_select(L, (const __nv_bfloat16*)q, stream));
     }
     if (e != cudaSuccess) return cuda_fail(L, e, "rtp_decode: select");
-    if (L->n_local > 0 && !L->prof_on) {  // the window attention needs only q_prep: fork it off
+    if (L->n_local > 0 && !L->prof_on) {  // the window attention needs only the RoPE'd queries: fork it off
       e = cudaEventRecord(L->ev_fork, stream);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_fork, 0);
       if (e == cudaSuccess) e = launch_decode_swa(L, out, L->side);
