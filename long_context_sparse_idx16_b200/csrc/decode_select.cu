@@ -590,21 +590,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
   }
   __syncthreads();
 
-  // ---- query preparation (q_raw set).  The index queries of this CTA's segments live in the
-  // candidate buffer, which is not used before the cut.
+  // ---- query preparation (q_raw set), first part: the index queries of this CTA's segments,
+  // kept in the candidate buffer (not used before the cut).  The RoPE'd rows follow the stream.
   float* s_qt = reinterpret_cast<float*>(S.sk);  // [kSelMaxSeg][r]
   if (a.q_raw) {
-    // RoPE'd rows b * Hq + h, 128 threads per row (rows spread over all CTAs): first half
-    // x cos - partner sin, second half x cos + partner sin, the angle reduced in fp64
-    const int n_rows = a.P / a.Hr * a.Hq, d = tid & (kD - 1);
-    for (int r = blockIdx.x * (kThreads / kD) + tid / kD; r < n_rows; r += gridDim.x * (kThreads / kD)) {
-      const int b = r / a.Hq;
-      const __nv_bfloat16* qr = a.q_raw + (int64_t)r * kD;
-      const float x = __bfloat162float(qr[d]), xp = __bfloat162float(qr[d ^ kHalfD]);
-      float cs, sn;
-      rope_cos_sin((int64_t)a.lens.v[b] - 1, a.theta[d & (kHalfD - 1)], &cs, &sn);
-      a.q_rot[(int64_t)r * kD + d] = d < kHalfD ? x * cs - xp * sn : x * cs + xp * sn;
-    }
     // index query of segment w (warp w): lane l holds dims 4l .. 4l + 3 of q and their 16
     // weights each, then the 16 sums are reduced over the warp
     if (warp < nseg) {
@@ -712,6 +701,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_select_kernel(SelectArgs a
     }
     mx = block_max(mx, S);
     if (tid == 0) a.seg_max[s.p + c] = mx;
+  }
+  if (a.q_raw) {
+    // query preparation, second part, while the slowest CTAs finish the stream: RoPE'd rows
+    // b * Hq + h for the attention kernels, 128 threads per row (rows spread over all CTAs):
+    // first half x cos - partner sin, second half x cos + partner sin, the angle reduced in fp64
+    const int n_rows = a.P / a.Hr * a.Hq, d = tid & (kD - 1);
+    for (int r = blockIdx.x * (kThreads / kD) + tid / kD; r < n_rows; r += gridDim.x * (kThreads / kD)) {
+      const int b = r / a.Hq;
+      const __nv_bfloat16* qr = a.q_raw + (int64_t)r * kD;
+      const float x = __bfloat162float(qr[d]), xp = __bfloat162float(qr[d ^ kHalfD]);
+      float cs, sn;
+      rope_cos_sin((int64_t)a.lens.v[b] - 1, a.theta[d & (kHalfD - 1)], &cs, &sn);
+      a.q_rot[(int64_t)r * kD + d] = d < kHalfD ? x * cs - xp * sn : x * cs + xp * sn;
+    }
   }
   if (!grid_sync(a.bar, G, a.err, a.wait_limit)) return;
 
