@@ -117,7 +117,6 @@ def _check_clustered_decode(x, layer, K, iters, lens, ncl, p, heads=None):
         n = lens[b]
         for h in (heads or range(s.n_q_heads)):
             if h not in s.retrieval_heads:
-                slot0 = 0
                 r = oracle.head_rows(x.k[b, :n], x.v[b, :n], x.q[b, 0, h], [n - 1], g=s.kv_head(h), retrieval=False,
                                      wq=None, wk=None, top_p=1.0, top_k=0, window=s.window, n_sink=s.n_sink,
                                      rope_base=s.rope_base, index_bf16=True)
@@ -244,3 +243,57 @@ def test_cluster_build_errors():
     with pytest.raises(RTPError):  # created without n_clusters
         plain.cluster_build(1)
     plain.close()
+
+
+def test_clustered_decode_overflow_and_dense_override():
+    from long_context_sparse_idx16_b200 import RTP_EOVERFLOW
+
+    x = synth.generate(synth.spec("decode_128k", batch=1, prefix=4095, index_bf16=True))
+    N = x.spec.n_total
+    K, cap = 32, 200
+    from long_context_sparse_idx16_b200 import Layer
+
+    layer = Layer.from_spec(x.spec, x, max_seq=N, max_chunk=1, n_clusters=K, max_select=cap)
+    build_cache(layer, x, N)
+    layer.cluster_build(3)
+    layer.set_top_p(0.99)  # most clusters: far more than 200 keys
+    _, st = layer.decode(torch_bf16(x.q[:, 0]), stats=True, sel_cap=cap)
+    assert layer.check() == RTP_EOVERFLOW
+    cnt, idx = st[0].cpu().numpy(), st[3].cpu().numpy()
+    slot = 0
+    r = oracle.cluster_row(x, 0, x.spec.retrieval_heads[slot], N, K, 3, p32(0.99))
+    assert int(cnt[0, slot]) == cap and len(r.sel) > cap
+    assert np.array_equal(idx[0, slot, :cap], r.sel[:cap])  # the truncated list is the set's prefix
+    # p = 1 keeps every causal key whatever the clustering
+    layer.set_top_p(1.0)
+    _, st = layer.decode(torch_bf16(x.q[:, 0]), stats=True, sel_cap=cap)
+    assert layer.check() == 0 and np.all(st[0].cpu().numpy() == N)
+    layer.close()
+
+
+def test_every_key_its_own_cluster():
+    # K = n: every centre is its key, so the clusters taken are single keys ordered by score
+    x = synth.generate(synth.spec("toy_decode_4k", prefix=511, index_bf16=True))
+    N = x.spec.n_total
+    layer = _layer(x, N)
+    build_cache(layer, x, N)
+    layer.cluster_build(2)
+    assert layer.check() == 0
+    _check_build(x, layer, N, 2, [N])
+    _check_clustered_decode(x, layer, N, 2, [N], [N], 0.9)
+    layer.close()
+
+
+def test_index_key_outside_the_clustering_range_is_reported():
+    from long_context_sparse_idx16_b200 import RTP_ERANGE, Layer
+
+    s = synth.spec("toy_decode_4k", prefix=255, index_bf16=True)
+    x = synth.generate(s)
+    big = (x.wk * 40000.0).astype(np.float32)  # many index keys of magnitude above 2^15
+    layer = Layer(batch=s.batch, n_q_heads=s.n_q_heads, n_kv_heads=s.n_kv_heads, head_class=s.head_class,
+                  wq=x.wq, wk=big, top_p=s.top_p, window=s.window, n_sink=s.n_sink, max_seq=s.n_total,
+                  rope_base=s.rope_base, index_bf16=True, max_chunk=1, n_clusters=8)
+    build_cache(layer, x, s.n_total)
+    layer.cluster_build(1)
+    assert layer.check() == RTP_ERANGE
+    layer.close()
