@@ -646,7 +646,7 @@ def measure_decode(s, x, steps: int, warmup: int, world: int, dev, *, top_ps=Non
         kern = {"decode_select": {"us_per_launch": sel_ms * 1e3 / max(sel_n, 1), "launches": sel_n}}
         other_n = 0
         for k in ("append_kv", "q_prep", "decode_topk", "decode_gather", "decode_swa", "swa_merge", "dense_fill",
-                  "cluster_select", "cluster_count", "cluster_write"):
+                  "cluster_select", "cluster_compact"):
             kms, kn = layer.profile_read(k)
             if kn:
                 kern[k] = {"us_per_launch": kms * 1e3 / kn, "launches": kn}

@@ -18,8 +18,8 @@
 // Clustered decode: the centre scores c_k = q~ . mu_k (fp64, from the fp32 index query), the
 // cluster weights n_k exp(c_k - max c), the clusters taken in (c desc, k asc) order while the
 // weight before them is below p of the total; the selected set is every clustered key of a hit
-// cluster plus every key cached after the clustering, in ascending position order, which the
-// sparse-attention gather then attends to exactly.
+// cluster plus every key cached after the clustering, in ascending position order (one
+// single-pass compaction), which the sparse-attention gather then attends to exactly.
 #include "rtp_device.cuh"
 #include "rtp_internal.h"
 
@@ -282,78 +282,53 @@ __device__ __forceinline__ uint32_t cl_mask(const uint16_t* __restrict__ asg, co
   return msk;
 }
 
-// Per-chunk counts; the last CTA of a problem (ticket) turns them into exclusive offsets in
-// place and writes the set size.
-__global__ void __launch_bounds__(kClThreads) cl_count_kernel(const uint16_t* __restrict__ assign,
-                                                              int64_t a_stride, const uint8_t* __restrict__ hit,
-                                                              int K, int Hr, int64_t max_select,
-                                                              const SeqPos lens, const SeqPos ncl_b,
-                                                              int32_t* __restrict__ chunk,
-                                                              uint32_t* __restrict__ ticket,
-                                                              int32_t* __restrict__ sel_cnt,
-                                                              uint32_t* __restrict__ err) {
-  __shared__ uint8_t s_hit[1024];
-  __shared__ int s_red[32];
-  __shared__ long long s_scan[kClThreads];
-  __shared__ bool s_last;
-  const int p = blockIdx.y, b = p / Hr;
-  const int64_t n = lens.v[b], ncl = ncl_b.v[b];
-  const int64_t j0 = (int64_t)blockIdx.x * kClChunk;
-  for (int i = threadIdx.x; i < K; i += kClThreads) s_hit[i] = hit[(int64_t)p * K + i];
-  __syncthreads();
-  int c = __popc(cl_mask(assign + (int64_t)p * a_stride, s_hit, j0 + (int64_t)threadIdx.x * kClPer, ncl, n));
-  c = cl_block_reduce(c, s_red, ISum());
-  const int nch = gridDim.x;
-  if (threadIdx.x == 0) {
-    chunk[(int64_t)p * nch + blockIdx.x] = c;
-    __threadfence();
-    s_last = atomicAdd(&ticket[p], 1u) == (uint32_t)(nch - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // exclusive scan of the nch counts, kClThreads at a time
-  long long base = 0;
-  for (int t0 = 0; t0 < nch; t0 += kClThreads) {
-    const int t = t0 + threadIdx.x;
-    const long long v = t < nch ? (long long)*((volatile int32_t*)&chunk[(int64_t)p * nch + t]) : 0;
-    s_scan[threadIdx.x] = v;
-    __syncthreads();
-    for (int o = 1; o < kClThreads; o <<= 1) {
-      const long long add = threadIdx.x >= o ? s_scan[threadIdx.x - o] : 0;
-      __syncthreads();
-      s_scan[threadIdx.x] += add;
-      __syncthreads();
-    }
-    if (t < nch) chunk[(int64_t)p * nch + t] = (int32_t)(base + s_scan[threadIdx.x] - v);
-    base += s_scan[kClThreads - 1];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    sel_cnt[p] = (int32_t)(base < max_select ? base : max_select);
-    if (base > max_select) atomicOr(err, kErrOverflow);
-    ticket[p] = 0u;
-  }
+// Chunk flags of the single-pass compaction: launch epoch (24 bits) | status (2 bits: 1 the
+// chunk's own count, 2 the inclusive count of chunks 0 .. this one) | value (38 bits).
+constexpr int kFlagEpochBits = 24;
+constexpr unsigned long long kFlagValueMask = (1ull << 38) - 1ull;
+
+__device__ __forceinline__ unsigned long long cl_flag(uint32_t epoch, uint32_t status, long long v) {
+  return ((unsigned long long)epoch << 40) | ((unsigned long long)status << 38) | ((unsigned long long)v & kFlagValueMask);
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
 
-// Ordered write of the selected positions: thread t owns positions j0 + 16 t .. j0 + 16 t + 15;
-// a block scan of the per-thread counts gives each thread its first slot.
-__global__ void __launch_bounds__(kClThreads) cl_write_kernel(const uint16_t* __restrict__ assign,
-                                                              int64_t a_stride, const uint8_t* __restrict__ hit,
-                                                              int K, int Hr, int64_t max_select,
-                                                              const SeqPos lens, const SeqPos ncl_b,
-                                                              const int32_t* __restrict__ chunk,
-                                                              int32_t* __restrict__ sel_idx) {
+// Single-pass ordered compaction of one problem's selected positions (chunks of kClChunk
+// positions, thread t of a chunk owning positions 16 t .. 16 t + 15).  A CTA takes the next
+// chunk of its problem from a counter, so every chunk it waits on belongs to a CTA that is
+// already running; it publishes its own count, then sums its predecessors' flags, 32 per step,
+// back to the first one that carries an inclusive count (decoupled look-back, every wait
+// bounded), publishes
+// its inclusive count and writes its positions.  The last chunk writes the set size; the last
+// CTA to finish resets the counters for the next launch.
+__global__ void __launch_bounds__(kClThreads) cl_compact_kernel(const uint16_t* __restrict__ assign,
+                                                                int64_t a_stride, const uint8_t* __restrict__ hit,
+                                                                int K, int Hr, int64_t max_select,
+                                                                const SeqPos lens, const SeqPos ncl_b,
+                                                                unsigned long long* __restrict__ flags,
+                                                                uint32_t* __restrict__ ctr, uint32_t epoch,
+                                                                long long wait_limit, int32_t* __restrict__ sel_idx,
+                                                                int32_t* __restrict__ sel_cnt,
+                                                                uint32_t* __restrict__ err) {
   __shared__ uint8_t s_hit[1024];
   __shared__ int s_wsum[kClThreads / 32];
-  const int p = blockIdx.y, b = p / Hr;
-  const int64_t n = lens.v[b], ncl = ncl_b.v[b];
-  const int64_t j0 = (int64_t)blockIdx.x * kClChunk;
-  if (j0 >= n) return;
+  __shared__ int s_chunk;
+  __shared__ long long s_base;
+  const int p = blockIdx.y, b = p / Hr, nch = gridDim.x;
+  if (threadIdx.x == 0) s_chunk = (int)atomicAdd(&ctr[2 * p], 1u);
   for (int i = threadIdx.x; i < K; i += kClThreads) s_hit[i] = hit[(int64_t)p * K + i];
   __syncthreads();
+  const int chunk = s_chunk;
+  const int64_t n = lens.v[b], ncl = ncl_b.v[b];
+  const int64_t j0 = (int64_t)chunk * kClChunk;
   const int64_t jb = j0 + (int64_t)threadIdx.x * kClPer;
-  uint32_t msk = cl_mask(assign + (int64_t)p * a_stride, s_hit, jb, ncl, n);
+  uint32_t msk = j0 < n ? cl_mask(assign + (int64_t)p * a_stride, s_hit, jb, ncl, n) : 0u;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c = __popc(msk);
   int incl = c;
@@ -364,15 +339,72 @@ __global__ void __launch_bounds__(kClThreads) cl_write_kernel(const uint16_t* __
   }
   if (lane == 31) s_wsum[warp] = incl;
   __syncthreads();
-  int off = incl - c;
-  for (int w = 0; w < warp; ++w) off += s_wsum[w];
-  int64_t slot = (int64_t)chunk[(int64_t)p * gridDim.x + blockIdx.x] + off;
+  int off = incl - c, tot = 0;
+  for (int w = 0; w < kClThreads / 32; ++w) {
+    off += w < warp ? s_wsum[w] : 0;
+    tot += s_wsum[w];
+  }
+  if (warp == 0) {
+    // warp 0: publish this chunk's count, then look back 32 predecessors at a time (lane l
+    // reads chunk top - l) down to the nearest one that carries an inclusive count
+    unsigned long long* fl = flags + (int64_t)p * nch;
+    long long prefix = 0;
+    if (chunk > 0) {
+      if (lane == 0) st_release_u64(fl + chunk, cl_flag(epoch, 1u, tot));
+      const long long t0 = clock64();
+      for (int top = chunk - 1; top >= 0;) {
+        const int j = top - lane;
+        unsigned long long f = 0ull;
+        bool ok = true, inc = true;  // before chunk 0: an inclusive count of 0
+        if (j >= 0) {
+          f = ld_acquire_u64(fl + j);
+          const uint32_t st = (uint32_t)(f >> 38) & 3u;
+          ok = (uint32_t)(f >> 40) == epoch && st != 0u;
+          inc = ok && st == 2u;
+        }
+        const uint32_t pub = __ballot_sync(0xffffffffu, ok), incm = __ballot_sync(0xffffffffu, inc);
+        const int L = incm ? __ffs(incm) - 1 : 31;  // lanes 0 .. L-1 add counts, lane L its inclusive
+        const uint32_t need = L == 31 ? 0xffffffffu : ((1u << (L + 1)) - 1u);
+        if ((pub & need) == need) {
+          long long v = (lane <= L && j >= 0) ? (long long)(f & kFlagValueMask) : 0;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          prefix += v;
+          if (incm) break;
+          top -= 32;
+        } else if (clock64() - t0 > wait_limit) {
+          if (lane == 0) atomicOr(err, kErrTimeout);  // the set of this call is invalid; rtp_check reports it
+          break;
+        } else {
+          __nanosleep(20);
+        }
+      }
+    }
+    if (lane == 0) {
+      st_release_u64(fl + chunk, cl_flag(epoch, 2u, prefix + tot));
+      s_base = prefix;
+      if (chunk == nch - 1) {
+        const long long total = prefix + tot;
+        sel_cnt[p] = (int32_t)(total < max_select ? total : max_select);
+        if (total > max_select) atomicOr(err, kErrOverflow);
+      }
+    }
+  }
+  __syncthreads();
+  int64_t slot = s_base + off;
   int32_t* dst = sel_idx + (int64_t)p * max_select;
   while (msk) {
     const int i = __ffs(msk) - 1;
     msk &= msk - 1u;
     if (slot < max_select) dst[slot] = (int32_t)(jb + i);
     ++slot;
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&ctr[2 * p + 1], 1u) == (uint32_t)(nch - 1)) {  // every chunk taken and done
+      ctr[2 * p] = 0u;
+      ctr[2 * p + 1] = 0u;
+    }
   }
 }
 
@@ -432,15 +464,17 @@ cudaError_t launch_cluster_select(rtp_layer* L, cudaStream_t st) {
   }
   const dim3 g((unsigned)((L->len + kClChunk - 1) / kClChunk), (unsigned)P);
   if (e == cudaSuccess) {
-    ProfScope ps(L, "cluster_count", st);
-    cl_count_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_stride, L->cl_hit, K, L->Hr, L->max_select, lens,
-                                              ncl, L->cl_chunk, L->cl_ticket, L->sel_cnt, L->err);
-    e = cudaGetLastError();
+    if (++L->cl_epoch >= (1u << kFlagEpochBits)) {  // epochs wrapped: clear every flag once
+      e = cudaMemsetAsync(L->cl_flags, 0, sizeof(unsigned long long) * (size_t)P * cluster_chunks(L->max_seq), st);
+      L->cl_epoch = 1u;
+    }
   }
   if (e == cudaSuccess) {
-    ProfScope ps(L, "cluster_write", st);
-    cl_write_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_stride, L->cl_hit, K, L->Hr, L->max_select, lens,
-                                              ncl, L->cl_chunk, L->sel_idx);
+    ProfScope ps(L, "cluster_compact", st);
+    cl_compact_kernel<<<g, kClThreads, 0, st>>>(L->cl_assign, L->cl_stride, L->cl_hit, K, L->Hr, L->max_select, lens,
+                                                ncl, L->cl_flags, L->cl_ctr, L->cl_epoch,
+                                                L->wait_limit > 0 ? L->wait_limit : kWaitLimitCycles, L->sel_idx,
+                                                L->sel_cnt, L->err);
     e = cudaGetLastError();
   }
   return e;

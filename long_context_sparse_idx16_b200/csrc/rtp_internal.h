@@ -149,8 +149,9 @@ struct rtp_layer {
   unsigned long long* cl_sum = nullptr;  // [P][K][r] integer centre sums (two's complement)
   unsigned long long* cl_acc = nullptr;  // [P][K] counts being accumulated
   uint8_t* cl_hit = nullptr;             // [P][K] clusters hit by the current decode query
-  int32_t* cl_chunk = nullptr;           // [P][max_seq / 4096] selected counts, then offsets
-  uint32_t* cl_ticket = nullptr;         // [P]
+  unsigned long long* cl_flags = nullptr;  // [P][max_seq / 4096] compaction chunk flags
+  uint32_t* cl_ctr = nullptr;              // [P][2] compaction chunk counter, finished chunks
+  uint32_t cl_epoch = 0;                   // compaction launches (flag epochs, 24 bits)
 
   // per-kernel event timing (rtp_profile_enable)
   bool prof_on = false;

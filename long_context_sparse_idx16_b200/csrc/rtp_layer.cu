@@ -103,7 +103,7 @@ static void free_all(rtp_layer* L) {
                   L->sel_keep, L->sel_flags, L->slot_cnt, L->bar, L->gscores, L->gpart, L->gticket, L->spart,
                   L->sticket, L->err, L->tk_keys, L->tk_hist, L->tk_cnt, L->pf_capture, L->attn_part,
                   L->attn_ticket, L->sel_cum, L->sel_psum, L->sel_pticket, L->sel_cres, L->cl_cent,
-                  L->cl_count, L->cl_assign, L->cl_sum, L->cl_acc, L->cl_hit, L->cl_chunk, L->cl_ticket};
+                  L->cl_count, L->cl_assign, L->cl_sum, L->cl_acc, L->cl_hit, L->cl_flags, L->cl_ctr};
   for (void* p : ptrs)
     if (p) cudaFree(p);
 }
@@ -294,9 +294,10 @@ rtp_status rtp_create(const rtp_config* cfg, rtp_layer** out) {
     RTP_ALLOC(L->cl_sum, P * K * kR);
     RTP_ALLOC(L->cl_acc, P * K);
     RTP_ALLOC(L->cl_hit, P * K);
-    RTP_ALLOC(L->cl_chunk, P * cluster_chunks(L->max_seq));
-    RTP_ALLOC(L->cl_ticket, P);
-    if (e == cudaSuccess) e = cudaMemset(L->cl_ticket, 0, sizeof(uint32_t) * (size_t)P);
+    RTP_ALLOC(L->cl_flags, P * cluster_chunks(L->max_seq));
+    RTP_ALLOC(L->cl_ctr, 2 * P);
+    if (e == cudaSuccess) e = cudaMemset(L->cl_flags, 0, sizeof(unsigned long long) * (size_t)(P * cluster_chunks(L->max_seq)));
+    if (e == cudaSuccess) e = cudaMemset(L->cl_ctr, 0, sizeof(uint32_t) * (size_t)(2 * P));
   }
   if (need_gscores) {
     L->gscores_elems = (size_t)(P * L->max_seq);
@@ -701,7 +702,7 @@ rtp_status rtp_check(rtp_layer* L, cudaStream_t stream) {
     // a barrier gave up: its counters are inconsistent; start the next launch from zero
     reset_select_scratch(L);
     cudaMemset(L->gticket, 0, sizeof(uint32_t) * (size_t)(L->B * L->Hr > 0 ? L->B * L->Hr : 1));
-    if (L->cl_ticket) cudaMemset(L->cl_ticket, 0, sizeof(uint32_t) * (size_t)(L->B * L->Hr));
+    if (L->cl_ctr) cudaMemset(L->cl_ctr, 0, sizeof(uint32_t) * (size_t)(2 * L->B * L->Hr));
     if (L->attn_ticket)
       cudaMemset(L->attn_ticket, 0, sizeof(uint32_t) * (size_t)L->B * L->Hr * ((L->max_chunk + 127) / 128));
     return fail(L, RTP_ETIMEOUT, "a bounded in-kernel wait gave up");
