@@ -190,7 +190,8 @@ rtp_status rtp_prefill_chunk(rtp_layer* layer, const void* q, int32_t C, float* 
 rtp_status rtp_set_top_p(rtp_layer* layer, float top_p);
 
 /* Test knob: the limit, in SM clock cycles, on each wait of the decode selection's grid-wide
- * barriers (0 restores the default, about one second).  A wait past its limit makes the
+ * barriers and of the clustered selection's compaction look-back (0 restores the default,
+ * about one second).  A wait past its limit makes the
  * kernel record RTP_ETIMEOUT and leave; the next rtp_check reports it and resets the
  * selection's scratch, so later calls start clean.  A tiny limit makes the barrier give up
  * at once, which is how the timeout path is tested.  The tensor-core completion waits of the
