@@ -194,9 +194,6 @@ struct DSum {
 struct IMax {
   __device__ int operator()(int a, int b) const { return a > b ? a : b; }
 };
-struct ISum {
-  __device__ int operator()(int a, int b) const { return a + b; }
-};
 
 // The coarse match of one problem's index query against its K centres: hit flags, the hit
 // clusters' weight fraction (sel_mass) and the weight fraction of the last cluster taken
