@@ -298,8 +298,8 @@ class ClusterRow:
 
 
 def cluster_row(inputs, b: int, h: int, n: int, K: int, iters: int, p: float,
-                n_clustered: Optional[int] = None) -> ClusterRow:
-    """The clustered selection and attention of the decode query of retrieval head h, sequence
+                n_clustered: Optional[int] = None, row: int = 0) -> ClusterRow:
+    """The clustered selection and attention of query row ``row`` of retrieval head h, sequence
     b, at position n - 1: keys 0 .. n_clustered - 1 clustered, the later ones always kept."""
     s = inputs.spec
     slot = s.retrieval_heads.index(h)
@@ -307,8 +307,8 @@ def cluster_row(inputs, b: int, h: int, n: int, K: int, iters: int, p: float,
     nc = n if n_clustered is None else n_clustered
     kt = index_keys_bf16(inputs.k[b], g, inputs.wk[slot], nc)
     cent, counts, assign = kmeans(kt, K, iters)
-    qt = index_query(inputs.q[b, 0, h], inputs.wq[slot])
+    qt = index_query(inputs.q[b, row, h], inputs.wq[slot])
     hit, w, wt = cluster_select(qt, cent, counts, p)
     sel = np.concatenate([np.flatnonzero(hit[assign]), np.arange(nc, n)]).astype(np.int64)
-    out = attend_set(inputs, b, h, 0, sel, pos=n - 1)
+    out = attend_set(inputs, b, h, row, sel, pos=n - 1)
     return ClusterRow(out, sel, hit, w, wt, cent, counts, assign)

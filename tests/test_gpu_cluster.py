@@ -103,10 +103,10 @@ def _order_before(r, qt):
     return before
 
 
-def _check_clustered_decode(x, layer, K, iters, lens, ncl, p, heads=None):
+def _check_clustered_decode(x, layer, K, iters, lens, ncl, p, heads=None, row=0):
     s = x.spec
     layer.set_top_p(p)
-    out, st = layer.decode(torch_bf16(x.q[:, 0]), stats=True, sel_cap=max(lens))
+    out, st = layer.decode(torch_bf16(x.q[:, row]), stats=True, sel_cap=max(lens))
     assert layer.check() == 0
     out = out.cpu().numpy()
     cnt, mass, thr, idx = (t.cpu().numpy() for t in (st[0], st[1], st[2], st[3]))
@@ -117,14 +117,14 @@ def _check_clustered_decode(x, layer, K, iters, lens, ncl, p, heads=None):
         n = lens[b]
         for h in (heads or range(s.n_q_heads)):
             if h not in s.retrieval_heads:
-                r = oracle.head_rows(x.k[b, :n], x.v[b, :n], x.q[b, 0, h], [n - 1], g=s.kv_head(h), retrieval=False,
+                r = oracle.head_rows(x.k[b, :n], x.v[b, :n], x.q[b, row, h], [n - 1], g=s.kv_head(h), retrieval=False,
                                      wq=None, wk=None, top_p=1.0, top_k=0, window=s.window, n_sink=s.n_sink,
                                      rope_base=s.rope_base, index_bf16=True)
                 gpus.append(out[b, h])
                 refs.append(r.out[0])
                 continue
             slot = s.retrieval_heads.index(h)
-            r = oracle.cluster_row(x, b, h, n, K, iters, p32(p), n_clustered=ncl[b])
+            r = oracle.cluster_row(x, b, h, n, K, iters, p32(p), n_clustered=ncl[b], row=row)
             k = int(cnt[b, slot])
             sel = idx[b, slot, :k].astype(np.int64)
             assert np.all(np.diff(sel) > 0), "selected positions must be strictly ascending"
@@ -135,12 +135,12 @@ def _check_clustered_decode(x, layer, K, iters, lens, ncl, p, heads=None):
             assert np.array_equal(sel, want), f"b={b} h={h}: the set is not a union of whole clusters"
             diff = np.flatnonzero(hit_gpu != r.hit)
             if len(diff):
-                qt = oracle.index_query(x.q[b, 0, h], x.wq[slot])
+                qt = oracle.index_query(x.q[b, row, h], x.wq[slot])
                 before = _order_before(r, qt)
                 bad = [int(c) for c in diff if not abs(before[c] - p32(p)) <= CUT_TOL]
                 assert not bad, f"b={b} h={h}: clusters {bad} differ beyond the cut tolerance"
                 n_moved += len(diff)
-                ref = oracle.attend_set(x, b, h, 0, sel, pos=n - 1)
+                ref = oracle.attend_set(x, b, h, row, sel, pos=n - 1)
             else:
                 assert abs(float(mass[b, slot]) - float(r.w[r.hit].sum())) <= W_TOL
                 assert abs(float(thr[b, slot]) - r.w_t) <= W_TOL
@@ -296,4 +296,28 @@ def test_index_key_outside_the_clustering_range_is_reported():
     build_cache(layer, x, s.n_total)
     layer.cluster_build(1)
     assert layer.check() == RTP_ERANGE
+    layer.close()
+
+
+def test_dense_prefill_then_clustered_decode():
+    # the page's own pipeline (aitntnews page, experiments): retrieval heads attend densely in
+    # prefill, the prefill's K cache is clustered, decode selects by clusters
+    from long_context_sparse_idx16_b200 import Layer
+
+    C, K = 2048, 64
+    s = synth.spec("prefill_32k", prefix=0, chunk=C + 1, window=512, index_bf16=True, prefill_dense=True)
+    x = synth.generate(s)
+    layer = Layer.from_spec(s, x, max_seq=C + 1, max_chunk=C, n_clusters=K)
+    build_cache(layer, x, C)
+    out = layer.prefill_chunk(torch_bf16(x.q[:, :C])).cpu().numpy()
+    assert layer.check() == 0
+    rows = [0, 1, 700, C - 1]
+    local = [h for h in range(s.n_q_heads) if h not in s.retrieval_heads][0]
+    for h in (s.retrieval_heads[0], s.retrieval_heads[-1], local):
+        r = oracle.layer_rows(x, 0, h, rows)  # dense prefill: p = 1 for the retrieval heads
+        check_outputs(out[0, rows, h], r.out, f"dense prefill h={h}")
+    layer.cluster_build(3)
+    build_cache(layer, x, C + 1)  # the decode token's key, cached after the clustering
+    assert layer.cluster_len(0) == C
+    _check_clustered_decode(x, layer, K, 3, [C + 1], [C], 0.9, row=C)
     layer.close()
