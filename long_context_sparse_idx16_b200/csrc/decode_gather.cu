@@ -73,16 +73,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float* f) {
   }
 }
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __global__ void __launch_bounds__(kIThreads) decode_gather_items_kernel(GatherArgs a) {
   __shared__ int s_base[kMaxProblems + 1];
   __shared__ int s_span[kMaxProblems];
@@ -393,8 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_gather_kernel(GatherArgs a
       for (int u = 0; u < kRowsPerStage; ++u) {
         const int row = hw + 32 * u;
         if (st.g0 + row < st.g1) {
-          cp_async16(sk + row * kD, kg + (int64_t)jv[u] * kD);
-          cp_async16(sv + row * kD, vg + (int64_t)jv[u] * kD);
+          cp_async16(sk + row * kD, kg + (int64_t)jv[u] * kD, 16);
+          cp_async16(sv + row * kD, vg + (int64_t)jv[u] * kD, 16);
         }
       }
     }

@@ -11,8 +11,9 @@
 //     (fp16 operands, fp32 accumulation).  Decode has at most 16 query rows per KV group, far
 //     below the 64/128-row tcgen05 tile, and the kernel is bound by HBM, so the warp-level MMA
 //     is the right size here.
-//   * Each warp streams its own 32-key slice of a 128-key tile with cp.async into an
-//     XOR-swizzled shared tile and reads fragments with ldmatrix, conflict-free.
+//   * Each warp streams its own 16-key slices with cp.async into XOR-swizzled shared tiles,
+//     two buffers deep: the next slice's copies are in flight while the current slice's MMAs
+//     run.  Fragments are read with ldmatrix, conflict-free.
 //   * The window is split into chunks over the grid (enough CTAs for all SMs even at B=1);
 //     per-chunk partials (m, l, o) are merged by a small second kernel.
 #include "rtp_device.cuh"
@@ -24,9 +25,11 @@ namespace {
 
 constexpr int kThreads = kSwaThreads;  // 4 warps
 constexpr int kWarps = kThreads / 32;
-constexpr int kTile = kSwaTile;        // keys per CTA step (32 per warp)
-constexpr int kWarpKeys = kTile / kWarps;
+constexpr int kTile = kSwaTile;        // keys per chunking unit (chunks are whole tiles)
+constexpr int kWarpKeys = 16;          // keys per warp stage
+constexpr int kStepKeys = kWarps * kWarpKeys;  // keys per CTA step (64)
 constexpr int kRowBytes = kD * 2;      // one fp16 row
+constexpr int kStageBytes = 2 * kWarpKeys * kRowBytes;  // one warp stage: K rows, then V rows (8 KB)
 
 struct SwaArgs {
   const __half* kc;
@@ -79,8 +82,7 @@ __global__ void __launch_bounds__(kThreads) decode_swa_kernel(SwaArgs a) {
   const int gr = lane >> 2, tq = lane & 3;  // mma groupID / thread-in-group
   const int n_rows = a.loc_cnt[g];
   if (n_rows == 0) return;
-  unsigned char* ksm = sm + warp * (2 * kWarpKeys * kRowBytes);
-  unsigned char* vsm = ksm + kWarpKeys * kRowBytes;
+  unsigned char* wsm = sm + warp * (2 * kStageBytes);  // this warp's two stage buffers
 
   // Q fragments: rows = local heads of this KV group (zero beyond n_rows)
   uint32_t qa[8][4];
@@ -113,9 +115,12 @@ __global__ void __launch_bounds__(kThreads) decode_swa_kernel(SwaArgs a) {
   const int64_t u_lo = (int64_t)chunk * a.chunk_keys;
   const int64_t u_hi = min(nJ, u_lo + a.chunk_keys);
 
-  for (int64_t t0 = u_lo; t0 < u_hi; t0 += kTile) {
+  // stage `it` of this warp: keys u_lo + it * kStepKeys + warp * kWarpKeys + (0 .. 15), into
+  // buffer it & 1 (keys past the chunk are zero-filled and masked below)
+  auto issue = [&](int64_t t0, int buf) {
+    unsigned char* ksm = wsm + buf * kStageBytes;
+    unsigned char* vsm = ksm + kWarpKeys * kRowBytes;
     const int64_t wbase = t0 + warp * kWarpKeys;
-    // stage this warp's 32 K rows and 32 V rows (16 chunks of 16 B each)
 #pragma unroll
     for (int i = 0; i < (kWarpKeys * 16) / 32; ++i) {
       const int idx = i * 32 + lane;
@@ -127,32 +132,39 @@ __global__ void __launch_bounds__(kThreads) decode_swa_kernel(SwaArgs a) {
       cp_async16(ksm + swz(r, ch), kb + safe * kD + ch * 8, ok ? 16 : 0);
       cp_async16(vsm + swz(r, ch), vb + safe * kD + ch * 8, ok ? 16 : 0);
     }
+  };
+  if (u_lo < u_hi) issue(u_lo, 0);
+  cp_async_commit();
+  int it = 0;
+  for (int64_t t0 = u_lo; t0 < u_hi; t0 += kStepKeys, ++it) {
+    const int buf = it & 1;
+    if (t0 + kStepKeys < u_hi) issue(t0 + kStepKeys, buf ^ 1);  // the next stage, into the other buffer
     cp_async_commit();
-    cp_async_wait<0>();
+    cp_async_wait<1>();  // every group but the newest: this stage has landed
     __syncwarp();
+    const unsigned char* ksm = wsm + buf * kStageBytes;
+    const unsigned char* vsm = ksm + kWarpKeys * kRowBytes;
+    const int64_t wbase = t0 + warp * kWarpKeys;
 
-    // S = Q K^T over 32 keys: 4 n-tiles of 8 keys
-    float s[4][4];
+    // S = Q K^T over 16 keys: 2 n-tiles of 8 keys
+    float s[2][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        // matrices: (ntile 2np, k lo), (2np, k hi), (2np+1, k lo), (2np+1, k hi)
-        const int mi = lane >> 3;
-        const int key = np * 16 + (mi >> 1) * 8 + (lane & 7);
-        const int ch = kk * 2 + (mi & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(smem_u32(ksm) + swz(key, ch), b0, b1, b2, b3);
-        mma16816(s[2 * np], qa[kk], b0, b1);
-        mma16816(s[2 * np + 1], qa[kk], b2, b3);
-      }
+      // matrices: (ntile 0, k lo), (0, k hi), (1, k lo), (1, k hi)
+      const int mi = lane >> 3;
+      const int key = (mi >> 1) * 8 + (lane & 7);
+      const int ch = kk * 2 + (mi & 1);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(smem_u32(ksm) + swz(key, ch), b0, b1, b2, b3);
+      mma16816(s[0], qa[kk], b0, b1);
+      mma16816(s[1], qa[kk], b2, b3);
     }
     // mask keys past the chunk, scale, online softmax (rows gr and gr+8)
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int64_t u = wbase + nt * 8 + 2 * tq + e;
@@ -172,20 +184,19 @@ __global__ void __launch_bounds__(kThreads) decode_swa_kernel(SwaArgs a) {
     const float c1 = mn1 == -INFINITY ? 1.f : fast_exp2(m1 - mn1);
     m0 = mn0;
     m1 = mn1;
-    uint32_t pa[2][4];
+    uint32_t pa[4];
     float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < 2; ++nt) {
       const float p0 = mn0 == -INFINITY ? 0.f : fast_exp2(s[nt][0] - mn0);
       const float p1 = mn0 == -INFINITY ? 0.f : fast_exp2(s[nt][1] - mn0);
       const float p2 = mn1 == -INFINITY ? 0.f : fast_exp2(s[nt][2] - mn1);
       const float p3 = mn1 == -INFINITY ? 0.f : fast_exp2(s[nt][3] - mn1);
       rs0 += p0 + p1;
       rs1 += p2 + p3;
-      // A fragment of P for k-step nt/2: (row gr, keys 2tq..) from even tile, (+8) from odd tile
-      const int ks = nt >> 1, hi = nt & 1;
-      pa[ks][hi ? 2 : 0] = pack_half2(p0, p1);
-      pa[ks][hi ? 3 : 1] = pack_half2(p2, p3);
+      // A fragment of P (one k-step of 16 keys): (row gr, keys 2tq..) from tile 0, (+8) from tile 1
+      pa[nt ? 2 : 0] = pack_half2(p0, p1);
+      pa[nt ? 3 : 1] = pack_half2(p2, p3);
     }
     l0 = l0 * c0 + rs0;
     l1 = l1 * c1 + rs1;
@@ -196,23 +207,21 @@ __global__ void __launch_bounds__(kThreads) decode_swa_kernel(SwaArgs a) {
       o[i][2] *= c1;
       o[i][3] *= c1;
     }
-    // O += P V: 2 k-steps of 16 keys; 8 pairs of 8-dim n-tiles
+    // O += P V: one k-step of 16 keys; 8 pairs of 8-dim n-tiles
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-#pragma unroll
-      for (int dp = 0; dp < 8; ++dp) {
-        // matrices: (keys lo, dims 16dp..+7), (keys hi, same), (keys lo, dims +8..), (keys hi, +8..)
-        const int mi = lane >> 3;
-        const int key = ks * 16 + (mi & 1) * 8 + (lane & 7);
-        const int ch = dp * 2 + (mi >> 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(smem_u32(vsm) + swz(key, ch), b0, b1, b2, b3);
-        mma16816(o[2 * dp], pa[ks], b0, b1);
-        mma16816(o[2 * dp + 1], pa[ks], b2, b3);
-      }
+    for (int dp = 0; dp < 8; ++dp) {
+      // matrices: (keys lo, dims 16dp..+7), (keys hi, same), (keys lo, dims +8..), (keys hi, +8..)
+      const int mi = lane >> 3;
+      const int key = (mi & 1) * 8 + (lane & 7);
+      const int ch = dp * 2 + (mi >> 1);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(vsm) + swz(key, ch), b0, b1, b2, b3);
+      mma16816(o[2 * dp], pa, b0, b1);
+      mma16816(o[2 * dp + 1], pa, b2, b3);
     }
-    __syncwarp();
+    __syncwarp();  // this buffer is refilled two stages on
   }
+  cp_async_wait<0>();  // no copy may still land in the tile space the merge below reuses
 
   // row sums across the 4 threads of a group
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -319,12 +328,13 @@ __global__ void __launch_bounds__(256) swa_merge_kernel(const float* __restrict_
 
 }  // namespace
 
-// Chunking, in whole 128-key tiles: at most two CTAs per SM over the whole grid, so the grid
-// runs as one wave (the kernel's registers -- about 254 per thread at 128 threads -- let two
-// CTAs share an SM; a third CTA on any SM would wait for a second wave).
+// Chunking, in whole 128-key tiles: at most three CTAs per SM over the whole grid, so the grid
+// runs as one wave (166 registers per thread at 128 threads and 64 KB of shared memory let
+// three CTAs share an SM; a fourth would wait for a second wave).
+constexpr int64_t kSwaCtasPerSm = 3;
 static void swa_chunks(const rtp_layer* L, int64_t nJ, int64_t* chunk_keys, int* n_chunks) {
   const int64_t pairs = (int64_t)L->B * L->Hkv;
-  int64_t want = (2LL * L->sm_count) / pairs;  // chunks per (b, g)
+  int64_t want = (kSwaCtasPerSm * L->sm_count) / pairs;  // chunks per (b, g)
   if (want < 1) want = 1;
   int64_t ck = (nJ + want - 1) / want;
   ck = (ck + kTile - 1) / kTile * kTile;
@@ -337,7 +347,7 @@ static void swa_chunks(const rtp_layer* L, int64_t nJ, int64_t* chunk_keys, int*
 // want is at most this.
 static int64_t swa_max_chunks(const rtp_layer* L) {
   const int64_t pairs = (int64_t)L->B * L->Hkv;
-  return (2LL * L->sm_count + pairs - 1) / pairs;
+  return (kSwaCtasPerSm * L->sm_count + pairs - 1) / pairs;
 }
 
 int64_t swa_part_elems(const rtp_layer* L) {
@@ -370,7 +380,7 @@ cudaError_t launch_decode_swa(const rtp_layer* L, float* out, cudaStream_t st) {
   a.scale_log2 = L->sm_scale * 1.4426950408889634f;
   a.part = L->spart;
   a.out = out;
-  const size_t tile_smem = (size_t)kWarps * 2 * kWarpKeys * kRowBytes;  // 64 KB
+  const size_t tile_smem = (size_t)kWarps * 2 * kStageBytes;  // 64 KB: two stage buffers per warp
   const size_t merge_smem = (size_t)kWarps * 16 * kD * 4 + kWarps * 16 * 2 * 4;
   const size_t smem = tile_smem > merge_smem ? tile_smem : merge_smem;
   cudaError_t e = cudaFuncSetAttribute(decode_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
